@@ -1,0 +1,15 @@
+"""Seeded synthetic STCA workloads shared by the oracle tests, the GPU tests and the bench.
+
+This package draws inputs only (history lengths, target counts, embeddings,
+weights) and stores them in the element type a configuration names.  It holds
+none of the method's arithmetic: no encoding, no attention, no fusion.
+"""
+from .workloads import (  # noqa: F401
+    CONFIGS,
+    Workload,
+    bf16_bits_to_f32,
+    f32_to_bf16_bits,
+    make_config_workload,
+    make_workload,
+    round_to_bf16,
+)
