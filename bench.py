@@ -1,0 +1,473 @@
+#!/usr/bin/env python
+"""STCA forward throughput on one or more B200s, through the C ABI.
+
+One step = stca_encode (the M history encodings, Eq. (2)) + stca_forward (the
+M stacked single-query cross-attention layers with query fusion, Eqs. (3)-(8))
+over one synthetic jagged batch shaped like the request-level-batched serving
+workload: 64 requests, L = 10000 history tokens each, 16 targets per request,
+d = 128, h = 8, M = 3, r = 4, bf16 storage with fp32 accumulation.
+
+Prints ONE JSON line (rank 0): history-tokens/s over all ranks, the targets/s
+companion, the roofline of the dominant kernel (timed live with CUDA events
+around its launches), the whole-step roofline, an end-to-end figure through
+the host-buffer entry point, the fp64 CPU oracle timed on a bounded sample, and
+the SM clocks sampled during the timed region.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--config c1..c5]
+Under torchrun (N > 1) every rank runs its own batch (weak scaling).
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from gen import CONFIGS, make_config_workload  # noqa: E402
+
+METRIC = "STCA fwd history-tokens/s & targets/s at L=10k; % of HBM/tensor roofline"
+UNIT = "history-tokens/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_BYTES = 126 * 2 ** 20
+
+
+def log(*a):
+    print(*a, file=sys.stderr, flush=True)
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in FALLBACK_PEAKS}, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ----------------------------------------------------------------- counts
+def counts(wl):
+    """Algorithmic FLOPs and bytes of one step (encode + forward)."""
+    N, T, d, h, M, rd = wl.N, wl.T, wl.d, wl.h, wl.M, wl.r * wl.d
+    s = 2 if wl.dtype == "bf16" else 4
+    TL = int(np.sum(wl.lengths.astype(np.int64) * wl.target_counts.astype(np.int64)))
+    enc_flops = M * N * 6 * d * rd                     # GEMM1 (2 x 2 d rd) + GEMM2 (2 rd d)
+    attn_flops = M * 4 * h * d * TL                    # u X~^T and alpha X~ over d, per head
+    tgt_flops = T * 6 * rd * d + T * sum(
+        8 * d * d + ((2 * (i + 2) * d * d + 6 * rd * d) if i + 1 < M else 0) for i in range(M))
+    return {
+        "N": N, "T": T, "TL": TL, "elem": s,
+        "enc_flops": enc_flops, "attn_flops": attn_flops, "tgt_flops": tgt_flops,
+        "tensor_flops": enc_flops + attn_flops + tgt_flops,
+        "enc_bytes_per_layer": 2 * N * d * s,          # read X, write X~(i)
+        "attn_bytes_per_layer": N * d * s,             # read X~(i) once for all T_r h rows
+        "bytes_min": M * N * d * s,
+        "bytes_materialised": (2 * M + 1) * N * d * s,
+        "io_bytes": T * d * s + T * M * d * 4,
+    }
+
+
+# ----------------------------------------------------------------- clocks
+_REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+            0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+            0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+            0x100: "display_clock_setting"}
+
+
+class ClockSampler:
+    """Samples SM clock, power and clock-event reasons through NVML (read only)."""
+
+    def __init__(self, torch_device_index=0, period_s=0.02):
+        self.samples, self.max_mhz, self.ok = [], None, False
+        self.period = period_s
+        try:
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            props = torch.cuda.get_device_properties(torch_device_index)
+            h = None
+            uuid = getattr(props, "uuid", None)
+            if uuid is not None:
+                try:
+                    h = pynvml.nvmlDeviceGetHandleByUUID("GPU-" + str(uuid))
+                except Exception:
+                    h = None
+            if h is None:
+                h = pynvml.nvmlDeviceGetHandleByIndex(torch_device_index)
+            self.h = h
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # pragma: no cover
+            log(f"clock sampling unavailable: {e}")
+        self._stop = threading.Event()
+        self._t = None
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                sm = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+                try:
+                    rs = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                except Exception:
+                    rs = nv.nvmlDeviceGetCurrentClocksThrottleReasons(self.h)
+                util = nv.nvmlDeviceGetUtilizationRates(self.h).gpu
+                self.samples.append((sm, int(rs), util))
+            except Exception:
+                pass
+            self._stop.wait(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self._t:
+            self._stop.set()
+            self._t.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
+        loaded = [s for s in self.samples if s[2] > 0] or self.samples
+        bits = 0
+        for s in loaded:
+            bits |= s[1]
+        reasons = sorted(n for b, n in _REASONS.items() if bits & b and n != "gpu_idle")
+        return {"sm_mhz": float(statistics.median(s[0] for s in loaded)),
+                "sm_max_mhz": self.max_mhz, "reasons": reasons, "samples": len(loaded)}
+
+
+# ----------------------------------------------------------------- oracle leg
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else os.cpu_count()
+    except Exception:
+        return os.cpu_count()
+
+
+def oracle_sample(wl, budget_s=15.0, seed=0):
+    """Time the fp64 oracle on whole requests of `wl` until ~budget_s of CPU work."""
+    from oracle import stca_oracle as O
+    rng = np.random.default_rng(seed)
+    order = [int(r) for r in rng.permutation(wl.R)]
+    done, t0 = [], time.perf_counter()
+    for r in order:
+        O.forward_workload(wl, requests=[r])
+        done.append(r)
+        if time.perf_counter() - t0 >= budget_s:
+            break
+    dt = time.perf_counter() - t0
+    toks = int(sum(int(wl.lengths[r]) for r in done))
+    tg = int(sum(int(wl.target_counts[r]) for r in done))
+    return {"value": toks / dt, "unit": UNIT, "targets_per_s": tg / dt, "cores": blas_threads(),
+            "kind": "oracle", "sample": f"{len(done)} of {wl.R} requests ({toks} history tokens, "
+                                        f"{tg} targets) of the same workload, {dt:.1f} s"}
+
+
+def run_reference(args, rank):
+    """The oracle as the reference arm: each step runs it on a bounded sample."""
+    if rank != 0:
+        return
+    wl = make_config_workload(args.config)
+    from oracle import stca_oracle as O
+    rng = np.random.default_rng(123)
+    # one step = the oracle on `per_step` whole requests, sized to keep the run short
+    t0 = time.perf_counter()
+    O.forward_workload(wl, requests=[0])
+    t1 = time.perf_counter() - t0
+    budget = 150.0 / max(1, args.steps + args.warmup)
+    per_step = int(max(1, min(wl.R, budget // max(t1, 1e-6))))
+    times, toks, tgs = [], 0, 0
+    for it in range(args.warmup + args.steps):
+        reqs = [int(x) for x in rng.choice(wl.R, size=per_step, replace=False)]
+        s0 = time.perf_counter()
+        O.forward_workload(wl, requests=reqs)
+        dt = time.perf_counter() - s0
+        if it >= args.warmup:
+            times.append(dt)
+            toks += int(sum(int(wl.lengths[r]) for r in reqs))
+            tgs += int(sum(int(wl.target_counts[r]) for r in reqs))
+    tot = sum(times)
+    value = toks / tot
+    cores = blas_threads()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * tot / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(wl, args.gpus),
+        "targets_per_s": tgs / tot,
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": f"each step: the oracle on {per_step} random whole requests "
+                                   f"of the workload, on {cores} host threads"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def workload_config(wl, n):
+    cfg = {"workload": wl.name, "R": wl.R, "history_tokens": wl.N, "targets": wl.T,
+           "L": (int(wl.lengths[0]) if np.all(wl.lengths == wl.lengths[0])
+                 else f"{int(wl.lengths.min())}..{int(wl.lengths.max())}"),
+           "d": wl.d, "h": wl.h, "M": wl.M, "r": wl.r, "storage": wl.dtype,
+           "parallelism": f"dp{n}"}
+    s = 2 if wl.dtype == "bf16" else 4
+    in_bytes = wl.N * wl.d * s
+    if in_bytes * (wl.M + 1) > L2_BYTES:
+        cfg["l2"] = (f"no flush: inputs larger than L2 (X {in_bytes / 1e6:.0f} MB and "
+                     f"X~ {wl.M * in_bytes / 1e6:.0f} MB per step vs 126 MB L2)")
+    else:
+        cfg["l2"] = "L2 flushed between steps (256 MB write)"
+    return cfg
+
+
+# ----------------------------------------------------------------- our arm
+def to_dev(wl, a, device):
+    import torch
+    t = torch.from_numpy(np.ascontiguousarray(wl.storage(a)))
+    if wl.dtype == "bf16":
+        t = t.view(torch.int16).view(torch.bfloat16)
+    return t.to(device)
+
+
+def storage_weights(wl):
+    out = {}
+    for k, v in wl.weights.items():
+        if v is None:
+            out[k] = None
+        elif isinstance(v, list):
+            out[k] = [None if a is None else wl.storage(a) for a in v]
+        else:
+            out[k] = wl.storage(v)
+    return out
+
+
+def roofline_of(kind, kt, c, wl, peaks, sustained, steps):
+    """Roofline object of kernel class `kind` from its live event timings.
+
+    Per launch, the algorithmic work is the class's per-step total divided by
+    its launches per step (e.g. the encoder: M N 6 d rd FLOPs and 2 N d s bytes
+    per layer; the attention: 4 h d sum_r T_r L_r FLOPs and N d s bytes per layer).
+    """
+    ms, n = kt[kind]
+    if n == 0 or ms <= 0:
+        return None
+    avg_s = ms / n / 1e3
+    per_step = n / steps
+    if kind == "encode":
+        flops, bytes_ = c["enc_flops"] / per_step, c["enc_bytes_per_layer"] * wl.M / per_step
+    elif kind == "attention":
+        flops, bytes_ = c["attn_flops"] / per_step, c["attn_bytes_per_layer"] * wl.M / per_step
+    else:
+        flops, bytes_ = c["tgt_flops"] / per_step, c["io_bytes"] / per_step
+    base = {"kernel": kind, "traffic": None, "avg_launch_ms": avg_s * 1e3,
+            "flops_per_launch": flops, "bytes_per_launch": bytes_}
+    if wl.dtype == "f32":
+        peak = 148 * 128 * 2 * 1.965e9 / 1e12     # FP32 FFMA lanes x clock (nominal)
+        ach = flops / avg_s / 1e12
+        return dict(base, bound="alu", achieved=ach, peak=peak, unit="TFLOP/s", frac=ach / peak,
+                    peak_source="nominal FP32 FFMA: 148 SMs x 128 lanes x 2 x 1.965 GHz")
+    tflops_peak = peaks["bf16_tflops_sustained" if sustained else "bf16_tflops"]
+    ridge = tflops_peak * 1e12 / (peaks["hbm_gbs"] * 1e9)
+    if flops / bytes_ >= ridge:
+        ach = flops / avg_s / 1e12
+        return dict(base, bound="tensor", achieved=ach, peak=tflops_peak, unit="TFLOP/s",
+                    frac=ach / tflops_peak,
+                    peak_source="bf16_tflops_sustained" if sustained else "bf16_tflops")
+    ach = bytes_ / avg_s / 1e9
+    return dict(base, bound="hbm", achieved=ach, peak=peaks["hbm_gbs"], unit="GB/s",
+                frac=ach / peaks["hbm_gbs"], peak_source="hbm_gbs")
+
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+    import target_attention_jagged_b200 as S
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    wl = make_config_workload(args.config, seed=CONFIGS[args.config]["seed"] + 1000 * rank)
+    c = counts(wl)
+    peaks, peak_src = load_peaks()
+    stream = torch.cuda.Stream(device=dev)
+    st = S.Stca(storage_weights(wl), wl.d, wl.h, wl.r, wl.M, wl.dtype)
+    X = to_dev(wl, wl.X, dev)
+    xt = to_dev(wl, wl.targets, dev)
+    Z = torch.empty((wl.T, wl.M, wl.d), dtype=torch.float32, device=dev)
+    s2 = 2 if wl.dtype == "bf16" else 4
+    flush = None
+    if wl.N * wl.d * s2 * (wl.M + 1) <= L2_BYTES:
+        flush = torch.empty(256 * 2 ** 20, dtype=torch.uint8, device=dev)
+
+    def step():
+        if flush is not None:
+            flush.fill_(1)
+        st.encode(X, wl.offsets, stream)
+        st.forward(xt, wl.target_offsets, Z, stream)
+
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            step()
+    torch.cuda.synchronize()
+    st.status(stream)
+    launches_per_step = st.get_option(S.STCA_OPT_LAUNCHES)
+    st.set_option(S.STCA_OPT_TIMING, 1)
+    S.stca_kernel_times(st.handle)          # drop anything recorded so far
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(local_rank)
+    with sampler, torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(args.steps):
+            step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    elapsed_ms = e0.elapsed_time(e1)
+    kt = S.stca_kernel_times(st.handle)
+    st.set_option(S.STCA_OPT_TIMING, 0)
+    st.status(stream)
+    if world > 1:
+        t = torch.tensor([elapsed_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed_ms = float(t.item())
+    sec = elapsed_ms / 1e3
+    value = world * wl.N * args.steps / sec
+    targets_per_s = world * wl.T * args.steps / sec
+    sustained = sec > 1.0
+    rooflines = {k: roofline_of(k, kt, c, wl, peaks, sustained, args.steps) for k in kt}
+    for r_ in rooflines.values():
+        if r_:
+            r_["peak_source"] += f" ({peak_src})"
+    dom = max(kt, key=lambda k: kt[k][0])
+    roof = dict(rooflines[dom])
+    tpeak = peaks["bf16_tflops_sustained" if sustained else "bf16_tflops"] * 1e12
+    t_flop = c["tensor_flops"] / tpeak
+    t_bytes = c["bytes_materialised"] / (peaks["hbm_gbs"] * 1e9)
+    t_roof = max(t_flop, t_bytes)
+    step_roof = {"t_roof_ms": t_roof * 1e3, "t_step_ms": elapsed_ms / args.steps,
+                 "frac": t_roof / (sec / args.steps),
+                 "bound": "tensor" if t_flop >= t_bytes else "hbm",
+                 "tensor_flops": c["tensor_flops"], "bytes_materialised": c["bytes_materialised"],
+                 "bytes_min": c["bytes_min"],
+                 "frac_bytes_min": (c["bytes_min"] / (peaks["hbm_gbs"] * 1e9)) / (sec / args.steps)}
+
+    # ---- forward only (the encoded history reused for a new set of targets)
+    torch.cuda.synchronize()
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        st.encode(X, wl.offsets, stream)
+        st.forward(xt, wl.target_offsets, Z, stream)
+        f0.record(stream)
+        for _ in range(args.steps):
+            st.forward(xt, wl.target_offsets, Z, stream)
+        f1.record(stream)
+    torch.cuda.synchronize()
+    fwd_ms = f0.elapsed_time(f1) / args.steps
+
+    # ---- end to end through the host-buffer entry point
+    Xh = torch.from_numpy(np.ascontiguousarray(wl.storage(wl.X))).pin_memory()
+    th = torch.from_numpy(np.ascontiguousarray(wl.storage(wl.targets))).pin_memory()
+    Zh = torch.empty((wl.T, wl.M, wl.d), dtype=torch.float32).pin_memory()
+    for _ in range(min(args.warmup, 3)):
+        S.stca_run_host(st.handle, Xh, wl.offsets, th, wl.target_offsets, Zh, stream)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    g0.record(stream)
+    for _ in range(args.steps):
+        S.stca_run_host(st.handle, Xh, wl.offsets, th, wl.target_offsets, Zh, stream)
+    g1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = g0.elapsed_time(g1)
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e = {"value": world * wl.N * args.steps / (e2e_ms / 1e3), "unit": UNIT,
+           "h2d_bytes_per_step": int(Xh.numel() * Xh.element_size() + th.numel() * th.element_size()
+                                     + 2 * 8 * (wl.R + 1)),
+           "d2h_bytes_per_step": int(Zh.numel() * Zh.element_size()),
+           "targets_per_s": world * wl.T * args.steps / (e2e_ms / 1e3)}
+    st.close()
+
+    if rank != 0:
+        return
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": wl.dtype,
+        "data": "synthetic (seeded N(0,1) embeddings, Xavier-uniform weights)",
+        "config": workload_config(wl, world),
+        "targets_per_s": targets_per_s,
+        "roofline": roof, "roofline_step": step_roof,
+        "kernels": {k: {"ms_total": v[0], "launches": v[1]} for k, v in kt.items()},
+        "forward_only": {"ms_per_forward": fwd_ms,
+                         "targets_per_s": world * wl.T / (fwd_ms / 1e3),
+                         "history_tokens_per_s": world * wl.N / (fwd_ms / 1e3)},
+        "e2e": e2e,
+        "gpu_launches": int(launches_per_step * args.steps),
+        "clocks": sampler.summary(),
+        "when": datetime.datetime.utcnow().isoformat() + "Z",
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = oracle_sample(wl, budget_s=args.cpu_budget)
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--config", default="c3", choices=sorted(CONFIGS))
+    ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        log(f"note: WORLD_SIZE={world} but --gpus={args.gpus}; using WORLD_SIZE")
+    if args.impl == "reference":
+        run_reference(args, rank)
+        return
+    if world > 1:
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,199 @@
+/*
+ * stca.h -- C ABI of the STCA forward library (libstca.so, sm_100a).
+ *
+ * Stacked Target Cross Attention over jagged user histories with
+ * request-level batching.  Sources:
+ *   [digest] "Make It Long, Keep It Fast: End-to-End 10k-Sequence Modeling at
+ *            Billion Scale on Douyin" (paper digest), §2.1 Eqs. (1)-(8), (13);
+ *            §2.2 (request-level batching); §2.3 (ragged target attention).
+ *   [blog]   "字节跳动-STCA：抖音 10k 长序列端到端建模的架构、系统与外推三件套"
+ *            (STCA blog), §2.2-§2.5.
+ *
+ * What the calls compute.  For request r with history X_r (L_r x d, the rows
+ * offsets[r] .. offsets[r+1]-1 of X) and targets x_t (rows target_offsets[r]
+ * .. target_offsets[r+1]-1 of `targets`), for every layer i = 1..M:
+ *   X~(i)   = LN_i(SwiGLUFFN_i(X_r))                        [digest] Eq. (2)
+ *   q(1)    = LN_q(SwiGLUFFN_q1(x_t))                        Eq. (3)
+ *   u_j     = (q(i) W_Q^(i,j)) W_K^(i,j)^T,  head j          Eq. (13)
+ *   alpha_j = softmax(u_j X~(i)^T / sqrt(d_h)) over the L_r history rows
+ *   o(i)    = [ (alpha_1 X~(i)) W_V^(i,1) || ... || (alpha_h X~(i)) W_V^(i,h) ] W_O^(i)
+ *                                                            Eqs. (6), (13)
+ *   q(i+1)  = SwiGLUFFN_q(i+1)([o(1) || ... || o(i) || x_t] W_C^(i+1))   Eq. (7)
+ * and writes Z[t, i, :] = o(i) for every target t (Eq. (8)).
+ *   SwiGLUFFN(x) = ((x W_u) * SiLU(x W_g)) W_d, no biases (Eq. (1) read with the
+ *   blog's shapes: W_u, W_g d x rd, W_d rd x d).  LN: eps 1e-5, biased variance,
+ *   affine (gamma, beta).  Head j owns columns [j d_h, (j+1) d_h) of W_Q, W_K, W_V.
+ *   The history encodings X~(i) read the raw X for every i; they are not chained.
+ *
+ * Conventions.  Row-major everywhere, x * W (row vector times matrix).
+ * Element type of X, targets and all weights: the handle's dtype (STCA_F32:
+ * IEEE fp32; STCA_BF16: bfloat16 bit patterns, uint16).  Z is always fp32.
+ * Return value: STCA_OK (0) or a negative STCA_E* code; stca_last_error()
+ * gives a message (thread-local).  No call aborts the process.
+ *
+ * Threading and streams.  A handle is used by one host thread at a time and
+ * orders its work on the stream passed to each call (NULL = the legacy
+ * default stream).  Separate handles are independent.
+ */
+#ifndef STCA_H_
+#define STCA_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct stca_handle stca_handle;
+
+typedef enum { STCA_F32 = 0, STCA_BF16 = 1 } stca_dtype;
+
+enum {
+  STCA_OK = 0,
+  STCA_EINVAL = -1,      /* bad argument: shape, dtype, pointer, offsets       */
+  STCA_ESTATE = -2,      /* call out of order, e.g. forward before encode      */
+  STCA_ENOMEM = -3,      /* device or pinned host allocation failed            */
+  STCA_ECUDA = -4,       /* a CUDA runtime or driver call failed               */
+  STCA_EDEVICE = -5      /* a kernel reported a failure (bounded wait ran out) */
+};
+
+/*
+ * Weights of all M layers.  Each field is a host array of M pointers, entry i
+ * belonging to layer i+1.  Pointers are host pointers unless stca_init's
+ * weights_on_device is nonzero; each points to dtype elements, row-major.
+ *   Wu[i], Wg[i]  d x rd       SwiGLU up and gate projections   Eq. (1)-(2)
+ *   Wd[i]         rd x d       SwiGLU down projection
+ *   ln_gamma[i], ln_beta[i]  d LayerNorm affine of layer i's history encoding;
+ *                 the field itself may be NULL: gamma = 1, beta = 0
+ *   Wq[i], Wk[i], Wv[i], Wo[i]  d x d   attention projections   Eqs. (4)-(6)
+ *   Wc[i]         (i+1)d x d   query fusion of layer i+1 (Eq. (7)); Wc[0] is
+ *                 ignored and may be NULL; the field may be NULL when M == 1
+ *   qWu, qWg, qWd optional query-side SwiGLU of each layer (Eqs. (3), (7));
+ *                 NULL field: the query uses the history FFN of that layer
+ *   q_ln_gamma, q_ln_beta  optional single pointers (d elements): the LN of
+ *                 Eq. (3); NULL: layer 1's ln_gamma / ln_beta
+ * stca_init copies everything; the caller may free its buffers afterwards.
+ */
+typedef struct {
+  const void* const* Wu;
+  const void* const* Wg;
+  const void* const* Wd;
+  const void* const* ln_gamma;
+  const void* const* ln_beta;
+  const void* const* Wq;
+  const void* const* Wk;
+  const void* const* Wv;
+  const void* const* Wo;
+  const void* const* Wc;
+  const void* const* qWu;
+  const void* const* qWg;
+  const void* const* qWd;
+  const void* q_ln_gamma;
+  const void* q_ln_beta;
+} stca_weights;
+
+/*
+ * Create a handle on the current CUDA device and copy the weights into it.
+ * d: model width; h: heads (d % h == 0); r: SwiGLU expansion (hidden rd = r*d);
+ * M: stacked layers (1..16); dtype: STCA_F32 or STCA_BF16.
+ * Supported sizes: d in [8, 1024] with d % 8 == 0, rd <= 4096.  The bf16
+ * tensor-core kernels additionally need d in {64, 128, 256} and rd % 64 == 0;
+ * other bf16 sizes run on the CUDA-core kernels.
+ * On success *out owns device memory until stca_destroy.
+ * Errors: STCA_EINVAL (sizes, NULL required field), STCA_ENOMEM, STCA_ECUDA.
+ */
+int stca_init(const stca_weights* w, int d, int h, int r, int M, int dtype,
+              int weights_on_device, stca_handle** out);
+
+/* Release everything the handle owns.  NULL is accepted. */
+void stca_destroy(stca_handle* handle);
+
+/*
+ * Encode a jagged batch of histories: computes X~(i) for i = 1..M (Eq. (2))
+ * into buffers the handle owns; they stay valid until the next stca_encode
+ * or stca_destroy, so any number of stca_forward calls can reuse them
+ * (request-level batching: one history, many targets).
+ *   X        device pointer, N x d dtype elements, requests concatenated
+ *   offsets  HOST pointer, R+1 int64: offsets[0] == 0, offsets[R] == N,
+ *            offsets[r+1] - offsets[r] = L_r >= 1 (an empty history has no
+ *            softmax and is rejected)
+ *   R >= 1 requests, N rows in total.  stream: a cudaStream_t or NULL.
+ * Asynchronous with respect to the host, except that a first call or a larger
+ * batch than before allocates device memory.
+ * Errors: STCA_EINVAL (offsets not monotone, L_r == 0, sizes), STCA_ENOMEM,
+ * STCA_ECUDA.
+ */
+int stca_encode(stca_handle* handle, const void* X, const int64_t* offsets,
+                int64_t R, int64_t N, void* stream);
+
+/*
+ * Run the stacked target attention for the targets of the encoded requests.
+ *   targets         device pointer, T x d dtype elements, grouped by request
+ *   target_offsets  HOST pointer, R+1 int64 with the R of the last encode:
+ *                   targets of request r are rows target_offsets[r] ..
+ *                   target_offsets[r+1]-1; T_r = 0 is allowed
+ *   T               total targets (target_offsets[R]); T == 0 is a no-op
+ *   Z               device pointer, caller-owned, T x M x d fp32; row t holds
+ *                   [o(1); ...; o(M)] of target t (Eq. (8))
+ * Errors: STCA_ESTATE (no encode yet), STCA_EINVAL, STCA_ENOMEM, STCA_ECUDA.
+ */
+int stca_forward(stca_handle* handle, const void* targets, const int64_t* target_offsets,
+                 int64_t T, float* Z, void* stream);
+
+/*
+ * End-to-end call on HOST buffers: copies X and targets from host memory to
+ * device staging buffers the handle owns, encodes, runs the forward, copies
+ * Z (T x M x d fp32) back to host memory and waits for the stream.  Host
+ * buffers should be page-locked for the copies to overlap; pageable memory
+ * works but is slower.  Same argument rules as stca_encode and stca_forward.
+ */
+int stca_run_host(stca_handle* handle, const void* X_host, const int64_t* offsets,
+                  int64_t R, int64_t N, const void* targets_host,
+                  const int64_t* target_offsets, int64_t T, float* Z_host, void* stream);
+
+/*
+ * Check offsets on the host without touching a device: offsets[0] == 0,
+ * non-decreasing, offsets[R] == total; with require_nonempty, every segment
+ * has at least one row.  Returns STCA_OK or STCA_EINVAL.
+ */
+int stca_validate_offsets(const int64_t* offsets, int64_t R, int64_t total,
+                          int require_nonempty);
+
+/*
+ * Wait for the handle's work on `stream` and read its device status word.
+ * STCA_OK, or STCA_EDEVICE if a kernel gave up a bounded wait (the message
+ * names the kernel), or STCA_ECUDA.  The status is cleared by the read.
+ */
+int stca_device_status(stca_handle* handle, void* stream);
+
+/* Tunables and introspection (STCA_OPT_*).  Values are validated. */
+enum {
+  STCA_OPT_ATTN_PATH = 1,     /* 0 auto, 1 CUDA cores, 2 tensor cores (bf16 only) */
+  STCA_OPT_ENCODE_PATH = 2,   /* 0 auto, 1 CUDA cores, 2 tensor cores (bf16 only) */
+  STCA_OPT_SPLIT_KEYS = 3,    /* keys per attention work item, 0 = auto; multiple of 128 */
+  STCA_OPT_TIMING = 4,        /* 1: record CUDA events around every kernel launch */
+  STCA_OPT_LAUNCHES = 100     /* read-only: kernels launched since the last encode */
+};
+int stca_set_option(stca_handle* handle, int option, int64_t value);
+int stca_get_option(stca_handle* handle, int option, int64_t* value);
+
+/* Kernel classes reported by stca_kernel_times. */
+enum { STCA_K_ENCODE = 0, STCA_K_ATTN = 1, STCA_K_STEP = 2, STCA_K_CLASSES = 3 };
+
+/*
+ * Device time of each kernel class since the previous call, from the CUDA
+ * events recorded (on the launch stream) around every launch while
+ * STCA_OPT_TIMING is 1.  Writes ms[c] (milliseconds, summed) and launches[c]
+ * for c < min(n, STCA_K_CLASSES); either array may be NULL.  Waits for the
+ * recorded events, then forgets them.
+ */
+int stca_kernel_times(stca_handle* handle, double* ms, int64_t* launches, int n);
+
+/* Message of the last error on this host thread ("" if none). */
+const char* stca_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* STCA_H_ */

@@ -1,0 +1,86 @@
+"""Build libstca.so in-tree with nvcc for sm_100a.
+
+    python target_attention_jagged_b200/build.py [--debug] [--verbose-ptxas] [--force]
+
+Compiles every .cu under csrc/ into target_attention_jagged_b200/libstca.so.
+"""
+from __future__ import annotations
+
+import argparse
+import glob
+import os
+import shutil
+import subprocess
+import sys
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+ROOT = os.path.dirname(PKG)
+LIB = os.path.join(PKG, "libstca.so")
+ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
+
+
+def nvcc() -> str:
+    for cand in (os.environ.get("NVCC"), "/usr/local/cuda/bin/nvcc", shutil.which("nvcc")):
+        if cand and os.path.exists(cand):
+            return cand
+    raise RuntimeError("nvcc not found")
+
+
+def sources():
+    return sorted(glob.glob(os.path.join(PKG, "csrc", "*.cu")))
+
+
+def headers():
+    return sorted(glob.glob(os.path.join(PKG, "csrc", "*.h")) +
+                  glob.glob(os.path.join(PKG, "csrc", "*.cuh")) +
+                  glob.glob(os.path.join(ROOT, "include", "*.h")))
+
+
+def up_to_date() -> bool:
+    if not os.path.exists(LIB):
+        return False
+    t = os.path.getmtime(LIB)
+    return all(os.path.getmtime(f) <= t for f in sources() + headers() + [__file__])
+
+
+def build(debug: bool = False, verbose_ptxas: bool = False, force: bool = False) -> str:
+    if not force and not debug and not verbose_ptxas and up_to_date():
+        return LIB
+    objdir = os.path.join(PKG, "_build")
+    os.makedirs(objdir, exist_ok=True)
+    flags = ARCH + ["-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC",
+                    "-I", os.path.join(ROOT, "include"), "-I", os.path.join(PKG, "csrc")]
+    flags += ["-O0", "-G"] if debug else ["-O3"]
+    if verbose_ptxas:
+        flags += ["-Xptxas", "-v"]
+    objs = []
+    for src in sources():
+        obj = os.path.join(objdir, os.path.basename(src) + ".o")
+        cmd = [nvcc()] + flags + ["-c", src, "-o", obj]
+        r = subprocess.run(cmd, capture_output=True, text=True)
+        if r.returncode != 0 or verbose_ptxas:
+            sys.stderr.write(r.stdout + r.stderr)
+        if r.returncode != 0:
+            raise RuntimeError(f"nvcc failed on {src}")
+        objs.append(obj)
+    tmp = LIB + ".tmp"
+    cmd = [nvcc()] + ARCH + ["-shared", "-o", tmp] + objs + ["-lcuda"]
+    r = subprocess.run(cmd, capture_output=True, text=True)
+    if r.returncode != 0:
+        sys.stderr.write(r.stdout + r.stderr)
+        raise RuntimeError("link failed")
+    os.replace(tmp, LIB)
+    return LIB
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--debug", action="store_true")
+    ap.add_argument("--verbose-ptxas", action="store_true")
+    ap.add_argument("--force", action="store_true")
+    a = ap.parse_args()
+    print(build(debug=a.debug, verbose_ptxas=a.verbose_ptxas, force=a.force))
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,617 @@
+// C ABI of the STCA forward library: argument checks, weight staging, the
+// attention work plan and the launch sequence.  See include/stca.h.
+#include <cuda_runtime.h>
+#include <string.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdint>
+#include <new>
+#include <string>
+#include <vector>
+
+#include "stca_internal.h"
+
+namespace stca {
+
+static thread_local std::string g_err;
+
+int set_error(int code, const std::string& msg) {
+  g_err = msg;
+  return code;
+}
+
+static int ok() {
+  g_err.clear();
+  return STCA_OK;
+}
+
+// Make the handle's device current for the duration of a call.
+struct DeviceGuard {
+  int prev = -1;
+  bool ok = true;
+  explicit DeviceGuard(int dev) {
+    if (cudaGetDevice(&prev) != cudaSuccess) { prev = -1; ok = false; return; }
+    if (prev != dev && cudaSetDevice(dev) != cudaSuccess) ok = false;
+  }
+  ~DeviceGuard() {
+    int cur = -1;
+    if (prev >= 0 && cudaGetDevice(&cur) == cudaSuccess && cur != prev) cudaSetDevice(prev);
+  }
+};
+
+static int check_launch(const char* what) {
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess)
+    return set_error(STCA_ECUDA, std::string(what) + ": " + cudaGetErrorString(e));
+  return STCA_OK;
+}
+
+// Grow-only device buffer.
+static int ensure_dev(void** p, size_t* cap, size_t need) {
+  if (need <= *cap && *p) return STCA_OK;
+  if (*p) { cudaFree(*p); *p = nullptr; *cap = 0; }
+  size_t bytes = std::max<size_t>(need, 256);
+  bytes = (bytes + (1u << 20) - 1) & ~static_cast<size_t>((1u << 20) - 1);
+  if (cudaMalloc(p, bytes) != cudaSuccess) {
+    cudaGetLastError();
+    *p = nullptr;
+    return set_error(STCA_ENOMEM, "cudaMalloc of " + std::to_string(bytes) + " bytes failed");
+  }
+  *cap = bytes;
+  return STCA_OK;
+}
+
+// Optional CUDA events around one launch (STCA_OPT_TIMING).
+static cudaEvent_t pool_event(stca_handle* H) {
+  if (!H->ev_pool.empty()) {
+    cudaEvent_t e = H->ev_pool.back();
+    H->ev_pool.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  if (cudaEventCreate(&e) != cudaSuccess) { cudaGetLastError(); return nullptr; }
+  return e;
+}
+
+struct TimedLaunch {
+  stca_handle* H;
+  int cls;
+  cudaStream_t s;
+  cudaEvent_t a = nullptr;
+  TimedLaunch(stca_handle* h, int c, cudaStream_t st) : H(h), cls(c), s(st) {
+    if (H->timing && (a = pool_event(H))) cudaEventRecord(a, s);
+  }
+  ~TimedLaunch() {
+    if (!a) return;
+    cudaEvent_t b = pool_event(H);
+    if (!b) { H->ev_pool.push_back(a); return; }
+    cudaEventRecord(b, s);
+    H->timed.push_back({cls, a, b});
+  }
+};
+
+static int validate_offsets(const int64_t* off, int64_t R, int64_t total, bool nonempty,
+                            const char* name) {
+  if (!off) return set_error(STCA_EINVAL, std::string(name) + " is NULL");
+  if (R < 1) return set_error(STCA_EINVAL, "R must be >= 1");
+  if (off[0] != 0) return set_error(STCA_EINVAL, std::string(name) + "[0] != 0");
+  for (int64_t r = 0; r < R; ++r) {
+    const int64_t len = off[r + 1] - off[r];
+    if (len < 0)
+      return set_error(STCA_EINVAL, std::string(name) + " decreases at index " +
+                                        std::to_string(r + 1));
+    if (nonempty && len == 0)
+      return set_error(STCA_EINVAL, std::string(name) + ": segment " + std::to_string(r) +
+                                        " is empty (an empty history has no softmax)");
+    if (len > INT32_MAX)
+      return set_error(STCA_EINVAL, std::string(name) + ": segment too long");
+  }
+  if (off[R] != total)
+    return set_error(STCA_EINVAL, std::string(name) + "[R] = " + std::to_string(off[R]) +
+                                      " != " + std::to_string(total));
+  return STCA_OK;
+}
+
+// ------------------------------------------------------------------ weights
+static float bf16_bits_to_float(uint16_t b) {
+  uint32_t u = static_cast<uint32_t>(b) << 16;
+  float f;
+  memcpy(&f, &u, 4);
+  return f;
+}
+
+// Copy `n` dtype elements from a host or device pointer into fp32.
+static int fetch(const void* src, size_t n, int dtype, bool on_device, std::vector<float>* out,
+                 const char* name) {
+  if (!src) return set_error(STCA_EINVAL, std::string("weight ") + name + " is NULL");
+  const size_t esz = dtype == STCA_BF16 ? 2 : 4;
+  std::vector<uint8_t> raw;
+  const uint8_t* p = static_cast<const uint8_t*>(src);
+  if (on_device) {
+    raw.resize(n * esz);
+    STCA_CUDA_TRY(cudaMemcpy(raw.data(), src, n * esz, cudaMemcpyDeviceToHost));
+    p = raw.data();
+  }
+  out->resize(n);
+  if (dtype == STCA_BF16) {
+    for (size_t i = 0; i < n; ++i) {
+      uint16_t b;
+      memcpy(&b, p + 2 * i, 2);
+      (*out)[i] = bf16_bits_to_float(b);
+    }
+  } else {
+    memcpy(out->data(), p, n * 4);
+  }
+  return STCA_OK;
+}
+
+static const void* layer_ptr(const void* const* field, int i) { return field ? field[i] : nullptr; }
+
+}  // namespace stca
+
+using namespace stca;
+
+// ====================================================================== ABI
+extern "C" const char* stca_last_error(void) { return g_err.c_str(); }
+
+extern "C" int stca_validate_offsets(const int64_t* offsets, int64_t R, int64_t total,
+                                     int require_nonempty) {
+  int rc = validate_offsets(offsets, R, total, require_nonempty != 0, "offsets");
+  return rc == STCA_OK ? ok() : rc;
+}
+
+extern "C" void stca_destroy(stca_handle* H) {
+  if (!H) return;
+  DeviceGuard g(H->device);
+  cudaDeviceSynchronize();
+  cudaFree(H->w32);
+  cudaFree(H->wtc);
+  cudaFree(H->xt);
+  cudaFree(H->q);
+  cudaFree(H->U);
+  cudaFree(H->Ubf);
+  cudaFree(H->part);
+  cudaFree(H->plan_d);
+  cudaFree(H->status_d);
+  cudaFree(H->x_stage);
+  cudaFree(H->t_stage);
+  cudaFree(H->z_stage);
+  if (H->plan_h) cudaFreeHost(H->plan_h);
+  if (H->plan_evt) cudaEventDestroy(H->plan_evt);
+  for (auto& t : H->timed) { cudaEventDestroy(t.a); cudaEventDestroy(t.b); }
+  for (auto e : H->ev_pool) cudaEventDestroy(e);
+  delete H;
+}
+
+extern "C" int stca_init(const stca_weights* w, int d, int h, int r, int M, int dtype,
+                         int weights_on_device, stca_handle** out) {
+  if (!out) return set_error(STCA_EINVAL, "out is NULL");
+  *out = nullptr;
+  if (!w) return set_error(STCA_EINVAL, "weights is NULL");
+  if (d < 8 || d > 1024 || d % 8) return set_error(STCA_EINVAL, "d must be in [8, 1024], d % 8 == 0");
+  if (h < 1 || d % h) return set_error(STCA_EINVAL, "h must divide d");
+  if (r < 1 || static_cast<int64_t>(r) * d > 4096) return set_error(STCA_EINVAL, "need 1 <= r, r*d <= 4096");
+  if (M < 1 || M > 16) return set_error(STCA_EINVAL, "M must be in [1, 16]");
+  if (dtype != STCA_F32 && dtype != STCA_BF16) return set_error(STCA_EINVAL, "dtype must be STCA_F32 or STCA_BF16");
+  if (!w->Wu || !w->Wg || !w->Wd || !w->Wq || !w->Wk || !w->Wv || !w->Wo)
+    return set_error(STCA_EINVAL, "a required weight field is NULL");
+  if (M > 1 && !w->Wc) return set_error(STCA_EINVAL, "Wc is NULL but M > 1");
+  const bool qffn = w->qWu || w->qWg || w->qWd;
+  if (qffn && !(w->qWu && w->qWg && w->qWd))
+    return set_error(STCA_EINVAL, "qWu, qWg and qWd must be given together");
+  if ((w->q_ln_gamma == nullptr) != (w->q_ln_beta == nullptr))
+    return set_error(STCA_EINVAL, "q_ln_gamma and q_ln_beta must be given together");
+  if ((w->ln_gamma == nullptr) != (w->ln_beta == nullptr))
+    return set_error(STCA_EINVAL, "ln_gamma and ln_beta must be given together");
+
+  stca_handle* H = new (std::nothrow) stca_handle();
+  if (!H) return set_error(STCA_ENOMEM, "host allocation failed");
+  if (cudaGetDevice(&H->device) != cudaSuccess) {
+    delete H;
+    cudaGetLastError();
+    return set_error(STCA_ECUDA, "no CUDA device");
+  }
+  H->d = d; H->h = h; H->r = r; H->M = M; H->dtype = dtype;
+  H->rd = r * d; H->dh = d / h;
+  H->elem = dtype == STCA_BF16 ? 2 : 4;
+  const int rd = H->rd, dh = H->dh;
+  const bool dev = weights_on_device != 0;
+  if (target_step_smem(H) > 227 * 1024) {
+    delete H;
+    return set_error(STCA_EINVAL, "per-target step needs more than 227 KB shared memory for these sizes");
+  }
+
+  // ---- fp32 slab: per layer Wu Wg Wd [qWu qWg qWd] ln_g ln_b Wq WkT Wv Wo [Wc]; then q_ln
+  std::vector<size_t> lay_off(M + 1, 0);
+  auto layer_floats = [&](int i) {
+    size_t n = 3 * static_cast<size_t>(d) * rd + 2 * static_cast<size_t>(d) + 4 * static_cast<size_t>(d) * d;
+    if (qffn) n += 3 * static_cast<size_t>(d) * rd;
+    if (i > 0) n += static_cast<size_t>(i + 1) * d * d;
+    return n;
+  };
+  for (int i = 0; i < M; ++i) lay_off[i + 1] = lay_off[i] + layer_floats(i);
+  const size_t total = lay_off[M] + 2 * static_cast<size_t>(d);
+  std::vector<float> slab(total, 0.f), tmp;
+  int rc = STCA_OK;
+  auto put = [&](size_t at, const void* src, size_t n, const char* name) -> int {
+    int e = fetch(src, n, dtype, dev, &tmp, name);
+    if (e) return e;
+    std::copy(tmp.begin(), tmp.end(), slab.begin() + at);
+    return STCA_OK;
+  };
+  struct Offs { size_t Wu, Wg, Wd, qWu, qWg, qWd, lg, lb, Wq, WkT, Wv, Wo, Wc; };
+  std::vector<Offs> offs(M);
+  for (int i = 0; i < M && rc == STCA_OK; ++i) {
+    size_t at = lay_off[i];
+    Offs& o = offs[i];
+    o.Wu = at; at += static_cast<size_t>(d) * rd;
+    o.Wg = at; at += static_cast<size_t>(d) * rd;
+    o.Wd = at; at += static_cast<size_t>(rd) * d;
+    if (qffn) {
+      o.qWu = at; at += static_cast<size_t>(d) * rd;
+      o.qWg = at; at += static_cast<size_t>(d) * rd;
+      o.qWd = at; at += static_cast<size_t>(rd) * d;
+    } else {
+      o.qWu = o.Wu; o.qWg = o.Wg; o.qWd = o.Wd;
+    }
+    o.lg = at; at += d;
+    o.lb = at; at += d;
+    o.Wq = at; at += static_cast<size_t>(d) * d;
+    o.WkT = at; at += static_cast<size_t>(d) * d;
+    o.Wv = at; at += static_cast<size_t>(d) * d;
+    o.Wo = at; at += static_cast<size_t>(d) * d;
+    o.Wc = 0;
+    if (i > 0) { o.Wc = at; at += static_cast<size_t>(i + 1) * d * d; }
+    if ((rc = put(o.Wu, w->Wu[i], static_cast<size_t>(d) * rd, "Wu"))) break;
+    if ((rc = put(o.Wg, w->Wg[i], static_cast<size_t>(d) * rd, "Wg"))) break;
+    if ((rc = put(o.Wd, w->Wd[i], static_cast<size_t>(rd) * d, "Wd"))) break;
+    if (qffn) {
+      if ((rc = put(o.qWu, w->qWu[i], static_cast<size_t>(d) * rd, "qWu"))) break;
+      if ((rc = put(o.qWg, w->qWg[i], static_cast<size_t>(d) * rd, "qWg"))) break;
+      if ((rc = put(o.qWd, w->qWd[i], static_cast<size_t>(rd) * d, "qWd"))) break;
+    }
+    if (w->ln_gamma) {
+      if ((rc = put(o.lg, layer_ptr(w->ln_gamma, i), d, "ln_gamma"))) break;
+      if ((rc = put(o.lb, layer_ptr(w->ln_beta, i), d, "ln_beta"))) break;
+    } else {
+      std::fill(slab.begin() + o.lg, slab.begin() + o.lg + d, 1.f);
+    }
+    if ((rc = put(o.Wq, w->Wq[i], static_cast<size_t>(d) * d, "Wq"))) break;
+    if ((rc = fetch(w->Wk[i], static_cast<size_t>(d) * d, dtype, dev, &tmp, "Wk"))) break;
+    for (int j = 0; j < h; ++j)          // WkT[j][c][k] = Wk[k][j*dh + c]
+      for (int c = 0; c < dh; ++c)
+        for (int k = 0; k < d; ++k)
+          slab[o.WkT + (static_cast<size_t>(j) * dh + c) * d + k] = tmp[static_cast<size_t>(k) * d + j * dh + c];
+    if ((rc = put(o.Wv, w->Wv[i], static_cast<size_t>(d) * d, "Wv"))) break;
+    if ((rc = put(o.Wo, w->Wo[i], static_cast<size_t>(d) * d, "Wo"))) break;
+    if (i > 0 && (rc = put(o.Wc, w->Wc[i], static_cast<size_t>(i + 1) * d * d, "Wc"))) break;
+  }
+  const size_t qlg = lay_off[M], qlb = qlg + d;
+  if (rc == STCA_OK) {
+    if (w->q_ln_gamma) {
+      if (!(rc = put(qlg, w->q_ln_gamma, d, "q_ln_gamma"))) rc = put(qlb, w->q_ln_beta, d, "q_ln_beta");
+    } else {
+      std::copy(slab.begin() + offs[0].lg, slab.begin() + offs[0].lg + d, slab.begin() + qlg);
+      std::copy(slab.begin() + offs[0].lb, slab.begin() + offs[0].lb + d, slab.begin() + qlb);
+    }
+  }
+  if (rc != STCA_OK) { delete H; return rc; }
+  if (cudaMalloc(&H->w32, total * sizeof(float)) != cudaSuccess ||
+      cudaMalloc(&H->status_d, sizeof(int)) != cudaSuccess) {
+    cudaGetLastError();
+    stca_destroy(H);
+    return set_error(STCA_ENOMEM, "weight allocation failed");
+  }
+  if (cudaMemcpy(H->w32, slab.data(), total * sizeof(float), cudaMemcpyHostToDevice) != cudaSuccess ||
+      cudaMemset(H->status_d, 0, sizeof(int)) != cudaSuccess ||
+      cudaEventCreateWithFlags(&H->plan_evt, cudaEventDisableTiming) != cudaSuccess) {
+    std::string m = cudaGetErrorString(cudaGetLastError());
+    stca_destroy(H);
+    return set_error(STCA_ECUDA, "weight upload failed: " + m);
+  }
+  H->L32.resize(M);
+  for (int i = 0; i < M; ++i) {
+    const Offs& o = offs[i];
+    LayerW32& L = H->L32[i];
+    L.Wu = H->w32 + o.Wu; L.Wg = H->w32 + o.Wg; L.Wd = H->w32 + o.Wd;
+    L.qWu = H->w32 + o.qWu; L.qWg = H->w32 + o.qWg; L.qWd = H->w32 + o.qWd;
+    L.ln_g = H->w32 + o.lg; L.ln_b = H->w32 + o.lb;
+    L.Wq = H->w32 + o.Wq; L.WkT = H->w32 + o.WkT;
+    L.Wv = H->w32 + o.Wv; L.Wo = H->w32 + o.Wo;
+    L.Wc = i > 0 ? H->w32 + o.Wc : nullptr;
+  }
+  H->q_ln_g = H->w32 + qlg;
+  H->q_ln_b = H->w32 + qlb;
+  *out = H;
+  return ok();
+}
+
+// ------------------------------------------------------------------ encode
+static int64_t choose_split(const stca_handle* H) {
+  if (H->opt_split_keys > 0) return H->opt_split_keys;
+  return 1024;
+}
+
+extern "C" int stca_encode(stca_handle* H, const void* X, const int64_t* offsets, int64_t R,
+                           int64_t N, void* stream) {
+  if (!H) return set_error(STCA_EINVAL, "handle is NULL");
+  if (!X) return set_error(STCA_EINVAL, "X is NULL");
+  if (reinterpret_cast<uintptr_t>(X) % 16) return set_error(STCA_EINVAL, "X must be 16-byte aligned");
+  if (N < 1) return set_error(STCA_EINVAL, "N must be >= 1");
+  if (int rc = validate_offsets(offsets, R, N, true, "offsets")) return rc;
+  DeviceGuard g(H->device);
+  if (!g.ok) return set_error(STCA_ECUDA, "cannot select the handle's device");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const size_t layer_bytes = static_cast<size_t>(N) * H->d * H->elem;
+  if (int rc = ensure_dev(&H->xt, &H->xt_cap, layer_bytes * H->M)) return rc;
+  H->encoded = false;
+  H->R = R;
+  H->N = N;
+  H->offsets_h.assign(offsets, offsets + R + 1);
+  // key ranges: each request's history cut into ranges of at most `split` keys
+  const int64_t split = choose_split(H);
+  H->items_h.clear();
+  H->req_item_begin.assign(R + 1, 0);
+  for (int64_t r = 0; r < R; ++r) {
+    H->req_item_begin[r] = static_cast<int32_t>(H->items_h.size());
+    for (int64_t k0 = offsets[r]; k0 < offsets[r + 1]; k0 += split) {
+      AttnItem it;
+      it.req = static_cast<int32_t>(r);
+      it.nkeys = static_cast<int32_t>(std::min<int64_t>(split, offsets[r + 1] - k0));
+      it.key0 = k0;
+      it.row_base = 0;
+      H->items_h.push_back(it);
+    }
+  }
+  H->req_item_begin[R] = static_cast<int32_t>(H->items_h.size());
+  H->last_toff.clear();          // plan must be rebuilt for the next forward
+  H->launches = 0;
+  const bool bf = H->dtype == STCA_BF16;
+  for (int i = 0; i < H->M; ++i) {
+    void* xti = static_cast<char*>(H->xt) + layer_bytes * i;
+    {
+      TimedLaunch tl(H, STCA_K_ENCODE, s);
+      launch_ffn_rows(X, bf, N, H->L32[i], true, H->L32[i].ln_g, H->L32[i].ln_b, xti, bf,
+                      H->d, H->rd, s);
+    }
+    H->launches++;
+    if (int rc = check_launch("encode")) return rc;
+  }
+  H->encoded = true;
+  return ok();
+}
+
+// ------------------------------------------------------------------ forward
+static size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+static int build_plan(stca_handle* H, const int64_t* toff, int64_t T, cudaStream_t s) {
+  const int64_t R = H->R;
+  if (!H->last_toff.empty() && static_cast<int64_t>(H->last_toff.size()) == R + 1 &&
+      std::equal(H->last_toff.begin(), H->last_toff.end(), toff))
+    return STCA_OK;   // same layout as the previous forward on this encode: plan is on device
+  const int h = H->h;
+  std::vector<AttnItem> items = H->items_h;
+  int64_t G = 0, npairs = 0;
+  for (auto& it : items) {
+    const int64_t Tr = toff[it.req + 1] - toff[it.req];
+    it.row_base = G;
+    G += Tr * h;
+    npairs += Tr;
+  }
+  const size_t n_items = items.size();
+  H->off_items = 0;
+  H->off_pairs = align256(H->off_items + n_items * sizeof(AttnItem));
+  H->off_treq = align256(H->off_pairs + static_cast<size_t>(npairs) * 2 * sizeof(int32_t));
+  H->off_toff = align256(H->off_treq + static_cast<size_t>(T) * sizeof(int32_t));
+  H->off_rib = align256(H->off_toff + static_cast<size_t>(R + 1) * sizeof(int64_t));
+  const size_t bytes = align256(H->off_rib + static_cast<size_t>(R + 1) * sizeof(int32_t));
+  // pinned staging: wait until the previous upload has left it
+  if (H->plan_h && cudaEventSynchronize(H->plan_evt) != cudaSuccess)
+    return set_error(STCA_ECUDA, "plan event wait failed");
+  if (bytes > H->plan_h_cap) {
+    if (H->plan_h) cudaFreeHost(H->plan_h);
+    H->plan_h = nullptr;
+    H->plan_h_cap = 0;
+    if (cudaMallocHost(&H->plan_h, bytes) != cudaSuccess) {
+      cudaGetLastError();
+      H->plan_h = nullptr;
+      return set_error(STCA_ENOMEM, "pinned plan buffer allocation failed");
+    }
+    H->plan_h_cap = bytes;
+  }
+  if (int rc = ensure_dev(&H->plan_d, &H->plan_cap, bytes)) return rc;
+  char* p = static_cast<char*>(H->plan_h);
+  memcpy(p + H->off_items, items.data(), n_items * sizeof(AttnItem));
+  int32_t* pairs = reinterpret_cast<int32_t*>(p + H->off_pairs);
+  int64_t q = 0;
+  for (size_t w = 0; w < n_items; ++w) {
+    const int64_t Tr = toff[items[w].req + 1] - toff[items[w].req];
+    for (int64_t tl = 0; tl < Tr; ++tl) {
+      pairs[2 * q] = static_cast<int32_t>(w);
+      pairs[2 * q + 1] = static_cast<int32_t>(tl);
+      ++q;
+    }
+  }
+  int32_t* treq = reinterpret_cast<int32_t*>(p + H->off_treq);
+  for (int64_t r = 0; r < R; ++r)
+    for (int64_t t = toff[r]; t < toff[r + 1]; ++t) treq[t] = static_cast<int32_t>(r);
+  memcpy(p + H->off_toff, toff, static_cast<size_t>(R + 1) * sizeof(int64_t));
+  memcpy(p + H->off_rib, H->req_item_begin.data(), static_cast<size_t>(R + 1) * sizeof(int32_t));
+  STCA_CUDA_TRY(cudaMemcpyAsync(H->plan_d, H->plan_h, bytes, cudaMemcpyHostToDevice, s));
+  STCA_CUDA_TRY(cudaEventRecord(H->plan_evt, s));
+  H->last_G = G;
+  H->last_pairs = npairs;
+  H->last_toff.assign(toff, toff + R + 1);
+  return STCA_OK;
+}
+
+extern "C" int stca_forward(stca_handle* H, const void* targets, const int64_t* target_offsets,
+                            int64_t T, float* Z, void* stream) {
+  if (!H) return set_error(STCA_EINVAL, "handle is NULL");
+  if (!H->encoded) return set_error(STCA_ESTATE, "stca_forward before a successful stca_encode");
+  if (T < 0) return set_error(STCA_EINVAL, "T must be >= 0");
+  if (int rc = validate_offsets(target_offsets, H->R, T, false, "target_offsets")) return rc;
+  if (T == 0) return ok();
+  if (!targets || !Z) return set_error(STCA_EINVAL, "targets or Z is NULL");
+  if (reinterpret_cast<uintptr_t>(targets) % 16 || reinterpret_cast<uintptr_t>(Z) % 16)
+    return set_error(STCA_EINVAL, "targets and Z must be 16-byte aligned");
+  DeviceGuard g(H->device);
+  if (!g.ok) return set_error(STCA_ECUDA, "cannot select the handle's device");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (attn_simt_smem(H) > 227 * 1024)
+    return set_error(STCA_EINVAL, "h * d too large for the CUDA-core attention kernel");
+  if (int rc = build_plan(H, target_offsets, T, s)) return rc;
+  const int d = H->d, h = H->h;
+  if (int rc = ensure_dev(reinterpret_cast<void**>(&H->U), &H->U_cap,
+                          static_cast<size_t>(T) * h * d * sizeof(float))) return rc;
+  if (int rc = ensure_dev(reinterpret_cast<void**>(&H->part), &H->part_cap,
+                          static_cast<size_t>(std::max<int64_t>(H->last_G, 1)) * (d + 2) * sizeof(float)))
+    return rc;
+  char* p = static_cast<char*>(H->plan_d);
+  const AttnItem* items_d = reinterpret_cast<const AttnItem*>(p + H->off_items);
+  const int32_t* pairs_d = reinterpret_cast<const int32_t*>(p + H->off_pairs);
+  const int32_t* treq_d = reinterpret_cast<const int32_t*>(p + H->off_treq);
+  const int64_t* toff_d = reinterpret_cast<const int64_t*>(p + H->off_toff);
+  const int32_t* rib_d = reinterpret_cast<const int32_t*>(p + H->off_rib);
+  const size_t layer_bytes = static_cast<size_t>(H->N) * d * H->elem;
+  {
+    TimedLaunch tl(H, STCA_K_STEP, s);
+    launch_target_step(H, -1, targets, T, treq_d, toff_d, rib_d, items_d, Z, s);
+  }
+  H->launches++;
+  if (int rc = check_launch("query init")) return rc;
+  for (int i = 0; i < H->M; ++i) {
+    const void* xti = static_cast<const char*>(H->xt) + layer_bytes * i;
+    {
+      TimedLaunch tl(H, STCA_K_ATTN, s);
+      launch_attn_simt(H, i, xti, items_d, pairs_d, H->last_pairs, toff_d, s);
+    }
+    H->launches++;
+    if (int rc = check_launch("attention")) return rc;
+    {
+      TimedLaunch tl(H, STCA_K_STEP, s);
+      launch_target_step(H, i, targets, T, treq_d, toff_d, rib_d, items_d, Z, s);
+    }
+    H->launches++;
+    if (int rc = check_launch("target step")) return rc;
+  }
+  return ok();
+}
+
+// ------------------------------------------------------------------ host entry
+extern "C" int stca_run_host(stca_handle* H, const void* X_host, const int64_t* offsets,
+                             int64_t R, int64_t N, const void* targets_host,
+                             const int64_t* target_offsets, int64_t T, float* Z_host,
+                             void* stream) {
+  if (!H) return set_error(STCA_EINVAL, "handle is NULL");
+  if (!X_host || (T > 0 && (!targets_host || !Z_host)))
+    return set_error(STCA_EINVAL, "a host buffer is NULL");
+  if (N < 1) return set_error(STCA_EINVAL, "N must be >= 1");
+  if (int rc = validate_offsets(offsets, R, N, true, "offsets")) return rc;
+  if (T < 0) return set_error(STCA_EINVAL, "T must be >= 0");
+  if (int rc = validate_offsets(target_offsets, R, T, false, "target_offsets")) return rc;
+  DeviceGuard g(H->device);
+  if (!g.ok) return set_error(STCA_ECUDA, "cannot select the handle's device");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const size_t xb = static_cast<size_t>(N) * H->d * H->elem;
+  const size_t tb = static_cast<size_t>(T) * H->d * H->elem;
+  const size_t zb = static_cast<size_t>(T) * H->M * H->d * sizeof(float);
+  if (int rc = ensure_dev(&H->x_stage, &H->x_stage_cap, xb)) return rc;
+  if (T > 0) {
+    if (int rc = ensure_dev(&H->t_stage, &H->t_stage_cap, tb)) return rc;
+    if (int rc = ensure_dev(reinterpret_cast<void**>(&H->z_stage), &H->z_stage_cap, zb)) return rc;
+  }
+  STCA_CUDA_TRY(cudaMemcpyAsync(H->x_stage, X_host, xb, cudaMemcpyHostToDevice, s));
+  if (T > 0) STCA_CUDA_TRY(cudaMemcpyAsync(H->t_stage, targets_host, tb, cudaMemcpyHostToDevice, s));
+  if (int rc = stca_encode(H, H->x_stage, offsets, R, N, stream)) return rc;
+  if (T > 0) {
+    if (int rc = stca_forward(H, H->t_stage, target_offsets, T, H->z_stage, stream)) return rc;
+    STCA_CUDA_TRY(cudaMemcpyAsync(Z_host, H->z_stage, zb, cudaMemcpyDeviceToHost, s));
+  }
+  STCA_CUDA_TRY(cudaStreamSynchronize(s));
+  return ok();
+}
+
+// ------------------------------------------------------------------ misc
+extern "C" int stca_device_status(stca_handle* H, void* stream) {
+  if (!H) return set_error(STCA_EINVAL, "handle is NULL");
+  DeviceGuard g(H->device);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  STCA_CUDA_TRY(cudaStreamSynchronize(s));
+  int st = 0;
+  STCA_CUDA_TRY(cudaMemcpy(&st, H->status_d, sizeof(int), cudaMemcpyDeviceToHost));
+  STCA_CUDA_TRY(cudaMemset(H->status_d, 0, sizeof(int)));
+  if (st) {
+    std::string m = "device status 0x" + std::to_string(st) + ":";
+    if (st & kStatusEncodeTimeout) m += " encoder gave up a bounded wait;";
+    if (st & kStatusAttnTimeout) m += " attention gave up a bounded wait;";
+    return set_error(STCA_EDEVICE, m);
+  }
+  return ok();
+}
+
+extern "C" int stca_set_option(stca_handle* H, int option, int64_t value) {
+  if (!H) return set_error(STCA_EINVAL, "handle is NULL");
+  switch (option) {
+    case STCA_OPT_ATTN_PATH:
+      if (value < 0 || value > 2) return set_error(STCA_EINVAL, "attention path must be 0, 1 or 2");
+      H->opt_attn_path = static_cast<int>(value);
+      return ok();
+    case STCA_OPT_ENCODE_PATH:
+      if (value < 0 || value > 2) return set_error(STCA_EINVAL, "encode path must be 0, 1 or 2");
+      H->opt_encode_path = static_cast<int>(value);
+      return ok();
+    case STCA_OPT_TIMING:
+      if (value != 0 && value != 1) return set_error(STCA_EINVAL, "timing must be 0 or 1");
+      H->timing = value != 0;
+      return ok();
+    case STCA_OPT_SPLIT_KEYS:
+      if (value < 0 || value % 128 || value > (int64_t(1) << 30))
+        return set_error(STCA_EINVAL, "split must be 0 or a positive multiple of 128");
+      H->opt_split_keys = value;
+      return ok();
+    default:
+      return set_error(STCA_EINVAL, "unknown or read-only option " + std::to_string(option));
+  }
+}
+
+extern "C" int stca_get_option(stca_handle* H, int option, int64_t* value) {
+  if (!H || !value) return set_error(STCA_EINVAL, "handle or value is NULL");
+  switch (option) {
+    case STCA_OPT_ATTN_PATH: *value = H->opt_attn_path; return ok();
+    case STCA_OPT_ENCODE_PATH: *value = H->opt_encode_path; return ok();
+    case STCA_OPT_SPLIT_KEYS: *value = H->opt_split_keys; return ok();
+    case STCA_OPT_TIMING: *value = H->timing ? 1 : 0; return ok();
+    case STCA_OPT_LAUNCHES: *value = H->launches; return ok();
+    default: return set_error(STCA_EINVAL, "unknown option " + std::to_string(option));
+  }
+}
+
+extern "C" int stca_kernel_times(stca_handle* H, double* ms, int64_t* launches, int n) {
+  if (!H) return set_error(STCA_EINVAL, "handle is NULL");
+  if (n < 0) return set_error(STCA_EINVAL, "n must be >= 0");
+  DeviceGuard g(H->device);
+  double acc[STCA_K_CLASSES] = {0, 0, 0};
+  int64_t cnt[STCA_K_CLASSES] = {0, 0, 0};
+  int rc = STCA_OK;
+  for (auto& t : H->timed) {
+    float v = 0.f;
+    if (rc == STCA_OK) {
+      cudaError_t e = cudaEventSynchronize(t.b);
+      if (e == cudaSuccess) e = cudaEventElapsedTime(&v, t.a, t.b);
+      if (e != cudaSuccess) rc = set_error(STCA_ECUDA, std::string("event timing: ") + cudaGetErrorString(e));
+    }
+    acc[t.cls] += v;
+    cnt[t.cls] += 1;
+    H->ev_pool.push_back(t.a);
+    H->ev_pool.push_back(t.b);
+  }
+  H->timed.clear();
+  if (rc != STCA_OK) return rc;
+  for (int c = 0; c < n && c < STCA_K_CLASSES; ++c) {
+    if (ms) ms[c] = acc[c];
+    if (launches) launches[c] = cnt[c];
+  }
+  return ok();
+}

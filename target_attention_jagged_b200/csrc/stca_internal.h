@@ -1,0 +1,125 @@
+// Internal declarations shared by the STCA library's translation units.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <string>
+#include <vector>
+
+#include "stca.h"
+
+namespace stca {
+
+// ---------------------------------------------------------------- errors
+int set_error(int code, const std::string& msg);
+
+#define STCA_CUDA_TRY(expr)                                                              \
+  do {                                                                                   \
+    cudaError_t _e = (expr);                                                             \
+    if (_e != cudaSuccess)                                                               \
+      return ::stca::set_error(STCA_ECUDA, std::string(#expr) + ": " + cudaGetErrorString(_e)); \
+  } while (0)
+
+// Device status word bits written by kernels that give up a bounded wait.
+enum : int { kStatusEncodeTimeout = 1, kStatusAttnTimeout = 2 };
+
+// ---------------------------------------------------------------- work plan
+// One attention work item: a contiguous key range of one request's history.
+struct AttnItem {
+  int32_t req;        // request index
+  int32_t nkeys;      // keys in this range (>= 1)
+  int64_t key0;       // first history row (absolute row in X~)
+  int64_t row_base;   // first partial row of this item (rows = T_r * h)
+};
+
+// Per-layer pointers into the handle's fp32 weight slab (CUDA-core kernels and
+// the per-target kernels).
+struct LayerW32 {
+  const float *Wu, *Wg, *Wd;        // history FFN: d x rd, d x rd, rd x d
+  const float *qWu, *qWg, *qWd;     // query FFN (aliases the history FFN by default)
+  const float *ln_g, *ln_b;         // d
+  const float *Wq;                  // d x d
+  const float *WkT;                 // h x d_h x d: WkT[j][c][k] = Wk[k][j*d_h + c]
+  const float *Wv, *Wo;             // d x d
+  const float *Wc;                  // (i+1)d x d, NULL for layer 0
+};
+
+// Per-layer pointers into the bf16 slab used by the tensor-core encoder.
+struct LayerWTc {
+  const uint16_t* W1;   // hidden-chunked [Wu | Wg] operand, see encode_tc.cu
+  const uint16_t* W2;   // Wd operand, see encode_tc.cu
+};
+
+}  // namespace stca
+
+struct stca_handle {
+  int device = 0;
+  int d = 0, h = 0, r = 0, M = 0, dtype = 0;
+  int rd = 0, dh = 0;
+  int elem = 4;                         // bytes per X / X~ element
+
+  // weights
+  float* w32 = nullptr;                 // fp32 slab
+  std::vector<stca::LayerW32> L32;
+  const float* q_ln_g = nullptr;
+  const float* q_ln_b = nullptr;
+  uint16_t* wtc = nullptr;              // bf16 slab for tensor-core kernels
+  std::vector<stca::LayerWTc> Ltc;
+
+  // options
+  int opt_attn_path = 0, opt_encode_path = 0;
+  int64_t opt_split_keys = 0;
+  int64_t launches = 0;
+  bool timing = false;
+  struct TimedRec { int cls; cudaEvent_t a, b; };
+  std::vector<TimedRec> timed;          // events recorded around launches
+  std::vector<cudaEvent_t> ev_pool;     // recycled events
+
+  // encoded state
+  bool encoded = false;
+  int64_t R = 0, N = 0;
+  std::vector<int64_t> offsets_h;
+  void* xt = nullptr;                   // M x N x d, elem bytes each
+  size_t xt_cap = 0;
+  std::vector<stca::AttnItem> items_h;  // key ranges of the last encode
+  std::vector<int32_t> req_item_begin;  // R+1
+
+  // forward workspace (device)
+  float* q = nullptr;       size_t q_cap = 0;      // T x d
+  float* U = nullptr;       size_t U_cap = 0;      // T x h x d (scaled)
+  uint16_t* Ubf = nullptr;  size_t Ubf_cap = 0;    // bf16 copy for tensor cores
+  float* part = nullptr;    size_t part_cap = 0;   // G x (d + 2)
+  void* plan_d = nullptr;   size_t plan_cap = 0;   // uploaded plan arrays
+  void* plan_h = nullptr;   size_t plan_h_cap = 0; // pinned staging
+  cudaEvent_t plan_evt = nullptr;
+  int* status_d = nullptr;
+
+  // host-buffer entry point staging
+  void* x_stage = nullptr;  size_t x_stage_cap = 0;
+  void* t_stage = nullptr;  size_t t_stage_cap = 0;
+  float* z_stage = nullptr; size_t z_stage_cap = 0;
+
+  // last forward's plan (reused when the same targets layout repeats)
+  std::vector<int64_t> last_toff;
+  int64_t last_G = 0, last_pairs = 0;
+  size_t off_items = 0, off_pairs = 0, off_treq = 0, off_toff = 0, off_rib = 0;
+};
+
+namespace stca {
+
+// ---------------------------------------------------------------- kernels
+// CUDA-core kernels (simt_kernels.cu)
+void launch_ffn_rows(const void* X, int x_is_bf16, int64_t nrows, const LayerW32& w,
+                     bool history_ffn, const float* ln_g, const float* ln_b, void* Y,
+                     int y_is_bf16, int d, int rd, cudaStream_t s);
+void launch_attn_simt(const stca_handle* H, int layer, const void* xt_layer,
+                      const AttnItem* items_d, const int32_t* pairs_d, int64_t npairs,
+                      const int64_t* toff_d, cudaStream_t s);
+void launch_target_step(const stca_handle* H, int layer, const void* targets, int64_t T,
+                        const int32_t* treq_d, const int64_t* toff_d, const int32_t* rib_d,
+                        const AttnItem* items_d, float* Z, cudaStream_t s);
+size_t target_step_smem(const stca_handle* H);
+size_t attn_simt_smem(const stca_handle* H);
+
+}  // namespace stca

@@ -1,0 +1,279 @@
+"""ctypes binding of libstca.so (include/stca.h): argument marshalling only.
+
+Every step of the STCA forward runs in the library's CUDA kernels; this module
+only turns tensors and arrays into pointers and sizes, and error codes into
+exceptions.  There is no fallback: if libstca.so is missing, importing this
+module raises.
+
+Functions carry the C names.  Device buffers are torch CUDA tensors; offsets
+are host int64 arrays; weights may be host numpy arrays or torch tensors
+(bf16 handles take torch.bfloat16 tensors or numpy uint16 bf16 bit patterns,
+fp32 handles take float32).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Sequence
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libstca.so")
+
+STCA_F32, STCA_BF16 = 0, 1
+STCA_OK, STCA_EINVAL, STCA_ESTATE, STCA_ENOMEM, STCA_ECUDA, STCA_EDEVICE = 0, -1, -2, -3, -4, -5
+STCA_OPT_ATTN_PATH, STCA_OPT_ENCODE_PATH, STCA_OPT_SPLIT_KEYS, STCA_OPT_TIMING = 1, 2, 3, 4
+STCA_OPT_LAUNCHES = 100
+STCA_K_ENCODE, STCA_K_ATTN, STCA_K_STEP, STCA_K_CLASSES = 0, 1, 2, 3
+_NAMES = {STCA_EINVAL: "EINVAL", STCA_ESTATE: "ESTATE", STCA_ENOMEM: "ENOMEM",
+          STCA_ECUDA: "ECUDA", STCA_EDEVICE: "EDEVICE"}
+
+EXPORTS = ("stca_init", "stca_destroy", "stca_encode", "stca_forward", "stca_run_host",
+           "stca_validate_offsets", "stca_device_status", "stca_set_option",
+           "stca_get_option", "stca_kernel_times", "stca_last_error")
+
+
+class StcaError(RuntimeError):
+    def __init__(self, code: int, msg: str):
+        super().__init__(f"STCA_{_NAMES.get(code, code)}: {msg}")
+        self.code = code
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with "
+                          "`python target_attention_jagged_b200/build.py`")
+    lib = ctypes.CDLL(LIB_PATH)
+    P, I, I64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64
+    PI64 = ctypes.POINTER(ctypes.c_int64)
+    lib.stca_init.argtypes = [P, I, I, I, I, I, I, ctypes.POINTER(P)]
+    lib.stca_destroy.argtypes = [P]
+    lib.stca_destroy.restype = None
+    lib.stca_encode.argtypes = [P, P, PI64, I64, I64, P]
+    lib.stca_forward.argtypes = [P, P, PI64, I64, P, P]
+    lib.stca_run_host.argtypes = [P, P, PI64, I64, I64, P, PI64, I64, P, P]
+    lib.stca_validate_offsets.argtypes = [PI64, I64, I64, I]
+    lib.stca_device_status.argtypes = [P, P]
+    lib.stca_set_option.argtypes = [P, I, I64]
+    lib.stca_get_option.argtypes = [P, I, PI64]
+    lib.stca_kernel_times.argtypes = [P, ctypes.POINTER(ctypes.c_double), PI64, I]
+    lib.stca_last_error.restype = ctypes.c_char_p
+    lib.stca_last_error.argtypes = []
+    for name in EXPORTS:
+        if name not in ("stca_destroy", "stca_last_error"):
+            getattr(lib, name).restype = ctypes.c_int
+    return lib
+
+
+_lib = _load()
+
+
+class _Weights(ctypes.Structure):
+    _fields_ = [(n, ctypes.POINTER(ctypes.c_void_p)) for n in (
+        "Wu", "Wg", "Wd", "ln_gamma", "ln_beta", "Wq", "Wk", "Wv", "Wo", "Wc",
+        "qWu", "qWg", "qWd")] + [("q_ln_gamma", ctypes.c_void_p), ("q_ln_beta", ctypes.c_void_p)]
+
+
+def stca_last_error() -> str:
+    return _lib.stca_last_error().decode()
+
+
+def _check(rc: int):
+    if rc != STCA_OK:
+        raise StcaError(rc, stca_last_error())
+
+
+def _offsets(a) -> np.ndarray:
+    a = np.ascontiguousarray(np.asarray(a, dtype=np.int64))
+    return a
+
+
+def _i64p(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_int64))
+
+
+def _stream_ptr(stream) -> Optional[int]:
+    if stream is None:
+        try:
+            import torch
+            if torch.cuda.is_available():
+                return torch.cuda.current_stream().cuda_stream
+        except Exception:
+            pass
+        return None
+    return getattr(stream, "cuda_stream", stream)
+
+
+def _host_buffer(a, dtype_code: int, keep: list) -> int:
+    """Pointer to a host copy of weight `a` in the handle's element type."""
+    try:
+        import torch
+        if isinstance(a, torch.Tensor):
+            a = a.detach().cpu()
+            if dtype_code == STCA_BF16:
+                if a.dtype != torch.bfloat16:
+                    raise TypeError("bf16 handle: weights must be torch.bfloat16")
+                a = a.contiguous().view(torch.int16).numpy().view(np.uint16)
+            else:
+                if a.dtype != torch.float32:
+                    raise TypeError("fp32 handle: weights must be torch.float32")
+                a = a.contiguous().numpy()
+    except ImportError:  # pragma: no cover
+        pass
+    a = np.ascontiguousarray(a)
+    want = np.uint16 if dtype_code == STCA_BF16 else np.float32
+    if a.dtype != want:
+        raise TypeError(f"weights must be {np.dtype(want).name} for this handle, got {a.dtype}")
+    keep.append(a)
+    return a.ctypes.data
+
+
+def stca_init(weights: dict, d: int, h: int, r: int, M: int, dtype: int) -> int:
+    """Create a handle from host weights (dict of per-layer lists, the keys of
+    stca_weights).  Returns the opaque handle (an int)."""
+    keep: list = []
+
+    def arr(key, optional=False, skip0=False):
+        v = weights.get(key)
+        if v is None:
+            if optional:
+                return None
+            raise ValueError(f"weight {key} missing")
+        if len(v) != M:
+            raise ValueError(f"weight {key} needs {M} entries")
+        ptrs = (ctypes.c_void_p * M)()
+        for i, a in enumerate(v):
+            if a is None:
+                if skip0 and i == 0:
+                    ptrs[i] = None
+                    continue
+                raise ValueError(f"weight {key}[{i}] is None")
+            ptrs[i] = _host_buffer(a, dtype, keep)
+        keep.append(ptrs)
+        return ctypes.cast(ptrs, ctypes.POINTER(ctypes.c_void_p))
+
+    w = _Weights()
+    for k in ("Wu", "Wg", "Wd", "Wq", "Wk", "Wv", "Wo"):
+        setattr(w, k, arr(k))
+    w.ln_gamma = arr("ln_g", optional=True)
+    w.ln_beta = arr("ln_b", optional=True)
+    w.Wc = arr("Wc", optional=(M == 1), skip0=True)
+    w.qWu = arr("qWu", optional=True)
+    w.qWg = arr("qWg", optional=True)
+    w.qWd = arr("qWd", optional=True)
+    w.q_ln_gamma = _host_buffer(weights["q_ln_g"], dtype, keep) if weights.get("q_ln_g") is not None else None
+    w.q_ln_beta = _host_buffer(weights["q_ln_b"], dtype, keep) if weights.get("q_ln_b") is not None else None
+    out = ctypes.c_void_p()
+    _check(_lib.stca_init(ctypes.byref(w), d, h, r, M, dtype, 0, ctypes.byref(out)))
+    return out.value
+
+
+def stca_destroy(handle: int) -> None:
+    _lib.stca_destroy(handle)
+
+
+def stca_encode(handle: int, X, offsets, stream=None) -> None:
+    """X: CUDA tensor (N x d) in the handle's dtype; offsets: host int64 (R+1)."""
+    off = _offsets(offsets)
+    R = off.shape[0] - 1
+    N = int(off[-1]) if R >= 0 else 0
+    _check(_lib.stca_encode(handle, X.data_ptr(), _i64p(off), R, N, _stream_ptr(stream)))
+
+
+def stca_forward(handle: int, targets, target_offsets, Z=None, stream=None):
+    """targets: CUDA tensor (T x d); returns Z (T x M x d fp32 CUDA tensor)."""
+    import torch
+    toff = _offsets(target_offsets)
+    T = int(toff[-1])
+    if Z is None:
+        raise ValueError("pass Z: a CUDA float32 tensor of shape (T, M, d)")
+    assert Z.dtype == torch.float32 and Z.is_cuda and Z.is_contiguous()
+    _check(_lib.stca_forward(handle, targets.data_ptr() if T > 0 else None, _i64p(toff), T,
+                             Z.data_ptr() if T > 0 else None, _stream_ptr(stream)))
+    return Z
+
+
+def stca_run_host(handle: int, X_host, offsets, targets_host, target_offsets, Z_host,
+                  stream=None) -> None:
+    """End-to-end on host buffers (numpy arrays or CPU tensors, ideally pinned)."""
+    off, toff = _offsets(offsets), _offsets(target_offsets)
+
+    def ptr(a):
+        return a.data_ptr() if hasattr(a, "data_ptr") else a.ctypes.data
+    _check(_lib.stca_run_host(handle, ptr(X_host), _i64p(off), off.shape[0] - 1, int(off[-1]),
+                              ptr(targets_host), _i64p(toff), int(toff[-1]), ptr(Z_host),
+                              _stream_ptr(stream)))
+
+
+def stca_validate_offsets(offsets, total: int, require_nonempty: bool = True) -> int:
+    off = _offsets(offsets)
+    return _lib.stca_validate_offsets(_i64p(off), off.shape[0] - 1, total, int(require_nonempty))
+
+
+def stca_device_status(handle: int, stream=None) -> None:
+    _check(_lib.stca_device_status(handle, _stream_ptr(stream)))
+
+
+def stca_set_option(handle: int, option: int, value: int) -> None:
+    _check(_lib.stca_set_option(handle, option, value))
+
+
+def stca_get_option(handle: int, option: int) -> int:
+    v = ctypes.c_int64()
+    _check(_lib.stca_get_option(handle, option, ctypes.byref(v)))
+    return v.value
+
+
+def stca_kernel_times(handle: int):
+    """{class: (ms, launches)} since the previous call (needs STCA_OPT_TIMING = 1)."""
+    ms = (ctypes.c_double * STCA_K_CLASSES)()
+    n = (ctypes.c_int64 * STCA_K_CLASSES)()
+    _check(_lib.stca_kernel_times(handle, ms, n, STCA_K_CLASSES))
+    names = ("encode", "attention", "target_step")
+    return {names[c]: (ms[c], n[c]) for c in range(STCA_K_CLASSES)}
+
+
+class Stca:
+    """Owning wrapper: Stca(weights, d, h, r, M, dtype) then encode / forward."""
+
+    def __init__(self, weights: dict, d: int, h: int, r: int, M: int, dtype: str = "bf16"):
+        self.d, self.h, self.r, self.M = d, h, r, M
+        self.dtype = STCA_BF16 if dtype == "bf16" else STCA_F32
+        self.handle = stca_init(weights, d, h, r, M, self.dtype)
+
+    def encode(self, X, offsets, stream=None):
+        stca_encode(self.handle, X, offsets, stream)
+
+    def forward(self, targets, target_offsets, Z=None, stream=None):
+        import torch
+        T = int(np.asarray(target_offsets)[-1])
+        if Z is None:
+            Z = torch.empty((T, self.M, self.d), dtype=torch.float32, device=targets.device)
+        return stca_forward(self.handle, targets, target_offsets, Z, stream)
+
+    def set_option(self, option: int, value: int):
+        stca_set_option(self.handle, option, value)
+
+    def get_option(self, option: int) -> int:
+        return stca_get_option(self.handle, option)
+
+    def status(self, stream=None):
+        stca_device_status(self.handle, stream)
+
+    def close(self):
+        if self.handle:
+            stca_destroy(self.handle)
+            self.handle = None
+
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *exc):
+        self.close()
+
+    def __del__(self):  # pragma: no cover
+        try:
+            self.close()
+        except Exception:
+            pass

@@ -1,0 +1,167 @@
+"""Parity of the CUDA path (through the C ABI) with the fp64 oracle.
+
+Every test runs the library on a seeded synthetic workload and compares Z
+element by element with the oracle on the same inputs (normwise per output
+vector; 1e-3 for fp32, 2e-2 for bf16).  The full-size configurations are
+compared on sampled requests (each request's Z depends only on its own
+history and targets), the small ones in full.
+"""
+import numpy as np
+import pytest
+
+from gen import make_config_workload, make_workload
+from oracle import stca_oracle as O
+from tests.gpu_helpers import TOL, normwise_err, rows_of, run_gpu, sampled_requests
+
+pytestmark = pytest.mark.gpu
+
+
+def check_full(wl, Z, tol=None):
+    want = O.forward_workload(wl)
+    err = normwise_err(Z, want)
+    assert err <= (tol or TOL[wl.dtype]), f"{wl.name}: normwise error {err:.3e}"
+    return err
+
+
+def check_sampled(wl, Z, k, seed=0):
+    reqs = sampled_requests(wl, k, seed)
+    got = O.forward_workload(wl, requests=reqs)
+    want = np.concatenate([got[r] for r in reqs])
+    err = normwise_err(Z[rows_of(wl, reqs)], want)
+    assert np.all(np.isfinite(Z)), "non-finite output"
+    assert err <= TOL[wl.dtype], f"{wl.name}: normwise error {err:.3e} on requests {reqs}"
+    return err
+
+
+# ------------------------------------------------------------ named configs
+
+def test_c1_full(gpu):
+    wl = make_config_workload("c1")
+    check_full(wl, run_gpu(wl, gpu))
+
+
+def test_c2_full(gpu):
+    wl = make_config_workload("c2")
+    check_full(wl, run_gpu(wl, gpu))
+
+
+@pytest.mark.parametrize("key,k", [("c3", 3), ("c4", 6), ("c5", 1)])
+def test_full_size_sampled(gpu, key, k):
+    wl = make_config_workload(key)
+    Z = run_gpu(wl, gpu)
+    check_sampled(wl, Z, k)
+
+
+# ------------------------------------------------------------ edge cases
+
+EDGE_L = [1, 2, 127, 128, 129, 257, 1000, 1021]
+EDGE_T = [1, 0, 3, 2, 1, 5, 2, 1]
+
+
+@pytest.mark.parametrize("dtype,d,h,M,r", [("bf16", 128, 4, 2, 2), ("f32", 64, 2, 3, 2),
+                                           ("bf16", 256, 8, 2, 2), ("bf16", 64, 4, 1, 4)])
+def test_ragged_edges(gpu, dtype, d, h, M, r):
+    wl = make_workload(lengths=EDGE_L, targets=EDGE_T, d=d, h=h, M=M, r=r, dtype=dtype,
+                       seed=100 + d + M)
+    check_full(wl, run_gpu(wl, gpu))
+
+
+def test_many_targets_per_request(gpu):
+    # T_r * h = 40 * 8 = 320 query rows: more than one 128-row tile
+    wl = make_workload(lengths=[700, 333], targets=[40, 17], d=128, h=8, M=2, r=2,
+                       dtype="bf16", seed=7)
+    check_full(wl, run_gpu(wl, gpu))
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_affine_ln_and_separate_query_ffn(gpu, dtype):
+    wl = make_workload(lengths=[300, 45, 1], targets=[2, 3, 1], d=128, h=4, M=3, r=2,
+                       dtype=dtype, seed=8, random_ln=True, distinct_query_ffn=True)
+    check_full(wl, run_gpu(wl, gpu))
+
+
+def test_small_width(gpu):
+    wl = make_workload(lengths=[37, 5], targets=[2, 1], d=16, h=2, M=2, r=1, dtype="f32",
+                       seed=9)
+    check_full(wl, run_gpu(wl, gpu))
+
+
+@pytest.mark.parametrize("split", [128, 256, 4096])
+def test_split_sizes_agree(gpu, split):
+    wl = make_workload(lengths=[1500, 129, 640], targets=[3, 2, 1], d=128, h=4, M=2, r=2,
+                       dtype="bf16", seed=10)
+    check_full(wl, run_gpu(wl, gpu, split=split))
+
+
+def test_single_token_history_equals_closed_form(gpu):
+    # L = 1: o = x~ W_V W_O whatever the query (softmax over one key)
+    wl = make_workload(lengths=[1, 1], targets=[3, 2], d=128, h=8, M=2, r=2, dtype="bf16",
+                       seed=11)
+    Z = run_gpu(wl, gpu)
+    W = wl.weights
+    for r in range(2):
+        Xr, _ = wl.request(r)
+        rows = slice(int(wl.target_offsets[r]), int(wl.target_offsets[r + 1]))
+        for i in range(2):
+            want = O.encode_history(Xr, W, i)[0] @ W["Wv"][i].astype(float) @ W["Wo"][i].astype(float)
+            assert normwise_err(Z[rows, i], np.broadcast_to(want, Z[rows, i].shape)) <= 2e-2
+
+
+# ------------------------------------------------------------ API behaviour
+
+def test_encode_once_forward_many(gpu):
+    import torch
+    import target_attention_jagged_b200 as S
+    from tests.gpu_helpers import storage_weights, to_device
+    wl = make_workload(lengths=[900, 50, 2000], targets=[4, 1, 2], d=128, h=4, M=2, r=2,
+                       dtype="bf16", seed=12)
+    wl2 = make_workload(lengths=[900, 50, 2000], targets=[0, 6, 3], d=128, h=4, M=2, r=2,
+                        dtype="bf16", seed=13)
+    wl2.X, wl2.weights = wl.X, wl.weights     # same histories, other targets
+    with S.Stca(storage_weights(wl), wl.d, wl.h, wl.r, wl.M, wl.dtype) as st:
+        st.encode(to_device(wl, wl.X, gpu), wl.offsets)
+        for w in (wl, wl2, wl):
+            Z = st.forward(to_device(w, w.targets, gpu), w.target_offsets)
+            torch.cuda.synchronize()
+            check_full(w, Z.cpu().numpy())
+        st.status()
+
+
+def test_run_host_matches_device(gpu):
+    import torch
+    import target_attention_jagged_b200 as S
+    from tests.gpu_helpers import storage_weights
+    wl = make_workload(lengths=[400, 77], targets=[3, 2], d=128, h=4, M=2, r=2, dtype="bf16",
+                       seed=14)
+    Zd = run_gpu(wl, gpu)
+    with S.Stca(storage_weights(wl), wl.d, wl.h, wl.r, wl.M, wl.dtype) as st:
+        Xh = torch.from_numpy(wl.storage(wl.X)).pin_memory()
+        th = torch.from_numpy(wl.storage(wl.targets)).pin_memory()
+        Zh = torch.empty((wl.T, wl.M, wl.d), dtype=torch.float32).pin_memory()
+        S.stca_run_host(st.handle, Xh, wl.offsets, th, wl.target_offsets, Zh)
+        assert np.array_equal(Zh.numpy(), Zd)
+
+
+def test_forward_before_encode_and_bad_offsets(gpu):
+    import torch
+    import target_attention_jagged_b200 as S
+    from tests.gpu_helpers import storage_weights, to_device
+    wl = make_workload(lengths=[10, 20], targets=[1, 1], d=64, h=2, M=1, r=1, dtype="f32",
+                       seed=15)
+    with S.Stca(storage_weights(wl), wl.d, wl.h, wl.r, wl.M, wl.dtype) as st:
+        xt = to_device(wl, wl.targets, gpu)
+        with pytest.raises(S.StcaError) as e:
+            st.forward(xt, wl.target_offsets)
+        assert e.value.code == -2
+        X = to_device(wl, wl.X, gpu)
+        with pytest.raises(S.StcaError) as e:
+            st.encode(X, [0, 30, 30])            # empty history
+        assert e.value.code == -1
+        with pytest.raises(S.StcaError):
+            st.encode(X, [0, 20, 10])            # decreasing
+        st.encode(X, wl.offsets)
+        with pytest.raises(S.StcaError):
+            st.forward(xt, [0, 1, 1, 2])         # wrong R
+        Z = torch.empty((0, 1, 64), device=gpu)
+        st.forward(xt[:0], [0, 0, 0], Z)         # T = 0 is a no-op
+        st.status()
