@@ -141,6 +141,14 @@ int stca_forward(stca_handle* handle, const void* targets, const int64_t* target
                  int64_t T, float* Z, void* stream);
 
 /*
+ * Copy the encoded history X~(layer+1) of the last stca_encode (N x d, dtype
+ * elements, the rows in the order of X) into `dst`, a device buffer the caller
+ * owns.  layer is 0-based.  Lets a caller keep or inspect the encoding of a
+ * request batch.  Errors: STCA_ESTATE (no encode yet), STCA_EINVAL, STCA_ECUDA.
+ */
+int stca_get_encoded(stca_handle* handle, int layer, void* dst, void* stream);
+
+/*
  * End-to-end call on HOST buffers: copies X and targets from host memory to
  * device staging buffers the handle owns, encodes, runs the forward, copies
  * Z (T x M x d fp32) back to host memory and waits for the stream.  Host

@@ -1,0 +1,469 @@
+// Tensor-core history encoder: X~(i) = LN_i(((X W_u) * SiLU(X W_g)) W_d) for all
+// M layers ("Make It Long, Keep It Fast" digest §2.1, Eqs. (1)-(2); the blog's
+// "high-throughput SwiGLU" and "optimised LayerNorm", §3.4).
+//
+// One persistent CTA per SM walks 128-row tiles of the jagged history buffer
+// (the rows of all requests, concatenated: the encoder is row-wise, so request
+// boundaries do not matter here).  Per tile it keeps the X tile in shared
+// memory for all M layers, and per layer streams the weights in hidden chunks
+// of 64 columns:
+//   GEMM1  acc1[128 x 128] = X_tile * [W_u | W_g/2]_chunk      (tcgen05, TMEM)
+//   gate   H[128 x 64]     = u * g' * (1 + tanh(g'))          (g' = g/2; CUDA cores)
+//   GEMM2  acc2[128 x d]  += H * W_d,chunk                    (tcgen05, TMEM)
+// then LayerNorm on acc2 and a bf16 store of the tile of X~(i).  The hidden
+// activations never leave the SM.  u * SiLU(g) = u * g' * (1 + tanh(g')) with
+// g' = g/2, so W_g is stored pre-halved (exact in bf16) and each gate value
+// costs one MUFU tanh.
+//
+// Warp roles (192 threads): warp 0 issues TMA loads, warp 1 issues the MMAs
+// (one thread) and owns the TMEM allocation, warps 2-5 run the gate and the
+// LayerNorm, each on its own 32-lane quarter of TMEM (one row per thread).
+// acc1 is double-buffered so GEMM1 of chunk c+1 overlaps the gate of chunk c.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <cstring>
+#include <string>
+#include <vector>
+
+#include "stca_internal.h"
+#include "tc_common.cuh"
+
+namespace stca {
+namespace {
+
+using namespace tc;
+
+struct EncParams {
+  int64_t N;                 // history rows
+  int ntiles;                // ceil(N / 128)
+  int M;                     // layers
+  int nchunk;                // rd / 64
+  uint8_t* xt;               // X~ base; layer i at xt + i * N * d * 2
+  const float* ln_g[16];
+  const float* ln_b[16];
+  int* status;
+};
+
+template <int D, int XB, int AB2, int S1, int S2>
+struct EncCfg {
+  static constexpr int KB = D / 64;                       // 64-wide K blocks of X
+  static constexpr uint32_t kBlock = 128u * 128u;         // [128 rows x 64] bf16
+  static constexpr uint32_t kXBytes = KB * kBlock;
+  static constexpr uint32_t kW1Stage = kBlock;            // [128 rows x 64]
+  static constexpr uint32_t kW2Stage = D * 128u;          // [D rows x 64]
+  static constexpr uint32_t oX = 0;
+  static constexpr uint32_t oW1 = oX + XB * kXBytes;
+  static constexpr uint32_t oW2 = oW1 + S1 * kW1Stage;
+  static constexpr uint32_t oH = oW2 + S2 * kW2Stage;
+  static constexpr uint32_t oBar = oH + 2 * kBlock;
+  static constexpr int kBars = 2 * S1 + 2 * S2 + 2 * XB + 4 + 4 + 2 * AB2 + 1;
+  static constexpr uint32_t oMisc = oBar + kBars * 8;
+  static constexpr uint32_t kSmem = oMisc + 16 + 1024;    // + alignment slack
+  static constexpr uint32_t kAcc1 = 0;                    // 2 x 128 columns
+  static constexpr uint32_t kAcc2 = 256;                  // AB2 x D columns
+  static_assert(kAcc2 + AB2 * D <= 512, "TMEM overflow");
+  static_assert(kSmem <= 227 * 1024, "shared memory overflow");
+};
+
+constexpr int kEncThreads = 192;
+
+__device__ __forceinline__ bool bwait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                      int* status) {
+  if (mbar_wait(bar, parity, abort_flag)) return true;
+  *abort_flag = 1;
+  atomicOr(status, kStatusEncodeTimeout);
+  return false;
+}
+
+// Wait without the abort shortcut, for at most `ns` (used while draining).
+__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, uint64_t ns) {
+  const uint64_t t0 = globaltimer();
+  while (!mbar_try_wait(bar, parity))
+    if (globaltimer() - t0 > ns) break;
+}
+
+template <int D, int XB, int AB2, int S1, int S2>
+__global__ void __launch_bounds__(kEncThreads, 1)
+encode_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW1,
+                 const __grid_constant__ CUtensorMap tmW2, const EncParams p) {
+  using C = EncCfg<D, XB, AB2, S1, S2>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                           ~static_cast<uintptr_t>(1023));
+  uint64_t* full1 = reinterpret_cast<uint64_t*>(sm + C::oBar);
+  uint64_t* empty1 = full1 + S1;
+  uint64_t* full2 = empty1 + S1;
+  uint64_t* empty2 = full2 + S2;
+  uint64_t* xfull = empty2 + S2;
+  uint64_t* xempty = xfull + XB;
+  uint64_t* a1full = xempty + XB;
+  uint64_t* a1empty = a1full + 2;
+  uint64_t* hfull = a1empty + 2;
+  uint64_t* hempty = hfull + 2;
+  uint64_t* a2full = hempty + 2;
+  uint64_t* a2empty = a2full + AB2;
+  uint64_t* mdrain = a2empty + AB2;         // completion of every MMA, before TMEM is freed
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + C::oMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + C::oMisc + 4);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < S1; ++i) { mbar_init(&full1[i], 1); mbar_init(&empty1[i], 1); }
+    for (int i = 0; i < S2; ++i) { mbar_init(&full2[i], 1); mbar_init(&empty2[i], 1); }
+    for (int i = 0; i < XB; ++i) { mbar_init(&xfull[i], 1); mbar_init(&xempty[i], 1); }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&a1full[i], 1); mbar_init(&a1empty[i], 4);
+      mbar_init(&hfull[i], 4); mbar_init(&hempty[i], 1);
+    }
+    for (int i = 0; i < AB2; ++i) { mbar_init(&a2full[i], 1); mbar_init(&a2empty[i], 4); }
+    mbar_init(mdrain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tmX);
+    prefetch_tmap(&tmW1);
+    prefetch_tmap(&tmW2);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t sbase = smem_u32(sm);
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      uint32_t r1 = 0, r2 = 0, xi = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < p.ntiles; tile += gridDim.x) {
+        const int xb = xi % XB;
+        if (!(ok = bwait(&xempty[xb], ((xi / XB) & 1) ^ 1, abort_flag, p.status))) break;
+        mbar_arrive_expect_tx(&xfull[xb], C::kXBytes);
+        for (int kb = 0; kb < C::KB; ++kb)
+          tma_load_2d(sm + C::oX + xb * C::kXBytes + kb * C::kBlock, &tmX, kb * 64, tile * 128,
+                      &xfull[xb]);
+        ++xi;
+        for (int layer = 0; ok && layer < p.M; ++layer) {
+          for (int c = 0; ok && c < p.nchunk; ++c) {
+            for (int kb = 0; kb < C::KB; ++kb) {
+              const int s = r1 % S1;
+              if (!(ok = bwait(&empty1[s], ((r1 / S1) & 1) ^ 1, abort_flag, p.status))) break;
+              mbar_arrive_expect_tx(&full1[s], C::kW1Stage);
+              tma_load_2d(sm + C::oW1 + s * C::kW1Stage, &tmW1, kb * 64,
+                          (layer * p.nchunk + c) * 128, &full1[s]);
+              ++r1;
+            }
+            if (!ok) break;
+            const int s = r2 % S2;
+            if (!(ok = bwait(&empty2[s], ((r2 / S2) & 1) ^ 1, abort_flag, p.status))) break;
+            mbar_arrive_expect_tx(&full2[s], C::kW2Stage);
+            tma_load_2d(sm + C::oW2 + s * C::kW2Stage, &tmW2, c * 64, layer * D, &full2[s]);
+            ++r2;
+          }
+        }
+      }
+      if (!ok) {   // let the copies already issued land before the CTA exits
+        for (uint32_t c = r1 > S1 ? r1 - S1 : 0; c < r1; ++c) drain_wait(&full1[c % S1], (c / S1) & 1, 100000000ull);
+        for (uint32_t c = r2 > S2 ? r2 - S2 : 0; c < r2; ++c) drain_wait(&full2[c % S2], (c / S2) & 1, 100000000ull);
+        for (uint32_t c = xi > XB ? xi - XB : 0; c < xi; ++c) drain_wait(&xfull[c % XB], (c / XB) & 1, 100000000ull);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc1 = idesc_bf16(128, 128);
+      constexpr uint32_t idesc2 = idesc_bf16(128, D);
+      uint32_t r1 = 0, r2 = 0, xc = 0, cc = 0, hc = 0, uc = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < p.ntiles; tile += gridDim.x, ++xc) {
+        const int xb = xc % XB;
+        if (!(ok = bwait(&xfull[xb], (xc / XB) & 1, abort_flag, p.status))) break;
+        tc_fence_after();
+        const uint32_t xaddr = sbase + C::oX + xb * C::kXBytes;
+        for (int layer = 0; ok && layer < p.M; ++layer, ++uc) {
+          const int b2 = uc % AB2;
+          const uint32_t acc2 = tmem + C::kAcc2 + b2 * D;
+          for (int c = 0; ok && c <= p.nchunk; ++c) {
+            if (c < p.nchunk) {
+              // GEMM1 of chunk c into acc1[cc & 1]
+              const int b = cc & 1;
+              if (!(ok = bwait(&a1empty[b], ((cc >> 1) & 1) ^ 1, abort_flag, p.status))) break;
+              tc_fence_after();
+              const uint32_t acc1 = tmem + C::kAcc1 + b * 128;
+              for (int kb = 0; kb < C::KB; ++kb) {
+                const int s = r1 % S1;
+                if (!(ok = bwait(&full1[s], (r1 / S1) & 1, abort_flag, p.status))) break;
+                tc_fence_after();
+                const uint32_t waddr = sbase + C::oW1 + s * C::kW1Stage;
+#pragma unroll
+                for (int k4 = 0; k4 < 4; ++k4)
+                  mma_bf16_ss(acc1, sdesc_sw128(xaddr + kb * C::kBlock + k4 * 32, 16, 1024),
+                              sdesc_sw128(waddr + k4 * 32, 16, 1024), idesc1, (kb | k4) != 0);
+                mma_commit(&empty1[s]);
+                ++r1;
+              }
+              if (!ok) break;
+              mma_commit(&a1full[b]);
+              if (layer == p.M - 1 && c == p.nchunk - 1) mma_commit(&xempty[xb]);
+              ++cc;
+            }
+            if (c >= 1) {
+              // GEMM2 of chunk c-1: acc2 += H[hc & 1] * W_d chunk
+              const int hb = hc & 1;
+              if (!(ok = bwait(&hfull[hb], (hc >> 1) & 1, abort_flag, p.status))) break;
+              tc_fence_after();
+              if (c == 1) {
+                if (!(ok = bwait(&a2empty[b2], ((uc / AB2) & 1) ^ 1, abort_flag, p.status))) break;
+                tc_fence_after();
+              }
+              const int s = r2 % S2;
+              if (!(ok = bwait(&full2[s], (r2 / S2) & 1, abort_flag, p.status))) break;
+              tc_fence_after();
+              const uint32_t haddr = sbase + C::oH + hb * C::kBlock;
+              const uint32_t waddr = sbase + C::oW2 + s * C::kW2Stage;
+#pragma unroll
+              for (int k4 = 0; k4 < 4; ++k4)
+                mma_bf16_ss(acc2, sdesc_sw128(haddr + k4 * 32, 16, 1024),
+                            sdesc_sw128(waddr + k4 * 32, 16, 1024), idesc2,
+                            ((c - 1) | k4) != 0);
+              mma_commit(&empty2[s]);
+              ++r2;
+              mma_commit(&hempty[hb]);
+              ++hc;
+            }
+          }
+          if (!ok) break;
+          mma_commit(&a2full[b2]);
+        }
+      }
+      // every MMA issued so far must finish before TMEM is released
+      mma_commit(mdrain);
+      drain_wait(mdrain, 0, 500000000ull);
+    }
+  } else {
+    // ------------------------------------------------------------ gate + LayerNorm
+    const int q = warp & 3;                    // TMEM lane quarter of this warp
+    const int row_in_tile = q * 32 + lane;
+    const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
+    uint32_t cc = 0, uc = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; ok && tile < p.ntiles; tile += gridDim.x) {
+      const int64_t row = static_cast<int64_t>(tile) * 128 + row_in_tile;
+      for (int layer = 0; ok && layer < p.M; ++layer, ++uc) {
+        for (int c = 0; c < p.nchunk; ++c, ++cc) {
+          const int b = cc & 1;
+          const uint32_t ph = (cc >> 1) & 1;
+          if (!(ok = bwait(&a1full[b], ph, abort_flag, p.status))) break;
+          __syncwarp();
+          tc_fence_after();
+          uint32_t packed[32];
+#pragma unroll
+          for (int half = 0; half < 2; ++half) {
+            uint32_t u[32], g[32];
+            const uint32_t a = tmem + lane_off + C::kAcc1 + b * 128 + half * 32;
+            tmem_ld32(a, u);
+            tmem_ld32(a + 64, g);
+            tmem_ld_wait();
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              const float g0 = __uint_as_float(g[2 * j]), g1 = __uint_as_float(g[2 * j + 1]);
+              const float p0 = __uint_as_float(u[2 * j]) * g0;
+              const float p1 = __uint_as_float(u[2 * j + 1]) * g1;
+              packed[half * 16 + j] =
+                  pack_bf16x2(fmaf(p0, tanh_approx(g0), p0), fmaf(p1, tanh_approx(g1), p1));
+            }
+          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&a1empty[b]);
+          if (!(ok = bwait(&hempty[b], ph ^ 1, abort_flag, p.status))) break;
+          __syncwarp();
+          const uint32_t hrow = sbase + C::oH + b * C::kBlock + row_in_tile * 128;
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            st_shared_v4(hrow + ((j ^ (row_in_tile & 7)) << 4), packed[4 * j], packed[4 * j + 1],
+                         packed[4 * j + 2], packed[4 * j + 3]);
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&hfull[b]);
+        }
+        if (!ok) break;
+        // LayerNorm of the finished rows, bf16 store of X~(layer)
+        const int b2 = uc % AB2;
+        if (!(ok = bwait(&a2full[b2], (uc / AB2) & 1, abort_flag, p.status))) break;
+        __syncwarp();
+        tc_fence_after();
+        const uint32_t a2 = tmem + lane_off + C::kAcc2 + b2 * D;
+        float shift = 0.f, s1 = 0.f, s2 = 0.f;
+#pragma unroll 1
+        for (int cb = 0; cb < D / 32; ++cb) {
+          uint32_t v[32];
+          tmem_ld32(a2 + cb * 32, v);
+          tmem_ld_wait();
+          if (cb == 0) shift = __uint_as_float(v[0]);
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const float x = __uint_as_float(v[j]) - shift;
+            s1 += x;
+            s2 = fmaf(x, x, s2);
+          }
+        }
+        const float m1 = s1 * (1.0f / D);
+        const float var = fmaxf(s2 * (1.0f / D) - m1 * m1, 0.f);
+        const float mean = shift + m1;
+        const float rstd = rsqrtf(var + 1e-5f);
+        const float* gam = p.ln_g[layer];
+        const float* bet = p.ln_b[layer];
+        uint8_t* orow = p.xt + (static_cast<int64_t>(layer) * p.N + row) * (D * 2);
+#pragma unroll 1
+        for (int cb = 0; cb < D / 32; ++cb) {
+          uint32_t v[32];
+          tmem_ld32(a2 + cb * 32, v);
+          tmem_ld_wait();
+          uint32_t o[16];
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const int k = cb * 32 + 2 * j;
+            const float y0 = (__uint_as_float(v[2 * j]) - mean) * rstd * __ldg(gam + k) + __ldg(bet + k);
+            const float y1 = (__uint_as_float(v[2 * j + 1]) - mean) * rstd * __ldg(gam + k + 1) +
+                             __ldg(bet + k + 1);
+            o[j] = pack_bf16x2(y0, y1);
+          }
+          if (row < p.N) {
+            uint4* dst = reinterpret_cast<uint4*>(orow + cb * 64);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) dst[k] = make_uint4(o[4 * k], o[4 * k + 1], o[4 * k + 2], o[4 * k + 3]);
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&a2empty[b2]);
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ------------------------------------------------------------------ host side
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+    else
+      cudaGetLastError();
+  }
+  return fn;
+}
+
+template <int D, int XB, int AB2, int S1, int S2>
+int launch_cfg(stca_handle* H, const CUtensorMap& tmX, const EncParams& p, cudaStream_t s) {
+  using C = EncCfg<D, XB, AB2, S1, S2>;
+  auto k = encode_tc_kernel<D, XB, AB2, S1, S2>;
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+  if (e != cudaSuccess) return set_error(STCA_ECUDA, std::string("encode_tc smem: ") + cudaGetErrorString(e));
+  const int grid = std::min(p.ntiles, H->num_sms);
+  k<<<grid, kEncThreads, C::kSmem, s>>>(tmX, H->tmW1, H->tmW2, p);
+  return STCA_OK;
+}
+
+}  // namespace
+
+int make_tmap_bf16_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer,
+                      uint32_t box_inner, uint32_t box_outer) {
+  auto fn = encode_fn();
+  if (!fn) return set_error(STCA_ECUDA, "cuTensorMapEncodeTiled is unavailable");
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {inner * 2};
+  const cuuint32_t box[2] = {box_inner, box_outer};
+  const cuuint32_t es[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+                  box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS)
+    return set_error(STCA_ECUDA, "cuTensorMapEncodeTiled failed (" + std::to_string(int(r)) + ")");
+  return STCA_OK;
+}
+
+bool encode_tc_supported(int d, int rd) {
+  return (d == 64 || d == 128 || d == 256) && rd % 64 == 0 && rd >= 64;
+}
+
+// Lay out the tensor-core operands of all layers and build their tensor maps.
+//   W1T: rows (layer, chunk c, j): j < 64 -> column c*64+j of W_u; j >= 64 ->
+//        column c*64+j-64 of W_g times 1/2; each row holds d values (K-major).
+//   W2T: rows (layer, n) = column n of W_d, rd values each (K-major).
+int encode_tc_setup(stca_handle* H, const std::vector<const float*>& Wu,
+                    const std::vector<const float*>& Wg, const std::vector<const float*>& Wd) {
+  const int d = H->d, rd = H->rd, M = H->M, nchunk = rd / 64;
+  const size_t w1_rows = static_cast<size_t>(M) * nchunk * 128;
+  const size_t w2_rows = static_cast<size_t>(M) * d;
+  std::vector<uint16_t> host(w1_rows * d + w2_rows * rd);
+  auto bf = [](float f) {
+    uint32_t u;
+    memcpy(&u, &f, 4);
+    return static_cast<uint16_t>(u >> 16);   // values are bf16-exact already
+  };
+  for (int i = 0; i < M; ++i)
+    for (int c = 0; c < nchunk; ++c)
+      for (int j = 0; j < 128; ++j) {
+        uint16_t* dst = host.data() + ((static_cast<size_t>(i) * nchunk + c) * 128 + j) * d;
+        const int col = c * 64 + (j & 63);
+        for (int k = 0; k < d; ++k)
+          dst[k] = j < 64 ? bf(Wu[i][static_cast<size_t>(k) * rd + col])
+                          : bf(0.5f * Wg[i][static_cast<size_t>(k) * rd + col]);
+      }
+  uint16_t* w2 = host.data() + w1_rows * d;
+  for (int i = 0; i < M; ++i)
+    for (int n = 0; n < d; ++n)
+      for (int k = 0; k < rd; ++k)
+        w2[(static_cast<size_t>(i) * d + n) * rd + k] = bf(Wd[i][static_cast<size_t>(k) * d + n]);
+  if (cudaMalloc(&H->wtc, host.size() * 2) != cudaSuccess) {
+    cudaGetLastError();
+    return set_error(STCA_ENOMEM, "tensor-core weight allocation failed");
+  }
+  STCA_CUDA_TRY(cudaMemcpy(H->wtc, host.data(), host.size() * 2, cudaMemcpyHostToDevice));
+  if (int rc = make_tmap_bf16_2d(&H->tmW1, H->wtc, d, w1_rows, 64, 128)) return rc;
+  if (int rc = make_tmap_bf16_2d(&H->tmW2, H->wtc + w1_rows * d, rd, w2_rows, 64, d)) return rc;
+  H->tc_encode_ready = true;
+  return STCA_OK;
+}
+
+int launch_encode_tc(stca_handle* H, const void* X, int64_t N, cudaStream_t s) {
+  CUtensorMap tmX;
+  if (int rc = make_tmap_bf16_2d(&tmX, X, H->d, N, 64, 128)) return rc;
+  EncParams p{};
+  p.N = N;
+  p.ntiles = static_cast<int>((N + 127) / 128);
+  p.M = H->M;
+  p.nchunk = H->rd / 64;
+  p.xt = static_cast<uint8_t*>(H->xt);
+  for (int i = 0; i < H->M; ++i) {
+    p.ln_g[i] = H->L32[i].ln_g;
+    p.ln_b[i] = H->L32[i].ln_b;
+  }
+  p.status = H->status_d;
+  switch (H->d) {
+    case 64: return launch_cfg<64, 2, 2, 4, 4>(H, tmX, p, s);
+    case 128: return launch_cfg<128, 2, 2, 4, 3>(H, tmX, p, s);
+    case 256: return launch_cfg<256, 1, 1, 3, 2>(H, tmX, p, s);
+    default: return set_error(STCA_EINVAL, "tensor-core encoder needs d in {64, 128, 256}");
+  }
+}
+
+}  // namespace stca

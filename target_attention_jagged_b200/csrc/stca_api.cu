@@ -323,6 +323,22 @@ extern "C" int stca_init(const stca_weights* w, int d, int h, int r, int M, int 
   }
   H->q_ln_g = H->w32 + qlg;
   H->q_ln_b = H->w32 + qlb;
+  if (cudaDeviceGetAttribute(&H->num_sms, cudaDevAttrMultiProcessorCount, H->device) != cudaSuccess) {
+    cudaGetLastError();
+    H->num_sms = 148;
+  }
+  if (dtype == STCA_BF16 && encode_tc_supported(d, rd)) {
+    std::vector<const float*> Wu(M), Wg(M), Wd(M);
+    for (int i = 0; i < M; ++i) {
+      Wu[i] = slab.data() + offs[i].Wu;
+      Wg[i] = slab.data() + offs[i].Wg;
+      Wd[i] = slab.data() + offs[i].Wd;
+    }
+    if (int rc2 = encode_tc_setup(H, Wu, Wg, Wd)) {
+      stca_destroy(H);
+      return rc2;
+    }
+  }
   *out = H;
   return ok();
 }
@@ -368,15 +384,28 @@ extern "C" int stca_encode(stca_handle* H, const void* X, const int64_t* offsets
   H->last_toff.clear();          // plan must be rebuilt for the next forward
   H->launches = 0;
   const bool bf = H->dtype == STCA_BF16;
-  for (int i = 0; i < H->M; ++i) {
-    void* xti = static_cast<char*>(H->xt) + layer_bytes * i;
+  if (H->opt_encode_path == 2 && !H->tc_encode_ready)
+    return set_error(STCA_EINVAL, "tensor-core encoder needs bf16 and d in {64,128,256}, rd % 64 == 0");
+  if (H->tc_encode_ready && H->opt_encode_path != 1) {
+    int rc;
     {
       TimedLaunch tl(H, STCA_K_ENCODE, s);
-      launch_ffn_rows(X, bf, N, H->L32[i], true, H->L32[i].ln_g, H->L32[i].ln_b, xti, bf,
-                      H->d, H->rd, s);
+      rc = launch_encode_tc(H, X, N, s);
     }
+    if (rc) return rc;
     H->launches++;
-    if (int rc = check_launch("encode")) return rc;
+    if (int rc2 = check_launch("encode (tensor cores)")) return rc2;
+  } else {
+    for (int i = 0; i < H->M; ++i) {
+      void* xti = static_cast<char*>(H->xt) + layer_bytes * i;
+      {
+        TimedLaunch tl(H, STCA_K_ENCODE, s);
+        launch_ffn_rows(X, bf, N, H->L32[i], true, H->L32[i].ln_g, H->L32[i].ln_b, xti, bf,
+                        H->d, H->rd, s);
+      }
+      H->launches++;
+      if (int rc = check_launch("encode")) return rc;
+    }
   }
   H->encoded = true;
   return ok();
@@ -496,6 +525,18 @@ extern "C" int stca_forward(stca_handle* H, const void* targets, const int64_t* 
     H->launches++;
     if (int rc = check_launch("target step")) return rc;
   }
+  return ok();
+}
+
+extern "C" int stca_get_encoded(stca_handle* H, int layer, void* dst, void* stream) {
+  if (!H) return set_error(STCA_EINVAL, "handle is NULL");
+  if (!H->encoded) return set_error(STCA_ESTATE, "no encoded history");
+  if (layer < 0 || layer >= H->M) return set_error(STCA_EINVAL, "layer out of range");
+  if (!dst) return set_error(STCA_EINVAL, "dst is NULL");
+  DeviceGuard g(H->device);
+  const size_t bytes = static_cast<size_t>(H->N) * H->d * H->elem;
+  STCA_CUDA_TRY(cudaMemcpyAsync(dst, static_cast<const char*>(H->xt) + bytes * layer, bytes,
+                                cudaMemcpyDeviceToDevice, static_cast<cudaStream_t>(stream)));
   return ok();
 }
 

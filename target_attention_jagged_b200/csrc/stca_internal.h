@@ -1,6 +1,7 @@
 // Internal declarations shared by the STCA library's translation units.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -45,12 +46,6 @@ struct LayerW32 {
   const float *Wc;                  // (i+1)d x d, NULL for layer 0
 };
 
-// Per-layer pointers into the bf16 slab used by the tensor-core encoder.
-struct LayerWTc {
-  const uint16_t* W1;   // hidden-chunked [Wu | Wg] operand, see encode_tc.cu
-  const uint16_t* W2;   // Wd operand, see encode_tc.cu
-};
-
 }  // namespace stca
 
 struct stca_handle {
@@ -64,8 +59,10 @@ struct stca_handle {
   std::vector<stca::LayerW32> L32;
   const float* q_ln_g = nullptr;
   const float* q_ln_b = nullptr;
-  uint16_t* wtc = nullptr;              // bf16 slab for tensor-core kernels
-  std::vector<stca::LayerWTc> Ltc;
+  uint16_t* wtc = nullptr;              // bf16 operands of the tensor-core encoder
+  CUtensorMap tmW1, tmW2;               // their TMA descriptors
+  bool tc_encode_ready = false;
+  int num_sms = 148;
 
   // options
   int opt_attn_path = 0, opt_encode_path = 0;
@@ -121,5 +118,13 @@ void launch_target_step(const stca_handle* H, int layer, const void* targets, in
                         const AttnItem* items_d, float* Z, cudaStream_t s);
 size_t target_step_smem(const stca_handle* H);
 size_t attn_simt_smem(const stca_handle* H);
+
+// Tensor-core encoder (encode_tc.cu)
+bool encode_tc_supported(int d, int rd);
+int encode_tc_setup(stca_handle* H, const std::vector<const float*>& Wu,
+                    const std::vector<const float*>& Wg, const std::vector<const float*>& Wd);
+int launch_encode_tc(stca_handle* H, const void* X, int64_t N, cudaStream_t s);
+int make_tmap_bf16_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer,
+                      uint32_t box_inner, uint32_t box_outer);
 
 }  // namespace stca

@@ -31,7 +31,7 @@ _NAMES = {STCA_EINVAL: "EINVAL", STCA_ESTATE: "ESTATE", STCA_ENOMEM: "ENOMEM",
 
 EXPORTS = ("stca_init", "stca_destroy", "stca_encode", "stca_forward", "stca_run_host",
            "stca_validate_offsets", "stca_device_status", "stca_set_option",
-           "stca_get_option", "stca_kernel_times", "stca_last_error")
+           "stca_get_option", "stca_kernel_times", "stca_get_encoded", "stca_last_error")
 
 
 class StcaError(RuntimeError):
@@ -57,6 +57,7 @@ def _load():
     lib.stca_device_status.argtypes = [P, P]
     lib.stca_set_option.argtypes = [P, I, I64]
     lib.stca_get_option.argtypes = [P, I, PI64]
+    lib.stca_get_encoded.argtypes = [P, I, P, P]
     lib.stca_kernel_times.argtypes = [P, ctypes.POINTER(ctypes.c_double), PI64, I]
     lib.stca_last_error.restype = ctypes.c_char_p
     lib.stca_last_error.argtypes = []
@@ -223,6 +224,12 @@ def stca_get_option(handle: int, option: int) -> int:
     v = ctypes.c_int64()
     _check(_lib.stca_get_option(handle, option, ctypes.byref(v)))
     return v.value
+
+
+def stca_get_encoded(handle: int, layer: int, dst, stream=None):
+    """Copy X~(layer+1) of the last encode into `dst` (CUDA tensor, N x d)."""
+    _check(_lib.stca_get_encoded(handle, layer, dst.data_ptr(), _stream_ptr(stream)))
+    return dst
 
 
 def stca_kernel_times(handle: int):
