@@ -8,6 +8,7 @@ from .workloads import (  # noqa: F401
     CONFIGS,
     Workload,
     bf16_bits_to_f32,
+    config_shapes,
     f32_to_bf16_bits,
     make_config_workload,
     make_workload,

@@ -223,6 +223,16 @@ def make_workload(*, lengths, targets, d, h, M, r, dtype="bf16", seed=0,
                     X=X, targets=xt, weights=W)
 
 
+def config_shapes(key: str, seed=None):
+    """History lengths and target counts of configuration `key` without drawing
+    the embeddings: the same first two draws as make_config_workload."""
+    cfg = CONFIGS[key]
+    rng = np.random.default_rng(cfg["seed"] if seed is None else seed)
+    L = _draw_lengths(cfg["lengths"], cfg["R"], rng)
+    Tr = _draw_targets(cfg["targets"], cfg["R"], rng)
+    return L, Tr, _offsets(L), _offsets(Tr)
+
+
 def make_config_workload(key: str, **overrides) -> Workload:
     """The named configuration `key` ("c1".."c5"), optionally with overrides."""
     cfg = dict(CONFIGS[key])

@@ -168,6 +168,25 @@ int stca_validate_offsets(const int64_t* offsets, int64_t R, int64_t total,
                           int require_nonempty);
 
 /*
+ * Host only, no device needed: the attention work split the library uses for a
+ * batch (the same planner stca_forward runs).  path 1: CUDA-core kernel, items
+ * are key ranges of at most split_keys (default 1024) keys over all T_r * h
+ * query rows.  path 2: tensor-core kernel, (request, 128-row query tile) pairs
+ * cut into num_ctas runs of equal numbers of 128-key tiles (capped at
+ * split_keys / 128 tiles when split_keys > 0), one run per CTA; each maximal
+ * run inside a pair is an item.  Outputs: *n_items, *grid (CTAs, path 2),
+ * *partial_rows; when `items` is not NULL, 7 int64 per item (request, query
+ * tile, first key row, keys, first query row, query rows, first partial row);
+ * when `cta_begin` is not NULL (path 2), grid + 1 item indices.  The plan is
+ * checked against the invariants the kernels rely on; a violation returns
+ * STCA_EINVAL.  Offsets follow stca_encode / stca_forward.
+ */
+int stca_plan_attention(const int64_t* offsets, const int64_t* target_offsets, int64_t R,
+                        int h, int path, int num_ctas, int64_t split_keys, int64_t* n_items,
+                        int64_t* grid, int64_t* partial_rows, int64_t* items, int64_t items_cap,
+                        int32_t* cta_begin, int64_t cta_cap);
+
+/*
  * Wait for the handle's work on `stream` and read its device status word.
  * STCA_OK, or STCA_EDEVICE if a kernel gave up a bounded wait (the message
  * names the kernel), or STCA_ECUDA.  The status is cleared by the read.

@@ -23,6 +23,7 @@ from .stca import (  # noqa: F401
     stca_kernel_times,
     stca_init,
     stca_last_error,
+    stca_plan_attention,
     stca_run_host,
     stca_set_option,
     stca_validate_offsets,

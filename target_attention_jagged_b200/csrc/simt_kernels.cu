@@ -205,10 +205,7 @@ struct StepArgs {
   int layer, M, d, h, dh, rd;
   int64_t T;
   const void* targets;
-  const int32_t* treq;
-  const int64_t* toff;
-  const int32_t* rib;
-  const AttnItem* items;
+  StepPlan plan;
   const float *pacc, *pm, *pl;
   float* Z;
   float* U;
@@ -272,25 +269,31 @@ __global__ void __launch_bounds__(kThreads) target_step_kernel(StepArgs a) {
   const int layer = a.layer;
   if (layer >= 0) {
     // split combine: c_j = sum_w e^{m_w - m} acc_w / sum_w e^{m_w - m} l_w
+    const StepPlan& P = a.plan;
     for (int pr = warp; pr < nb * h; pr += blockDim.x / 32) {
       const int b = pr / h, j = pr - b * h;
       const int64_t t = t0 + b;
-      const int r = a.treq[t];
-      const int64_t row = (t - a.toff[r]) * h + j;
-      const int w0 = a.rib[r], w1 = a.rib[r + 1];
+      const int r = P.treq[t];
+      const int64_t qrow = (t - P.toff[r]) * h + j;
+      const int64_t mt = qrow / P.mtile_rows;
+      const int64_t row = qrow - mt * P.mtile_rows;
+      const int pair = P.req_pair_begin[r] + static_cast<int>(mt);
+      const int w0 = P.pair_item_begin[pair], w1 = P.pair_item_begin[pair + 1];
       float mx = -INFINITY;
-      for (int w = w0; w < w1; ++w) mx = fmaxf(mx, a.pm[a.items[w].row_base + row]);
+      for (int w = w0; w < w1; ++w) mx = fmaxf(mx, a.pm[P.items[w].row_base + row]);
       float l = 0.f;
       for (int w = w0; w < w1; ++w) {
-        const int64_t g = a.items[w].row_base + row;
-        l = fmaf(a.pl[g], expf(a.pm[g] - mx), l);
+        const int64_t g = P.items[w].row_base + row;
+        const float f = P.log2_partials ? exp2f(a.pm[g] - mx) : expf(a.pm[g] - mx);
+        l = fmaf(a.pl[g], f, l);
       }
       const float inv = 1.0f / l;
       for (int k = lane; k < d; k += 32) {
         float v = 0.f;
         for (int w = w0; w < w1; ++w) {
-          const int64_t g = a.items[w].row_base + row;
-          v = fmaf(a.pacc[g * d + k], expf(a.pm[g] - mx), v);
+          const int64_t g = P.items[w].row_base + row;
+          const float f = P.log2_partials ? exp2f(a.pm[g] - mx) : expf(a.pm[g] - mx);
+          v = fmaf(a.pacc[g * d + k], f, v);
         }
         A[b * a.wa + j * d + k] = v * inv;
       }
@@ -366,7 +369,7 @@ __global__ void __launch_bounds__(kThreads) target_step_kernel(StepArgs a) {
     for (int b = 0; b < nb; ++b) {
       const float u = acc[b] * a.uscale;
       const int64_t gi = (t0 + b) * h * d + cc;
-      a.U[gi] = u;
+      if (a.U) a.U[gi] = u;
       if (a.Ubf) a.Ubf[gi] = f32_to_bf16(u);
     }
   }
@@ -442,23 +445,24 @@ size_t target_step_smem(const stca_handle* H) {
 }
 
 void launch_target_step(const stca_handle* H, int layer, const void* targets, int64_t T,
-                        const int32_t* treq_d, const int64_t* toff_d, const int32_t* rib_d,
-                        const AttnItem* items_d, float* Z, cudaStream_t s) {
+                        const StepPlan& plan, float* Z, cudaStream_t s) {
   if (T <= 0) return;
   StepArgs a{};
   a.layer = layer;
   a.M = H->M; a.d = H->d; a.h = H->h; a.dh = H->dh; a.rd = H->rd;
   a.T = T;
   a.targets = targets;
-  a.treq = treq_d; a.toff = toff_d; a.rib = rib_d; a.items = items_d;
+  a.plan = plan;
   const int64_t G = H->last_G;
   a.pacc = H->part;
   a.pm = H->part + G * H->d;
   a.pl = a.pm + G;
   a.Z = Z;
-  a.U = H->U;
-  a.Ubf = H->Ubf;
-  a.uscale = 1.0f / sqrtf(static_cast<float>(H->dh));
+  const bool tc = plan.log2_partials != 0;
+  a.U = tc ? nullptr : H->U;
+  a.Ubf = tc ? H->Ubf : nullptr;
+  // fold 1/sqrt(d_h) (and log2(e) for the exp2-based tensor-core kernel) into u
+  a.uscale = (tc ? 1.4426950408889634f : 1.0f) / sqrtf(static_cast<float>(H->dh));
   if (layer >= 0) a.cur = H->L32[layer];
   if (layer + 1 < H->M) a.nxt = H->L32[layer + 1];
   a.q_ln_g = H->q_ln_g;

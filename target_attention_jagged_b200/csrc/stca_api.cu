@@ -344,10 +344,6 @@ extern "C" int stca_init(const stca_weights* w, int d, int h, int r, int M, int 
 }
 
 // ------------------------------------------------------------------ encode
-static int64_t choose_split(const stca_handle* H) {
-  if (H->opt_split_keys > 0) return H->opt_split_keys;
-  return 1024;
-}
 
 extern "C" int stca_encode(stca_handle* H, const void* X, const int64_t* offsets, int64_t R,
                            int64_t N, void* stream) {
@@ -365,24 +361,14 @@ extern "C" int stca_encode(stca_handle* H, const void* X, const int64_t* offsets
   H->R = R;
   H->N = N;
   H->offsets_h.assign(offsets, offsets + R + 1);
-  // key ranges: each request's history cut into ranges of at most `split` keys
-  const int64_t split = choose_split(H);
-  H->items_h.clear();
-  H->req_item_begin.assign(R + 1, 0);
-  for (int64_t r = 0; r < R; ++r) {
-    H->req_item_begin[r] = static_cast<int32_t>(H->items_h.size());
-    for (int64_t k0 = offsets[r]; k0 < offsets[r + 1]; k0 += split) {
-      AttnItem it;
-      it.req = static_cast<int32_t>(r);
-      it.nkeys = static_cast<int32_t>(std::min<int64_t>(split, offsets[r + 1] - k0));
-      it.key0 = k0;
-      it.row_base = 0;
-      H->items_h.push_back(it);
-    }
-  }
-  H->req_item_begin[R] = static_cast<int32_t>(H->items_h.size());
   H->last_toff.clear();          // plan must be rebuilt for the next forward
   H->launches = 0;
+  if (H->dtype == STCA_BF16 && attn_tc_supported(H->d)) {
+    for (int i = 0; i < H->M; ++i)
+      if (int rc = make_tmap_bf16_2d(&H->tmXt[i], static_cast<char*>(H->xt) + layer_bytes * i,
+                                     H->d, N, 64, 128))
+        return rc;
+  }
   const bool bf = H->dtype == STCA_BF16;
   if (H->opt_encode_path == 2 && !H->tc_encode_ready)
     return set_error(STCA_EINVAL, "tensor-core encoder needs bf16 and d in {64,128,256}, rd % 64 == 0");
@@ -414,27 +400,202 @@ extern "C" int stca_encode(stca_handle* H, const void* X, const int64_t* offsets
 // ------------------------------------------------------------------ forward
 static size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
-static int build_plan(stca_handle* H, const int64_t* toff, int64_t T, cudaStream_t s) {
+// Attention path of a forward: 2 tensor cores, 1 CUDA cores.
+static int attn_path(const stca_handle* H) {
+  const bool tc = H->dtype == STCA_BF16 && attn_tc_supported(H->d);
+  if (H->opt_attn_path == 1) return 1;
+  if (H->opt_attn_path == 2) return tc ? 2 : -1;
+  return tc ? 2 : 1;
+}
+
+// Host-side attention work plan (see build_plan_host).
+struct PlanHost {
+  std::vector<AttnItem> items;
+  std::vector<int32_t> pairs_simt;       // (item, target) pairs, CUDA-core grid
+  std::vector<int32_t> cta_begin;        // tensor-core grid + 1
+  std::vector<int32_t> req_pair_begin;   // R + 1
+  std::vector<int32_t> pair_item_begin;  // pairs + 1
+  int64_t G = 0;                         // partial rows
+  int grid = 0;                          // tensor-core CTAs
+};
+
+// Cut the attention of one forward into work items.
+//  CUDA cores (path 1): each request's keys cut into ranges of at most `split`
+//    keys (1024 by default); one item per range covers all T_r * h query rows;
+//    the kernel grid is the list of (item, target) pairs.
+//  Tensor cores (path 2): (request, 128-row query tile) pairs, each over all
+//    its key tiles, laid end to end and cut into runs of equal numbers of key
+//    tiles, one run per CTA (stream-K); every maximal run inside one pair is
+//    an item.  `split`, when set, caps a run at split/128 key tiles.
+static void build_plan_host(const int64_t* off, const int64_t* toff, int64_t R, int h, int path,
+                            int num_ctas, int64_t split_keys, PlanHost& P) {
+  P = PlanHost();
+  P.req_pair_begin.assign(R + 1, 0);
+  auto& items = P.items;
+  int64_t& G = P.G;
+  if (path == 1) {
+    const int64_t split = split_keys > 0 ? split_keys : 1024;
+    for (int64_t r = 0; r < R; ++r) {
+      P.req_pair_begin[r] = static_cast<int32_t>(r);
+      P.pair_item_begin.push_back(static_cast<int32_t>(items.size()));
+      const int64_t Tr = toff[r + 1] - toff[r];
+      for (int64_t k0 = off[r]; k0 < off[r + 1]; k0 += split) {
+        AttnItem it{};
+        it.req = static_cast<int32_t>(r);
+        it.nkeys = static_cast<int32_t>(std::min<int64_t>(split, off[r + 1] - k0));
+        it.key0 = k0;
+        it.row_base = G;
+        it.qrow0 = toff[r] * h;
+        it.mt = 0;
+        it.rows = static_cast<int32_t>(Tr * h);
+        G += Tr * h;
+        for (int64_t tl = 0; tl < Tr; ++tl) {
+          P.pairs_simt.push_back(static_cast<int32_t>(items.size()));
+          P.pairs_simt.push_back(static_cast<int32_t>(tl));
+        }
+        items.push_back(it);
+      }
+    }
+    P.req_pair_begin[R] = static_cast<int32_t>(R);
+    P.pair_item_begin.push_back(static_cast<int32_t>(items.size()));
+    return;
+  }
+  struct Pair { int64_t r, mt, ntiles; };
+  std::vector<Pair> pairs;
+  int64_t W = 0;
+  for (int64_t r = 0; r < R; ++r) {
+    P.req_pair_begin[r] = static_cast<int32_t>(pairs.size());
+    const int64_t rows = (toff[r + 1] - toff[r]) * h;
+    const int64_t nt = (off[r + 1] - off[r] + 127) / 128;
+    for (int64_t mt = 0; mt * 128 < rows; ++mt) {
+      pairs.push_back({r, mt, nt});
+      W += nt;
+    }
+  }
+  P.req_pair_begin[R] = static_cast<int32_t>(pairs.size());
+  int64_t cs = (W + num_ctas - 1) / std::max(num_ctas, 1);      // key tiles per CTA
+  if (split_keys > 0) cs = std::min<int64_t>(cs, std::max<int64_t>(1, split_keys / 128));
+  cs = std::max<int64_t>(cs, 1);
+  P.grid = static_cast<int>((W + cs - 1) / cs);
+  P.cta_begin.assign(P.grid + 1, 0);
+  int64_t cursor = 0;     // global key-tile index of the pair's first tile
+  int next_cta = 0;
+  for (const Pair& pr : pairs) {
+    P.pair_item_begin.push_back(static_cast<int32_t>(items.size()));
+    const int64_t L = off[pr.r + 1] - off[pr.r];
+    const int64_t rows = std::min<int64_t>(128, (toff[pr.r + 1] - toff[pr.r]) * h - pr.mt * 128);
+    int64_t a = 0;
+    while (a < pr.ntiles) {
+      const int64_t g0 = cursor + a;
+      const int64_t b = std::min<int64_t>(pr.ntiles, (g0 / cs + 1) * cs - cursor);
+      while (next_cta <= g0 / cs) P.cta_begin[next_cta++] = static_cast<int32_t>(items.size());
+      AttnItem it{};
+      it.req = static_cast<int32_t>(pr.r);
+      it.key0 = off[pr.r] + a * 128;
+      it.nkeys = static_cast<int32_t>(std::min<int64_t>(b * 128, L) - a * 128);
+      it.row_base = G;
+      it.qrow0 = toff[pr.r] * h + pr.mt * 128;
+      it.mt = static_cast<int32_t>(pr.mt);
+      it.rows = static_cast<int32_t>(rows);
+      G += rows;
+      items.push_back(it);
+      a = b;
+    }
+    cursor += pr.ntiles;
+  }
+  while (next_cta <= P.grid) P.cta_begin[next_cta++] = static_cast<int32_t>(items.size());
+  P.pair_item_begin.push_back(static_cast<int32_t>(items.size()));
+}
+
+// Invariants every kernel relies on for in-bounds access; a violation is a
+// library bug and is reported instead of launched.
+static int check_plan(const PlanHost& P, const int64_t* off, const int64_t* toff, int64_t R,
+                      int h, int path) {
+  const int64_t N = off[R], T = toff[R];
+  auto bad = [](const std::string& m) { return set_error(STCA_EINVAL, "internal plan check: " + m); };
+  int64_t rows_sum = 0;
+  for (size_t w = 0; w < P.items.size(); ++w) {
+    const AttnItem& it = P.items[w];
+    if (it.req < 0 || it.req >= R) return bad("request index");
+    if (it.nkeys < 1 || it.key0 < off[it.req] || it.key0 + it.nkeys > off[it.req + 1])
+      return bad("key range outside its request");
+    if (it.rows < 0 || it.row_base != rows_sum) return bad("partial rows not contiguous");
+    rows_sum += it.rows;
+    const int64_t req_rows = (toff[it.req + 1] - toff[it.req]) * h;
+    if (path == 2) {
+      if (it.rows < 1 || it.rows > 128 || int64_t(it.mt) * 128 + it.rows > req_rows ||
+          it.qrow0 != toff[it.req] * h + int64_t(it.mt) * 128 || it.qrow0 + it.rows > T * h)
+        return bad("query tile");
+    } else if (it.rows != req_rows) {
+      return bad("query rows");
+    }
+  }
+  if (rows_sum != P.G) return bad("partial row count");
+  if (static_cast<int64_t>(P.req_pair_begin.size()) != R + 1) return bad("request pairs");
+  const int64_t npairs = static_cast<int64_t>(P.pair_item_begin.size()) - 1;
+  if (P.req_pair_begin[R] != npairs) return bad("pair count");
+  for (int64_t p = 0; p < npairs; ++p)
+    if (P.pair_item_begin[p] > P.pair_item_begin[p + 1]) return bad("pair items");
+  if (P.pair_item_begin[npairs] != static_cast<int32_t>(P.items.size())) return bad("pair end");
+  for (int64_t r = 0; r < R; ++r) {
+    const int64_t rows = (toff[r + 1] - toff[r]) * h;
+    const int64_t want = path == 2 ? (rows + 127) / 128 : 1;
+    if (P.req_pair_begin[r + 1] - P.req_pair_begin[r] != want) return bad("pairs of a request");
+    for (int32_t p = P.req_pair_begin[r]; p < P.req_pair_begin[r + 1]; ++p) {
+      // the pair's items cover the request's keys exactly once, in order
+      int64_t k = off[r];
+      for (int32_t w = P.pair_item_begin[p]; w < P.pair_item_begin[p + 1]; ++w) {
+        if (P.items[w].req != r || P.items[w].key0 != k) return bad("key coverage");
+        k += P.items[w].nkeys;
+      }
+      if (rows > 0 && k != off[r + 1]) return bad("keys not covered");
+    }
+  }
+  if (path == 2) {
+    if (static_cast<int>(P.cta_begin.size()) != P.grid + 1 || P.cta_begin[0] != 0 ||
+        P.cta_begin[P.grid] != static_cast<int32_t>(P.items.size()))
+      return bad("CTA ranges");
+    for (int c = 0; c < P.grid; ++c)
+      if (P.cta_begin[c] > P.cta_begin[c + 1]) return bad("CTA ranges order");
+  } else {
+    for (size_t q = 0; q < P.pairs_simt.size(); q += 2) {
+      const int32_t w = P.pairs_simt[q], tl = P.pairs_simt[q + 1];
+      if (w < 0 || w >= static_cast<int32_t>(P.items.size()) || tl < 0 ||
+          tl >= toff[P.items[w].req + 1] - toff[P.items[w].req])
+        return bad("(item, target) pair");
+    }
+  }
+  (void)N;
+  return STCA_OK;
+}
+
+// Build (or reuse) the plan for the targets layout `toff` and upload it.
+static int build_plan(stca_handle* H, const int64_t* toff, int64_t T, int path, cudaStream_t s) {
   const int64_t R = H->R;
-  if (!H->last_toff.empty() && static_cast<int64_t>(H->last_toff.size()) == R + 1 &&
+  if (path == H->last_path && !H->last_toff.empty() &&
+      static_cast<int64_t>(H->last_toff.size()) == R + 1 &&
       std::equal(H->last_toff.begin(), H->last_toff.end(), toff))
     return STCA_OK;   // same layout as the previous forward on this encode: plan is on device
-  const int h = H->h;
-  std::vector<AttnItem> items = H->items_h;
-  int64_t G = 0, npairs = 0;
-  for (auto& it : items) {
-    const int64_t Tr = toff[it.req + 1] - toff[it.req];
-    it.row_base = G;
-    G += Tr * h;
-    npairs += Tr;
-  }
+  const int64_t* off = H->offsets_h.data();
+  PlanHost P;
+  build_plan_host(off, toff, R, H->h, path, H->num_sms, H->opt_split_keys, P);
+  if (int rc = check_plan(P, off, toff, R, H->h, path)) return rc;
+  const auto& items = P.items;
+  const auto& pairs_simt = P.pairs_simt;
+  const auto& cta_begin = P.cta_begin;
+  const auto& req_pair_begin = P.req_pair_begin;
+  const auto& pair_item_begin = P.pair_item_begin;
+  const int64_t G = P.G;
+  const int grid = P.grid;
   const size_t n_items = items.size();
   H->off_items = 0;
   H->off_pairs = align256(H->off_items + n_items * sizeof(AttnItem));
-  H->off_treq = align256(H->off_pairs + static_cast<size_t>(npairs) * 2 * sizeof(int32_t));
+  H->off_cta = align256(H->off_pairs + pairs_simt.size() * sizeof(int32_t));
+  H->off_treq = align256(H->off_cta + cta_begin.size() * sizeof(int32_t));
   H->off_toff = align256(H->off_treq + static_cast<size_t>(T) * sizeof(int32_t));
-  H->off_rib = align256(H->off_toff + static_cast<size_t>(R + 1) * sizeof(int64_t));
-  const size_t bytes = align256(H->off_rib + static_cast<size_t>(R + 1) * sizeof(int32_t));
+  H->off_rpb = align256(H->off_toff + static_cast<size_t>(R + 1) * sizeof(int64_t));
+  H->off_pib = align256(H->off_rpb + static_cast<size_t>(R + 1) * sizeof(int32_t));
+  const size_t bytes = align256(H->off_pib + pair_item_begin.size() * sizeof(int32_t));
   // pinned staging: wait until the previous upload has left it
   if (H->plan_h && cudaEventSynchronize(H->plan_evt) != cudaSuccess)
     return set_error(STCA_ECUDA, "plan event wait failed");
@@ -452,25 +613,20 @@ static int build_plan(stca_handle* H, const int64_t* toff, int64_t T, cudaStream
   if (int rc = ensure_dev(&H->plan_d, &H->plan_cap, bytes)) return rc;
   char* p = static_cast<char*>(H->plan_h);
   memcpy(p + H->off_items, items.data(), n_items * sizeof(AttnItem));
-  int32_t* pairs = reinterpret_cast<int32_t*>(p + H->off_pairs);
-  int64_t q = 0;
-  for (size_t w = 0; w < n_items; ++w) {
-    const int64_t Tr = toff[items[w].req + 1] - toff[items[w].req];
-    for (int64_t tl = 0; tl < Tr; ++tl) {
-      pairs[2 * q] = static_cast<int32_t>(w);
-      pairs[2 * q + 1] = static_cast<int32_t>(tl);
-      ++q;
-    }
-  }
+  memcpy(p + H->off_pairs, pairs_simt.data(), pairs_simt.size() * sizeof(int32_t));
+  memcpy(p + H->off_cta, cta_begin.data(), cta_begin.size() * sizeof(int32_t));
   int32_t* treq = reinterpret_cast<int32_t*>(p + H->off_treq);
   for (int64_t r = 0; r < R; ++r)
     for (int64_t t = toff[r]; t < toff[r + 1]; ++t) treq[t] = static_cast<int32_t>(r);
   memcpy(p + H->off_toff, toff, static_cast<size_t>(R + 1) * sizeof(int64_t));
-  memcpy(p + H->off_rib, H->req_item_begin.data(), static_cast<size_t>(R + 1) * sizeof(int32_t));
+  memcpy(p + H->off_rpb, req_pair_begin.data(), static_cast<size_t>(R + 1) * sizeof(int32_t));
+  memcpy(p + H->off_pib, pair_item_begin.data(), pair_item_begin.size() * sizeof(int32_t));
   STCA_CUDA_TRY(cudaMemcpyAsync(H->plan_d, H->plan_h, bytes, cudaMemcpyHostToDevice, s));
   STCA_CUDA_TRY(cudaEventRecord(H->plan_evt, s));
   H->last_G = G;
-  H->last_pairs = npairs;
+  H->last_pairs = static_cast<int64_t>(pairs_simt.size() / 2);
+  H->last_grid = grid;
+  H->last_path = path;
   H->last_toff.assign(toff, toff + R + 1);
   return STCA_OK;
 }
@@ -488,42 +644,63 @@ extern "C" int stca_forward(stca_handle* H, const void* targets, const int64_t* 
   DeviceGuard g(H->device);
   if (!g.ok) return set_error(STCA_ECUDA, "cannot select the handle's device");
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (attn_simt_smem(H) > 227 * 1024)
+  const int path = attn_path(H);
+  if (path < 0)
+    return set_error(STCA_EINVAL, "tensor-core attention needs bf16 and d in {64, 128, 256}");
+  if (path == 1 && attn_simt_smem(H) > 227 * 1024)
     return set_error(STCA_EINVAL, "h * d too large for the CUDA-core attention kernel");
-  if (int rc = build_plan(H, target_offsets, T, s)) return rc;
+  if (int rc = build_plan(H, target_offsets, T, path, s)) return rc;
   const int d = H->d, h = H->h;
-  if (int rc = ensure_dev(reinterpret_cast<void**>(&H->U), &H->U_cap,
-                          static_cast<size_t>(T) * h * d * sizeof(float))) return rc;
+  const size_t urows = static_cast<size_t>(T) * h;
+  if (path == 1) {
+    if (int rc = ensure_dev(reinterpret_cast<void**>(&H->U), &H->U_cap, urows * d * sizeof(float)))
+      return rc;
+  } else {
+    if (int rc = ensure_dev(reinterpret_cast<void**>(&H->Ubf), &H->Ubf_cap, urows * d * 2)) return rc;
+    if (int rc = make_tmap_bf16_2d(&H->tmU, H->Ubf, d, urows, 64, 128)) return rc;
+  }
   if (int rc = ensure_dev(reinterpret_cast<void**>(&H->part), &H->part_cap,
                           static_cast<size_t>(std::max<int64_t>(H->last_G, 1)) * (d + 2) * sizeof(float)))
     return rc;
   char* p = static_cast<char*>(H->plan_d);
   const AttnItem* items_d = reinterpret_cast<const AttnItem*>(p + H->off_items);
   const int32_t* pairs_d = reinterpret_cast<const int32_t*>(p + H->off_pairs);
-  const int32_t* treq_d = reinterpret_cast<const int32_t*>(p + H->off_treq);
-  const int64_t* toff_d = reinterpret_cast<const int64_t*>(p + H->off_toff);
-  const int32_t* rib_d = reinterpret_cast<const int32_t*>(p + H->off_rib);
+  const int32_t* cta_d = reinterpret_cast<const int32_t*>(p + H->off_cta);
+  StepPlan plan;
+  plan.treq = reinterpret_cast<const int32_t*>(p + H->off_treq);
+  plan.toff = reinterpret_cast<const int64_t*>(p + H->off_toff);
+  plan.req_pair_begin = reinterpret_cast<const int32_t*>(p + H->off_rpb);
+  plan.pair_item_begin = reinterpret_cast<const int32_t*>(p + H->off_pib);
+  plan.items = items_d;
+  plan.mtile_rows = path == 2 ? 128 : (1 << 30);
+  plan.log2_partials = path == 2 ? 1 : 0;
   const size_t layer_bytes = static_cast<size_t>(H->N) * d * H->elem;
   {
     TimedLaunch tl(H, STCA_K_STEP, s);
-    launch_target_step(H, -1, targets, T, treq_d, toff_d, rib_d, items_d, Z, s);
+    launch_target_step(H, -1, targets, T, plan, Z, s);
   }
   H->launches++;
   if (int rc = check_launch("query init")) return rc;
   for (int i = 0; i < H->M; ++i) {
-    const void* xti = static_cast<const char*>(H->xt) + layer_bytes * i;
+    int rc = STCA_OK;
     {
       TimedLaunch tl(H, STCA_K_ATTN, s);
-      launch_attn_simt(H, i, xti, items_d, pairs_d, H->last_pairs, toff_d, s);
+      if (path == 2) {
+        rc = launch_attn_tc(H, i, items_d, cta_d, H->last_grid, s);
+      } else {
+        const void* xti = static_cast<const char*>(H->xt) + layer_bytes * i;
+        launch_attn_simt(H, i, xti, items_d, pairs_d, H->last_pairs, plan.toff, s);
+      }
     }
+    if (rc) return rc;
     H->launches++;
-    if (int rc = check_launch("attention")) return rc;
+    if (int rc2 = check_launch("attention")) return rc2;
     {
       TimedLaunch tl(H, STCA_K_STEP, s);
-      launch_target_step(H, i, targets, T, treq_d, toff_d, rib_d, items_d, Z, s);
+      launch_target_step(H, i, targets, T, plan, Z, s);
     }
     H->launches++;
-    if (int rc = check_launch("target step")) return rc;
+    if (int rc2 = check_launch("target step")) return rc2;
   }
   return ok();
 }
@@ -537,6 +714,40 @@ extern "C" int stca_get_encoded(stca_handle* H, int layer, void* dst, void* stre
   const size_t bytes = static_cast<size_t>(H->N) * H->d * H->elem;
   STCA_CUDA_TRY(cudaMemcpyAsync(dst, static_cast<const char*>(H->xt) + bytes * layer, bytes,
                                 cudaMemcpyDeviceToDevice, static_cast<cudaStream_t>(stream)));
+  return ok();
+}
+
+extern "C" int stca_plan_attention(const int64_t* offsets, const int64_t* target_offsets,
+                                   int64_t R, int h, int path, int num_ctas, int64_t split_keys,
+                                   int64_t* n_items, int64_t* grid, int64_t* partial_rows,
+                                   int64_t* items, int64_t items_cap, int32_t* cta_begin,
+                                   int64_t cta_cap) {
+  if (!n_items || !grid || !partial_rows) return set_error(STCA_EINVAL, "NULL output count");
+  if (path != 1 && path != 2) return set_error(STCA_EINVAL, "path must be 1 or 2");
+  if (h < 1 || num_ctas < 1 || split_keys < 0) return set_error(STCA_EINVAL, "bad h, num_ctas or split_keys");
+  if (int rc = validate_offsets(offsets, R, offsets ? offsets[R] : 0, true, "offsets")) return rc;
+  if (int rc = validate_offsets(target_offsets, R, target_offsets ? target_offsets[R] : 0, false,
+                                "target_offsets"))
+    return rc;
+  PlanHost P;
+  build_plan_host(offsets, target_offsets, R, h, path, num_ctas, split_keys, P);
+  if (int rc = check_plan(P, offsets, target_offsets, R, h, path)) return rc;
+  *n_items = static_cast<int64_t>(P.items.size());
+  *grid = P.grid;
+  *partial_rows = P.G;
+  if (items) {
+    if (items_cap < *n_items) return set_error(STCA_EINVAL, "items_cap too small");
+    for (size_t w = 0; w < P.items.size(); ++w) {
+      const AttnItem& it = P.items[w];
+      int64_t* o = items + 7 * w;
+      o[0] = it.req; o[1] = it.mt; o[2] = it.key0; o[3] = it.nkeys;
+      o[4] = it.qrow0; o[5] = it.rows; o[6] = it.row_base;
+    }
+  }
+  if (cta_begin && path == 2) {
+    if (cta_cap < P.grid + 1) return set_error(STCA_EINVAL, "cta_cap too small");
+    std::copy(P.cta_begin.begin(), P.cta_begin.end(), cta_begin);
+  }
   return ok();
 }
 

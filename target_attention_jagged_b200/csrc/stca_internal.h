@@ -26,12 +26,17 @@ int set_error(int code, const std::string& msg);
 enum : int { kStatusEncodeTimeout = 1, kStatusAttnTimeout = 2 };
 
 // ---------------------------------------------------------------- work plan
-// One attention work item: a contiguous key range of one request's history.
+// One attention work item: a contiguous key range of one request's history
+// against one tile of its query rows (all T_r * h rows on the CUDA-core path,
+// up to 128 rows on the tensor-core path).
 struct AttnItem {
   int32_t req;        // request index
   int32_t nkeys;      // keys in this range (>= 1)
   int64_t key0;       // first history row (absolute row in X~)
-  int64_t row_base;   // first partial row of this item (rows = T_r * h)
+  int64_t row_base;   // first partial row written by this item
+  int64_t qrow0;      // first query row (row of U: target * h + head)
+  int32_t mt;         // query tile index within the request
+  int32_t rows;       // query rows of this tile that belong to the request
 };
 
 // Per-layer pointers into the handle's fp32 weight slab (CUDA-core kernels and
@@ -61,6 +66,8 @@ struct stca_handle {
   const float* q_ln_b = nullptr;
   uint16_t* wtc = nullptr;              // bf16 operands of the tensor-core encoder
   CUtensorMap tmW1, tmW2;               // their TMA descriptors
+  CUtensorMap tmXt[16];                 // X~(i) of the last encode (tensor-core attention)
+  CUtensorMap tmU;                      // bf16 query rows of the current forward
   bool tc_encode_ready = false;
   int num_sms = 148;
 
@@ -79,8 +86,6 @@ struct stca_handle {
   std::vector<int64_t> offsets_h;
   void* xt = nullptr;                   // M x N x d, elem bytes each
   size_t xt_cap = 0;
-  std::vector<stca::AttnItem> items_h;  // key ranges of the last encode
-  std::vector<int32_t> req_item_begin;  // R+1
 
   // forward workspace (device)
   float* q = nullptr;       size_t q_cap = 0;      // T x d
@@ -99,8 +104,11 @@ struct stca_handle {
 
   // last forward's plan (reused when the same targets layout repeats)
   std::vector<int64_t> last_toff;
+  int last_path = 0;                    // 1 CUDA cores, 2 tensor cores
   int64_t last_G = 0, last_pairs = 0;
-  size_t off_items = 0, off_pairs = 0, off_treq = 0, off_toff = 0, off_rib = 0;
+  int last_grid = 0;                    // CTAs of the tensor-core attention
+  size_t off_items = 0, off_pairs = 0, off_cta = 0, off_treq = 0, off_toff = 0, off_rpb = 0,
+         off_pib = 0;
 };
 
 namespace stca {
@@ -113,11 +121,24 @@ void launch_ffn_rows(const void* X, int x_is_bf16, int64_t nrows, const LayerW32
 void launch_attn_simt(const stca_handle* H, int layer, const void* xt_layer,
                       const AttnItem* items_d, const int32_t* pairs_d, int64_t npairs,
                       const int64_t* toff_d, cudaStream_t s);
+struct StepPlan {
+  const int32_t* treq;              // T: request of each target
+  const int64_t* toff;              // R+1
+  const int32_t* req_pair_begin;    // R+1: first (request, query tile) pair of r
+  const int32_t* pair_item_begin;   // pairs+1: first item of each pair
+  const AttnItem* items;
+  int mtile_rows;                   // query rows per tile (1 << 30: one tile per request)
+  int log2_partials;                // partial maxima are in log2 units
+};
 void launch_target_step(const stca_handle* H, int layer, const void* targets, int64_t T,
-                        const int32_t* treq_d, const int64_t* toff_d, const int32_t* rib_d,
-                        const AttnItem* items_d, float* Z, cudaStream_t s);
+                        const StepPlan& plan, float* Z, cudaStream_t s);
 size_t target_step_smem(const stca_handle* H);
 size_t attn_simt_smem(const stca_handle* H);
+
+// Tensor-core attention (attn_tc.cu)
+bool attn_tc_supported(int d);
+int launch_attn_tc(stca_handle* H, int layer, const AttnItem* items_d, const int32_t* cta_begin_d,
+                   int grid, cudaStream_t s);
 
 // Tensor-core encoder (encode_tc.cu)
 bool encode_tc_supported(int d, int rd);

@@ -31,7 +31,8 @@ _NAMES = {STCA_EINVAL: "EINVAL", STCA_ESTATE: "ESTATE", STCA_ENOMEM: "ENOMEM",
 
 EXPORTS = ("stca_init", "stca_destroy", "stca_encode", "stca_forward", "stca_run_host",
            "stca_validate_offsets", "stca_device_status", "stca_set_option",
-           "stca_get_option", "stca_kernel_times", "stca_get_encoded", "stca_last_error")
+           "stca_get_option", "stca_kernel_times", "stca_get_encoded", "stca_plan_attention",
+           "stca_last_error")
 
 
 class StcaError(RuntimeError):
@@ -58,6 +59,8 @@ def _load():
     lib.stca_set_option.argtypes = [P, I, I64]
     lib.stca_get_option.argtypes = [P, I, PI64]
     lib.stca_get_encoded.argtypes = [P, I, P, P]
+    lib.stca_plan_attention.argtypes = [PI64, PI64, I64, I, I, I, I64, PI64, PI64, PI64, PI64,
+                                        I64, ctypes.POINTER(ctypes.c_int32), I64]
     lib.stca_kernel_times.argtypes = [P, ctypes.POINTER(ctypes.c_double), PI64, I]
     lib.stca_last_error.restype = ctypes.c_char_p
     lib.stca_last_error.argtypes = []
@@ -230,6 +233,27 @@ def stca_get_encoded(handle: int, layer: int, dst, stream=None):
     """Copy X~(layer+1) of the last encode into `dst` (CUDA tensor, N x d)."""
     _check(_lib.stca_get_encoded(handle, layer, dst.data_ptr(), _stream_ptr(stream)))
     return dst
+
+
+def stca_plan_attention(offsets, target_offsets, h: int, path: int, num_ctas: int = 148,
+                        split_keys: int = 0) -> dict:
+    """The attention work split for a batch (host only).  Returns items as an
+    (n, 7) int64 array: request, query tile, first key row, keys, first query
+    row, query rows, first partial row; plus grid, partial_rows, cta_begin."""
+    off, toff = _offsets(offsets), _offsets(target_offsets)
+    R = off.shape[0] - 1
+    n, g, rows = ctypes.c_int64(), ctypes.c_int64(), ctypes.c_int64()
+    _check(_lib.stca_plan_attention(_i64p(off), _i64p(toff), R, h, path, num_ctas, split_keys,
+                                    ctypes.byref(n), ctypes.byref(g), ctypes.byref(rows),
+                                    None, 0, None, 0))
+    items = np.zeros((n.value, 7), dtype=np.int64)
+    cta = np.zeros(g.value + 1, dtype=np.int32)
+    _check(_lib.stca_plan_attention(_i64p(off), _i64p(toff), R, h, path, num_ctas, split_keys,
+                                    ctypes.byref(n), ctypes.byref(g), ctypes.byref(rows),
+                                    _i64p(items), items.shape[0],
+                                    cta.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)),
+                                    cta.shape[0]))
+    return {"items": items, "grid": g.value, "partial_rows": rows.value, "cta_begin": cta}
 
 
 def stca_kernel_times(handle: int):

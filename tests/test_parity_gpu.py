@@ -58,19 +58,25 @@ EDGE_L = [1, 2, 127, 128, 129, 257, 1000, 1021]
 EDGE_T = [1, 0, 3, 2, 1, 5, 2, 1]
 
 
+ATTN_AUTO, ATTN_SIMT, ATTN_TC = 0, 1, 2
+
+
+@pytest.mark.parametrize("attn", [ATTN_AUTO, ATTN_SIMT])
 @pytest.mark.parametrize("dtype,d,h,M,r", [("bf16", 128, 4, 2, 2), ("f32", 64, 2, 3, 2),
-                                           ("bf16", 256, 8, 2, 2), ("bf16", 64, 4, 1, 4)])
-def test_ragged_edges(gpu, dtype, d, h, M, r):
+                                           ("bf16", 256, 8, 2, 2), ("bf16", 64, 4, 1, 4),
+                                           ("bf16", 128, 16, 3, 1)])
+def test_ragged_edges(gpu, dtype, d, h, M, r, attn):
     wl = make_workload(lengths=EDGE_L, targets=EDGE_T, d=d, h=h, M=M, r=r, dtype=dtype,
                        seed=100 + d + M)
-    check_full(wl, run_gpu(wl, gpu))
+    check_full(wl, run_gpu(wl, gpu, attn_path=attn))
 
 
-def test_many_targets_per_request(gpu):
-    # T_r * h = 40 * 8 = 320 query rows: more than one 128-row tile
+@pytest.mark.parametrize("attn", [ATTN_TC, ATTN_SIMT])
+def test_many_targets_per_request(gpu, attn):
+    # T_r * h = 40 * 8 = 320 query rows: three 128-row tiles, the last ragged
     wl = make_workload(lengths=[700, 333], targets=[40, 17], d=128, h=8, M=2, r=2,
                        dtype="bf16", seed=7)
-    check_full(wl, run_gpu(wl, gpu))
+    check_full(wl, run_gpu(wl, gpu, attn_path=attn))
 
 
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
@@ -86,11 +92,34 @@ def test_small_width(gpu):
     check_full(wl, run_gpu(wl, gpu))
 
 
+@pytest.mark.parametrize("attn", [ATTN_TC, ATTN_SIMT])
 @pytest.mark.parametrize("split", [128, 256, 4096])
-def test_split_sizes_agree(gpu, split):
+def test_split_sizes_agree(gpu, split, attn):
     wl = make_workload(lengths=[1500, 129, 640], targets=[3, 2, 1], d=128, h=4, M=2, r=2,
                        dtype="bf16", seed=10)
-    check_full(wl, run_gpu(wl, gpu, split=split))
+    check_full(wl, run_gpu(wl, gpu, split=split, attn_path=attn))
+
+
+def test_sharp_softmax_rescaling(gpu):
+    # The first key tile of each request repeats one token, so its scores are
+    # all equal and the running max jumps by far more than the lazy-rescale
+    # threshold in later tiles: exercises the O / l correction path.
+    wl = make_workload(lengths=[3000, 900], targets=[4, 3], d=128, h=4, M=2, r=2,
+                       dtype="bf16", seed=16)
+    wl.weights["Wq"] = [w * 3.0 for w in wl.weights["Wq"]]
+    for r in range(2):
+        lo = int(wl.offsets[r])
+        wl.X[lo:lo + 256] = wl.X[lo]
+    check_full(wl, run_gpu(wl, gpu, attn_path=ATTN_TC, split=1024))
+    check_full(wl, run_gpu(wl, gpu, attn_path=ATTN_SIMT))
+
+
+def test_attention_paths_agree_on_c2(gpu):
+    wl = make_config_workload("c2")
+    a = run_gpu(wl, gpu, attn_path=ATTN_TC)
+    b = run_gpu(wl, gpu, attn_path=ATTN_SIMT)
+    check_full(wl, a)
+    assert normwise_err(a, b) <= 2e-2
 
 
 def test_single_token_history_equals_closed_form(gpu):
