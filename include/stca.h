@@ -149,6 +149,27 @@ int stca_forward(stca_handle* handle, const void* targets, const int64_t* target
 int stca_get_encoded(stca_handle* handle, int layer, void* dst, void* stream);
 
 /*
+ * stca_forward without device allocation.  (An addition of this library: the
+ * STCA pages have no counterpart; it changes where the workspace lives, not
+ * what is computed.)  Same arguments, result and errors as stca_forward, for
+ * bf16 handles with d in {64, 128, 256} (the tensor-core path); other handles
+ * get STCA_EINVAL.  For callers that cannot call cudaMalloc after start-up --
+ * their device memory belongs to another allocator's pool, their memory budget
+ * is fixed, or they cannot afford the synchronisation cudaMalloc / cudaFree
+ * may imply -- the query rows, split partials and work plan of the call live in
+ * a 32 MiB file-scope device array built into the library: every GPU that
+ * loads the library holds it until the process exits.  A batch whose
+ * workspace does not fit returns STCA_EINVAL with the size it needs.  All
+ * calls on a device share the array: calls whose work overlaps on the GPU
+ * (other streams, other handles) race, so keep them on one stream.  The first
+ * call on a device looks up the array's address (cudaGetSymbolAddress); make
+ * it before any stream capture.  Nothing a call reads is left over from an
+ * earlier call.  stca_init and stca_encode still allocate as documented.
+ */
+int stca_forward_static(stca_handle* handle, const void* targets,
+                        const int64_t* target_offsets, int64_t T, float* Z, void* stream);
+
+/*
  * End-to-end call on HOST buffers: copies X and targets from host memory to
  * device staging buffers the handle owns, encodes, runs the forward, copies
  * Z (T x M x d fp32) back to host memory and waits for the stream.  Host

@@ -18,6 +18,7 @@ from .stca import (  # noqa: F401
     stca_device_status,
     stca_encode,
     stca_forward,
+    stca_forward_static,
     stca_get_encoded,
     stca_get_option,
     stca_kernel_times,

@@ -408,4 +408,23 @@ int launch_attn_tc(stca_handle* H, int layer, const AttnItem* items_d, const int
   }
 }
 
+// The same kernel with every buffer given explicitly (no handle state).
+int launch_attn_tc_ws(int d, const CUtensorMap& tmQ, const CUtensorMap& tmK,
+                      const AttnItem* items_d, const int32_t* cta_begin_d, int grid, float* part,
+                      int64_t G, int* status, cudaStream_t s) {
+  AttnParams p{};
+  p.items = items_d;
+  p.cta_item_begin = cta_begin_d;
+  p.pacc = part;
+  p.pm = part + G * d;
+  p.pl = p.pm + G;
+  p.status = status;
+  switch (d) {
+    case 64: return launch_cfg<64, 2, 6, 2>(nullptr, tmQ, tmK, p, grid, s);
+    case 128: return launch_cfg<128, 2, 3, 2>(nullptr, tmQ, tmK, p, grid, s);
+    case 256: return launch_cfg<256, 1, 2, 1>(nullptr, tmQ, tmK, p, grid, s);
+    default: return set_error(STCA_EINVAL, "tensor-core attention needs d in {64, 128, 256}");
+  }
+}
+
 }  // namespace stca

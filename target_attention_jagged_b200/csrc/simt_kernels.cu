@@ -481,4 +481,35 @@ void launch_target_step(const stca_handle* H, int layer, const void* targets, in
   }
 }
 
+// Same launch as launch_target_step for the tensor-core partial layout, with
+// the bf16 query rows and the split partials in caller-given buffers.
+void launch_target_step_ws(const stca_handle* H, int layer, const void* targets, int64_t T,
+                           const StepPlan& plan, float* Z, uint16_t* Ubf, float* part,
+                           int64_t G, cudaStream_t s) {
+  if (T <= 0) return;
+  StepArgs a{};
+  a.layer = layer;
+  a.M = H->M; a.d = H->d; a.h = H->h; a.dh = H->dh; a.rd = H->rd;
+  a.T = T;
+  a.targets = targets;
+  a.plan = plan;
+  a.pacc = part;
+  a.pm = part + G * H->d;
+  a.pl = a.pm + G;
+  a.Z = Z;
+  a.U = nullptr;
+  a.Ubf = Ubf;
+  a.uscale = 1.4426950408889634f / sqrtf(static_cast<float>(H->dh));
+  if (layer >= 0) a.cur = H->L32[layer];
+  if (layer + 1 < H->M) a.nxt = H->L32[layer + 1];
+  a.q_ln_g = H->q_ln_g;
+  a.q_ln_b = H->q_ln_b;
+  step_widths(H, &a.wa, &a.wb);
+  const size_t smem = target_step_smem(H);
+  const unsigned grid = static_cast<unsigned>((T + kTB - 1) / kTB);
+  cudaFuncSetAttribute(target_step_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                       (int)smem);
+  target_step_kernel<true><<<grid, kThreads, smem, s>>>(a);
+}
+
 }  // namespace stca

@@ -408,17 +408,6 @@ static int attn_path(const stca_handle* H) {
   return tc ? 2 : 1;
 }
 
-// Host-side attention work plan (see build_plan_host).
-struct PlanHost {
-  std::vector<AttnItem> items;
-  std::vector<int32_t> pairs_simt;       // (item, target) pairs, CUDA-core grid
-  std::vector<int32_t> cta_begin;        // tensor-core grid + 1
-  std::vector<int32_t> req_pair_begin;   // R + 1
-  std::vector<int32_t> pair_item_begin;  // pairs + 1
-  int64_t G = 0;                         // partial rows
-  int grid = 0;                          // tensor-core CTAs
-};
-
 // Cut the attention of one forward into work items.
 //  CUDA cores (path 1): each request's keys cut into ranges of at most `split`
 //    keys (1024 by default); one item per range covers all T_r * h query rows;
@@ -427,7 +416,7 @@ struct PlanHost {
 //    its key tiles, laid end to end and cut into runs of equal numbers of key
 //    tiles, one run per CTA (stream-K); every maximal run inside one pair is
 //    an item.  `split`, when set, caps a run at split/128 key tiles.
-static void build_plan_host(const int64_t* off, const int64_t* toff, int64_t R, int h, int path,
+void stca::build_plan_host(const int64_t* off, const int64_t* toff, int64_t R, int h, int path,
                             int num_ctas, int64_t split_keys, PlanHost& P) {
   P = PlanHost();
   P.req_pair_begin.assign(R + 1, 0);
@@ -509,7 +498,7 @@ static void build_plan_host(const int64_t* off, const int64_t* toff, int64_t R, 
 
 // Invariants every kernel relies on for in-bounds access; a violation is a
 // library bug and is reported instead of launched.
-static int check_plan(const PlanHost& P, const int64_t* off, const int64_t* toff, int64_t R,
+int stca::check_plan(const PlanHost& P, const int64_t* off, const int64_t* toff, int64_t R,
                       int h, int path) {
   const int64_t N = off[R], T = toff[R];
   auto bad = [](const std::string& m) { return set_error(STCA_EINVAL, "internal plan check: " + m); };

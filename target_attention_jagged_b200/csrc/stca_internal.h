@@ -135,6 +135,27 @@ void launch_target_step(const stca_handle* H, int layer, const void* targets, in
 size_t target_step_smem(const stca_handle* H);
 size_t attn_simt_smem(const stca_handle* H);
 
+// Host-side attention work plan (stca_api.cu).
+struct PlanHost {
+  std::vector<AttnItem> items;
+  std::vector<int32_t> pairs_simt;       // (item, target) pairs, CUDA-core grid
+  std::vector<int32_t> cta_begin;        // tensor-core grid + 1
+  std::vector<int32_t> req_pair_begin;   // R + 1
+  std::vector<int32_t> pair_item_begin;  // pairs + 1
+  int64_t G = 0;                         // partial rows
+  int grid = 0;                          // tensor-core CTAs
+};
+void build_plan_host(const int64_t* off, const int64_t* toff, int64_t R, int h, int path,
+                     int num_ctas, int64_t split_keys, PlanHost& P);
+int check_plan(const PlanHost& P, const int64_t* off, const int64_t* toff, int64_t R, int h,
+               int path);
+void launch_target_step_ws(const stca_handle* H, int layer, const void* targets, int64_t T,
+                           const StepPlan& plan, float* Z, uint16_t* Ubf, float* part,
+                           int64_t G, cudaStream_t s);
+int launch_attn_tc_ws(int d, const CUtensorMap& tmQ, const CUtensorMap& tmK,
+                      const AttnItem* items_d, const int32_t* cta_begin_d, int grid, float* part,
+                      int64_t G, int* status, cudaStream_t s);
+
 // Tensor-core attention (attn_tc.cu)
 bool attn_tc_supported(int d);
 int launch_attn_tc(stca_handle* H, int layer, const AttnItem* items_d, const int32_t* cta_begin_d,

@@ -32,7 +32,7 @@ _NAMES = {STCA_EINVAL: "EINVAL", STCA_ESTATE: "ESTATE", STCA_ENOMEM: "ENOMEM",
 EXPORTS = ("stca_init", "stca_destroy", "stca_encode", "stca_forward", "stca_run_host",
            "stca_validate_offsets", "stca_device_status", "stca_set_option",
            "stca_get_option", "stca_kernel_times", "stca_get_encoded", "stca_plan_attention",
-           "stca_last_error")
+           "stca_forward_static", "stca_last_error")
 
 
 class StcaError(RuntimeError):
@@ -53,6 +53,7 @@ def _load():
     lib.stca_destroy.restype = None
     lib.stca_encode.argtypes = [P, P, PI64, I64, I64, P]
     lib.stca_forward.argtypes = [P, P, PI64, I64, P, P]
+    lib.stca_forward_static.argtypes = [P, P, PI64, I64, P, P]
     lib.stca_run_host.argtypes = [P, P, PI64, I64, I64, P, PI64, I64, P, P]
     lib.stca_validate_offsets.argtypes = [PI64, I64, I64, I]
     lib.stca_device_status.argtypes = [P, P]
@@ -195,6 +196,18 @@ def stca_forward(handle: int, targets, target_offsets, Z=None, stream=None):
     assert Z.dtype == torch.float32 and Z.is_cuda and Z.is_contiguous()
     _check(_lib.stca_forward(handle, targets.data_ptr() if T > 0 else None, _i64p(toff), T,
                              Z.data_ptr() if T > 0 else None, _stream_ptr(stream)))
+    return Z
+
+
+def stca_forward_static(handle: int, targets, target_offsets, Z, stream=None):
+    """stca_forward with its workspace in the library's static device array
+    (no device allocation); Z: CUDA float32 (T, M, d)."""
+    import torch
+    toff = _offsets(target_offsets)
+    T = int(toff[-1])
+    assert Z.dtype == torch.float32 and Z.is_cuda and Z.is_contiguous()
+    _check(_lib.stca_forward_static(handle, targets.data_ptr() if T > 0 else None, _i64p(toff),
+                                    T, Z.data_ptr() if T > 0 else None, _stream_ptr(stream)))
     return Z
 
 
