@@ -99,9 +99,6 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
       : "memory");
 }
 
-__device__ __forceinline__ void tmem_st_wait() {
-  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
-}
 
 template <int D, int QB, int KS, int PB>
 __global__ void __launch_bounds__(kAttnThreads, 1)
@@ -279,12 +276,18 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         if (lane == 0) mbar_arrive(&sempty[sb]);
         ++sc;
         const int nvalid = min(128, item.nkeys - j * 128);
+        if (nvalid < 128) {   // the request's last tile: keys past its end take no weight
+#pragma unroll
+          for (int cb = 0; cb < 4; ++cb)
+#pragma unroll
+            for (int k = 0; k < 32; ++k)
+              if (cb * 32 + k >= nvalid) sv[cb][k] = __float_as_uint(-INFINITY);
+        }
         float mx = -INFINITY;
 #pragma unroll
         for (int cb = 0; cb < 4; ++cb)
 #pragma unroll
-          for (int k = 0; k < 32; ++k)
-            if (cb * 32 + k < nvalid) mx = fmaxf(mx, __uint_as_float(sv[cb][k]));
+          for (int k = 0; k < 32; ++k) mx = fmaxf(mx, __uint_as_float(sv[cb][k]));
         const bool resc = mx > m_used + kRescaleThreshold;
         const float m_new = resc ? mx : m_used;
         const float corr = resc ? ex2(m_used - m_new) : 1.f;
@@ -296,11 +299,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         for (int cb = 0; cb < 4; ++cb)
 #pragma unroll
           for (int k = 0; k < 32; k += 2) {
-            const int kk = cb * 32 + k;
-            const float p0 = kk < nvalid ? ex2(__uint_as_float(sv[cb][k]) - m_new) : 0.f;
-            const float p1 = kk + 1 < nvalid ? ex2(__uint_as_float(sv[cb][k + 1]) - m_new) : 0.f;
+            const float p0 = ex2(__uint_as_float(sv[cb][k]) - m_new);      // exp2(-inf) = 0
+            const float p1 = ex2(__uint_as_float(sv[cb][k + 1]) - m_new);
             lsum += p0 + p1;
-            pk[kk >> 1] = pack_bf16x2(p0, p1);
+            pk[(cb * 32 + k) >> 1] = pack_bf16x2(p0, p1);
           }
         l += lsum;
         const int pb = pc % PB;

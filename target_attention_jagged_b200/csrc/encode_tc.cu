@@ -7,18 +7,25 @@
 // boundaries do not matter here).  Per tile it keeps the X tile in shared
 // memory for all M layers, and per layer streams the weights in hidden chunks
 // of 64 columns:
-//   GEMM1  acc1[128 x 128] = X_tile * [W_u | W_g/2]_chunk      (tcgen05, TMEM)
+//   GEMM1  acc1[128 x 128] = X_tile * [W_u | W_g/2]_chunk      (tcgen05, SMEM operands)
 //   gate   H[128 x 64]     = u * g' * (1 + tanh(g'))          (g' = g/2; CUDA cores)
-//   GEMM2  acc2[128 x d]  += H * W_d,chunk                    (tcgen05, TMEM)
+//   GEMM2  acc2[128 x d]  += H * W_d,chunk                    (tcgen05, H read from TMEM)
 // then LayerNorm on acc2 and a bf16 store of the tile of X~(i).  The hidden
-// activations never leave the SM.  u * SiLU(g) = u * g' * (1 + tanh(g')) with
+// activations never leave the SM, and never touch shared memory: the gate
+// warps write H as packed bf16 back into the TMEM columns of u they have just
+// read, and GEMM2 takes its A operand from there.  Shared-memory bandwidth
+// (operand reads plus TMA writes of the streamed weights) is what bounds this
+// kernel, so keeping H out of it leaves room for deeper weight pipelines.  u * SiLU(g) = u * g' * (1 + tanh(g')) with
 // g' = g/2, so W_g is stored pre-halved (exact in bf16) and each gate value
 // costs one MUFU tanh.
 //
-// Warp roles (192 threads): warp 0 issues TMA loads, warp 1 issues the MMAs
-// (one thread) and owns the TMEM allocation, warps 2-5 run the gate and the
-// LayerNorm, each on its own 32-lane quarter of TMEM (one row per thread).
-// acc1 is double-buffered so GEMM1 of chunk c+1 overlaps the gate of chunk c.
+// Warp roles (448 threads): warp 0 issues TMA loads, warp 1 issues the MMAs
+// (one thread) and owns the TMEM allocation, warps 2-9 run the gate and warps
+// 10-13 the LayerNorm.  A warp may only touch its own 32-lane quarter of TMEM
+// (one row per thread), so two gate warps share each quarter and split its
+// columns in halves.  acc1 is double-buffered so GEMM1 of chunk c+1 overlaps
+// the gate of chunk c; acc2 is double-buffered (d <= 128) so the LayerNorm of
+// one (tile, layer) overlaps the GEMMs of the next.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -55,18 +62,19 @@ struct EncCfg {
   static constexpr uint32_t oX = 0;
   static constexpr uint32_t oW1 = oX + XB * kXBytes;
   static constexpr uint32_t oW2 = oW1 + S1 * kW1Stage;
-  static constexpr uint32_t oH = oW2 + S2 * kW2Stage;
-  static constexpr uint32_t oBar = oH + 2 * kBlock;
-  static constexpr int kBars = 2 * S1 + 2 * S2 + 2 * XB + 4 + 4 + 2 * AB2 + 1;
+  static constexpr uint32_t oBar = oW2 + S2 * kW2Stage;
+  static constexpr int kBars = 2 * S1 + 2 * S2 + 2 * XB + 2 + 2 + 2 * AB2 + 1;
   static constexpr uint32_t oMisc = oBar + kBars * 8;
   static constexpr uint32_t kSmem = oMisc + 16 + 1024;    // + alignment slack
-  static constexpr uint32_t kAcc1 = 0;                    // 2 x 128 columns
+  static constexpr uint32_t kAcc1 = 0;                    // 2 x 128 columns (H aliases u)
   static constexpr uint32_t kAcc2 = 256;                  // AB2 x D columns
   static_assert(kAcc2 + AB2 * D <= 512, "TMEM overflow");
   static_assert(kSmem <= 227 * 1024, "shared memory overflow");
 };
 
-constexpr int kEncThreads = 192;
+constexpr int kEpiWarps = 8;                          // gate: two per TMEM lane quarter
+constexpr int kLnWarps = 4;                           // LayerNorm: one per lane quarter
+constexpr int kEncThreads = 64 + 32 * (kEpiWarps + kLnWarps);
 
 __device__ __forceinline__ bool bwait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
                                       int* status) {
@@ -97,11 +105,9 @@ encode_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
   uint64_t* empty2 = full2 + S2;
   uint64_t* xfull = empty2 + S2;
   uint64_t* xempty = xfull + XB;
-  uint64_t* a1full = xempty + XB;
-  uint64_t* a1empty = a1full + 2;
-  uint64_t* hfull = a1empty + 2;
-  uint64_t* hempty = hfull + 2;
-  uint64_t* a2full = hempty + 2;
+  uint64_t* a1full = xempty + XB;     // GEMM1 of a chunk done
+  uint64_t* hfull = a1full + 2;       // its gate written to TMEM (and u, g read)
+  uint64_t* a2full = hfull + 2;
   uint64_t* a2empty = a2full + AB2;
   uint64_t* mdrain = a2empty + AB2;         // completion of every MMA, before TMEM is freed
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + C::oMisc);
@@ -112,11 +118,8 @@ encode_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
     for (int i = 0; i < S1; ++i) { mbar_init(&full1[i], 1); mbar_init(&empty1[i], 1); }
     for (int i = 0; i < S2; ++i) { mbar_init(&full2[i], 1); mbar_init(&empty2[i], 1); }
     for (int i = 0; i < XB; ++i) { mbar_init(&xfull[i], 1); mbar_init(&xempty[i], 1); }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&a1full[i], 1); mbar_init(&a1empty[i], 4);
-      mbar_init(&hfull[i], 4); mbar_init(&hempty[i], 1);
-    }
-    for (int i = 0; i < AB2; ++i) { mbar_init(&a2full[i], 1); mbar_init(&a2empty[i], 4); }
+    for (int i = 0; i < 2; ++i) { mbar_init(&a1full[i], 1); mbar_init(&hfull[i], kEpiWarps); }
+    for (int i = 0; i < AB2; ++i) { mbar_init(&a2full[i], 1); mbar_init(&a2empty[i], kLnWarps); }
     mbar_init(mdrain, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -191,10 +194,11 @@ encode_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
           const uint32_t acc2 = tmem + C::kAcc2 + b2 * D;
           for (int c = 0; ok && c <= p.nchunk; ++c) {
             if (c < p.nchunk) {
-              // GEMM1 of chunk c into acc1[cc & 1]
+              // GEMM1 of chunk c into acc1[cc & 1].  That buffer last held chunk
+              // c-2: its gate was waited for (hfull) before GEMM2 of c-2 was
+              // issued, and MMAs of one thread run in issue order, so GEMM2 of
+              // c-2 has read its H before this GEMM1 overwrites it.
               const int b = cc & 1;
-              if (!(ok = bwait(&a1empty[b], ((cc >> 1) & 1) ^ 1, abort_flag, p.status))) break;
-              tc_fence_after();
               const uint32_t acc1 = tmem + C::kAcc1 + b * 128;
               for (int kb = 0; kb < C::KB; ++kb) {
                 const int s = r1 % S1;
@@ -225,16 +229,17 @@ encode_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
               const int s = r2 % S2;
               if (!(ok = bwait(&full2[s], (r2 / S2) & 1, abort_flag, p.status))) break;
               tc_fence_after();
-              const uint32_t haddr = sbase + C::oH + hb * C::kBlock;
+              // H of the chunk: hidden columns 0..31 in TMEM columns 0..15 of
+              // acc1[hb], columns 32..63 in 32..47 (each gate warp's own u columns)
+              const uint32_t haddr = tmem + C::kAcc1 + hb * 128;
               const uint32_t waddr = sbase + C::oW2 + s * C::kW2Stage;
 #pragma unroll
               for (int k4 = 0; k4 < 4; ++k4)
-                mma_bf16_ss(acc2, sdesc_sw128(haddr + k4 * 32, 16, 1024),
+                mma_bf16_ts(acc2, haddr + (k4 >> 1) * 32 + (k4 & 1) * 8,
                             sdesc_sw128(waddr + k4 * 32, 16, 1024), idesc2,
                             ((c - 1) | k4) != 0);
               mma_commit(&empty2[s]);
               ++r2;
-              mma_commit(&hempty[hb]);
               ++hc;
             }
           }
@@ -247,105 +252,111 @@ encode_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
       drain_wait(mdrain, 0, 500000000ull);
     }
   } else {
-    // ------------------------------------------------------------ gate + LayerNorm
-    const int q = warp & 3;                    // TMEM lane quarter of this warp
+    // ------------------------------------------------------------ gate / LayerNorm
+    // A warp may only touch TMEM lanes 32 * (warp % 4) .. +31 (one row per
+    // thread).  Gate warps 2-9: two per lane quarter, each on half (`ch`) of the
+    // chunk's hidden columns.  LayerNorm warps 10-13: one per lane quarter, on
+    // acc2 of the previous (tile, layer) while the gate warps work on the next.
+    const int q = warp & 3;
     const int row_in_tile = q * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
-    uint32_t cc = 0, uc = 0;
     bool ok = true;
-    for (int tile = blockIdx.x; ok && tile < p.ntiles; tile += gridDim.x) {
-      const int64_t row = static_cast<int64_t>(tile) * 128 + row_in_tile;
-      for (int layer = 0; ok && layer < p.M; ++layer, ++uc) {
-        for (int c = 0; c < p.nchunk; ++c, ++cc) {
-          const int b = cc & 1;
-          const uint32_t ph = (cc >> 1) & 1;
-          if (!(ok = bwait(&a1full[b], ph, abort_flag, p.status))) break;
+    if (warp < 2 + kEpiWarps) {
+      const int ch = (warp - 2) >> 2;
+      uint32_t cc = 0;
+      for (int tile = blockIdx.x; ok && tile < p.ntiles; tile += gridDim.x) {
+        for (int layer = 0; ok && layer < p.M; ++layer) {
+          for (int c = 0; c < p.nchunk; ++c, ++cc) {
+            const int b = cc & 1;
+            if (!(ok = bwait(&a1full[b], (cc >> 1) & 1, abort_flag, p.status))) break;
+            __syncwarp();
+            tc_fence_after();
+            uint32_t packed[16];
+            {
+              uint32_t u[32], g[32];
+              const uint32_t a = tmem + lane_off + C::kAcc1 + b * 128 + ch * 32;
+              tmem_ld32(a, u);
+              tmem_ld32(a + 64, g);
+              tmem_ld_wait();
+#pragma unroll
+              for (int j = 0; j < 16; ++j) {
+                const float g0 = __uint_as_float(g[2 * j]), g1 = __uint_as_float(g[2 * j + 1]);
+                const float p0 = __uint_as_float(u[2 * j]) * g0;
+                const float p1 = __uint_as_float(u[2 * j + 1]) * g1;
+                packed[j] = pack_bf16x2(fmaf(p0, tanh_approx(g0), p0), fmaf(p1, tanh_approx(g1), p1));
+              }
+            }
+            // H (bf16 pairs) over this warp's own u columns, read above
+            tmem_st16(tmem + lane_off + C::kAcc1 + b * 128 + ch * 32, packed);
+            tmem_st_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&hfull[b]);
+          }
+        }
+      }
+    } else {
+      uint32_t uc = 0;
+      for (int tile = blockIdx.x; ok && tile < p.ntiles; tile += gridDim.x) {
+        const int64_t row = static_cast<int64_t>(tile) * 128 + row_in_tile;
+        for (int layer = 0; ok && layer < p.M; ++layer, ++uc) {
+          const int b2 = uc % AB2;
+          if (!(ok = bwait(&a2full[b2], (uc / AB2) & 1, abort_flag, p.status))) break;
           __syncwarp();
           tc_fence_after();
-          uint32_t packed[32];
-#pragma unroll
-          for (int half = 0; half < 2; ++half) {
-            uint32_t u[32], g[32];
-            const uint32_t a = tmem + lane_off + C::kAcc1 + b * 128 + half * 32;
-            tmem_ld32(a, u);
-            tmem_ld32(a + 64, g);
+          // row statistics, sums shifted by the row's first value against cancellation
+          const uint32_t arow = tmem + lane_off + C::kAcc2 + b2 * D;
+          float shift = 0.f, s1 = 0.f, s2 = 0.f;
+#pragma unroll 1
+          for (int cb = 0; cb < D / 32; ++cb) {
+            uint32_t v[32];
+            tmem_ld32(arow + cb * 32, v);
             tmem_ld_wait();
+            if (cb == 0) shift = __uint_as_float(v[0]);
 #pragma unroll
-            for (int j = 0; j < 16; ++j) {
-              const float g0 = __uint_as_float(g[2 * j]), g1 = __uint_as_float(g[2 * j + 1]);
-              const float p0 = __uint_as_float(u[2 * j]) * g0;
-              const float p1 = __uint_as_float(u[2 * j + 1]) * g1;
-              packed[half * 16 + j] =
-                  pack_bf16x2(fmaf(p0, tanh_approx(g0), p0), fmaf(p1, tanh_approx(g1), p1));
+            for (int j = 0; j < 32; ++j) {
+              const float x = __uint_as_float(v[j]) - shift;
+              s1 += x;
+              s2 = fmaf(x, x, s2);
+            }
+          }
+          const float m1 = s1 * (1.0f / D);
+          const float var = fmaxf(s2 * (1.0f / D) - m1 * m1, 0.f);
+          const float mean = shift + m1;
+          const float rstd = rsqrtf(var + 1e-5f);
+          const float4* gam = reinterpret_cast<const float4*>(p.ln_g[layer]);
+          const float4* bet = reinterpret_cast<const float4*>(p.ln_b[layer]);
+          uint8_t* orow = p.xt + (static_cast<int64_t>(layer) * p.N + row) * (D * 2);
+#pragma unroll 1
+          for (int cb = 0; cb < D / 32; ++cb) {
+            uint32_t v[32];
+            tmem_ld32(arow + cb * 32, v);
+            tmem_ld_wait();
+            uint32_t o[16];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              const float4 gg = __ldg(gam + cb * 8 + j);
+              const float4 bb = __ldg(bet + cb * 8 + j);
+              const float y0 = (__uint_as_float(v[4 * j]) - mean) * rstd * gg.x + bb.x;
+              const float y1 = (__uint_as_float(v[4 * j + 1]) - mean) * rstd * gg.y + bb.y;
+              const float y2 = (__uint_as_float(v[4 * j + 2]) - mean) * rstd * gg.z + bb.z;
+              const float y3 = (__uint_as_float(v[4 * j + 3]) - mean) * rstd * gg.w + bb.w;
+              o[2 * j] = pack_bf16x2(y0, y1);
+              o[2 * j + 1] = pack_bf16x2(y2, y3);
+            }
+            if (row < p.N) {
+              uint4* dst = reinterpret_cast<uint4*>(orow + cb * 64);
+#pragma unroll
+              for (int k = 0; k < 4; ++k) dst[k] = make_uint4(o[4 * k], o[4 * k + 1], o[4 * k + 2], o[4 * k + 3]);
             }
           }
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(&a1empty[b]);
-          if (!(ok = bwait(&hempty[b], ph ^ 1, abort_flag, p.status))) break;
-          __syncwarp();
-          const uint32_t hrow = sbase + C::oH + b * C::kBlock + row_in_tile * 128;
-#pragma unroll
-          for (int j = 0; j < 8; ++j)
-            st_shared_v4(hrow + ((j ^ (row_in_tile & 7)) << 4), packed[4 * j], packed[4 * j + 1],
-                         packed[4 * j + 2], packed[4 * j + 3]);
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&hfull[b]);
+          if (lane == 0) mbar_arrive(&a2empty[b2]);
         }
-        if (!ok) break;
-        // LayerNorm of the finished rows, bf16 store of X~(layer)
-        const int b2 = uc % AB2;
-        if (!(ok = bwait(&a2full[b2], (uc / AB2) & 1, abort_flag, p.status))) break;
-        __syncwarp();
-        tc_fence_after();
-        const uint32_t a2 = tmem + lane_off + C::kAcc2 + b2 * D;
-        float shift = 0.f, s1 = 0.f, s2 = 0.f;
-#pragma unroll 1
-        for (int cb = 0; cb < D / 32; ++cb) {
-          uint32_t v[32];
-          tmem_ld32(a2 + cb * 32, v);
-          tmem_ld_wait();
-          if (cb == 0) shift = __uint_as_float(v[0]);
-#pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const float x = __uint_as_float(v[j]) - shift;
-            s1 += x;
-            s2 = fmaf(x, x, s2);
-          }
-        }
-        const float m1 = s1 * (1.0f / D);
-        const float var = fmaxf(s2 * (1.0f / D) - m1 * m1, 0.f);
-        const float mean = shift + m1;
-        const float rstd = rsqrtf(var + 1e-5f);
-        const float* gam = p.ln_g[layer];
-        const float* bet = p.ln_b[layer];
-        uint8_t* orow = p.xt + (static_cast<int64_t>(layer) * p.N + row) * (D * 2);
-#pragma unroll 1
-        for (int cb = 0; cb < D / 32; ++cb) {
-          uint32_t v[32];
-          tmem_ld32(a2 + cb * 32, v);
-          tmem_ld_wait();
-          uint32_t o[16];
-#pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const int k = cb * 32 + 2 * j;
-            const float y0 = (__uint_as_float(v[2 * j]) - mean) * rstd * __ldg(gam + k) + __ldg(bet + k);
-            const float y1 = (__uint_as_float(v[2 * j + 1]) - mean) * rstd * __ldg(gam + k + 1) +
-                             __ldg(bet + k + 1);
-            o[j] = pack_bf16x2(y0, y1);
-          }
-          if (row < p.N) {
-            uint4* dst = reinterpret_cast<uint4*>(orow + cb * 64);
-#pragma unroll
-            for (int k = 0; k < 4; ++k) dst[k] = make_uint4(o[4 * k], o[4 * k + 1], o[4 * k + 2], o[4 * k + 3]);
-          }
-        }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&a2empty[b2]);
       }
     }
+    if (!ok) *abort_flag = 1;
   }
   tc_fence_before();
   __syncthreads();
@@ -459,9 +470,9 @@ int launch_encode_tc(stca_handle* H, const void* X, int64_t N, cudaStream_t s) {
   }
   p.status = H->status_d;
   switch (H->d) {
-    case 64: return launch_cfg<64, 2, 2, 4, 4>(H, tmX, p, s);
-    case 128: return launch_cfg<128, 2, 2, 4, 3>(H, tmX, p, s);
-    case 256: return launch_cfg<256, 1, 1, 3, 2>(H, tmX, p, s);
+    case 64: return launch_cfg<64, 2, 2, 8, 6>(H, tmX, p, s);
+    case 128: return launch_cfg<128, 2, 2, 6, 4>(H, tmX, p, s);
+    case 256: return launch_cfg<256, 1, 1, 6, 2>(H, tmX, p, s);
     default: return set_error(STCA_EINVAL, "tensor-core encoder needs d in {64, 128, 256}");
   }
 }

@@ -1,9 +1,7 @@
-// CUDA-core kernels of the STCA forward: the row-wise SwiGLU+LayerNorm encoder,
-// the split-L single-query attention and the per-target step (split combine,
-// W_V / W_O epilogue, Eq. (7) query fusion, the u = (q W_Q) W_K^T projection).
-//
-// These run the fp32 configuration (where tensor-core TF32 would not hold the
-// 1e-3 bound) and the per-target work of every configuration.  Sources: "Make
+// CUDA-core kernels of the STCA forward: the row-wise SwiGLU+LayerNorm encoder
+// and the split-L single-query attention.  They run the fp32 configuration
+// (where tensor-core TF32 would not hold the 1e-3 bound) and the sizes the
+// tensor-core kernels do not cover.  Sources: "Make
 // It Long, Keep It Fast" digest §2.1, Eqs. (1)-(8) and (13).
 #include <cuda_bf16.h>
 #include <math.h>
@@ -193,188 +191,6 @@ attn_simt_kernel(const void* __restrict__ Xt, const float* __restrict__ U,
   }
 }
 
-// ---------------------------------------------------------------- per-target
-// The per-target step after layer `layer`'s attention (layer >= 0): merge the
-// split partials into c_j = alpha_j X~ (Eq. (13)), o = [c_j W_V^j]_j W_O (Eq. (6)),
-// Z[t, layer, :] = o (Eq. (8)); then, unless layer is the last, the Eq. (7)
-// query fusion of layer+1 and its u projection.  layer == -1 computes
-// q(1) = LN(FFN_1(x_t)) (Eq. (3)) and the u projection of layer 0.
-constexpr int kTB = 4;   // targets per CTA
-
-struct StepArgs {
-  int layer, M, d, h, dh, rd;
-  int64_t T;
-  const void* targets;
-  StepPlan plan;
-  const float *pacc, *pm, *pl;
-  float* Z;
-  float* U;
-  uint16_t* Ubf;      // optional bf16 copy of U (tensor-core attention)
-  float uscale;       // folded into U: 1/sqrt(d_h), times log2(e) for exp2 kernels
-  LayerW32 cur, nxt;  // weights of `layer` (post) and `layer+1` (prep)
-  const float *q_ln_g, *q_ln_b;
-  int wa;             // width of buffer A per target
-  int wb;             // width of buffer B per target
-};
-
-// out[b][c] = sum_k in[b][k] * W[k][c] for c < n, b < nb.
-__device__ __forceinline__ void rows_matmul(const float* in, int ldin, int K, const float* W,
-                                            int64_t ldw, float* out, int ldout, int n, int nb) {
-  for (int c = threadIdx.x; c < n; c += blockDim.x) {
-    float acc[kTB];
-#pragma unroll
-    for (int b = 0; b < kTB; ++b) acc[b] = 0.f;
-    for (int k = 0; k < K; ++k) {
-      const float w = W[static_cast<int64_t>(k) * ldw + c];
-#pragma unroll
-      for (int b = 0; b < kTB; ++b) acc[b] = fmaf(in[b * ldin + k], w, acc[b]);
-    }
-    for (int b = 0; b < nb; ++b) out[b * ldout + c] = acc[b];
-  }
-}
-
-// x (nb rows of width d in `in`) -> SwiGLU FFN -> out (width d); scratch: 2rd + rd.
-__device__ void rows_ffn(const float* in, int ldin, const float* Wu, const float* Wg,
-                         const float* Wd, float* tmp2, float* tmp1, float* out, int ldout,
-                         int d, int rd, int nb) {
-  rows_matmul(in, ldin, d, Wu, rd, tmp2, 2 * rd, rd, nb);
-  rows_matmul(in, ldin, d, Wg, rd, tmp2 + rd, 2 * rd, rd, nb);
-  __syncthreads();
-  for (int e = threadIdx.x; e < nb * rd; e += blockDim.x) {
-    const int b = e / rd, c = e - b * rd;
-    tmp1[b * rd + c] = tmp2[b * 2 * rd + c] * silu_acc(tmp2[b * 2 * rd + rd + c]);
-  }
-  __syncthreads();
-  rows_matmul(tmp1, rd, rd, Wd, d, out, ldout, d, nb);
-  __syncthreads();
-}
-
-template <bool XBF>
-__global__ void __launch_bounds__(kThreads) target_step_kernel(StepArgs a) {
-  extern __shared__ float sm[];
-  const int d = a.d, h = a.h, dh = a.dh, rd = a.rd;
-  float* xs = sm;                       // kTB x d: raw x_t
-  float* A = xs + kTB * d;              // kTB x wa
-  float* B = A + kTB * a.wa;            // kTB x wb
-  float* C = B + kTB * a.wb;            // kTB x d
-  float* D = C + kTB * d;               // kTB x 2rd, then kTB x rd (FFN scratch)
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int64_t t0 = static_cast<int64_t>(blockIdx.x) * kTB;
-  const int nb = a.T - t0 < kTB ? static_cast<int>(a.T - t0) : kTB;
-  for (int e = tid; e < kTB * d; e += blockDim.x) {
-    const int b = e / d, k = e - b * d;
-    xs[e] = b < nb ? ld_elem<XBF>(a.targets, (t0 + b) * d + k) : 0.f;
-  }
-  __syncthreads();
-  const int layer = a.layer;
-  if (layer >= 0) {
-    // split combine: c_j = sum_w e^{m_w - m} acc_w / sum_w e^{m_w - m} l_w
-    const StepPlan& P = a.plan;
-    for (int pr = warp; pr < nb * h; pr += blockDim.x / 32) {
-      const int b = pr / h, j = pr - b * h;
-      const int64_t t = t0 + b;
-      const int r = P.treq[t];
-      const int64_t qrow = (t - P.toff[r]) * h + j;
-      const int64_t mt = qrow / P.mtile_rows;
-      const int64_t row = qrow - mt * P.mtile_rows;
-      const int pair = P.req_pair_begin[r] + static_cast<int>(mt);
-      const int w0 = P.pair_item_begin[pair], w1 = P.pair_item_begin[pair + 1];
-      float mx = -INFINITY;
-      for (int w = w0; w < w1; ++w) mx = fmaxf(mx, a.pm[P.items[w].row_base + row]);
-      float l = 0.f;
-      for (int w = w0; w < w1; ++w) {
-        const int64_t g = P.items[w].row_base + row;
-        const float f = P.log2_partials ? exp2f(a.pm[g] - mx) : expf(a.pm[g] - mx);
-        l = fmaf(a.pl[g], f, l);
-      }
-      const float inv = 1.0f / l;
-      for (int k = lane; k < d; k += 32) {
-        float v = 0.f;
-        for (int w = w0; w < w1; ++w) {
-          const int64_t g = P.items[w].row_base + row;
-          const float f = P.log2_partials ? exp2f(a.pm[g] - mx) : expf(a.pm[g] - mx);
-          v = fmaf(a.pacc[g * d + k], f, v);
-        }
-        A[b * a.wa + j * d + k] = v * inv;
-      }
-    }
-    __syncthreads();
-    // o_head[b][j dh + c] = sum_k c_j[k] W_V[k][j dh + c]
-    for (int cc = tid; cc < d; cc += blockDim.x) {
-      const int j = cc / dh;
-      float acc[kTB];
-#pragma unroll
-      for (int b = 0; b < kTB; ++b) acc[b] = 0.f;
-      for (int k = 0; k < d; ++k) {
-        const float w = a.cur.Wv[static_cast<int64_t>(k) * d + cc];
-#pragma unroll
-        for (int b = 0; b < kTB; ++b) acc[b] = fmaf(A[b * a.wa + j * d + k], w, acc[b]);
-      }
-      for (int b = 0; b < nb; ++b) B[b * a.wb + cc] = acc[b];
-    }
-    __syncthreads();
-    rows_matmul(B, a.wb, d, a.cur.Wo, d, C, d, d, nb);
-    __syncthreads();
-    for (int e = tid; e < nb * d; e += blockDim.x) {
-      const int b = e / d, k = e - b * d;
-      a.Z[((t0 + b) * a.M + layer) * d + k] = C[b * d + k];
-    }
-    __syncthreads();
-    if (layer + 1 >= a.M) return;
-    // Eq. (7): [o(1) || ... || o(layer+1) || x_t] W_C^(layer+2)
-    const int wcat = (layer + 2) * d;
-    for (int e = tid; e < nb * wcat; e += blockDim.x) {
-      const int b = e / wcat, k = e - b * wcat;
-      const int blk = k / d, kk = k - blk * d;
-      float v;
-      if (blk < layer) v = a.Z[((t0 + b) * a.M + blk) * d + kk];
-      else if (blk == layer) v = C[b * d + kk];
-      else v = xs[b * d + kk];
-      A[b * a.wa + k] = v;
-    }
-    __syncthreads();
-    rows_matmul(A, a.wa, wcat, a.nxt.Wc, d, B, a.wb, d, nb);
-    __syncthreads();
-    rows_ffn(B, a.wb, a.nxt.qWu, a.nxt.qWg, a.nxt.qWd, D, D + kTB * 2 * rd, C, d, d, rd, nb);
-  } else {
-    rows_ffn(xs, d, a.nxt.qWu, a.nxt.qWg, a.nxt.qWd, D, D + kTB * 2 * rd, C, d, d, rd, nb);
-    // LayerNorm of Eq. (3)
-    for (int b = warp; b < nb; b += blockDim.x / 32) {
-      float s = 0.f;
-      for (int k = lane; k < d; k += 32) s += C[b * d + k];
-      const float mean = warp_sum(s) / d;
-      float v = 0.f;
-      for (int k = lane; k < d; k += 32) { const float u = C[b * d + k] - mean; v = fmaf(u, u, v); }
-      const float rstd = 1.0f / sqrtf(warp_sum(v) / d + 1e-5f);
-      __syncwarp();
-      for (int k = lane; k < d; k += 32)
-        C[b * d + k] = (C[b * d + k] - mean) * rstd * a.q_ln_g[k] + a.q_ln_b[k];
-    }
-    __syncthreads();
-  }
-  // P = q W_Q of the next layer; u_j = P_j W_K^j^T, scaled (Eq. (13))
-  rows_matmul(C, d, d, a.nxt.Wq, d, B, a.wb, d, nb);
-  __syncthreads();
-  for (int cc = tid; cc < h * d; cc += blockDim.x) {
-    const int j = cc / d, k = cc - j * d;
-    float acc[kTB];
-#pragma unroll
-    for (int b = 0; b < kTB; ++b) acc[b] = 0.f;
-    const float* wk = a.nxt.WkT + static_cast<int64_t>(j) * dh * d + k;
-    for (int c = 0; c < dh; ++c) {
-      const float w = wk[static_cast<int64_t>(c) * d];
-#pragma unroll
-      for (int b = 0; b < kTB; ++b) acc[b] = fmaf(B[b * a.wb + j * dh + c], w, acc[b]);
-    }
-    for (int b = 0; b < nb; ++b) {
-      const float u = acc[b] * a.uscale;
-      const int64_t gi = (t0 + b) * h * d + cc;
-      if (a.U) a.U[gi] = u;
-      if (a.Ubf) a.Ubf[gi] = f32_to_bf16(u);
-    }
-  }
-}
-
 }  // namespace
 
 // ------------------------------------------------------------------ launchers
@@ -430,86 +246,6 @@ void launch_attn_simt(const stca_handle* H, int layer, const void* xt_layer,
     attn_simt_kernel<false><<<static_cast<unsigned>(npairs), kAttnWarps * 32, smem, s>>>(
         xt_layer, H->U, items_d, pairs_d, toff_d, pacc, pm, pl, H->d, H->h);
   }
-}
-
-static void step_widths(const stca_handle* H, int* wa, int* wb) {
-  const int d = H->d;
-  *wa = std::max(std::max(H->h * d, (H->M + 1) * d), d);
-  *wb = d;
-}
-
-size_t target_step_smem(const stca_handle* H) {
-  int wa, wb;
-  step_widths(H, &wa, &wb);
-  return static_cast<size_t>(kTB) * (H->d + wa + wb + H->d + 3 * H->rd) * sizeof(float);
-}
-
-void launch_target_step(const stca_handle* H, int layer, const void* targets, int64_t T,
-                        const StepPlan& plan, float* Z, cudaStream_t s) {
-  if (T <= 0) return;
-  StepArgs a{};
-  a.layer = layer;
-  a.M = H->M; a.d = H->d; a.h = H->h; a.dh = H->dh; a.rd = H->rd;
-  a.T = T;
-  a.targets = targets;
-  a.plan = plan;
-  const int64_t G = H->last_G;
-  a.pacc = H->part;
-  a.pm = H->part + G * H->d;
-  a.pl = a.pm + G;
-  a.Z = Z;
-  const bool tc = plan.log2_partials != 0;
-  a.U = tc ? nullptr : H->U;
-  a.Ubf = tc ? H->Ubf : nullptr;
-  // fold 1/sqrt(d_h) (and log2(e) for the exp2-based tensor-core kernel) into u
-  a.uscale = (tc ? 1.4426950408889634f : 1.0f) / sqrtf(static_cast<float>(H->dh));
-  if (layer >= 0) a.cur = H->L32[layer];
-  if (layer + 1 < H->M) a.nxt = H->L32[layer + 1];
-  a.q_ln_g = H->q_ln_g;
-  a.q_ln_b = H->q_ln_b;
-  step_widths(H, &a.wa, &a.wb);
-  const size_t smem = target_step_smem(H);
-  const unsigned grid = static_cast<unsigned>((T + kTB - 1) / kTB);
-  if (H->elem == 2) {
-    cudaFuncSetAttribute(target_step_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         (int)smem);
-    target_step_kernel<true><<<grid, kThreads, smem, s>>>(a);
-  } else {
-    cudaFuncSetAttribute(target_step_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         (int)smem);
-    target_step_kernel<false><<<grid, kThreads, smem, s>>>(a);
-  }
-}
-
-// Same launch as launch_target_step for the tensor-core partial layout, with
-// the bf16 query rows and the split partials in caller-given buffers.
-void launch_target_step_ws(const stca_handle* H, int layer, const void* targets, int64_t T,
-                           const StepPlan& plan, float* Z, uint16_t* Ubf, float* part,
-                           int64_t G, cudaStream_t s) {
-  if (T <= 0) return;
-  StepArgs a{};
-  a.layer = layer;
-  a.M = H->M; a.d = H->d; a.h = H->h; a.dh = H->dh; a.rd = H->rd;
-  a.T = T;
-  a.targets = targets;
-  a.plan = plan;
-  a.pacc = part;
-  a.pm = part + G * H->d;
-  a.pl = a.pm + G;
-  a.Z = Z;
-  a.U = nullptr;
-  a.Ubf = Ubf;
-  a.uscale = 1.4426950408889634f / sqrtf(static_cast<float>(H->dh));
-  if (layer >= 0) a.cur = H->L32[layer];
-  if (layer + 1 < H->M) a.nxt = H->L32[layer + 1];
-  a.q_ln_g = H->q_ln_g;
-  a.q_ln_b = H->q_ln_b;
-  step_widths(H, &a.wa, &a.wb);
-  const size_t smem = target_step_smem(H);
-  const unsigned grid = static_cast<unsigned>((T + kTB - 1) / kTB);
-  cudaFuncSetAttribute(target_step_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                       (int)smem);
-  target_step_kernel<true><<<grid, kThreads, smem, s>>>(a);
 }
 
 }  // namespace stca

@@ -166,6 +166,7 @@ extern "C" void stca_destroy(stca_handle* H) {
   DeviceGuard g(H->device);
   cudaDeviceSynchronize();
   cudaFree(H->w32);
+  cudaFree(H->wstep);
   cudaFree(H->wtc);
   cudaFree(H->xt);
   cudaFree(H->q);
@@ -191,6 +192,7 @@ extern "C" int stca_init(const stca_weights* w, int d, int h, int r, int M, int 
   if (!w) return set_error(STCA_EINVAL, "weights is NULL");
   if (d < 8 || d > 1024 || d % 8) return set_error(STCA_EINVAL, "d must be in [8, 1024], d % 8 == 0");
   if (h < 1 || d % h) return set_error(STCA_EINVAL, "h must divide d");
+  if ((d / h) % 2) return set_error(STCA_EINVAL, "h must divide d with an even d / h");
   if (r < 1 || static_cast<int64_t>(r) * d > 4096) return set_error(STCA_EINVAL, "need 1 <= r, r*d <= 4096");
   if (M < 1 || M > 16) return set_error(STCA_EINVAL, "M must be in [1, 16]");
   if (dtype != STCA_F32 && dtype != STCA_BF16) return set_error(STCA_EINVAL, "dtype must be STCA_F32 or STCA_BF16");
@@ -326,6 +328,33 @@ extern "C" int stca_init(const stca_weights* w, int d, int h, int r, int M, int 
   if (cudaDeviceGetAttribute(&H->num_sms, cudaDevAttrMultiProcessorCount, H->device) != cudaSuccess) {
     cudaGetLastError();
     H->num_sms = 148;
+  }
+  {
+    std::vector<StepHostW> sw(M);
+    for (int i = 0; i < M; ++i) {
+      sw[i].Wq = slab.data() + offs[i].Wq;
+      sw[i].Wk = nullptr;
+      sw[i].Wv = slab.data() + offs[i].Wv;
+      sw[i].Wo = slab.data() + offs[i].Wo;
+      sw[i].Wc = i > 0 ? slab.data() + offs[i].Wc : nullptr;
+      sw[i].qWu = slab.data() + offs[i].qWu;
+      sw[i].qWg = slab.data() + offs[i].qWg;
+      sw[i].qWd = slab.data() + offs[i].qWd;
+    }
+    // W_K in its original [d x d] layout, recovered from the per-head transpose
+    std::vector<std::vector<float>> wk(M, std::vector<float>(static_cast<size_t>(d) * d));
+    for (int i = 0; i < M; ++i) {
+      for (int j = 0; j < h; ++j)
+        for (int c = 0; c < dh; ++c)
+          for (int k = 0; k < d; ++k)
+            wk[i][static_cast<size_t>(k) * d + j * dh + c] =
+                slab[offs[i].WkT + (static_cast<size_t>(j) * dh + c) * d + k];
+      sw[i].Wk = wk[i].data();
+    }
+    if (int rc2 = step_weights_setup(H, sw)) {
+      stca_destroy(H);
+      return rc2;
+    }
   }
   if (dtype == STCA_BF16 && encode_tc_supported(d, rd)) {
     std::vector<const float*> Wu(M), Wg(M), Wd(M);

@@ -51,6 +51,23 @@ struct LayerW32 {
   const float *Wc;                  // (i+1)d x d, NULL for layer 0
 };
 
+// Per-layer weights of the per-target step, in the handle's element type
+// (bf16 bits or fp32), laid out by step_weights_setup (target_step.cu).
+struct LayerStep {
+  const void *Wq;    // d x d
+  const void *WkT;   // d_h x h d: WkT[c][j d + k] = W_K[k][j d_h + c]
+  const void *Wv;    // d x d
+  const void *Wo;    // d x d
+  const void *Wc;    // (i+1) d x d, NULL for layer 0
+  const void *Wug;   // d x 2rd: [query W_u | query W_g]
+  const void *Wd;    // rd x d: query W_d
+};
+
+// Host fp32 weights of one layer handed to step_weights_setup.
+struct StepHostW {
+  const float *Wq, *Wk, *Wv, *Wo, *Wc, *qWu, *qWg, *qWd;
+};
+
 }  // namespace stca
 
 struct stca_handle {
@@ -61,6 +78,8 @@ struct stca_handle {
 
   // weights
   float* w32 = nullptr;                 // fp32 slab
+  void* wstep = nullptr;                // per-target step weights (dtype)
+  std::vector<stca::LayerStep> Lstep;
   std::vector<stca::LayerW32> L32;
   const float* q_ln_g = nullptr;
   const float* q_ln_b = nullptr;
@@ -130,9 +149,11 @@ struct StepPlan {
   int mtile_rows;                   // query rows per tile (1 << 30: one tile per request)
   int log2_partials;                // partial maxima are in log2 units
 };
+// Per-target step (target_step.cu)
 void launch_target_step(const stca_handle* H, int layer, const void* targets, int64_t T,
                         const StepPlan& plan, float* Z, cudaStream_t s);
 size_t target_step_smem(const stca_handle* H);
+int step_weights_setup(stca_handle* H, const std::vector<StepHostW>& layers);
 size_t attn_simt_smem(const stca_handle* H);
 
 // Host-side attention work plan (stca_api.cu).

@@ -1,0 +1,469 @@
+// Per-target step of the STCA forward, between two attention layers:
+//   split combine   c_j = sum_w 2^{m_w - m} acc_w / sum_w 2^{m_w - m} l_w       (Eq. (13) alpha X~)
+//   output          o = [c_1 W_V^1 || ... || c_h W_V^h] W_O; Z[t, i, :] = o   (Eqs. (6), (8))
+//   query fusion    q = SwiGLUFFN_{i+1}([o(1) || ... || o(i+1) || x_t] W_C)  (Eq. (7))
+//   u projection    u_j = (q W_Q^j) W_K^j^T, scaled for the next attention     (Eq. (13))
+// and, before the first layer, q(1) = LN(SwiGLUFFN_1(x_t)) (Eq. (3)) and its u.
+// Sources: "Make It Long, Keep It Fast" digest §2.1.
+//
+// A CTA takes kTB targets and runs the whole chain for them with fp32
+// activations in shared memory.  Every matrix product goes through gemm_tb,
+// which streams the weight matrix (bf16 for bf16 handles, fp32 otherwise)
+// through a double-buffered shared-memory ring with cp.async and gives each
+// thread a pair of output columns for all kTB rows; narrow outputs split the K
+// range over thread groups and reduce in shared memory.
+#include <cuda_bf16.h>
+#include <math.h>
+
+#include <algorithm>
+#include <vector>
+
+#include "stca_internal.h"
+
+namespace stca {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kNB = 512;               // output columns per GEMM block (256 pairs)
+constexpr int kChunk = 16384;          // weight bytes per pipeline stage
+constexpr int kStages = 4;             // weight chunks in flight
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+__device__ __forceinline__ float silu_acc(float z) { return z / (1.0f + expf(-z)); }
+
+template <typename WT>
+__device__ __forceinline__ float2 load_pair(const unsigned char* p);
+template <>
+__device__ __forceinline__ float2 load_pair<uint16_t>(const unsigned char* p) {
+  const uint32_t v = *reinterpret_cast<const uint32_t*>(p);
+  return make_float2(__uint_as_float(v << 16), __uint_as_float(v & 0xFFFF0000u));
+}
+template <>
+__device__ __forceinline__ float2 load_pair<float>(const unsigned char* p) {
+  return *reinterpret_cast<const float2*>(p);
+}
+
+template <bool BF>
+__device__ __forceinline__ float ld_elem(const void* p, int64_t i) {
+  if constexpr (BF) return __uint_as_float(static_cast<uint32_t>(static_cast<const uint16_t*>(p)[i]) << 16);
+  else return static_cast<const float*>(p)[i];
+}
+
+// out[b][n] = sum_{k < K} in[b * ldin + (n / hc) * hs + k] * W[k * N + n], b < kTB, n < N.
+// `hc` columns share one input slice (a head), placed `hs` floats apart; a plain
+// product has hc = N, hs = 0.  W is row-major K x N in global memory.  Every
+// thread of the CTA must call this; it ends with the CTA synchronised.
+template <typename WT, int kTB>
+__device__ void gemm_tb(const float* in, int ldin, int hc, int hs, int K, const WT* W, int N,
+                        float* out, int ldout, unsigned char* wbuf, float* red) {
+  const int tid = threadIdx.x;
+  const bool vec4 = (ldin % 4 == 0) && (hs % 4 == 0) && (reinterpret_cast<uintptr_t>(in) % 16 == 0);
+  for (int n0 = 0; n0 < N; n0 += kNB) {
+    const int nb = min(kNB, N - n0);
+    const int np = nb >> 1;
+    const int gk = max(1, kThreads / np);                  // K groups
+    const int p = tid % np, g = tid / np;
+    const bool active = g < gk;
+    const int row_bytes = nb * static_cast<int>(sizeof(WT));
+    const int rows = max(1, kChunk / row_bytes);
+    const int nchunks = (K + rows - 1) / rows;
+    const int pieces_per_row = row_bytes >> 4;
+    auto issue = [&](int c) {
+      if (c >= nchunks) {          // keep one commit group per chunk slot
+        cp_async_commit();
+        return;
+      }
+      const int k0 = c * rows, kr = min(rows, K - k0);
+      unsigned char* dst = wbuf + (c % kStages) * kChunk;
+      const unsigned char* src = reinterpret_cast<const unsigned char*>(W + static_cast<int64_t>(k0) * N + n0);
+      for (int q = tid; q < kr * pieces_per_row; q += kThreads) {
+        const int rr = q / pieces_per_row, pc = q - rr * pieces_per_row;
+        cp_async16(dst + rr * row_bytes + pc * 16,
+                   src + static_cast<int64_t>(rr) * N * sizeof(WT) + pc * 16);
+      }
+      cp_async_commit();
+    };
+    float acc[kTB][2];
+#pragma unroll
+    for (int b = 0; b < kTB; ++b) acc[b][0] = acc[b][1] = 0.f;
+    const int col = n0 + 2 * p;
+    const float* inb = in + (col / hc) * hs;
+    for (int c = 0; c < kStages - 1; ++c) issue(c);
+    for (int c = 0; c < nchunks; ++c) {
+      issue(c + kStages - 1);
+      cp_async_wait<kStages - 1>();
+      __syncthreads();
+      const unsigned char* wb = wbuf + (c % kStages) * kChunk + p * 2 * sizeof(WT);
+      const int k0 = c * rows, kr = min(rows, K - k0);
+      if (active) {
+        // group g takes a contiguous slice of the chunk's rows, in steps of 4
+        const int per = ((kr + gk - 1) / gk + 3) & ~3;
+        const int kb = g * per, ke = min(kr, kb + per);
+        int kk = kb;
+        if (vec4 && ((k0 + kb) & 3) == 0) {
+          for (; kk + 4 <= ke; kk += 4) {
+            float2 w[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) w[u] = load_pair<WT>(wb + (kk + u) * row_bytes);
+#pragma unroll
+            for (int b = 0; b < kTB; ++b) {
+              const float4 x = *reinterpret_cast<const float4*>(inb + b * ldin + k0 + kk);
+              acc[b][0] = fmaf(x.x, w[0].x, acc[b][0]);
+              acc[b][1] = fmaf(x.x, w[0].y, acc[b][1]);
+              acc[b][0] = fmaf(x.y, w[1].x, acc[b][0]);
+              acc[b][1] = fmaf(x.y, w[1].y, acc[b][1]);
+              acc[b][0] = fmaf(x.z, w[2].x, acc[b][0]);
+              acc[b][1] = fmaf(x.z, w[2].y, acc[b][1]);
+              acc[b][0] = fmaf(x.w, w[3].x, acc[b][0]);
+              acc[b][1] = fmaf(x.w, w[3].y, acc[b][1]);
+            }
+          }
+        }
+        for (; kk < ke; ++kk) {
+          const float2 w = load_pair<WT>(wb + kk * row_bytes);
+#pragma unroll
+          for (int b = 0; b < kTB; ++b) {
+            const float x = inb[b * ldin + k0 + kk];
+            acc[b][0] = fmaf(x, w.x, acc[b][0]);
+            acc[b][1] = fmaf(x, w.y, acc[b][1]);
+          }
+        }
+      }
+      __syncthreads();
+    }
+    if (gk > 1) {
+      if (active) {
+#pragma unroll
+        for (int b = 0; b < kTB; ++b) {
+          red[(g * kTB + b) * nb + 2 * p] = acc[b][0];
+          red[(g * kTB + b) * nb + 2 * p + 1] = acc[b][1];
+        }
+      }
+      __syncthreads();
+      for (int e = tid; e < kTB * nb; e += kThreads) {
+        const int b = e / nb, n = e - b * nb;
+        float s = 0.f;
+        for (int q = 0; q < gk; ++q) s += red[(q * kTB + b) * nb + n];
+        out[b * ldout + n0 + n] = s;
+      }
+    } else if (active) {
+#pragma unroll
+      for (int b = 0; b < kTB; ++b) {
+        out[b * ldout + col] = acc[b][0];
+        out[b * ldout + col + 1] = acc[b][1];
+      }
+    }
+    __syncthreads();
+  }
+}
+
+struct StepArgs {
+  int layer, M, d, h, dh, rd;
+  int64_t T;
+  const void* targets;
+  StepPlan plan;
+  const float *pacc, *pm, *pl;
+  float* Z;
+  float* U;           // fp32 query rows (CUDA-core attention) or NULL
+  uint16_t* Ubf;      // bf16 query rows (tensor-core attention) or NULL
+  float uscale;       // 1/sqrt(d_h), times log2(e) for the exp2 kernels
+  LayerStep cur, nxt; // weights of `layer` (output) and `layer + 1` (query)
+  const float *q_ln_g, *q_ln_b;
+  int wa, wb;         // widths of buffers A and B per target
+};
+
+template <bool XBF, typename WT, int kTB>
+__global__ void __launch_bounds__(kThreads) target_step_kernel(StepArgs a) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  const int d = a.d, h = a.h, dh = a.dh, rd = a.rd;
+  unsigned char* wbuf = smem;                                       // kStages x kChunk
+  float* red = reinterpret_cast<float*>(smem + kStages * kChunk);   // kTB x kNB
+  float* xs = red + kTB * kNB;                                // kTB x d: raw x_t
+  float* A = xs + kTB * d;                                    // kTB x wa
+  float* B = A + kTB * a.wa;                                  // kTB x wb
+  float* C = B + kTB * a.wb;                                  // kTB x d
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int64_t t0 = static_cast<int64_t>(blockIdx.x) * kTB;
+  const int nb = a.T - t0 < kTB ? static_cast<int>(a.T - t0) : kTB;
+  for (int e = tid; e < kTB * d; e += blockDim.x) {
+    const int b = e / d, k = e - b * d;
+    xs[e] = b < nb ? ld_elem<XBF>(a.targets, (t0 + b) * d + k) : 0.f;
+  }
+  __syncthreads();
+  const int layer = a.layer;
+  if (layer >= 0) {
+    // split combine into A[b][j * d + k]
+    const StepPlan& P = a.plan;
+    for (int pr = warp; pr < kTB * h; pr += blockDim.x / 32) {
+      const int b = pr / h, j = pr - b * h;
+      if (b >= nb) {
+        for (int k = lane; k < d; k += 32) A[b * a.wa + j * d + k] = 0.f;
+        continue;
+      }
+      const int64_t t = t0 + b;
+      const int r = P.treq[t];
+      const int64_t qrow = (t - P.toff[r]) * h + j;
+      const int64_t mt = qrow / P.mtile_rows;
+      const int64_t row = qrow - mt * P.mtile_rows;
+      const int pair = P.req_pair_begin[r] + static_cast<int>(mt);
+      const int w0 = P.pair_item_begin[pair], w1 = P.pair_item_begin[pair + 1];
+      float mx = -INFINITY;
+      for (int w = w0; w < w1; ++w) mx = fmaxf(mx, a.pm[P.items[w].row_base + row]);
+      float l = 0.f;
+      for (int w = w0; w < w1; ++w) {
+        const int64_t g = P.items[w].row_base + row;
+        const float f = P.log2_partials ? exp2f(a.pm[g] - mx) : expf(a.pm[g] - mx);
+        l = fmaf(a.pl[g], f, l);
+      }
+      const float inv = 1.0f / l;
+      for (int k = lane; k < d; k += 32) {
+        float v = 0.f;
+        for (int w = w0; w < w1; ++w) {
+          const int64_t g = P.items[w].row_base + row;
+          const float f = P.log2_partials ? exp2f(a.pm[g] - mx) : expf(a.pm[g] - mx);
+          v = fmaf(a.pacc[g * d + k], f, v);
+        }
+        A[b * a.wa + j * d + k] = v * inv;
+      }
+    }
+    __syncthreads();
+    // o_head[b][j dh + c] = c_j . W_V[:, j dh + c]; o = o_head W_O
+    gemm_tb<WT, kTB>(A, a.wa, dh, d, d, static_cast<const WT*>(a.cur.Wv), d, B, a.wb, wbuf, red);
+    gemm_tb<WT, kTB>(B, a.wb, d, 0, d, static_cast<const WT*>(a.cur.Wo), d, C, d, wbuf, red);
+    for (int e = tid; e < nb * d; e += blockDim.x) {
+      const int b = e / d, k = e - b * d;
+      a.Z[((t0 + b) * a.M + layer) * d + k] = C[b * d + k];
+    }
+    if (layer + 1 >= a.M) return;
+    // Eq. (7): [o(1) || ... || o(layer+1) || x_t] W_C^(layer+2), then SwiGLU
+    const int wcat = (layer + 2) * d;
+    __syncthreads();
+    for (int e = tid; e < kTB * wcat; e += blockDim.x) {
+      const int b = e / wcat, k = e - b * wcat;
+      const int blk = k / d, kk = k - blk * d;
+      float v = 0.f;
+      if (b < nb) {
+        if (blk < layer) v = a.Z[((t0 + b) * a.M + blk) * d + kk];
+        else if (blk == layer) v = C[b * d + kk];
+        else v = xs[b * d + kk];
+      }
+      A[b * a.wa + k] = v;
+    }
+    __syncthreads();
+    gemm_tb<WT, kTB>(A, a.wa, wcat, 0, wcat, static_cast<const WT*>(a.nxt.Wc), d, B, a.wb, wbuf, red);
+    gemm_tb<WT, kTB>(B, a.wb, 2 * rd, 0, d, static_cast<const WT*>(a.nxt.Wug), 2 * rd, A, a.wa, wbuf, red);
+  } else {
+    gemm_tb<WT, kTB>(xs, d, 2 * rd, 0, d, static_cast<const WT*>(a.nxt.Wug), 2 * rd, A, a.wa, wbuf, red);
+  }
+  // gate: B[b][c] = u * SiLU(g); then the down projection into C
+  for (int e = tid; e < kTB * rd; e += blockDim.x) {
+    const int b = e / rd, c = e - b * rd;
+    B[b * a.wb + c] = A[b * a.wa + c] * silu_acc(A[b * a.wa + rd + c]);
+  }
+  __syncthreads();
+  gemm_tb<WT, kTB>(B, a.wb, d, 0, rd, static_cast<const WT*>(a.nxt.Wd), d, C, d, wbuf, red);
+  if (layer < 0) {
+    // LayerNorm of Eq. (3)
+    for (int b = warp; b < kTB; b += blockDim.x / 32) {
+      float s = 0.f;
+      for (int k = lane; k < d; k += 32) s += C[b * d + k];
+      const float mean = warp_sum(s) / d;
+      float v = 0.f;
+      for (int k = lane; k < d; k += 32) { const float u = C[b * d + k] - mean; v = fmaf(u, u, v); }
+      const float rstd = 1.0f / sqrtf(warp_sum(v) / d + 1e-5f);
+      __syncwarp();
+      for (int k = lane; k < d; k += 32)
+        C[b * d + k] = (C[b * d + k] - mean) * rstd * a.q_ln_g[k] + a.q_ln_b[k];
+    }
+    __syncthreads();
+  }
+  // P = q W_Q (into B); u_j = P_j W_K^j^T (into A, [b][j][k]); store scaled
+  gemm_tb<WT, kTB>(C, d, d, 0, d, static_cast<const WT*>(a.nxt.Wq), d, B, a.wb, wbuf, red);
+  gemm_tb<WT, kTB>(B, a.wb, d, dh, dh, static_cast<const WT*>(a.nxt.WkT), h * d, A, a.wa, wbuf, red);
+  for (int e = tid; e < nb * h * d; e += blockDim.x) {
+    const int b = e / (h * d), cc = e - b * (h * d);
+    const float u = A[b * a.wa + cc] * a.uscale;
+    const int64_t gi = (t0 + b) * h * d + cc;
+    if (a.U) a.U[gi] = u;
+    if (a.Ubf) a.Ubf[gi] = __bfloat16_as_ushort(__float2bfloat16_rn(u));
+  }
+}
+
+void step_widths(const stca_handle* H, int* wa, int* wb) {
+  const int d = H->d;
+  *wa = std::max(std::max(H->h * d, H->M * d), 2 * H->rd);
+  *wb = std::max(d, H->rd);
+}
+
+size_t smem_for(const stca_handle* H, int tb) {
+  int wa, wb;
+  step_widths(H, &wa, &wb);
+  return static_cast<size_t>(kStages) * kChunk + static_cast<size_t>(tb) * kNB * sizeof(float) +
+         static_cast<size_t>(tb) * (H->d + wa + wb + H->d) * sizeof(float);
+}
+
+// Targets per CTA: 8, or 4 when 8 do not fit in shared memory.
+int choose_tb(const stca_handle* H) { return smem_for(H, 8) <= 227 * 1024 ? 8 : 4; }
+
+template <int TB>
+void launch_tb(const stca_handle* H, const StepArgs& a, cudaStream_t s) {
+  const size_t smem = smem_for(H, TB);
+  const unsigned grid = static_cast<unsigned>((a.T + TB - 1) / TB);
+  if (H->elem == 2) {
+    auto k = target_step_kernel<true, uint16_t, TB>;
+    cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    k<<<grid, kThreads, smem, s>>>(a);
+  } else {
+    auto k = target_step_kernel<false, float, TB>;
+    cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    k<<<grid, kThreads, smem, s>>>(a);
+  }
+}
+
+void launch(const stca_handle* H, const StepArgs& a0, cudaStream_t s) {
+  StepArgs a = a0;
+  step_widths(H, &a.wa, &a.wb);
+  if (choose_tb(H) == 8) launch_tb<8>(H, a, s);
+  else launch_tb<4>(H, a, s);
+}
+
+StepArgs base_args(const stca_handle* H, int layer, const void* targets, int64_t T,
+                   const StepPlan& plan, float* Z) {
+  StepArgs a{};
+  a.layer = layer;
+  a.M = H->M; a.d = H->d; a.h = H->h; a.dh = H->dh; a.rd = H->rd;
+  a.T = T;
+  a.targets = targets;
+  a.plan = plan;
+  a.Z = Z;
+  if (layer >= 0) a.cur = H->Lstep[layer];
+  if (layer + 1 < H->M) a.nxt = H->Lstep[layer + 1];
+  a.q_ln_g = H->q_ln_g;
+  a.q_ln_b = H->q_ln_b;
+  return a;
+}
+
+}  // namespace
+
+size_t target_step_smem(const stca_handle* H) { return smem_for(H, choose_tb(H)); }
+
+void launch_target_step(const stca_handle* H, int layer, const void* targets, int64_t T,
+                        const StepPlan& plan, float* Z, cudaStream_t s) {
+  if (T <= 0) return;
+  StepArgs a = base_args(H, layer, targets, T, plan, Z);
+  const int64_t G = H->last_G;
+  a.pacc = H->part;
+  a.pm = H->part + G * H->d;
+  a.pl = a.pm + G;
+  const bool tc = plan.log2_partials != 0;
+  a.U = tc ? nullptr : H->U;
+  a.Ubf = tc ? H->Ubf : nullptr;
+  a.uscale = (tc ? 1.4426950408889634f : 1.0f) / sqrtf(static_cast<float>(H->dh));
+  launch(H, a, s);
+}
+
+void launch_target_step_ws(const stca_handle* H, int layer, const void* targets, int64_t T,
+                           const StepPlan& plan, float* Z, uint16_t* Ubf, float* part,
+                           int64_t G, cudaStream_t s) {
+  if (T <= 0) return;
+  StepArgs a = base_args(H, layer, targets, T, plan, Z);
+  a.pacc = part;
+  a.pm = part + G * H->d;
+  a.pl = a.pm + G;
+  a.U = nullptr;
+  a.Ubf = Ubf;
+  a.uscale = 1.4426950408889634f / sqrtf(static_cast<float>(H->dh));
+  launch(H, a, s);
+}
+
+// Lay out the per-target weights of every layer in the handle's element type:
+// W_Q, W_K^T per head as one [d_h x h d] matrix, W_V, W_O, W_C, the query
+// SwiGLU up/gate as one [d x 2rd] matrix [W_u | W_g], and W_d.
+int step_weights_setup(stca_handle* H, const std::vector<StepHostW>& layers) {
+  const int d = H->d, h = H->h, dh = H->dh, rd = H->rd, M = H->M;
+  auto pad = [](size_t n) { return (n + 15) & ~size_t(15); };
+  std::vector<float> host;
+  struct Off { size_t Wq, WkT, Wv, Wo, Wc, Wug, Wd; };
+  std::vector<Off> offs(M);
+  for (int i = 0; i < M; ++i) {
+    const StepHostW& L = layers[i];
+    Off& o = offs[i];
+    auto put = [&](const float* src, size_t n) {
+      const size_t at = host.size();
+      host.resize(at + pad(n), 0.f);
+      if (src) std::copy(src, src + n, host.begin() + at);
+      return at;
+    };
+    o.Wq = put(L.Wq, static_cast<size_t>(d) * d);
+    o.WkT = put(nullptr, static_cast<size_t>(dh) * h * d);
+    for (int c = 0; c < dh; ++c)          // WkT[c][j d + k] = W_K[k][j dh + c]
+      for (int j = 0; j < h; ++j)
+        for (int k = 0; k < d; ++k)
+          host[o.WkT + static_cast<size_t>(c) * h * d + j * d + k] = L.Wk[static_cast<size_t>(k) * d + j * dh + c];
+    o.Wv = put(L.Wv, static_cast<size_t>(d) * d);
+    o.Wo = put(L.Wo, static_cast<size_t>(d) * d);
+    o.Wc = i > 0 ? put(L.Wc, static_cast<size_t>(i + 1) * d * d) : 0;
+    o.Wug = put(nullptr, static_cast<size_t>(d) * 2 * rd);
+    for (int k = 0; k < d; ++k)
+      for (int c = 0; c < rd; ++c) {
+        host[o.Wug + static_cast<size_t>(k) * 2 * rd + c] = L.qWu[static_cast<size_t>(k) * rd + c];
+        host[o.Wug + static_cast<size_t>(k) * 2 * rd + rd + c] = L.qWg[static_cast<size_t>(k) * rd + c];
+      }
+    o.Wd = put(L.qWd, static_cast<size_t>(rd) * d);
+  }
+  const size_t n = host.size();
+  const size_t esz = H->elem == 2 ? 2 : 4;
+  std::vector<unsigned char> bytes(n * esz);
+  if (esz == 2) {
+    uint16_t* dst = reinterpret_cast<uint16_t*>(bytes.data());
+    for (size_t k = 0; k < n; ++k) {
+      uint32_t u;
+      memcpy(&u, &host[k], 4);
+      dst[k] = static_cast<uint16_t>(u >> 16);     // values are bf16-exact
+    }
+  } else {
+    memcpy(bytes.data(), host.data(), n * 4);
+  }
+  if (cudaMalloc(&H->wstep, bytes.size()) != cudaSuccess) {
+    cudaGetLastError();
+    return set_error(STCA_ENOMEM, "per-target weight allocation failed");
+  }
+  STCA_CUDA_TRY(cudaMemcpy(H->wstep, bytes.data(), bytes.size(), cudaMemcpyHostToDevice));
+  H->Lstep.resize(M);
+  const unsigned char* base = static_cast<const unsigned char*>(H->wstep);
+  for (int i = 0; i < M; ++i) {
+    const Off& o = offs[i];
+    LayerStep& L = H->Lstep[i];
+    L.Wq = base + o.Wq * esz;
+    L.WkT = base + o.WkT * esz;
+    L.Wv = base + o.Wv * esz;
+    L.Wo = base + o.Wo * esz;
+    L.Wc = i > 0 ? base + o.Wc * esz : nullptr;
+    L.Wug = base + o.Wug * esz;
+    L.Wd = base + o.Wd * esz;
+  }
+  return STCA_OK;
+}
+
+}  // namespace stca

@@ -66,6 +66,7 @@ def _weights(d, r, M, dtype=np.float32):
 @pytest.mark.parametrize("d,h,r,M,dtype,word", [
     (12, 2, 1, 1, S.STCA_F32, "d must"),      # d % 8
     (16, 3, 1, 1, S.STCA_F32, "h must"),      # h does not divide d
+    (16, 16, 1, 1, S.STCA_F32, "even"),       # odd d / h
     (16, 2, 0, 1, S.STCA_F32, "r"),           # r < 1
     (16, 2, 1, 0, S.STCA_F32, "M must"),      # M < 1
     (16, 2, 1, 17, S.STCA_F32, "M must"),     # M too large
