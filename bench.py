@@ -428,7 +428,7 @@ def run_ours(args, rank, world, local_rank):
         "e2e": e2e,
         "gpu_launches": int(launches_per_step * args.steps),
         "clocks": sampler.summary(),
-        "when": datetime.datetime.utcnow().isoformat() + "Z",
+        "when": datetime.datetime.now(datetime.timezone.utc).isoformat(),
     }
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = oracle_sample(wl, budget_s=args.cpu_budget)

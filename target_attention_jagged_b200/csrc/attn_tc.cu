@@ -154,6 +154,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
+      const uint64_t stream_policy = policy_evict_first();   // X~ is read once per layer
       uint32_t qi = 0, ki = 0;
       bool ok = true;
       for (int it = it0; ok && it < it1; ++it) {
@@ -171,8 +172,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           if (!(ok = bwait(&kempty[s], ((ki / KS) & 1) ^ 1, abort_flag, p.status))) break;
           mbar_arrive_expect_tx(&kfull[s], C::kTile);
           for (int kb = 0; kb < C::KB; ++kb)
-            tma_load_2d(sm + C::oK + s * C::kTile + kb * C::kBlock, &tmK, kb * 64,
-                        static_cast<int>(item.key0 + j * 128), &kfull[s]);
+            tma_load_2d_hint(sm + C::oK + s * C::kTile + kb * C::kBlock, &tmK, kb * 64,
+                             static_cast<int>(item.key0 + j * 128), &kfull[s], stream_policy);
           ++ki;
         }
       }

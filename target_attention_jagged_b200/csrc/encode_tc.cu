@@ -142,6 +142,7 @@ encode_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
+      const uint64_t stream_policy = policy_evict_first();   // X is read once
       uint32_t r1 = 0, r2 = 0, xi = 0;
       bool ok = true;
       for (int tile = blockIdx.x; ok && tile < p.ntiles; tile += gridDim.x) {
@@ -149,8 +150,8 @@ encode_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
         if (!(ok = bwait(&xempty[xb], ((xi / XB) & 1) ^ 1, abort_flag, p.status))) break;
         mbar_arrive_expect_tx(&xfull[xb], C::kXBytes);
         for (int kb = 0; kb < C::KB; ++kb)
-          tma_load_2d(sm + C::oX + xb * C::kXBytes + kb * C::kBlock, &tmX, kb * 64, tile * 128,
-                      &xfull[xb]);
+          tma_load_2d_hint(sm + C::oX + xb * C::kXBytes + kb * C::kBlock, &tmX, kb * 64,
+                           tile * 128, &xfull[xb], stream_policy);
         ++xi;
         for (int layer = 0; ok && layer < p.M; ++layer) {
           for (int c = 0; ok && c < p.nchunk; ++c) {
@@ -296,6 +297,7 @@ encode_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
         }
       }
     } else {
+      const uint64_t out_policy = policy_evict_first();      // X~ is written once here
       uint32_t uc = 0;
       for (int tile = blockIdx.x; ok && tile < p.ntiles; tile += gridDim.x) {
         const int64_t row = static_cast<int64_t>(tile) * 128 + row_in_tile;
@@ -347,7 +349,9 @@ encode_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
             if (row < p.N) {
               uint4* dst = reinterpret_cast<uint4*>(orow + cb * 64);
 #pragma unroll
-              for (int k = 0; k < 4; ++k) dst[k] = make_uint4(o[4 * k], o[4 * k + 1], o[4 * k + 2], o[4 * k + 3]);
+              for (int k = 0; k < 4; ++k)
+                st_global_v4_hint(dst + k, make_uint4(o[4 * k], o[4 * k + 1], o[4 * k + 2], o[4 * k + 3]),
+                                  out_policy);
             }
           }
           tc_fence_before();

@@ -173,6 +173,7 @@ extern "C" void stca_destroy(stca_handle* H) {
   cudaFree(H->U);
   cudaFree(H->Ubf);
   cudaFree(H->part);
+  cudaFree(H->cbuf);
   cudaFree(H->plan_d);
   cudaFree(H->status_d);
   cudaFree(H->x_stage);
@@ -680,6 +681,8 @@ extern "C" int stca_forward(stca_handle* H, const void* targets, const int64_t* 
   if (int rc = ensure_dev(reinterpret_cast<void**>(&H->part), &H->part_cap,
                           static_cast<size_t>(std::max<int64_t>(H->last_G, 1)) * (d + 2) * sizeof(float)))
     return rc;
+  if (int rc = ensure_dev(reinterpret_cast<void**>(&H->cbuf), &H->cbuf_cap, urows * d * sizeof(float)))
+    return rc;
   char* p = static_cast<char*>(H->plan_d);
   const AttnItem* items_d = reinterpret_cast<const AttnItem*>(p + H->off_items);
   const int32_t* pairs_d = reinterpret_cast<const int32_t*>(p + H->off_pairs);
@@ -695,7 +698,7 @@ extern "C" int stca_forward(stca_handle* H, const void* targets, const int64_t* 
   const size_t layer_bytes = static_cast<size_t>(H->N) * d * H->elem;
   {
     TimedLaunch tl(H, STCA_K_STEP, s);
-    launch_target_step(H, -1, targets, T, plan, Z, s);
+    launch_target_step(H, -1, targets, T, plan, nullptr, Z, s);
   }
   H->launches++;
   if (int rc = check_launch("query init")) return rc;
@@ -715,9 +718,10 @@ extern "C" int stca_forward(stca_handle* H, const void* targets, const int64_t* 
     if (int rc2 = check_launch("attention")) return rc2;
     {
       TimedLaunch tl(H, STCA_K_STEP, s);
-      launch_target_step(H, i, targets, T, plan, Z, s);
+      launch_combine(H, plan, H->part, H->last_G, T, H->cbuf, s);
+      launch_target_step(H, i, targets, T, plan, H->cbuf, Z, s);
     }
-    H->launches++;
+    H->launches += 2;
     if (int rc2 = check_launch("target step")) return rc2;
   }
   return ok();
@@ -816,6 +820,7 @@ extern "C" int stca_device_status(stca_handle* H, void* stream) {
     std::string m = "device status 0x" + std::to_string(st) + ":";
     if (st & kStatusEncodeTimeout) m += " encoder gave up a bounded wait;";
     if (st & kStatusAttnTimeout) m += " attention gave up a bounded wait;";
+    if (st & kStatusStepTimeout) m += " per-target step gave up a bounded wait;";
     return set_error(STCA_EDEVICE, m);
   }
   return ok();

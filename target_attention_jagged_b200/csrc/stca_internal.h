@@ -23,7 +23,7 @@ int set_error(int code, const std::string& msg);
   } while (0)
 
 // Device status word bits written by kernels that give up a bounded wait.
-enum : int { kStatusEncodeTimeout = 1, kStatusAttnTimeout = 2 };
+enum : int { kStatusEncodeTimeout = 1, kStatusAttnTimeout = 2, kStatusStepTimeout = 4 };
 
 // ---------------------------------------------------------------- work plan
 // One attention work item: a contiguous key range of one request's history
@@ -111,6 +111,7 @@ struct stca_handle {
   float* U = nullptr;       size_t U_cap = 0;      // T x h x d (scaled)
   uint16_t* Ubf = nullptr;  size_t Ubf_cap = 0;    // bf16 copy for tensor cores
   float* part = nullptr;    size_t part_cap = 0;   // G x (d + 2)
+  float* cbuf = nullptr;    size_t cbuf_cap = 0;   // T x h x d: merged alpha X~ rows
   void* plan_d = nullptr;   size_t plan_cap = 0;   // uploaded plan arrays
   void* plan_h = nullptr;   size_t plan_h_cap = 0; // pinned staging
   cudaEvent_t plan_evt = nullptr;
@@ -150,8 +151,10 @@ struct StepPlan {
   int log2_partials;                // partial maxima are in log2 units
 };
 // Per-target step (target_step.cu)
+void launch_combine(const stca_handle* H, const StepPlan& plan, const float* part, int64_t G,
+                    int64_t T, float* out, cudaStream_t s);
 void launch_target_step(const stca_handle* H, int layer, const void* targets, int64_t T,
-                        const StepPlan& plan, float* Z, cudaStream_t s);
+                        const StepPlan& plan, const float* cmerged, float* Z, cudaStream_t s);
 size_t target_step_smem(const stca_handle* H);
 int step_weights_setup(stca_handle* H, const std::vector<StepHostW>& layers);
 size_t attn_simt_smem(const stca_handle* H);
@@ -171,8 +174,7 @@ void build_plan_host(const int64_t* off, const int64_t* toff, int64_t R, int h, 
 int check_plan(const PlanHost& P, const int64_t* off, const int64_t* toff, int64_t R, int h,
                int path);
 void launch_target_step_ws(const stca_handle* H, int layer, const void* targets, int64_t T,
-                           const StepPlan& plan, float* Z, uint16_t* Ubf, float* part,
-                           int64_t G, cudaStream_t s);
+                           const float* cmerged, float* Z, uint16_t* Ubf, cudaStream_t s);
 int launch_attn_tc_ws(int d, const CUtensorMap& tmQ, const CUtensorMap& tmK,
                       const AttnItem* items_d, const int32_t* cta_begin_d, int grid, float* part,
                       int64_t G, int* status, cudaStream_t s);

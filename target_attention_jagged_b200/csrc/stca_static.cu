@@ -21,7 +21,8 @@
 // (different streams, or different handles on one device) race on it, so
 // order such calls on one stream or serialise them.  A call reads nothing that
 // an earlier call left there: the plan, the query rows and every partial row
-// it reads are written by the same call first.
+// it reads are written by the same call first.  Workspace per call: the plan,
+// T*h*d bf16 query rows, T*h*d fp32 merged rows and the split partials.
 #include <cuda_runtime.h>
 #include <string.h>
 
@@ -64,7 +65,7 @@ size_t up256(size_t x) { return (x + 255) & ~size_t(255); }
 
 // Scratch layout of one call.
 struct StaticLayout {
-  size_t items, cta, treq, toff, rpb, pib, plan_end, ubf, part, total;
+  size_t items, cta, treq, toff, rpb, pib, plan_end, ubf, cbuf, part, total;
 };
 
 StaticLayout layout_for(const PlanHost& P, int64_t R, int64_t T, int h, int d) {
@@ -77,7 +78,8 @@ StaticLayout layout_for(const PlanHost& P, int64_t R, int64_t T, int h, int d) {
   L.pib = up256(L.rpb + static_cast<size_t>(R + 1) * sizeof(int32_t));
   L.plan_end = up256(L.pib + P.pair_item_begin.size() * sizeof(int32_t));
   L.ubf = L.plan_end;
-  L.part = up256(L.ubf + static_cast<size_t>(T) * h * d * 2);
+  L.cbuf = up256(L.ubf + static_cast<size_t>(T) * h * d * 2);
+  L.part = up256(L.cbuf + static_cast<size_t>(T) * h * d * sizeof(float));
   L.total = up256(L.part + static_cast<size_t>(std::max<int64_t>(P.G, 1)) * (d + 2) * sizeof(float));
   return L;
 }
@@ -153,6 +155,7 @@ extern "C" int stca_forward_static(stca_handle* H, const void* targets,
   const int32_t* cta_d = reinterpret_cast<const int32_t*>(sc + L.cta);
   uint16_t* Ubf = reinterpret_cast<uint16_t*>(sc + L.ubf);
   float* part = reinterpret_cast<float*>(sc + L.part);
+  float* cbuf = reinterpret_cast<float*>(sc + L.cbuf);
   CUtensorMap tmU;
   if (int rc = make_tmap_bf16_2d(&tmU, Ubf, d, static_cast<uint64_t>(T) * h, 64, 128)) return rc;
   StepPlan plan;
@@ -164,7 +167,7 @@ extern "C" int stca_forward_static(stca_handle* H, const void* targets,
   plan.mtile_rows = 128;
   plan.log2_partials = 1;
 
-  launch_target_step_ws(H, -1, targets, T, plan, Z, Ubf, part, P.G, s);
+  launch_target_step_ws(H, -1, targets, T, nullptr, Z, Ubf, s);
   if (cudaError_t e = cudaGetLastError())
     return set_error(STCA_ECUDA, std::string("query init: ") + cudaGetErrorString(e));
   for (int i = 0; i < H->M; ++i) {
@@ -173,7 +176,8 @@ extern "C" int stca_forward_static(stca_handle* H, const void* targets,
       return rc;
     if (cudaError_t e = cudaGetLastError())
       return set_error(STCA_ECUDA, std::string("attention: ") + cudaGetErrorString(e));
-    launch_target_step_ws(H, i, targets, T, plan, Z, Ubf, part, P.G, s);
+    launch_combine(H, plan, part, P.G, T, cbuf, s);
+    launch_target_step_ws(H, i, targets, T, cbuf, Z, Ubf, s);
     if (cudaError_t e = cudaGetLastError())
       return set_error(STCA_ECUDA, std::string("target step: ") + cudaGetErrorString(e));
   }

@@ -7,11 +7,11 @@
 // Sources: "Make It Long, Keep It Fast" digest §2.1.
 //
 // A CTA takes kTB targets and runs the whole chain for them with fp32
-// activations in shared memory.  Every matrix product goes through gemm_tb,
-// which streams the weight matrix (bf16 for bf16 handles, fp32 otherwise)
-// through a double-buffered shared-memory ring with cp.async and gives each
-// thread a pair of output columns for all kTB rows; narrow outputs split the K
-// range over thread groups and reduce in shared memory.
+// activations in shared memory.  Every matrix product streams its weight
+// matrix (bf16 for bf16 handles, fp32 otherwise) through a 4-stage ring of
+// bulk TMA copies, and gives each thread a pair of output columns for all kTB
+// rows; narrow outputs split the K range over thread groups and reduce in
+// shared memory.
 #include <cuda_bf16.h>
 #include <math.h>
 
@@ -19,29 +19,66 @@
 #include <vector>
 
 #include "stca_internal.h"
+#include "tc_common.cuh"
 
 namespace stca {
 namespace {
 
-constexpr int kThreads = 256;
+constexpr int kThreads = 512;
 constexpr int kNB = 512;               // output columns per GEMM block (256 pairs)
 constexpr int kChunk = 16384;          // weight bytes per pipeline stage
 constexpr int kStages = 4;             // weight chunks in flight
 
-__device__ __forceinline__ uint32_t smem_u32(const void* p) {
-  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+using stca::tc::smem_u32;
+
+// Weight ring: kStages shared-memory stages filled by bulk TMA copies (one per
+// row segment, or one per stage when the rows are contiguous), each stage
+// completing on its own mbarrier.  Chunk q of the kernel's whole sequence of
+// products lands in stage q % kStages; its phase parity is (q / kStages) & 1.
+struct Ring {
+  unsigned char* buf;     // kStages x stage bytes
+  uint64_t* bar;          // kStages mbarriers
+  int* status;            // device status word (bounded waits)
+  uint32_t q;             // chunks consumed so far in this kernel
+};
+
+__device__ __forceinline__ void bulk_copy(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
 }
 
-__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src)
-               : "memory");
+// Issue chunk q: `rows` rows of `row_bytes` from src (row pitch src_pitch) to
+// stage q % kStages (row pitch dst_pitch).  Called by every thread; thread 0 issues.
+__device__ __forceinline__ void ring_issue(Ring& R, uint32_t q, int stage_bytes, const unsigned char* src,
+                                           int rows, int row_bytes, int64_t src_pitch, int dst_pitch) {
+  if (threadIdx.x != 0) return;
+  const int st = q % kStages;
+  unsigned char* dst = R.buf + st * stage_bytes;
+  uint64_t* bar = &R.bar[st];
+  stca::tc::mbar_arrive_expect_tx(bar, static_cast<uint32_t>(rows * row_bytes));
+  if (src_pitch == row_bytes && dst_pitch == row_bytes) {
+    bulk_copy(dst, src, static_cast<uint32_t>(rows * row_bytes), bar);
+  } else {
+    for (int r = 0; r < rows; ++r)
+      bulk_copy(dst + r * dst_pitch, src + r * src_pitch, static_cast<uint32_t>(row_bytes), bar);
+  }
 }
-__device__ __forceinline__ void cp_async_commit() {
-  asm volatile("cp.async.commit_group;" ::: "memory");
-}
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+
+// Wait until chunk q has landed (bounded; a timeout is reported and skipped).
+__device__ __forceinline__ void ring_wait(Ring& R, uint32_t q) {
+  uint64_t* bar = &R.bar[q % kStages];
+  const uint32_t parity = (q / kStages) & 1;
+  if (stca::tc::mbar_try_wait(bar, parity)) return;
+  const uint64_t t0 = stca::tc::globaltimer();
+  while (!stca::tc::mbar_try_wait(bar, parity)) {
+    if (stca::tc::globaltimer() - t0 > stca::tc::kWaitTimeoutNs) {
+      atomicOr(R.status, kStatusStepTimeout);
+      return;
+    }
+  }
 }
 
 __device__ __forceinline__ float warp_sum(float v) {
@@ -74,35 +111,27 @@ __device__ __forceinline__ float ld_elem(const void* p, int64_t i) {
 // `hc` columns share one input slice (a head), placed `hs` floats apart; a plain
 // product has hc = N, hs = 0.  W is row-major K x N in global memory.  Every
 // thread of the CTA must call this; it ends with the CTA synchronised.
-template <typename WT, int kTB>
+template <typename WT, int kTB, int NT>
 __device__ void gemm_tb(const float* in, int ldin, int hc, int hs, int K, const WT* W, int N,
-                        float* out, int ldout, unsigned char* wbuf, float* red) {
+                        float* out, int ldout, Ring& R, float* red) {
+  unsigned char* wbuf = R.buf;
   const int tid = threadIdx.x;
   const bool vec4 = (ldin % 4 == 0) && (hs % 4 == 0) && (reinterpret_cast<uintptr_t>(in) % 16 == 0);
   for (int n0 = 0; n0 < N; n0 += kNB) {
     const int nb = min(kNB, N - n0);
     const int np = nb >> 1;
-    const int gk = max(1, kThreads / np);                  // K groups
+    const int gk = max(1, NT / np);                        // K groups
     const int p = tid % np, g = tid / np;
     const bool active = g < gk;
     const int row_bytes = nb * static_cast<int>(sizeof(WT));
     const int rows = max(1, kChunk / row_bytes);
     const int nchunks = (K + rows - 1) / rows;
-    const int pieces_per_row = row_bytes >> 4;
     auto issue = [&](int c) {
-      if (c >= nchunks) {          // keep one commit group per chunk slot
-        cp_async_commit();
-        return;
-      }
+      if (c >= nchunks) return;
       const int k0 = c * rows, kr = min(rows, K - k0);
-      unsigned char* dst = wbuf + (c % kStages) * kChunk;
-      const unsigned char* src = reinterpret_cast<const unsigned char*>(W + static_cast<int64_t>(k0) * N + n0);
-      for (int q = tid; q < kr * pieces_per_row; q += kThreads) {
-        const int rr = q / pieces_per_row, pc = q - rr * pieces_per_row;
-        cp_async16(dst + rr * row_bytes + pc * 16,
-                   src + static_cast<int64_t>(rr) * N * sizeof(WT) + pc * 16);
-      }
-      cp_async_commit();
+      ring_issue(R, R.q + c, kChunk,
+                 reinterpret_cast<const unsigned char*>(W + static_cast<int64_t>(k0) * N + n0), kr,
+                 row_bytes, static_cast<int64_t>(N) * sizeof(WT), row_bytes);
     };
     float acc[kTB][2];
 #pragma unroll
@@ -112,9 +141,8 @@ __device__ void gemm_tb(const float* in, int ldin, int hc, int hs, int K, const 
     for (int c = 0; c < kStages - 1; ++c) issue(c);
     for (int c = 0; c < nchunks; ++c) {
       issue(c + kStages - 1);
-      cp_async_wait<kStages - 1>();
-      __syncthreads();
-      const unsigned char* wb = wbuf + (c % kStages) * kChunk + p * 2 * sizeof(WT);
+      ring_wait(R, R.q + c);
+      const unsigned char* wb = wbuf + ((R.q + c) % kStages) * kChunk + p * 2 * sizeof(WT);
       const int k0 = c * rows, kr = min(rows, K - k0);
       if (active) {
         // group g takes a contiguous slice of the chunk's rows, in steps of 4
@@ -152,6 +180,7 @@ __device__ void gemm_tb(const float* in, int ldin, int hc, int hs, int K, const 
       }
       __syncthreads();
     }
+    R.q += nchunks;
     if (gk > 1) {
       if (active) {
 #pragma unroll
@@ -161,7 +190,7 @@ __device__ void gemm_tb(const float* in, int ldin, int hc, int hs, int K, const 
         }
       }
       __syncthreads();
-      for (int e = tid; e < kTB * nb; e += kThreads) {
+      for (int e = tid; e < kTB * nb; e += NT) {
         const int b = e / nb, n = e - b * nb;
         float s = 0.f;
         for (int q = 0; q < gk; ++q) s += red[(q * kTB + b) * nb + n];
@@ -178,13 +207,92 @@ __device__ void gemm_tb(const float* in, int ldin, int hc, int hs, int K, const 
   }
 }
 
+template <typename WT, int kTB>
+__device__ __forceinline__ void gemm(const float* in, int ldin, int hc, int hs, int K, const void* W,
+                                     int N, float* out, int ldout, Ring& R, float* red) {
+  gemm_tb<WT, kTB, kThreads>(in, ldin, hc, hs, K, static_cast<const WT*>(W), N, out, ldout, R, red);
+}
+
+// ---------------------------------------------------------------- split combine
+// c_j = sum_w s_w acc_w / sum_w s_w l_w with s_w = e^(m_w - m) (2^ for the
+// tensor-core partials) over the items w that cover query row (t, j): the
+// attention-weighted history alpha_j X~ of Eq. (13).  One CTA per query row;
+// the first warp reads the items' (m, l) with one lane per item.
+constexpr int kCombineThreads = 128;
+constexpr int kCombineMaxItems = 32;
+
+__global__ void __launch_bounds__(kCombineThreads)
+combine_kernel(StepPlan P, const float* __restrict__ pacc, const float* __restrict__ pm,
+               const float* __restrict__ pl, float* __restrict__ out, int d, int h) {
+  __shared__ int64_t sg[kCombineMaxItems];
+  __shared__ float sf[kCombineMaxItems];
+  __shared__ int s_nw;
+  const int64_t qr = blockIdx.x;          // target t, head j: row t * h + j of U
+  const int64_t t = qr / h;
+  const int j = static_cast<int>(qr - t * h);
+  const int r = P.treq[t];
+  const int64_t qrow = (t - P.toff[r]) * h + j;
+  const int64_t mt = qrow / P.mtile_rows;
+  const int64_t row = qrow - mt * P.mtile_rows;
+  const int pair = P.req_pair_begin[r] + static_cast<int>(mt);
+  const int w0 = P.pair_item_begin[pair], w1 = P.pair_item_begin[pair + 1];
+  const int nw = w1 - w0;
+  const int tid = threadIdx.x;
+  if (nw <= kCombineMaxItems) {
+    if (tid < 32) {
+      int64_t g = 0;
+      float m = -INFINITY, l = 0.f;
+      if (tid < nw) {
+        g = P.items[w0 + tid].row_base + row;
+        m = pm[g];
+        l = pl[g];
+      }
+      float mx = m;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+      const float f = tid < nw ? (P.log2_partials ? exp2f(m - mx) : expf(m - mx)) : 0.f;
+      float ls = l * f;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) ls += __shfl_xor_sync(0xffffffffu, ls, o);
+      if (tid < nw) {
+        sg[tid] = g;
+        sf[tid] = f / ls;
+      }
+      if (tid == 0) s_nw = nw;
+    }
+    __syncthreads();
+    for (int k = tid; k < d; k += kCombineThreads) {
+      float v = 0.f;
+      for (int w = 0; w < s_nw; ++w) v = fmaf(pacc[sg[w] * d + k], sf[w], v);
+      out[qr * d + k] = v;
+    }
+  } else {
+    // many splits of one pair: serial over the items
+    float mx = -INFINITY;
+    for (int w = w0; w < w1; ++w) mx = fmaxf(mx, pm[P.items[w].row_base + row]);
+    float l = 0.f;
+    for (int w = w0; w < w1; ++w) {
+      const int64_t g = P.items[w].row_base + row;
+      l = fmaf(pl[g], P.log2_partials ? exp2f(pm[g] - mx) : expf(pm[g] - mx), l);
+    }
+    for (int k = tid; k < d; k += kCombineThreads) {
+      float v = 0.f;
+      for (int w = w0; w < w1; ++w) {
+        const int64_t g = P.items[w].row_base + row;
+        v = fmaf(pacc[g * d + k], P.log2_partials ? exp2f(pm[g] - mx) : expf(pm[g] - mx), v);
+      }
+      out[qr * d + k] = v / l;
+    }
+  }
+}
+
 struct StepArgs {
   int layer, M, d, h, dh, rd;
   int64_t T;
   const void* targets;
-  StepPlan plan;
-  const float *pacc, *pm, *pl;
+  const float* cmerged;   // T x h x d: c_j = alpha_j X~ of the layer just attended
   float* Z;
+  int* status;        // device status word
   float* U;           // fp32 query rows (CUDA-core attention) or NULL
   uint16_t* Ubf;      // bf16 query rows (tensor-core attention) or NULL
   float uscale;       // 1/sqrt(d_h), times log2(e) for the exp2 kernels
@@ -197,63 +305,46 @@ template <bool XBF, typename WT, int kTB>
 __global__ void __launch_bounds__(kThreads) target_step_kernel(StepArgs a) {
   extern __shared__ __align__(16) unsigned char smem[];
   const int d = a.d, h = a.h, dh = a.dh, rd = a.rd;
-  unsigned char* wbuf = smem;                                       // kStages x kChunk
-  float* red = reinterpret_cast<float*>(smem + kStages * kChunk);   // kTB x kNB
-  float* xs = red + kTB * kNB;                                // kTB x d: raw x_t
-  float* A = xs + kTB * d;                                    // kTB x wa
+  const int ldd = d + 8;     // padded row strides spread rows over the shared-memory banks
+  constexpr int kRing = kStages * kChunk;
+  constexpr int kRed = kTB * 2 * kThreads;
+  unsigned char* wbuf = smem;                                 // weight ring
+  uint64_t* rbar = reinterpret_cast<uint64_t*>(smem + kRing); // kStages ring mbarriers
+  float* red = reinterpret_cast<float*>(smem + kRing + 128);  // K-split partials
+  float* xs = red + kRed;                                     // kTB x ldd: raw x_t
+  float* A = xs + kTB * ldd;                                  // kTB x wa
   float* B = A + kTB * a.wa;                                  // kTB x wb
-  float* C = B + kTB * a.wb;                                  // kTB x d
+  float* C = B + kTB * a.wb;                                  // kTB x ldd
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  if (tid == 0) {
+    for (int i = 0; i < kStages; ++i) stca::tc::mbar_init(&rbar[i], 1);
+    stca::tc::fence_mbar_init();
+  }
+  Ring R{wbuf, rbar, a.status, 0};
   const int64_t t0 = static_cast<int64_t>(blockIdx.x) * kTB;
   const int nb = a.T - t0 < kTB ? static_cast<int>(a.T - t0) : kTB;
   for (int e = tid; e < kTB * d; e += blockDim.x) {
     const int b = e / d, k = e - b * d;
-    xs[e] = b < nb ? ld_elem<XBF>(a.targets, (t0 + b) * d + k) : 0.f;
+    xs[b * ldd + k] = b < nb ? ld_elem<XBF>(a.targets, (t0 + b) * d + k) : 0.f;
   }
   __syncthreads();
   const int layer = a.layer;
   if (layer >= 0) {
-    // split combine into A[b][j * d + k]
-    const StepPlan& P = a.plan;
-    for (int pr = warp; pr < kTB * h; pr += blockDim.x / 32) {
-      const int b = pr / h, j = pr - b * h;
-      if (b >= nb) {
-        for (int k = lane; k < d; k += 32) A[b * a.wa + j * d + k] = 0.f;
-        continue;
-      }
-      const int64_t t = t0 + b;
-      const int r = P.treq[t];
-      const int64_t qrow = (t - P.toff[r]) * h + j;
-      const int64_t mt = qrow / P.mtile_rows;
-      const int64_t row = qrow - mt * P.mtile_rows;
-      const int pair = P.req_pair_begin[r] + static_cast<int>(mt);
-      const int w0 = P.pair_item_begin[pair], w1 = P.pair_item_begin[pair + 1];
-      float mx = -INFINITY;
-      for (int w = w0; w < w1; ++w) mx = fmaxf(mx, a.pm[P.items[w].row_base + row]);
-      float l = 0.f;
-      for (int w = w0; w < w1; ++w) {
-        const int64_t g = P.items[w].row_base + row;
-        const float f = P.log2_partials ? exp2f(a.pm[g] - mx) : expf(a.pm[g] - mx);
-        l = fmaf(a.pl[g], f, l);
-      }
-      const float inv = 1.0f / l;
-      for (int k = lane; k < d; k += 32) {
-        float v = 0.f;
-        for (int w = w0; w < w1; ++w) {
-          const int64_t g = P.items[w].row_base + row;
-          const float f = P.log2_partials ? exp2f(a.pm[g] - mx) : expf(a.pm[g] - mx);
-          v = fmaf(a.pacc[g * d + k], f, v);
-        }
-        A[b * a.wa + j * d + k] = v * inv;
-      }
+    // c_j rows of these targets (merged by combine_kernel) into A[b][j * d + k]
+    const int hd = h * d;
+    for (int e = tid * 4; e < kTB * hd; e += blockDim.x * 4) {
+      const int b = e / hd, c = e - b * hd;
+      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (b < nb) v = *reinterpret_cast<const float4*>(a.cmerged + (t0 + b) * hd + c);
+      *reinterpret_cast<float4*>(A + b * a.wa + c) = v;
     }
     __syncthreads();
     // o_head[b][j dh + c] = c_j . W_V[:, j dh + c]; o = o_head W_O
-    gemm_tb<WT, kTB>(A, a.wa, dh, d, d, static_cast<const WT*>(a.cur.Wv), d, B, a.wb, wbuf, red);
-    gemm_tb<WT, kTB>(B, a.wb, d, 0, d, static_cast<const WT*>(a.cur.Wo), d, C, d, wbuf, red);
+    gemm<WT, kTB>(A, a.wa, dh, d, d, a.cur.Wv, d, B, a.wb, R, red);
+    gemm<WT, kTB>(B, a.wb, d, 0, d, a.cur.Wo, d, C, ldd, R, red);
     for (int e = tid; e < nb * d; e += blockDim.x) {
       const int b = e / d, k = e - b * d;
-      a.Z[((t0 + b) * a.M + layer) * d + k] = C[b * d + k];
+      a.Z[((t0 + b) * a.M + layer) * d + k] = C[b * ldd + k];
     }
     if (layer + 1 >= a.M) return;
     // Eq. (7): [o(1) || ... || o(layer+1) || x_t] W_C^(layer+2), then SwiGLU
@@ -265,16 +356,16 @@ __global__ void __launch_bounds__(kThreads) target_step_kernel(StepArgs a) {
       float v = 0.f;
       if (b < nb) {
         if (blk < layer) v = a.Z[((t0 + b) * a.M + blk) * d + kk];
-        else if (blk == layer) v = C[b * d + kk];
-        else v = xs[b * d + kk];
+        else if (blk == layer) v = C[b * ldd + kk];
+        else v = xs[b * ldd + kk];
       }
       A[b * a.wa + k] = v;
     }
     __syncthreads();
-    gemm_tb<WT, kTB>(A, a.wa, wcat, 0, wcat, static_cast<const WT*>(a.nxt.Wc), d, B, a.wb, wbuf, red);
-    gemm_tb<WT, kTB>(B, a.wb, 2 * rd, 0, d, static_cast<const WT*>(a.nxt.Wug), 2 * rd, A, a.wa, wbuf, red);
+    gemm<WT, kTB>(A, a.wa, wcat, 0, wcat, a.nxt.Wc, d, B, a.wb, R, red);
+    gemm<WT, kTB>(B, a.wb, 2 * rd, 0, d, a.nxt.Wug, 2 * rd, A, a.wa, R, red);
   } else {
-    gemm_tb<WT, kTB>(xs, d, 2 * rd, 0, d, static_cast<const WT*>(a.nxt.Wug), 2 * rd, A, a.wa, wbuf, red);
+    gemm<WT, kTB>(xs, ldd, 2 * rd, 0, d, a.nxt.Wug, 2 * rd, A, a.wa, R, red);
   }
   // gate: B[b][c] = u * SiLU(g); then the down projection into C
   for (int e = tid; e < kTB * rd; e += blockDim.x) {
@@ -282,25 +373,25 @@ __global__ void __launch_bounds__(kThreads) target_step_kernel(StepArgs a) {
     B[b * a.wb + c] = A[b * a.wa + c] * silu_acc(A[b * a.wa + rd + c]);
   }
   __syncthreads();
-  gemm_tb<WT, kTB>(B, a.wb, d, 0, rd, static_cast<const WT*>(a.nxt.Wd), d, C, d, wbuf, red);
+  gemm<WT, kTB>(B, a.wb, d, 0, rd, a.nxt.Wd, d, C, ldd, R, red);
   if (layer < 0) {
     // LayerNorm of Eq. (3)
     for (int b = warp; b < kTB; b += blockDim.x / 32) {
       float s = 0.f;
-      for (int k = lane; k < d; k += 32) s += C[b * d + k];
+      for (int k = lane; k < d; k += 32) s += C[b * ldd + k];
       const float mean = warp_sum(s) / d;
       float v = 0.f;
-      for (int k = lane; k < d; k += 32) { const float u = C[b * d + k] - mean; v = fmaf(u, u, v); }
+      for (int k = lane; k < d; k += 32) { const float u = C[b * ldd + k] - mean; v = fmaf(u, u, v); }
       const float rstd = 1.0f / sqrtf(warp_sum(v) / d + 1e-5f);
       __syncwarp();
       for (int k = lane; k < d; k += 32)
-        C[b * d + k] = (C[b * d + k] - mean) * rstd * a.q_ln_g[k] + a.q_ln_b[k];
+        C[b * ldd + k] = (C[b * ldd + k] - mean) * rstd * a.q_ln_g[k] + a.q_ln_b[k];
     }
     __syncthreads();
   }
   // P = q W_Q (into B); u_j = P_j W_K^j^T (into A, [b][j][k]); store scaled
-  gemm_tb<WT, kTB>(C, d, d, 0, d, static_cast<const WT*>(a.nxt.Wq), d, B, a.wb, wbuf, red);
-  gemm_tb<WT, kTB>(B, a.wb, d, dh, dh, static_cast<const WT*>(a.nxt.WkT), h * d, A, a.wa, wbuf, red);
+  gemm<WT, kTB>(C, ldd, d, 0, d, a.nxt.Wq, d, B, a.wb, R, red);
+  gemm<WT, kTB>(B, a.wb, d, dh, dh, a.nxt.WkT, h * d, A, a.wa, R, red);
   for (int e = tid; e < nb * h * d; e += blockDim.x) {
     const int b = e / (h * d), cc = e - b * (h * d);
     const float u = A[b * a.wa + cc] * a.uscale;
@@ -312,15 +403,16 @@ __global__ void __launch_bounds__(kThreads) target_step_kernel(StepArgs a) {
 
 void step_widths(const stca_handle* H, int* wa, int* wb) {
   const int d = H->d;
-  *wa = std::max(std::max(H->h * d, H->M * d), 2 * H->rd);
-  *wb = std::max(d, H->rd);
+  *wa = std::max(std::max(H->h * d, H->M * d), 2 * H->rd) + 8;
+  *wb = std::max(d, H->rd) + 8;
 }
 
 size_t smem_for(const stca_handle* H, int tb) {
   int wa, wb;
   step_widths(H, &wa, &wb);
-  return static_cast<size_t>(kStages) * kChunk + static_cast<size_t>(tb) * kNB * sizeof(float) +
-         static_cast<size_t>(tb) * (H->d + wa + wb + H->d) * sizeof(float);
+  return static_cast<size_t>(kStages) * kChunk + 128 +
+         static_cast<size_t>(tb) * 2 * kThreads * sizeof(float) +
+         static_cast<size_t>(tb) * (2 * (H->d + 8) + wa + wb) * sizeof(float);
 }
 
 // Targets per CTA: 8, or 4 when 8 do not fit in shared memory.
@@ -349,14 +441,15 @@ void launch(const stca_handle* H, const StepArgs& a0, cudaStream_t s) {
 }
 
 StepArgs base_args(const stca_handle* H, int layer, const void* targets, int64_t T,
-                   const StepPlan& plan, float* Z) {
+                   const float* cmerged, float* Z) {
   StepArgs a{};
   a.layer = layer;
   a.M = H->M; a.d = H->d; a.h = H->h; a.dh = H->dh; a.rd = H->rd;
   a.T = T;
   a.targets = targets;
-  a.plan = plan;
+  a.cmerged = cmerged;
   a.Z = Z;
+  a.status = H->status_d;
   if (layer >= 0) a.cur = H->Lstep[layer];
   if (layer + 1 < H->M) a.nxt = H->Lstep[layer + 1];
   a.q_ln_g = H->q_ln_g;
@@ -366,16 +459,22 @@ StepArgs base_args(const stca_handle* H, int layer, const void* targets, int64_t
 
 }  // namespace
 
-size_t target_step_smem(const stca_handle* H) { return smem_for(H, choose_tb(H)); }
+size_t target_step_smem(const stca_handle* H) { return smem_for(H, 4); }
+
+void launch_combine(const stca_handle* H, const StepPlan& plan, const float* part, int64_t G,
+                    int64_t T, float* out, cudaStream_t s) {
+  if (T <= 0) return;
+  const float* pacc = part;
+  const float* pm = part + G * H->d;
+  const float* pl = pm + G;
+  combine_kernel<<<static_cast<unsigned>(T * H->h), kCombineThreads, 0, s>>>(plan, pacc, pm, pl,
+                                                                              out, H->d, H->h);
+}
 
 void launch_target_step(const stca_handle* H, int layer, const void* targets, int64_t T,
-                        const StepPlan& plan, float* Z, cudaStream_t s) {
+                        const StepPlan& plan, const float* cmerged, float* Z, cudaStream_t s) {
   if (T <= 0) return;
-  StepArgs a = base_args(H, layer, targets, T, plan, Z);
-  const int64_t G = H->last_G;
-  a.pacc = H->part;
-  a.pm = H->part + G * H->d;
-  a.pl = a.pm + G;
+  StepArgs a = base_args(H, layer, targets, T, cmerged, Z);
   const bool tc = plan.log2_partials != 0;
   a.U = tc ? nullptr : H->U;
   a.Ubf = tc ? H->Ubf : nullptr;
@@ -384,13 +483,9 @@ void launch_target_step(const stca_handle* H, int layer, const void* targets, in
 }
 
 void launch_target_step_ws(const stca_handle* H, int layer, const void* targets, int64_t T,
-                           const StepPlan& plan, float* Z, uint16_t* Ubf, float* part,
-                           int64_t G, cudaStream_t s) {
+                           const float* cmerged, float* Z, uint16_t* Ubf, cudaStream_t s) {
   if (T <= 0) return;
-  StepArgs a = base_args(H, layer, targets, T, plan, Z);
-  a.pacc = part;
-  a.pm = part + G * H->d;
-  a.pl = a.pm + G;
+  StepArgs a = base_args(H, layer, targets, T, cmerged, Z);
   a.U = nullptr;
   a.Ubf = Ubf;
   a.uscale = 1.4426950408889634f / sqrtf(static_cast<float>(H->dh));
