@@ -258,12 +258,48 @@ def storage_weights(wl):
     return out
 
 
-def roofline_of(kind, kt, c, wl, peaks, sustained, steps):
+KERNEL_SOURCES = {"encode": "encode_tc.cu", "attention": "attn_tc.cu", "target_step": "target_step.cu"}
+
+
+def source_hash(kind):
+    """sha256 (first 16 hex digits) of a kernel class's sources: its .cu file
+    followed by the shared tcgen05/TMA helper header."""
+    import hashlib
+    h = hashlib.sha256()
+    for f in (KERNEL_SOURCES[kind], "tc_common.cuh"):
+        with open(os.path.join(ROOT, "target_attention_jagged_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kind, config_key):
+    """DRAM bytes per launch from the committed ncu summary, or None when the
+    summary is for another workload or the kernel's sources changed since.
+    The per-target class times combine + step together, so only the encoder
+    and attention classes (one kernel per timed launch) carry a figure."""
+    p = os.path.join(ROOT, "profiles", "traffic.md")
+    if kind not in ("encode", "attention") or config_key != "c3" or not os.path.exists(p):
+        return None
+    with open(p) as f:
+        for line in f:
+            cells = [x.strip() for x in line.strip().strip("|").split("|")]
+            if len(cells) == 4 and cells[0] == kind:
+                try:
+                    nbytes = int(cells[2])
+                except ValueError:
+                    return None
+                return nbytes if cells[3] == source_hash(kind) else None
+    return None
+
+
+def roofline_of(kind, kt, c, wl, peaks, sustained, steps, config_key=None):
     """Roofline object of kernel class `kind` from its live event timings.
 
     Per launch, the algorithmic work is the class's per-step total divided by
     its launches per step (e.g. the encoder: M N 6 d rd FLOPs and 2 N d s bytes
     per layer; the attention: 4 h d sum_r T_r L_r FLOPs and N d s bytes per layer).
+    The tensor-core encoder runs all M layers in one launch and reads X once:
+    (M + 1) N d s bytes per launch.
     """
     ms, n = kt[kind]
     if n == 0 or ms <= 0:
@@ -271,12 +307,15 @@ def roofline_of(kind, kt, c, wl, peaks, sustained, steps):
     avg_s = ms / n / 1e3
     per_step = n / steps
     if kind == "encode":
-        flops, bytes_ = c["enc_flops"] / per_step, c["enc_bytes_per_layer"] * wl.M / per_step
+        enc_bytes = (wl.M + 1) * c["N"] * wl.d * c["elem"] if per_step == 1 else \
+            c["enc_bytes_per_layer"] * wl.M
+        flops, bytes_ = c["enc_flops"] / per_step, enc_bytes / per_step
     elif kind == "attention":
         flops, bytes_ = c["attn_flops"] / per_step, c["attn_bytes_per_layer"] * wl.M / per_step
     else:
         flops, bytes_ = c["tgt_flops"] / per_step, c["io_bytes"] / per_step
-    base = {"kernel": kind, "traffic": None, "avg_launch_ms": avg_s * 1e3,
+    traffic = recorded_traffic(kind, config_key) if wl.dtype == "bf16" else None
+    base = {"kernel": kind, "traffic": traffic, "avg_launch_ms": avg_s * 1e3,
             "flops_per_launch": flops, "bytes_per_launch": bytes_}
     if wl.dtype == "f32":
         peak = 148 * 128 * 2 * 1.965e9 / 1e12     # FP32 FFMA lanes x clock (nominal)
@@ -299,6 +338,7 @@ def run_ours(args, rank, world, local_rank):
     import torch
     import torch.distributed as dist
     import target_attention_jagged_b200 as S
+    from target_attention_jagged_b200.shard import max_over_ranks
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
@@ -342,19 +382,15 @@ def run_ours(args, rank, world, local_rank):
         torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
-    elapsed_ms = e0.elapsed_time(e1)
     kt = S.stca_kernel_times(st.handle)
     st.set_option(S.STCA_OPT_TIMING, 0)
     st.status(stream)
-    if world > 1:
-        t = torch.tensor([elapsed_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed_ms = float(t.item())
+    elapsed_ms = max_over_ranks(e0.elapsed_time(e1), dev)
     sec = elapsed_ms / 1e3
     value = world * wl.N * args.steps / sec
     targets_per_s = world * wl.T * args.steps / sec
     sustained = sec > 1.0
-    rooflines = {k: roofline_of(k, kt, c, wl, peaks, sustained, args.steps) for k in kt}
+    rooflines = {k: roofline_of(k, kt, c, wl, peaks, sustained, args.steps, args.config) for k in kt}
     for r_ in rooflines.values():
         if r_:
             r_["peak_source"] += f" ({peak_src})"
@@ -399,11 +435,7 @@ def run_ours(args, rank, world, local_rank):
         S.stca_run_host(st.handle, Xh, wl.offsets, th, wl.target_offsets, Zh, stream)
     g1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = g0.elapsed_time(g1)
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(g0.elapsed_time(g1), dev)
     e2e = {"value": world * wl.N * args.steps / (e2e_ms / 1e3), "unit": UNIT,
            "h2d_bytes_per_step": int(Xh.numel() * Xh.element_size() + th.numel() * th.element_size()
                                      + 2 * 8 * (wl.R + 1)),

@@ -1,0 +1,64 @@
+"""Data-parallel sharding of a jagged STCA batch over ranks (host logic only).
+
+Requests never interact: each request's output depends only on its own
+history and targets ("Make It Long, Keep It Fast" digest §2.2), so a batch
+shards over GPUs by whole requests with no exchange on the data path.  This
+module balances requests by their work and cuts the jagged arrays; the
+per-rank forward is the ordinary single-GPU call.
+"""
+from __future__ import annotations
+
+import heapq
+from typing import List, Sequence
+
+import numpy as np
+
+
+def request_work(lengths, target_counts, d: int, h: int, M: int, r: int) -> np.ndarray:
+    """Work estimate per request: M layers of the encoder (6 d rd per history
+    token) plus the attention (4 h d per history token and target)."""
+    L = np.asarray(lengths, dtype=np.float64)
+    T = np.asarray(target_counts, dtype=np.float64)
+    return M * (6.0 * d * r * d * L + 4.0 * h * d * T * L)
+
+
+def partition_requests(work: Sequence[float], world: int) -> List[np.ndarray]:
+    """Greedy longest-processing-time: each request, heaviest first, goes to the
+    rank with the least work so far.  Returns each rank's request indices in
+    increasing order (the order of the original batch)."""
+    if world < 1:
+        raise ValueError("world must be >= 1")
+    w = np.asarray(work, dtype=np.float64)
+    heap = [(0.0, k) for k in range(world)]
+    owned: List[list] = [[] for _ in range(world)]
+    for i in np.argsort(-w, kind="stable"):
+        load, k = heapq.heappop(heap)
+        owned[k].append(int(i))
+        heapq.heappush(heap, (load + float(w[i]), k))
+    return [np.asarray(sorted(o), dtype=np.int64) for o in owned]
+
+
+def shard_offsets(offsets, target_offsets, requests):
+    """Rows of X, rows of the targets and the new offset arrays of a shard."""
+    off = np.asarray(offsets, dtype=np.int64)
+    toff = np.asarray(target_offsets, dtype=np.int64)
+    reqs = np.asarray(requests, dtype=np.int64)
+    x_rows = np.concatenate([np.arange(off[q], off[q + 1]) for q in reqs]) if len(reqs) else \
+        np.zeros(0, dtype=np.int64)
+    t_rows = np.concatenate([np.arange(toff[q], toff[q + 1]) for q in reqs]) if len(reqs) else \
+        np.zeros(0, dtype=np.int64)
+    new_off = np.concatenate([[0], np.cumsum(off[reqs + 1] - off[reqs])]).astype(np.int64)
+    new_toff = np.concatenate([[0], np.cumsum(toff[reqs + 1] - toff[reqs])]).astype(np.int64)
+    return x_rows, t_rows, new_off, new_toff
+
+
+def max_over_ranks(value: float, device=None) -> float:
+    """The maximum of `value` over the default process group (identity
+    without one): a timed region ends when its slowest rank does."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
