@@ -13,11 +13,16 @@
 // then LayerNorm on acc2 and a bf16 store of the tile of X~(i).  The hidden
 // activations never leave the SM, and never touch shared memory: the gate
 // warps write H as packed bf16 back into the TMEM columns of u they have just
-// read, and GEMM2 takes its A operand from there.  Shared-memory bandwidth
-// (operand reads plus TMA writes of the streamed weights) is what bounds this
-// kernel, so keeping H out of it leaves room for deeper weight pipelines.  u * SiLU(g) = u * g' * (1 + tanh(g')) with
-// g' = g/2, so W_g is stored pre-halved (exact in bf16) and each gate value
-// costs one MUFU tanh.
+// read, and GEMM2 takes its A operand from there.  u * SiLU(g) =
+// u * g' * (1 + tanh(g')) with g' = g/2, so W_g is stored pre-halved (exact in
+// bf16) and each gate value costs one MUFU tanh.
+//
+// What paces the kernel is the one thread that issues the MMAs: the tensor
+// pipe queues little work ahead, a 128 x 128 x 16 MMA lasts 64 cycles, and a
+// wait on an mbarrier that has already completed costs about as much.  So the
+// weights of a chunk travel as one pipeline stage (W1 and W2 of the chunk
+// together for d <= 128; for d = 256 three stages of 32 KB), and each chunk
+// costs the issuer two waits (its stage, the gate) and no more.
 //
 // Warp roles (448 threads): warp 0 issues TMA loads, warp 1 issues the MMAs
 // (one thread) and owns the TMEM allocation, warps 2-9 run the gate and warps
@@ -52,24 +57,33 @@ struct EncParams {
   int* status;
 };
 
-template <int D, int XB, int AB2, int S1, int S2>
+// Shared-memory pipeline of one configuration.  A chunk's weights are KB
+// blocks of W1 ([128 rows x 64] bf16, 16 KB each) and one block of W2
+// ([d rows x 64]).  SPC stages per chunk: 1 (W1 and W2 together) for d <= 128,
+// 3 for d = 256 (W1 blocks 0-1, W1 blocks 2-3, W2).
+template <int D, int XB, int AB2, int S>
 struct EncCfg {
   static constexpr int KB = D / 64;                       // 64-wide K blocks of X
   static constexpr uint32_t kBlock = 128u * 128u;         // [128 rows x 64] bf16
   static constexpr uint32_t kXBytes = KB * kBlock;
-  static constexpr uint32_t kW1Stage = kBlock;            // [128 rows x 64]
-  static constexpr uint32_t kW2Stage = D * 128u;          // [D rows x 64]
+  static constexpr uint32_t kW1Bytes = KB * kBlock;
+  static constexpr uint32_t kW2Bytes = D * 128u;          // [D rows x 64]
+  static constexpr int SPC = D == 256 ? 3 : 1;
+  static constexpr uint32_t kStage = SPC == 1 ? kW1Bytes + kW2Bytes : 2 * kBlock;
+  static_assert(SPC == 1 || kW2Bytes == kStage, "d = 256 stages are 32 KB");
   static constexpr uint32_t oX = 0;
-  static constexpr uint32_t oW1 = oX + XB * kXBytes;
-  static constexpr uint32_t oW2 = oW1 + S1 * kW1Stage;
-  static constexpr uint32_t oBar = oW2 + S2 * kW2Stage;
-  static constexpr int kBars = 2 * S1 + 2 * S2 + 2 * XB + 2 + 2 + 2 * AB2 + 1;
+  static constexpr uint32_t oW = oX + XB * kXBytes;
+  static constexpr uint32_t oBar = oW + S * kStage;
+  static constexpr int kBars = 2 * S + 2 * XB + 2 + 2 + 2 * AB2 + 1;
   static constexpr uint32_t oMisc = oBar + kBars * 8;
   static constexpr uint32_t kSmem = oMisc + 16 + 1024;    // + alignment slack
   static constexpr uint32_t kAcc1 = 0;                    // 2 x 128 columns (H aliases u)
   static constexpr uint32_t kAcc2 = 256;                  // AB2 x D columns
   static_assert(kAcc2 + AB2 * D <= 512, "TMEM overflow");
   static_assert(kSmem <= 227 * 1024, "shared memory overflow");
+  // While GEMM1 of chunk c+1 runs, W2 of chunk c is still held: the stages
+  // live at once are 2 for SPC = 1 and SPC (W2 of c, W1 of c+1) otherwise.
+  static_assert(S >= (SPC == 1 ? 2 : SPC), "too few stages to make progress");
 };
 
 constexpr int kEpiWarps = 8;                          // gate: two per TMEM lane quarter
@@ -91,32 +105,30 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, uint6
     if (globaltimer() - t0 > ns) break;
 }
 
-template <int D, int XB, int AB2, int S1, int S2>
+template <int D, int XB, int AB2, int S>
 __global__ void __launch_bounds__(kEncThreads, 1)
 encode_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW1,
                  const __grid_constant__ CUtensorMap tmW2, const EncParams p) {
-  using C = EncCfg<D, XB, AB2, S1, S2>;
+  using C = EncCfg<D, XB, AB2, S>;
+  constexpr int SPC = C::SPC;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                            ~static_cast<uintptr_t>(1023));
-  uint64_t* full1 = reinterpret_cast<uint64_t*>(sm + C::oBar);
-  uint64_t* empty1 = full1 + S1;
-  uint64_t* full2 = empty1 + S1;
-  uint64_t* empty2 = full2 + S2;
-  uint64_t* xfull = empty2 + S2;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sm + C::oBar);
+  uint64_t* empty = full + S;
+  uint64_t* xfull = empty + S;
   uint64_t* xempty = xfull + XB;
   uint64_t* a1full = xempty + XB;     // GEMM1 of a chunk done
   uint64_t* hfull = a1full + 2;       // its gate written to TMEM (and u, g read)
   uint64_t* a2full = hfull + 2;
   uint64_t* a2empty = a2full + AB2;
-  uint64_t* mdrain = a2empty + AB2;         // completion of every MMA, before TMEM is freed
+  uint64_t* mdrain = a2empty + AB2;   // completion of every MMA, before TMEM is freed
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + C::oMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + C::oMisc + 4);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
-    for (int i = 0; i < S1; ++i) { mbar_init(&full1[i], 1); mbar_init(&empty1[i], 1); }
-    for (int i = 0; i < S2; ++i) { mbar_init(&full2[i], 1); mbar_init(&empty2[i], 1); }
+    for (int i = 0; i < S; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
     for (int i = 0; i < XB; ++i) { mbar_init(&xfull[i], 1); mbar_init(&xempty[i], 1); }
     for (int i = 0; i < 2; ++i) { mbar_init(&a1full[i], 1); mbar_init(&hfull[i], kEpiWarps); }
     for (int i = 0; i < AB2; ++i) { mbar_init(&a2full[i], 1); mbar_init(&a2empty[i], kLnWarps); }
@@ -142,8 +154,9 @@ encode_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      const uint64_t stream_policy = policy_evict_first();   // X is read once
-      uint32_t r1 = 0, r2 = 0, xi = 0;
+      const uint64_t x_policy = policy_evict_first();    // X is read once
+      const uint64_t w_policy = policy_evict_last();     // weights: re-read by every SM
+      uint32_t g = 0, xi = 0;
       bool ok = true;
       for (int tile = blockIdx.x; ok && tile < p.ntiles; tile += gridDim.x) {
         const int xb = xi % XB;
@@ -151,30 +164,32 @@ encode_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
         mbar_arrive_expect_tx(&xfull[xb], C::kXBytes);
         for (int kb = 0; kb < C::KB; ++kb)
           tma_load_2d_hint(sm + C::oX + xb * C::kXBytes + kb * C::kBlock, &tmX, kb * 64,
-                           tile * 128, &xfull[xb], stream_policy);
+                           tile * 128, &xfull[xb], x_policy);
         ++xi;
         for (int layer = 0; ok && layer < p.M; ++layer) {
           for (int c = 0; ok && c < p.nchunk; ++c) {
-            for (int kb = 0; kb < C::KB; ++kb) {
-              const int s = r1 % S1;
-              if (!(ok = bwait(&empty1[s], ((r1 / S1) & 1) ^ 1, abort_flag, p.status))) break;
-              mbar_arrive_expect_tx(&full1[s], C::kW1Stage);
-              tma_load_2d(sm + C::oW1 + s * C::kW1Stage, &tmW1, kb * 64,
-                          (layer * p.nchunk + c) * 128, &full1[s]);
-              ++r1;
+            const int w1row = (layer * p.nchunk + c) * 128;
+            for (int j = 0; j < SPC; ++j, ++g) {
+              const int s = g % S;
+              if (!(ok = bwait(&empty[s], ((g / S) & 1) ^ 1, abort_flag, p.status))) break;
+              mbar_arrive_expect_tx(&full[s], C::kStage);
+              uint8_t* st = sm + C::oW + s * C::kStage;
+              if (SPC == 1) {
+                for (int kb = 0; kb < C::KB; ++kb)
+                  tma_load_2d_hint(st + kb * C::kBlock, &tmW1, kb * 64, w1row, &full[s], w_policy);
+                tma_load_2d_hint(st + C::kW1Bytes, &tmW2, c * 64, layer * D, &full[s], w_policy);
+              } else if (j < 2) {
+                tma_load_2d_hint(st, &tmW1, 2 * j * 64, w1row, &full[s], w_policy);
+                tma_load_2d_hint(st + C::kBlock, &tmW1, (2 * j + 1) * 64, w1row, &full[s], w_policy);
+              } else {
+                tma_load_2d_hint(st, &tmW2, c * 64, layer * D, &full[s], w_policy);
+              }
             }
-            if (!ok) break;
-            const int s = r2 % S2;
-            if (!(ok = bwait(&empty2[s], ((r2 / S2) & 1) ^ 1, abort_flag, p.status))) break;
-            mbar_arrive_expect_tx(&full2[s], C::kW2Stage);
-            tma_load_2d(sm + C::oW2 + s * C::kW2Stage, &tmW2, c * 64, layer * D, &full2[s]);
-            ++r2;
           }
         }
       }
       if (!ok) {   // let the copies already issued land before the CTA exits
-        for (uint32_t c = r1 > S1 ? r1 - S1 : 0; c < r1; ++c) drain_wait(&full1[c % S1], (c / S1) & 1, 100000000ull);
-        for (uint32_t c = r2 > S2 ? r2 - S2 : 0; c < r2; ++c) drain_wait(&full2[c % S2], (c / S2) & 1, 100000000ull);
+        for (uint32_t c = g > S ? g - S : 0; c < g; ++c) drain_wait(&full[c % S], (c / S) & 1, 100000000ull);
         for (uint32_t c = xi > XB ? xi - XB : 0; c < xi; ++c) drain_wait(&xfull[c % XB], (c / XB) & 1, 100000000ull);
       }
     }
@@ -183,7 +198,7 @@ encode_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
     if (lane == 0) {
       constexpr uint32_t idesc1 = idesc_bf16(128, 128);
       constexpr uint32_t idesc2 = idesc_bf16(128, D);
-      uint32_t r1 = 0, r2 = 0, xc = 0, cc = 0, hc = 0, uc = 0;
+      uint32_t g = 0, xc = 0, cc = 0, hc = 0, uc = 0;
       bool ok = true;
       for (int tile = blockIdx.x; ok && tile < p.ntiles; tile += gridDim.x, ++xc) {
         const int xb = xc % XB;
@@ -194,6 +209,7 @@ encode_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
           const int b2 = uc % AB2;
           const uint32_t acc2 = tmem + C::kAcc2 + b2 * D;
           for (int c = 0; ok && c <= p.nchunk; ++c) {
+            // g = first stage of chunk c; chunk c-1 started at g - SPC
             if (c < p.nchunk) {
               // GEMM1 of chunk c into acc1[cc & 1].  That buffer last held chunk
               // c-2: its gate was waited for (hfull) before GEMM2 of c-2 was
@@ -201,17 +217,23 @@ encode_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
               // c-2 has read its H before this GEMM1 overwrites it.
               const int b = cc & 1;
               const uint32_t acc1 = tmem + C::kAcc1 + b * 128;
-              for (int kb = 0; kb < C::KB; ++kb) {
-                const int s = r1 % S1;
-                if (!(ok = bwait(&full1[s], (r1 / S1) & 1, abort_flag, p.status))) break;
+              for (int j = 0; j < (SPC == 1 ? 1 : 2); ++j) {
+                const uint32_t gs = g + j;
+                const int s = gs % S;
+                if (!(ok = bwait(&full[s], (gs / S) & 1, abort_flag, p.status))) break;
                 tc_fence_after();
-                const uint32_t waddr = sbase + C::oW1 + s * C::kW1Stage;
+                const uint32_t waddr = sbase + C::oW + s * C::kStage;
+                constexpr int kbn = SPC == 1 ? C::KB : 2;
 #pragma unroll
-                for (int k4 = 0; k4 < 4; ++k4)
-                  mma_bf16_ss(acc1, sdesc_sw128(xaddr + kb * C::kBlock + k4 * 32, 16, 1024),
-                              sdesc_sw128(waddr + k4 * 32, 16, 1024), idesc1, (kb | k4) != 0);
-                mma_commit(&empty1[s]);
-                ++r1;
+                for (int kk = 0; kk < kbn; ++kk) {
+                  const int kb = j * 2 + kk;
+#pragma unroll
+                  for (int k4 = 0; k4 < 4; ++k4)
+                    mma_bf16_ss(acc1, sdesc_sw128(xaddr + kb * C::kBlock + k4 * 32, 16, 1024),
+                                sdesc_sw128(waddr + kk * C::kBlock + k4 * 32, 16, 1024), idesc1,
+                                (kb | k4) != 0);
+                }
+                if (SPC != 1) mma_commit(&empty[s]);   // these W1 blocks are done with
               }
               if (!ok) break;
               mma_commit(&a1full[b]);
@@ -227,22 +249,29 @@ encode_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
                 if (!(ok = bwait(&a2empty[b2], ((uc / AB2) & 1) ^ 1, abort_flag, p.status))) break;
                 tc_fence_after();
               }
-              const int s = r2 % S2;
-              if (!(ok = bwait(&full2[s], (r2 / S2) & 1, abort_flag, p.status))) break;
-              tc_fence_after();
+              uint32_t w2addr;
+              int s;
+              if (SPC == 1) {   // W2 rides in chunk c-1's stage, waited for at its GEMM1
+                s = (g - 1) % S;
+                w2addr = sbase + C::oW + s * C::kStage + C::kW1Bytes;
+              } else {
+                const uint32_t gs = g - SPC + 2;
+                s = gs % S;
+                if (!(ok = bwait(&full[s], (gs / S) & 1, abort_flag, p.status))) break;
+                tc_fence_after();
+                w2addr = sbase + C::oW + s * C::kStage;
+              }
               // H of the chunk: hidden columns 0..31 in TMEM columns 0..15 of
               // acc1[hb], columns 32..63 in 32..47 (each gate warp's own u columns)
               const uint32_t haddr = tmem + C::kAcc1 + hb * 128;
-              const uint32_t waddr = sbase + C::oW2 + s * C::kW2Stage;
 #pragma unroll
               for (int k4 = 0; k4 < 4; ++k4)
                 mma_bf16_ts(acc2, haddr + (k4 >> 1) * 32 + (k4 & 1) * 8,
-                            sdesc_sw128(waddr + k4 * 32, 16, 1024), idesc2,
-                            ((c - 1) | k4) != 0);
-              mma_commit(&empty2[s]);
-              ++r2;
+                            sdesc_sw128(w2addr + k4 * 32, 16, 1024), idesc2, ((c - 1) | k4) != 0);
+              mma_commit(&empty[s]);
               ++hc;
             }
+            if (c < p.nchunk) g += SPC;
           }
           if (!ok) break;
           mma_commit(&a2full[b2]);
@@ -370,6 +399,7 @@ encode_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
   }
 }
 
+
 // ------------------------------------------------------------------ host side
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
@@ -386,10 +416,10 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-template <int D, int XB, int AB2, int S1, int S2>
+template <int D, int XB, int AB2, int S>
 int launch_cfg(stca_handle* H, const CUtensorMap& tmX, const EncParams& p, cudaStream_t s) {
-  using C = EncCfg<D, XB, AB2, S1, S2>;
-  auto k = encode_tc_kernel<D, XB, AB2, S1, S2>;
+  using C = EncCfg<D, XB, AB2, S>;
+  auto k = encode_tc_kernel<D, XB, AB2, S>;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
   if (e != cudaSuccess) return set_error(STCA_ECUDA, std::string("encode_tc smem: ") + cudaGetErrorString(e));
   const int grid = std::min(p.ntiles, H->num_sms);
@@ -474,9 +504,9 @@ int launch_encode_tc(stca_handle* H, const void* X, int64_t N, cudaStream_t s) {
   }
   p.status = H->status_d;
   switch (H->d) {
-    case 64: return launch_cfg<64, 2, 2, 8, 6>(H, tmX, p, s);
-    case 128: return launch_cfg<128, 2, 2, 6, 4>(H, tmX, p, s);
-    case 256: return launch_cfg<256, 1, 1, 6, 2>(H, tmX, p, s);
+    case 64: return launch_cfg<64, 2, 2, 8>(H, tmX, p, s);      // 24 KB stages
+    case 128: return launch_cfg<128, 2, 2, 3>(H, tmX, p, s);    // 48 KB stages
+    case 256: return launch_cfg<256, 1, 1, 5>(H, tmX, p, s);    // 32 KB stages
     default: return set_error(STCA_EINVAL, "tensor-core encoder needs d in {64, 128, 256}");
   }
 }
