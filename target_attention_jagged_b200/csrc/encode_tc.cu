@@ -17,20 +17,24 @@
 // u * g' * (1 + tanh(g')) with g' = g/2, so W_g is stored pre-halved (exact in
 // bf16) and each gate value costs one MUFU tanh.
 //
-// What paces the kernel is the one thread that issues the MMAs: the tensor
-// pipe queues little work ahead, a 128 x 128 x 16 MMA lasts 64 cycles, and a
-// wait on an mbarrier that has already completed costs about as much.  So the
+// What paces the kernel is the issue of the MMAs: the tensor pipe queues
+// little work ahead, a 128 x 128 x 16 MMA lasts 64 cycles, and each wait on an
+// mbarrier or commit costs about as much to the thread that issues it.  So the
 // weights of a chunk travel as one pipeline stage (W1 and W2 of the chunk
-// together for d <= 128; for d = 256 three stages of 32 KB), and each chunk
-// costs the issuer two waits (its stage, the gate) and no more.
+// together for d <= 128; for d = 256 three stages of 32 KB), and two threads
+// in different warps issue the MMAs -- one GEMM1, the other GEMM2 -- so that
+// the waits of each overlap the MMAs of the other.  The GEMM1 issuer does not
+// overwrite an acc1 buffer before the GEMM2 issuer reports (g2done) that the
+// GEMM2 reading its H has completed.
 //
-// Warp roles (448 threads): warp 0 issues TMA loads, warp 1 issues the MMAs
-// (one thread) and owns the TMEM allocation, warps 2-9 run the gate and warps
-// 10-13 the LayerNorm.  A warp may only touch its own 32-lane quarter of TMEM
-// (one row per thread), so two gate warps share each quarter and split its
-// columns in halves.  acc1 is double-buffered so GEMM1 of chunk c+1 overlaps
-// the gate of chunk c; acc2 is double-buffered (d <= 128) so the LayerNorm of
-// one (tile, layer) overlaps the GEMMs of the next.
+// Warp roles (480 threads): warp 0 issues TMA loads, warp 1 issues GEMM1 (one
+// thread) and owns the TMEM allocation, warps 2-9 run the gate, warps 10-13
+// the LayerNorm and warp 14 issues GEMM2 (one thread).  A warp may only touch
+// its own 32-lane quarter of TMEM (one row per thread), so two gate warps
+// share each quarter and split its columns in halves.  acc1 is
+// double-buffered so GEMM1 of chunk c+1 overlaps the gate of chunk c; acc2 is
+// double-buffered (d <= 128) so the LayerNorm of one (tile, layer) overlaps
+// the GEMMs of the next.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -74,7 +78,7 @@ struct EncCfg {
   static constexpr uint32_t oX = 0;
   static constexpr uint32_t oW = oX + XB * kXBytes;
   static constexpr uint32_t oBar = oW + S * kStage;
-  static constexpr int kBars = 2 * S + 2 * XB + 2 + 2 + 2 * AB2 + 1;
+  static constexpr int kBars = 2 * S + 2 * XB + 2 + 2 + 2 + 2 * AB2 + 1;
   static constexpr uint32_t oMisc = oBar + kBars * 8;
   static constexpr uint32_t kSmem = oMisc + 16 + 1024;    // + alignment slack
   static constexpr uint32_t kAcc1 = 0;                    // 2 x 128 columns (H aliases u)
@@ -88,7 +92,8 @@ struct EncCfg {
 
 constexpr int kEpiWarps = 8;                          // gate: two per TMEM lane quarter
 constexpr int kLnWarps = 4;                           // LayerNorm: one per lane quarter
-constexpr int kEncThreads = 64 + 32 * (kEpiWarps + kLnWarps);
+constexpr int kIssuer2Warp = 2 + kEpiWarps + kLnWarps;  // issues GEMM2
+constexpr int kEncThreads = 32 * (kIssuer2Warp + 1);
 
 __device__ __forceinline__ bool bwait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
                                       int* status) {
@@ -122,17 +127,20 @@ encode_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
   uint64_t* hfull = a1full + 2;       // its gate written to TMEM (and u, g read)
   uint64_t* a2full = hfull + 2;
   uint64_t* a2empty = a2full + AB2;
-  uint64_t* mdrain = a2empty + AB2;   // completion of every MMA, before TMEM is freed
+  uint64_t* g2done = a2empty + AB2;  // GEMM2 of a chunk done: its H may be overwritten
+  uint64_t* mdrain = g2done + 2;     // completion of every MMA, before TMEM is freed
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + C::oMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + C::oMisc + 4);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
-    for (int i = 0; i < S; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
+    // a d <= 128 stage is released by both issuers (W1 and W2 ride together)
+    for (int i = 0; i < S; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], SPC == 1 ? 2 : 1); }
     for (int i = 0; i < XB; ++i) { mbar_init(&xfull[i], 1); mbar_init(&xempty[i], 1); }
     for (int i = 0; i < 2; ++i) { mbar_init(&a1full[i], 1); mbar_init(&hfull[i], kEpiWarps); }
     for (int i = 0; i < AB2; ++i) { mbar_init(&a2full[i], 1); mbar_init(&a2empty[i], kLnWarps); }
-    mbar_init(mdrain, 1);
+    for (int i = 0; i < 2; ++i) mbar_init(&g2done[i], 1);
+    mbar_init(mdrain, 2);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -194,90 +202,85 @@ encode_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
       }
     }
   } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
+    // ------------------------------------------------------------ GEMM1 issuer
     if (lane == 0) {
       constexpr uint32_t idesc1 = idesc_bf16(128, 128);
-      constexpr uint32_t idesc2 = idesc_bf16(128, D);
-      uint32_t g = 0, xc = 0, cc = 0, hc = 0, uc = 0;
+      uint32_t g = 0, xc = 0, cc = 0;
       bool ok = true;
       for (int tile = blockIdx.x; ok && tile < p.ntiles; tile += gridDim.x, ++xc) {
         const int xb = xc % XB;
         if (!(ok = bwait(&xfull[xb], (xc / XB) & 1, abort_flag, p.status))) break;
-        tc_fence_after();
         const uint32_t xaddr = sbase + C::oX + xb * C::kXBytes;
+        for (int layer = 0; ok && layer < p.M; ++layer) {
+          for (int c = 0; ok && c < p.nchunk; ++c, ++cc, g += SPC) {
+            // acc1[cc & 1] last held chunk cc-2, whose H GEMM2 reads from there
+            const int b = cc & 1;
+            if (cc >= 2 && !(ok = bwait(&g2done[b], ((cc >> 1) & 1) ^ 1, abort_flag, p.status))) break;
+            const uint32_t acc1 = tmem + C::kAcc1 + b * 128;
+            for (int j = 0; j < (SPC == 1 ? 1 : 2); ++j) {
+              const uint32_t gs = g + j;
+              const int s = gs % S;
+              if (!(ok = bwait(&full[s], (gs / S) & 1, abort_flag, p.status))) break;
+              tc_fence_after();
+              const uint32_t waddr = sbase + C::oW + s * C::kStage;
+              constexpr int kbn = SPC == 1 ? C::KB : 2;
+#pragma unroll
+              for (int kk = 0; kk < kbn; ++kk) {
+                const int kb = j * 2 + kk;
+#pragma unroll
+                for (int k4 = 0; k4 < 4; ++k4)
+                  mma_bf16_ss(acc1, sdesc_sw128(xaddr + kb * C::kBlock + k4 * 32, 16, 1024),
+                              sdesc_sw128(waddr + kk * C::kBlock + k4 * 32, 16, 1024), idesc1,
+                              (kb | k4) != 0);
+              }
+              mma_commit(&empty[s]);   // GEMM1's share of the stage is done with
+            }
+            if (!ok) break;
+            mma_commit(&a1full[b]);
+            if (layer == p.M - 1 && c == p.nchunk - 1) mma_commit(&xempty[xb]);
+          }
+        }
+      }
+      mma_commit(mdrain);
+      drain_wait(mdrain, 0, 500000000ull);
+    }
+  } else if (warp == kIssuer2Warp) {
+    // ------------------------------------------------------------ GEMM2 issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc2 = idesc_bf16(128, D);
+      uint32_t g = 0, hc = 0, uc = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < p.ntiles; tile += gridDim.x) {
         for (int layer = 0; ok && layer < p.M; ++layer, ++uc) {
           const int b2 = uc % AB2;
           const uint32_t acc2 = tmem + C::kAcc2 + b2 * D;
-          for (int c = 0; ok && c <= p.nchunk; ++c) {
-            // g = first stage of chunk c; chunk c-1 started at g - SPC
-            if (c < p.nchunk) {
-              // GEMM1 of chunk c into acc1[cc & 1].  That buffer last held chunk
-              // c-2: its gate was waited for (hfull) before GEMM2 of c-2 was
-              // issued, and MMAs of one thread run in issue order, so GEMM2 of
-              // c-2 has read its H before this GEMM1 overwrites it.
-              const int b = cc & 1;
-              const uint32_t acc1 = tmem + C::kAcc1 + b * 128;
-              for (int j = 0; j < (SPC == 1 ? 1 : 2); ++j) {
-                const uint32_t gs = g + j;
-                const int s = gs % S;
-                if (!(ok = bwait(&full[s], (gs / S) & 1, abort_flag, p.status))) break;
-                tc_fence_after();
-                const uint32_t waddr = sbase + C::oW + s * C::kStage;
-                constexpr int kbn = SPC == 1 ? C::KB : 2;
+          for (int c = 0; ok && c < p.nchunk; ++c, ++hc, g += SPC) {
+            // acc2 += H[hc & 1] * W_d chunk, once the gate has written H
+            const int hb = hc & 1;
+            if (!(ok = bwait(&hfull[hb], (hc >> 1) & 1, abort_flag, p.status))) break;
+            if (c == 0 && !(ok = bwait(&a2empty[b2], ((uc / AB2) & 1) ^ 1, abort_flag, p.status)))
+              break;
+            // W2 of the chunk: in the chunk's stage for SPC = 1 (long complete:
+            // GEMM1 of the chunk, before the gate, waited for it), else in its
+            // third stage
+            const uint32_t gs = g + (SPC == 1 ? 0 : 2);
+            const int s = gs % S;
+            if (!(ok = bwait(&full[s], (gs / S) & 1, abort_flag, p.status))) break;
+            tc_fence_after();
+            const uint32_t w2addr = sbase + C::oW + s * C::kStage + (SPC == 1 ? C::kW1Bytes : 0);
+            // H of the chunk: hidden columns 0..31 in TMEM columns 0..15 of
+            // acc1[hb], columns 32..63 in 32..47 (each gate warp's own u columns)
+            const uint32_t haddr = tmem + C::kAcc1 + hb * 128;
 #pragma unroll
-                for (int kk = 0; kk < kbn; ++kk) {
-                  const int kb = j * 2 + kk;
-#pragma unroll
-                  for (int k4 = 0; k4 < 4; ++k4)
-                    mma_bf16_ss(acc1, sdesc_sw128(xaddr + kb * C::kBlock + k4 * 32, 16, 1024),
-                                sdesc_sw128(waddr + kk * C::kBlock + k4 * 32, 16, 1024), idesc1,
-                                (kb | k4) != 0);
-                }
-                if (SPC != 1) mma_commit(&empty[s]);   // these W1 blocks are done with
-              }
-              if (!ok) break;
-              mma_commit(&a1full[b]);
-              if (layer == p.M - 1 && c == p.nchunk - 1) mma_commit(&xempty[xb]);
-              ++cc;
-            }
-            if (c >= 1) {
-              // GEMM2 of chunk c-1: acc2 += H[hc & 1] * W_d chunk
-              const int hb = hc & 1;
-              if (!(ok = bwait(&hfull[hb], (hc >> 1) & 1, abort_flag, p.status))) break;
-              tc_fence_after();
-              if (c == 1) {
-                if (!(ok = bwait(&a2empty[b2], ((uc / AB2) & 1) ^ 1, abort_flag, p.status))) break;
-                tc_fence_after();
-              }
-              uint32_t w2addr;
-              int s;
-              if (SPC == 1) {   // W2 rides in chunk c-1's stage, waited for at its GEMM1
-                s = (g - 1) % S;
-                w2addr = sbase + C::oW + s * C::kStage + C::kW1Bytes;
-              } else {
-                const uint32_t gs = g - SPC + 2;
-                s = gs % S;
-                if (!(ok = bwait(&full[s], (gs / S) & 1, abort_flag, p.status))) break;
-                tc_fence_after();
-                w2addr = sbase + C::oW + s * C::kStage;
-              }
-              // H of the chunk: hidden columns 0..31 in TMEM columns 0..15 of
-              // acc1[hb], columns 32..63 in 32..47 (each gate warp's own u columns)
-              const uint32_t haddr = tmem + C::kAcc1 + hb * 128;
-#pragma unroll
-              for (int k4 = 0; k4 < 4; ++k4)
-                mma_bf16_ts(acc2, haddr + (k4 >> 1) * 32 + (k4 & 1) * 8,
-                            sdesc_sw128(w2addr + k4 * 32, 16, 1024), idesc2, ((c - 1) | k4) != 0);
-              mma_commit(&empty[s]);
-              ++hc;
-            }
-            if (c < p.nchunk) g += SPC;
+            for (int k4 = 0; k4 < 4; ++k4)
+              mma_bf16_ts(acc2, haddr + (k4 >> 1) * 32 + (k4 & 1) * 8,
+                          sdesc_sw128(w2addr + k4 * 32, 16, 1024), idesc2, (c | k4) != 0);
+            mma_commit(&empty[s]);
+            mma_commit(&g2done[hb]);
+            if (c == p.nchunk - 1) mma_commit(&a2full[b2]);
           }
-          if (!ok) break;
-          mma_commit(&a2full[b2]);
         }
       }
-      // every MMA issued so far must finish before TMEM is released
       mma_commit(mdrain);
       drain_wait(mdrain, 0, 500000000ull);
     }
