@@ -80,3 +80,21 @@ def test_tensor_core_path_rejected_when_unsupported(gpu):
         st.set_option(S.STCA_OPT_ENCODE_PATH, ENCODE_TC)
         with pytest.raises(S.StcaError):
             st.encode(to_device(wl, wl.X, gpu), wl.offsets)
+
+
+@pytest.mark.parametrize("d,M,r", [(64, 2, 2), (128, 3, 4), (256, 3, 2)])
+def test_encoder_many_tiles_per_cta(gpu, d, M, r):
+    """Several 128-row tiles per persistent CTA (every weight ring wraps many
+    times, the X buffers are reused): sampled rows against the oracle.  The
+    encoder is row-wise, so the oracle runs on the sampled rows alone."""
+    n = 148 * 128 * 3 + 77
+    wl = make_workload(lengths=[n - 5000, 5000], targets=[1, 1], d=d, h=4, M=M, r=r,
+                       dtype="bf16", seed=11 + d, random_ln=True)
+    got = encoded_layers(wl, gpu, ENCODE_TC)
+    rng = np.random.default_rng(d)
+    rows = np.unique(np.concatenate([rng.integers(0, n, 400), np.arange(n - 80, n),
+                                     np.arange(0, 40)]))
+    for i in range(M):
+        want = O.encode_history(wl.X[rows], wl.weights, i)
+        err = rowwise_err(got[i][rows], want)
+        assert err <= TOL["bf16"], f"d={d} layer {i}: row-wise error {err:.3e}"
