@@ -220,6 +220,8 @@ enum {
   STCA_OPT_ENCODE_PATH = 2,   /* 0 auto, 1 CUDA cores, 2 tensor cores (bf16 only) */
   STCA_OPT_SPLIT_KEYS = 3,    /* keys per attention work item, 0 = auto; multiple of 128 */
   STCA_OPT_TIMING = 4,        /* 1: record CUDA events around every kernel launch */
+  STCA_OPT_STEP_PATH = 5,     /* per-target step: 0 auto, 1 CUDA cores, 2 tensor cores (bf16,
+                                 d in {128, 256}, r d <= 512, with the tensor-core attention) */
   STCA_OPT_LAUNCHES = 100     /* read-only: kernels launched since the last encode */
 };
 int stca_set_option(stca_handle* handle, int option, int64_t value);

@@ -11,6 +11,7 @@ from .stca import (  # noqa: F401
     STCA_OPT_ENCODE_PATH,
     STCA_OPT_LAUNCHES,
     STCA_OPT_SPLIT_KEYS,
+    STCA_OPT_STEP_PATH,
     STCA_OPT_TIMING,
     Stca,
     StcaError,

@@ -356,6 +356,12 @@ extern "C" int stca_init(const stca_weights* w, int d, int h, int r, int M, int 
       stca_destroy(H);
       return rc2;
     }
+    if (step_tc_supported(H)) {
+      if (int rc2 = step_tc_setup(H, sw)) {
+        stca_destroy(H);
+        return rc2;
+      }
+    }
   }
   if (dtype == STCA_BF16 && encode_tc_supported(d, rd)) {
     std::vector<const float*> Wu(M), Wg(M), Wd(M);
@@ -696,9 +702,19 @@ extern "C" int stca_forward(stca_handle* H, const void* targets, const int64_t* 
   plan.mtile_rows = path == 2 ? 128 : (1 << 30);
   plan.log2_partials = path == 2 ? 1 : 0;
   const size_t layer_bytes = static_cast<size_t>(H->N) * d * H->elem;
+  // per-target step: tensor cores when the attention is (their query units)
+  if (H->opt_step_path == 2 && !(path == 2 && H->step_tc_ready))
+    return set_error(STCA_EINVAL, "tensor-core step needs the tensor-core attention, bf16, "
+                                  "d in {128, 256} and r d <= 512");
+  const bool step_tc = path == 2 && H->step_tc_ready && H->opt_step_path != 1;
+  auto step = [&](int layer, const float* cm) {
+    if (step_tc) return launch_step_tc(H, layer, targets, T, cm, Z, H->Ubf, s);
+    launch_target_step(H, layer, targets, T, plan, cm, Z, s);
+    return static_cast<int>(STCA_OK);
+  };
   {
     TimedLaunch tl(H, STCA_K_STEP, s);
-    launch_target_step(H, -1, targets, T, plan, nullptr, Z, s);
+    if (int rc = step(-1, nullptr)) return rc;
   }
   H->launches++;
   if (int rc = check_launch("query init")) return rc;
@@ -719,8 +735,9 @@ extern "C" int stca_forward(stca_handle* H, const void* targets, const int64_t* 
     {
       TimedLaunch tl(H, STCA_K_STEP, s);
       launch_combine(H, plan, H->part, H->last_G, T, H->cbuf, s);
-      launch_target_step(H, i, targets, T, plan, H->cbuf, Z, s);
+      rc = step(i, H->cbuf);
     }
+    if (rc) return rc;
     H->launches += 2;
     if (int rc2 = check_launch("target step")) return rc2;
   }
@@ -837,6 +854,10 @@ extern "C" int stca_set_option(stca_handle* H, int option, int64_t value) {
       if (value < 0 || value > 2) return set_error(STCA_EINVAL, "encode path must be 0, 1 or 2");
       H->opt_encode_path = static_cast<int>(value);
       return ok();
+    case STCA_OPT_STEP_PATH:
+      if (value < 0 || value > 2) return set_error(STCA_EINVAL, "step path must be 0, 1 or 2");
+      H->opt_step_path = static_cast<int>(value);
+      return ok();
     case STCA_OPT_TIMING:
       if (value != 0 && value != 1) return set_error(STCA_EINVAL, "timing must be 0 or 1");
       H->timing = value != 0;
@@ -856,6 +877,7 @@ extern "C" int stca_get_option(stca_handle* H, int option, int64_t* value) {
   switch (option) {
     case STCA_OPT_ATTN_PATH: *value = H->opt_attn_path; return ok();
     case STCA_OPT_ENCODE_PATH: *value = H->opt_encode_path; return ok();
+    case STCA_OPT_STEP_PATH: *value = H->opt_step_path; return ok();
     case STCA_OPT_SPLIT_KEYS: *value = H->opt_split_keys; return ok();
     case STCA_OPT_TIMING: *value = H->timing ? 1 : 0; return ok();
     case STCA_OPT_LAUNCHES: *value = H->launches; return ok();

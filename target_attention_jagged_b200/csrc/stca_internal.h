@@ -68,6 +68,14 @@ struct StepHostW {
   const float *Wq, *Wk, *Wv, *Wo, *Wc, *qWu, *qWg, *qWd;
 };
 
+// One product of the tensor-core per-target step: MB blocks of 128 output
+// features times KC chunks of 64 inputs, stored as A tiles tile0 ..
+// tile0 + MB * KC - 1 (block-major) of the handle's step tile stream.
+struct TcGemm {
+  int mb = 0, kc = 0;
+  int64_t tile0 = -1;
+};
+
 }  // namespace stca
 
 struct stca_handle {
@@ -88,10 +96,13 @@ struct stca_handle {
   CUtensorMap tmXt[16];                 // X~(i) of the last encode (tensor-core attention)
   CUtensorMap tmU;                      // bf16 query rows of the current forward
   bool tc_encode_ready = false;
+  uint16_t* wstep_tc = nullptr;         // A-tile stream of the tensor-core per-target step
+  std::vector<stca::TcGemm> tcO, tcC, tcUG, tcD, tcQ;   // per layer
+  bool step_tc_ready = false;
   int num_sms = 148;
 
   // options
-  int opt_attn_path = 0, opt_encode_path = 0;
+  int opt_attn_path = 0, opt_encode_path = 0, opt_step_path = 0;
   int64_t opt_split_keys = 0;
   int64_t launches = 0;
   bool timing = false;
@@ -158,6 +169,12 @@ void launch_target_step(const stca_handle* H, int layer, const void* targets, in
 size_t target_step_smem(const stca_handle* H);
 int step_weights_setup(stca_handle* H, const std::vector<StepHostW>& layers);
 size_t attn_simt_smem(const stca_handle* H);
+
+// Tensor-core per-target step (step_tc.cu)
+bool step_tc_supported(const stca_handle* H);
+int step_tc_setup(stca_handle* H, const std::vector<StepHostW>& layers);
+int launch_step_tc(const stca_handle* H, int layer, const void* targets, int64_t T,
+                   const float* cmerged, float* Z, uint16_t* Ubf, cudaStream_t s);
 
 // Host-side attention work plan (stca_api.cu).
 struct PlanHost {

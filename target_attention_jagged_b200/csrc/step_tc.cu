@@ -1,0 +1,623 @@
+// Tensor-core per-target step of the STCA forward, between two attention
+// layers ("Make It Long, Keep It Fast" digest §2.1):
+//   output          o = [c_1 W_V^1 || ... || c_h W_V^h] W_O; Z[t, i, :] = o   (Eqs. (6), (8), (13))
+//   query fusion    q = SwiGLUFFN_{i+1}([o(1) || ... || o(i+1) || x_t] W_C)  (Eq. (7))
+//   u projection    u_j = (q W_Q^j) W_K^j^T, scaled for the next attention     (Eq. (13))
+// and, before the first layer, q(1) = LN(SwiGLUFFN_1(x_t)) (Eq. (3)) and its u.
+//
+// A CTA takes 16 targets.  The dense products run on the tensor cores in
+// transposed form, Y^T[features x 16] = W^T[features x K] X^T[K x 16]: one
+// tcgen05.mma is a 128-feature block x 16 targets x 16 inputs, so a handful of
+// targets still fills the MMA's M side (features) and the 16 targets are its N.
+// The weights are laid out once, at set-up, as a stream of ready-made A tiles
+// ([128 features x 64 inputs] bf16, 128-byte swizzle, 16 KB) in the order the
+// kernel consumes them, and reach shared memory by plain bulk copies through a
+// ring.  The activations X^T are written by the worker warps, as bf16, straight
+// into the B-operand layout ([16 targets x 64 inputs] tiles, 2 KB); outputs
+// come back from TMEM one feature per lane, 16 targets per lane.  The
+// per-head products c_j W_V^j and P_j W_K^j^T are too narrow for an MMA (d_h
+// columns) and stay on the CUDA cores.
+//
+// Warp roles (320 threads): warp 0 streams the weight tiles, warp 1 owns TMEM
+// and issues the MMAs (one thread), warps 2-9 are workers (prologue,
+// epilogues, the CUDA-core products).  Worker warp w reads TMEM lane quarter
+// w % 4 and target columns 8 ((w - 2) / 4) .. +7.
+#include <cuda_bf16.h>
+#include <math.h>
+
+#include <algorithm>
+#include <cstring>
+#include <vector>
+
+#include "stca_internal.h"
+#include "tc_common.cuh"
+
+namespace stca {
+namespace {
+
+using namespace tc;
+
+constexpr int kTgt = 16;                  // targets per CTA (the MMA's N)
+constexpr int kWorkers = 8;               // worker warps
+constexpr int kStepThreads = 32 * (2 + kWorkers);
+constexpr uint32_t kATile = 128u * 128u;  // A tile: 128 rows x 64 bf16
+constexpr uint32_t kBTile = kTgt * 128u;  // B tile: 16 rows x 64 bf16
+constexpr int kMaxRing = 8;               // A tiles in flight, at most
+
+// Byte offset of element (row r, column c) of a K-major tile whose rows hold
+// 64 bf16 (128 B) with the 128-byte swizzle: 8-row atoms of 1024 B, the
+// 16-byte chunk j of row r stored at chunk j ^ (r % 8).
+__host__ __device__ inline uint32_t sw128_off(int r, int c) {
+  return static_cast<uint32_t>((r >> 3) * 1024 + (r & 7) * 128 + ((((c >> 3) ^ r) & 7) << 4) +
+                               (c & 7) * 2);
+}
+
+}  // namespace
+
+// ------------------------------------------------------------------ set-up
+// A tiles of Y^T = W^T X^T for a row-major W [K x N] (K inputs, N outputs):
+// tile (m, kc) holds output features r in [0, 128) of block m and inputs k in
+// [64 kc, 64 kc + 64).  Block m is read from columns col0 .. col0 + 127 of the
+// matrix src (row length ld): element (r, c) = src[(64 kc + c) ld + col0 + r].
+namespace {
+struct ColBlock {
+  const float* src;
+  int ld, col0;
+};
+
+TcGemm put_tiles(std::vector<uint16_t>& out, int K, const std::vector<ColBlock>& blocks) {
+  TcGemm g;
+  g.mb = static_cast<int>(blocks.size());
+  g.kc = K / 64;
+  g.tile0 = static_cast<int64_t>(out.size() / (kATile / 2));
+  for (const ColBlock& b : blocks)
+    for (int kc = 0; kc < g.kc; ++kc) {
+      const size_t base = out.size();
+      out.resize(base + kATile / 2, 0);
+      uint16_t* t = out.data() + base;
+      for (int r = 0; r < 128; ++r)
+        for (int c = 0; c < 64; ++c) {
+          const float f = b.src[static_cast<size_t>(kc * 64 + c) * b.ld + b.col0 + r];
+          uint32_t u;
+          memcpy(&u, &f, 4);
+          t[sw128_off(r, c) / 2] = static_cast<uint16_t>(u >> 16);   // bf16-exact values
+        }
+    }
+  return g;
+}
+
+std::vector<ColBlock> col_blocks(const float* W, int N) {
+  std::vector<ColBlock> v;
+  for (int m = 0; m < N / 128; ++m) v.push_back({W, N, 128 * m});
+  return v;
+}
+}  // namespace
+
+bool step_tc_supported(const stca_handle* H) {
+  // d: one or two 128-feature blocks; rd <= 512: the FFN's 2 rd / 128 blocks
+  // of 16 columns fit the 128 TMEM columns; M <= 8 bounds the W_C operand
+  return H->elem == 2 && (H->d == 128 || H->d == 256) && H->rd % 128 == 0 && H->rd <= 512 &&
+         H->d % H->h == 0 && H->dh % 2 == 0 && H->M <= 8;
+}
+
+// Lay out, per layer i, the A tiles of W_O, W_C (i >= 1), the query FFN
+// (W_u and W_g blocks interleaved: block 2m = u features 128m.., block 2m+1 =
+// g features of the same range, so one TMEM lane holds a matching u, g pair)
+// and W_d, and W_Q.
+int step_tc_setup(stca_handle* H, const std::vector<StepHostW>& layers) {
+  const int d = H->d, rd = H->rd, M = H->M;
+  std::vector<uint16_t> tiles;
+  H->tcO.assign(M, TcGemm());
+  H->tcC.assign(M, TcGemm());
+  H->tcUG.assign(M, TcGemm());
+  H->tcD.assign(M, TcGemm());
+  H->tcQ.assign(M, TcGemm());
+  for (int i = 0; i < M; ++i) {
+    const StepHostW& L = layers[i];
+    H->tcO[i] = put_tiles(tiles, d, col_blocks(L.Wo, d));
+    if (i > 0) H->tcC[i] = put_tiles(tiles, (i + 1) * d, col_blocks(L.Wc, d));
+    std::vector<ColBlock> ug;
+    for (int m = 0; m < rd / 128; ++m) {
+      ug.push_back({L.qWu, rd, 128 * m});
+      ug.push_back({L.qWg, rd, 128 * m});
+    }
+    H->tcUG[i] = put_tiles(tiles, d, ug);
+    H->tcD[i] = put_tiles(tiles, rd, col_blocks(L.qWd, d));
+    H->tcQ[i] = put_tiles(tiles, d, col_blocks(L.Wq, d));
+  }
+  if (cudaMalloc(&H->wstep_tc, tiles.size() * 2) != cudaSuccess) {
+    cudaGetLastError();
+    return set_error(STCA_ENOMEM, "tensor-core step weight allocation failed");
+  }
+  STCA_CUDA_TRY(cudaMemcpy(H->wstep_tc, tiles.data(), tiles.size() * 2, cudaMemcpyHostToDevice));
+  H->step_tc_ready = true;
+  return STCA_OK;
+}
+
+// ------------------------------------------------------------------ kernel
+namespace {
+
+enum : int { kO = 0, kC = 1, kUG = 2, kD = 3, kQ = 4 };
+
+struct StepTcArgs {
+  int layer, M, d, h, dh, rd;
+  int64_t T;
+  const uint16_t* targets;      // T x d
+  const float* cmerged;         // T x h x d: c_j = alpha_j X~ of the layer just attended
+  float* Z;                     // T x M x d
+  uint16_t* Ubf;                // T x h x d: scaled u rows for the next attention
+  const uint16_t* tiles;        // A-tile stream
+  const uint16_t* Wv;           // d x d (this layer), layer >= 0
+  const uint16_t* WkT;          // d_h x h d (next layer), layer < M - 1
+  const float *q_ln_g, *q_ln_b;
+  float uscale;
+  int* status;
+  int ng;                       // products in this launch
+  TcGemm g[5];
+  int kind[5];
+  int nring;                    // A-tile ring stages
+  int kch;                      // inputs per W_V staging chunk
+};
+
+// Shared memory, in bytes (1024-aligned base): the A-tile ring, then the
+// B-operand buffers of the five products, an fp32 scratch of d x 16 (the
+// query projection P^T, features by targets), a reduction scratch, then the
+// mbarriers.  bU .. the end of the scratch are not in use before the output
+// product, so the W_V prologue stages its operands there.
+struct StepLayout {
+  uint32_t ring, bO, bC, bU, bH, bQ, scr, red, bar, total;
+};
+
+__host__ __device__ inline StepLayout step_layout(int d, int rd, int M, int nring) {
+  StepLayout L;
+  L.ring = 0;
+  L.bO = L.ring + nring * kATile;
+  L.bC = L.bO + (d / 64) * kBTile;
+  L.bU = L.bC + (M * d / 64) * kBTile;
+  L.bH = L.bU + (d / 64) * kBTile;
+  L.bQ = L.bH + (rd / 64) * kBTile;
+  L.scr = L.bQ + (d / 64) * kBTile;
+  L.red = L.scr + kTgt * d * 4;
+  L.bar = L.red + 2 * 2 * 4 * 8 * 4;             // [2 stats][2 halves][4 quarters][8 targets]
+  L.total = L.bar + (2 * kMaxRing + 4) * 8 + 16;
+  return L;
+}
+
+// Worker-only barrier (the 256 worker threads; id 1).  Every worker executes
+// the same sequence of these, whatever its mbarrier waits returned.
+__device__ __forceinline__ void workers_sync() {
+  asm volatile("bar.sync 1, %0;" ::"n"(32 * kWorkers) : "memory");
+}
+
+// Write a worker thread's 8 fp32 values (targets t8 .. t8 + 7 of input feature
+// f of the next product) into the bf16 B-operand buffer `b` (tiles of 16
+// targets x 64 inputs).  Lanes f and f ^ 1 pair up into bf16x2 words: the even
+// lane stores targets t8 .. t8 + 3, the odd one t8 + 4 .. t8 + 7.
+__device__ __forceinline__ void put_b8(uint8_t* b, int f, int t8, const float (&v)[8], int lane) {
+  const bool even = (lane & 1) == 0;
+  const int f0 = f & ~1;
+  uint8_t* tile = b + (f0 >> 6) * kBTile;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const float other = __shfl_xor_sync(0xffffffffu, v[j], 1);
+    const float lo = even ? v[j] : other, hi = even ? other : v[j];
+    if ((j < 4) == even) {
+      const uint32_t w = pack_bf16x2(lo, hi);
+      *reinterpret_cast<uint32_t*>(tile + sw128_off(t8 + j, f0 & 63)) = w;
+    }
+  }
+}
+
+// Element (target t, input k) of a B buffer, bf16.
+__device__ __forceinline__ void put_b1(uint8_t* b, int t, int k, float v) {
+  *reinterpret_cast<__nv_bfloat16*>(b + (k >> 6) * kBTile + sw128_off(t, k & 63)) =
+      __float2bfloat16_rn(v);
+}
+
+__device__ __forceinline__ float bf2f(uint16_t u) { return __uint_as_float(static_cast<uint32_t>(u) << 16); }
+
+__device__ __forceinline__ bool step_wait(uint64_t* bar, uint32_t parity, int* status) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer();
+  while (!mbar_try_wait(bar, parity))
+    if (globaltimer() - t0 > kWaitTimeoutNs) {
+      atomicOr(status, kStatusStepTimeout);
+      return false;
+    }
+  return true;
+}
+
+__global__ void __launch_bounds__(kStepThreads, 1) step_tc_kernel(const StepTcArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                           ~static_cast<uintptr_t>(1023));
+  const int d = a.d, h = a.h, dh = a.dh, rd = a.rd, L = a.layer;
+  const int R = a.nring;
+  const StepLayout Y = step_layout(d, rd, a.M, R);
+  uint64_t* full = reinterpret_cast<uint64_t*>(sm + Y.bar);
+  uint64_t* empty = full + R;
+  uint64_t* bready = empty + R;   // the workers have written a product's B operand
+  uint64_t* aready = bready + 1;      // a product's MMAs are complete
+  uint64_t* mdrain = aready + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mdrain + 2);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t t0 = static_cast<int64_t>(blockIdx.x) * kTgt;
+  const int nb = a.T - t0 < kTgt ? static_cast<int>(a.T - t0) : kTgt;
+  uint8_t* bufs[5] = {sm + Y.bO, sm + Y.bC, sm + Y.bU, sm + Y.bH, sm + Y.bQ};
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < R; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
+    mbar_init(bready, kWorkers);
+    mbar_init(aready, 1);
+    mbar_init(mdrain, 1);
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 128);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ weight streamer
+    if (lane == 0) {
+      uint32_t q = 0;
+      bool ok = true;
+      for (int gi = 0; ok && gi < a.ng; ++gi) {
+        const TcGemm G = a.g[gi];
+        const int n = G.mb * G.kc;
+        for (int t = 0; ok && t < n; ++t, ++q) {
+          const int s = q % R;
+          if (!(ok = step_wait(&empty[s], ((q / R) & 1) ^ 1, a.status))) break;
+          mbar_arrive_expect_tx(&full[s], kATile);
+          const uint16_t* src = a.tiles + (G.tile0 + t) * (kATile / 2);
+          asm volatile(
+              "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                  smem_u32(sm + Y.ring + s * kATile)),
+              "l"(src), "r"(kATile), "r"(smem_u32(&full[s]))
+              : "memory");
+        }
+      }
+      // let the copies in flight land before the CTA can exit
+      for (uint32_t c = q > static_cast<uint32_t>(R) ? q - R : 0; c < q; ++c)
+        step_wait(&full[c % R], (c / R) & 1, a.status);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16(128, kTgt);
+      uint32_t q = 0;
+      bool ok = true;
+      for (int gi = 0; ok && gi < a.ng; ++gi) {
+        const TcGemm G = a.g[gi];
+        if (!(ok = step_wait(bready, gi & 1, a.status))) break;
+        tc_fence_after();
+        const uint32_t bbase = smem_u32(bufs[a.kind[gi]]);
+        for (int m = 0; ok && m < G.mb; ++m) {
+          const uint32_t acc = tmem + m * kTgt;
+          for (int kc = 0; kc < G.kc; ++kc, ++q) {
+            const int s = q % R;
+            if (!(ok = step_wait(&full[s], (q / R) & 1, a.status))) break;
+            tc_fence_after();
+            const uint32_t aaddr = smem_u32(sm + Y.ring + s * kATile);
+            const uint32_t baddr = bbase + kc * kBTile;
+#pragma unroll
+            for (int k4 = 0; k4 < 4; ++k4)
+              mma_bf16_ss(acc, sdesc_sw128(aaddr + k4 * 32, 16, 1024),
+                          sdesc_sw128(baddr + k4 * 32, 16, 1024), idesc, (kc | k4) != 0);
+            mma_commit(&empty[s]);
+          }
+        }
+        if (!ok) break;
+        mma_commit(aready);
+      }
+      mma_commit(mdrain);
+      step_wait(mdrain, 0, a.status);
+    }
+  } else {
+    // ------------------------------------------------------------ workers
+    const int wid = warp - 2;                 // 0..7
+    const int tid = threadIdx.x - 64;         // 0..255
+    const int q4 = warp & 3;                  // TMEM lane quarter
+    const int t8 = 8 * (wid >> 2);            // target columns t8 .. t8 + 7
+    const uint32_t lane_base = static_cast<uint32_t>(q4 * 32) << 16;
+    float* scr = reinterpret_cast<float*>(sm + Y.scr);
+    float* red = reinterpret_cast<float*>(sm + Y.red);
+    const int M = a.M;
+    bool ok = true;
+    // ---- prologue: the B operand of the launch's first product
+    if (L < 0) {
+      for (int e = tid; e < kTgt * d; e += 32 * kWorkers) {
+        const int t = e / d, k = e - t * d;
+        put_b1(bufs[kUG], t, k, t < nb ? bf2f(a.targets[(t0 + t) * d + k]) : 0.f);
+      }
+    } else {
+      if (L + 1 < M) {
+        // [o(1) .. o(L) | o(L+1): by the output epilogue | x_t] of Eq. (7)
+        const int wcat = (L + 2) * d;
+        for (int e = tid; e < kTgt * wcat; e += 32 * kWorkers) {
+          const int t = e / wcat, k = e - t * wcat;
+          const int blk = k / d, kk = k - blk * d;
+          if (blk == L) continue;
+          float v = 0.f;
+          if (t < nb) v = blk < L ? a.Z[((t0 + t) * M + blk) * d + kk] : bf2f(a.targets[(t0 + t) * d + kk]);
+          put_b1(bufs[kC], t, k, v);
+        }
+      }
+      // o_head = c_j W_V^j into the B operand of W_O.  Output column n belongs
+      // to head n / d_h; a thread owns blocks of 4 targets x 2 columns and
+      // accumulates them over the d inputs, which arrive in chunks of kch:
+      // cs[j][k][t] (all heads' c_j, 16 targets contiguous) and ws[k][n]
+      // (rows of W_V), staged in the buffers the later products use.
+      const int kch = a.kch;
+      float* cs = reinterpret_cast<float*>(sm + Y.bU);
+      uint16_t* ws = reinterpret_cast<uint16_t*>(sm + Y.bU + kTgt * h * kch * 4);
+      constexpr int kMaxBlk = 2;                      // 2 d / 256 blocks per thread, d <= 256
+      float acc[kMaxBlk][4][2];
+#pragma unroll
+      for (int bi = 0; bi < kMaxBlk; ++bi)
+#pragma unroll
+        for (int t = 0; t < 4; ++t) acc[bi][t][0] = acc[bi][t][1] = 0.f;
+      const int nblk = 2 * d;                         // (16 / 4) x (d / 2) blocks
+      for (int k0 = 0; k0 < d; k0 += kch) {
+        // c_j[t][k0 .. k0 + kch): one float4 of 4 inputs per (t, j, k4)
+        for (int e = tid; e < kTgt * h * (kch / 4); e += 32 * kWorkers) {
+          const int t = e % kTgt, rest = e / kTgt;
+          const int j = rest % h, k4 = rest / h;
+          float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+          if (t < nb)
+            v = *reinterpret_cast<const float4*>(a.cmerged + ((t0 + t) * h + j) * d + k0 + 4 * k4);
+          float* dst = cs + (j * kch + 4 * k4) * kTgt + t;
+          dst[0] = v.x;
+          dst[kTgt] = v.y;
+          dst[2 * kTgt] = v.z;
+          dst[3 * kTgt] = v.w;
+        }
+        // W_V rows k0 .. k0 + kch, 16 bytes at a time
+        for (int e = tid; e < kch * d / 8; e += 32 * kWorkers) {
+          const int k = e / (d / 8), c8 = e - k * (d / 8);
+          *reinterpret_cast<uint4*>(ws + k * d + 8 * c8) =
+              *reinterpret_cast<const uint4*>(a.Wv + (k0 + k) * d + 8 * c8);
+        }
+        workers_sync();
+#pragma unroll
+        for (int bi = 0; bi < kMaxBlk; ++bi) {
+          const int b = tid + bi * 32 * kWorkers;
+          if (b < nblk) {
+            const int t4 = b & 3, n = 2 * (b >> 2), j = n / dh;
+            const float* cp = cs + j * kch * kTgt + 4 * t4;
+            const uint16_t* wp = ws + n;
+            for (int k = 0; k < kch; ++k) {
+              const float4 c = *reinterpret_cast<const float4*>(cp + k * kTgt);
+              const uint32_t w2 = *reinterpret_cast<const uint32_t*>(wp + k * d);
+              const float w0 = __uint_as_float(w2 << 16), w1 = __uint_as_float(w2 & 0xFFFF0000u);
+              acc[bi][0][0] = fmaf(c.x, w0, acc[bi][0][0]); acc[bi][0][1] = fmaf(c.x, w1, acc[bi][0][1]);
+              acc[bi][1][0] = fmaf(c.y, w0, acc[bi][1][0]); acc[bi][1][1] = fmaf(c.y, w1, acc[bi][1][1]);
+              acc[bi][2][0] = fmaf(c.z, w0, acc[bi][2][0]); acc[bi][2][1] = fmaf(c.z, w1, acc[bi][2][1]);
+              acc[bi][3][0] = fmaf(c.w, w0, acc[bi][3][0]); acc[bi][3][1] = fmaf(c.w, w1, acc[bi][3][1]);
+            }
+          }
+        }
+        workers_sync();
+      }
+#pragma unroll
+      for (int bi = 0; bi < kMaxBlk; ++bi) {
+        const int b = tid + bi * 32 * kWorkers;
+        if (b < nblk) {
+          const int t4 = b & 3, n = 2 * (b >> 2);
+          uint8_t* tile = bufs[kO] + (n >> 6) * kBTile;
+#pragma unroll
+          for (int t = 0; t < 4; ++t)
+            *reinterpret_cast<uint32_t*>(tile + sw128_off(4 * t4 + t, n & 63)) =
+                pack_bf16x2(acc[bi][t][0], acc[bi][t][1]);
+        }
+      }
+    }
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(bready);
+
+    // ---- epilogues
+    for (int gi = 0; gi < a.ng; ++gi) {
+      const int kind = a.kind[gi];
+      const TcGemm G = a.g[gi];
+      if (ok) ok = step_wait(aready, gi & 1, a.status);
+      __syncwarp();
+      tc_fence_after();
+      float vals[2][8];                       // up to two blocks of 128 features (d <= 256)
+      if (kind == kUG) {
+        for (int p = 0; p < G.mb / 2; ++p) {
+          uint32_t u[8], g[8];
+          tmem_ld8(tmem + lane_base + (2 * p) * kTgt + t8, u);
+          tmem_ld8(tmem + lane_base + (2 * p + 1) * kTgt + t8, g);
+          tmem_ld_wait();
+          float hv[8];
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const float gg = __uint_as_float(g[j]);
+            hv[j] = __uint_as_float(u[j]) * gg / (1.0f + __expf(-gg));
+          }
+          put_b8(bufs[kD], 128 * p + 32 * q4 + lane, t8, hv, lane);
+        }
+      } else {
+        for (int m = 0; m < G.mb; ++m) {
+          uint32_t r[8];
+          tmem_ld8(tmem + lane_base + m * kTgt + t8, r);
+          tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 8; ++j) vals[m][j] = __uint_as_float(r[j]);
+        }
+        if (kind == kD && L < 0) {
+          // LayerNorm of Eq. (3) over the d features of each target column:
+          // features are spread over lanes, lane quarters and blocks
+          float s[8];
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            s[j] = vals[0][j] + (G.mb > 1 ? vals[1][j] : 0.f);
+            for (int o = 16; o > 0; o >>= 1) s[j] += __shfl_xor_sync(0xffffffffu, s[j], o);
+          }
+          if (lane == 0)
+            for (int j = 0; j < 8; ++j) red[((0 * 2 + (wid >> 2)) * 4 + q4) * 8 + j] = s[j];
+          workers_sync();
+          float mean[8], s2[8];
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            float tot = 0.f;
+            for (int qq = 0; qq < 4; ++qq) tot += red[((0 * 2 + (wid >> 2)) * 4 + qq) * 8 + j];
+            mean[j] = tot / d;
+            float e0 = vals[0][j] - mean[j];
+            s2[j] = e0 * e0;
+            if (G.mb > 1) { const float e1 = vals[1][j] - mean[j]; s2[j] = fmaf(e1, e1, s2[j]); }
+            for (int o = 16; o > 0; o >>= 1) s2[j] += __shfl_xor_sync(0xffffffffu, s2[j], o);
+          }
+          if (lane == 0)
+            for (int j = 0; j < 8; ++j) red[((1 * 2 + (wid >> 2)) * 4 + q4) * 8 + j] = s2[j];
+          workers_sync();
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            float tot = 0.f;
+            for (int qq = 0; qq < 4; ++qq) tot += red[((1 * 2 + (wid >> 2)) * 4 + qq) * 8 + j];
+            const float rstd = rsqrtf(tot / d + 1e-5f);
+            for (int m = 0; m < G.mb; ++m) {
+              const int f = 128 * m + 32 * q4 + lane;
+              vals[m][j] = (vals[m][j] - mean[j]) * rstd * a.q_ln_g[f] + a.q_ln_b[f];
+            }
+          }
+        }
+        for (int m = 0; m < G.mb; ++m) {
+          const int f = 128 * m + 32 * q4 + lane;
+          if (kind == kO) {
+            for (int j = 0; j < 8; ++j)
+              if (t8 + j < nb) a.Z[((t0 + t8 + j) * M + L) * d + f] = vals[m][j];
+            if (L + 1 < M) put_b8(bufs[kC], L * d + f, t8, vals[m], lane);
+          } else if (kind == kC) {
+            put_b8(bufs[kUG], f, t8, vals[m], lane);
+          } else if (kind == kD) {
+            put_b8(bufs[kQ], f, t8, vals[m], lane);
+          } else {   // kQ: P = q W_Q in fp32, as P^T[feature][target] for the W_K products
+            float4* dst = reinterpret_cast<float4*>(scr + f * kTgt + t8);
+            dst[0] = make_float4(vals[m][0], vals[m][1], vals[m][2], vals[m][3]);
+            dst[1] = make_float4(vals[m][4], vals[m][5], vals[m][6], vals[m][7]);
+          }
+        }
+      }
+      tc_fence_before();
+      if (gi + 1 < a.ng) {
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bready);
+      }
+    }
+    // ---- u_j = P_j W_K^j^T (Eq. (13)), scaled, as bf16 rows for the attention.
+    // A thread owns blocks of 16 targets x 4 outputs (head j, columns k..k+3):
+    // per c < d_h, one 8-byte load of W_K^T and the 16 targets' P[j d_h + c].
+    if (L + 1 < M) {
+      workers_sync();
+      const int hd = h * d;
+      for (int b = tid; b < hd / 4; b += 32 * kWorkers) {
+        const int jk = 4 * b, j = jk / d;
+        float acc[kTgt][4];
+#pragma unroll
+        for (int t = 0; t < kTgt; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.f;
+        for (int c = 0; c < dh; ++c) {
+          const uint2 w = *reinterpret_cast<const uint2*>(a.WkT + c * hd + jk);
+          const float w0 = __uint_as_float(w.x << 16), w1 = __uint_as_float(w.x & 0xFFFF0000u);
+          const float w2 = __uint_as_float(w.y << 16), w3 = __uint_as_float(w.y & 0xFFFF0000u);
+          const float4* pp = reinterpret_cast<const float4*>(scr + (j * dh + c) * kTgt);
+#pragma unroll
+          for (int t4 = 0; t4 < 4; ++t4) {
+            const float4 pv = pp[t4];
+            const float pt[4] = {pv.x, pv.y, pv.z, pv.w};
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              float* ac = acc[4 * t4 + u];
+              ac[0] = fmaf(pt[u], w0, ac[0]);
+              ac[1] = fmaf(pt[u], w1, ac[1]);
+              ac[2] = fmaf(pt[u], w2, ac[2]);
+              ac[3] = fmaf(pt[u], w3, ac[3]);
+            }
+          }
+        }
+#pragma unroll
+        for (int t = 0; t < kTgt; ++t)
+          if (t < nb) {
+            uint2 o;
+            o.x = pack_bf16x2(acc[t][0] * a.uscale, acc[t][1] * a.uscale);
+            o.y = pack_bf16x2(acc[t][2] * a.uscale, acc[t][3] * a.uscale);
+            *reinterpret_cast<uint2*>(a.Ubf + (t0 + t) * hd + jk) = o;
+          }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 128);
+  }
+}
+
+}  // namespace
+
+// ------------------------------------------------------------------ launch
+// layer < 0: q(1) and its u; 0 <= layer < M-1: output of layer `layer`, then
+// q(layer+2) and its u; layer = M-1: output only.  Writes the bf16 query rows
+// scaled by log2(e) / sqrt(d_h) (the tensor-core attention's units).
+int launch_step_tc(const stca_handle* H, int layer, const void* targets, int64_t T,
+                   const float* cmerged, float* Z, uint16_t* Ubf, cudaStream_t s) {
+  if (T <= 0) return STCA_OK;
+  if (!H->step_tc_ready) return set_error(STCA_ESTATE, "tensor-core step weights are not set up");
+  const int M = H->M;
+  StepTcArgs a{};
+  a.layer = layer;
+  a.M = M; a.d = H->d; a.h = H->h; a.dh = H->dh; a.rd = H->rd;
+  a.T = T;
+  a.targets = static_cast<const uint16_t*>(targets);
+  a.cmerged = cmerged;
+  a.Z = Z;
+  a.Ubf = Ubf;
+  a.tiles = H->wstep_tc;
+  a.Wv = layer >= 0 ? static_cast<const uint16_t*>(H->Lstep[layer].Wv) : nullptr;
+  a.WkT = layer + 1 < M ? static_cast<const uint16_t*>(H->Lstep[layer + 1].WkT) : nullptr;
+  a.q_ln_g = H->q_ln_g;
+  a.q_ln_b = H->q_ln_b;
+  a.uscale = 1.4426950408889634f / sqrtf(static_cast<float>(H->dh));
+  a.status = H->status_d;
+  auto add = [&](int kind, const TcGemm& g) {
+    a.kind[a.ng] = kind;
+    a.g[a.ng] = g;
+    ++a.ng;
+  };
+  if (layer >= 0) add(kO, H->tcO[layer]);
+  if (layer + 1 < M) {
+    const int n = layer + 1;
+    if (layer >= 0) add(kC, H->tcC[n]);
+    add(kUG, H->tcUG[n]);
+    add(kD, H->tcD[n]);
+    add(kQ, H->tcQ[n]);
+  }
+  // the deepest ring that fits, and the widest W_V staging chunk that fits
+  // in the buffers it borrows
+  int nring = kMaxRing;
+  while (nring > 2 && step_layout(H->d, H->rd, M, nring).total + 1024 > 227u * 1024) --nring;
+  const StepLayout Y = step_layout(H->d, H->rd, M, nring);
+  if (Y.total + 1024 > 227u * 1024) return set_error(STCA_EINVAL, "tensor-core step: shared memory");
+  int kch = 32;
+  while (kch > 4 && static_cast<uint32_t>(kTgt * H->h * kch * 4 + kch * H->d * 2) > Y.red - Y.bU) kch /= 2;
+  if (static_cast<uint32_t>(kTgt * H->h * kch * 4 + kch * H->d * 2) > Y.red - Y.bU)
+    return set_error(STCA_EINVAL, "tensor-core step: too many heads for the W_V staging");
+  a.nring = nring;
+  a.kch = kch;
+  const size_t smem = Y.total + 1024;
+  cudaError_t e = cudaFuncSetAttribute(step_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return set_error(STCA_ECUDA, std::string("step_tc smem: ") + cudaGetErrorString(e));
+  const unsigned grid = static_cast<unsigned>((T + kTgt - 1) / kTgt);
+  step_tc_kernel<<<grid, kStepThreads, smem, s>>>(a);
+  return STCA_OK;
+}
+
+}  // namespace stca

@@ -31,7 +31,7 @@ def to_device(wl, a, device):
     return t.to(device)
 
 
-def run_gpu(wl, device, attn_path=0, encode_path=0, split=0, handle=None, keep=False):
+def run_gpu(wl, device, attn_path=0, encode_path=0, split=0, handle=None, keep=False, step_path=0):
     """Z (T x M x d, numpy fp32) from the CUDA path through the C ABI."""
     import torch
     import target_attention_jagged_b200 as S
@@ -43,6 +43,8 @@ def run_gpu(wl, device, attn_path=0, encode_path=0, split=0, handle=None, keep=F
             st.set_option(S.STCA_OPT_ENCODE_PATH, encode_path)
         if split:
             st.set_option(S.STCA_OPT_SPLIT_KEYS, split)
+        if step_path:
+            st.set_option(S.STCA_OPT_STEP_PATH, step_path)
         X = to_device(wl, wl.X, device)
         xt = to_device(wl, wl.targets, device)
         st.encode(X, wl.offsets)

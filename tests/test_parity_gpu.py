@@ -194,3 +194,30 @@ def test_forward_before_encode_and_bad_offsets(gpu):
         Z = torch.empty((0, 1, 64), device=gpu)
         st.forward(xt[:0], [0, 0, 0], Z)         # T = 0 is a no-op
         st.status()
+
+
+STEP_CC, STEP_TC = 1, 2
+
+
+@pytest.mark.parametrize("step", [STEP_TC, STEP_CC])
+@pytest.mark.parametrize("d,h,M,r,rln,dq", [(128, 8, 3, 4, False, False), (128, 4, 2, 2, True, True),
+                                            (256, 16, 4, 2, True, False), (256, 8, 1, 1, False, True),
+                                            (128, 2, 5, 1, True, True)])
+def test_step_paths(gpu, step, d, h, M, r, rln, dq):
+    """Both per-target step implementations against the oracle: 37 targets in
+    requests of 1 to 17 targets (16-target CTAs, the last one ragged), heads of
+    16 to 64 columns, one to five layers, affine LayerNorm, separate query FFN."""
+    wl = make_workload(lengths=[900, 130, 1, 2100, 64], targets=[9, 1, 3, 17, 7], d=d, h=h, M=M,
+                       r=r, dtype="bf16", seed=300 + d + h + M, random_ln=rln,
+                       distinct_query_ffn=dq)
+    check_full(wl, run_gpu(wl, gpu, step_path=step))
+
+
+def test_tensor_core_step_rejected_when_unsupported(gpu):
+    import target_attention_jagged_b200 as S
+    wl = make_workload(lengths=[50], targets=[2], d=64, h=4, M=1, r=2, dtype="bf16", seed=13)
+    with pytest.raises(S.StcaError):
+        run_gpu(wl, gpu, step_path=STEP_TC)
+    wl = make_workload(lengths=[50], targets=[2], d=128, h=4, M=1, r=2, dtype="bf16", seed=13)
+    with pytest.raises(S.StcaError):
+        run_gpu(wl, gpu, step_path=STEP_TC, attn_path=ATTN_SIMT)
