@@ -337,14 +337,24 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_tc_kernel(const StepTcAr
     } else {
       if (L + 1 < M) {
         // [o(1) .. o(L) | o(L+1): by the output epilogue | x_t] of Eq. (7)
-        const int wcat = (L + 2) * d;
-        for (int e = tid; e < kTgt * wcat; e += 32 * kWorkers) {
-          const int t = e / wcat, k = e - t * wcat;
-          const int blk = k / d, kk = k - blk * d;
+        // 8 inputs (one 16-byte chunk of a B row) per item
+        const int wcat8 = (L + 2) * d / 8, d8 = d / 8;
+        for (int e = tid; e < kTgt * wcat8; e += 32 * kWorkers) {
+          const int t = e / wcat8, k8 = e - t * wcat8;
+          const int blk = k8 / d8, kk = 8 * (k8 - blk * d8);
           if (blk == L) continue;
-          float v = 0.f;
-          if (t < nb) v = blk < L ? a.Z[((t0 + t) * M + blk) * d + kk] : bf2f(a.targets[(t0 + t) * d + kk]);
-          put_b1(bufs[kC], t, k, v);
+          uint4 v = make_uint4(0u, 0u, 0u, 0u);
+          if (t < nb) {
+            if (blk < L) {
+              const float4* z = reinterpret_cast<const float4*>(a.Z + ((t0 + t) * M + blk) * d + kk);
+              const float4 z0 = z[0], z1 = z[1];
+              v = make_uint4(pack_bf16x2(z0.x, z0.y), pack_bf16x2(z0.z, z0.w),
+                             pack_bf16x2(z1.x, z1.y), pack_bf16x2(z1.z, z1.w));
+            } else {
+              v = *reinterpret_cast<const uint4*>(a.targets + (t0 + t) * d + kk);
+            }
+          }
+          *reinterpret_cast<uint4*>(bufs[kC] + (8 * k8 >> 6) * kBTile + sw128_off(t, (8 * k8) & 63)) = v;
         }
       }
       // o_head = c_j W_V^j into the B operand of W_O.  Output column n belongs
@@ -362,26 +372,54 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_tc_kernel(const StepTcAr
 #pragma unroll
         for (int t = 0; t < 4; ++t) acc[bi][t][0] = acc[bi][t][1] = 0.f;
       const int nblk = 2 * d;                         // (16 / 4) x (d / 2) blocks
+      // per thread and chunk: at most kMaxC float4 of c_j and kMaxW uint4 of
+      // W_V, all loaded before any is stored so the loads overlap
+      constexpr int kMaxC = 8, kMaxW = 4;
+      const int nc = kTgt * h * (kch / 4), nw = kch * d / 8;
+      // the items of this thread are the same in every chunk: their source
+      // offsets (at k0 = 0) and destinations, once; -1 marks no item
+      int c_src[kMaxC], c_dst[kMaxC], w_src[kMaxW], w_dst[kMaxW];
+#pragma unroll
+      for (int i = 0; i < kMaxC; ++i) {
+        const int e = tid + i * 32 * kWorkers;
+        const int t = e % kTgt, rest = e / kTgt;
+        const int j = rest % h, k4 = rest / h;
+        c_dst[i] = e < nc ? (j * kch + 4 * k4) * kTgt + t : -1;
+        c_src[i] = e < nc && t < nb ? (t * h + j) * d + 4 * k4 : -1;   // from this CTA's rows
+      }
+#pragma unroll
+      for (int i = 0; i < kMaxW; ++i) {
+        const int e = tid + i * 32 * kWorkers;
+        const int k = e / (d / 8), c8 = e - k * (d / 8);
+        w_src[i] = e < nw ? k * d + 8 * c8 : -1;
+        w_dst[i] = w_src[i];
+      }
+      const float* cm = a.cmerged + t0 * h * d;
       for (int k0 = 0; k0 < d; k0 += kch) {
-        // c_j[t][k0 .. k0 + kch): one float4 of 4 inputs per (t, j, k4)
-        for (int e = tid; e < kTgt * h * (kch / 4); e += 32 * kWorkers) {
-          const int t = e % kTgt, rest = e / kTgt;
-          const int j = rest % h, k4 = rest / h;
-          float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-          if (t < nb)
-            v = *reinterpret_cast<const float4*>(a.cmerged + ((t0 + t) * h + j) * d + k0 + 4 * k4);
-          float* dst = cs + (j * kch + 4 * k4) * kTgt + t;
-          dst[0] = v.x;
-          dst[kTgt] = v.y;
-          dst[2 * kTgt] = v.z;
-          dst[3 * kTgt] = v.w;
+        float4 cv[kMaxC];
+        uint4 wv[kMaxW];
+#pragma unroll
+        for (int i = 0; i < kMaxC; ++i) {
+          cv[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+          if (c_src[i] >= 0) cv[i] = __ldg(reinterpret_cast<const float4*>(cm + c_src[i] + k0));
         }
-        // W_V rows k0 .. k0 + kch, 16 bytes at a time
-        for (int e = tid; e < kch * d / 8; e += 32 * kWorkers) {
-          const int k = e / (d / 8), c8 = e - k * (d / 8);
-          *reinterpret_cast<uint4*>(ws + k * d + 8 * c8) =
-              *reinterpret_cast<const uint4*>(a.Wv + (k0 + k) * d + 8 * c8);
-        }
+#pragma unroll
+        for (int i = 0; i < kMaxW; ++i)
+          if (w_src[i] >= 0) wv[i] = __ldg(reinterpret_cast<const uint4*>(a.Wv + k0 * d + w_src[i]));
+        // c_j[t][k0 .. k0 + kch) as cs[j][k][t]
+#pragma unroll
+        for (int i = 0; i < kMaxC; ++i)
+          if (c_dst[i] >= 0) {
+            float* dst = cs + c_dst[i];
+            dst[0] = cv[i].x;
+            dst[kTgt] = cv[i].y;
+            dst[2 * kTgt] = cv[i].z;
+            dst[3 * kTgt] = cv[i].w;
+          }
+        // W_V rows k0 .. k0 + kch
+#pragma unroll
+        for (int i = 0; i < kMaxW; ++i)
+          if (w_dst[i] >= 0) *reinterpret_cast<uint4*>(ws + w_dst[i]) = wv[i];
         workers_sync();
 #pragma unroll
         for (int bi = 0; bi < kMaxBlk; ++bi) {
@@ -390,6 +428,7 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_tc_kernel(const StepTcAr
             const int t4 = b & 3, n = 2 * (b >> 2), j = n / dh;
             const float* cp = cs + j * kch * kTgt + 4 * t4;
             const uint16_t* wp = ws + n;
+#pragma unroll 8
             for (int k = 0; k < kch; ++k) {
               const float4 c = *reinterpret_cast<const float4*>(cp + k * kTgt);
               const uint32_t w2 = *reinterpret_cast<const uint32_t*>(wp + k * d);
@@ -522,22 +561,31 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_tc_kernel(const StepTcAr
         float acc[kTgt][4];
 #pragma unroll
         for (int t = 0; t < kTgt; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.f;
-        for (int c = 0; c < dh; ++c) {
-          const uint2 w = *reinterpret_cast<const uint2*>(a.WkT + c * hd + jk);
-          const float w0 = __uint_as_float(w.x << 16), w1 = __uint_as_float(w.x & 0xFFFF0000u);
-          const float w2 = __uint_as_float(w.y << 16), w3 = __uint_as_float(w.y & 0xFFFF0000u);
-          const float4* pp = reinterpret_cast<const float4*>(scr + (j * dh + c) * kTgt);
+        for (int c0 = 0; c0 < dh; c0 += 8) {        // d_h is even; 8 loads in flight
+          uint2 wk[8];
 #pragma unroll
-          for (int t4 = 0; t4 < 4; ++t4) {
-            const float4 pv = pp[t4];
-            const float pt[4] = {pv.x, pv.y, pv.z, pv.w};
+          for (int u = 0; u < 8; ++u)
+            if (c0 + u < dh) wk[u] = __ldg(reinterpret_cast<const uint2*>(a.WkT + (c0 + u) * hd + jk));
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              float* ac = acc[4 * t4 + u];
-              ac[0] = fmaf(pt[u], w0, ac[0]);
-              ac[1] = fmaf(pt[u], w1, ac[1]);
-              ac[2] = fmaf(pt[u], w2, ac[2]);
-              ac[3] = fmaf(pt[u], w3, ac[3]);
+          for (int u8 = 0; u8 < 8; ++u8) {
+            const int c = c0 + u8;
+            if (c >= dh) break;
+            const uint2 w = wk[u8];
+            const float w0 = __uint_as_float(w.x << 16), w1 = __uint_as_float(w.x & 0xFFFF0000u);
+            const float w2 = __uint_as_float(w.y << 16), w3 = __uint_as_float(w.y & 0xFFFF0000u);
+            const float4* pp = reinterpret_cast<const float4*>(scr + (j * dh + c) * kTgt);
+#pragma unroll
+            for (int t4 = 0; t4 < 4; ++t4) {
+              const float4 pv = pp[t4];
+              const float pt[4] = {pv.x, pv.y, pv.z, pv.w};
+#pragma unroll
+              for (int u = 0; u < 4; ++u) {
+                float* ac = acc[4 * t4 + u];
+                ac[0] = fmaf(pt[u], w0, ac[0]);
+                ac[1] = fmaf(pt[u], w1, ac[1]);
+                ac[2] = fmaf(pt[u], w2, ac[2]);
+                ac[3] = fmaf(pt[u], w3, ac[3]);
+              }
             }
           }
         }
@@ -605,9 +653,15 @@ int launch_step_tc(const stca_handle* H, int layer, const void* targets, int64_t
   while (nring > 2 && step_layout(H->d, H->rd, M, nring).total + 1024 > 227u * 1024) --nring;
   const StepLayout Y = step_layout(H->d, H->rd, M, nring);
   if (Y.total + 1024 > 227u * 1024) return set_error(STCA_EINVAL, "tensor-core step: shared memory");
+  // the W_V staging loads at most 8 float4 of c_j and 4 x 16 bytes of W_V per
+  // worker thread and chunk
+  auto stage_ok = [&](int k) {
+    return static_cast<uint32_t>(kTgt * H->h * k * 4 + k * H->d * 2) <= Y.red - Y.bU &&
+           kTgt * H->h * (k / 4) <= 8 * 32 * kWorkers && k * H->d / 8 <= 4 * 32 * kWorkers;
+  };
   int kch = 32;
-  while (kch > 4 && static_cast<uint32_t>(kTgt * H->h * kch * 4 + kch * H->d * 2) > Y.red - Y.bU) kch /= 2;
-  if (static_cast<uint32_t>(kTgt * H->h * kch * 4 + kch * H->d * 2) > Y.red - Y.bU)
+  while (kch > 4 && !stage_ok(kch)) kch /= 2;
+  if (!stage_ok(kch))
     return set_error(STCA_EINVAL, "tensor-core step: too many heads for the W_V staging");
   a.nring = nring;
   a.kch = kch;
