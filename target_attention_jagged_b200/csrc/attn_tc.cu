@@ -8,18 +8,23 @@
 //   P = exp2(S - m), online max / sum per row (CUDA cores, one row per thread)
 //   O += P X~_tile               (tcgen05, M = 128, N = d, K = 128 keys)
 // The same shared-memory copy of each X~ tile is the K-major B operand of the
-// first MMA and the MN-major B operand of the second.  Work is cut stream-K
-// style: every CTA gets an equal run of (query tile, key tile) units in
-// (request, query tile, key) order, so ragged lengths do not unbalance the SMs;
-// each maximal run inside one (request, query tile) pair is an item that
-// writes an unnormalised partial (O, m, l) for the split combine.
+// first MMA and the MN-major B operand of the second.  With d <= 128, P stays
+// in TMEM (packed bf16) and the second MMA takes it from there, which keeps
+// shared-memory bandwidth for the MMAs' operands and the TMA writes.  Work is
+// cut stream-K style: every CTA gets an equal run of (query tile, key tile)
+// units in (request, query tile, key) order, so ragged lengths do not
+// unbalance the SMs; each maximal run inside one (request, query tile) pair is
+// an item that writes an unnormalised partial (O, m, l) for the split combine.
 //
 // The running max is rescaled lazily: O and l are corrected only when a row's
 // max grows by more than 8 (log2 units); otherwise P uses the stale max and
 // stays below 2^8, well inside bf16 and fp32 range.
 //
-// Warp roles (192 threads): warp 0 TMA, warp 1 MMA issue + TMEM owner, warps
-// 2-5 softmax / correction / partial store, one query row per thread.
+// Warp roles (352 threads): warp 0 TMA, warp 1 issues S (and owns TMEM),
+// warps 2-9 softmax / correction / partial store (one query row per thread,
+// two warps -- key halves -- per row), warp 10 issues P X~.  Two issuers let
+// S of later tiles run ahead of the P X~ products, which wait for the
+// softmax.
 #include <cuda.h>
 
 #include <algorithm>
@@ -43,8 +48,14 @@ struct AttnParams {
   int* status;
 };
 
+// P_TMEM: P lives in TMEM (packed bf16, 64 columns per buffer) and the P X~
+// product reads it from there; with d = 256 TMEM is full (S and O) and P goes
+// through shared memory.  Keeping P out of shared memory matters: the MMAs'
+// operand reads, the TMA writes of X~ and the P writes would otherwise all
+// share its bandwidth.
 template <int D, int QB, int KS, int PB>
 struct AttnCfg {
+  static constexpr bool P_TMEM = D <= 128;
   static constexpr int KB = D / 64;
   static constexpr uint32_t kBlock = 128u * 128u;       // [128 rows x 64] bf16
   static constexpr uint32_t kTile = KB * kBlock;         // [128 rows x D]
@@ -52,17 +63,24 @@ struct AttnCfg {
   static constexpr uint32_t oQ = 0;
   static constexpr uint32_t oK = oQ + QB * kTile;
   static constexpr uint32_t oP = oK + KS * kTile;
-  static constexpr uint32_t oBar = oP + PB * kPBytes;
-  static constexpr int kBars = 2 * QB + 2 * KS + 4 + 2 * PB + 3 + 1;
+  static constexpr uint32_t oX = oP + (P_TMEM ? 0 : PB * kPBytes);   // pair exchange: 2 x 2 x 128 floats
+  static constexpr uint32_t oBar = oX + 2 * 2 * 128 * 4;
+  static constexpr int kBars = 2 * QB + 2 * KS + 4 + 2 * PB + 3 + 1 + 8;
   static constexpr uint32_t oMisc = oBar + kBars * 8;
-  static constexpr uint32_t kSmem = oMisc + 16 + 1024;
+  // No alignment slack: the dynamic shared memory of a block starts at a
+  // 1024-byte boundary (after the 1 KB the system reserves), and the kernel
+  // checks that before it uses any of it.
+  static constexpr uint32_t kSmem = oMisc + 16;
   static constexpr uint32_t kS = 0;        // 2 x 128 TMEM columns of scores
   static constexpr uint32_t kO = 256;      // D columns of the output accumulator
-  static_assert(kO + D <= 512, "TMEM overflow");
+  static constexpr uint32_t kPt = kO + D;  // P_TMEM: PB x 64 columns of P
+  static_assert(kO + D + (P_TMEM ? PB * 64 : 0) <= 512, "TMEM overflow");
   static_assert(kSmem <= 227 * 1024, "shared memory overflow");
 };
 
-constexpr int kAttnThreads = 192;
+constexpr int kSoftWarps = 8;               // two per TMEM lane quarter
+constexpr int kPvWarp = 2 + kSoftWarps;     // issues the P X~ products
+constexpr int kAttnThreads = 32 * (kPvWarp + 1);
 constexpr float kRescaleThreshold = 8.0f;   // log2 units
 
 __device__ __forceinline__ bool bwait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
@@ -85,6 +103,23 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
+// 2^x on the FMA pipe, for x <= 8 (a score is at most 8 above the row's
+// running max): x = j + f with j = round(x) (magic-number rounding) and
+// f in [-1/2, 1/2]; 2^f by a degree-3 polynomial fitted here to a relative
+// error of 7.5e-5 (1.5e-4 with the fp32 evaluation) on that interval; j is
+// added to the exponent bits.  Below -126 the result is held at 2^-126, which
+// is zero at the precision of P (bf16).  A share of the softmax's
+// exponentials goes this way so that they do not all queue on the MUFU.
+__device__ __forceinline__ float ex2_fma(float x) {
+  x = fmaxf(x, -126.0f);
+  const float t = x + 12582912.0f;                 // 1.5 * 2^23: round(x) in the low bits
+  const float f = x - (t - 12582912.0f);
+  float p = fmaf(f, 0.05517259240150452f, 0.24261370301246643f);
+  p = fmaf(f, p, 0.6932610273361206f);
+  p = fmaf(f, p, 0.9999278783798218f);
+  return __uint_as_float(__float_as_uint(p) + (__float_as_uint(t) << 23));
+}
+
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
@@ -105,9 +140,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const AttnParams p) {
   using C = AttnCfg<D, QB, KS, PB>;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                           ~static_cast<uintptr_t>(1023));
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  if (smem_u32(smem_raw) & 1023u) {      // the swizzled tiles need 1024-byte alignment
+    if (threadIdx.x == 0) atomicOr(p.status, kStatusAttnTimeout);
+    return;
+  }
+  uint8_t* sm = smem_raw;
   uint64_t* qfull = reinterpret_cast<uint64_t*>(sm + C::oBar);
   uint64_t* qempty = qfull + QB;
   uint64_t* kfull = qempty + QB;
@@ -120,6 +158,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   uint64_t* ofinal = odone + 1;       // one phase per item
   uint64_t* oempty = ofinal + 1;      // one phase per item (partial stored)
   uint64_t* mdrain = oempty + 1;
+  uint64_t* xmax = mdrain + 1;        // [quarter][parity]: the pair's exchange
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + C::oMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + C::oMisc + 4);
 
@@ -128,12 +167,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   if (threadIdx.x == 0) {
     for (int i = 0; i < QB; ++i) { mbar_init(&qfull[i], 1); mbar_init(&qempty[i], 1); }
     for (int i = 0; i < KS; ++i) { mbar_init(&kfull[i], 1); mbar_init(&kempty[i], 1); }
-    for (int i = 0; i < 2; ++i) { mbar_init(&sfull[i], 1); mbar_init(&sempty[i], 4); }
-    for (int i = 0; i < PB; ++i) { mbar_init(&pfull[i], 4); mbar_init(&pempty[i], 1); }
+    for (int i = 0; i < 2; ++i) { mbar_init(&sfull[i], 1); mbar_init(&sempty[i], kSoftWarps); }
+    for (int i = 0; i < PB; ++i) { mbar_init(&pfull[i], kSoftWarps); mbar_init(&pempty[i], 1); }
     mbar_init(odone, 1);
     mbar_init(ofinal, 1);
-    mbar_init(oempty, 4);
-    mbar_init(mdrain, 1);
+    mbar_init(oempty, kSoftWarps);
+    mbar_init(mdrain, 2);
+    for (int i = 0; i < 8; ++i) mbar_init(&xmax[i], 2);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -183,27 +223,25 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       }
     }
   } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
+    // ------------------------------------------------------------ S issuer
+    // S of the next tile is issued as soon as its TMEM buffer is free (the
+    // softmax has loaded the tile two back), ahead of the P X~ products.
     if (lane == 0) {
       constexpr uint32_t idS = idesc_bf16(128, 128);                 // Q K-major, X~ K-major
-      constexpr uint32_t idO = idesc_bf16(128, D, false, true);      // P K-major, X~ MN-major
-      uint32_t qi = 0, ki = 0, sc = 0, pc = 0, ic = 0;
+      uint32_t qi = 0, ki = 0, sc = 0;
       bool ok = true;
-      for (int it = it0; ok && it < it1; ++it, ++ic) {
+      for (int it = it0; ok && it < it1; ++it) {
         const AttnItem item = p.items[it];
         const int nt = (item.nkeys + 127) >> 7;
         const int qb = qi % QB;
         if (!(ok = bwait(&qfull[qb], (qi / QB) & 1, abort_flag, p.status))) break;
         tc_fence_after();
         const uint32_t qaddr = sbase + C::oQ + qb * C::kTile;
-        uint32_t stage_prev = 0;
-        // S(0)
-        auto issue_s = [&](uint32_t& stage_out) -> bool {
+        for (int j = 0; ok && j < nt; ++j, ++sc, ++ki) {
           const int sb = sc & 1;
-          if (!bwait(&sempty[sb], ((sc >> 1) & 1) ^ 1, abort_flag, p.status)) return false;
-          tc_fence_after();
+          if (!(ok = bwait(&sempty[sb], ((sc >> 1) & 1) ^ 1, abort_flag, p.status))) break;
           const int s = ki % KS;
-          if (!bwait(&kfull[s], (ki / KS) & 1, abort_flag, p.status)) return false;
+          if (!(ok = bwait(&kfull[s], (ki / KS) & 1, abort_flag, p.status))) break;
           tc_fence_after();
           const uint32_t kaddr = sbase + C::oK + s * C::kTile;
 #pragma unroll
@@ -213,109 +251,152 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                         sdesc_sw128(kaddr + (kk >> 2) * C::kBlock + (kk & 3) * 32, 16, 1024),
                         idS, kk != 0);
           mma_commit(&sfull[sb]);
-          stage_out = s;
-          ++sc;
-          ++ki;
-          return true;
-        };
-        if (!(ok = issue_s(stage_prev))) break;
-        for (int j = 0; ok && j < nt; ++j) {
-          const uint32_t stage_j = stage_prev;
-          if (j + 1 < nt) {
-            if (!(ok = issue_s(stage_prev))) break;
-          }
           if (j + 1 == nt) mma_commit(&qempty[qb]);
+        }
+        ++qi;
+      }
+      mma_commit(mdrain);
+      drain_wait(mdrain, 0, 500000000ull);
+    }
+  } else if (warp == kPvWarp) {
+    // ------------------------------------------------------------ P X~ issuer
+    // The K tile of S(j) is the V tile of this product; its arrival is known
+    // from the S issuer's wait (S(j) -> softmax(j) -> pfull), and its stage is
+    // released here.
+    if (lane == 0) {
+      constexpr uint32_t idO = idesc_bf16(128, D, false, true);      // P K-major, X~ MN-major
+      uint32_t ki = 0, pc = 0, ic = 0;
+      bool ok = true;
+      for (int it = it0; ok && it < it1; ++it, ++ic) {
+        const AttnItem item = p.items[it];
+        const int nt = (item.nkeys + 127) >> 7;
+        for (int j = 0; ok && j < nt; ++j, ++pc, ++ki) {
           const int pb = pc % PB;
           if (!(ok = bwait(&pfull[pb], (pc / PB) & 1, abort_flag, p.status))) break;
+          if (j == 0 && !(ok = bwait(oempty, (ic & 1) ^ 1, abort_flag, p.status))) break;
           tc_fence_after();
-          if (j == 0) {
-            if (!(ok = bwait(oempty, (ic & 1) ^ 1, abort_flag, p.status))) break;
-            tc_fence_after();
-          }
-          const uint32_t paddr = sbase + C::oP + pb * C::kPBytes;
-          const uint32_t vaddr = sbase + C::oK + stage_j * C::kTile;
+          const int s = ki % KS;
+          const uint32_t vaddr = sbase + C::oK + s * C::kTile;
+          if constexpr (C::P_TMEM) {
+            // P: keys 2c, 2c+1 in column c of the buffer; 16 keys = 8 columns per MMA
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk)   // 16 keys per MMA
-            mma_bf16_ss(tmem + C::kO,
-                        sdesc_sw128(paddr + (kk >> 2) * C::kBlock + (kk & 3) * 32, 16, 1024),
-                        sdesc_sw128(vaddr + kk * 2048, C::kBlock, 1024), idO,
-                        (j | kk) != 0);
-          mma_commit(&kempty[stage_j]);
+            for (int kk = 0; kk < 8; ++kk)
+              mma_bf16_ts(tmem + C::kO, tmem + C::kPt + pb * 64 + kk * 8,
+                          sdesc_sw128(vaddr + kk * 2048, C::kBlock, 1024), idO, (j | kk) != 0);
+          } else {
+            const uint32_t paddr = sbase + C::oP + pb * C::kPBytes;
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk)   // 16 keys per MMA
+              mma_bf16_ss(tmem + C::kO,
+                          sdesc_sw128(paddr + (kk >> 2) * C::kBlock + (kk & 3) * 32, 16, 1024),
+                          sdesc_sw128(vaddr + kk * 2048, C::kBlock, 1024), idO,
+                          (j | kk) != 0);
+          }
+          mma_commit(&kempty[s]);
           mma_commit(&pempty[pb]);
           mma_commit(odone);
-          ++pc;
         }
         if (!ok) break;
         mma_commit(ofinal);
-        ++qi;
       }
       mma_commit(mdrain);
       drain_wait(mdrain, 0, 500000000ull);
     }
   } else {
     // ------------------------------------------------------------ softmax + partials
+    // Two warps per TMEM lane quarter: half hf of the pair takes keys
+    // [64 hf, 64 hf + 64) of every tile for the quarter's 32 query rows, and
+    // columns [hf D/2, (hf + 1) D/2) of O when it is rescaled or stored.  The
+    // pair swaps row maxima (and, at the end of an item, row sums) through
+    // shared memory; both then take identical rescaling decisions.
     const int q = warp & 3;
+    const int hf = (warp - 2) >> 2;
     const int r = q * 32 + lane;              // query row of the tile (TMEM lane)
     const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
+    float* xbuf = reinterpret_cast<float*>(sm + C::oX);   // [2 parity][2 halves][128 rows]
+    uint64_t* xbar = xmax + q * 2;            // this pair's exchange barriers
+    uint32_t xp = 0;                          // exchanges so far
+    // swap v with the partner warp: returns the partner's value for row r
+    auto swap_with_pair = [&](float v, bool& okk) -> float {
+      float* xs = xbuf + (xp & 1) * 256;
+      xs[hf * 128 + r] = v;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&xbar[xp & 1]);
+      okk = bwait(&xbar[xp & 1], (xp >> 1) & 1, abort_flag, p.status);
+      const float o = xs[(hf ^ 1) * 128 + r];
+      ++xp;
+      return o;
+    };
     uint32_t sc = 0, pc = 0, ic = 0;
     bool ok = true;
     for (int it = it0; ok && it < it1; ++it, ++ic) {
       const AttnItem item = p.items[it];
       const int nt = (item.nkeys + 127) >> 7;
-      float m_used = -1e30f, l = 0.f;
+      float m_used = -1e30f, l = 0.f;         // l: this half's share of the row sum
       for (int j = 0; j < nt; ++j) {
         const int sb = sc & 1;
         if (!(ok = bwait(&sfull[sb], (sc >> 1) & 1, abort_flag, p.status))) break;
         __syncwarp();
         tc_fence_after();
-        uint32_t sv[4][32];
+        uint32_t sv[2][32];
 #pragma unroll
-        for (int cb = 0; cb < 4; ++cb) tmem_ld32(tmem + lane_off + C::kS + sb * 128 + cb * 32, sv[cb]);
+        for (int cb = 0; cb < 2; ++cb)
+          tmem_ld32(tmem + lane_off + C::kS + sb * 128 + hf * 64 + cb * 32, sv[cb]);
         tmem_ld_wait();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&sempty[sb]);
         ++sc;
-        const int nvalid = min(128, item.nkeys - j * 128);
-        if (nvalid < 128) {   // the request's last tile: keys past its end take no weight
+        const int nvalid = min(128, item.nkeys - j * 128) - hf * 64;
+        if (nvalid < 64) {   // the request's last tile: keys past its end take no weight
 #pragma unroll
-          for (int cb = 0; cb < 4; ++cb)
+          for (int cb = 0; cb < 2; ++cb)
 #pragma unroll
             for (int k = 0; k < 32; ++k)
               if (cb * 32 + k >= nvalid) sv[cb][k] = __float_as_uint(-INFINITY);
         }
-        float mx = -INFINITY;
+        float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-        for (int cb = 0; cb < 4; ++cb)
+        for (int cb = 0; cb < 2; ++cb)
 #pragma unroll
-          for (int k = 0; k < 32; ++k) mx = fmaxf(mx, __uint_as_float(sv[cb][k]));
+          for (int k = 0; k < 32; ++k) m4[k & 3] = fmaxf(m4[k & 3], __uint_as_float(sv[cb][k]));
+        const float mloc = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+        const float mx = fmaxf(mloc, swap_with_pair(mloc, ok));
+        if (!ok) break;
         const bool resc = mx > m_used + kRescaleThreshold;
         const float m_new = resc ? mx : m_used;
         const float corr = resc ? ex2(m_used - m_new) : 1.f;
         l *= corr;
         m_used = m_new;
-        uint32_t pk[64];
-        float lsum = 0.f;
+        uint32_t pk[32];
+        float ls[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int cb = 0; cb < 4; ++cb)
+        for (int cb = 0; cb < 2; ++cb)
 #pragma unroll
           for (int k = 0; k < 32; k += 2) {
             const float p0 = ex2(__uint_as_float(sv[cb][k]) - m_new);      // exp2(-inf) = 0
-            const float p1 = ex2(__uint_as_float(sv[cb][k + 1]) - m_new);
-            lsum += p0 + p1;
+            const float x1 = __uint_as_float(sv[cb][k + 1]) - m_new;
+            // with d <= 128, 1 in 4 on the FMA pipe (MUFU-bound); with d = 256 the
+            // softmax is bound by instruction issue, and all go to the MUFU
+            const float p1 = (C::P_TMEM && (k & 2)) ? ex2_fma(x1) : ex2(x1);
+            ls[(k >> 1) & 3] += p0 + p1;
             pk[(cb * 32 + k) >> 1] = pack_bf16x2(p0, p1);
           }
-        l += lsum;
+        l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
         const int pb = pc % PB;
         if (!(ok = bwait(&pempty[pb], ((pc / PB) & 1) ^ 1, abort_flag, p.status))) break;
         __syncwarp();
-        // P row: keys 0..63 in block 0, 64..127 in block 1, K-major, 128-B swizzle
-        const uint32_t prow = sbase + C::oP + pb * C::kPBytes + r * 128;
+        if constexpr (C::P_TMEM) {
+          // P row, keys 64 hf .. 64 hf + 63: columns 32 hf .. 32 hf + 31 of the buffer
+          tmem_st32(tmem + lane_off + C::kPt + pb * 64 + hf * 32, pk);
+          tmem_st_wait();
+        } else {
+          // P row, keys 64 hf .. 64 hf + 63: block hf of the tile, K-major, 128-B swizzle
+          const uint32_t prow = sbase + C::oP + pb * C::kPBytes + hf * C::kBlock + r * 128;
 #pragma unroll
-        for (int c = 0; c < 16; ++c) {
-          const uint32_t blk = (c >> 3) * C::kBlock;
-          st_shared_v4(prow + blk + (((c & 7) ^ (r & 7)) << 4), pk[4 * c], pk[4 * c + 1],
-                       pk[4 * c + 2], pk[4 * c + 3]);
+          for (int c = 0; c < 8; ++c)
+            st_shared_v4(prow + ((c ^ (r & 7)) << 4), pk[4 * c], pk[4 * c + 1], pk[4 * c + 2],
+                         pk[4 * c + 3]);
         }
         if (j > 0 && __any_sync(0xffffffffu, resc)) {
           // O holds the rows' sums up to tile j-1: wait for that MMA, then rescale
@@ -323,7 +404,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           __syncwarp();
           tc_fence_after();
 #pragma unroll 1
-          for (int cb = 0; cb < D / 32; ++cb) {
+          for (int cb = hf * (D / 64); cb < (hf + 1) * (D / 64); ++cb) {
             uint32_t ov[32];
             tmem_ld32(tmem + lane_off + C::kO + cb * 32, ov);
             tmem_ld_wait();
@@ -340,7 +421,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         ++pc;
       }
       if (!ok) break;
-      // item done: store the unnormalised partial of the valid rows
+      // item done: the row sum is both halves' shares
+      l += swap_with_pair(l, ok);
+      if (!ok) break;
+      // store the unnormalised partial of the valid rows, this half's columns
       if (!(ok = bwait(ofinal, ic & 1, abort_flag, p.status))) break;
       __syncwarp();
       tc_fence_after();
@@ -348,7 +432,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       const int64_t g = item.row_base + r;
       float* dst = p.pacc + g * D;
 #pragma unroll 1
-      for (int cb = 0; cb < D / 32; ++cb) {
+      for (int cb = hf * (D / 64); cb < (hf + 1) * (D / 64); ++cb) {
         uint32_t ov[32];
         tmem_ld32(tmem + lane_off + C::kO + cb * 32, ov);
         tmem_ld_wait();
@@ -360,7 +444,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                                 __uint_as_float(ov[4 * k + 2]), __uint_as_float(ov[4 * k + 3]));
         }
       }
-      if (valid) {
+      if (valid && hf == 0) {
         p.pm[g] = m_used;
         p.pl[g] = l;
       }
@@ -404,8 +488,8 @@ int launch_attn_tc(stca_handle* H, int layer, const AttnItem* items_d, const int
   p.status = H->status_d;
   const CUtensorMap& tmK = H->tmXt[layer];
   switch (H->d) {
-    case 64: return launch_cfg<64, 2, 6, 2>(H, H->tmU, tmK, p, grid, s);
-    case 128: return launch_cfg<128, 2, 3, 2>(H, H->tmU, tmK, p, grid, s);
+    case 64: return launch_cfg<64, 2, 10, 2>(H, H->tmU, tmK, p, grid, s);
+    case 128: return launch_cfg<128, 2, 5, 2>(H, H->tmU, tmK, p, grid, s);
     case 256: return launch_cfg<256, 1, 2, 1>(H, H->tmU, tmK, p, grid, s);
     default: return set_error(STCA_EINVAL, "tensor-core attention needs d in {64, 128, 256}");
   }
@@ -423,8 +507,8 @@ int launch_attn_tc_ws(int d, const CUtensorMap& tmQ, const CUtensorMap& tmK,
   p.pl = p.pm + G;
   p.status = status;
   switch (d) {
-    case 64: return launch_cfg<64, 2, 6, 2>(nullptr, tmQ, tmK, p, grid, s);
-    case 128: return launch_cfg<128, 2, 3, 2>(nullptr, tmQ, tmK, p, grid, s);
+    case 64: return launch_cfg<64, 2, 10, 2>(nullptr, tmQ, tmK, p, grid, s);
+    case 128: return launch_cfg<128, 2, 5, 2>(nullptr, tmQ, tmK, p, grid, s);
     case 256: return launch_cfg<256, 1, 2, 1>(nullptr, tmQ, tmK, p, grid, s);
     default: return set_error(STCA_EINVAL, "tensor-core attention needs d in {64, 128, 256}");
   }
