@@ -191,8 +191,9 @@ int stca_validate_offsets(const int64_t* offsets, int64_t R, int64_t total,
 /*
  * Host only, no device needed: the attention work split the library uses for a
  * batch (the same planner stca_forward runs).  path 1: CUDA-core kernel, items
- * are key ranges of at most split_keys (default 1024) keys over all T_r * h
- * query rows.  path 2: tensor-core kernel, (request, 128-row query tile) pairs
+ * are key ranges of at most split_keys keys over all T_r * h query rows (by
+ * default 1024, or down to 128 when a batch has fewer than 2 num_ctas
+ * (range, target) pairs of 1024 keys).  path 2: tensor-core kernel, (request, 128-row query tile) pairs
  * cut into num_ctas runs of equal numbers of 128-key tiles (capped at
  * split_keys / 128 tiles when split_keys > 0), one run per CTA; each maximal
  * run inside a pair is an item.  Outputs: *n_items, *grid (CTAs, path 2),

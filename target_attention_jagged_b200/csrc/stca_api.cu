@@ -446,8 +446,9 @@ static int attn_path(const stca_handle* H) {
 
 // Cut the attention of one forward into work items.
 //  CUDA cores (path 1): each request's keys cut into ranges of at most `split`
-//    keys (1024 by default); one item per range covers all T_r * h query rows;
-//    the kernel grid is the list of (item, target) pairs.
+//    keys (by default 1024, or down to 128 for small batches so that the grid
+//    has two entries per CTA); one item per range covers all T_r * h query
+//    rows; the kernel grid is the list of (item, target) pairs.
 //  Tensor cores (path 2): (request, 128-row query tile) pairs, each over all
 //    its key tiles, laid end to end and cut into runs of equal numbers of key
 //    tiles, one run per CTA (stream-K); every maximal run inside one pair is
@@ -459,7 +460,15 @@ void stca::build_plan_host(const int64_t* off, const int64_t* toff, int64_t R, i
   auto& items = P.items;
   int64_t& G = P.G;
   if (path == 1) {
-    const int64_t split = split_keys > 0 ? split_keys : 1024;
+    // default: 1024 keys, or shorter ranges (down to 128) when that leaves
+    // fewer than two (item, target) grid entries per CTA
+    int64_t split = split_keys;
+    if (split <= 0) {
+      int64_t work = 0;                 // key-target pairs
+      for (int64_t r = 0; r < R; ++r) work += (toff[r + 1] - toff[r]) * (off[r + 1] - off[r]);
+      const int64_t per = (work + 2 * num_ctas - 1) / (2 * std::max(num_ctas, 1));
+      split = std::min<int64_t>(1024, std::max<int64_t>(128, (per + 127) / 128 * 128));
+    }
     for (int64_t r = 0; r < R; ++r) {
       P.req_pair_begin[r] = static_cast<int32_t>(r);
       P.pair_item_begin.push_back(static_cast<int32_t>(items.size()));
@@ -650,6 +659,9 @@ static int build_plan(stca_handle* H, const int64_t* toff, int64_t T, int path, 
   STCA_CUDA_TRY(cudaEventRecord(H->plan_evt, s));
   H->last_G = G;
   H->last_pairs = static_cast<int64_t>(pairs_simt.size() / 2);
+  H->last_max_items = 0;
+  for (size_t k = 0; k + 1 < pair_item_begin.size(); ++k)
+    H->last_max_items = std::max(H->last_max_items, pair_item_begin[k + 1] - pair_item_begin[k]);
   H->last_grid = grid;
   H->last_path = path;
   H->last_toff.assign(toff, toff + R + 1);
@@ -707,8 +719,14 @@ extern "C" int stca_forward(stca_handle* H, const void* targets, const int64_t* 
     return set_error(STCA_EINVAL, "tensor-core step needs the tensor-core attention, bf16, "
                                   "d in {128, 256} and r d <= 512");
   const bool step_tc = path == 2 && H->step_tc_ready && H->opt_step_path != 1;
+  // the tensor-core step merges the split partials itself when every query
+  // tile has few enough items; otherwise combine_kernel merges them first
+  const bool fused = step_tc && H->last_max_items <= step_tc_max_items() &&
+                     H->last_G < (int64_t(1) << 31);
   auto step = [&](int layer, const float* cm) {
-    if (step_tc) return launch_step_tc(H, layer, targets, T, cm, Z, H->Ubf, s);
+    if (step_tc)
+      return launch_step_tc(H, layer, targets, T, fused ? nullptr : cm, &plan, H->part, H->last_G,
+                            Z, H->Ubf, s);
     launch_target_step(H, layer, targets, T, plan, cm, Z, s);
     return static_cast<int>(STCA_OK);
   };
@@ -734,11 +752,14 @@ extern "C" int stca_forward(stca_handle* H, const void* targets, const int64_t* 
     if (int rc2 = check_launch("attention")) return rc2;
     {
       TimedLaunch tl(H, STCA_K_STEP, s);
-      launch_combine(H, plan, H->part, H->last_G, T, H->cbuf, s);
+      if (!fused) {
+        launch_combine(H, plan, H->part, H->last_G, T, H->cbuf, s);
+        H->launches++;
+      }
       rc = step(i, H->cbuf);
     }
     if (rc) return rc;
-    H->launches += 2;
+    H->launches++;
     if (int rc2 = check_launch("target step")) return rc2;
   }
   return ok();

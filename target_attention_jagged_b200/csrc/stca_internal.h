@@ -137,6 +137,7 @@ struct stca_handle {
   std::vector<int64_t> last_toff;
   int last_path = 0;                    // 1 CUDA cores, 2 tensor cores
   int64_t last_G = 0, last_pairs = 0;
+  int last_max_items = 0;               // most items of one (request, query tile) pair
   int last_grid = 0;                    // CTAs of the tensor-core attention
   size_t off_items = 0, off_pairs = 0, off_cta = 0, off_treq = 0, off_toff = 0, off_rpb = 0,
          off_pib = 0;
@@ -173,8 +174,13 @@ size_t attn_simt_smem(const stca_handle* H);
 // Tensor-core per-target step (step_tc.cu)
 bool step_tc_supported(const stca_handle* H);
 int step_tc_setup(stca_handle* H, const std::vector<StepHostW>& layers);
+// cmerged: the merged rows c_j (T x h x d), or NULL to merge the split
+// partials (part: G x d accumulators, then G maxima, G sums) inside the step;
+// that needs at most step_tc_max_items() items per (request, query tile).
+int step_tc_max_items();
 int launch_step_tc(const stca_handle* H, int layer, const void* targets, int64_t T,
-                   const float* cmerged, float* Z, uint16_t* Ubf, cudaStream_t s);
+                   const float* cmerged, const StepPlan* plan, const float* part, int64_t G,
+                   float* Z, uint16_t* Ubf, cudaStream_t s);
 
 // Host-side attention work plan (stca_api.cu).
 struct PlanHost {

@@ -143,7 +143,10 @@ struct StepTcArgs {
   int layer, M, d, h, dh, rd;
   int64_t T;
   const uint16_t* targets;      // T x d
-  const float* cmerged;         // T x h x d: c_j = alpha_j X~ of the layer just attended
+  const float* cmerged;         // T x h x d: c_j = alpha_j X~ of the layer just attended,
+                                // or NULL: merge the split partials here (plan, pacc, pm, pl)
+  StepPlan plan;
+  const float *pacc, *pm, *pl;  // split partials: G x d, G, G (log2 units)
   float* Z;                     // T x M x d
   uint16_t* Ubf;                // T x h x d: scaled u rows for the next attention
   const uint16_t* tiles;        // A-tile stream
@@ -165,10 +168,18 @@ struct StepTcArgs {
 // mbarriers.  bU .. the end of the scratch are not in use before the output
 // product, so the W_V prologue stages its operands there.
 struct StepLayout {
-  uint32_t ring, bO, bC, bU, bH, bQ, scr, red, bar, total;
+  uint32_t ring, bO, bC, bU, bH, bQ, scr, red, cw, bar, total;
 };
 
-__host__ __device__ inline StepLayout step_layout(int d, int rd, int M, int nring) {
+// Split partials merged in the step: at most kMaxItems items per query row.
+// For query row (t, j) of the CTA: cw_g[q][w] = partial row of item w (this
+// row of it), cw_f[q][w] = its weight 2^(m_w - m) / L, cw_n[q] = items.  With
+// more items per row the merge reads more partial rows than the separate
+// combine kernel (spread over every SM) takes to read and merge them, so the
+// host keeps that kernel then.
+constexpr int kMaxItems = 2;
+
+__host__ __device__ inline StepLayout step_layout(int d, int rd, int M, int h, int nring) {
   StepLayout L;
   L.ring = 0;
   L.bO = L.ring + nring * kATile;
@@ -178,7 +189,9 @@ __host__ __device__ inline StepLayout step_layout(int d, int rd, int M, int nrin
   L.bQ = L.bH + (rd / 64) * kBTile;
   L.scr = L.bQ + (d / 64) * kBTile;
   L.red = L.scr + kTgt * d * 4;
-  L.bar = L.red + 2 * 2 * 4 * 8 * 4;             // [2 stats][2 halves][4 quarters][8 targets]
+  L.cw = L.red + 2 * 2 * 4 * 8 * 4;              // [2 stats][2 halves][4 quarters][8 targets]
+  L.bar = L.cw + kTgt * h * (kMaxItems * 8 + 4);
+  L.bar = (L.bar + 7) & ~7u;
   L.total = L.bar + (2 * kMaxRing + 4) * 8 + 16;
   return L;
 }
@@ -233,7 +246,7 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_tc_kernel(const StepTcAr
                                            ~static_cast<uintptr_t>(1023));
   const int d = a.d, h = a.h, dh = a.dh, rd = a.rd, L = a.layer;
   const int R = a.nring;
-  const StepLayout Y = step_layout(d, rd, a.M, R);
+  const StepLayout Y = step_layout(d, rd, a.M, h, R);
   uint64_t* full = reinterpret_cast<uint64_t*>(sm + Y.bar);
   uint64_t* empty = full + R;
   uint64_t* bready = empty + R;   // the workers have written a product's B operand
@@ -328,6 +341,49 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_tc_kernel(const StepTcAr
     float* red = reinterpret_cast<float*>(sm + Y.red);
     const int M = a.M;
     bool ok = true;
+    const int nq = kTgt * h;                  // query rows of this CTA
+    int32_t* cw_g = reinterpret_cast<int32_t*>(sm + Y.cw);
+    float* cw_f = reinterpret_cast<float*>(cw_g + nq * kMaxItems);
+    int32_t* cw_n = reinterpret_cast<int32_t*>(cw_f + nq * kMaxItems);
+    if (L >= 0 && a.cmerged == nullptr) {
+      // split combine of Eq. (13)'s alpha_j X~: c_j = sum_w 2^(m_w - m) acc_w / L,
+      // L = sum_w 2^(m_w - m) l_w, over the items w that cover query row (t, j)
+      for (int qi = tid; qi < nq; qi += 32 * kWorkers) {
+        const int t = qi / h, j = qi - t * h;
+        int n = 0;
+        if (t < nb) {
+          const StepPlan& P = a.plan;
+          const int r = P.treq[t0 + t];
+          const int64_t qrow = (t0 + t - P.toff[r]) * h + j;
+          const int64_t mt = qrow / P.mtile_rows, row = qrow - mt * P.mtile_rows;
+          const int pair = P.req_pair_begin[r] + static_cast<int>(mt);
+          const int w0 = P.pair_item_begin[pair];
+          n = P.pair_item_begin[pair + 1] - w0;
+          float mw[kMaxItems], lw[kMaxItems], mx = -INFINITY;
+#pragma unroll
+          for (int w = 0; w < kMaxItems; ++w)
+            if (w < n) {
+              const int64_t g = P.items[w0 + w].row_base + row;
+              cw_g[qi * kMaxItems + w] = static_cast<int32_t>(g);
+              mw[w] = a.pm[g];
+              lw[w] = a.pl[g];
+              mx = fmaxf(mx, mw[w]);
+            }
+          float ls = 0.f;
+#pragma unroll
+          for (int w = 0; w < kMaxItems; ++w)
+            if (w < n) {
+              mw[w] = exp2f(mw[w] - mx);
+              ls = fmaf(lw[w], mw[w], ls);
+            }
+#pragma unroll
+          for (int w = 0; w < kMaxItems; ++w)
+            if (w < n) cw_f[qi * kMaxItems + w] = mw[w] / ls;
+        }
+        cw_n[qi] = n;
+      }
+      workers_sync();
+    }
     // ---- prologue: the B operand of the launch's first product
     if (L < 0) {
       for (int e = tid; e < kTgt * d; e += 32 * kWorkers) {
@@ -378,7 +434,7 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_tc_kernel(const StepTcAr
       const int nc = kTgt * h * (kch / 4), nw = kch * d / 8;
       // the items of this thread are the same in every chunk: their source
       // offsets (at k0 = 0) and destinations, once; -1 marks no item
-      int c_src[kMaxC], c_dst[kMaxC], w_src[kMaxW], w_dst[kMaxW];
+      int c_src[kMaxC], c_dst[kMaxC], c_q[kMaxC], c_k[kMaxC], w_src[kMaxW], w_dst[kMaxW];
 #pragma unroll
       for (int i = 0; i < kMaxC; ++i) {
         const int e = tid + i * 32 * kWorkers;
@@ -386,7 +442,10 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_tc_kernel(const StepTcAr
         const int j = rest % h, k4 = rest / h;
         c_dst[i] = e < nc ? (j * kch + 4 * k4) * kTgt + t : -1;
         c_src[i] = e < nc && t < nb ? (t * h + j) * d + 4 * k4 : -1;   // from this CTA's rows
+        c_q[i] = t * h + j;                                            // its query row
+        c_k[i] = 4 * k4;
       }
+      const bool fused = a.cmerged == nullptr;
 #pragma unroll
       for (int i = 0; i < kMaxW; ++i) {
         const int e = tid + i * 32 * kWorkers;
@@ -394,14 +453,31 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_tc_kernel(const StepTcAr
         w_src[i] = e < nw ? k * d + 8 * c8 : -1;
         w_dst[i] = w_src[i];
       }
-      const float* cm = a.cmerged + t0 * h * d;
+      const float* cm = fused ? nullptr : a.cmerged + t0 * h * d;
       for (int k0 = 0; k0 < d; k0 += kch) {
         float4 cv[kMaxC];
         uint4 wv[kMaxW];
 #pragma unroll
         for (int i = 0; i < kMaxC; ++i) {
           cv[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-          if (c_src[i] >= 0) cv[i] = __ldg(reinterpret_cast<const float4*>(cm + c_src[i] + k0));
+          if (c_src[i] < 0) continue;
+          if (!fused) {
+            cv[i] = __ldg(reinterpret_cast<const float4*>(cm + c_src[i] + k0));
+          } else {
+            const int q = c_q[i], n = cw_n[q];
+            const int koff = c_k[i] + k0;
+#pragma unroll
+            for (int w = 0; w < kMaxItems; ++w)
+              if (w < n) {
+                const float f = cw_f[q * kMaxItems + w];
+                const float4 v = __ldg(reinterpret_cast<const float4*>(
+                    a.pacc + static_cast<int64_t>(cw_g[q * kMaxItems + w]) * d + koff));
+                cv[i].x = fmaf(f, v.x, cv[i].x);
+                cv[i].y = fmaf(f, v.y, cv[i].y);
+                cv[i].z = fmaf(f, v.z, cv[i].z);
+                cv[i].w = fmaf(f, v.w, cv[i].w);
+              }
+          }
         }
 #pragma unroll
         for (int i = 0; i < kMaxW; ++i)
@@ -614,8 +690,11 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_tc_kernel(const StepTcAr
 // layer < 0: q(1) and its u; 0 <= layer < M-1: output of layer `layer`, then
 // q(layer+2) and its u; layer = M-1: output only.  Writes the bf16 query rows
 // scaled by log2(e) / sqrt(d_h) (the tensor-core attention's units).
+int step_tc_max_items() { return kMaxItems; }
+
 int launch_step_tc(const stca_handle* H, int layer, const void* targets, int64_t T,
-                   const float* cmerged, float* Z, uint16_t* Ubf, cudaStream_t s) {
+                   const float* cmerged, const StepPlan* plan, const float* part, int64_t G,
+                   float* Z, uint16_t* Ubf, cudaStream_t s) {
   if (T <= 0) return STCA_OK;
   if (!H->step_tc_ready) return set_error(STCA_ESTATE, "tensor-core step weights are not set up");
   const int M = H->M;
@@ -625,6 +704,14 @@ int launch_step_tc(const stca_handle* H, int layer, const void* targets, int64_t
   a.T = T;
   a.targets = static_cast<const uint16_t*>(targets);
   a.cmerged = cmerged;
+  if (layer >= 0 && cmerged == nullptr) {
+    if (!plan || !part || G >= (int64_t(1) << 31))
+      return set_error(STCA_EINVAL, "tensor-core step: no split partials to merge");
+    a.plan = *plan;
+    a.pacc = part;
+    a.pm = part + G * H->d;
+    a.pl = a.pm + G;
+  }
   a.Z = Z;
   a.Ubf = Ubf;
   a.tiles = H->wstep_tc;
@@ -650,8 +737,8 @@ int launch_step_tc(const stca_handle* H, int layer, const void* targets, int64_t
   // the deepest ring that fits, and the widest W_V staging chunk that fits
   // in the buffers it borrows
   int nring = kMaxRing;
-  while (nring > 2 && step_layout(H->d, H->rd, M, nring).total + 1024 > 227u * 1024) --nring;
-  const StepLayout Y = step_layout(H->d, H->rd, M, nring);
+  while (nring > 2 && step_layout(H->d, H->rd, M, H->h, nring).total + 1024 > 227u * 1024) --nring;
+  const StepLayout Y = step_layout(H->d, H->rd, M, H->h, nring);
   if (Y.total + 1024 > 227u * 1024) return set_error(STCA_EINVAL, "tensor-core step: shared memory");
   // the W_V staging loads at most 8 float4 of c_j and 4 x 16 bytes of W_V per
   // worker thread and chunk
