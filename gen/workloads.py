@@ -208,6 +208,13 @@ def make_workload(*, lengths, targets, d, h, M, r, dtype="bf16", seed=0,
         W["qWd"] = [_xavier(rng, rd, d) for _ in range(M)]
         W["q_ln_g"] = rng.uniform(0.5, 1.5, size=d).astype(np.float32)
         W["q_ln_b"] = rng.uniform(-0.5, 0.5, size=d).astype(np.float32)
+    # prediction-head weights of Eq. (9), from a stream of their own so that
+    # the draws above do not depend on them
+    hrng = np.random.default_rng([seed, 9])
+    W["Wz"] = _xavier(hrng, (M + 1) * d, d)
+    W["zWu"] = _xavier(hrng, d, rd)
+    W["zWg"] = _xavier(hrng, d, rd)
+    W["zWd"] = _xavier(hrng, rd, d)
     if dtype == "bf16":
         X = round_to_bf16(X)
         xt = round_to_bf16(xt)

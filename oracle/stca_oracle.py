@@ -38,6 +38,9 @@ Readings taken where the pages are silent or garbled:
   O10 A request with an empty history is rejected (softmax over no keys is
       undefined); a request with no targets produces no rows.
   O11 The output per target is Z_H = [o^(1); ...; o^(M)] (Eq. (8)), M x d.
+  O12 The prediction-head token z of Eq. (9) is a separate output, computed
+      from Z_H and x_t; its SwiGLU FFN has weights of its own (zW_u, zW_g,
+      zW_d), not shared with the history or query FFNs.
 """
 from __future__ import annotations
 
@@ -177,6 +180,23 @@ def query_fusion(outs: Sequence[np.ndarray], xt, W, i_next):
     """
     cat = np.concatenate([_f64(o) for o in outs] + [_f64(xt)], axis=-1)
     return swiglu_ffn(cat @ _f64(W["Wc"][i_next]), *_query_ffn(W, i_next))
+
+
+def prediction_head(outs: Sequence[np.ndarray], xt, W):
+    """z = SwiGLUFFN([o^(1) || ... || o^(M) || x_t] W_Z), W_Z of (M+1)d x d.
+
+    [digest] §2.1 Eq. (9) (the prediction head).  The head's SwiGLU FFN has
+    weights of its own, zW_u, zW_g (d x rd) and zW_d (rd x d) (reading O12);
+    as in Eq. (7), no LayerNorm (O5) and the raw x_t as the last block (O8).
+    """
+    cat = np.concatenate([_f64(o) for o in outs] + [_f64(xt)], axis=-1)
+    return swiglu_ffn(cat @ _f64(W["Wz"]), _f64(W["zWu"]), _f64(W["zWg"]), _f64(W["zWd"]))
+
+
+def head_from_outputs(Z, targets, W):
+    """z (T, d) of Eq. (9) for every target, from Z (T, M, d) of Eq. (8)."""
+    Z = _f64(Z)
+    return prediction_head([Z[:, i, :] for i in range(Z.shape[1])], targets, W)
 
 
 # --------------------------------------------------------------------------

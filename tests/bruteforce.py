@@ -100,3 +100,14 @@ def forward_request(X, xt, W, h):
                 q = _ffn(_vecmat(cat, Wl["Wc"][i + 1]), *qffn(i + 1))
         Z.append(outs)
     return Z
+
+
+def prediction_head(outs, xt, W):
+    """z of Eq. (9) for one target: outs = [o(1), ..., o(M)] (lists of d),
+    xt (d); the head's FFN weights zWu, zWg, zWd and W_Z ((M+1) d x d)."""
+    cat = []
+    for o in outs:
+        cat += [float(v) for v in o]
+    cat += [float(v) for v in xt]
+    y = _vecmat(cat, _tolist(W["Wz"]))
+    return _ffn(y, _tolist(W["zWu"]), _tolist(W["zWg"]), _tolist(W["zWd"]))

@@ -153,3 +153,62 @@ def test_pins_reject_mutant(name, monkeypatch):
         fn = chained
     monkeypatch.setattr(O, attr, fn)
     assert pins_reject(), f"mutant not caught: {name}"
+
+
+
+# ------------------------------------------------------------ prediction head, Eq. (9)
+
+def head_pins_reject():
+    """True when a head pin fails: brute force on tiny cases, the PyTorch cross-check."""
+    for seed, M in ((31, 1), (32, 3)):
+        wl = make_workload(lengths=[3], targets=[2], d=4, h=2, M=M, r=2, dtype="f32", seed=seed)
+        Z = O.forward_request(wl.X, wl.targets, wl.weights, wl.h)
+        z = O.head_from_outputs(Z, wl.targets, wl.weights)
+        bf = np.array([bruteforce.prediction_head([Z[t, i] for i in range(M)], wl.targets[t],
+                                                  wl.weights) for t in range(2)])
+        if z.shape != bf.shape or _rel(z, bf) > 1e-10:
+            return True
+    wl = make_workload(lengths=[20], targets=[3], d=8, h=2, M=2, r=2, dtype="f32", seed=33)
+    Z = O.forward_request(wl.X, wl.targets, wl.weights, wl.h)
+    if _rel(O.head_from_outputs(Z, wl.targets, wl.weights),
+            torch_reference.prediction_head(Z, wl.targets, wl.weights)) > 1e-10:
+        return True
+    return False
+
+
+def _head_xt_first(outs, xt, W):
+    cat = np.concatenate([_f(xt)] + [_f(o) for o in outs], axis=-1)
+    return O.swiglu_ffn(cat @ _f(W["Wz"]), _f(W["zWu"]), _f(W["zWg"]), _f(W["zWd"]))
+
+
+def _head_last_only(outs, xt, W):
+    d = _f(xt).shape[-1]
+    cat = np.concatenate([_f(outs[-1]), _f(xt)], axis=-1)
+    return O.swiglu_ffn(cat @ _f(W["Wz"])[-2 * d:], _f(W["zWu"]), _f(W["zWg"]), _f(W["zWd"]))
+
+
+def _head_query_ffn(outs, xt, W):
+    cat = np.concatenate([_f(o) for o in outs] + [_f(xt)], axis=-1)
+    return O.swiglu_ffn(cat @ _f(W["Wz"]), _f(W["Wu"][-1]), _f(W["Wg"][-1]), _f(W["Wd"][-1]))
+
+
+def _head_with_ln(outs, xt, W):
+    cat = np.concatenate([_f(o) for o in outs] + [_f(xt)], axis=-1)
+    y = O.swiglu_ffn(cat @ _f(W["Wz"]), _f(W["zWu"]), _f(W["zWg"]), _f(W["zWd"]))
+    d = y.shape[-1]
+    return O.layer_norm(y, np.ones(d), np.zeros(d))
+
+
+HEAD_MUTANTS = {
+    "x_t first in the head concat": _head_xt_first,
+    "head keeps only the last layer's output": _head_last_only,
+    "head reuses the history FFN weights": _head_query_ffn,
+    "head adds a LayerNorm": _head_with_ln,
+}
+
+
+@pytest.mark.parametrize("name", sorted(HEAD_MUTANTS))
+def test_head_pins_reject_mutant(name, monkeypatch):
+    assert not head_pins_reject(), "head pins must accept the unmodified oracle"
+    monkeypatch.setattr(O, "prediction_head", HEAD_MUTANTS[name])
+    assert head_pins_reject(), f"mutant not caught: {name}"

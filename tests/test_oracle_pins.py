@@ -280,3 +280,53 @@ def test_length_flop_model():
         assert r == 4 * 1000 * d * h
         assert n == h * 1000 * (4 * d * dh + 4 * dh)
         assert abs(n / r - dh) < 1e-9 * dh + dh / d
+
+
+# ------------------------------------------------------------ prediction head, Eq. (9)
+
+def _z_of(wl):
+    Z = O.forward_request(wl.X, wl.targets, wl.weights, wl.h)
+    return Z, O.head_from_outputs(Z, wl.targets, wl.weights)
+
+
+@pytest.mark.parametrize("seed,M,r", [(21, 1, 1), (22, 2, 2), (23, 3, 1)])
+def test_head_bruteforce_tiny(seed, M, r):
+    wl = make_workload(lengths=[3], targets=[2], d=4, h=2, M=M, r=r, dtype="f32", seed=seed)
+    Z, z = _z_of(wl)
+    want = np.array([bruteforce.prediction_head([Z[t, i] for i in range(M)], wl.targets[t],
+                                                wl.weights) for t in range(2)])
+    assert z.shape == (2, 4)
+    assert np.abs(z - want).max() <= 1e-12 * max(1.0, np.abs(want).max())
+
+
+def test_head_torch_library_crosscheck():
+    wl = make_workload(lengths=[30], targets=[5], d=16, h=4, M=3, r=2, dtype="f32", seed=24)
+    Z, z = _z_of(wl)
+    want = torch_reference.prediction_head(Z, wl.targets, wl.weights)
+    assert np.abs(z - want).max() <= 1e-12 * np.abs(want).max()
+
+
+def test_head_block_order():
+    # W_Z with one nonzero row block: z then depends on that block's input alone.
+    # Blocks are o(1), ..., o(M), then x_t (Eq. (9)).
+    wl = make_workload(lengths=[10], targets=[3], d=8, h=2, M=3, r=1, dtype="f32", seed=25)
+    d, M = 8, 3
+    Z, _ = _z_of(wl)
+    rng = np.random.default_rng(0)
+    for blk in range(M + 1):
+        W = dict(wl.weights)
+        Wz = np.zeros_like(np.asarray(W["Wz"], dtype=np.float64))
+        Wz[blk * d:(blk + 1) * d] = np.asarray(wl.weights["Wz"])[blk * d:(blk + 1) * d]
+        W["Wz"] = Wz
+        base = O.head_from_outputs(Z, wl.targets, W)
+        for other in range(M + 1):
+            Z2, xt2 = Z.copy(), np.array(wl.targets, dtype=np.float64)
+            if other < M:
+                Z2[:, other] += rng.standard_normal((3, d))
+            else:
+                xt2 += rng.standard_normal((3, d))
+            moved = np.abs(O.head_from_outputs(Z2, xt2, W) - base).max()
+            if other == blk:
+                assert moved > 1e-6, (blk, other)
+            else:
+                assert moved == 0.0, (blk, other)

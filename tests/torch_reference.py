@@ -45,3 +45,12 @@ def forward_request(X, xt, W, h, eps=1e-5):
         if i + 1 < M:
             q = ffn(torch.cat(outs + [xt], dim=-1) @ _t(W["Wc"][i + 1]), i + 1, True)
     return torch.stack(outs, dim=1).numpy()
+
+
+def prediction_head(Z, xt, W):
+    """z of Eq. (9) for every target: Z (T, M, d), xt (T, d); F.silu for the gate."""
+    Z, xt = _t(Z), _t(xt)
+    T, M, d = Z.shape
+    cat = torch.cat([Z.reshape(T, M * d), xt], dim=-1)
+    y = cat @ _t(W["Wz"])
+    return (((y @ _t(W["zWu"])) * F.silu(y @ _t(W["zWg"]))) @ _t(W["zWd"])).numpy()
