@@ -74,6 +74,8 @@ def counts(wl):
         "bytes_min": M * N * d * s,
         "bytes_materialised": (2 * M + 1) * N * d * s,
         "io_bytes": T * d * s + T * M * d * 4,
+        # prediction head of Eq. (9): v W_Z, v' [zW_u | zW_g], h zW_d per target
+        "head_flops": T * 2 * ((M + 1) * d * d + 3 * d * rd),
     }
 
 
@@ -401,7 +403,7 @@ def run_ours(args, rank, world, local_rank):
         local_ms = timed_steps(args.steps)
     if world > 1:
         dist.barrier()
-    kt = S.stca_kernel_times(st.handle)
+    kt = {k: v for k, v in S.stca_kernel_times(st.handle).items() if v[1] > 0}
     st.set_option(S.STCA_OPT_TIMING, 0)
     st.status(stream)
     elapsed_ms = max_over_ranks(local_ms, dev)
@@ -438,6 +440,29 @@ def run_ours(args, rank, world, local_rank):
         f1.record(stream)
     torch.cuda.synchronize()
     fwd_ms = f0.elapsed_time(f1) / args.steps
+
+    # ---- prediction-head token of Eq. (9) on the forward's Z (outside the step)
+    zout = torch.empty((wl.T, wl.d), dtype=torch.float32, device=dev)
+    h0, h1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        st.forward(xt, wl.target_offsets, Z, stream)
+        for _ in range(3):
+            st.head(xt, Z, zout, stream)
+        h0.record(stream)
+        for _ in range(args.steps):
+            st.head(xt, Z, zout, stream)
+        h1.record(stream)
+    torch.cuda.synchronize()
+    st.status(stream)
+    head_ms = h0.elapsed_time(h1) / args.steps
+    head_peak = 148 * 128 * 2 * 1.965e9 / 1e12
+    head_ach = c["head_flops"] / (head_ms / 1e3) / 1e12
+    head = {"ms_per_head": head_ms, "targets_per_s": world * wl.T / (head_ms / 1e3),
+            "kernel": "head_kernel", "inputs": "Z and weights L2-resident (back-to-back calls)",
+            "roofline": {"bound": "alu", "achieved": head_ach, "peak": head_peak,
+                         "unit": "TFLOP/s", "frac": head_ach / head_peak,
+                         "flops_per_launch": c["head_flops"],
+                         "peak_source": "nominal FP32 FFMA: 148 SMs x 128 lanes x 2 x 1.965 GHz"}}
 
     # ---- end to end through the host-buffer entry point
     Xh = torch.from_numpy(np.ascontiguousarray(wl.storage(wl.X))).pin_memory()
@@ -476,6 +501,7 @@ def run_ours(args, rank, world, local_rank):
         "forward_only": {"ms_per_forward": fwd_ms,
                          "targets_per_s": world * wl.T / (fwd_ms / 1e3),
                          "history_tokens_per_s": world * wl.N / (fwd_ms / 1e3)},
+        "head": head,
         "e2e": e2e,
         "gpu_launches": int(launches_per_step * args.steps),
         "clocks": sampler.summary(),

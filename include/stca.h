@@ -72,6 +72,13 @@ enum {
  *                 NULL field: the query uses the history FFN of that layer
  *   q_ln_gamma, q_ln_beta  optional single pointers (d elements): the LN of
  *                 Eq. (3); NULL: layer 1's ln_gamma / ln_beta
+ *   Wz, zWu, zWg, zWd  optional single pointers: the prediction-head token of
+ *                 Eq. (9) ("Make It Long, Keep It Fast" digest, §2.1, Eq. (9)),
+ *                 z = SwiGLUFFN([o(1) || ... || o(M) || x_t] W_Z), with
+ *                 Wz (M+1)d x d, zWu and zWg d x rd, zWd rd x d.  The head's
+ *                 SwiGLU has weights of its own and no LayerNorm (the pages
+ *                 name no norm there).  All four NULL: stca_head is rejected;
+ *                 some NULL: stca_init fails with STCA_EINVAL.
  * stca_init copies everything; the caller may free its buffers afterwards.
  */
 typedef struct {
@@ -90,6 +97,10 @@ typedef struct {
   const void* const* qWd;
   const void* q_ln_gamma;
   const void* q_ln_beta;
+  const void* Wz;
+  const void* zWu;
+  const void* zWg;
+  const void* zWd;
 } stca_weights;
 
 /*
@@ -139,6 +150,23 @@ int stca_encode(stca_handle* handle, const void* X, const int64_t* offsets,
  */
 int stca_forward(stca_handle* handle, const void* targets, const int64_t* target_offsets,
                  int64_t T, float* Z, void* stream);
+
+/*
+ * Prediction-head token of Eq. (9) ("Make It Long, Keep It Fast" digest,
+ * §2.1, Eq. (9)) for T targets:
+ *   zout[t] = SwiGLUFFN_z([Z[t, 0, :] || ... || Z[t, M-1, :] || x_t] W_Z)
+ * where SwiGLUFFN_z(v) = ((v zWu) * SiLU(v zWg)) zWd with the head weights
+ * given to stca_init.
+ *   targets  device pointer, T x d dtype elements (x_t, the rows given to
+ *            stca_forward)
+ *   Z        device pointer, T x M x d fp32: the output of stca_forward
+ *   zout     device pointer, caller-owned, T x d fp32
+ *   T >= 0 (0 is a no-op).  Needs no stca_encode; asynchronous on `stream`.
+ * Errors: STCA_EINVAL (NULL pointer, T < 0, no head weights in the handle),
+ * STCA_ECUDA.
+ */
+int stca_head(stca_handle* handle, const void* targets, int64_t T, const float* Z,
+              float* zout, void* stream);
 
 /*
  * Copy the encoded history X~(layer+1) of the last stca_encode (N x d, dtype
@@ -229,7 +257,7 @@ int stca_set_option(stca_handle* handle, int option, int64_t value);
 int stca_get_option(stca_handle* handle, int option, int64_t* value);
 
 /* Kernel classes reported by stca_kernel_times. */
-enum { STCA_K_ENCODE = 0, STCA_K_ATTN = 1, STCA_K_STEP = 2, STCA_K_CLASSES = 3 };
+enum { STCA_K_ENCODE = 0, STCA_K_ATTN = 1, STCA_K_STEP = 2, STCA_K_HEAD = 3, STCA_K_CLASSES = 4 };
 
 /*
  * Device time of each kernel class since the previous call, from the CUDA

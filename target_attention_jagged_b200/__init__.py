@@ -22,6 +22,7 @@ from .stca import (  # noqa: F401
     stca_forward_static,
     stca_get_encoded,
     stca_get_option,
+    stca_head,
     stca_kernel_times,
     stca_init,
     stca_last_error,

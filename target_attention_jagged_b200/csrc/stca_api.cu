@@ -167,6 +167,8 @@ extern "C" void stca_destroy(stca_handle* H) {
   cudaDeviceSynchronize();
   cudaFree(H->w32);
   cudaFree(H->wstep);
+  cudaFree(H->wstep_tc);
+  cudaFree(H->whead);
   cudaFree(H->wtc);
   cudaFree(H->xt);
   cudaFree(H->q);
@@ -207,6 +209,9 @@ extern "C" int stca_init(const stca_weights* w, int d, int h, int r, int M, int 
     return set_error(STCA_EINVAL, "q_ln_gamma and q_ln_beta must be given together");
   if ((w->ln_gamma == nullptr) != (w->ln_beta == nullptr))
     return set_error(STCA_EINVAL, "ln_gamma and ln_beta must be given together");
+  const int nhead = (w->Wz != nullptr) + (w->zWu != nullptr) + (w->zWg != nullptr) + (w->zWd != nullptr);
+  if (nhead != 0 && nhead != 4)
+    return set_error(STCA_EINVAL, "Wz, zWu, zWg and zWd must be given together");
 
   stca_handle* H = new (std::nothrow) stca_handle();
   if (!H) return set_error(STCA_ENOMEM, "host allocation failed");
@@ -361,6 +366,18 @@ extern "C" int stca_init(const stca_weights* w, int d, int h, int r, int M, int 
         stca_destroy(H);
         return rc2;
       }
+    }
+  }
+  if (nhead == 4) {
+    std::vector<float> wz, zu, zg, zd;
+    int rc2 = fetch(w->Wz, static_cast<size_t>(M + 1) * d * d, dtype, dev, &wz, "Wz");
+    if (!rc2) rc2 = fetch(w->zWu, static_cast<size_t>(d) * rd, dtype, dev, &zu, "zWu");
+    if (!rc2) rc2 = fetch(w->zWg, static_cast<size_t>(d) * rd, dtype, dev, &zg, "zWg");
+    if (!rc2) rc2 = fetch(w->zWd, static_cast<size_t>(rd) * d, dtype, dev, &zd, "zWd");
+    if (!rc2) rc2 = head_weights_setup(H, wz.data(), zu.data(), zg.data(), zd.data());
+    if (rc2) {
+      stca_destroy(H);
+      return rc2;
     }
   }
   if (dtype == STCA_BF16 && encode_tc_supported(d, rd)) {
@@ -765,6 +782,25 @@ extern "C" int stca_forward(stca_handle* H, const void* targets, const int64_t* 
   return ok();
 }
 
+extern "C" int stca_head(stca_handle* H, const void* targets, int64_t T, const float* Z,
+                         float* zout, void* stream) {
+  if (!H) return set_error(STCA_EINVAL, "handle is NULL");
+  if (!H->whead) return set_error(STCA_EINVAL, "stca_head: the handle has no head weights (Wz, zWu, zWg, zWd)");
+  if (T < 0) return set_error(STCA_EINVAL, "T must be >= 0");
+  if (T == 0) return ok();
+  if (!targets || !Z || !zout) return set_error(STCA_EINVAL, "stca_head: targets, Z and zout must not be NULL");
+  if (T > (int64_t(1) << 40)) return set_error(STCA_EINVAL, "stca_head: T too large");
+  DeviceGuard g(H->device);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  {
+    TimedLaunch tl(H, STCA_K_HEAD, s);
+    launch_head(H, targets, T, Z, zout, s);
+  }
+  H->launches++;
+  STCA_CUDA_TRY(cudaGetLastError());
+  return ok();
+}
+
 extern "C" int stca_get_encoded(stca_handle* H, int layer, void* dst, void* stream) {
   if (!H) return set_error(STCA_EINVAL, "handle is NULL");
   if (!H->encoded) return set_error(STCA_ESTATE, "no encoded history");
@@ -910,8 +946,8 @@ extern "C" int stca_kernel_times(stca_handle* H, double* ms, int64_t* launches, 
   if (!H) return set_error(STCA_EINVAL, "handle is NULL");
   if (n < 0) return set_error(STCA_EINVAL, "n must be >= 0");
   DeviceGuard g(H->device);
-  double acc[STCA_K_CLASSES] = {0, 0, 0};
-  int64_t cnt[STCA_K_CLASSES] = {0, 0, 0};
+  double acc[STCA_K_CLASSES] = {};
+  int64_t cnt[STCA_K_CLASSES] = {};
   int rc = STCA_OK;
   for (auto& t : H->timed) {
     float v = 0.f;

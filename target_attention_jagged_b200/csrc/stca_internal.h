@@ -99,6 +99,8 @@ struct stca_handle {
   uint16_t* wstep_tc = nullptr;         // A-tile stream of the tensor-core per-target step
   std::vector<stca::TcGemm> tcO, tcC, tcUG, tcD, tcQ;   // per layer
   bool step_tc_ready = false;
+  void* whead = nullptr;                // prediction-head weights (dtype): Wz, [zWu | zWg], zWd
+  const void *hWz = nullptr, *hWug = nullptr, *hWd = nullptr;
   int num_sms = 148;
 
   // options
@@ -169,6 +171,11 @@ void launch_target_step(const stca_handle* H, int layer, const void* targets, in
                         const StepPlan& plan, const float* cmerged, float* Z, cudaStream_t s);
 size_t target_step_smem(const stca_handle* H);
 int step_weights_setup(stca_handle* H, const std::vector<StepHostW>& layers);
+// Prediction head of Eq. (9): host fp32 Wz ((M+1)d x d), zWu, zWg (d x rd), zWd (rd x d).
+int head_weights_setup(stca_handle* H, const float* Wz, const float* zWu, const float* zWg,
+                       const float* zWd);
+void launch_head(const stca_handle* H, const void* targets, int64_t T, const float* Z, float* zout,
+                 cudaStream_t s);
 size_t attn_simt_smem(const stca_handle* H);
 
 // Tensor-core per-target step (step_tc.cu)

@@ -3,7 +3,9 @@
 //   output          o = [c_1 W_V^1 || ... || c_h W_V^h] W_O; Z[t, i, :] = o   (Eqs. (6), (8))
 //   query fusion    q = SwiGLUFFN_{i+1}([o(1) || ... || o(i+1) || x_t] W_C)  (Eq. (7))
 //   u projection    u_j = (q W_Q^j) W_K^j^T, scaled for the next attention     (Eq. (13))
-// and, before the first layer, q(1) = LN(SwiGLUFFN_1(x_t)) (Eq. (3)) and its u.
+// and, before the first layer, q(1) = LN(SwiGLUFFN_1(x_t)) (Eq. (3)) and its u;
+// after the last layer, optionally, the prediction-head token
+//   z = SwiGLUFFN_z([o(1) || ... || o(M) || x_t] W_Z)                         (Eq. (9)).
 // Sources: "Make It Long, Keep It Fast" digest §2.1.
 //
 // A CTA takes kTB targets and runs the whole chain for them with fp32
@@ -401,6 +403,115 @@ __global__ void __launch_bounds__(kThreads) target_step_kernel(StepArgs a) {
   }
 }
 
+// ---------------------------------------------------------------- prediction head
+// z = ((v W_Z) zW_u * SiLU((v W_Z) zW_g)) zW_d with v = [o(1) || ... || o(M) || x_t]
+// (Eq. (9)).  Row t of Z already holds o(1..M) back to back, so v is that row
+// followed by x_t.  Organised like the step: kTB targets per CTA, fp32
+// activations in shared memory, each weight matrix streamed once per CTA.
+struct HeadArgs {
+  int M, d, rd;
+  int64_t T;
+  const void* targets;
+  const float* Z;
+  float* zout;
+  int* status;
+  const void *Wz, *Wug, *Wd;
+  int wa, wb;         // widths of buffers A and B per target
+};
+
+template <bool XBF, typename WT, int kTB>
+__global__ void __launch_bounds__(kThreads) head_kernel(HeadArgs a) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  constexpr int kRing = kStages * kChunk;
+  constexpr int kRed = kTB * 2 * kThreads;
+  unsigned char* wbuf = smem;                                 // weight ring
+  uint64_t* rbar = reinterpret_cast<uint64_t*>(smem + kRing); // kStages ring mbarriers
+  float* red = reinterpret_cast<float*>(smem + kRing + 128);  // K-split partials
+  float* A = red + kRed;        // kTB x wa: v, then [u | g], then z
+  float* B = A + kTB * a.wa;    // kTB x wb: v W_Z, then u * SiLU(g)
+  const int tid = threadIdx.x;
+  const int d = a.d, rd = a.rd, md = a.M * d, vd = md + d;
+  if (tid == 0) {
+    for (int i = 0; i < kStages; ++i) stca::tc::mbar_init(&rbar[i], 1);
+    stca::tc::fence_mbar_init();
+  }
+  Ring R{wbuf, rbar, a.status, 0};
+  const int64_t t0 = static_cast<int64_t>(blockIdx.x) * kTB;
+  const int nb = a.T - t0 < kTB ? static_cast<int>(a.T - t0) : kTB;
+  for (int e = tid; e < kTB * vd; e += blockDim.x) {
+    const int b = e / vd, k = e - b * vd;
+    float v = 0.f;
+    if (b < nb) v = k < md ? a.Z[(t0 + b) * md + k] : ld_elem<XBF>(a.targets, (t0 + b) * d + k - md);
+    A[b * a.wa + k] = v;
+  }
+  __syncthreads();
+  gemm<WT, kTB>(A, a.wa, d, 0, vd, a.Wz, d, B, a.wb, R, red);
+  gemm<WT, kTB>(B, a.wb, 2 * rd, 0, d, a.Wug, 2 * rd, A, a.wa, R, red);
+  for (int e = tid; e < kTB * rd; e += blockDim.x) {
+    const int b = e / rd, c = e - b * rd;
+    B[b * a.wb + c] = A[b * a.wa + c] * silu_acc(A[b * a.wa + rd + c]);
+  }
+  __syncthreads();
+  gemm<WT, kTB>(B, a.wb, d, 0, rd, a.Wd, d, A, a.wa, R, red);
+  for (int e = tid; e < nb * d; e += blockDim.x) {
+    const int b = e / d, k = e - b * d;
+    a.zout[(t0 + b) * d + k] = A[b * a.wa + k];
+  }
+}
+
+void head_widths(const stca_handle* H, int* wa, int* wb) {
+  *wa = std::max((H->M + 1) * H->d, 2 * H->rd) + 8;
+  *wb = std::max(H->d, H->rd) + 8;
+}
+
+size_t head_smem(const stca_handle* H, int tb) {
+  int wa, wb;
+  head_widths(H, &wa, &wb);
+  return static_cast<size_t>(kStages) * kChunk + 128 +
+         static_cast<size_t>(tb) * 2 * kThreads * sizeof(float) +
+         static_cast<size_t>(tb) * (wa + wb) * sizeof(float);
+}
+
+template <int TB>
+void launch_head_tb(const stca_handle* H, const HeadArgs& a, cudaStream_t s) {
+  const size_t smem = head_smem(H, TB);
+  const unsigned grid = static_cast<unsigned>((a.T + TB - 1) / TB);
+  if (H->elem == 2) {
+    auto k = head_kernel<true, uint16_t, TB>;
+    cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    k<<<grid, kThreads, smem, s>>>(a);
+  } else {
+    auto k = head_kernel<false, float, TB>;
+    cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    k<<<grid, kThreads, smem, s>>>(a);
+  }
+}
+
+// Convert fp32 host values (bf16-exact for bf16 handles) to the handle's
+// element type and copy them to a new device allocation.
+int upload_elems(const stca_handle* H, const std::vector<float>& host, void** dst, const char* what) {
+  const size_t n = host.size();
+  const size_t esz = H->elem == 2 ? 2 : 4;
+  std::vector<unsigned char> bytes(n * esz);
+  if (esz == 2) {
+    uint16_t* out = reinterpret_cast<uint16_t*>(bytes.data());
+    for (size_t k = 0; k < n; ++k) {
+      uint32_t u;
+      memcpy(&u, &host[k], 4);
+      out[k] = static_cast<uint16_t>(u >> 16);
+    }
+  } else {
+    memcpy(bytes.data(), host.data(), n * 4);
+  }
+  if (cudaMalloc(dst, bytes.size()) != cudaSuccess) {
+    cudaGetLastError();
+    *dst = nullptr;
+    return set_error(STCA_ENOMEM, std::string(what) + " weight allocation failed");
+  }
+  STCA_CUDA_TRY(cudaMemcpy(*dst, bytes.data(), bytes.size(), cudaMemcpyHostToDevice));
+  return STCA_OK;
+}
+
 void step_widths(const stca_handle* H, int* wa, int* wb) {
   const int d = H->d;
   *wa = std::max(std::max(H->h * d, H->M * d), 2 * H->rd) + 8;
@@ -527,24 +638,8 @@ int step_weights_setup(stca_handle* H, const std::vector<StepHostW>& layers) {
       }
     o.Wd = put(L.qWd, static_cast<size_t>(rd) * d);
   }
-  const size_t n = host.size();
   const size_t esz = H->elem == 2 ? 2 : 4;
-  std::vector<unsigned char> bytes(n * esz);
-  if (esz == 2) {
-    uint16_t* dst = reinterpret_cast<uint16_t*>(bytes.data());
-    for (size_t k = 0; k < n; ++k) {
-      uint32_t u;
-      memcpy(&u, &host[k], 4);
-      dst[k] = static_cast<uint16_t>(u >> 16);     // values are bf16-exact
-    }
-  } else {
-    memcpy(bytes.data(), host.data(), n * 4);
-  }
-  if (cudaMalloc(&H->wstep, bytes.size()) != cudaSuccess) {
-    cudaGetLastError();
-    return set_error(STCA_ENOMEM, "per-target weight allocation failed");
-  }
-  STCA_CUDA_TRY(cudaMemcpy(H->wstep, bytes.data(), bytes.size(), cudaMemcpyHostToDevice));
+  if (int rc = upload_elems(H, host, &H->wstep, "per-target")) return rc;
   H->Lstep.resize(M);
   const unsigned char* base = static_cast<const unsigned char*>(H->wstep);
   for (int i = 0; i < M; ++i) {
@@ -559,6 +654,54 @@ int step_weights_setup(stca_handle* H, const std::vector<StepHostW>& layers) {
     L.Wd = base + o.Wd * esz;
   }
   return STCA_OK;
+}
+
+// Head weights in the handle's element type: W_Z, [zW_u | zW_g] as one
+// [d x 2rd] matrix, zW_d; each starts on a 64-byte boundary.
+int head_weights_setup(stca_handle* H, const float* Wz, const float* zWu, const float* zWg,
+                       const float* zWd) {
+  const int d = H->d, rd = H->rd;
+  if (head_smem(H, 4) > 227 * 1024)
+    return set_error(STCA_EINVAL, "prediction head needs more than 227 KB shared memory for these sizes");
+  auto pad = [](size_t n) { return (n + 15) & ~size_t(15); };
+  const size_t nz = static_cast<size_t>(H->M + 1) * d * d, nug = static_cast<size_t>(d) * 2 * rd,
+               nd = static_cast<size_t>(rd) * d;
+  const size_t oz = 0, oug = pad(nz), od = oug + pad(nug);
+  std::vector<float> host(od + pad(nd), 0.f);
+  std::copy(Wz, Wz + nz, host.begin() + oz);
+  for (int k = 0; k < d; ++k)
+    for (int c = 0; c < rd; ++c) {
+      host[oug + static_cast<size_t>(k) * 2 * rd + c] = zWu[static_cast<size_t>(k) * rd + c];
+      host[oug + static_cast<size_t>(k) * 2 * rd + rd + c] = zWg[static_cast<size_t>(k) * rd + c];
+    }
+  std::copy(zWd, zWd + nd, host.begin() + od);
+  if (int rc = upload_elems(H, host, &H->whead, "prediction-head")) return rc;
+  const size_t esz = H->elem == 2 ? 2 : 4;
+  const unsigned char* base = static_cast<const unsigned char*>(H->whead);
+  H->hWz = base + oz * esz;
+  H->hWug = base + oug * esz;
+  H->hWd = base + od * esz;
+  return STCA_OK;
+}
+
+// Targets per CTA: 8, else 4.  Four always fit when the step's four-target
+// layout does (stca_init checks that): the head's widths are (M+1)d and
+// max(d, rd) against the step's 2d + max(hd, Md, 2rd) + max(d, rd).
+void launch_head(const stca_handle* H, const void* targets, int64_t T, const float* Z, float* zout,
+                 cudaStream_t s) {
+  if (T <= 0) return;
+  HeadArgs a{};
+  a.M = H->M; a.d = H->d; a.rd = H->rd;
+  a.T = T;
+  a.targets = targets;
+  a.Z = Z;
+  a.zout = zout;
+  a.status = H->status_d;
+  a.Wz = H->hWz; a.Wug = H->hWug; a.Wd = H->hWd;
+  head_widths(H, &a.wa, &a.wb);
+  constexpr size_t kMax = 227 * 1024;
+  if (head_smem(H, 8) <= kMax) launch_head_tb<8>(H, a, s);
+  else launch_head_tb<4>(H, a, s);
 }
 
 }  // namespace stca

@@ -26,14 +26,14 @@ STCA_OK, STCA_EINVAL, STCA_ESTATE, STCA_ENOMEM, STCA_ECUDA, STCA_EDEVICE = 0, -1
 STCA_OPT_ATTN_PATH, STCA_OPT_ENCODE_PATH, STCA_OPT_SPLIT_KEYS, STCA_OPT_TIMING = 1, 2, 3, 4
 STCA_OPT_STEP_PATH = 5
 STCA_OPT_LAUNCHES = 100
-STCA_K_ENCODE, STCA_K_ATTN, STCA_K_STEP, STCA_K_CLASSES = 0, 1, 2, 3
+STCA_K_ENCODE, STCA_K_ATTN, STCA_K_STEP, STCA_K_HEAD, STCA_K_CLASSES = 0, 1, 2, 3, 4
 _NAMES = {STCA_EINVAL: "EINVAL", STCA_ESTATE: "ESTATE", STCA_ENOMEM: "ENOMEM",
           STCA_ECUDA: "ECUDA", STCA_EDEVICE: "EDEVICE"}
 
 EXPORTS = ("stca_init", "stca_destroy", "stca_encode", "stca_forward", "stca_run_host",
            "stca_validate_offsets", "stca_device_status", "stca_set_option",
            "stca_get_option", "stca_kernel_times", "stca_get_encoded", "stca_plan_attention",
-           "stca_forward_static", "stca_last_error")
+           "stca_forward_static", "stca_head", "stca_last_error")
 
 
 class StcaError(RuntimeError):
@@ -55,6 +55,7 @@ def _load():
     lib.stca_encode.argtypes = [P, P, PI64, I64, I64, P]
     lib.stca_forward.argtypes = [P, P, PI64, I64, P, P]
     lib.stca_forward_static.argtypes = [P, P, PI64, I64, P, P]
+    lib.stca_head.argtypes = [P, P, I64, P, P, P]
     lib.stca_run_host.argtypes = [P, P, PI64, I64, I64, P, PI64, I64, P, P]
     lib.stca_validate_offsets.argtypes = [PI64, I64, I64, I]
     lib.stca_device_status.argtypes = [P, P]
@@ -78,7 +79,8 @@ _lib = _load()
 class _Weights(ctypes.Structure):
     _fields_ = [(n, ctypes.POINTER(ctypes.c_void_p)) for n in (
         "Wu", "Wg", "Wd", "ln_gamma", "ln_beta", "Wq", "Wk", "Wv", "Wo", "Wc",
-        "qWu", "qWg", "qWd")] + [("q_ln_gamma", ctypes.c_void_p), ("q_ln_beta", ctypes.c_void_p)]
+        "qWu", "qWg", "qWd")] + [(n, ctypes.c_void_p) for n in (
+        "q_ln_gamma", "q_ln_beta", "Wz", "zWu", "zWg", "zWd")]
 
 
 def stca_last_error() -> str:
@@ -170,6 +172,9 @@ def stca_init(weights: dict, d: int, h: int, r: int, M: int, dtype: int) -> int:
     w.qWd = arr("qWd", optional=True)
     w.q_ln_gamma = _host_buffer(weights["q_ln_g"], dtype, keep) if weights.get("q_ln_g") is not None else None
     w.q_ln_beta = _host_buffer(weights["q_ln_b"], dtype, keep) if weights.get("q_ln_b") is not None else None
+    for k in ("Wz", "zWu", "zWg", "zWd"):     # optional prediction head (Eq. (9))
+        if weights.get(k) is not None:
+            setattr(w, k, _host_buffer(weights[k], dtype, keep))
     out = ctypes.c_void_p()
     _check(_lib.stca_init(ctypes.byref(w), d, h, r, M, dtype, 0, ctypes.byref(out)))
     return out.value
@@ -210,6 +215,20 @@ def stca_forward_static(handle: int, targets, target_offsets, Z, stream=None):
     _check(_lib.stca_forward_static(handle, targets.data_ptr() if T > 0 else None, _i64p(toff),
                                     T, Z.data_ptr() if T > 0 else None, _stream_ptr(stream)))
     return Z
+
+
+def stca_head(handle: int, targets, Z, zout, stream=None):
+    """Prediction-head token of Eq. (9): zout (T x d fp32 CUDA) from Z (T x M x d
+    fp32 CUDA, the forward's output) and targets (T x d CUDA, handle dtype)."""
+    import torch
+    T = int(Z.shape[0])
+    assert Z.dtype == torch.float32 and Z.is_cuda and Z.is_contiguous()
+    assert zout.dtype == torch.float32 and zout.is_cuda and zout.is_contiguous()
+    assert targets.is_contiguous() and int(targets.shape[0]) == T and int(zout.shape[0]) == T
+    _check(_lib.stca_head(handle, targets.data_ptr() if T > 0 else None, T,
+                          Z.data_ptr() if T > 0 else None, zout.data_ptr() if T > 0 else None,
+                          _stream_ptr(stream)))
+    return zout
 
 
 def stca_run_host(handle: int, X_host, offsets, targets_host, target_offsets, Z_host,
@@ -275,7 +294,7 @@ def stca_kernel_times(handle: int):
     ms = (ctypes.c_double * STCA_K_CLASSES)()
     n = (ctypes.c_int64 * STCA_K_CLASSES)()
     _check(_lib.stca_kernel_times(handle, ms, n, STCA_K_CLASSES))
-    names = ("encode", "attention", "target_step")
+    names = ("encode", "attention", "target_step", "head")
     return {names[c]: (ms[c], n[c]) for c in range(STCA_K_CLASSES)}
 
 
@@ -296,6 +315,13 @@ class Stca:
         if Z is None:
             Z = torch.empty((T, self.M, self.d), dtype=torch.float32, device=targets.device)
         return stca_forward(self.handle, targets, target_offsets, Z, stream)
+
+    def head(self, targets, Z, zout=None, stream=None):
+        """z of Eq. (9) for every target: (T, d) fp32."""
+        import torch
+        if zout is None:
+            zout = torch.empty((int(Z.shape[0]), self.d), dtype=torch.float32, device=Z.device)
+        return stca_head(self.handle, targets, Z, zout, stream)
 
     def set_option(self, option: int, value: int):
         stca_set_option(self.handle, option, value)

@@ -105,7 +105,21 @@ def test_null_handle_calls_fail_cleanly():
     v = ctypes.c_int64()
     assert lib.stca_get_option(None, 1, ctypes.byref(v)) == B.STCA_EINVAL
     assert lib.stca_device_status(None, None) == B.STCA_EINVAL
+    assert lib.stca_head(None, None, 4, None, None, None) == B.STCA_EINVAL
     lib.stca_destroy(None)   # accepted
+
+
+@pytest.mark.parametrize("given", [("Wz",), ("Wz", "zWu", "zWg"), ("zWd",)])
+def test_init_rejects_partial_head_weights_on_host(given):
+    # the four prediction-head matrices of Eq. (9) come together or not at all
+    d, r, M = 8, 1, 1
+    w = _weights(d, r, M)
+    shapes = {"Wz": ((M + 1) * d, d), "zWu": (d, r * d), "zWg": (d, r * d), "zWd": (r * d, d)}
+    for k in given:
+        w[k] = np.ones(shapes[k], dtype=np.float32)
+    with pytest.raises(S.StcaError) as e:
+        B.stca_init(w, d, 2, r, M, S.STCA_F32)
+    assert e.value.code == B.STCA_EINVAL and "together" in str(e.value)
 
 
 def test_weight_dtype_checked_by_binding():
