@@ -6,11 +6,14 @@ none of the method's arithmetic: no encoding, no attention, no fusion.
 """
 from .workloads import (  # noqa: F401
     CONFIGS,
+    TRAIN_BATCH,
+    TrainingHistories,
     Workload,
     bf16_bits_to_f32,
     config_shapes,
     f32_to_bf16_bits,
     make_config_workload,
+    make_training_histories,
     make_workload,
     round_to_bf16,
 )

@@ -230,6 +230,48 @@ def make_workload(*, lengths, targets, d, h, M, r, dtype="bf16", seed=0,
                     X=X, targets=xt, weights=W)
 
 
+# A sparse-training batch ("Make It Long, Keep It Fast" digest §2.3; STCA blog
+# §2.6, §3.3): full histories cut to L_infer = 10k at inference, trained at an
+# average length of 2k (SS = 20%) with L_max = L_infer, the U-shaped Beta
+# curriculum of alpha = 0.02, 8 targets per user (request-level batching,
+# m = 8), and the recommended 4-layer, d = 256, h = 8, r = 4 encoder.  The
+# full-history lengths and L_min are not given on the pages: lognormal with
+# mean 6000 clipped to [100, 20000], and L_min = 64.
+TRAIN_BATCH = dict(name="sparse-train-B256-Lavg2000-Lmax10000-a0.02-T8-d256-h8-M4-r4-bf16",
+                   B=256, hist=("lognormal", 6000.0, 0.8, 100, 20000), L_min=64,
+                   L_max=10000, L_avg=2000, L_infer=10000, alpha=0.02, targets=8,
+                   d=256, h=8, M=4, r=4, dtype="bf16", seed=5)
+
+
+@dataclasses.dataclass
+class TrainingHistories:
+    """Full user histories of one training batch and the per-user Beta draws."""
+    hist_lengths: np.ndarray   # B int64
+    hist_offsets: np.ndarray   # B+1 int64
+    s: np.ndarray              # B float64, s_b ~ Beta(alpha, beta)
+    X: np.ndarray              # N x d float32 values (bf16-valued for bf16)
+    dtype: str
+
+    def storage(self, a):
+        return f32_to_bf16_bits(a) if self.dtype == "bf16" else np.ascontiguousarray(a, np.float32)
+
+
+def make_training_histories(*, B, hist, d, alpha, beta, dtype="bf16", seed=0, with_x=True):
+    """Draw, in this order, the B full-history lengths (a length spec as in
+    CONFIGS, or a list), the B Beta(alpha, beta) draws and the N x d history
+    rows (iid N(0, 1)).  beta is the caller's: this module does not derive it."""
+    rng = np.random.default_rng(seed)
+    if isinstance(hist, (list, tuple, np.ndarray)) and (len(hist) == 0 or not isinstance(hist[0], str)):
+        hist = ("list", list(hist))
+    H = _draw_lengths(hist, B, rng)
+    s = rng.beta(alpha, beta, size=B).astype(np.float64)
+    N = int(H.sum())
+    X = rng.standard_normal((N, d), dtype=np.float32) if with_x else np.zeros((0, d), np.float32)
+    if dtype == "bf16":
+        X = round_to_bf16(X)
+    return TrainingHistories(hist_lengths=H, hist_offsets=_offsets(H), s=s, X=X, dtype=dtype)
+
+
 def config_shapes(key: str, seed=None):
     """History lengths and target counts of configuration `key` without drawing
     the embeddings: the same first two draws as make_config_workload."""
