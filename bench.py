@@ -34,7 +34,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
-from gen import CONFIGS, make_config_workload  # noqa: E402
+from gen import CONFIGS, TRAIN_BATCH, make_config_workload, make_training_histories  # noqa: E402
 
 METRIC = "STCA fwd history-tokens/s & targets/s at L=10k; % of HBM/tensor roofline"
 UNIT = "history-tokens/s"
@@ -336,6 +336,74 @@ def roofline_of(kind, kt, c, wl, peaks, sustained, steps, config_key=None):
                 frac=ach / peaks["hbm_gbs"], peak_source="hbm_gbs")
 
 
+def measure_train_batch(S, torch, dev, stream, peaks, steps):
+    """The sparse-training batch builder on its workload (B = 256 users, L_avg =
+    2000, L_max = L_infer = 10000, alpha = 0.02, d = 256 bf16): the host plan,
+    the device gather of the packed stream (HBM-bound: every packed row is read
+    once and written once, plus a 4-byte user index), and the STCA forward
+    (encode + forward, 8 targets per user) over the packed batch."""
+    cfg = TRAIN_BATCH
+    beta, ss = S.stca_sl_beta(cfg["alpha"], cfg["L_min"], cfg["L_max"], cfg["L_avg"])
+    th = make_training_histories(B=cfg["B"], hist=cfg["hist"], d=cfg["d"], alpha=cfg["alpha"],
+                                 beta=beta, dtype=cfg["dtype"], seed=cfg["seed"])
+    X = torch.from_numpy(th.storage(th.X)).view(torch.int16).view(torch.bfloat16).to(dev)
+    args = (cfg["L_min"], cfg["L_max"], cfg["L_avg"], cfg["L_infer"])
+    t0 = time.perf_counter()
+    for _ in range(steps):
+        plan = S.stca_sl_plan(th.hist_offsets, th.s, *args)
+    plan_ms = (time.perf_counter() - t0) * 1e3 / steps
+    P = int(plan["packed_offsets"][-1])
+    src = torch.from_numpy(plan["src_start"]).to(dev)
+    poff = torch.from_numpy(plan["packed_offsets"]).to(dev)
+    Xp = torch.empty((P, cfg["d"]), dtype=torch.bfloat16, device=dev)
+    seg = torch.empty(P, dtype=torch.int32, device=dev)
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            S.stca_sl_gather(X, src, poff, Xp, seg, stream)
+        evs = []
+        for _ in range(steps):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            S.stca_sl_gather(X, src, poff, Xp, seg, stream)
+            b.record(stream)
+            evs.append((a, b))
+    torch.cuda.synchronize()
+    g_ms = statistics.median(a.elapsed_time(b) for a, b in evs)
+    nbytes = 2 * P * cfg["d"] * 2 + 4 * P
+    ach = nbytes / (g_ms / 1e3) / 1e9
+    # the forward over the packed batch
+    from gen import make_workload
+    wl = make_workload(lengths=plan["lengths"].tolist(), targets=[cfg["targets"]] * cfg["B"],
+                       d=cfg["d"], h=cfg["h"], M=cfg["M"], r=cfg["r"], dtype="bf16",
+                       seed=cfg["seed"], name=cfg["name"])
+    st = S.Stca(storage_weights(wl), wl.d, wl.h, wl.r, wl.M, wl.dtype)
+    xt = to_dev(wl, wl.targets, dev)
+    Z = torch.empty((wl.T, wl.M, wl.d), dtype=torch.float32, device=dev)
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            st.encode(Xp, plan["packed_offsets"], stream)
+            st.forward(xt, wl.target_offsets, Z, stream)
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        f0.record(stream)
+        for _ in range(steps):
+            S.stca_sl_gather(X, src, poff, Xp, seg, stream)
+            st.encode(Xp, plan["packed_offsets"], stream)
+            st.forward(xt, wl.target_offsets, Z, stream)
+        f1.record(stream)
+    torch.cuda.synchronize()
+    st.status(stream)
+    st.close()
+    step_ms = f0.elapsed_time(f1) / steps
+    return {"workload": cfg["name"], "users": cfg["B"], "packed_rows": P,
+            "sequence_sparsity": ss, "beta": beta, "plan_ms_host": plan_ms,
+            "gather": {"ms": g_ms, "kernel": "sl_gather_kernel",
+                       "roofline": {"bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"],
+                                    "unit": "GB/s", "frac": ach / peaks["hbm_gbs"],
+                                    "bytes_per_launch": nbytes, "peak_source": "hbm_gbs"}},
+            "gather_encode_forward": {"ms": step_ms, "history_tokens_per_s": P / (step_ms / 1e3),
+                                      "targets_per_s": wl.T / (step_ms / 1e3)}}
+
+
 def run_ours(args, rank, world, local_rank):
     import torch
     import torch.distributed as dist
@@ -464,6 +532,11 @@ def run_ours(args, rank, world, local_rank):
                          "flops_per_launch": c["head_flops"],
                          "peak_source": "nominal FP32 FFMA: 148 SMs x 128 lanes x 2 x 1.965 GHz"}}
 
+    # ---- the sparse-training batch builder and a forward over its packed batch
+    train_batch = None
+    if not args.no_train_batch:
+        train_batch = measure_train_batch(S, torch, dev, stream, peaks, args.steps)
+
     # ---- end to end through the host-buffer entry point
     Xh = torch.from_numpy(np.ascontiguousarray(wl.storage(wl.X))).pin_memory()
     th = torch.from_numpy(np.ascontiguousarray(wl.storage(wl.targets))).pin_memory()
@@ -502,6 +575,7 @@ def run_ours(args, rank, world, local_rank):
                          "targets_per_s": world * wl.T / (fwd_ms / 1e3),
                          "history_tokens_per_s": world * wl.N / (fwd_ms / 1e3)},
         "head": head,
+        "train_batch": train_batch,
         "e2e": e2e,
         "gpu_launches": int(launches_per_step * args.steps),
         "clocks": sampler.summary(),
@@ -521,6 +595,8 @@ def main():
     ap.add_argument("--config", default="c3", choices=sorted(CONFIGS))
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-train-batch", action="store_true",
+                    help="skip the sparse-training batch builder measurement")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -243,6 +243,69 @@ int stca_plan_attention(const int64_t* offsets, const int64_t* target_offsets, i
  */
 int stca_device_status(stca_handle* handle, void* stream);
 
+/* ------------------------------------------------------------------------
+ * Sparse-training batch builder ("Make It Long, Keep It Fast" digest, §2.3
+ * "Extrapolation: Train Sparsely, Infer Densely"; STCA blog, §2.6): per-user
+ * training lengths from the stochastic length curriculum, the temporal-suffix
+ * selection, and the two-step batch-level load balance, producing the packed,
+ * padding-free history stream and offsets that stca_encode takes.  Random
+ * numbers are the caller's: it draws s_b ~ Beta(alpha, beta).
+ * ------------------------------------------------------------------------ */
+
+/*
+ * Eq. (17): *beta = alpha (L_max - L_avg) / (L_avg - L_min), the Beta shape
+ * that makes the mean of Eq. (16)'s L_raw equal L_avg; Eq. (15): *ss (may be
+ * NULL) = L_avg / L_max, the sequence sparsity.  Host only.
+ * Errors: STCA_EINVAL unless alpha > 0 and 0 <= L_min < L_avg < L_max.
+ */
+int stca_sl_beta(double alpha, int64_t L_min, int64_t L_max, int64_t L_avg, double* beta,
+                 double* ss);
+
+/*
+ * Host only: the packed layout of one training batch of B users.
+ *   hist_offsets  B+1 int64: user b's full history is rows hist_offsets[b] ..
+ *                 hist_offsets[b+1]-1 of X, oldest first; every user has >= 1 row
+ *   s             B doubles in [0, 1]: the user's Beta draw
+ *   L_min, L_max, L_avg   0 <= L_min < L_avg < L_max; L_infer >= 1
+ * For each user: L_raw = L_min + s (L_max - L_min) (Eq. (16), in double, in
+ * that order), aligned down to a multiple of 8 (at least 8), capped by the
+ * usable history min(H_b, L_infer).  Then the batch is brought to exactly
+ * B * L_avg rows: a surplus is removed by keeping one row per user and sharing
+ * the other B * L_avg - B rows in proportion to (length - 1), a shortfall is
+ * filled in proportion to each user's unused usable history, both by the
+ * largest-remainder method (ties to the lower user index); when the usable
+ * histories hold fewer rows than the budget, every user takes all of its own.
+ * Outputs (caller-owned host arrays): train[B] (the aligned Eq. (16) lengths,
+ * may be NULL), lengths[B] (final, each >= 1), packed_offsets[B+1] (prefix
+ * sums of lengths) and src_start[B] = hist_offsets[b+1] - lengths[b] (the
+ * first row of the user's temporal suffix).  Deterministic: the same inputs
+ * give the same integers on every machine.
+ * Errors: STCA_EINVAL (bad offsets, empty history, s outside [0, 1] or not
+ * finite, bad lengths, B < 1, NULL output).
+ */
+int stca_sl_plan(const int64_t* hist_offsets, int64_t B, const double* s, int64_t L_min,
+                 int64_t L_max, int64_t L_avg, int64_t L_infer, int64_t* train, int64_t* lengths,
+                 int64_t* packed_offsets, int64_t* src_start);
+
+/*
+ * Device gather of the packed stream: for user b and 0 <= k < packed_offsets[b+1]
+ * - packed_offsets[b], row packed_offsets[b] + k of X_packed is row
+ * src_start[b] + k of X, copied bit for bit, and seg[packed_offsets[b] + k] = b
+ * (the index tensor of the ragged attention; seg may be NULL).
+ *   X          device, N rows of row_bytes bytes (row_bytes a multiple of 16,
+ *              X and X_packed 16-byte aligned)
+ *   src_start, packed_offsets   DEVICE int64 arrays of B and B+1 entries, as
+ *              stca_sl_plan writes them (caller-owned; the library does not check
+ *              them on the device: every source row must lie in [0, N))
+ *   P          packed rows, packed_offsets[B]
+ *   X_packed   device, P rows of row_bytes (caller-owned); seg: device int32 P
+ * Asynchronous on `stream`.  Errors: STCA_EINVAL (sizes, alignment, NULL),
+ * STCA_ECUDA.
+ */
+int stca_sl_gather(const void* X, int64_t N, int64_t row_bytes, const int64_t* src_start,
+                   const int64_t* packed_offsets, int64_t B, int64_t P, void* X_packed,
+                   int32_t* seg, void* stream);
+
 /* Tunables and introspection (STCA_OPT_*).  Values are validated. */
 enum {
   STCA_OPT_ATTN_PATH = 1,     /* 0 auto, 1 CUDA cores, 2 tensor cores (bf16 only) */

@@ -48,7 +48,9 @@ def build(debug: bool = False, verbose_ptxas: bool = False, force: bool = False)
         return LIB
     objdir = os.path.join(PKG, "_build")
     os.makedirs(objdir, exist_ok=True)
-    flags = ARCH + ["-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC",
+    # -ffp-contract=off: host arithmetic that decides integers (the training
+    # lengths of the batch builder) rounds every operation, as numpy does
+    flags = ARCH + ["-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-Xcompiler", "-ffp-contract=off",
                     "-I", os.path.join(ROOT, "include"), "-I", os.path.join(PKG, "csrc")]
     flags += ["-O0", "-G"] if debug else ["-O3"]
     if verbose_ptxas:

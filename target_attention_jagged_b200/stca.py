@@ -33,7 +33,8 @@ _NAMES = {STCA_EINVAL: "EINVAL", STCA_ESTATE: "ESTATE", STCA_ENOMEM: "ENOMEM",
 EXPORTS = ("stca_init", "stca_destroy", "stca_encode", "stca_forward", "stca_run_host",
            "stca_validate_offsets", "stca_device_status", "stca_set_option",
            "stca_get_option", "stca_kernel_times", "stca_get_encoded", "stca_plan_attention",
-           "stca_forward_static", "stca_head", "stca_last_error")
+           "stca_forward_static", "stca_head", "stca_sl_beta", "stca_sl_plan",
+           "stca_sl_gather", "stca_last_error")
 
 
 class StcaError(RuntimeError):
@@ -56,6 +57,10 @@ def _load():
     lib.stca_forward.argtypes = [P, P, PI64, I64, P, P]
     lib.stca_forward_static.argtypes = [P, P, PI64, I64, P, P]
     lib.stca_head.argtypes = [P, P, I64, P, P, P]
+    D, PD = ctypes.c_double, ctypes.POINTER(ctypes.c_double)
+    lib.stca_sl_beta.argtypes = [D, I64, I64, I64, PD, PD]
+    lib.stca_sl_plan.argtypes = [PI64, I64, PD, I64, I64, I64, I64, PI64, PI64, PI64, PI64]
+    lib.stca_sl_gather.argtypes = [P, I64, I64, P, P, I64, I64, P, P, P]
     lib.stca_run_host.argtypes = [P, P, PI64, I64, I64, P, PI64, I64, P, P]
     lib.stca_validate_offsets.argtypes = [PI64, I64, I64, I]
     lib.stca_device_status.argtypes = [P, P]
@@ -229,6 +234,61 @@ def stca_head(handle: int, targets, Z, zout, stream=None):
                           Z.data_ptr() if T > 0 else None, zout.data_ptr() if T > 0 else None,
                           _stream_ptr(stream)))
     return zout
+
+
+def stca_sl_beta(alpha: float, L_min: int, L_max: int, L_avg: int):
+    """Eq. (17) beta and Eq. (15) sequence sparsity: returns (beta, ss)."""
+    beta, ss = ctypes.c_double(), ctypes.c_double()
+    _check(_lib.stca_sl_beta(alpha, L_min, L_max, L_avg, ctypes.byref(beta), ctypes.byref(ss)))
+    return beta.value, ss.value
+
+
+def stca_sl_plan(hist_offsets, s, L_min: int, L_max: int, L_avg: int, L_infer: int) -> dict:
+    """Host plan of a training batch: int64 arrays train, lengths, packed_offsets, src_start."""
+    off = _offsets(hist_offsets)
+    B = off.shape[0] - 1
+    sd = np.ascontiguousarray(np.asarray(s, dtype=np.float64))
+    if sd.shape != (B,):
+        raise ValueError("one draw per user")
+    out = {k: np.zeros(B + (k == "packed_offsets"), dtype=np.int64)
+           for k in ("train", "lengths", "packed_offsets", "src_start")}
+    _check(_lib.stca_sl_plan(_i64p(off), B, sd.ctypes.data_as(ctypes.POINTER(ctypes.c_double)),
+                             L_min, L_max, L_avg, L_infer, _i64p(out["train"]),
+                             _i64p(out["lengths"]), _i64p(out["packed_offsets"]),
+                             _i64p(out["src_start"])))
+    return out
+
+
+def stca_sl_gather(X, src_start, packed_offsets, X_packed, seg=None, stream=None):
+    """Device gather of the packed stream.  X, X_packed: CUDA tensors (rows x d);
+    src_start, packed_offsets: CUDA int64 tensors (B, B+1); seg: CUDA int32 (P) or None."""
+    import torch
+    assert X.is_cuda and X_packed.is_cuda and X.is_contiguous() and X_packed.is_contiguous()
+    assert src_start.dtype == torch.int64 and packed_offsets.dtype == torch.int64
+    B = int(src_start.shape[0])
+    P = int(X_packed.shape[0])
+    row_bytes = X.element_size() * (X.numel() // max(1, X.shape[0])) if X.shape[0] else \
+        X_packed.element_size() * (X_packed.numel() // max(1, P))
+    _check(_lib.stca_sl_gather(X.data_ptr(), int(X.shape[0]), row_bytes, src_start.data_ptr(),
+                               packed_offsets.data_ptr(), B, P, X_packed.data_ptr(),
+                               seg.data_ptr() if seg is not None else None, _stream_ptr(stream)))
+    return X_packed
+
+
+def build_training_batch(X, hist_offsets, s, L_min: int, L_max: int, L_avg: int, L_infer: int,
+                         stream=None):
+    """Plan (host) and gather (device) one sparse-training batch: returns
+    (X_packed, seg, plan) with plan's packed_offsets the stca_encode offsets."""
+    import torch
+    plan = stca_sl_plan(hist_offsets, s, L_min, L_max, L_avg, L_infer)
+    P = int(plan["packed_offsets"][-1])
+    dev = X.device
+    src = torch.from_numpy(plan["src_start"]).to(dev)
+    poff = torch.from_numpy(plan["packed_offsets"]).to(dev)
+    Xp = torch.empty((P,) + tuple(X.shape[1:]), dtype=X.dtype, device=dev)
+    seg = torch.empty(P, dtype=torch.int32, device=dev)
+    stca_sl_gather(X, src, poff, Xp, seg, stream)
+    return Xp, seg, plan
 
 
 def stca_run_host(handle: int, X_host, offsets, targets_host, target_offsets, Z_host,
