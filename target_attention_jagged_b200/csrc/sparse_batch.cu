@@ -50,10 +50,18 @@ void share_rows(const std::vector<int64_t>& w, int64_t total, std::vector<int64_
 // Packed row p -> its user, then the row copy.  A warp owns a contiguous run
 // of packed rows; it finds the user of its first row by binary search over the
 // packed offsets and walks forward.  Rows move as 16-byte vectors with
-// streaming (evict-first) loads and stores; four rows are in flight per warp
+// streaming (evict-first) loads and stores; eight rows are in flight per warp
 // when a row is at most 32 vectors long.  A source row outside [0, N) is not
 // read: its packed row is left as it was and its seg entry is -1.
 constexpr int kGatherThreads = 256;
+// u[lane] without dynamic register indexing
+template <int N>
+__device__ __forceinline__ int32_t user_sel(const int32_t (&u)[N], int lane) {
+  int32_t r = -1;
+#pragma unroll
+  for (int i = 0; i < N; ++i) r = lane == i ? u[i] : r;
+  return r;
+}
 
 __device__ __forceinline__ int64_t user_of(const int64_t* poff, int64_t B, int64_t p) {
   int64_t lo = 0, hi = B;                 // poff[lo] <= p < poff[hi] when offsets are valid
@@ -78,7 +86,7 @@ __global__ void __launch_bounds__(kGatherThreads) sl_gather_kernel(
   int64_t b = user_of(poff, B, p0);
   int64_t next = b + 1 < B ? __ldg(poff + b + 1) : P;   // first row of the next user
   int64_t base = __ldg(poff + b), src = __ldg(src_start + b);
-  constexpr int kRows = 4;
+  constexpr int kRows = 8;
   for (int64_t p = p0; p < p1; p += kRows) {
     int64_t srow[kRows];
     int32_t user[kRows];
@@ -102,7 +110,7 @@ __global__ void __launch_bounds__(kGatherThreads) sl_gather_kernel(
       }
     }
     if (seg && lane < kRows && p + lane < p1)
-      seg[p + lane] = lane == 0 ? user[0] : lane == 1 ? user[1] : lane == 2 ? user[2] : user[3];
+      seg[p + lane] = user_sel(user, lane);
     for (int c = lane; c < row16; c += 32) {
       uint4 v[kRows];
 #pragma unroll

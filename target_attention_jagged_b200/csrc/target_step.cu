@@ -218,18 +218,20 @@ __device__ __forceinline__ void gemm(const float* in, int ldin, int hc, int hs, 
 // ---------------------------------------------------------------- split combine
 // c_j = sum_w s_w acc_w / sum_w s_w l_w with s_w = e^(m_w - m) (2^ for the
 // tensor-core partials) over the items w that cover query row (t, j): the
-// attention-weighted history alpha_j X~ of Eq. (13).  One CTA per query row;
-// the first warp reads the items' (m, l) with one lane per item.
-constexpr int kCombineThreads = 128;
-constexpr int kCombineMaxItems = 32;
+// attention-weighted history alpha_j X~ of Eq. (13).  One warp per query row,
+// eight rows per CTA: the lanes first read the items' (m, l), one item per
+// lane, and turn them into weights; then each lane owns 4 columns (a float4)
+// of every 128 and sums the items' partial rows, one coalesced 16-byte load
+// per lane and item.
+constexpr int kCombineThreads = 256;
+constexpr int kCombineRows = kCombineThreads / 32;
 
 __global__ void __launch_bounds__(kCombineThreads)
 combine_kernel(StepPlan P, const float* __restrict__ pacc, const float* __restrict__ pm,
-               const float* __restrict__ pl, float* __restrict__ out, int d, int h) {
-  __shared__ int64_t sg[kCombineMaxItems];
-  __shared__ float sf[kCombineMaxItems];
-  __shared__ int s_nw;
-  const int64_t qr = blockIdx.x;          // target t, head j: row t * h + j of U
+               const float* __restrict__ pl, float* __restrict__ out, int d, int h, int64_t nq) {
+  const int lane = threadIdx.x & 31;
+  const int64_t qr = static_cast<int64_t>(blockIdx.x) * kCombineRows + (threadIdx.x >> 5);
+  if (qr >= nq) return;                   // target t, head j: row t * h + j of U
   const int64_t t = qr / h;
   const int j = static_cast<int>(qr - t * h);
   const int r = P.treq[t];
@@ -237,53 +239,51 @@ combine_kernel(StepPlan P, const float* __restrict__ pacc, const float* __restri
   const int64_t mt = qrow / P.mtile_rows;
   const int64_t row = qrow - mt * P.mtile_rows;
   const int pair = P.req_pair_begin[r] + static_cast<int>(mt);
-  const int w0 = P.pair_item_begin[pair], w1 = P.pair_item_begin[pair + 1];
-  const int nw = w1 - w0;
-  const int tid = threadIdx.x;
-  if (nw <= kCombineMaxItems) {
-    if (tid < 32) {
-      int64_t g = 0;
-      float m = -INFINITY, l = 0.f;
-      if (tid < nw) {
-        g = P.items[w0 + tid].row_base + row;
-        m = pm[g];
-        l = pl[g];
-      }
-      float mx = m;
+  const int w0 = P.pair_item_begin[pair], nw = P.pair_item_begin[pair + 1] - w0;
+  // the row's maximum and normaliser over all items, 32 items at a time
+  float mx = -INFINITY;
+  for (int b = 0; b < nw; b += 32)
+    if (b + lane < nw) mx = fmaxf(mx, pm[P.items[w0 + b + lane].row_base + row]);
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-      const float f = tid < nw ? (P.log2_partials ? exp2f(m - mx) : expf(m - mx)) : 0.f;
-      float ls = l * f;
+  for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  float ls = 0.f;
+  for (int b = 0; b < nw; b += 32)
+    if (b + lane < nw) {
+      const int64_t g = P.items[w0 + b + lane].row_base + row;
+      const float m = pm[g];
+      ls = fmaf(pl[g], P.log2_partials ? exp2f(m - mx) : expf(m - mx), ls);
+    }
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) ls += __shfl_xor_sync(0xffffffffu, ls, o);
-      if (tid < nw) {
-        sg[tid] = g;
-        sf[tid] = f / ls;
+  for (int o = 16; o > 0; o >>= 1) ls += __shfl_xor_sync(0xffffffffu, ls, o);
+  const float inv = 1.0f / ls;
+  float* orow = out + qr * d;
+  for (int b = 0; b < nw; b += 32) {
+    // item b + lane: its partial row and weight, handed round the warp below
+    int64_t g = 0;
+    float f = 0.f;
+    if (b + lane < nw) {
+      g = P.items[w0 + b + lane].row_base + row;
+      const float m = pm[g];
+      f = (P.log2_partials ? exp2f(m - mx) : expf(m - mx)) * inv;
+    }
+    const int n = min(32, nw - b);
+    for (int k0 = 0; k0 < d; k0 += 128) {      // the whole warp walks the same k0 (shuffles)
+      const int k = k0 + 4 * lane;
+      const bool on = k < d;
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (on && b > 0) acc = *reinterpret_cast<const float4*>(orow + k);
+      for (int w = 0; w < n; ++w) {
+        const int64_t gw = __shfl_sync(0xffffffffu, g, w);
+        const float fw = __shfl_sync(0xffffffffu, f, w);
+        if (on) {
+          const float4 v = __ldg(reinterpret_cast<const float4*>(pacc + gw * d + k));
+          acc.x = fmaf(fw, v.x, acc.x);
+          acc.y = fmaf(fw, v.y, acc.y);
+          acc.z = fmaf(fw, v.z, acc.z);
+          acc.w = fmaf(fw, v.w, acc.w);
+        }
       }
-      if (tid == 0) s_nw = nw;
-    }
-    __syncthreads();
-    for (int k = tid; k < d; k += kCombineThreads) {
-      float v = 0.f;
-      for (int w = 0; w < s_nw; ++w) v = fmaf(pacc[sg[w] * d + k], sf[w], v);
-      out[qr * d + k] = v;
-    }
-  } else {
-    // many splits of one pair: serial over the items
-    float mx = -INFINITY;
-    for (int w = w0; w < w1; ++w) mx = fmaxf(mx, pm[P.items[w].row_base + row]);
-    float l = 0.f;
-    for (int w = w0; w < w1; ++w) {
-      const int64_t g = P.items[w].row_base + row;
-      l = fmaf(pl[g], P.log2_partials ? exp2f(pm[g] - mx) : expf(pm[g] - mx), l);
-    }
-    for (int k = tid; k < d; k += kCombineThreads) {
-      float v = 0.f;
-      for (int w = w0; w < w1; ++w) {
-        const int64_t g = P.items[w].row_base + row;
-        v = fmaf(pacc[g * d + k], P.log2_partials ? exp2f(pm[g] - mx) : expf(pm[g] - mx), v);
-      }
-      out[qr * d + k] = v / l;
+      if (on) *reinterpret_cast<float4*>(orow + k) = acc;
     }
   }
 }
@@ -578,8 +578,9 @@ void launch_combine(const stca_handle* H, const StepPlan& plan, const float* par
   const float* pacc = part;
   const float* pm = part + G * H->d;
   const float* pl = pm + G;
-  combine_kernel<<<static_cast<unsigned>(T * H->h), kCombineThreads, 0, s>>>(plan, pacc, pm, pl,
-                                                                              out, H->d, H->h);
+  const int64_t nq = T * H->h;
+  combine_kernel<<<static_cast<unsigned>((nq + kCombineRows - 1) / kCombineRows), kCombineThreads, 0,
+                   s>>>(plan, pacc, pm, pl, out, H->d, H->h, nq);
 }
 
 void launch_target_step(const stca_handle* H, int layer, const void* targets, int64_t T,
