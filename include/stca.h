@@ -314,7 +314,16 @@ enum {
   STCA_OPT_TIMING = 4,        /* 1: record CUDA events around every kernel launch */
   STCA_OPT_STEP_PATH = 5,     /* per-target step: 0 auto, 1 CUDA cores, 2 tensor cores (bf16,
                                  d in {128, 256}, r d <= 512, with the tensor-core attention) */
-  STCA_OPT_LAUNCHES = 100     /* read-only: kernels launched since the last encode */
+  STCA_OPT_ATTN_FORM = 6,     /* 0: the reordered single-query form of Eq. (13) (default);
+                                 1: the naive form of Eq. (12) -- K = X~ W_K and V = X~ W_V
+                                 projected once per layer for all targets, then attention per
+                                 head over d_h features (the pages' K/V-cache serving idea);
+                                 2: whichever of the two has fewer FLOPs for the batch.
+                                 The naive form needs the tensor-core step (see above) and
+                                 d_h in {16, 32, 64}; form 1 without them is rejected, form 2
+                                 falls back to the reordered form */
+  STCA_OPT_LAUNCHES = 100,    /* read-only: kernels launched since the last encode */
+  STCA_OPT_LAST_FORM = 101    /* read-only: 1 if the last forward ran the naive form, else 0 */
 };
 int stca_set_option(stca_handle* handle, int option, int64_t value);
 int stca_get_option(stca_handle* handle, int option, int64_t* value);

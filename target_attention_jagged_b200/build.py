@@ -66,7 +66,7 @@ def build(debug: bool = False, verbose_ptxas: bool = False, force: bool = False)
             raise RuntimeError(f"nvcc failed on {src}")
         objs.append(obj)
     tmp = LIB + ".tmp"
-    cmd = [nvcc()] + ARCH + ["-shared", "-o", tmp] + objs + ["-lcuda"]
+    cmd = [nvcc()] + ARCH + ["-shared", "-o", tmp] + objs + ["-lcuda", "-lcublasLt"]
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         sys.stderr.write(r.stdout + r.stderr)

@@ -20,6 +20,12 @@
 // max grows by more than 8 (log2 units); otherwise P uses the stale max and
 // stays below 2^8, well inside bf16 and fp32 range.
 //
+// The naive form (Eq. (12), SEPV) runs the same kernel on projected keys and
+// values: the query rows are q W_Q of G = 64 / d_h heads packed into one tile
+// (each row non-zero only in its own head's d_h features), S contracts the
+// tile's 64 head-group features of K = X~ W_K, and O += P V takes the same 64
+// features of V = X~ W_V from a second shared-memory tile loaded beside K.
+//
 // Warp roles (352 threads): warp 0 TMA, warp 1 issues S (and owns TMEM),
 // warps 2-9 softmax / correction / partial store (one query row per thread,
 // two warps -- key halves -- per row), warp 10 issues P X~.  Two issuers let
@@ -53,16 +59,17 @@ struct AttnParams {
 // through shared memory.  Keeping P out of shared memory matters: the MMAs'
 // operand reads, the TMA writes of X~ and the P writes would otherwise all
 // share its bandwidth.
-template <int D, int QB, int KS, int PB>
+template <int D, int QB, int KS, int PB, bool SEPV>
 struct AttnCfg {
   static constexpr bool P_TMEM = D <= 128;
   static constexpr int KB = D / 64;
   static constexpr uint32_t kBlock = 128u * 128u;       // [128 rows x 64] bf16
   static constexpr uint32_t kTile = KB * kBlock;         // [128 rows x D]
+  static constexpr uint32_t kStage = SEPV ? 2 * kTile : kTile;   // key tile (+ value tile)
   static constexpr uint32_t kPBytes = 2 * kBlock;        // [128 rows x 128 keys]
   static constexpr uint32_t oQ = 0;
   static constexpr uint32_t oK = oQ + QB * kTile;
-  static constexpr uint32_t oP = oK + KS * kTile;
+  static constexpr uint32_t oP = oK + KS * kStage;
   static constexpr uint32_t oX = oP + (P_TMEM ? 0 : PB * kPBytes);   // pair exchange: 2 x 2 x 128 floats
   static constexpr uint32_t oBar = oX + 2 * 2 * 128 * 4;
   static constexpr int kBars = 2 * QB + 2 * KS + 4 + 2 * PB + 3 + 1 + 8;
@@ -135,11 +142,11 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
 }
 
 
-template <int D, int QB, int KS, int PB>
+template <int D, int QB, int KS, int PB, bool SEPV>
 __global__ void __launch_bounds__(kAttnThreads, 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-               const AttnParams p) {
-  using C = AttnCfg<D, QB, KS, PB>;
+               const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
+  using C = AttnCfg<D, QB, KS, PB, SEPV>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   if (smem_u32(smem_raw) & 1023u) {      // the swizzled tiles need 1024-byte alignment
     if (threadIdx.x == 0) atomicOr(p.status, kStatusAttnTimeout);
@@ -180,6 +187,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   if (warp == 0 && lane == 0) {
     prefetch_tmap(&tmQ);
     prefetch_tmap(&tmK);
+    if constexpr (SEPV) prefetch_tmap(&tmV);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, 512);
@@ -210,10 +218,16 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         for (int j = 0; j < nt; ++j) {
           const int s = ki % KS;
           if (!(ok = bwait(&kempty[s], ((ki / KS) & 1) ^ 1, abort_flag, p.status))) break;
-          mbar_arrive_expect_tx(&kfull[s], C::kTile);
+          mbar_arrive_expect_tx(&kfull[s], C::kStage);
+          const int kx = SEPV ? item.kcol : 0;      // head-group features (naive form)
           for (int kb = 0; kb < C::KB; ++kb)
-            tma_load_2d_hint(sm + C::oK + s * C::kTile + kb * C::kBlock, &tmK, kb * 64,
+            tma_load_2d_hint(sm + C::oK + s * C::kStage + kb * C::kBlock, &tmK, kx + kb * 64,
                              static_cast<int>(item.key0 + j * 128), &kfull[s], stream_policy);
+          if constexpr (SEPV)
+            for (int kb = 0; kb < C::KB; ++kb)
+              tma_load_2d_hint(sm + C::oK + s * C::kStage + C::kTile + kb * C::kBlock, &tmV,
+                               kx + kb * 64, static_cast<int>(item.key0 + j * 128), &kfull[s],
+                               stream_policy);
           ++ki;
         }
       }
@@ -243,7 +257,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           const int s = ki % KS;
           if (!(ok = bwait(&kfull[s], (ki / KS) & 1, abort_flag, p.status))) break;
           tc_fence_after();
-          const uint32_t kaddr = sbase + C::oK + s * C::kTile;
+          const uint32_t kaddr = sbase + C::oK + s * C::kStage;
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk)
             mma_bf16_ss(tmem + C::kS + sb * 128,
@@ -276,7 +290,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           if (j == 0 && !(ok = bwait(oempty, (ic & 1) ^ 1, abort_flag, p.status))) break;
           tc_fence_after();
           const int s = ki % KS;
-          const uint32_t vaddr = sbase + C::oK + s * C::kTile;
+          const uint32_t vaddr = sbase + C::oK + s * C::kStage + (SEPV ? C::kTile : 0u);
           if constexpr (C::P_TMEM) {
             // P: keys 2c, 2c+1 in column c of the buffer; 16 keys = 8 columns per MMA
 #pragma unroll
@@ -461,14 +475,14 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   }
 }
 
-template <int D, int QB, int KS, int PB>
+template <int D, int QB, int KS, int PB, bool SEPV = false>
 int launch_cfg(stca_handle* H, const CUtensorMap& tmQ, const CUtensorMap& tmK, const AttnParams& p,
-               int grid, cudaStream_t s) {
-  using C = AttnCfg<D, QB, KS, PB>;
-  auto k = attn_tc_kernel<D, QB, KS, PB>;
+               int grid, cudaStream_t s, const CUtensorMap* tmV = nullptr) {
+  using C = AttnCfg<D, QB, KS, PB, SEPV>;
+  auto k = attn_tc_kernel<D, QB, KS, PB, SEPV>;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
   if (e != cudaSuccess) return set_error(STCA_ECUDA, std::string("attn_tc smem: ") + cudaGetErrorString(e));
-  k<<<grid, kAttnThreads, C::kSmem, s>>>(tmQ, tmK, p);
+  k<<<grid, kAttnThreads, C::kSmem, s>>>(tmQ, tmK, tmV ? *tmV : tmK, p);
   return STCA_OK;
 }
 
@@ -493,6 +507,21 @@ int launch_attn_tc(stca_handle* H, int layer, const AttnItem* items_d, const int
     case 256: return launch_cfg<256, 1, 2, 1>(H, H->tmU, tmK, p, grid, s);
     default: return set_error(STCA_EINVAL, "tensor-core attention needs d in {64, 128, 256}");
   }
+}
+
+// Naive form: packed query rows (H->tmU over the [rows x 64] layout), keys and
+// values of the projection (H->tmKn, H->tmVn); partial rows are 64 wide.
+int launch_attn_tc_naive(stca_handle* H, const AttnItem* items_d, const int32_t* cta_begin_d,
+                         int grid, cudaStream_t s) {
+  AttnParams p{};
+  p.items = items_d;
+  p.cta_item_begin = cta_begin_d;
+  const int64_t G = H->last_G;
+  p.pacc = H->part;
+  p.pm = H->part + G * 64;
+  p.pl = p.pm + G;
+  p.status = H->status_d;
+  return launch_cfg<64, 2, 5, 2, true>(H, H->tmU, H->tmKn, p, grid, s, &H->tmVn);
 }
 
 // The same kernel with every buffer given explicitly (no handle state).

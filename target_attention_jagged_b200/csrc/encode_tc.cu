@@ -518,10 +518,15 @@ int launch_cfg(stca_handle* H, const CUtensorMap& tmX, const EncParams& p, cudaS
 
 int make_tmap_bf16_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer,
                       uint32_t box_inner, uint32_t box_outer) {
+  return make_tmap_bf16_2d_strided(m, base, inner, outer, inner * 2, box_inner, box_outer);
+}
+
+int make_tmap_bf16_2d_strided(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer,
+                              uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer) {
   auto fn = encode_fn();
   if (!fn) return set_error(STCA_ECUDA, "cuTensorMapEncodeTiled is unavailable");
   const cuuint64_t dims[2] = {inner, outer};
-  const cuuint64_t strides[1] = {inner * 2};
+  const cuuint64_t strides[1] = {row_bytes};
   const cuuint32_t box[2] = {box_inner, box_outer};
   const cuuint32_t es[2] = {1, 1};
   CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,

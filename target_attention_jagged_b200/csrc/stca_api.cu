@@ -10,6 +10,8 @@
 #include <string>
 #include <vector>
 
+#include <cublasLt.h>
+
 #include "stca_internal.h"
 
 namespace stca {
@@ -169,6 +171,10 @@ extern "C" void stca_destroy(stca_handle* H) {
   cudaFree(H->wstep);
   cudaFree(H->wstep_tc);
   cudaFree(H->whead);
+  cudaFree(H->wkv);
+  cudaFree(H->kv);
+  cudaFree(H->lt_ws);
+  if (H->lt) cublasLtDestroy(static_cast<cublasLtHandle_t>(H->lt));
   cudaFree(H->wtc);
   cudaFree(H->xt);
   cudaFree(H->q);
@@ -366,6 +372,26 @@ extern "C" int stca_init(const stca_weights* w, int d, int h, int r, int M, int 
         stca_destroy(H);
         return rc2;
       }
+      if (naive_layout(dh).G > 0) {
+        // naive form (Eq. (12)): [W_K | W_V] of every layer, d x 2d bf16
+        std::vector<uint16_t> kvw(static_cast<size_t>(M) * d * 2 * d);
+        auto bf = [](float f) {
+          uint32_t u;
+          memcpy(&u, &f, 4);
+          return static_cast<uint16_t>(u >> 16);     // bf16-valued already
+        };
+        for (int i = 0; i < M; ++i)
+          for (int k = 0; k < d; ++k)
+            for (int m = 0; m < 2 * d; ++m)
+              kvw[(static_cast<size_t>(i) * d + k) * 2 * d + m] =
+                  bf(m < d ? sw[i].Wk[static_cast<size_t>(k) * d + m] : sw[i].Wv[static_cast<size_t>(k) * d + m - d]);
+        if (cudaMalloc(&H->wkv, kvw.size() * 2) != cudaSuccess ||
+            cudaMemcpy(H->wkv, kvw.data(), kvw.size() * 2, cudaMemcpyHostToDevice) != cudaSuccess) {
+          cudaGetLastError();
+          stca_destroy(H);
+          return set_error(STCA_ENOMEM, "naive-form weight upload failed");
+        }
+      }
     }
   }
   if (nhead == 4) {
@@ -470,8 +496,17 @@ static int attn_path(const stca_handle* H) {
 //    its key tiles, laid end to end and cut into runs of equal numbers of key
 //    tiles, one run per CTA (stream-K); every maximal run inside one pair is
 //    an item.  `split`, when set, caps a run at split/128 key tiles.
+NaiveLayout stca::naive_layout(int dh) {
+  NaiveLayout L;
+  if (dh == 16 || dh == 32 || dh == 64) {
+    L.G = 64 / dh;
+    L.Tq = 128 / L.G;
+  }
+  return L;
+}
+
 void stca::build_plan_host(const int64_t* off, const int64_t* toff, int64_t R, int h, int path,
-                            int num_ctas, int64_t split_keys, PlanHost& P) {
+                            int num_ctas, int64_t split_keys, PlanHost& P, int dh) {
   P = PlanHost();
   P.req_pair_begin.assign(R + 1, 0);
   auto& items = P.items;
@@ -511,18 +546,29 @@ void stca::build_plan_host(const int64_t* off, const int64_t* toff, int64_t R, i
     P.pair_item_begin.push_back(static_cast<int32_t>(items.size()));
     return;
   }
+  // path 2: a request's T_r h query rows in tiles of 128; path 3 (naive form):
+  // (h / G) nslots tiles of 128 rows each (NaiveLayout)
+  const NaiveLayout NL = naive_layout(dh);
+  auto tiles_of = [&](int64_t r) -> int64_t {
+    const int64_t Tr = toff[r + 1] - toff[r];
+    if (path == 3) return Tr == 0 ? 0 : (h / NL.G) * ((Tr + NL.Tq - 1) / NL.Tq);
+    return (Tr * h + 127) / 128;
+  };
   struct Pair { int64_t r, mt, ntiles; };
   std::vector<Pair> pairs;
   int64_t W = 0;
+  if (path == 3) P.qbase.assign(R + 1, 0);
   for (int64_t r = 0; r < R; ++r) {
     P.req_pair_begin[r] = static_cast<int32_t>(pairs.size());
-    const int64_t rows = (toff[r + 1] - toff[r]) * h;
     const int64_t nt = (off[r + 1] - off[r] + 127) / 128;
-    for (int64_t mt = 0; mt * 128 < rows; ++mt) {
+    const int64_t ntile = tiles_of(r);
+    for (int64_t mt = 0; mt < ntile; ++mt) {
       pairs.push_back({r, mt, nt});
       W += nt;
     }
+    if (path == 3) P.qbase[r + 1] = P.qbase[r] + 128 * ntile;
   }
+  if (path == 3) P.qrows = P.qbase[R];
   P.req_pair_begin[R] = static_cast<int32_t>(pairs.size());
   int64_t cs = (W + num_ctas - 1) / std::max(num_ctas, 1);      // key tiles per CTA
   if (split_keys > 0) cs = std::min<int64_t>(cs, std::max<int64_t>(1, split_keys / 128));
@@ -534,7 +580,8 @@ void stca::build_plan_host(const int64_t* off, const int64_t* toff, int64_t R, i
   for (const Pair& pr : pairs) {
     P.pair_item_begin.push_back(static_cast<int32_t>(items.size()));
     const int64_t L = off[pr.r + 1] - off[pr.r];
-    const int64_t rows = std::min<int64_t>(128, (toff[pr.r + 1] - toff[pr.r]) * h - pr.mt * 128);
+    const int64_t rows = path == 3 ? 128
+                                   : std::min<int64_t>(128, (toff[pr.r + 1] - toff[pr.r]) * h - pr.mt * 128);
     int64_t a = 0;
     while (a < pr.ntiles) {
       const int64_t g0 = cursor + a;
@@ -545,9 +592,15 @@ void stca::build_plan_host(const int64_t* off, const int64_t* toff, int64_t R, i
       it.key0 = off[pr.r] + a * 128;
       it.nkeys = static_cast<int32_t>(std::min<int64_t>(b * 128, L) - a * 128);
       it.row_base = G;
-      it.qrow0 = toff[pr.r] * h + pr.mt * 128;
       it.mt = static_cast<int32_t>(pr.mt);
       it.rows = static_cast<int32_t>(rows);
+      if (path == 3) {
+        const int64_t nslots = (toff[pr.r + 1] - toff[pr.r] + NL.Tq - 1) / NL.Tq;
+        it.qrow0 = P.qbase[pr.r] + pr.mt * 128;
+        it.kcol = static_cast<int32_t>((pr.mt / nslots) * 64);
+      } else {
+        it.qrow0 = toff[pr.r] * h + pr.mt * 128;
+      }
       G += rows;
       items.push_back(it);
       a = b;
@@ -564,6 +617,7 @@ int stca::check_plan(const PlanHost& P, const int64_t* off, const int64_t* toff,
                       int h, int path) {
   const int64_t N = off[R], T = toff[R];
   auto bad = [](const std::string& m) { return set_error(STCA_EINVAL, "internal plan check: " + m); };
+  if (path == 3 && static_cast<int64_t>(P.qbase.size()) != R + 1) return bad("naive query layout");
   int64_t rows_sum = 0;
   for (size_t w = 0; w < P.items.size(); ++w) {
     const AttnItem& it = P.items[w];
@@ -573,7 +627,13 @@ int stca::check_plan(const PlanHost& P, const int64_t* off, const int64_t* toff,
     if (it.rows < 0 || it.row_base != rows_sum) return bad("partial rows not contiguous");
     rows_sum += it.rows;
     const int64_t req_rows = (toff[it.req + 1] - toff[it.req]) * h;
-    if (path == 2) {
+    if (path == 3) {
+      const int64_t ntile = P.req_pair_begin[it.req + 1] - P.req_pair_begin[it.req];
+      if (it.rows != 128 || it.mt < 0 || it.mt >= ntile ||
+          it.qrow0 != P.qbase[it.req] + int64_t(it.mt) * 128 || it.qrow0 + 128 > P.qrows ||
+          it.kcol < 0 || it.kcol % 64 != 0 || it.kcol + 64 > int64_t(h) * 64)
+        return bad("naive query tile");
+    } else if (path == 2) {
       if (it.rows < 1 || it.rows > 128 || int64_t(it.mt) * 128 + it.rows > req_rows ||
           it.qrow0 != toff[it.req] * h + int64_t(it.mt) * 128 || it.qrow0 + it.rows > T * h)
         return bad("query tile");
@@ -590,7 +650,7 @@ int stca::check_plan(const PlanHost& P, const int64_t* off, const int64_t* toff,
   if (P.pair_item_begin[npairs] != static_cast<int32_t>(P.items.size())) return bad("pair end");
   for (int64_t r = 0; r < R; ++r) {
     const int64_t rows = (toff[r + 1] - toff[r]) * h;
-    const int64_t want = path == 2 ? (rows + 127) / 128 : 1;
+    const int64_t want = path == 2 ? (rows + 127) / 128 : path == 3 ? (P.qbase[r + 1] - P.qbase[r]) / 128 : 1;
     if (P.req_pair_begin[r + 1] - P.req_pair_begin[r] != want) return bad("pairs of a request");
     for (int32_t p = P.req_pair_begin[r]; p < P.req_pair_begin[r + 1]; ++p) {
       // the pair's items cover the request's keys exactly once, in order
@@ -602,7 +662,7 @@ int stca::check_plan(const PlanHost& P, const int64_t* off, const int64_t* toff,
       if (rows > 0 && k != off[r + 1]) return bad("keys not covered");
     }
   }
-  if (path == 2) {
+  if (path >= 2) {
     if (static_cast<int>(P.cta_begin.size()) != P.grid + 1 || P.cta_begin[0] != 0 ||
         P.cta_begin[P.grid] != static_cast<int32_t>(P.items.size()))
       return bad("CTA ranges");
@@ -629,7 +689,7 @@ static int build_plan(stca_handle* H, const int64_t* toff, int64_t T, int path, 
     return STCA_OK;   // same layout as the previous forward on this encode: plan is on device
   const int64_t* off = H->offsets_h.data();
   PlanHost P;
-  build_plan_host(off, toff, R, H->h, path, H->num_sms, H->opt_split_keys, P);
+  build_plan_host(off, toff, R, H->h, path, H->num_sms, H->opt_split_keys, P, H->dh);
   if (int rc = check_plan(P, off, toff, R, H->h, path)) return rc;
   const auto& items = P.items;
   const auto& pairs_simt = P.pairs_simt;
@@ -646,7 +706,8 @@ static int build_plan(stca_handle* H, const int64_t* toff, int64_t T, int path, 
   H->off_toff = align256(H->off_treq + static_cast<size_t>(T) * sizeof(int32_t));
   H->off_rpb = align256(H->off_toff + static_cast<size_t>(R + 1) * sizeof(int64_t));
   H->off_pib = align256(H->off_rpb + static_cast<size_t>(R + 1) * sizeof(int32_t));
-  const size_t bytes = align256(H->off_pib + pair_item_begin.size() * sizeof(int32_t));
+  H->off_qbase = align256(H->off_pib + pair_item_begin.size() * sizeof(int32_t));
+  const size_t bytes = align256(H->off_qbase + P.qbase.size() * sizeof(int64_t));
   // pinned staging: wait until the previous upload has left it
   if (H->plan_h && cudaEventSynchronize(H->plan_evt) != cudaSuccess)
     return set_error(STCA_ECUDA, "plan event wait failed");
@@ -672,6 +733,8 @@ static int build_plan(stca_handle* H, const int64_t* toff, int64_t T, int path, 
   memcpy(p + H->off_toff, toff, static_cast<size_t>(R + 1) * sizeof(int64_t));
   memcpy(p + H->off_rpb, req_pair_begin.data(), static_cast<size_t>(R + 1) * sizeof(int32_t));
   memcpy(p + H->off_pib, pair_item_begin.data(), pair_item_begin.size() * sizeof(int32_t));
+  if (!P.qbase.empty()) memcpy(p + H->off_qbase, P.qbase.data(), P.qbase.size() * sizeof(int64_t));
+  H->last_qrows = P.qrows;
   STCA_CUDA_TRY(cudaMemcpyAsync(H->plan_d, H->plan_h, bytes, cudaMemcpyHostToDevice, s));
   STCA_CUDA_TRY(cudaEventRecord(H->plan_evt, s));
   H->last_G = G;
@@ -683,6 +746,75 @@ static int build_plan(stca_handle* H, const int64_t* toff, int64_t T, int path, 
   H->last_path = path;
   H->last_toff.assign(toff, toff + R + 1);
   return STCA_OK;
+}
+
+// Naive form, Eq. (12): K = X~(layer+1) W_K and V = X~(layer+1) W_V for every
+// history row at once, into H->kv (row n: [K_n | V_n], bf16).  A plain GEMM,
+// [N x d] x [d x 2d], run by cuBLASLt (bf16 operands, fp32 accumulation).
+static int kv_project(stca_handle* H, int layer, cudaStream_t s) {
+  const int d = H->d;
+  const int64_t N = H->N;
+  if (!H->lt) {
+    cublasLtHandle_t lt = nullptr;
+    if (cublasLtCreate(&lt) != CUBLAS_STATUS_SUCCESS) return set_error(STCA_ECUDA, "cublasLtCreate failed");
+    H->lt = lt;
+  }
+  constexpr size_t kWs = size_t(32) << 20;
+  if (int rc = ensure_dev(&H->lt_ws, &H->lt_ws_cap, kWs)) return rc;
+  cublasLtHandle_t lt = static_cast<cublasLtHandle_t>(H->lt);
+  cublasLtMatmulDesc_t op = nullptr;
+  cublasLtMatrixLayout_t la = nullptr, lb = nullptr, lc = nullptr;
+  cublasLtMatmulPreference_t pref = nullptr;
+  int rc = STCA_OK;
+  // column-major view: KV^T (2d x N) = W^T (2d x d) * X~^T (d x N)
+  if (cublasLtMatmulDescCreate(&op, CUBLAS_COMPUTE_32F, CUDA_R_32F) != CUBLAS_STATUS_SUCCESS ||
+      cublasLtMatrixLayoutCreate(&la, CUDA_R_16BF, 2 * d, d, 2 * d) != CUBLAS_STATUS_SUCCESS ||
+      cublasLtMatrixLayoutCreate(&lb, CUDA_R_16BF, d, N, d) != CUBLAS_STATUS_SUCCESS ||
+      cublasLtMatrixLayoutCreate(&lc, CUDA_R_16BF, 2 * d, N, 2 * d) != CUBLAS_STATUS_SUCCESS ||
+      cublasLtMatmulPreferenceCreate(&pref) != CUBLAS_STATUS_SUCCESS) {
+    rc = set_error(STCA_ECUDA, "cuBLASLt descriptor set-up failed");
+  }
+  cublasLtMatmulHeuristicResult_t heur{};
+  int found = 0;
+  if (rc == STCA_OK) {
+    size_t ws = kWs;
+    cublasLtMatmulPreferenceSetAttribute(pref, CUBLASLT_MATMUL_PREF_MAX_WORKSPACE_BYTES, &ws, sizeof(ws));
+    if (cublasLtMatmulAlgoGetHeuristic(lt, op, la, lb, lc, lc, pref, 1, &heur, &found) !=
+            CUBLAS_STATUS_SUCCESS || found < 1)
+      rc = set_error(STCA_ECUDA, "cuBLASLt found no algorithm for the K/V projection");
+  }
+  if (rc == STCA_OK) {
+    const float alpha = 1.f, beta = 0.f;
+    const uint16_t* w = static_cast<const uint16_t*>(H->wkv) + static_cast<size_t>(layer) * d * 2 * d;
+    const void* x = static_cast<const char*>(H->xt) + static_cast<size_t>(N) * d * 2 * layer;
+    if (cublasLtMatmul(lt, op, &alpha, w, la, x, lb, &beta, H->kv, lc, H->kv, lc, &heur.algo, H->lt_ws,
+                       kWs, s) != CUBLAS_STATUS_SUCCESS)
+      rc = set_error(STCA_ECUDA, "cuBLASLt K/V projection failed");
+  }
+  if (pref) cublasLtMatmulPreferenceDestroy(pref);
+  if (lc) cublasLtMatrixLayoutDestroy(lc);
+  if (lb) cublasLtMatrixLayoutDestroy(lb);
+  if (la) cublasLtMatrixLayoutDestroy(la);
+  if (op) cublasLtMatmulDescDestroy(op);
+  return rc;
+}
+
+// FLOPs of one layer's attention in either form: the reordered form contracts
+// d features for each of the T_r h query rows; the naive form projects K and V
+// (4 L d^2) and then contracts the tile's 64 head-group features for the
+// padded query rows of its layout.
+static bool naive_cheaper(const stca_handle* H, const int64_t* toff) {
+  const NaiveLayout NL = naive_layout(H->dh);
+  double re = 0, nv = 0;
+  const double d = H->d, h = H->h;
+  for (int64_t r = 0; r < H->R; ++r) {
+    const double L = static_cast<double>(H->offsets_h[r + 1] - H->offsets_h[r]);
+    const int64_t Tr = toff[r + 1] - toff[r];
+    re += 4.0 * Tr * h * L * d;
+    const double rows = Tr == 0 ? 0.0 : 128.0 * (h / NL.G) * ((Tr + NL.Tq - 1) / NL.Tq);
+    nv += 4.0 * L * d * d + 4.0 * rows * L * 64.0;
+  }
+  return nv < re;
 }
 
 extern "C" int stca_forward(stca_handle* H, const void* targets, const int64_t* target_offsets,
@@ -703,10 +835,31 @@ extern "C" int stca_forward(stca_handle* H, const void* targets, const int64_t* 
     return set_error(STCA_EINVAL, "tensor-core attention needs bf16 and d in {64, 128, 256}");
   if (path == 1 && attn_simt_smem(H) > 227 * 1024)
     return set_error(STCA_EINVAL, "h * d too large for the CUDA-core attention kernel");
-  if (int rc = build_plan(H, target_offsets, T, path, s)) return rc;
+  // attention form: the reordered Eq. (13) unless the naive Eq. (12) is asked for
+  const NaiveLayout NL = naive_layout(H->dh);
+  const bool naive_ok = path == 2 && H->step_tc_ready && H->opt_step_path != 1 && NL.G > 0 &&
+                        H->wkv != nullptr;
+  if (H->opt_attn_form == 1 && !naive_ok)
+    return set_error(STCA_EINVAL, "the naive attention form needs the tensor-core attention and step "
+                                  "(bf16, d in {128, 256}, r d <= 512) and d_h in {16, 32, 64}");
+  const bool naive = naive_ok && (H->opt_attn_form == 1 ||
+                                  (H->opt_attn_form == 2 && naive_cheaper(H, target_offsets)));
+  H->last_naive = naive;
+  if (int rc = build_plan(H, target_offsets, T, naive ? 3 : path, s)) return rc;
   const int d = H->d, h = H->h;
   const size_t urows = static_cast<size_t>(T) * h;
-  if (path == 1) {
+  if (naive) {
+    const size_t qrows = static_cast<size_t>(H->last_qrows);
+    if (int rc = ensure_dev(reinterpret_cast<void**>(&H->Ubf), &H->Ubf_cap, std::max<size_t>(qrows, 1) * 128))
+      return rc;
+    if (int rc = make_tmap_bf16_2d(&H->tmU, H->Ubf, 64, qrows, 64, 128)) return rc;
+    if (int rc = ensure_dev(&H->kv, &H->kv_cap, static_cast<size_t>(H->N) * 4 * d)) return rc;
+    if (int rc = make_tmap_bf16_2d_strided(&H->tmKn, H->kv, d, H->N, 4 * d, 64, 128)) return rc;
+    if (int rc = make_tmap_bf16_2d_strided(&H->tmVn, static_cast<char*>(H->kv) + 2 * d, d, H->N, 4 * d,
+                                           64, 128))
+      return rc;
+    STCA_CUDA_TRY(cudaMemsetAsync(H->Ubf, 0, qrows * 128, s));   // padding rows stay zero
+  } else if (path == 1) {
     if (int rc = ensure_dev(reinterpret_cast<void**>(&H->U), &H->U_cap, urows * d * sizeof(float)))
       return rc;
   } else {
@@ -714,7 +867,8 @@ extern "C" int stca_forward(stca_handle* H, const void* targets, const int64_t* 
     if (int rc = make_tmap_bf16_2d(&H->tmU, H->Ubf, d, urows, 64, 128)) return rc;
   }
   if (int rc = ensure_dev(reinterpret_cast<void**>(&H->part), &H->part_cap,
-                          static_cast<size_t>(std::max<int64_t>(H->last_G, 1)) * (d + 2) * sizeof(float)))
+                          static_cast<size_t>(std::max<int64_t>(H->last_G, 1)) * ((naive ? 64 : d) + 2) *
+                              sizeof(float)))
     return rc;
   if (int rc = ensure_dev(reinterpret_cast<void**>(&H->cbuf), &H->cbuf_cap, urows * d * sizeof(float)))
     return rc;
@@ -738,12 +892,13 @@ extern "C" int stca_forward(stca_handle* H, const void* targets, const int64_t* 
   const bool step_tc = path == 2 && H->step_tc_ready && H->opt_step_path != 1;
   // the tensor-core step merges the split partials itself when every query
   // tile has few enough items; otherwise combine_kernel merges them first
-  const bool fused = step_tc && H->last_max_items <= step_tc_max_items() &&
+  const bool fused = !naive && step_tc && H->last_max_items <= step_tc_max_items() &&
                      H->last_G < (int64_t(1) << 31);
+  NaiveStep ns{NL.G, NL.Tq, reinterpret_cast<const int64_t*>(p + H->off_qbase), H->Ubf};
   auto step = [&](int layer, const float* cm) {
     if (step_tc)
       return launch_step_tc(H, layer, targets, T, fused ? nullptr : cm, &plan, H->part, H->last_G,
-                            Z, H->Ubf, s);
+                            Z, H->Ubf, s, naive ? &ns : nullptr);
     launch_target_step(H, layer, targets, T, plan, cm, Z, s);
     return static_cast<int>(STCA_OK);
   };
@@ -757,7 +912,11 @@ extern "C" int stca_forward(stca_handle* H, const void* targets, const int64_t* 
     int rc = STCA_OK;
     {
       TimedLaunch tl(H, STCA_K_ATTN, s);
-      if (path == 2) {
+      if (naive) {
+        rc = kv_project(H, i, s);
+        if (!rc) rc = launch_attn_tc_naive(H, items_d, cta_d, H->last_grid, s);
+        H->launches++;
+      } else if (path == 2) {
         rc = launch_attn_tc(H, i, items_d, cta_d, H->last_grid, s);
       } else {
         const void* xti = static_cast<const char*>(H->xt) + layer_bytes * i;
@@ -769,7 +928,10 @@ extern "C" int stca_forward(stca_handle* H, const void* targets, const int64_t* 
     if (int rc2 = check_launch("attention")) return rc2;
     {
       TimedLaunch tl(H, STCA_K_STEP, s);
-      if (!fused) {
+      if (naive) {
+        launch_combine_naive(H, plan, H->part, H->last_G, T, H->cbuf, s);
+        H->launches++;
+      } else if (!fused) {
         launch_combine(H, plan, H->part, H->last_G, T, H->cbuf, s);
         H->launches++;
       }
@@ -919,6 +1081,10 @@ extern "C" int stca_set_option(stca_handle* H, int option, int64_t value) {
       if (value != 0 && value != 1) return set_error(STCA_EINVAL, "timing must be 0 or 1");
       H->timing = value != 0;
       return ok();
+    case STCA_OPT_ATTN_FORM:
+      if (value < 0 || value > 2) return set_error(STCA_EINVAL, "attention form must be 0, 1 or 2");
+      H->opt_attn_form = static_cast<int>(value);
+      return ok();
     case STCA_OPT_SPLIT_KEYS:
       if (value < 0 || value % 128 || value > (int64_t(1) << 30))
         return set_error(STCA_EINVAL, "split must be 0 or a positive multiple of 128");
@@ -938,6 +1104,8 @@ extern "C" int stca_get_option(stca_handle* H, int option, int64_t* value) {
     case STCA_OPT_SPLIT_KEYS: *value = H->opt_split_keys; return ok();
     case STCA_OPT_TIMING: *value = H->timing ? 1 : 0; return ok();
     case STCA_OPT_LAUNCHES: *value = H->launches; return ok();
+    case STCA_OPT_ATTN_FORM: *value = H->opt_attn_form; return ok();
+    case STCA_OPT_LAST_FORM: *value = H->last_naive ? 1 : 0; return ok();
     default: return set_error(STCA_EINVAL, "unknown option " + std::to_string(option));
   }
 }

@@ -37,6 +37,17 @@ struct AttnItem {
   int64_t qrow0;      // first query row (row of U: target * h + head)
   int32_t mt;         // query tile index within the request
   int32_t rows;       // query rows of this tile that belong to the request
+  int32_t kcol;       // naive form: first feature of the tile's head group in K and V
+  int32_t pad_;
+};
+
+// Query layout of the naive-form attention (Eq. (12) with K = X~ W_K and
+// V = X~ W_V projected once per request): G = 64 / d_h heads share a tile, each
+// with Tq = 128 / G query positions.  Request r has nslots = ceil(T_r / Tq)
+// slots and (h / G) * nslots tiles of 128 rows, tile mt = jg * nslots + qs
+// holding rows s * Tq + tt for head j = jg * G + s and target qs * Tq + tt.
+struct NaiveLayout {
+  int G = 0, Tq = 0;
 };
 
 // Per-layer pointers into the handle's fp32 weight slab (CUDA-core kernels and
@@ -95,6 +106,13 @@ struct stca_handle {
   CUtensorMap tmW1, tmW2;               // their TMA descriptors
   CUtensorMap tmXt[16];                 // X~(i) of the last encode (tensor-core attention)
   CUtensorMap tmU;                      // bf16 query rows of the current forward
+  CUtensorMap tmKn, tmVn;               // naive form: keys and values of the current layer
+  int opt_attn_form = 0;                // 0 reordered (Eq. (13)), 1 naive (Eq. (12)), 2 auto
+  bool last_naive = false;              // the last forward ran the naive form
+  void* kv = nullptr;       size_t kv_cap = 0;     // naive form: N x 2d bf16, [K | V] per row
+  void* wkv = nullptr;                  // naive form: per layer [W_K | W_V], d x 2d bf16
+  void* lt = nullptr;                   // cuBLASLt handle (naive-form projection)
+  void* lt_ws = nullptr;    size_t lt_ws_cap = 0;  // its workspace
   bool tc_encode_ready = false;
   uint16_t* wstep_tc = nullptr;         // A-tile stream of the tensor-core per-target step
   std::vector<stca::TcGemm> tcO, tcC, tcUG, tcD, tcQ;   // per layer
@@ -142,7 +160,8 @@ struct stca_handle {
   int last_max_items = 0;               // most items of one (request, query tile) pair
   int last_grid = 0;                    // CTAs of the tensor-core attention
   size_t off_items = 0, off_pairs = 0, off_cta = 0, off_treq = 0, off_toff = 0, off_rpb = 0,
-         off_pib = 0;
+         off_pib = 0, off_qbase = 0;
+  int64_t last_qrows = 0;               // naive form: rows of the packed query layout
 };
 
 namespace stca {
@@ -167,6 +186,9 @@ struct StepPlan {
 // Per-target step (target_step.cu)
 void launch_combine(const stca_handle* H, const StepPlan& plan, const float* part, int64_t G,
                     int64_t T, float* out, cudaStream_t s);
+// Naive form: per-head outputs o_head (T x d fp32) from 64-wide partials.
+void launch_combine_naive(const stca_handle* H, const StepPlan& plan, const float* part, int64_t G,
+                          int64_t T, float* out, cudaStream_t s);
 void launch_target_step(const stca_handle* H, int layer, const void* targets, int64_t T,
                         const StepPlan& plan, const float* cmerged, float* Z, cudaStream_t s);
 size_t target_step_smem(const stca_handle* H);
@@ -185,9 +207,17 @@ int step_tc_setup(stca_handle* H, const std::vector<StepHostW>& layers);
 // partials (part: G x d accumulators, then G maxima, G sums) inside the step;
 // that needs at most step_tc_max_items() items per (request, query tile).
 int step_tc_max_items();
+// Naive form of the step: `naive` not NULL; cmerged then holds o_head (T x d, the
+// per-head outputs of Eq. (12)), and the query rows of the next layer are written
+// into the packed layout (NaiveLayout) at naive->upk, request r from row qbase[r].
+struct NaiveStep {
+  int G, Tq;
+  const int64_t* qbase;     // device, R + 1
+  uint16_t* upk;            // device, [rows x 64] bf16
+};
 int launch_step_tc(const stca_handle* H, int layer, const void* targets, int64_t T,
                    const float* cmerged, const StepPlan* plan, const float* part, int64_t G,
-                   float* Z, uint16_t* Ubf, cudaStream_t s);
+                   float* Z, uint16_t* Ubf, cudaStream_t s, const NaiveStep* naive = nullptr);
 
 // Host-side attention work plan (stca_api.cu).
 struct PlanHost {
@@ -196,11 +226,14 @@ struct PlanHost {
   std::vector<int32_t> cta_begin;        // tensor-core grid + 1
   std::vector<int32_t> req_pair_begin;   // R + 1
   std::vector<int32_t> pair_item_begin;  // pairs + 1
+  std::vector<int64_t> qbase;            // naive form (path 3): first query row of each request
+  int64_t qrows = 0;                     // naive form: query rows of the padded layout
   int64_t G = 0;                         // partial rows
   int grid = 0;                          // tensor-core CTAs
 };
 void build_plan_host(const int64_t* off, const int64_t* toff, int64_t R, int h, int path,
-                     int num_ctas, int64_t split_keys, PlanHost& P);
+                     int num_ctas, int64_t split_keys, PlanHost& P, int dh = 0);
+NaiveLayout naive_layout(int dh);
 int check_plan(const PlanHost& P, const int64_t* off, const int64_t* toff, int64_t R, int h,
                int path);
 void launch_target_step_ws(const stca_handle* H, int layer, const void* targets, int64_t T,
@@ -213,6 +246,8 @@ int launch_attn_tc_ws(int d, const CUtensorMap& tmQ, const CUtensorMap& tmK,
 bool attn_tc_supported(int d);
 int launch_attn_tc(stca_handle* H, int layer, const AttnItem* items_d, const int32_t* cta_begin_d,
                    int grid, cudaStream_t s);
+int launch_attn_tc_naive(stca_handle* H, const AttnItem* items_d, const int32_t* cta_begin_d,
+                         int grid, cudaStream_t s);
 
 // Tensor-core encoder (encode_tc.cu)
 bool encode_tc_supported(int d, int rd);
@@ -221,5 +256,8 @@ int encode_tc_setup(stca_handle* H, const std::vector<const float*>& Wu,
 int launch_encode_tc(stca_handle* H, const void* X, int64_t N, cudaStream_t s);
 int make_tmap_bf16_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer,
                       uint32_t box_inner, uint32_t box_outer);
+// The same with rows `row_bytes` apart (a multiple of 16).
+int make_tmap_bf16_2d_strided(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer,
+                              uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer);
 
 }  // namespace stca

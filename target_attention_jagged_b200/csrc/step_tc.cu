@@ -160,6 +160,10 @@ struct StepTcArgs {
   int kind[5];
   int nring;                    // A-tile ring stages
   int kch;                      // inputs per W_V staging chunk
+  int naive;                    // naive form: cmerged is o_head (T x d); write packed q rows
+  int nG, nTq;                  // its layout (NaiveLayout)
+  const int64_t* qbase;         // first packed row of each request
+  uint16_t* upk;                // packed query rows [rows x 64] bf16
 };
 
 // Shared memory, in bytes (1024-aligned base): the A-tile ring, then the
@@ -413,6 +417,22 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_tc_kernel(const StepTcAr
           *reinterpret_cast<uint4*>(bufs[kC] + (8 * k8 >> 6) * kBTile + sw128_off(t, (8 * k8) & 63)) = v;
         }
       }
+      if (a.naive) {
+        // naive form: the per-head outputs o_head[t] (already alpha V per head)
+        // are the B operand of W_O as they are
+        const int d8 = d / 8;
+        for (int e = tid; e < kTgt * d8; e += 32 * kWorkers) {
+          const int t = e / d8, k8 = e - t * d8;
+          uint4 v = make_uint4(0u, 0u, 0u, 0u);
+          if (t < nb) {
+            const float4* z = reinterpret_cast<const float4*>(a.cmerged + (t0 + t) * d + 8 * k8);
+            const float4 z0 = z[0], z1 = z[1];
+            v = make_uint4(pack_bf16x2(z0.x, z0.y), pack_bf16x2(z0.z, z0.w),
+                           pack_bf16x2(z1.x, z1.y), pack_bf16x2(z1.z, z1.w));
+          }
+          *reinterpret_cast<uint4*>(bufs[kO] + (8 * k8 >> 6) * kBTile + sw128_off(t, (8 * k8) & 63)) = v;
+        }
+      } else {
       // o_head = c_j W_V^j into the B operand of W_O.  Output column n belongs
       // to head n / d_h; a thread owns blocks of 4 targets x 2 columns and
       // accumulates them over the d inputs, which arrive in chunks of kch:
@@ -530,6 +550,7 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_tc_kernel(const StepTcAr
                 pack_bf16x2(acc[bi][t][0], acc[bi][t][1]);
         }
       }
+      }   // reordered form
     }
     fence_proxy_async_smem();
     __syncwarp();
@@ -629,7 +650,33 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_tc_kernel(const StepTcAr
     // ---- u_j = P_j W_K^j^T (Eq. (13)), scaled, as bf16 rows for the attention.
     // A thread owns blocks of 16 targets x 4 outputs (head j, columns k..k+3):
     // per c < d_h, one 8-byte load of W_K^T and the 16 targets' P[j d_h + c].
-    if (L + 1 < M) {
+    if (L + 1 < M && a.naive) {
+      // naive form: q W_Q of head j as row (j % G) Tq + tt of tile (j / G) nslots + qs
+      // of the packed layout (target qs Tq + tt of its request), non-zero only in
+      // the head's own d_h of the tile's 64 columns, scaled like u
+      workers_sync();
+      const int G = a.nG, Tq = a.nTq, ng8 = h * 8;
+      for (int e = tid; e < kTgt * ng8; e += 32 * kWorkers) {
+        const int t = e / ng8, rest = e - t * ng8;
+        const int j = rest >> 3, c8 = rest & 7;
+        if (t >= nb) continue;
+        const int64_t tg = t0 + t;
+        const int r = a.plan.treq[tg];
+        const int64_t tl = tg - a.plan.toff[r], Tr = a.plan.toff[r + 1] - a.plan.toff[r];
+        const int64_t nslots = (Tr + Tq - 1) / Tq, qs = tl / Tq, tt = tl - qs * Tq;
+        const int jg = j / G, sl = j - jg * G;
+        const int64_t row = a.qbase[r] + (jg * nslots + qs) * 128 + static_cast<int64_t>(sl) * Tq + tt;
+        float v[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int c = 8 * c8 + u;                // column of the 64-wide packed row
+          v[u] = c / dh == sl ? scr[(jg * 64 + c) * kTgt + t] * a.uscale : 0.f;
+        }
+        *reinterpret_cast<uint4*>(a.upk + row * 64 + 8 * c8) =
+            make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
+                       pack_bf16x2(v[6], v[7]));
+      }
+    } else if (L + 1 < M) {
       workers_sync();
       const int hd = h * d;
       for (int b = tid; b < hd / 4; b += 32 * kWorkers) {
@@ -694,7 +741,7 @@ int step_tc_max_items() { return kMaxItems; }
 
 int launch_step_tc(const stca_handle* H, int layer, const void* targets, int64_t T,
                    const float* cmerged, const StepPlan* plan, const float* part, int64_t G,
-                   float* Z, uint16_t* Ubf, cudaStream_t s) {
+                   float* Z, uint16_t* Ubf, cudaStream_t s, const NaiveStep* naive) {
   if (T <= 0) return STCA_OK;
   if (!H->step_tc_ready) return set_error(STCA_ESTATE, "tensor-core step weights are not set up");
   const int M = H->M;
@@ -711,6 +758,16 @@ int launch_step_tc(const stca_handle* H, int layer, const void* targets, int64_t
     a.pacc = part;
     a.pm = part + G * H->d;
     a.pl = a.pm + G;
+  }
+  if (plan) a.plan = *plan;
+  if (naive) {
+    if (!plan || (layer >= 0 && !cmerged))
+      return set_error(STCA_EINVAL, "tensor-core step: the naive form needs o_head and the plan");
+    a.naive = 1;
+    a.nG = naive->G;
+    a.nTq = naive->Tq;
+    a.qbase = naive->qbase;
+    a.upk = naive->upk;
   }
   a.Z = Z;
   a.Ubf = Ubf;

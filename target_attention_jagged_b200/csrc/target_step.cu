@@ -288,6 +288,63 @@ combine_kernel(StepPlan P, const float* __restrict__ pacc, const float* __restri
   }
 }
 
+// Naive-form merge (Eq. (12) with projected K, V): o_j[t] = sum_w s_w acc_w / sum_w
+// s_w l_w over the items of head j's row of target t, where acc_w holds the
+// tile's 64 head-group features of alpha V and head j owns d_h of them.  One
+// warp per (target, head) query row, eight per CTA; writes o_head[t][j d_h + c].
+__global__ void __launch_bounds__(kCombineThreads)
+combine_naive_kernel(StepPlan P, const float* __restrict__ pacc, const float* __restrict__ pm,
+                     const float* __restrict__ pl, float* __restrict__ out, int d, int h, int dh,
+                     int G, int Tq, int64_t nq) {
+  const int lane = threadIdx.x & 31;
+  const int64_t qr = static_cast<int64_t>(blockIdx.x) * kCombineRows + (threadIdx.x >> 5);
+  if (qr >= nq) return;
+  const int64_t t = qr / h;
+  const int j = static_cast<int>(qr - t * h);
+  const int r = P.treq[t];
+  const int64_t tl = t - P.toff[r], Tr = P.toff[r + 1] - P.toff[r];
+  const int64_t nslots = (Tr + Tq - 1) / Tq, qs = tl / Tq, tt = tl - qs * Tq;
+  const int jg = j / G, sl = j - jg * G;
+  const int64_t row = static_cast<int64_t>(sl) * Tq + tt;
+  const int pair = P.req_pair_begin[r] + static_cast<int>(jg * nslots + qs);
+  const int w0 = P.pair_item_begin[pair], nw = P.pair_item_begin[pair + 1] - w0;
+  float mx = -INFINITY;
+  for (int b = 0; b < nw; b += 32)
+    if (b + lane < nw) mx = fmaxf(mx, pm[P.items[w0 + b + lane].row_base + row]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  float ls = 0.f;
+  for (int b = 0; b < nw; b += 32)
+    if (b + lane < nw) {
+      const int64_t g = P.items[w0 + b + lane].row_base + row;
+      ls = fmaf(pl[g], exp2f(pm[g] - mx), ls);
+    }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) ls += __shfl_xor_sync(0xffffffffu, ls, o);
+  const float inv = 1.0f / ls;
+  float* orow = out + t * d + static_cast<int64_t>(j) * dh;
+  for (int b = 0; b < nw; b += 32) {
+    int64_t g = 0;
+    float f = 0.f;
+    if (b + lane < nw) {
+      g = P.items[w0 + b + lane].row_base + row;
+      f = exp2f(pm[g] - mx) * inv;
+    }
+    const int n = min(32, nw - b);
+    for (int c0 = 0; c0 < dh; c0 += 32) {      // warp-uniform: the shuffles below
+      const int c = c0 + lane;
+      const bool on = c < dh;
+      float acc = (on && b > 0) ? orow[c] : 0.f;
+      for (int w = 0; w < n; ++w) {
+        const int64_t gw = __shfl_sync(0xffffffffu, g, w);
+        const float fw = __shfl_sync(0xffffffffu, f, w);
+        if (on) acc = fmaf(fw, __ldg(pacc + gw * 64 + sl * dh + c), acc);
+      }
+      if (on) orow[c] = acc;
+    }
+  }
+}
+
 struct StepArgs {
   int layer, M, d, h, dh, rd;
   int64_t T;
@@ -581,6 +638,19 @@ void launch_combine(const stca_handle* H, const StepPlan& plan, const float* par
   const int64_t nq = T * H->h;
   combine_kernel<<<static_cast<unsigned>((nq + kCombineRows - 1) / kCombineRows), kCombineThreads, 0,
                    s>>>(plan, pacc, pm, pl, out, H->d, H->h, nq);
+}
+
+void launch_combine_naive(const stca_handle* H, const StepPlan& plan, const float* part, int64_t G,
+                          int64_t T, float* out, cudaStream_t s) {
+  if (T <= 0) return;
+  const NaiveLayout NL = naive_layout(H->dh);
+  const float* pacc = part;
+  const float* pm = part + G * 64;
+  const float* pl = pm + G;
+  const int64_t nq = T * H->h;
+  combine_naive_kernel<<<static_cast<unsigned>((nq + kCombineRows - 1) / kCombineRows),
+                         kCombineThreads, 0, s>>>(plan, pacc, pm, pl, out, H->d, H->h, H->dh, NL.G,
+                                                  NL.Tq, nq);
 }
 
 void launch_target_step(const stca_handle* H, int layer, const void* targets, int64_t T,

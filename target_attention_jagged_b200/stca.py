@@ -25,7 +25,9 @@ STCA_F32, STCA_BF16 = 0, 1
 STCA_OK, STCA_EINVAL, STCA_ESTATE, STCA_ENOMEM, STCA_ECUDA, STCA_EDEVICE = 0, -1, -2, -3, -4, -5
 STCA_OPT_ATTN_PATH, STCA_OPT_ENCODE_PATH, STCA_OPT_SPLIT_KEYS, STCA_OPT_TIMING = 1, 2, 3, 4
 STCA_OPT_STEP_PATH = 5
+STCA_OPT_ATTN_FORM = 6
 STCA_OPT_LAUNCHES = 100
+STCA_OPT_LAST_FORM = 101
 STCA_K_ENCODE, STCA_K_ATTN, STCA_K_STEP, STCA_K_HEAD, STCA_K_CLASSES = 0, 1, 2, 3, 4
 _NAMES = {STCA_EINVAL: "EINVAL", STCA_ESTATE: "ESTATE", STCA_ENOMEM: "ENOMEM",
           STCA_ECUDA: "ECUDA", STCA_EDEVICE: "EDEVICE"}
