@@ -76,6 +76,12 @@ def counts(wl):
         "io_bytes": T * d * s + T * M * d * 4,
         # prediction head of Eq. (9): v W_Z, v' [zW_u | zW_g], h zW_d per target
         "head_flops": T * 2 * ((M + 1) * d * d + 3 * d * rd),
+        # naive form (Eq. (12)) of the attention: K, V projection (4 L d^2) and the
+        # packed query tiles' 64 head-group features (G = 64 / d_h heads per tile)
+        "attn_flops_naive": M * sum(
+            4 * int(L) * d * d + 4 * 128 * (h // (64 // (d // h))) *
+            ((int(t) + 128 // (64 // (d // h)) - 1) // (128 // (64 // (d // h)))) * int(L) * 64
+            for L, t in zip(wl.lengths, wl.target_counts) if t > 0) if (d // h) in (16, 32, 64) else None,
     }
 
 
@@ -313,7 +319,8 @@ def roofline_of(kind, kt, c, wl, peaks, sustained, steps, config_key=None):
             c["enc_bytes_per_layer"] * wl.M
         flops, bytes_ = c["enc_flops"] / per_step, enc_bytes / per_step
     elif kind == "attention":
-        flops, bytes_ = c["attn_flops"] / per_step, c["attn_bytes_per_layer"] * wl.M / per_step
+        fl = c["attn_flops_naive"] if c.get("naive") else c["attn_flops"]
+        flops, bytes_ = fl / per_step, c["attn_bytes_per_layer"] * wl.M / per_step
     else:
         flops, bytes_ = c["tgt_flops"] / per_step, c["io_bytes"] / per_step
     traffic = recorded_traffic(kind, config_key) if wl.dtype == "bf16" else None
@@ -417,6 +424,8 @@ def run_ours(args, rank, world, local_rank):
     peaks, peak_src = load_peaks()
     stream = torch.cuda.Stream(device=dev)
     st = S.Stca(storage_weights(wl), wl.d, wl.h, wl.r, wl.M, wl.dtype)
+    if args.attn_form:
+        st.set_option(S.STCA_OPT_ATTN_FORM, args.attn_form)
     X = to_dev(wl, wl.X, dev)
     xt = to_dev(wl, wl.targets, dev)
     Z = torch.empty((wl.T, wl.M, wl.d), dtype=torch.float32, device=dev)
@@ -473,6 +482,8 @@ def run_ours(args, rank, world, local_rank):
         dist.barrier()
     kt = {k: v for k, v in S.stca_kernel_times(st.handle).items() if v[1] > 0}
     st.set_option(S.STCA_OPT_TIMING, 0)
+    naive_used = st.get_option(S.STCA_OPT_LAST_FORM) == 1
+    c["naive"] = naive_used
     st.status(stream)
     elapsed_ms = max_over_ranks(local_ms, dev)
     sec = elapsed_ms / 1e3
@@ -567,7 +578,8 @@ def run_ours(args, rank, world, local_rank):
         "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": wl.dtype,
         "data": "synthetic (seeded N(0,1) embeddings, Xavier-uniform weights)",
-        "config": workload_config(wl, world),
+        "config": dict(workload_config(wl, world),
+                       attn_form="naive (Eq. 12)" if naive_used else "reordered (Eq. 13)"),
         "targets_per_s": targets_per_s,
         "roofline": roof, "roofline_step": step_roof,
         "kernels": {k: {"ms_total": v[0], "launches": v[1]} for k, v in kt.items()},
@@ -595,6 +607,8 @@ def main():
     ap.add_argument("--config", default="c3", choices=sorted(CONFIGS))
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--attn-form", type=int, default=0, choices=[0, 1, 2],
+                    help="attention form: 0 reordered (Eq. 13, default), 1 naive (Eq. 12), 2 auto")
     ap.add_argument("--no-train-batch", action="store_true",
                     help="skip the sparse-training batch builder measurement")
     args = ap.parse_args()
