@@ -474,9 +474,12 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_tc_kernel(const StepTcAr
         w_dst[i] = w_src[i];
       }
       const float* cm = fused ? nullptr : a.cmerged + t0 * h * d;
-      for (int k0 = 0; k0 < d; k0 += kch) {
-        float4 cv[kMaxC];
-        uint4 wv[kMaxW];
+      // chunk k0's operands into registers; with merged rows (no in-step merge)
+      // the next chunk's loads are issued before this chunk's products, so they
+      // are in flight while the products run
+      float4 cv[kMaxC];
+      uint4 wv[kMaxW];
+      auto load_chunk = [&](int k0) {
 #pragma unroll
         for (int i = 0; i < kMaxC; ++i) {
           cv[i] = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -502,6 +505,10 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_tc_kernel(const StepTcAr
 #pragma unroll
         for (int i = 0; i < kMaxW; ++i)
           if (w_src[i] >= 0) wv[i] = __ldg(reinterpret_cast<const uint4*>(a.Wv + k0 * d + w_src[i]));
+      };
+      if (!fused) load_chunk(0);
+      for (int k0 = 0; k0 < d; k0 += kch) {
+        if (fused) load_chunk(k0);
         // c_j[t][k0 .. k0 + kch) as cs[j][k][t]
 #pragma unroll
         for (int i = 0; i < kMaxC; ++i)
@@ -517,6 +524,7 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_tc_kernel(const StepTcAr
         for (int i = 0; i < kMaxW; ++i)
           if (w_dst[i] >= 0) *reinterpret_cast<uint4*>(ws + w_dst[i]) = wv[i];
         workers_sync();
+        if (!fused && k0 + kch < d) load_chunk(k0 + kch);
 #pragma unroll
         for (int bi = 0; bi < kMaxBlk; ++bi) {
           const int b = tid + bi * 32 * kWorkers;
