@@ -197,6 +197,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  pdl_wait();                          // the predecessor's results are visible from here on
   const uint32_t sbase = smem_u32(sm);
 
   if (warp == 0) {
@@ -469,6 +470,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   }
   tc_fence_before();
   __syncthreads();
+  pdl_trigger();
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
@@ -482,7 +484,8 @@ int launch_cfg(stca_handle* H, const CUtensorMap& tmQ, const CUtensorMap& tmK, c
   auto k = attn_tc_kernel<D, QB, KS, PB, SEPV>;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
   if (e != cudaSuccess) return set_error(STCA_ECUDA, std::string("attn_tc smem: ") + cudaGetErrorString(e));
-  k<<<grid, kAttnThreads, C::kSmem, s>>>(tmQ, tmK, tmV ? *tmV : tmK, p);
+  e = launch_pdl(k, dim3(grid), dim3(kAttnThreads), C::kSmem, s, tmQ, tmK, tmV ? *tmV : tmK, p);
+  if (e != cudaSuccess) return set_error(STCA_ECUDA, std::string("attn_tc launch: ") + cudaGetErrorString(e));
   return STCA_OK;
 }
 

@@ -167,6 +167,7 @@ encode_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  pdl_wait();                          // the predecessor's results are visible from here on
   const uint32_t sbase = smem_u32(sm);
 
   if (warp == 0) {
@@ -480,6 +481,7 @@ encode_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
   }
   tc_fence_before();
   __syncthreads();
+  pdl_trigger();
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
@@ -510,7 +512,8 @@ int launch_cfg(stca_handle* H, const CUtensorMap& tmX, const EncParams& p, cudaS
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
   if (e != cudaSuccess) return set_error(STCA_ECUDA, std::string("encode_tc smem: ") + cudaGetErrorString(e));
   const int grid = std::min(p.ntiles, H->num_sms);
-  k<<<grid, kEncThreads, C::kSmem, s>>>(tmX, H->tmW1, H->tmW2, p);
+  e = launch_pdl(k, dim3(grid), dim3(kEncThreads), C::kSmem, s, tmX, H->tmW1, H->tmW2, p);
+  if (e != cudaSuccess) return set_error(STCA_ECUDA, std::string("encode_tc launch: ") + cudaGetErrorString(e));
   return STCA_OK;
 }
 

@@ -277,6 +277,7 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_tc_kernel(const StepTcAr
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  pdl_wait();                          // the predecessor's results are visible from here on
 
   if (warp == 0) {
     // ------------------------------------------------------------ weight streamer
@@ -733,6 +734,7 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_tc_kernel(const StepTcAr
   }
   tc_fence_before();
   __syncthreads();
+  pdl_trigger();
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, 128);
@@ -822,7 +824,8 @@ int launch_step_tc(const stca_handle* H, int layer, const void* targets, int64_t
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return set_error(STCA_ECUDA, std::string("step_tc smem: ") + cudaGetErrorString(e));
   const unsigned grid = static_cast<unsigned>((T + kTgt - 1) / kTgt);
-  step_tc_kernel<<<grid, kStepThreads, smem, s>>>(a);
+  e = launch_pdl(step_tc_kernel, dim3(grid), dim3(kStepThreads), smem, s, a);
+  if (e != cudaSuccess) return set_error(STCA_ECUDA, std::string("step_tc launch: ") + cudaGetErrorString(e));
   return STCA_OK;
 }
 

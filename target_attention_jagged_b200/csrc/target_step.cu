@@ -231,6 +231,7 @@ combine_kernel(StepPlan P, const float* __restrict__ pacc, const float* __restri
                const float* __restrict__ pl, float* __restrict__ out, int d, int h, int64_t nq) {
   const int lane = threadIdx.x & 31;
   const int64_t qr = static_cast<int64_t>(blockIdx.x) * kCombineRows + (threadIdx.x >> 5);
+  tc::pdl_wait();
   if (qr >= nq) return;                   // target t, head j: row t * h + j of U
   const int64_t t = qr / h;
   const int j = static_cast<int>(qr - t * h);
@@ -286,6 +287,7 @@ combine_kernel(StepPlan P, const float* __restrict__ pacc, const float* __restri
       if (on) *reinterpret_cast<float4*>(orow + k) = acc;
     }
   }
+  tc::pdl_trigger();
 }
 
 // Naive-form merge (Eq. (12) with projected K, V): o_j[t] = sum_w s_w acc_w / sum_w
@@ -636,8 +638,8 @@ void launch_combine(const stca_handle* H, const StepPlan& plan, const float* par
   const float* pm = part + G * H->d;
   const float* pl = pm + G;
   const int64_t nq = T * H->h;
-  combine_kernel<<<static_cast<unsigned>((nq + kCombineRows - 1) / kCombineRows), kCombineThreads, 0,
-                   s>>>(plan, pacc, pm, pl, out, H->d, H->h, nq);
+  tc::launch_pdl(combine_kernel, dim3(static_cast<unsigned>((nq + kCombineRows - 1) / kCombineRows)),
+                 dim3(kCombineThreads), 0, s, plan, pacc, pm, pl, out, H->d, H->h, nq);
 }
 
 void launch_combine_naive(const stca_handle* H, const StepPlan& plan, const float* part, int64_t G,
