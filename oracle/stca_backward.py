@@ -1,0 +1,102 @@
+"""Plain fp64 CPU oracle of the backward pass of two pieces of the STCA forward
+-- TEST INFRASTRUCTURE ONLY.
+
+Only tests/, __graft_entry__.smoke() and bench.py's CPU-baseline / reference
+legs may import or run this module.  The product path (the CUDA library and its
+Python binding) never calls it and shares no code with it.
+
+Sources: "Make It Long, Keep It Fast" digest §2.1, Eqs. (1)-(2) (the history
+encoding X~ = LN(SwiGLUFFN(X))) and Eq. (13) (the reordered single-query
+attention, alpha = softmax(u X~^T), c = alpha X~); the STCA blog §2.5 (request-
+level batching trains with the history encoded once for all of a request's
+targets, so the gradient of X~ sums over every target and head).
+
+Readings (the pages give the forward only):
+  B1  The backward is the exact derivative of the forward as this oracle's
+      forward module defines it (readings O1-O3 for the encoder: no biases,
+      LN with affine (gamma, beta), eps 1e-5, biased variance).
+  B2  The loss is synthetic: <output, G> for a given tensor G, so the gradient
+      that enters each piece is G itself.  The pages train with BCE on the
+      prediction head, which needs labels.
+  B3  Attention: a query row is u with its scale already in it (the forward's
+      u_j = (q W_Q^j) W_K^j^T / sqrt(d_h)); its output is the merged
+      c = softmax(u X~^T) X~ before W_V and W_O.  The backward gives dU and dX~
+      for one request's rows against its own keys.
+
+Everything is float64 from the (bf16- or fp32-valued) inputs; matrix products
+use numpy's matmul as a library primitive.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+from .stca_oracle import LN_EPS, sigmoid, softmax
+
+
+def _f64(a):
+    return np.asarray(a, dtype=np.float64)
+
+
+def encode_history_backward(X, W, i, dXt, eps=LN_EPS):
+    """Gradients of <LN(((X W_u) * SiLU(X W_g)) W_d), dXt> (Eqs. (1)-(2), layer i).
+
+    Returns dX (N x d), dWu, dWg (d x rd), dWd (rd x d), dgamma, dbeta (d)."""
+    x = _f64(X)
+    Wu, Wg, Wd = _f64(W["Wu"][i]), _f64(W["Wg"][i]), _f64(W["Wd"][i])
+    gamma = _f64(W["ln_g"][i])
+    dxt = _f64(dXt)
+    a = x @ Wu                                   # up projection
+    g = x @ Wg                                   # gate pre-activation
+    sg = sigmoid(g)
+    s = g * sg                                   # SiLU(g)
+    H = a * s
+    y = H @ Wd
+    mu = y.mean(axis=-1, keepdims=True)
+    var = ((y - mu) ** 2).mean(axis=-1, keepdims=True)
+    rstd = 1.0 / np.sqrt(var + eps)
+    yh = (y - mu) * rstd                         # normalised, before the affine
+    dgamma = (dxt * yh).sum(axis=0)
+    dbeta = dxt.sum(axis=0)
+    dyh = dxt * gamma
+    # LayerNorm: dy = rstd (dyh - mean(dyh) - yh mean(dyh * yh)) over the d features
+    dy = rstd * (dyh - dyh.mean(axis=-1, keepdims=True) - yh * (dyh * yh).mean(axis=-1, keepdims=True))
+    dWd = H.T @ dy
+    dH = dy @ Wd.T
+    da = dH * s
+    # d SiLU(g) / dg = sigmoid(g) (1 + g (1 - sigmoid(g)))
+    dg = dH * a * sg * (1.0 + g * (1.0 - sg))
+    dWu = x.T @ da
+    dWg = x.T @ dg
+    dX = da @ Wu.T + dg @ Wg.T
+    return {"dX": dX, "dWu": dWu, "dWg": dWg, "dWd": dWd, "dgamma": dgamma, "dbeta": dbeta}
+
+
+def attention_rows_backward(U, Xt, dC):
+    """Gradients of <softmax(U X~^T) X~, dC> for one request (Eq. (13), reading B3).
+
+    U: (R, d) query rows, Xt: (L, d) keys (the encoded history), dC: (R, d).
+    With P = softmax(U X~^T) and C = P X~:
+      dP = dC X~^T,  dS = P (dP - rowsum(P dP)),  dU = dS X~,  dX~ = P^T dC + dS^T U."""
+    U, Xt, dC = _f64(U), _f64(Xt), _f64(dC)
+    P = softmax(U @ Xt.T)
+    dP = dC @ Xt.T
+    dS = P * (dP - (P * dP).sum(axis=-1, keepdims=True))
+    return dS @ Xt, P.T @ dC + dS.T @ U
+
+
+def attention_backward_batch(U, Xt, offsets, target_offsets, h, dC):
+    """attention_rows_backward over a jagged batch: request r's rows are the
+    T_r h rows of U starting at target_offsets[r] * h, its keys rows
+    offsets[r] .. offsets[r+1]-1 of X~.  Returns dU (T h x d) and dX~ (N x d)."""
+    U, Xt, dC = _f64(U), _f64(Xt), _f64(dC)
+    dU = np.zeros_like(U)
+    dX = np.zeros_like(Xt)
+    for r in range(len(offsets) - 1):
+        q0, q1 = int(target_offsets[r]) * h, int(target_offsets[r + 1]) * h
+        k0, k1 = int(offsets[r]), int(offsets[r + 1])
+        if q1 == q0:
+            continue
+        du, dx = attention_rows_backward(U[q0:q1], Xt[k0:k1], dC[q0:q1])
+        dU[q0:q1] = du
+        dX[k0:k1] = dx
+    return dU, dX

@@ -1,0 +1,219 @@
+"""Pins of the backward oracle (oracle/stca_backward.py) against things other
+than itself: central finite differences of the fp64 forward (the oracle's own
+forward module, pinned elsewhere), PyTorch float64 autograd through library
+routines (F.layer_norm, F.silu, torch.softmax), and the invariances of
+LayerNorm and softmax.  Planted mistakes must fail at least one pin."""
+import numpy as np
+import pytest
+
+from oracle import stca_backward as B
+from oracle import stca_oracle as O
+
+
+def _small_weights(rng, d, rd):
+    return {"Wu": [rng.standard_normal((d, rd)) / np.sqrt(d)], "Wg": [rng.standard_normal((d, rd)) / np.sqrt(d)],
+            "Wd": [rng.standard_normal((rd, d)) / np.sqrt(rd)],
+            "ln_g": [rng.uniform(0.5, 1.5, d)], "ln_b": [rng.uniform(-0.5, 0.5, d)]}
+
+
+def pin_encoder_finite_differences():
+    rng = np.random.default_rng(1)
+    N, d, rd = 5, 6, 8
+    X = rng.standard_normal((N, d))
+    W = _small_weights(rng, d, rd)
+    G = rng.standard_normal((N, d))
+    loss = lambda X_, W_: float((O.encode_history(X_, W_, 0) * G).sum())  # noqa: E731
+    g = B.encode_history_backward(X, W, 0, G)
+    eps = 1e-6
+    for name, arr in [("dX", None), ("dWu", "Wu"), ("dWg", "Wg"), ("dWd", "Wd"),
+                      ("dgamma", "ln_g"), ("dbeta", "ln_b")]:
+        base = X if arr is None else W[arr][0]
+        V = rng.standard_normal(base.shape)
+        def shifted(sgn):
+            if arr is None:
+                return loss(X + sgn * eps * V, W)
+            W2 = {k: [v[0].copy()] for k, v in W.items()}
+            W2[arr][0] = W2[arr][0] + sgn * eps * V
+            return loss(X, W2)
+        fd = (shifted(1) - shifted(-1)) / (2 * eps)
+        an = float((g[name] * V).sum())
+        assert abs(fd - an) <= 1e-6 * max(1.0, abs(fd)), (name, fd, an)
+
+
+def pin_attention_finite_differences():
+    rng = np.random.default_rng(2)
+    R, L, d = 4, 7, 5
+    U = rng.standard_normal((R, d))
+    Xt = rng.standard_normal((L, d))
+    G = rng.standard_normal((R, d))
+    loss = lambda U_, X_: float(((O.softmax(U_ @ X_.T) @ X_) * G).sum())  # noqa: E731
+    dU, dX = B.attention_rows_backward(U, Xt, G)
+    eps = 1e-6
+    for an_grad, which in [(dU, "U"), (dX, "X")]:
+        V = rng.standard_normal(an_grad.shape)
+        if which == "U":
+            fd = (loss(U + eps * V, Xt) - loss(U - eps * V, Xt)) / (2 * eps)
+        else:
+            fd = (loss(U, Xt + eps * V) - loss(U, Xt - eps * V)) / (2 * eps)
+        an = float((an_grad * V).sum())
+        assert abs(fd - an) <= 1e-6 * max(1.0, abs(fd)), (which, fd, an)
+
+
+def pin_torch_autograd():
+    torch = pytest.importorskip("torch")
+    import torch.nn.functional as F
+    rng = np.random.default_rng(3)
+    N, d, rd = 9, 8, 16
+    X = rng.standard_normal((N, d))
+    W = _small_weights(rng, d, rd)
+    G = rng.standard_normal((N, d))
+    t = {k: torch.tensor(v[0], dtype=torch.float64, requires_grad=True) for k, v in W.items()}
+    tx = torch.tensor(X, dtype=torch.float64, requires_grad=True)
+    y = ((tx @ t["Wu"]) * F.silu(tx @ t["Wg"])) @ t["Wd"]
+    out = F.layer_norm(y, (d,), t["ln_g"], t["ln_b"], eps=1e-5)
+    (out * torch.tensor(G)).sum().backward()
+    g = B.encode_history_backward(X, W, 0, G)
+    for name, ref in [("dX", tx.grad), ("dWu", t["Wu"].grad), ("dWg", t["Wg"].grad),
+                      ("dWd", t["Wd"].grad), ("dgamma", t["ln_g"].grad), ("dbeta", t["ln_b"].grad)]:
+        np.testing.assert_allclose(g[name], ref.numpy(), rtol=1e-10, atol=1e-12, err_msg=name)
+    R, L = 6, 11
+    U = torch.tensor(rng.standard_normal((R, d)), requires_grad=True)
+    Xt = torch.tensor(rng.standard_normal((L, d)), requires_grad=True)
+    Gc = rng.standard_normal((R, d))
+    ((torch.softmax(U @ Xt.T, dim=-1) @ Xt) * torch.tensor(Gc)).sum().backward()
+    dU, dX = B.attention_rows_backward(U.detach().numpy(), Xt.detach().numpy(), Gc)
+    np.testing.assert_allclose(dU, U.grad.numpy(), rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(dX, Xt.grad.numpy(), rtol=1e-10, atol=1e-12)
+
+
+def pin_invariances():
+    rng = np.random.default_rng(4)
+    N, d, rd = 6, 8, 12
+    X = rng.standard_normal((N, d))
+    W = _small_weights(rng, d, rd)
+    G = rng.standard_normal((N, d))
+    g = B.encode_history_backward(X, W, 0, G)
+    # LN(y + c 1) = LN(y): the gradient reaching y sums to zero in every row, so
+    # dW_d = H^T dy has zero row sums
+    assert np.allclose(g["dWd"].sum(axis=1), 0.0, atol=1e-10)
+    # adding one vector v to every key shifts each row's scores by u.v (softmax
+    # unchanged) and each output c by v: d<C, G>/dv = sum of the key gradients
+    R, L = 3, 9
+    U = rng.standard_normal((R, d))
+    Xt = rng.standard_normal((L, d))
+    Gc = rng.standard_normal((R, d))
+    dU, dX = B.attention_rows_backward(U, Xt, Gc)
+    np.testing.assert_allclose(dX.sum(axis=0), Gc.sum(axis=0), rtol=1e-10, atol=1e-10)
+    # scaling every key by (1 + t) scales the scores: along U the derivative is
+    # <dU, U> = d/dt <C(U (1 + t)), G> at t = 0, by the chain rule on the scores
+    eps = 1e-6
+    f = lambda t: float(((O.softmax(U * (1 + t) @ Xt.T) @ Xt) * Gc).sum())  # noqa: E731
+    assert abs((f(eps) - f(-eps)) / (2 * eps) - float((dU * U).sum())) < 1e-6
+
+
+def test_encoder_backward_finite_differences():
+    pin_encoder_finite_differences()
+
+
+def test_attention_backward_finite_differences():
+    pin_attention_finite_differences()
+
+
+def test_backward_torch_autograd():
+    pin_torch_autograd()
+
+
+def test_backward_invariances():
+    pin_invariances()
+
+
+def test_attention_batch_matches_per_request():
+    rng = np.random.default_rng(5)
+    off = np.array([0, 5, 5 + 1, 5 + 1 + 9])
+    toff = np.array([0, 2, 2, 3])
+    h, d = 2, 4
+    U = rng.standard_normal((3 * h, d))
+    Xt = rng.standard_normal((15, d))
+    dC = rng.standard_normal((3 * h, d))
+    dU, dX = B.attention_backward_batch(U, Xt, off, toff, h, dC)
+    du0, dx0 = B.attention_rows_backward(U[:4], Xt[:5], dC[:4])
+    np.testing.assert_allclose(dU[:4], du0)
+    np.testing.assert_allclose(dX[:5], dx0)
+    assert np.all(dX[5:6] == 0)                 # request 1 has no targets: no gradient
+    du2, dx2 = B.attention_rows_backward(U[4:], Xt[6:], dC[4:])
+    np.testing.assert_allclose(dX[6:], dx2)
+
+
+# ------------------------------------------------------------------ mutations
+
+def _enc_no_mean_term(X, W, i, dXt, eps=1e-5):
+    x = np.asarray(X, float)
+    Wu, Wg, Wd = (np.asarray(W[k][i], float) for k in ("Wu", "Wg", "Wd"))
+    a, g = x @ Wu, x @ Wg
+    sg = O.sigmoid(g); s = g * sg; H = a * s; y = H @ Wd
+    mu = y.mean(-1, keepdims=True); rstd = 1 / np.sqrt(((y - mu) ** 2).mean(-1, keepdims=True) + eps)
+    yh = (y - mu) * rstd
+    dyh = dXt * np.asarray(W["ln_g"][i])
+    dy = rstd * (dyh - yh * (dyh * yh).mean(-1, keepdims=True))      # mean(dyh) dropped
+    dH = dy @ Wd.T; da = dH * s; dg = dH * a * sg * (1 + g * (1 - sg))
+    return {"dX": da @ Wu.T + dg @ Wg.T, "dWu": x.T @ da, "dWg": x.T @ dg, "dWd": H.T @ dy,
+            "dgamma": (dXt * yh).sum(0), "dbeta": np.asarray(dXt).sum(0)}
+
+
+def _enc_sigmoid_derivative(X, W, i, dXt, eps=1e-5):
+    x = np.asarray(X, float)
+    Wu, Wg, Wd = (np.asarray(W[k][i], float) for k in ("Wu", "Wg", "Wd"))
+    a, g = x @ Wu, x @ Wg
+    sg = O.sigmoid(g); s = g * sg; H = a * s; y = H @ Wd
+    mu = y.mean(-1, keepdims=True); rstd = 1 / np.sqrt(((y - mu) ** 2).mean(-1, keepdims=True) + eps)
+    yh = (y - mu) * rstd
+    dyh = dXt * np.asarray(W["ln_g"][i])
+    dy = rstd * (dyh - dyh.mean(-1, keepdims=True) - yh * (dyh * yh).mean(-1, keepdims=True))
+    dH = dy @ Wd.T; da = dH * s
+    dg = dH * a * sg                                     # d SiLU / dg taken as sigmoid(g)
+    return {"dX": da @ Wu.T + dg @ Wg.T, "dWu": x.T @ da, "dWg": x.T @ dg, "dWd": H.T @ dy,
+            "dgamma": (dXt * yh).sum(0), "dbeta": np.asarray(dXt).sum(0)}
+
+
+def _attn_sign(U, Xt, dC):
+    U, Xt, dC = (np.asarray(a, float) for a in (U, Xt, dC))
+    P = O.softmax(U @ Xt.T); dP = dC @ Xt.T
+    dS = P * (dP + (P * dP).sum(-1, keepdims=True))        # wrong sign
+    return dS @ Xt, P.T @ dC + dS.T @ U
+
+
+def _attn_no_value_term(U, Xt, dC):
+    U, Xt, dC = (np.asarray(a, float) for a in (U, Xt, dC))
+    P = O.softmax(U @ Xt.T); dP = dC @ Xt.T
+    dS = P * (dP - (P * dP).sum(-1, keepdims=True))
+    return dS @ Xt, dS.T @ U                                 # P^T dC dropped
+
+
+def _attn_transposed(U, Xt, dC):
+    U, Xt, dC = (np.asarray(a, float) for a in (U, Xt, dC))
+    P = O.softmax(U @ Xt.T); dP = dC @ Xt.T
+    dS = P * (dP - (P * dP).sum(-1, keepdims=True))
+    return dS @ Xt, P.T @ dC + dS.T @ dC                     # U replaced by dC
+
+
+MUTANTS = {
+    "ln_mean_term_dropped": ("encode_history_backward", _enc_no_mean_term),
+    "silu_derivative_wrong": ("encode_history_backward", _enc_sigmoid_derivative),
+    "softmax_sign": ("attention_rows_backward", _attn_sign),
+    "value_path_dropped": ("attention_rows_backward", _attn_no_value_term),
+    "query_replaced": ("attention_rows_backward", _attn_transposed),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_pins_reject_mutant(name, monkeypatch):
+    attr, fn = MUTANTS[name]
+    monkeypatch.setattr(B, attr, fn)
+    failed = 0
+    for pin in (pin_encoder_finite_differences, pin_attention_finite_differences, pin_torch_autograd,
+                pin_invariances):
+        try:
+            pin()
+        except AssertionError:
+            failed += 1
+    assert failed, f"mutant {name} passes every pin"
