@@ -306,6 +306,41 @@ int stca_sl_gather(const void* X, int64_t N, int64_t row_bytes, const int64_t* s
                    const int64_t* packed_offsets, int64_t B, int64_t P, void* X_packed,
                    int32_t* seg, void* stream);
 
+/* ------------------------------------------------------------------------
+ * Backward pass of two pieces of the forward, under a loss whose gradient is
+ * given ("Make It Long, Keep It Fast" digest §2.1, Eqs. (1)-(2) and (13);
+ * request-level batching sums a history's gradient over all its targets).
+ * All gradients are fp32 device buffers the caller owns; they are overwritten.
+ * ------------------------------------------------------------------------ */
+
+/*
+ * History encoding of layer `layer` (0-based): X~ = LN(((X W_u) * SiLU(X W_g)) W_d).
+ * Given dXt (N x d fp32, the gradient of X~), writes dX (N x d; may be NULL),
+ * dWu, dWg (d x rd), dWd (rd x d), dgamma, dbeta (d), for the handle's weights
+ * of that layer.  X: device, N x d in the handle's dtype (the rows given to
+ * stca_encode, or any others).  The products run on cuBLASLt in fp32 (TF32
+ * tensor cores for bf16 handles); the workspace (about N (2d + 3 rd) floats)
+ * is the handle's.  Errors: STCA_EINVAL, STCA_ENOMEM, STCA_ECUDA.
+ */
+int stca_encode_backward(stca_handle* handle, int layer, const void* X, int64_t N,
+                         const float* dXt, float* dX, float* dWu, float* dWg, float* dWd,
+                         float* dgamma, float* dbeta, void* stream);
+
+/*
+ * Single-query attention of layer `layer` on merged rows (Eq. (13)): for each
+ * request r and each of its T_r h query rows u (row t h + j of U: target t,
+ * head j, scale included, u = (q W_Q^j) W_K^j^T / sqrt(d_h)),
+ * c = softmax(u X~_r^T) X~_r with X~ the last stca_encode's encoding of that
+ * layer.  Given dC (T h x d fp32, the gradient of c), writes dU (T h x d) and
+ * dXt (N x d: every history row; rows of requests without targets get 0).
+ * target_offsets: HOST, R+1 int64 as for stca_forward.  Needs d in {64, 128,
+ * 256}.  Synchronises `stream` once to upload its work list.
+ * Errors: STCA_ESTATE (no encode yet), STCA_EINVAL, STCA_ENOMEM, STCA_ECUDA.
+ */
+int stca_attention_backward(stca_handle* handle, int layer, const float* U,
+                            const int64_t* target_offsets, int64_t T, const float* dC,
+                            float* dU, float* dXt, void* stream);
+
 /* Tunables and introspection (STCA_OPT_*).  Values are validated. */
 enum {
   STCA_OPT_ATTN_PATH = 1,     /* 0 auto, 1 CUDA cores, 2 tensor cores (bf16 only) */

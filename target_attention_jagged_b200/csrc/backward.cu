@@ -1,0 +1,460 @@
+// Backward pass of two pieces of the STCA forward ("Make It Long, Keep It Fast"
+// digest §2.1; training with request-level batching, STCA blog §2.5), under a
+// loss whose gradient is given:
+//
+//  * the history encoding X~ = LN(((X W_u) * SiLU(X W_g)) W_d) (Eqs. (1)-(2)):
+//      dX, dW_u, dW_g, dW_d, dgamma, dbeta from dX~.  The products are plain
+//      fp32 GEMMs run by cuBLASLt (TF32 tensor cores for bf16 handles, exact
+//      fp32 otherwise); the SwiGLU and LayerNorm derivatives are two kernels here.
+//  * the single-query attention of Eq. (13) on merged rows c = softmax(u X~^T) X~:
+//      dU and dX~ from dC, with the softmax recomputed flash-style:
+//        row kernel: per query row, pass 1 over the keys gives m, l and
+//          delta = sum_l P_l dP_l (dP_l = dc . x~_l); pass 2 gives
+//          dU = sum_l dS_l x~_l with dS_l = P_l (dP_l - delta);
+//        key kernel: per key, dX~_l = sum_rows (P dc + dS u) over the request's rows.
+//    Both run on the CUDA cores: a thread holds a quarter of a row's (or key's)
+//    d features, and four lanes reduce the dot products by shuffles.
+#include <cublasLt.h>
+#include <math.h>
+
+#include <algorithm>
+#include <string>
+#include <vector>
+
+#include "stca_internal.h"
+
+namespace stca {
+namespace {
+
+constexpr int kBwThreads = 256;     // 64 rows (or keys) x 4 lanes
+constexpr int kBwTile = 32;         // keys (or rows) staged per shared-memory tile
+
+__device__ __forceinline__ float ld_x(const void* X, bool bf, int64_t i) {
+  if (bf) return __uint_as_float(static_cast<uint32_t>(static_cast<const uint16_t*>(X)[i]) << 16);
+  return static_cast<const float*>(X)[i];
+}
+
+__device__ __forceinline__ float quad_sum(float v) {
+  v += __shfl_xor_sync(0xffffffffu, v, 1);
+  v += __shfl_xor_sync(0xffffffffu, v, 2);
+  return v;
+}
+
+// Work unit of the attention backward: request, first row (or key) of the
+// block, rows (or keys) in it.
+struct BwUnit {
+  int32_t req;
+  int32_t n;
+  int64_t first;
+};
+
+struct AttnBwArgs {
+  const void* Xt;           // N x d (bf16 or fp32): X~ of the layer
+  int xbf;
+  const float* U;           // T h x d
+  const float* dC;          // T h x d
+  float* dU;                // T h x d
+  float* dX;                // N x d
+  float* stats;             // T h x 3: m, l, delta
+  const int64_t* off;       // R + 1 (keys)
+  const int64_t* qoff;      // R + 1 (query rows: toff * h)
+  const BwUnit* units;
+  int d;
+};
+
+// Row kernel: block of up to 64 query rows of one request; thread (row, quarter
+// of the d = 4 DQ features).
+template <int DQ>
+__global__ void __launch_bounds__(kBwThreads) attn_bw_rows_kernel(AttnBwArgs a) {
+  extern __shared__ float sk[];                 // kBwTile x d keys (fp32)
+  const BwUnit un = a.units[blockIdx.x];
+  constexpr int kMaxQ = DQ;
+  const int d = 4 * DQ, dq = DQ;
+  const int tid = threadIdx.x, rl = tid >> 2, qu = tid & 3;
+  const bool active = rl < un.n;
+  const int64_t row = un.first + rl;
+  const int64_t k0 = a.off[un.req], L = a.off[un.req + 1] - k0;
+  float u[kMaxQ], dc[kMaxQ], du[kMaxQ];
+#pragma unroll
+  for (int f = 0; f < kMaxQ; ++f) {
+    u[f] = dc[f] = du[f] = 0.f;
+    if (f < dq && active) {
+      u[f] = a.U[row * d + qu * dq + f];
+      dc[f] = a.dC[row * d + qu * dq + f];
+    }
+  }
+  float m = -INFINITY, l = 0.f, dl = 0.f;       // running max, sum, sum of P dP (unnormalised)
+  for (int pass = 0; pass < 2; ++pass) {
+    const float inv_l = pass ? 1.f / l : 0.f, delta = pass ? dl / l : 0.f;
+    for (int64_t kt = 0; kt < L; kt += kBwTile) {
+      const int nk = static_cast<int>(L - kt < kBwTile ? L - kt : kBwTile);
+      __syncthreads();
+      for (int e = tid; e < nk * d; e += kBwThreads) sk[e] = ld_x(a.Xt, a.xbf, (k0 + kt) * d + e);
+      __syncthreads();
+      for (int k = 0; k < nk; ++k) {
+        const float* xk = sk + k * d + qu * dq;
+        float s = 0.f, dp = 0.f;
+#pragma unroll
+        for (int f = 0; f < kMaxQ; ++f)
+          if (f < dq) {
+            s = fmaf(u[f], xk[f], s);
+            dp = fmaf(dc[f], xk[f], dp);
+          }
+        s = quad_sum(s);
+        dp = quad_sum(dp);
+        if (pass == 0) {
+          if (s > m) {
+            const float c = __expf(m - s);
+            l *= c;
+            dl *= c;
+            m = s;
+          }
+          const float e = __expf(s - m);
+          l += e;
+          dl = fmaf(e, dp, dl);
+        } else {
+          const float p = __expf(s - m) * inv_l;
+          const float ds = p * (dp - delta);
+#pragma unroll
+          for (int f = 0; f < kMaxQ; ++f)
+            if (f < dq) du[f] = fmaf(ds, xk[f], du[f]);
+        }
+      }
+    }
+  }
+  if (!active) return;
+#pragma unroll
+  for (int f = 0; f < kMaxQ; ++f)
+    if (f < dq) a.dU[row * d + qu * dq + f] = du[f];
+  if (qu == 0) {
+    a.stats[row * 3 + 0] = m;
+    a.stats[row * 3 + 1] = l;
+    a.stats[row * 3 + 2] = dl / l;
+  }
+}
+
+// Key kernel: block of up to 64 keys of one request; thread (key, quarter).
+template <int DQ>
+__global__ void __launch_bounds__(kBwThreads) attn_bw_keys_kernel(AttnBwArgs a) {
+  extern __shared__ float sr[];                 // kBwTile rows x (2 d + 3): u, dc, m l delta
+  const BwUnit un = a.units[blockIdx.x];
+  constexpr int kMaxQ = DQ;
+  const int d = 4 * DQ, dq = DQ, w = 2 * d + 3;
+  const int tid = threadIdx.x, kl = tid >> 2, qu = tid & 3;
+  const bool active = kl < un.n;
+  const int64_t key = un.first + kl;
+  const int64_t r0 = a.qoff[un.req], R = a.qoff[un.req + 1] - r0;
+  float x[kMaxQ], dx[kMaxQ];
+#pragma unroll
+  for (int f = 0; f < kMaxQ; ++f) {
+    x[f] = dx[f] = 0.f;
+    if (f < dq && active) x[f] = ld_x(a.Xt, a.xbf, key * d + qu * dq + f);
+  }
+  for (int64_t rt = 0; rt < R; rt += kBwTile) {
+    const int nr = static_cast<int>(R - rt < kBwTile ? R - rt : kBwTile);
+    __syncthreads();
+    for (int e = tid; e < nr * w; e += kBwThreads) {
+      const int r = e / w, c = e - r * w;
+      const int64_t row = r0 + rt + r;
+      float v;
+      if (c < d) v = a.U[row * d + c];
+      else if (c < 2 * d) v = a.dC[row * d + c - d];
+      else v = a.stats[row * 3 + (c - 2 * d)];
+      sr[e] = v;
+    }
+    __syncthreads();
+    for (int r = 0; r < nr; ++r) {
+      const float* ur = sr + r * w + qu * dq;
+      const float* cr = ur + d;
+      const float m = sr[r * w + 2 * d], l = sr[r * w + 2 * d + 1], delta = sr[r * w + 2 * d + 2];
+      float s = 0.f, dp = 0.f;
+#pragma unroll
+      for (int f = 0; f < kMaxQ; ++f)
+        if (f < dq) {
+          s = fmaf(ur[f], x[f], s);
+          dp = fmaf(cr[f], x[f], dp);
+        }
+      s = quad_sum(s);
+      dp = quad_sum(dp);
+      const float p = __expf(s - m) / l;
+      const float ds = p * (dp - delta);
+#pragma unroll
+      for (int f = 0; f < kMaxQ; ++f)
+        if (f < dq) dx[f] = fmaf(p, cr[f], fmaf(ds, ur[f], dx[f]));
+    }
+  }
+  if (!active) return;
+#pragma unroll
+  for (int f = 0; f < kMaxQ; ++f)
+    if (f < dq) a.dX[key * d + qu * dq + f] = dx[f];
+}
+
+// ---------------------------------------------------------------- encoder
+__device__ __forceinline__ float sigm(float z) { return 1.0f / (1.0f + __expf(-z)); }
+
+// H = A * SiLU(G), elementwise over n values.
+__global__ void swiglu_fwd_kernel(const float* __restrict__ A, const float* __restrict__ G,
+                                  float* __restrict__ H, int64_t n) {
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const float g = G[i];
+    H[i] = A[i] * g * sigm(g);
+  }
+}
+
+// dA = dH * SiLU(G), dG = dH * A * SiLU'(G), written over A and G.
+__global__ void swiglu_bwd_kernel(float* __restrict__ A, float* __restrict__ G,
+                                  const float* __restrict__ dH, int64_t n) {
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const float g = G[i], a = A[i], dh = dH[i], sg = sigm(g);
+    A[i] = dh * g * sg;
+    G[i] = dh * a * sg * (1.0f + g * (1.0f - sg));
+  }
+}
+
+// LayerNorm backward, one warp per row: Y holds y on entry and dy on exit;
+// dgamma += dX~ * yhat, dbeta += dX~ (column sums, per-warp atomics).
+__global__ void ln_bwd_kernel(float* __restrict__ Y, const float* __restrict__ dXt,
+                              const float* __restrict__ gamma, float* __restrict__ dgamma,
+                              float* __restrict__ dbeta, int64_t N, int d) {
+  const int lane = threadIdx.x & 31;
+  const int64_t row = blockIdx.x * static_cast<int64_t>(blockDim.x / 32) + (threadIdx.x >> 5);
+  if (row >= N) return;
+  float* y = Y + row * d;
+  const float* g = dXt + row * d;
+  float s = 0.f;
+  for (int c = lane; c < d; c += 32) s += y[c];
+  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  const float mu = s / d;
+  float v = 0.f;
+  for (int c = lane; c < d; c += 32) { const float t = y[c] - mu; v = fmaf(t, t, v); }
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  const float rstd = rsqrtf(v / d + 1e-5f);
+  float m1 = 0.f, m2 = 0.f;                      // mean(dyh), mean(dyh * yhat)
+  for (int c = lane; c < d; c += 32) {
+    const float yh = (y[c] - mu) * rstd, dyh = g[c] * gamma[c];
+    m1 += dyh;
+    m2 = fmaf(dyh, yh, m2);
+    atomicAdd(&dgamma[c], g[c] * yh);
+    atomicAdd(&dbeta[c], g[c]);
+  }
+  for (int o = 16; o > 0; o >>= 1) {
+    m1 += __shfl_xor_sync(0xffffffffu, m1, o);
+    m2 += __shfl_xor_sync(0xffffffffu, m2, o);
+  }
+  m1 /= d;
+  m2 /= d;
+  for (int c = lane; c < d; c += 32) {
+    const float yh = (y[c] - mu) * rstd, dyh = g[c] * gamma[c];
+    y[c] = rstd * (dyh - m1 - yh * m2);
+  }
+}
+
+__global__ void to_f32_kernel(const uint16_t* __restrict__ x, float* __restrict__ y, int64_t n) {
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x)
+    y[i] = __uint_as_float(static_cast<uint32_t>(x[i]) << 16);
+}
+
+unsigned grid_for(int64_t n) { return static_cast<unsigned>(std::min<int64_t>((n + 255) / 256, 148 * 16)); }
+
+// Row-major C (m x n) = op(A) op(B) (+ C when beta = 1), fp32, through cuBLASLt's
+// column-major view C^T = op(B)^T op(A)^T.  ta / tb: A / B stored transposed.
+int gemm_rm(stca_handle* H, bool ta, bool tb, int64_t m, int64_t n, int64_t k, const float* A,
+            int64_t lda, const float* B, int64_t ldb, float* C, int64_t ldc, float beta,
+            cudaStream_t s) {
+  if (!H->lt) {
+    cublasLtHandle_t lt = nullptr;
+    if (cublasLtCreate(&lt) != CUBLAS_STATUS_SUCCESS) return set_error(STCA_ECUDA, "cublasLtCreate failed");
+    H->lt = lt;
+  }
+  constexpr size_t kWs = size_t(32) << 20;
+  if (!H->lt_ws || H->lt_ws_cap < kWs) {
+    cudaFree(H->lt_ws);
+    H->lt_ws = nullptr;
+    H->lt_ws_cap = 0;
+    if (cudaMalloc(&H->lt_ws, kWs) != cudaSuccess) {
+      cudaGetLastError();
+      return set_error(STCA_ENOMEM, "cuBLASLt workspace");
+    }
+    H->lt_ws_cap = kWs;
+  }
+  cublasLtHandle_t lt = static_cast<cublasLtHandle_t>(H->lt);
+  const cublasComputeType_t ct = H->elem == 2 ? CUBLAS_COMPUTE_32F_FAST_TF32 : CUBLAS_COMPUTE_32F;
+  cublasLtMatmulDesc_t op = nullptr;
+  cublasLtMatrixLayout_t l1 = nullptr, l2 = nullptr, lc = nullptr;
+  cublasLtMatmulPreference_t pref = nullptr;
+  int rc = STCA_OK;
+  // first cuBLAS operand: B (n x k after op), second: A (k x m after op)
+  const cublasOperation_t o1 = tb ? CUBLAS_OP_T : CUBLAS_OP_N, o2 = ta ? CUBLAS_OP_T : CUBLAS_OP_N;
+  if (cublasLtMatmulDescCreate(&op, ct, CUDA_R_32F) != CUBLAS_STATUS_SUCCESS ||
+      cublasLtMatmulDescSetAttribute(op, CUBLASLT_MATMUL_DESC_TRANSA, &o1, sizeof(o1)) != CUBLAS_STATUS_SUCCESS ||
+      cublasLtMatmulDescSetAttribute(op, CUBLASLT_MATMUL_DESC_TRANSB, &o2, sizeof(o2)) != CUBLAS_STATUS_SUCCESS ||
+      cublasLtMatrixLayoutCreate(&l1, CUDA_R_32F, tb ? k : n, tb ? n : k, ldb) != CUBLAS_STATUS_SUCCESS ||
+      cublasLtMatrixLayoutCreate(&l2, CUDA_R_32F, ta ? m : k, ta ? k : m, lda) != CUBLAS_STATUS_SUCCESS ||
+      cublasLtMatrixLayoutCreate(&lc, CUDA_R_32F, n, m, ldc) != CUBLAS_STATUS_SUCCESS ||
+      cublasLtMatmulPreferenceCreate(&pref) != CUBLAS_STATUS_SUCCESS)
+    rc = set_error(STCA_ECUDA, "cuBLASLt descriptor set-up failed");
+  cublasLtMatmulHeuristicResult_t heur{};
+  int found = 0;
+  if (rc == STCA_OK) {
+    size_t ws = kWs;
+    cublasLtMatmulPreferenceSetAttribute(pref, CUBLASLT_MATMUL_PREF_MAX_WORKSPACE_BYTES, &ws, sizeof(ws));
+    if (cublasLtMatmulAlgoGetHeuristic(lt, op, l1, l2, lc, lc, pref, 1, &heur, &found) !=
+            CUBLAS_STATUS_SUCCESS || found < 1)
+      rc = set_error(STCA_ECUDA, "cuBLASLt found no algorithm for a backward product");
+  }
+  if (rc == STCA_OK) {
+    const float alpha = 1.f;
+    if (cublasLtMatmul(lt, op, &alpha, B, l1, A, l2, &beta, C, lc, C, lc, &heur.algo, H->lt_ws, kWs, s) !=
+        CUBLAS_STATUS_SUCCESS)
+      rc = set_error(STCA_ECUDA, "cuBLASLt backward product failed");
+  }
+  if (pref) cublasLtMatmulPreferenceDestroy(pref);
+  if (lc) cublasLtMatrixLayoutDestroy(lc);
+  if (l2) cublasLtMatrixLayoutDestroy(l2);
+  if (l1) cublasLtMatrixLayoutDestroy(l1);
+  if (op) cublasLtMatmulDescDestroy(op);
+  return rc;
+}
+
+int ensure(void** p, size_t* cap, size_t bytes) {
+  if (*cap >= bytes && *p) return STCA_OK;
+  cudaFree(*p);
+  *p = nullptr;
+  *cap = 0;
+  if (cudaMalloc(p, bytes) != cudaSuccess) {
+    cudaGetLastError();
+    return set_error(STCA_ENOMEM, "backward workspace allocation failed");
+  }
+  *cap = bytes;
+  return STCA_OK;
+}
+
+}  // namespace
+}  // namespace stca
+
+using namespace stca;
+
+extern "C" int stca_encode_backward(stca_handle* H, int layer, const void* X, int64_t N,
+                                    const float* dXt, float* dX, float* dWu, float* dWg,
+                                    float* dWd, float* dgamma, float* dbeta, void* stream) {
+  if (!H) return set_error(STCA_EINVAL, "handle is NULL");
+  if (layer < 0 || layer >= H->M) return set_error(STCA_EINVAL, "layer out of range");
+  if (N < 1 || N > (int64_t(1) << 31)) return set_error(STCA_EINVAL, "N must be in [1, 2^31]");
+  if (!X || !dXt || !dWu || !dWg || !dWd || !dgamma || !dbeta)
+    return set_error(STCA_EINVAL, "stca_encode_backward: NULL argument");
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev != H->device) cudaSetDevice(H->device);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int d = H->d, rd = H->rd;
+  const LayerW32& Wl = H->L32[layer];
+  // workspace: Xf (N d), A (N rd), G (N rd), Hh (N rd), Y (N d)
+  const size_t nd = static_cast<size_t>(N) * d, nr = static_cast<size_t>(N) * rd;
+  if (int rc = ensure(&H->bw_ws, &H->bw_ws_cap, (2 * nd + 3 * nr) * sizeof(float))) return rc;
+  float* Xf = static_cast<float*>(H->bw_ws);
+  float* A = Xf + nd;
+  float* G = A + nr;
+  float* Hh = G + nr;
+  float* Y = Hh + nr;
+  if (H->elem == 2) {
+    to_f32_kernel<<<grid_for(nd), 256, 0, s>>>(static_cast<const uint16_t*>(X), Xf, nd);
+  } else {
+    STCA_CUDA_TRY(cudaMemcpyAsync(Xf, X, nd * sizeof(float), cudaMemcpyDeviceToDevice, s));
+  }
+  // forward recomputation: A = X W_u, G = X W_g, H = A SiLU(G), Y = H W_d
+  if (int rc = gemm_rm(H, false, false, N, rd, d, Xf, d, Wl.Wu, rd, A, rd, 0.f, s)) return rc;
+  if (int rc = gemm_rm(H, false, false, N, rd, d, Xf, d, Wl.Wg, rd, G, rd, 0.f, s)) return rc;
+  swiglu_fwd_kernel<<<grid_for(nr), 256, 0, s>>>(A, G, Hh, nr);
+  if (int rc = gemm_rm(H, false, false, N, d, rd, Hh, rd, Wl.Wd, d, Y, d, 0.f, s)) return rc;
+  // LayerNorm: Y <- dy; dgamma, dbeta
+  STCA_CUDA_TRY(cudaMemsetAsync(dgamma, 0, d * sizeof(float), s));
+  STCA_CUDA_TRY(cudaMemsetAsync(dbeta, 0, d * sizeof(float), s));
+  ln_bwd_kernel<<<static_cast<unsigned>((N + 7) / 8), 256, 0, s>>>(Y, dXt, Wl.ln_g, dgamma, dbeta, N, d);
+  // dW_d = H^T dy; dH = dy W_d^T (over H)
+  if (int rc = gemm_rm(H, true, false, rd, d, N, Hh, rd, Y, d, dWd, d, 0.f, s)) return rc;
+  if (int rc = gemm_rm(H, false, true, N, rd, d, Y, d, Wl.Wd, d, Hh, rd, 0.f, s)) return rc;
+  swiglu_bwd_kernel<<<grid_for(nr), 256, 0, s>>>(A, G, Hh, nr);
+  // dW_u = X^T dA, dW_g = X^T dG; dX = dA W_u^T + dG W_g^T
+  if (int rc = gemm_rm(H, true, false, d, rd, N, Xf, d, A, rd, dWu, rd, 0.f, s)) return rc;
+  if (int rc = gemm_rm(H, true, false, d, rd, N, Xf, d, G, rd, dWg, rd, 0.f, s)) return rc;
+  if (dX) {
+    if (int rc = gemm_rm(H, false, true, N, d, rd, A, rd, Wl.Wu, rd, dX, d, 0.f, s)) return rc;
+    if (int rc = gemm_rm(H, false, true, N, d, rd, G, rd, Wl.Wg, rd, dX, d, 1.f, s)) return rc;
+  }
+  STCA_CUDA_TRY(cudaGetLastError());
+  set_error(STCA_OK, "");
+  return STCA_OK;
+}
+
+extern "C" int stca_attention_backward(stca_handle* H, int layer, const float* U,
+                                       const int64_t* target_offsets, int64_t T, const float* dC,
+                                       float* dU, float* dXt, void* stream) {
+  if (!H) return set_error(STCA_EINVAL, "handle is NULL");
+  if (!H->encoded) return set_error(STCA_ESTATE, "stca_attention_backward before a successful stca_encode");
+  if (layer < 0 || layer >= H->M) return set_error(STCA_EINVAL, "layer out of range");
+  if (H->d != 64 && H->d != 128 && H->d != 256)
+    return set_error(STCA_EINVAL, "attention backward needs d in {64, 128, 256}");
+  if (int rc = stca_validate_offsets(target_offsets, H->R, T, 0)) return rc;
+  if (!dXt || (T > 0 && (!U || !dC || !dU)))
+    return set_error(STCA_EINVAL, "stca_attention_backward: NULL argument");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int d = H->d, h = H->h;
+  const int64_t R = H->R, N = H->N;
+  // work units and offsets, uploaded through the handle's backward plan buffer
+  std::vector<BwUnit> rows, keys;
+  std::vector<int64_t> offs(2 * (R + 1));
+  for (int64_t r = 0; r <= R; ++r) {
+    offs[r] = H->offsets_h[r];
+    offs[R + 1 + r] = target_offsets[r] * h;
+  }
+  for (int64_t r = 0; r < R; ++r) {
+    const int64_t q0 = target_offsets[r] * h, q1 = target_offsets[r + 1] * h;
+    for (int64_t q = q0; q < q1; q += 64)
+      rows.push_back({static_cast<int32_t>(r), static_cast<int32_t>(std::min<int64_t>(64, q1 - q)), q});
+    for (int64_t k = H->offsets_h[r]; k < H->offsets_h[r + 1]; k += 64)
+      keys.push_back({static_cast<int32_t>(r), static_cast<int32_t>(std::min<int64_t>(64, H->offsets_h[r + 1] - k)), k});
+  }
+  const size_t b_off = offs.size() * sizeof(int64_t);
+  const size_t b_rows = rows.size() * sizeof(BwUnit), b_keys = keys.size() * sizeof(BwUnit);
+  const size_t bytes = b_off + b_rows + b_keys + static_cast<size_t>(std::max<int64_t>(T * h, 1)) * 3 * sizeof(float) + 64;
+  if (int rc = ensure(&H->bw_plan, &H->bw_plan_cap, bytes)) return rc;
+  char* p = static_cast<char*>(H->bw_plan);
+  STCA_CUDA_TRY(cudaMemcpyAsync(p, offs.data(), b_off, cudaMemcpyHostToDevice, s));
+  if (!rows.empty()) STCA_CUDA_TRY(cudaMemcpyAsync(p + b_off, rows.data(), b_rows, cudaMemcpyHostToDevice, s));
+  if (!keys.empty())
+    STCA_CUDA_TRY(cudaMemcpyAsync(p + b_off + b_rows, keys.data(), b_keys, cudaMemcpyHostToDevice, s));
+  // the host vectors must outlive the copies: wait for them (a small upload)
+  STCA_CUDA_TRY(cudaStreamSynchronize(s));
+  AttnBwArgs a{};
+  a.Xt = static_cast<const char*>(H->xt) + static_cast<size_t>(N) * d * H->elem * layer;
+  a.xbf = H->elem == 2;
+  a.U = U;
+  a.dC = dC;
+  a.dU = dU;
+  a.dX = dXt;
+  a.off = reinterpret_cast<const int64_t*>(p);
+  a.qoff = a.off + R + 1;
+  a.stats = reinterpret_cast<float*>(p + ((b_off + b_rows + b_keys + 15) & ~size_t(15)));
+  a.d = d;
+  auto run = [&](auto rows_k, auto keys_k) {
+    if (!rows.empty()) {
+      a.units = reinterpret_cast<const BwUnit*>(p + b_off);
+      rows_k<<<static_cast<unsigned>(rows.size()), kBwThreads, kBwTile * d * sizeof(float), s>>>(a);
+    }
+    if (!keys.empty()) {
+      a.units = reinterpret_cast<const BwUnit*>(p + b_off + b_rows);
+      const size_t smem = static_cast<size_t>(kBwTile) * (2 * d + 3) * sizeof(float);
+      cudaFuncSetAttribute(keys_k, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+      keys_k<<<static_cast<unsigned>(keys.size()), kBwThreads, smem, s>>>(a);
+    }
+  };
+  if (d == 64) run(attn_bw_rows_kernel<16>, attn_bw_keys_kernel<16>);
+  else if (d == 128) run(attn_bw_rows_kernel<32>, attn_bw_keys_kernel<32>);
+  else run(attn_bw_rows_kernel<64>, attn_bw_keys_kernel<64>);
+  STCA_CUDA_TRY(cudaGetLastError());
+  set_error(STCA_OK, "");
+  return STCA_OK;
+}

@@ -174,6 +174,8 @@ extern "C" void stca_destroy(stca_handle* H) {
   cudaFree(H->wkv);
   cudaFree(H->kv);
   cudaFree(H->lt_ws);
+  cudaFree(H->bw_ws);
+  cudaFree(H->bw_plan);
   if (H->lt) cublasLtDestroy(static_cast<cublasLtHandle_t>(H->lt));
   cudaFree(H->wtc);
   cudaFree(H->xt);

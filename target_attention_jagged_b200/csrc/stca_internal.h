@@ -113,6 +113,8 @@ struct stca_handle {
   void* wkv = nullptr;                  // naive form: per layer [W_K | W_V], d x 2d bf16
   void* lt = nullptr;                   // cuBLASLt handle (naive-form projection)
   void* lt_ws = nullptr;    size_t lt_ws_cap = 0;  // its workspace
+  void* bw_ws = nullptr;    size_t bw_ws_cap = 0;  // encoder backward workspace (fp32)
+  void* bw_plan = nullptr;  size_t bw_plan_cap = 0;  // attention backward units and statistics
   bool tc_encode_ready = false;
   uint16_t* wstep_tc = nullptr;         // A-tile stream of the tensor-core per-target step
   std::vector<stca::TcGemm> tcO, tcC, tcUG, tcD, tcQ;   // per layer

@@ -36,7 +36,8 @@ EXPORTS = ("stca_init", "stca_destroy", "stca_encode", "stca_forward", "stca_run
            "stca_validate_offsets", "stca_device_status", "stca_set_option",
            "stca_get_option", "stca_kernel_times", "stca_get_encoded", "stca_plan_attention",
            "stca_forward_static", "stca_head", "stca_sl_beta", "stca_sl_plan",
-           "stca_sl_gather", "stca_last_error")
+           "stca_sl_gather", "stca_encode_backward", "stca_attention_backward",
+           "stca_last_error")
 
 
 class StcaError(RuntimeError):
@@ -63,6 +64,8 @@ def _load():
     lib.stca_sl_beta.argtypes = [D, I64, I64, I64, PD, PD]
     lib.stca_sl_plan.argtypes = [PI64, I64, PD, I64, I64, I64, I64, PI64, PI64, PI64, PI64]
     lib.stca_sl_gather.argtypes = [P, I64, I64, P, P, I64, I64, P, P, P]
+    lib.stca_encode_backward.argtypes = [P, I, P, I64, P, P, P, P, P, P, P, P]
+    lib.stca_attention_backward.argtypes = [P, I, P, PI64, I64, P, P, P, P]
     lib.stca_run_host.argtypes = [P, P, PI64, I64, I64, P, PI64, I64, P, P]
     lib.stca_validate_offsets.argtypes = [PI64, I64, I64, I]
     lib.stca_device_status.argtypes = [P, P]
@@ -291,6 +294,40 @@ def build_training_batch(X, hist_offsets, s, L_min: int, L_max: int, L_avg: int,
     seg = torch.empty(P, dtype=torch.int32, device=dev)
     stca_sl_gather(X, src, poff, Xp, seg, stream)
     return Xp, seg, plan
+
+
+def stca_encode_backward(handle: int, layer: int, X, dXt, d: int, rd: int, with_dx=True, stream=None):
+    """Gradients of the layer's history encoding (Eqs. (1)-(2)) from dXt (N x d
+    fp32 CUDA); X: the CUDA rows (N x d, handle dtype).  Returns a dict of fp32
+    CUDA tensors dX (or None), dWu, dWg, dWd, dgamma, dbeta."""
+    import torch
+    N = int(X.shape[0])
+    dev = X.device
+    f = lambda *sh: torch.empty(sh, dtype=torch.float32, device=dev)  # noqa: E731
+    out = {"dX": f(N, d) if with_dx else None, "dWu": f(d, rd), "dWg": f(d, rd), "dWd": f(rd, d),
+           "dgamma": f(d), "dbeta": f(d)}
+    assert dXt.dtype == torch.float32 and dXt.is_contiguous() and X.is_contiguous()
+    ptr = lambda t: t.data_ptr() if t is not None else None  # noqa: E731
+    _check(_lib.stca_encode_backward(handle, layer, X.data_ptr(), N, dXt.data_ptr(), ptr(out["dX"]),
+                                     ptr(out["dWu"]), ptr(out["dWg"]), ptr(out["dWd"]),
+                                     ptr(out["dgamma"]), ptr(out["dbeta"]), _stream_ptr(stream)))
+    return out
+
+
+def stca_attention_backward(handle: int, layer: int, U, target_offsets, dC, N: int, stream=None):
+    """Gradients of the merged attention rows (Eq. (13)) of the last encode's
+    layer: dU (T h x d) and dXt (N x d), fp32 CUDA tensors."""
+    import torch
+    toff = _offsets(target_offsets)
+    T = int(toff[-1])
+    assert U.dtype == torch.float32 and dC.dtype == torch.float32
+    dU = torch.empty_like(U)
+    dX = torch.empty((N, U.shape[1]), dtype=torch.float32, device=U.device)
+    _check(_lib.stca_attention_backward(handle, layer, U.data_ptr() if T > 0 else None, _i64p(toff), T,
+                                        dC.data_ptr() if T > 0 else None,
+                                        dU.data_ptr() if T > 0 else None, dX.data_ptr(),
+                                        _stream_ptr(stream)))
+    return dU, dX
 
 
 def stca_run_host(handle: int, X_host, offsets, targets_host, target_offsets, Z_host,
