@@ -549,6 +549,45 @@ def run_ours(args, rank, world, local_rank):
                          "flops_per_launch": c["head_flops"],
                          "peak_source": "nominal FP32 FFMA: 148 SMs x 128 lanes x 2 x 1.965 GHz"}}
 
+    # ---- backward of layer 1 (history encoding and merged attention), synthetic loss
+    backward = None
+    if not args.no_backward:
+        rng = np.random.default_rng(11)
+        dXt = torch.from_numpy(rng.standard_normal((wl.N, wl.d)).astype(np.float32)).to(dev)
+        rows = wl.T * wl.h
+        Ub = torch.from_numpy((rng.standard_normal((rows, wl.d)) * (2.0 / np.sqrt(wl.d))).astype(np.float32)).to(dev)
+        dC = torch.from_numpy(rng.standard_normal((rows, wl.d)).astype(np.float32)).to(dev)
+        st.encode(X, wl.offsets, stream)
+        with torch.cuda.stream(stream):
+            for _ in range(2):
+                S.stca_encode_backward(st.handle, 0, X, dXt, wl.d, wl.r * wl.d, stream=stream)
+                S.stca_attention_backward(st.handle, 0, Ub, wl.target_offsets, dC, wl.N, stream)
+            b0, b1, b2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+            nrep = max(1, min(args.steps, 5))
+            b0.record(stream)
+            for _ in range(nrep):
+                S.stca_encode_backward(st.handle, 0, X, dXt, wl.d, wl.r * wl.d, stream=stream)
+            b1.record(stream)
+            for _ in range(nrep):
+                S.stca_attention_backward(st.handle, 0, Ub, wl.target_offsets, dC, wl.N, stream)
+            b2.record(stream)
+        torch.cuda.synchronize()
+        st.status(stream)
+        enc_ms, att_ms = b0.elapsed_time(b1) / nrep, b1.elapsed_time(b2) / nrep
+        rd = wl.r * wl.d
+        enc_fl = 18 * wl.N * wl.d * rd              # recomputed forward (6 N d rd) + 6 backward products
+        att_fl = 18 * wl.d * c["TL"] * wl.h         # per (row, key): 2 passes of 2 dots + dU; 2 dots + dX~
+        tf32 = 1100.0
+        fp32 = 148 * 128 * 2 * 1.965e9 / 1e12
+        backward = {
+            "layer": 1, "loss": "synthetic <output, G>, G ~ N(0, 1)",
+            "encode": {"ms": enc_ms, "flops": enc_fl, "tflops": enc_fl / (enc_ms / 1e3) / 1e12,
+                       "frac_of_nominal_tf32": enc_fl / (enc_ms / 1e3) / 1e12 / tf32,
+                       "note": "cuBLASLt TF32 products + SwiGLU / LayerNorm derivative kernels"},
+            "attention": {"ms": att_ms, "flops": att_fl, "tflops": att_fl / (att_ms / 1e3) / 1e12,
+                          "frac_of_nominal_fp32": att_fl / (att_ms / 1e3) / 1e12 / fp32,
+                          "note": "CUDA-core flash-style kernels (softmax recomputed)"}}
+
     # ---- the sparse-training batch builder and a forward over its packed batch
     train_batch = None
     if not args.no_train_batch:
@@ -595,6 +634,7 @@ def run_ours(args, rank, world, local_rank):
                          "history_tokens_per_s": world * wl.N / (fwd_ms / 1e3)},
         "head": head,
         "train_batch": train_batch,
+        "backward": backward,
         "e2e": e2e,
         "gpu_launches": int(launches_per_step * args.steps),
         "clocks": sampler.summary(),
@@ -616,6 +656,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--attn-form", type=int, default=0, choices=[0, 1, 2],
                     help="attention form: 0 reordered (Eq. 13, default), 1 naive (Eq. 12), 2 auto")
+    ap.add_argument("--no-backward", action="store_true", help="skip the backward measurement")
     ap.add_argument("--no-train-batch", action="store_true",
                     help="skip the sparse-training batch builder measurement")
     args = ap.parse_args()
