@@ -13,7 +13,8 @@
 //          dU = sum_l dS_l x~_l with dS_l = P_l (dP_l - delta);
 //        key kernel: per key, dX~_l = sum_rows (P dc + dS u) over the request's rows.
 //    Both run on the CUDA cores: a thread holds a quarter of a row's (or key's)
-//    d features, and four lanes reduce the dot products by shuffles.
+//    d features, and four lanes reduce the dot products by shuffles; operands
+//    are staged in shared memory with 16-byte loads.
 #include <cublasLt.h>
 #include <math.h>
 
@@ -26,12 +27,35 @@
 namespace stca {
 namespace {
 
-constexpr int kBwThreads = 256;     // 64 rows (or keys) x 4 lanes
+constexpr int kBwThreads = 128;     // 32 rows (or keys) x 4 lanes
+constexpr int kBwBlock = kBwThreads / 4;
 constexpr int kBwTile = 32;         // keys (or rows) staged per shared-memory tile
 
 __device__ __forceinline__ float ld_x(const void* X, bool bf, int64_t i) {
   if (bf) return __uint_as_float(static_cast<uint32_t>(static_cast<const uint16_t*>(X)[i]) << 16);
   return static_cast<const float*>(X)[i];
+}
+
+// Stage n rows of d values of X (bf16 or fp32) as fp32 into s, 8 values per
+// 16-byte load (d % 8 == 0, rows 16-byte aligned).
+__device__ __forceinline__ void stage_rows(float* s, const void* X, bool bf, int64_t row0, int n, int d) {
+  const int n8 = n * d / 8;
+  for (int e = threadIdx.x; e < n8; e += blockDim.x) {
+    float4 lo, hi;
+    if (bf) {
+      const uint4 v = __ldg(reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(X) + row0 * d) + e);
+      lo = make_float4(__uint_as_float(v.x << 16), __uint_as_float(v.x & 0xFFFF0000u),
+                       __uint_as_float(v.y << 16), __uint_as_float(v.y & 0xFFFF0000u));
+      hi = make_float4(__uint_as_float(v.z << 16), __uint_as_float(v.z & 0xFFFF0000u),
+                       __uint_as_float(v.w << 16), __uint_as_float(v.w & 0xFFFF0000u));
+    } else {
+      const float4* src = reinterpret_cast<const float4*>(static_cast<const float*>(X) + row0 * d) + 2 * e;
+      lo = __ldg(src);
+      hi = __ldg(src + 1);
+    }
+    reinterpret_cast<float4*>(s)[2 * e] = lo;
+    reinterpret_cast<float4*>(s)[2 * e + 1] = hi;
+  }
 }
 
 __device__ __forceinline__ float quad_sum(float v) {
@@ -62,7 +86,7 @@ struct AttnBwArgs {
   int d;
 };
 
-// Row kernel: block of up to 64 query rows of one request; thread (row, quarter
+// Row kernel: block of up to 32 query rows of one request; thread (row, quarter
 // of the d = 4 DQ features).
 template <int DQ>
 __global__ void __launch_bounds__(kBwThreads) attn_bw_rows_kernel(AttnBwArgs a) {
@@ -89,7 +113,7 @@ __global__ void __launch_bounds__(kBwThreads) attn_bw_rows_kernel(AttnBwArgs a) 
     for (int64_t kt = 0; kt < L; kt += kBwTile) {
       const int nk = static_cast<int>(L - kt < kBwTile ? L - kt : kBwTile);
       __syncthreads();
-      for (int e = tid; e < nk * d; e += kBwThreads) sk[e] = ld_x(a.Xt, a.xbf, (k0 + kt) * d + e);
+      stage_rows(sk, a.Xt, a.xbf, k0 + kt, nk, d);
       __syncthreads();
       for (int k = 0; k < nk; ++k) {
         const float* xk = sk + k * d + qu * dq;
@@ -133,7 +157,7 @@ __global__ void __launch_bounds__(kBwThreads) attn_bw_rows_kernel(AttnBwArgs a) 
   }
 }
 
-// Key kernel: block of up to 64 keys of one request; thread (key, quarter).
+// Key kernel: block of up to 32 keys of one request; thread (key, quarter).
 template <int DQ>
 __global__ void __launch_bounds__(kBwThreads) attn_bw_keys_kernel(AttnBwArgs a) {
   extern __shared__ float sr[];                 // kBwTile rows x (2 d + 3): u, dc, m l delta
@@ -153,14 +177,21 @@ __global__ void __launch_bounds__(kBwThreads) attn_bw_keys_kernel(AttnBwArgs a) 
   for (int64_t rt = 0; rt < R; rt += kBwTile) {
     const int nr = static_cast<int>(R - rt < kBwTile ? R - rt : kBwTile);
     __syncthreads();
-    for (int e = tid; e < nr * w; e += kBwThreads) {
-      const int r = e / w, c = e - r * w;
-      const int64_t row = r0 + rt + r;
-      float v;
-      if (c < d) v = a.U[row * d + c];
-      else if (c < 2 * d) v = a.dC[row * d + c - d];
-      else v = a.stats[row * 3 + (c - 2 * d)];
-      sr[e] = v;
+    {
+      // u and dc of the tile's rows as float4, then their statistics
+      const int d4 = d / 4;
+      for (int e = tid; e < nr * 2 * d4; e += kBwThreads) {
+        const int r = e / (2 * d4), c4 = e - r * 2 * d4;
+        const int64_t row = r0 + rt + r;
+        const float4 v = c4 < d4 ? __ldg(reinterpret_cast<const float4*>(a.U + row * d) + c4)
+                                 : __ldg(reinterpret_cast<const float4*>(a.dC + row * d) + c4 - d4);
+        float* dst = sr + r * w + 4 * c4;
+        dst[0] = v.x; dst[1] = v.y; dst[2] = v.z; dst[3] = v.w;
+      }
+      for (int e = tid; e < nr * 3; e += kBwThreads) {
+        const int r = e / 3, c = e - r * 3;
+        sr[r * w + 2 * d + c] = a.stats[(r0 + rt + r) * 3 + c];
+      }
     }
     __syncthreads();
     for (int r = 0; r < nr; ++r) {
@@ -213,41 +244,82 @@ __global__ void swiglu_bwd_kernel(float* __restrict__ A, float* __restrict__ G,
   }
 }
 
-// LayerNorm backward, one warp per row: Y holds y on entry and dy on exit;
-// dgamma += dX~ * yhat, dbeta += dX~ (column sums, per-warp atomics).
-__global__ void ln_bwd_kernel(float* __restrict__ Y, const float* __restrict__ dXt,
-                              const float* __restrict__ gamma, float* __restrict__ dgamma,
-                              float* __restrict__ dbeta, int64_t N, int d) {
-  const int lane = threadIdx.x & 31;
-  const int64_t row = blockIdx.x * static_cast<int64_t>(blockDim.x / 32) + (threadIdx.x >> 5);
-  if (row >= N) return;
-  float* y = Y + row * d;
-  const float* g = dXt + row * d;
-  float s = 0.f;
-  for (int c = lane; c < d; c += 32) s += y[c];
-  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-  const float mu = s / d;
-  float v = 0.f;
-  for (int c = lane; c < d; c += 32) { const float t = y[c] - mu; v = fmaf(t, t, v); }
-  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-  const float rstd = rsqrtf(v / d + 1e-5f);
-  float m1 = 0.f, m2 = 0.f;                      // mean(dyh), mean(dyh * yhat)
-  for (int c = lane; c < d; c += 32) {
-    const float yh = (y[c] - mu) * rstd, dyh = g[c] * gamma[c];
-    m1 += dyh;
-    m2 = fmaf(dyh, yh, m2);
-    atomicAdd(&dgamma[c], g[c] * yh);
-    atomicAdd(&dbeta[c], g[c]);
+// LayerNorm backward: a CTA of 8 warps takes kLnRows consecutive rows, one warp
+// per row at a time.  Y holds y on entry and dy on exit.  Each lane keeps its
+// columns' sums of dX~ * yhat and dX~ in registers over the CTA's rows, the
+// warps add them in shared memory, and the CTA adds its totals to dgamma and
+// dbeta with one atomic per column.
+constexpr int kLnRows = 256;
+constexpr int kLnMaxCols = 8;                  // d / 32, d <= 256
+
+__global__ void __launch_bounds__(256) ln_bwd_kernel(float* __restrict__ Y, const float* __restrict__ dXt,
+                                                     const float* __restrict__ gamma, float* __restrict__ dgamma,
+                                                     float* __restrict__ dbeta, int64_t N, int d) {
+  __shared__ float sg[256], sb[256];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  for (int c = threadIdx.x; c < d; c += 256) sg[c] = sb[c] = 0.f;
+  __syncthreads();
+  float ag[kLnMaxCols], ab[kLnMaxCols];
+#pragma unroll
+  for (int j = 0; j < kLnMaxCols; ++j) ag[j] = ab[j] = 0.f;
+  const int64_t r0 = static_cast<int64_t>(blockIdx.x) * kLnRows;
+  for (int64_t row = r0 + warp; row < N && row < r0 + kLnRows; row += 8) {
+    float* y = Y + row * d;
+    const float* g = dXt + row * d;
+    float yv[kLnMaxCols], gv[kLnMaxCols];
+    float s = 0.f;
+#pragma unroll
+    for (int j = 0; j < kLnMaxCols; ++j) {
+      const int c = lane + 32 * j;
+      yv[j] = c < d ? y[c] : 0.f;
+      gv[j] = c < d ? g[c] : 0.f;
+      s += yv[j];
+    }
+    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    const float mu = s / d;
+    float v = 0.f;
+#pragma unroll
+    for (int j = 0; j < kLnMaxCols; ++j)
+      if (lane + 32 * j < d) { const float t = yv[j] - mu; v = fmaf(t, t, v); }
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    const float rstd = rsqrtf(v / d + 1e-5f);
+    float m1 = 0.f, m2 = 0.f;                    // sums of dyh and dyh * yhat
+#pragma unroll
+    for (int j = 0; j < kLnMaxCols; ++j) {
+      const int c = lane + 32 * j;
+      if (c >= d) continue;
+      const float yh = (yv[j] - mu) * rstd, dyh = gv[j] * gamma[c];
+      m1 += dyh;
+      m2 = fmaf(dyh, yh, m2);
+      ag[j] = fmaf(gv[j], yh, ag[j]);
+      ab[j] += gv[j];
+    }
+    for (int o = 16; o > 0; o >>= 1) {
+      m1 += __shfl_xor_sync(0xffffffffu, m1, o);
+      m2 += __shfl_xor_sync(0xffffffffu, m2, o);
+    }
+    m1 /= d;
+    m2 /= d;
+#pragma unroll
+    for (int j = 0; j < kLnMaxCols; ++j) {
+      const int c = lane + 32 * j;
+      if (c >= d) continue;
+      const float yh = (yv[j] - mu) * rstd, dyh = gv[j] * gamma[c];
+      y[c] = rstd * (dyh - m1 - yh * m2);
+    }
   }
-  for (int o = 16; o > 0; o >>= 1) {
-    m1 += __shfl_xor_sync(0xffffffffu, m1, o);
-    m2 += __shfl_xor_sync(0xffffffffu, m2, o);
+#pragma unroll
+  for (int j = 0; j < kLnMaxCols; ++j) {
+    const int c = lane + 32 * j;
+    if (c < d) {
+      atomicAdd(&sg[c], ag[j]);
+      atomicAdd(&sb[c], ab[j]);
+    }
   }
-  m1 /= d;
-  m2 /= d;
-  for (int c = lane; c < d; c += 32) {
-    const float yh = (y[c] - mu) * rstd, dyh = g[c] * gamma[c];
-    y[c] = rstd * (dyh - m1 - yh * m2);
+  __syncthreads();
+  for (int c = threadIdx.x; c < d; c += 256) {
+    atomicAdd(&dgamma[c], sg[c]);
+    atomicAdd(&dbeta[c], sb[c]);
   }
 }
 
@@ -372,7 +444,9 @@ extern "C" int stca_encode_backward(stca_handle* H, int layer, const void* X, in
   // LayerNorm: Y <- dy; dgamma, dbeta
   STCA_CUDA_TRY(cudaMemsetAsync(dgamma, 0, d * sizeof(float), s));
   STCA_CUDA_TRY(cudaMemsetAsync(dbeta, 0, d * sizeof(float), s));
-  ln_bwd_kernel<<<static_cast<unsigned>((N + 7) / 8), 256, 0, s>>>(Y, dXt, Wl.ln_g, dgamma, dbeta, N, d);
+  if (d > 32 * kLnMaxCols) return set_error(STCA_EINVAL, "encoder backward needs d <= 256");
+  ln_bwd_kernel<<<static_cast<unsigned>((N + kLnRows - 1) / kLnRows), 256, 0, s>>>(Y, dXt, Wl.ln_g, dgamma,
+                                                                                   dbeta, N, d);
   // dW_d = H^T dy; dH = dy W_d^T (over H)
   if (int rc = gemm_rm(H, true, false, rd, d, N, Hh, rd, Y, d, dWd, d, 0.f, s)) return rc;
   if (int rc = gemm_rm(H, false, true, N, rd, d, Y, d, Wl.Wd, d, Hh, rd, 0.f, s)) return rc;
@@ -412,10 +486,11 @@ extern "C" int stca_attention_backward(stca_handle* H, int layer, const float* U
   }
   for (int64_t r = 0; r < R; ++r) {
     const int64_t q0 = target_offsets[r] * h, q1 = target_offsets[r + 1] * h;
-    for (int64_t q = q0; q < q1; q += 64)
-      rows.push_back({static_cast<int32_t>(r), static_cast<int32_t>(std::min<int64_t>(64, q1 - q)), q});
-    for (int64_t k = H->offsets_h[r]; k < H->offsets_h[r + 1]; k += 64)
-      keys.push_back({static_cast<int32_t>(r), static_cast<int32_t>(std::min<int64_t>(64, H->offsets_h[r + 1] - k)), k});
+    for (int64_t q = q0; q < q1; q += kBwBlock)
+      rows.push_back({static_cast<int32_t>(r), static_cast<int32_t>(std::min<int64_t>(kBwBlock, q1 - q)), q});
+    for (int64_t k = H->offsets_h[r]; k < H->offsets_h[r + 1]; k += kBwBlock)
+      keys.push_back({static_cast<int32_t>(r),
+                      static_cast<int32_t>(std::min<int64_t>(kBwBlock, H->offsets_h[r + 1] - k)), k});
   }
   const size_t b_off = offs.size() * sizeof(int64_t);
   const size_t b_rows = rows.size() * sizeof(BwUnit), b_keys = keys.size() * sizeof(BwUnit);
