@@ -12,8 +12,8 @@
 //          delta = sum_l P_l dP_l (dP_l = dc . x~_l); pass 2 gives
 //          dU = sum_l dS_l x~_l with dS_l = P_l (dP_l - delta);
 //        key kernel: per key, dX~_l = sum_rows (P dc + dS u) over the request's rows.
-//    Both run on the CUDA cores: a thread holds a quarter of a row's (or key's)
-//    d features, and four lanes reduce the dot products by shuffles; operands
+//    Both run on the CUDA cores: a thread holds an eighth of a row's (or key's)
+//    d features, and eight lanes reduce the dot products by shuffles; operands
 //    are staged in shared memory with 16-byte loads.
 #include <cublasLt.h>
 #include <math.h>
@@ -27,8 +27,9 @@
 namespace stca {
 namespace {
 
-constexpr int kBwThreads = 128;     // 32 rows (or keys) x 4 lanes
-constexpr int kBwBlock = kBwThreads / 4;
+constexpr int kLanes = 8;           // lanes per row (or key), each with d / 8 features
+constexpr int kBwThreads = 128;     // 16 rows (or keys) x 8 lanes
+constexpr int kBwBlock = kBwThreads / kLanes;
 constexpr int kBwTile = 32;         // keys (or rows) staged per shared-memory tile
 
 __device__ __forceinline__ float ld_x(const void* X, bool bf, int64_t i) {
@@ -58,9 +59,11 @@ __device__ __forceinline__ void stage_rows(float* s, const void* X, bool bf, int
   }
 }
 
+// Sum over the kLanes lanes that share a row (or key).
 __device__ __forceinline__ float quad_sum(float v) {
   v += __shfl_xor_sync(0xffffffffu, v, 1);
   v += __shfl_xor_sync(0xffffffffu, v, 2);
+  v += __shfl_xor_sync(0xffffffffu, v, 4);
   return v;
 }
 
@@ -86,15 +89,15 @@ struct AttnBwArgs {
   int d;
 };
 
-// Row kernel: block of up to 32 query rows of one request; thread (row, quarter
-// of the d = 4 DQ features).
+// Row kernel: block of up to 16 query rows of one request; thread (row, eighth
+// of the d = 8 DQ features).
 template <int DQ>
 __global__ void __launch_bounds__(kBwThreads) attn_bw_rows_kernel(AttnBwArgs a) {
   extern __shared__ float sk[];                 // kBwTile x d keys (fp32)
   const BwUnit un = a.units[blockIdx.x];
   constexpr int kMaxQ = DQ;
-  const int d = 4 * DQ, dq = DQ;
-  const int tid = threadIdx.x, rl = tid >> 2, qu = tid & 3;
+  const int d = kLanes * DQ, dq = DQ;
+  const int tid = threadIdx.x, rl = tid / kLanes, qu = tid % kLanes;
   const bool active = rl < un.n;
   const int64_t row = un.first + rl;
   const int64_t k0 = a.off[un.req], L = a.off[un.req + 1] - k0;
@@ -157,14 +160,14 @@ __global__ void __launch_bounds__(kBwThreads) attn_bw_rows_kernel(AttnBwArgs a) 
   }
 }
 
-// Key kernel: block of up to 32 keys of one request; thread (key, quarter).
+// Key kernel: block of up to 16 keys of one request; thread (key, eighth).
 template <int DQ>
 __global__ void __launch_bounds__(kBwThreads) attn_bw_keys_kernel(AttnBwArgs a) {
   extern __shared__ float sr[];                 // kBwTile rows x (2 d + 3): u, dc, m l delta
   const BwUnit un = a.units[blockIdx.x];
   constexpr int kMaxQ = DQ;
-  const int d = 4 * DQ, dq = DQ, w = 2 * d + 3;
-  const int tid = threadIdx.x, kl = tid >> 2, qu = tid & 3;
+  const int d = kLanes * DQ, dq = DQ, w = 2 * d + 3;
+  const int tid = threadIdx.x, kl = tid / kLanes, qu = tid % kLanes;
   const bool active = kl < un.n;
   const int64_t key = un.first + kl;
   const int64_t r0 = a.qoff[un.req], R = a.qoff[un.req + 1] - r0;
@@ -526,9 +529,9 @@ extern "C" int stca_attention_backward(stca_handle* H, int layer, const float* U
       keys_k<<<static_cast<unsigned>(keys.size()), kBwThreads, smem, s>>>(a);
     }
   };
-  if (d == 64) run(attn_bw_rows_kernel<16>, attn_bw_keys_kernel<16>);
-  else if (d == 128) run(attn_bw_rows_kernel<32>, attn_bw_keys_kernel<32>);
-  else run(attn_bw_rows_kernel<64>, attn_bw_keys_kernel<64>);
+  if (d == 64) run(attn_bw_rows_kernel<8>, attn_bw_keys_kernel<8>);
+  else if (d == 128) run(attn_bw_rows_kernel<16>, attn_bw_keys_kernel<16>);
+  else run(attn_bw_rows_kernel<32>, attn_bw_keys_kernel<32>);
   STCA_CUDA_TRY(cudaGetLastError());
   set_error(STCA_OK, "");
   return STCA_OK;
