@@ -391,9 +391,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           for (int k = 0; k < 32; k += 2) {
             const float p0 = ex2(__uint_as_float(sv[cb][k]) - m_new);      // exp2(-inf) = 0
             const float x1 = __uint_as_float(sv[cb][k + 1]) - m_new;
-            // with d <= 128, 1 in 4 on the FMA pipe (MUFU-bound); with d = 256 the
-            // softmax is bound by instruction issue, and all go to the MUFU
-            const float p1 = (C::P_TMEM && (k & 2)) ? ex2_fma(x1) : ex2(x1);
+            // with d <= 128, 3 in 8 on the FMA pipe (MUFU-bound; 1 in 4 and 1 in 2
+            // measured slower); with d = 256 the softmax is bound by instruction
+            // issue, and all go to the MUFU
+            const float p1 = (C::P_TMEM && (k & 6) != 0) ? ex2_fma(x1) : ex2(x1);
             ls[(k >> 1) & 3] += p0 + p1;
             pk[(cb * 32 + k) >> 1] = pack_bf16x2(p0, p1);
           }
