@@ -169,6 +169,17 @@ int stca_head(stca_handle* handle, const void* targets, int64_t T, const float* 
               float* zout, void* stream);
 
 /*
+ * stca_forward followed by the prediction-head token of Eq. (9): writes Z as
+ * stca_forward does and zout (T x d fp32, caller-owned, 16-byte aligned) as
+ * stca_head would.  On the tensor-core step path the head runs inside the last
+ * layer's step launch (its [o(1) .. o(M) | x_t] operand is already on chip);
+ * elsewhere the head kernel runs after the forward.  Same errors as
+ * stca_forward, plus STCA_EINVAL when the handle has no head weights.
+ */
+int stca_forward_head(stca_handle* handle, const void* targets, const int64_t* target_offsets,
+                      int64_t T, float* Z, float* zout, void* stream);
+
+/*
  * Copy the encoded history X~(layer+1) of the last stca_encode (N x d, dtype
  * elements, the rows in the order of X) into `dst`, a device buffer the caller
  * owns.  layer is 0-based.  Lets a caller keep or inspect the encoding of a

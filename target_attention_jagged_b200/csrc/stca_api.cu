@@ -343,6 +343,23 @@ extern "C" int stca_init(const stca_weights* w, int d, int h, int r, int M, int 
     cudaGetLastError();
     H->num_sms = 148;
   }
+  // prediction-head weights of Eq. (9), when given (fp32 host copies)
+  std::vector<float> wz, zu, zg, zd;
+  HeadHostW hw;
+  if (nhead == 4) {
+    int rc2 = fetch(w->Wz, static_cast<size_t>(M + 1) * d * d, dtype, dev, &wz, "Wz");
+    if (!rc2) rc2 = fetch(w->zWu, static_cast<size_t>(d) * rd, dtype, dev, &zu, "zWu");
+    if (!rc2) rc2 = fetch(w->zWg, static_cast<size_t>(d) * rd, dtype, dev, &zg, "zWg");
+    if (!rc2) rc2 = fetch(w->zWd, static_cast<size_t>(rd) * d, dtype, dev, &zd, "zWd");
+    if (rc2) {
+      stca_destroy(H);
+      return rc2;
+    }
+    hw.Wz = wz.data();
+    hw.zWu = zu.data();
+    hw.zWg = zg.data();
+    hw.zWd = zd.data();
+  }
   {
     std::vector<StepHostW> sw(M);
     for (int i = 0; i < M; ++i) {
@@ -370,7 +387,7 @@ extern "C" int stca_init(const stca_weights* w, int d, int h, int r, int M, int 
       return rc2;
     }
     if (step_tc_supported(H)) {
-      if (int rc2 = step_tc_setup(H, sw)) {
+      if (int rc2 = step_tc_setup(H, sw, hw)) {
         stca_destroy(H);
         return rc2;
       }
@@ -397,13 +414,7 @@ extern "C" int stca_init(const stca_weights* w, int d, int h, int r, int M, int 
     }
   }
   if (nhead == 4) {
-    std::vector<float> wz, zu, zg, zd;
-    int rc2 = fetch(w->Wz, static_cast<size_t>(M + 1) * d * d, dtype, dev, &wz, "Wz");
-    if (!rc2) rc2 = fetch(w->zWu, static_cast<size_t>(d) * rd, dtype, dev, &zu, "zWu");
-    if (!rc2) rc2 = fetch(w->zWg, static_cast<size_t>(d) * rd, dtype, dev, &zg, "zWg");
-    if (!rc2) rc2 = fetch(w->zWd, static_cast<size_t>(rd) * d, dtype, dev, &zd, "zWd");
-    if (!rc2) rc2 = head_weights_setup(H, wz.data(), zu.data(), zg.data(), zd.data());
-    if (rc2) {
+    if (int rc2 = head_weights_setup(H, wz.data(), zu.data(), zg.data(), zd.data())) {
       stca_destroy(H);
       return rc2;
     }
@@ -819,8 +830,11 @@ static bool naive_cheaper(const stca_handle* H, const int64_t* toff) {
   return nv < re;
 }
 
-extern "C" int stca_forward(stca_handle* H, const void* targets, const int64_t* target_offsets,
-                            int64_t T, float* Z, void* stream) {
+// The forward of stca_forward; with zout, also the prediction-head token of
+// Eq. (9), inside the last per-target step when that runs on the tensor cores,
+// else by the separate head kernel after it.
+static int forward_impl(stca_handle* H, const void* targets, const int64_t* target_offsets,
+                        int64_t T, float* Z, float* zout, void* stream) {
   if (!H) return set_error(STCA_EINVAL, "handle is NULL");
   if (!H->encoded) return set_error(STCA_ESTATE, "stca_forward before a successful stca_encode");
   if (T < 0) return set_error(STCA_EINVAL, "T must be >= 0");
@@ -897,10 +911,12 @@ extern "C" int stca_forward(stca_handle* H, const void* targets, const int64_t* 
   const bool fused = !naive && step_tc && H->last_max_items <= step_tc_max_items() &&
                      H->last_G < (int64_t(1) << 31);
   NaiveStep ns{NL.G, NL.Tq, reinterpret_cast<const int64_t*>(p + H->off_qbase), H->Ubf};
+  const bool head_in_step = zout && step_tc && H->head_tc;
   auto step = [&](int layer, const float* cm) {
     if (step_tc)
       return launch_step_tc(H, layer, targets, T, fused ? nullptr : cm, &plan, H->part, H->last_G,
-                            Z, H->Ubf, s, naive ? &ns : nullptr);
+                            Z, H->Ubf, s, naive ? &ns : nullptr,
+                            head_in_step && layer == H->M - 1 ? zout : nullptr);
     launch_target_step(H, layer, targets, T, plan, cm, Z, s);
     return static_cast<int>(STCA_OK);
   };
@@ -943,7 +959,29 @@ extern "C" int stca_forward(stca_handle* H, const void* targets, const int64_t* 
     H->launches++;
     if (int rc2 = check_launch("target step")) return rc2;
   }
+  if (zout && !head_in_step) {
+    {
+      TimedLaunch tl(H, STCA_K_HEAD, s);
+      launch_head(H, targets, T, Z, zout, s);
+    }
+    H->launches++;
+    if (int rc2 = check_launch("prediction head")) return rc2;
+  }
   return ok();
+}
+
+extern "C" int stca_forward(stca_handle* H, const void* targets, const int64_t* target_offsets,
+                            int64_t T, float* Z, void* stream) {
+  return forward_impl(H, targets, target_offsets, T, Z, nullptr, stream);
+}
+
+extern "C" int stca_forward_head(stca_handle* H, const void* targets, const int64_t* target_offsets,
+                                 int64_t T, float* Z, float* zout, void* stream) {
+  if (!H) return set_error(STCA_EINVAL, "handle is NULL");
+  if (!H->whead) return set_error(STCA_EINVAL, "stca_forward_head: the handle has no head weights (Wz, zWu, zWg, zWd)");
+  if (T > 0 && !zout) return set_error(STCA_EINVAL, "stca_forward_head: zout is NULL");
+  if (reinterpret_cast<uintptr_t>(zout) % 16) return set_error(STCA_EINVAL, "zout must be 16-byte aligned");
+  return forward_impl(H, targets, target_offsets, T, Z, zout, stream);
 }
 
 extern "C" int stca_head(stca_handle* H, const void* targets, int64_t T, const float* Z,

@@ -118,6 +118,8 @@ struct stca_handle {
   bool tc_encode_ready = false;
   uint16_t* wstep_tc = nullptr;         // A-tile stream of the tensor-core per-target step
   std::vector<stca::TcGemm> tcO, tcC, tcUG, tcD, tcQ;   // per layer
+  stca::TcGemm tcZC, tcZUG, tcZD;       // prediction head (Eq. (9)): W_Z, [zW_u | zW_g], zW_d
+  bool head_tc = false;
   bool step_tc_ready = false;
   void* whead = nullptr;                // prediction-head weights (dtype): Wz, [zWu | zWg], zWd
   const void *hWz = nullptr, *hWug = nullptr, *hWd = nullptr;
@@ -204,7 +206,11 @@ size_t attn_simt_smem(const stca_handle* H);
 
 // Tensor-core per-target step (step_tc.cu)
 bool step_tc_supported(const stca_handle* H);
-int step_tc_setup(stca_handle* H, const std::vector<StepHostW>& layers);
+// head: fp32 host W_Z ((M+1)d x d), zW_u, zW_g (d x rd), zW_d (rd x d), or all NULL.
+struct HeadHostW {
+  const float *Wz = nullptr, *zWu = nullptr, *zWg = nullptr, *zWd = nullptr;
+};
+int step_tc_setup(stca_handle* H, const std::vector<StepHostW>& layers, const HeadHostW& head);
 // cmerged: the merged rows c_j (T x h x d), or NULL to merge the split
 // partials (part: G x d accumulators, then G maxima, G sums) inside the step;
 // that needs at most step_tc_max_items() items per (request, query tile).
@@ -219,7 +225,8 @@ struct NaiveStep {
 };
 int launch_step_tc(const stca_handle* H, int layer, const void* targets, int64_t T,
                    const float* cmerged, const StepPlan* plan, const float* part, int64_t G,
-                   float* Z, uint16_t* Ubf, cudaStream_t s, const NaiveStep* naive = nullptr);
+                   float* Z, uint16_t* Ubf, cudaStream_t s, const NaiveStep* naive = nullptr,
+                   float* zout = nullptr);
 
 // Host-side attention work plan (stca_api.cu).
 struct PlanHost {

@@ -104,7 +104,7 @@ bool step_tc_supported(const stca_handle* H) {
 // (W_u and W_g blocks interleaved: block 2m = u features 128m.., block 2m+1 =
 // g features of the same range, so one TMEM lane holds a matching u, g pair)
 // and W_d, and W_Q.
-int step_tc_setup(stca_handle* H, const std::vector<StepHostW>& layers) {
+int step_tc_setup(stca_handle* H, const std::vector<StepHostW>& layers, const HeadHostW& head) {
   const int d = H->d, rd = H->rd, M = H->M;
   std::vector<uint16_t> tiles;
   H->tcO.assign(M, TcGemm());
@@ -125,6 +125,20 @@ int step_tc_setup(stca_handle* H, const std::vector<StepHostW>& layers) {
     H->tcD[i] = put_tiles(tiles, rd, col_blocks(L.qWd, d));
     H->tcQ[i] = put_tiles(tiles, d, col_blocks(L.Wq, d));
   }
+  if (head.Wz) {
+    // prediction head of Eq. (9), run by the last layer's step: W_Z over the
+    // (M+1) d inputs [o(1) .. o(M) | x_t], its SwiGLU up/gate (blocks
+    // interleaved as for the query FFN) and down projection
+    H->tcZC = put_tiles(tiles, (M + 1) * d, col_blocks(head.Wz, d));
+    std::vector<ColBlock> ug;
+    for (int m = 0; m < rd / 128; ++m) {
+      ug.push_back({head.zWu, rd, 128 * m});
+      ug.push_back({head.zWg, rd, 128 * m});
+    }
+    H->tcZUG = put_tiles(tiles, d, ug);
+    H->tcZD = put_tiles(tiles, rd, col_blocks(head.zWd, d));
+    H->head_tc = true;
+  }
   if (cudaMalloc(&H->wstep_tc, tiles.size() * 2) != cudaSuccess) {
     cudaGetLastError();
     return set_error(STCA_ENOMEM, "tensor-core step weight allocation failed");
@@ -137,7 +151,7 @@ int step_tc_setup(stca_handle* H, const std::vector<StepHostW>& layers) {
 // ------------------------------------------------------------------ kernel
 namespace {
 
-enum : int { kO = 0, kC = 1, kUG = 2, kD = 3, kQ = 4 };
+enum : int { kO = 0, kC = 1, kUG = 2, kD = 3, kQ = 4, kZ = 5 };   // kZ: the head's down product
 
 struct StepTcArgs {
   int layer, M, d, h, dh, rd;
@@ -156,14 +170,15 @@ struct StepTcArgs {
   float uscale;
   int* status;
   int ng;                       // products in this launch
-  TcGemm g[5];
-  int kind[5];
+  TcGemm g[8];
+  int kind[8];
   int nring;                    // A-tile ring stages
   int kch;                      // inputs per W_V staging chunk
   int naive;                    // naive form: cmerged is o_head (T x d); write packed q rows
   int nG, nTq;                  // its layout (NaiveLayout)
   const int64_t* qbase;         // first packed row of each request
   uint16_t* upk;                // packed query rows [rows x 64] bf16
+  float* zout;                  // prediction head z (T x d) when the last layer runs it, or NULL
 };
 
 // Shared memory, in bytes (1024-aligned base): the A-tile ring, then the
@@ -188,7 +203,7 @@ __host__ __device__ inline StepLayout step_layout(int d, int rd, int M, int h, i
   L.ring = 0;
   L.bO = L.ring + nring * kATile;
   L.bC = L.bO + (d / 64) * kBTile;
-  L.bU = L.bC + (M * d / 64) * kBTile;
+  L.bU = L.bC + ((M + 1) * d / 64) * kBTile;     // fusion inputs, up to the head's M + 1 blocks
   L.bH = L.bU + (d / 64) * kBTile;
   L.bQ = L.bH + (rd / 64) * kBTile;
   L.scr = L.bQ + (d / 64) * kBTile;
@@ -260,7 +275,7 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_tc_kernel(const StepTcAr
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t t0 = static_cast<int64_t>(blockIdx.x) * kTgt;
   const int nb = a.T - t0 < kTgt ? static_cast<int>(a.T - t0) : kTgt;
-  uint8_t* bufs[5] = {sm + Y.bO, sm + Y.bC, sm + Y.bU, sm + Y.bH, sm + Y.bQ};
+  uint8_t* bufs[6] = {sm + Y.bO, sm + Y.bC, sm + Y.bU, sm + Y.bH, sm + Y.bQ, sm + Y.bH};
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < R; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
@@ -396,8 +411,9 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_tc_kernel(const StepTcAr
         put_b1(bufs[kUG], t, k, t < nb ? bf2f(a.targets[(t0 + t) * d + k]) : 0.f);
       }
     } else {
-      if (L + 1 < M) {
-        // [o(1) .. o(L) | o(L+1): by the output epilogue | x_t] of Eq. (7)
+      if (L + 1 < M || a.zout) {
+        // [o(1) .. o(L) | o(L+1): by the output epilogue | x_t] of Eq. (7), or of
+        // the head's Eq. (9) after the last layer
         // 8 inputs (one 16-byte chunk of a B row) per item
         const int wcat8 = (L + 2) * d / 8, d8 = d / 8;
         for (int e = tid; e < kTgt * wcat8; e += 32 * kWorkers) {
@@ -637,11 +653,14 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_tc_kernel(const StepTcAr
           if (kind == kO) {
             for (int j = 0; j < 8; ++j)
               if (t8 + j < nb) a.Z[((t0 + t8 + j) * M + L) * d + f] = vals[m][j];
-            if (L + 1 < M) put_b8(bufs[kC], L * d + f, t8, vals[m], lane);
+            if (L + 1 < M || a.zout) put_b8(bufs[kC], L * d + f, t8, vals[m], lane);
           } else if (kind == kC) {
             put_b8(bufs[kUG], f, t8, vals[m], lane);
           } else if (kind == kD) {
             put_b8(bufs[kQ], f, t8, vals[m], lane);
+          } else if (kind == kZ) {   // the head's token z of Eq. (9)
+            for (int j = 0; j < 8; ++j)
+              if (t8 + j < nb) a.zout[(t0 + t8 + j) * d + f] = vals[m][j];
           } else {   // kQ: P = q W_Q in fp32, as P^T[feature][target] for the W_K products
             float4* dst = reinterpret_cast<float4*>(scr + f * kTgt + t8);
             dst[0] = make_float4(vals[m][0], vals[m][1], vals[m][2], vals[m][3]);
@@ -751,7 +770,7 @@ int step_tc_max_items() { return kMaxItems; }
 
 int launch_step_tc(const stca_handle* H, int layer, const void* targets, int64_t T,
                    const float* cmerged, const StepPlan* plan, const float* part, int64_t G,
-                   float* Z, uint16_t* Ubf, cudaStream_t s, const NaiveStep* naive) {
+                   float* Z, uint16_t* Ubf, cudaStream_t s, const NaiveStep* naive, float* zout) {
   if (T <= 0) return STCA_OK;
   if (!H->step_tc_ready) return set_error(STCA_ESTATE, "tensor-core step weights are not set up");
   const int M = H->M;
@@ -794,6 +813,14 @@ int launch_step_tc(const stca_handle* H, int layer, const void* targets, int64_t
     ++a.ng;
   };
   if (layer >= 0) add(kO, H->tcO[layer]);
+  if (zout) {
+    if (layer != M - 1 || !H->head_tc)
+      return set_error(STCA_EINVAL, "tensor-core step: the head runs after the last layer, with head weights");
+    a.zout = zout;
+    add(kC, H->tcZC);
+    add(kUG, H->tcZUG);
+    add(kZ, H->tcZD);
+  }
   if (layer + 1 < M) {
     const int n = layer + 1;
     if (layer >= 0) add(kC, H->tcC[n]);

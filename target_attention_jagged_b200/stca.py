@@ -35,7 +35,7 @@ _NAMES = {STCA_EINVAL: "EINVAL", STCA_ESTATE: "ESTATE", STCA_ENOMEM: "ENOMEM",
 EXPORTS = ("stca_init", "stca_destroy", "stca_encode", "stca_forward", "stca_run_host",
            "stca_validate_offsets", "stca_device_status", "stca_set_option",
            "stca_get_option", "stca_kernel_times", "stca_get_encoded", "stca_plan_attention",
-           "stca_forward_static", "stca_head", "stca_sl_beta", "stca_sl_plan",
+           "stca_forward_static", "stca_head", "stca_forward_head", "stca_sl_beta", "stca_sl_plan",
            "stca_sl_gather", "stca_encode_backward", "stca_attention_backward",
            "stca_last_error")
 
@@ -60,6 +60,7 @@ def _load():
     lib.stca_forward.argtypes = [P, P, PI64, I64, P, P]
     lib.stca_forward_static.argtypes = [P, P, PI64, I64, P, P]
     lib.stca_head.argtypes = [P, P, I64, P, P, P]
+    lib.stca_forward_head.argtypes = [P, P, PI64, I64, P, P, P]
     D, PD = ctypes.c_double, ctypes.POINTER(ctypes.c_double)
     lib.stca_sl_beta.argtypes = [D, I64, I64, I64, PD, PD]
     lib.stca_sl_plan.argtypes = [PI64, I64, PD, I64, I64, I64, I64, PI64, PI64, PI64, PI64]
@@ -330,6 +331,18 @@ def stca_attention_backward(handle: int, layer: int, U, target_offsets, dC, N: i
     return dU, dX
 
 
+def stca_forward_head(handle: int, targets, target_offsets, Z, zout, stream=None):
+    """stca_forward and the Eq. (9) head token: Z (T, M, d) and zout (T, d), fp32 CUDA."""
+    import torch
+    toff = _offsets(target_offsets)
+    T = int(toff[-1])
+    assert Z.dtype == torch.float32 and zout.dtype == torch.float32
+    _check(_lib.stca_forward_head(handle, targets.data_ptr() if T > 0 else None, _i64p(toff), T,
+                                  Z.data_ptr() if T > 0 else None, zout.data_ptr() if T > 0 else None,
+                                  _stream_ptr(stream)))
+    return Z, zout
+
+
 def stca_run_host(handle: int, X_host, offsets, targets_host, target_offsets, Z_host,
                   stream=None) -> None:
     """End-to-end on host buffers (numpy arrays or CPU tensors, ideally pinned)."""
@@ -414,6 +427,16 @@ class Stca:
         if Z is None:
             Z = torch.empty((T, self.M, self.d), dtype=torch.float32, device=targets.device)
         return stca_forward(self.handle, targets, target_offsets, Z, stream)
+
+    def forward_head(self, targets, target_offsets, Z=None, zout=None, stream=None):
+        """Z of the forward and z of Eq. (9) in one call."""
+        import torch
+        T = int(np.asarray(target_offsets)[-1])
+        if Z is None:
+            Z = torch.empty((T, self.M, self.d), dtype=torch.float32, device=targets.device)
+        if zout is None:
+            zout = torch.empty((T, self.d), dtype=torch.float32, device=targets.device)
+        return stca_forward_head(self.handle, targets, target_offsets, Z, zout, stream)
 
     def head(self, targets, Z, zout=None, stream=None):
         """z of Eq. (9) for every target: (T, d) fp32."""

@@ -105,3 +105,33 @@ def test_head_empty_and_missing_weights(gpu):
         assert err.value.code == S.stca.STCA_EINVAL and "head weights" in str(err.value)
     finally:
         st.close()
+
+
+@pytest.mark.parametrize("dtype,d,h,M,r,step_path", [
+    ("bf16", 128, 8, 3, 4, 0),     # tensor-core step: the head runs in the last step launch
+    ("bf16", 256, 16, 6, 2, 0),    # the widest W_Z operand the fused head takes ((M+1) d = 1792)
+    ("bf16", 128, 4, 1, 2, 0),     # one layer: the query-init step is followed by the head step
+    ("bf16", 128, 8, 2, 2, 1),     # CUDA-core step: the head kernel after the forward
+    ("f32", 64, 2, 2, 2, 0),
+])
+def test_forward_head_matches_oracle(gpu, dtype, d, h, M, r, step_path):
+    import torch
+    import target_attention_jagged_b200 as S
+    wl = make_workload(lengths=[300, 1, 129, 2000], targets=[5, 2, 0, 17], d=d, h=h, M=M, r=r,
+                       dtype=dtype, seed=41 + d + M)
+    st = S.Stca(storage_weights(wl), d, h, r, M, dtype)
+    try:
+        if step_path:
+            st.set_option(S.STCA_OPT_STEP_PATH, step_path)
+        st.encode(to_device(wl, wl.X, gpu), wl.offsets)
+        Z, z = st.forward_head(to_device(wl, wl.targets, gpu), wl.target_offsets)
+        torch.cuda.synchronize()
+        st.status()
+        Z, z = Z.cpu().numpy(), z.cpu().numpy()
+    finally:
+        st.close()
+    wantZ = O.forward_workload(wl)
+    wantz = O.head_from_outputs(wantZ, wl.targets, wl.weights)
+    assert normwise_err(Z, wantZ) <= TOL[dtype]
+    err = normwise_err(z, wantz)
+    assert err <= TOL[dtype], f"forward + head normwise error {err:.3e}"
