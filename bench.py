@@ -540,9 +540,26 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.synchronize()
     st.status(stream)
     head_ms = h0.elapsed_time(h1) / args.steps
+    # the head fused into the last per-target step (stca_forward_head): its cost
+    # is the difference to the plain forward on the same encoded history
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            S.stca_forward_head(st.handle, xt, wl.target_offsets, Z, zout, stream)
+        q0, q1, q2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+        q0.record(stream)
+        for _ in range(args.steps):
+            st.forward(xt, wl.target_offsets, Z, stream)
+        q1.record(stream)
+        for _ in range(args.steps):
+            S.stca_forward_head(st.handle, xt, wl.target_offsets, Z, zout, stream)
+        q2.record(stream)
+    torch.cuda.synchronize()
+    st.status(stream)
+    fused_head_ms = (q1.elapsed_time(q2) - q0.elapsed_time(q1)) / args.steps
     head_peak = 148 * 128 * 2 * 1.965e9 / 1e12
     head_ach = c["head_flops"] / (head_ms / 1e3) / 1e12
     head = {"ms_per_head": head_ms, "targets_per_s": world * wl.T / (head_ms / 1e3),
+            "fused_in_last_step_ms": fused_head_ms,
             "kernel": "head_kernel", "inputs": "Z and weights L2-resident (back-to-back calls)",
             "roofline": {"bound": "alu", "achieved": head_ach, "peak": head_peak,
                          "unit": "TFLOP/s", "frac": head_ach / head_peak,
