@@ -106,8 +106,8 @@ __global__ void __launch_bounds__(kBwThreads) attn_bw_rows_kernel(AttnBwArgs a) 
   for (int f = 0; f < kMaxQ; ++f) {
     u[f] = dc[f] = du[f] = 0.f;
     if (f < dq && active) {
-      u[f] = a.U[row * d + qu * dq + f];
-      dc[f] = a.dC[row * d + qu * dq + f];
+      u[f] = a.U[row * d + f * kLanes + qu];      // features interleaved across the lanes:
+      dc[f] = a.dC[row * d + f * kLanes + qu];    // conflict-free shared-memory reads
     }
   }
   float m = -INFINITY, l = 0.f, dl = 0.f;       // running max, sum, sum of P dP (unnormalised)
@@ -119,13 +119,13 @@ __global__ void __launch_bounds__(kBwThreads) attn_bw_rows_kernel(AttnBwArgs a) 
       stage_rows(sk, a.Xt, a.xbf, k0 + kt, nk, d);
       __syncthreads();
       for (int k = 0; k < nk; ++k) {
-        const float* xk = sk + k * d + qu * dq;
+        const float* xk = sk + k * d + qu;
         float s = 0.f, dp = 0.f;
 #pragma unroll
         for (int f = 0; f < kMaxQ; ++f)
           if (f < dq) {
-            s = fmaf(u[f], xk[f], s);
-            dp = fmaf(dc[f], xk[f], dp);
+            s = fmaf(u[f], xk[f * kLanes], s);
+            dp = fmaf(dc[f], xk[f * kLanes], dp);
           }
         s = quad_sum(s);
         dp = quad_sum(dp);
@@ -144,7 +144,7 @@ __global__ void __launch_bounds__(kBwThreads) attn_bw_rows_kernel(AttnBwArgs a) 
           const float ds = p * (dp - delta);
 #pragma unroll
           for (int f = 0; f < kMaxQ; ++f)
-            if (f < dq) du[f] = fmaf(ds, xk[f], du[f]);
+            if (f < dq) du[f] = fmaf(ds, xk[f * kLanes], du[f]);
         }
       }
     }
@@ -152,7 +152,7 @@ __global__ void __launch_bounds__(kBwThreads) attn_bw_rows_kernel(AttnBwArgs a) 
   if (!active) return;
 #pragma unroll
   for (int f = 0; f < kMaxQ; ++f)
-    if (f < dq) a.dU[row * d + qu * dq + f] = du[f];
+    if (f < dq) a.dU[row * d + f * kLanes + qu] = du[f];
   if (qu == 0) {
     a.stats[row * 3 + 0] = m;
     a.stats[row * 3 + 1] = l;
@@ -175,7 +175,7 @@ __global__ void __launch_bounds__(kBwThreads) attn_bw_keys_kernel(AttnBwArgs a) 
 #pragma unroll
   for (int f = 0; f < kMaxQ; ++f) {
     x[f] = dx[f] = 0.f;
-    if (f < dq && active) x[f] = ld_x(a.Xt, a.xbf, key * d + qu * dq + f);
+    if (f < dq && active) x[f] = ld_x(a.Xt, a.xbf, key * d + f * kLanes + qu);
   }
   for (int64_t rt = 0; rt < R; rt += kBwTile) {
     const int nr = static_cast<int>(R - rt < kBwTile ? R - rt : kBwTile);
@@ -198,15 +198,15 @@ __global__ void __launch_bounds__(kBwThreads) attn_bw_keys_kernel(AttnBwArgs a) 
     }
     __syncthreads();
     for (int r = 0; r < nr; ++r) {
-      const float* ur = sr + r * w + qu * dq;
+      const float* ur = sr + r * w + qu;
       const float* cr = ur + d;
       const float m = sr[r * w + 2 * d], l = sr[r * w + 2 * d + 1], delta = sr[r * w + 2 * d + 2];
       float s = 0.f, dp = 0.f;
 #pragma unroll
       for (int f = 0; f < kMaxQ; ++f)
         if (f < dq) {
-          s = fmaf(ur[f], x[f], s);
-          dp = fmaf(cr[f], x[f], dp);
+          s = fmaf(ur[f * kLanes], x[f], s);
+          dp = fmaf(cr[f * kLanes], x[f], dp);
         }
       s = quad_sum(s);
       dp = quad_sum(dp);
@@ -214,13 +214,13 @@ __global__ void __launch_bounds__(kBwThreads) attn_bw_keys_kernel(AttnBwArgs a) 
       const float ds = p * (dp - delta);
 #pragma unroll
       for (int f = 0; f < kMaxQ; ++f)
-        if (f < dq) dx[f] = fmaf(p, cr[f], fmaf(ds, ur[f], dx[f]));
+        if (f < dq) dx[f] = fmaf(p, cr[f * kLanes], fmaf(ds, ur[f * kLanes], dx[f]));
     }
   }
   if (!active) return;
 #pragma unroll
   for (int f = 0; f < kMaxQ; ++f)
-    if (f < dq) a.dX[key * d + qu * dq + f] = dx[f];
+    if (f < dq) a.dX[key * d + f * kLanes + qu] = dx[f];
 }
 
 // ---------------------------------------------------------------- encoder
