@@ -78,3 +78,41 @@ def test_naive_form_rejected_when_unsupported(gpu):
         run_gpu(wl, gpu, attn_form=FORM_NAIVE)
     Z = run_gpu(wl, gpu, attn_form=FORM_AUTO)      # auto falls back to the reordered form
     assert normwise_err(Z, O.forward_workload(wl)) <= TOL["f32"]
+
+
+def test_naive_form_with_fused_head(gpu):
+    """The naive form's last step also runs the Eq. (9) head (stca_forward_head)."""
+    import torch
+    import target_attention_jagged_b200 as S
+    from tests.gpu_helpers import to_device
+    wl = make_workload(lengths=LENGTHS, targets=TARGETS, d=256, h=16, M=2, r=2, dtype="bf16", seed=61)
+    st = S.Stca(storage_weights(wl), 256, 16, 2, 2, "bf16")
+    try:
+        st.set_option(S.STCA_OPT_ATTN_FORM, FORM_NAIVE)
+        st.encode(to_device(wl, wl.X, gpu), wl.offsets)
+        Z, z = st.forward_head(to_device(wl, wl.targets, gpu), wl.target_offsets)
+        torch.cuda.synchronize()
+        st.status()
+        assert st.get_option(S.STCA_OPT_LAST_FORM) == 1
+        Z, z = Z.cpu().numpy(), z.cpu().numpy()
+    finally:
+        st.close()
+    wantZ = O.forward_workload(wl)
+    assert normwise_err(Z, wantZ) <= TOL["bf16"]
+    assert normwise_err(z, O.head_from_outputs(wantZ, wl.targets, wl.weights)) <= TOL["bf16"]
+
+
+def test_forward_head_without_head_weights(gpu):
+    import torch
+    import target_attention_jagged_b200 as S
+    from tests.gpu_helpers import to_device
+    wl = make_workload(lengths=[40], targets=[2], d=128, h=8, M=1, r=2, dtype="bf16", seed=62)
+    w = {k: v for k, v in storage_weights(wl).items() if k not in ("Wz", "zWu", "zWg", "zWd")}
+    st = S.Stca(w, 128, 8, 2, 1, "bf16")
+    try:
+        st.encode(to_device(wl, wl.X, gpu), wl.offsets)
+        with pytest.raises(S.StcaError) as e:
+            st.forward_head(to_device(wl, wl.targets, gpu), wl.target_offsets)
+        assert e.value.code == S.stca.STCA_EINVAL
+    finally:
+        st.close()
