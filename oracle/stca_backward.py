@@ -100,3 +100,34 @@ def attention_backward_batch(U, Xt, offsets, target_offsets, h, dC):
         dU[q0:q1] = du
         dX[k0:k1] = dx
     return dU, dX
+
+
+def output_backward(C, Wv, Wo, h, dZ):
+    """Gradients of <o, dZ> with o = [c_1 W_V^1 || ... || c_h W_V^h] W_O (Eqs. (6), (13)).
+
+    C: (T, h, d) merged rows c_j (row t h + j of the attention output), W_V, W_O:
+    (d, d), head j on columns [j d_h, (j+1) d_h) of W_V (reading O7).  Returns
+    dC (T, h, d), dWv, dWo (d, d)."""
+    C, Wv, Wo, dZ = _f64(C), _f64(Wv), _f64(Wo), _f64(dZ)
+    T, hh, d = C.shape
+    dh = d // h
+    Oh = np.concatenate([C[:, j, :] @ Wv[:, j * dh:(j + 1) * dh] for j in range(h)], axis=-1)
+    dOh = dZ @ Wo.T
+    dWo = Oh.T @ dZ
+    dC = np.stack([dOh[:, j * dh:(j + 1) * dh] @ Wv[:, j * dh:(j + 1) * dh].T for j in range(h)], axis=1)
+    dWv = np.concatenate([C[:, j, :].T @ dOh[:, j * dh:(j + 1) * dh] for j in range(h)], axis=-1)
+    return dC, dWv, dWo
+
+
+def query_backward(Q, Wq, Wk, h, dU):
+    """Gradients of <U, dU> with u_j = (q W_Q^j) W_K^j^T / sqrt(d_h) (Eq. (13)).
+
+    Q: (T, d) query vectors q, dU: (T, h, d).  Returns dQ (T, d), dWq, dWk (d, d)."""
+    Q, Wq, Wk, dU = _f64(Q), _f64(Wq), _f64(Wk), _f64(dU)
+    T, d = Q.shape
+    dh = d // h
+    s = 1.0 / np.sqrt(dh)
+    P = Q @ Wq                                             # (T, d): heads' q W_Q^j side by side
+    dP = np.concatenate([s * dU[:, j, :] @ Wk[:, j * dh:(j + 1) * dh] for j in range(h)], axis=-1)
+    dWk = np.concatenate([s * dU[:, j, :].T @ P[:, j * dh:(j + 1) * dh] for j in range(h)], axis=-1)
+    return dP @ Wq.T, Q.T @ dP, dWk

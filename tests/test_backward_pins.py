@@ -111,6 +111,73 @@ def pin_invariances():
     assert abs((f(eps) - f(-eps)) / (2 * eps) - float((dU * U).sum())) < 1e-6
 
 
+def pin_output_query_finite_differences():
+    rng = np.random.default_rng(7)
+    T, h, d = 3, 2, 6
+    dh = d // h
+    C = rng.standard_normal((T, h, d))
+    Wv, Wo, Wq, Wk = (rng.standard_normal((d, d)) for _ in range(4))
+    Q = rng.standard_normal((T, d))
+    dZ = rng.standard_normal((T, d))
+    dUg = rng.standard_normal((T, h, d))
+
+    def out(C_, Wv_, Wo_):
+        return np.concatenate([C_[:, j] @ Wv_[:, j * dh:(j + 1) * dh] for j in range(h)], -1) @ Wo_
+
+    def uq(Q_, Wq_, Wk_):
+        return np.stack([(Q_ @ Wq_[:, j * dh:(j + 1) * dh]) @ Wk_[:, j * dh:(j + 1) * dh].T / np.sqrt(dh)
+                         for j in range(h)], axis=1)
+    dC, dWv, dWo = B.output_backward(C, Wv, Wo, h, dZ)
+    dQ, dWq, dWk = B.query_backward(Q, Wq, Wk, h, dUg)
+    eps = 1e-6
+    for grad, f, args, i in [(dC, out, [C, Wv, Wo], 0), (dWv, out, [C, Wv, Wo], 1),
+                             (dWo, out, [C, Wv, Wo], 2), (dQ, uq, [Q, Wq, Wk], 0),
+                             (dWq, uq, [Q, Wq, Wk], 1), (dWk, uq, [Q, Wq, Wk], 2)]:
+        G = dZ if f is out else dUg
+        V = rng.standard_normal(grad.shape)
+        a1 = list(args); a1[i] = a1[i] + eps * V
+        a2 = list(args); a2[i] = a2[i] - eps * V
+        fd = float(((f(*a1) - f(*a2)) * G).sum()) / (2 * eps)
+        assert abs(fd - float((grad * V).sum())) <= 1e-6 * max(1.0, abs(fd)), (f.__name__, i)
+
+
+def pin_layer_chain():
+    """The three pieces composed give the gradient of the forward oracle's
+    reordered attention layer (queries, keys and all four projections)."""
+    rng = np.random.default_rng(8)
+    T, L, h, d = 2, 5, 2, 4
+    dh = d // h
+    q = rng.standard_normal((T, d))
+    Xt = rng.standard_normal((L, d))
+    Ws = [rng.standard_normal((d, d)) / np.sqrt(d) for _ in range(4)]
+    dZ = rng.standard_normal((T, d))
+    Wq, Wk, Wv, Wo = Ws
+    U = np.stack([(q @ Wq[:, j * dh:(j + 1) * dh]) @ Wk[:, j * dh:(j + 1) * dh].T / np.sqrt(dh)
+                  for j in range(h)], axis=1)                       # (T, h, d), row t h + j
+    C = np.stack([O.softmax(U[:, j] @ Xt.T) @ Xt for j in range(h)], axis=1)
+    dC, dWv, dWo = B.output_backward(C, Wv, Wo, h, dZ)
+    dU, dXt = B.attention_rows_backward(U.reshape(T * h, d), Xt, dC.reshape(T * h, d))
+    dq, dWq, dWk = B.query_backward(q, Wq, Wk, h, dU.reshape(T, h, d))
+    args = [q, Xt, Wq, Wk, Wv, Wo]
+    grads = [dq, dXt, dWq, dWk, dWv, dWo]
+    loss = lambda a: float((O.attention_reordered(a[0], a[1], a[2], a[3], a[4], a[5], h) * dZ).sum())  # noqa: E731
+    eps = 1e-6
+    for i, g in enumerate(grads):
+        V = rng.standard_normal(g.shape)
+        a1 = list(args); a1[i] = a1[i] + eps * V
+        a2 = list(args); a2[i] = a2[i] - eps * V
+        fd = (loss(a1) - loss(a2)) / (2 * eps)
+        assert abs(fd - float((g * V).sum())) <= 1e-6 * max(1.0, abs(fd)), i
+
+
+def test_attention_layer_chain_matches_forward_oracle():
+    pin_layer_chain()
+
+
+def test_output_and_query_backward_finite_differences():
+    pin_output_query_finite_differences()
+
+
 def test_encoder_backward_finite_differences():
     pin_encoder_finite_differences()
 
@@ -175,6 +242,21 @@ def _enc_sigmoid_derivative(X, W, i, dXt, eps=1e-5):
             "dgamma": (dXt * yh).sum(0), "dbeta": np.asarray(dXt).sum(0)}
 
 
+_output_backward = B.output_backward
+_query_backward = B.query_backward
+
+
+def _out_wrong_transpose(C, Wv, Wo, h, dZ):
+    dC, dWv, dWo = _output_backward(C, Wv, Wo, h, dZ)
+    return dC, dWv, dWo.T                                   # dW_O transposed
+
+
+def _query_no_scale(Q, Wq, Wk, h, dU):
+    dQ, dWq, dWk = _query_backward(Q, Wq, Wk, h, dU)
+    d = np.asarray(Q).shape[1]
+    return dQ * np.sqrt(d // h), dWq * np.sqrt(d // h), dWk * np.sqrt(d // h)   # 1/sqrt(d_h) dropped
+
+
 def _attn_sign(U, Xt, dC):
     U, Xt, dC = (np.asarray(a, float) for a in (U, Xt, dC))
     P = O.softmax(U @ Xt.T); dP = dC @ Xt.T
@@ -202,6 +284,8 @@ MUTANTS = {
     "softmax_sign": ("attention_rows_backward", _attn_sign),
     "value_path_dropped": ("attention_rows_backward", _attn_no_value_term),
     "query_replaced": ("attention_rows_backward", _attn_transposed),
+    "wo_gradient_transposed": ("output_backward", _out_wrong_transpose),
+    "query_scale_dropped": ("query_backward", _query_no_scale),
 }
 
 
@@ -211,7 +295,7 @@ def test_pins_reject_mutant(name, monkeypatch):
     monkeypatch.setattr(B, attr, fn)
     failed = 0
     for pin in (pin_encoder_finite_differences, pin_attention_finite_differences, pin_torch_autograd,
-                pin_invariances):
+                pin_invariances, pin_output_query_finite_differences, pin_layer_chain):
         try:
             pin()
         except AssertionError:
