@@ -574,12 +574,16 @@ def run_ours(args, rank, world, local_rank):
         rows = wl.T * wl.h
         Ub = torch.from_numpy((rng.standard_normal((rows, wl.d)) * (2.0 / np.sqrt(wl.d))).astype(np.float32)).to(dev)
         dC = torch.from_numpy(rng.standard_normal((rows, wl.d)).astype(np.float32)).to(dev)
+        Qb = torch.from_numpy(rng.standard_normal((wl.T, wl.d)).astype(np.float32)).to(dev)
+        dZb = torch.from_numpy(rng.standard_normal((wl.T, wl.d)).astype(np.float32)).to(dev)
         st.encode(X, wl.offsets, stream)
         with torch.cuda.stream(stream):
             for _ in range(2):
                 S.stca_encode_backward(st.handle, 0, X, dXt, wl.d, wl.r * wl.d, stream=stream)
                 S.stca_attention_backward(st.handle, 0, Ub, wl.target_offsets, dC, wl.N, stream)
-            b0, b1, b2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+                S.stca_output_backward(st.handle, 0, dC, dZb, wl.h, stream)
+                S.stca_query_backward(st.handle, 0, Qb, Ub, wl.h, stream)
+            b0, b1, b2, b3 = (torch.cuda.Event(enable_timing=True) for _ in range(4))
             nrep = max(1, min(args.steps, 5))
             b0.record(stream)
             for _ in range(nrep):
@@ -588,9 +592,14 @@ def run_ours(args, rank, world, local_rank):
             for _ in range(nrep):
                 S.stca_attention_backward(st.handle, 0, Ub, wl.target_offsets, dC, wl.N, stream)
             b2.record(stream)
+            for _ in range(nrep):
+                S.stca_output_backward(st.handle, 0, dC, dZb, wl.h, stream)
+                S.stca_query_backward(st.handle, 0, Qb, Ub, wl.h, stream)
+            b3.record(stream)
         torch.cuda.synchronize()
         st.status(stream)
         enc_ms, att_ms = b0.elapsed_time(b1) / nrep, b1.elapsed_time(b2) / nrep
+        proj_ms = b2.elapsed_time(b3) / nrep
         rd = wl.r * wl.d
         enc_fl = 18 * wl.N * wl.d * rd              # recomputed forward (6 N d rd) + 6 backward products
         att_fl = 18 * wl.d * c["TL"] * wl.h         # per (row, key): 2 passes of 2 dots + dU; 2 dots + dX~
@@ -603,7 +612,10 @@ def run_ours(args, rank, world, local_rank):
                        "note": "cuBLASLt TF32 products + SwiGLU / LayerNorm derivative kernels"},
             "attention": {"ms": att_ms, "flops": att_fl, "tflops": att_fl / (att_ms / 1e3) / 1e12,
                           "frac_of_nominal_fp32": att_fl / (att_ms / 1e3) / 1e12 / fp32,
-                          "note": "CUDA-core flash-style kernels (softmax recomputed)"}}
+                          "note": "CUDA-core flash-style kernels (softmax recomputed)"},
+            "projections": {"ms": proj_ms, "flops": 20 * wl.T * wl.d * wl.d,
+                            "note": "output side (W_V, W_O) and query side (W_Q, W_K): "
+                                    "cuBLASLt TF32 products, one per head for the per-head slices"}}
 
     # ---- the sparse-training batch builder and a forward over its packed batch
     train_batch = None

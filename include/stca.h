@@ -352,6 +352,31 @@ int stca_attention_backward(stca_handle* handle, int layer, const float* U,
                             const int64_t* target_offsets, int64_t T, const float* dC,
                             float* dU, float* dXt, void* stream);
 
+/*
+ * Output side of attention layer `layer` (digest Eqs. (6) and (13)): with the
+ * merged rows C (T h x d fp32: row t h + j holds c_j = alpha_j X~ of target t,
+ * head j), the layer output is o = [c_1 W_V^1 || ... || c_h W_V^h] W_O, head j
+ * on columns [j d_h, (j+1) d_h) of W_V.  Given dZ (T x d fp32, the gradient of
+ * o), writes dC (T h x d: the dC that stca_attention_backward takes), dWv and
+ * dWo (d x d, row-major like the weights).  All pointers are DEVICE memory the
+ * caller owns; W_V and W_O are the handle's.  T = 0 writes zero weight
+ * gradients.  Errors: STCA_EINVAL, STCA_ENOMEM, STCA_ECUDA.
+ */
+int stca_output_backward(stca_handle* handle, int layer, const float* C, int64_t T,
+                         const float* dZ, float* dC, float* dWv, float* dWo, void* stream);
+
+/*
+ * Query side of attention layer `layer` (digest Eq. (13)): the merged rows are
+ * u_j = (q W_Q^j) W_K^j^T / sqrt(d_h) for each target's query vector q.
+ * Given Q (T x d fp32, the layer's q as the forward formed it) and dU
+ * (T h x d fp32, row t h + j; the dU stca_attention_backward returns), writes
+ * dQ (T x d), dWq and dWk (d x d).  DEVICE pointers the caller owns; W_Q and
+ * W_K are the handle's.  T = 0 writes zero weight gradients.
+ * Errors: STCA_EINVAL, STCA_ENOMEM, STCA_ECUDA.
+ */
+int stca_query_backward(stca_handle* handle, int layer, const float* Q, int64_t T,
+                        const float* dU, float* dQ, float* dWq, float* dWk, void* stream);
+
 /* Tunables and introspection (STCA_OPT_*).  Values are validated. */
 enum {
   STCA_OPT_ATTN_PATH = 1,     /* 0 auto, 1 CUDA cores, 2 tensor cores (bf16 only) */

@@ -18,6 +18,8 @@
 #include <cublasLt.h>
 #include <math.h>
 
+#include <cmath>
+
 #include <algorithm>
 #include <string>
 #include <vector>
@@ -338,7 +340,7 @@ unsigned grid_for(int64_t n) { return static_cast<unsigned>(std::min<int64_t>((n
 // column-major view C^T = op(B)^T op(A)^T.  ta / tb: A / B stored transposed.
 int gemm_rm(stca_handle* H, bool ta, bool tb, int64_t m, int64_t n, int64_t k, const float* A,
             int64_t lda, const float* B, int64_t ldb, float* C, int64_t ldc, float beta,
-            cudaStream_t s) {
+            cudaStream_t s, float alpha = 1.f) {
   if (!H->lt) {
     cublasLtHandle_t lt = nullptr;
     if (cublasLtCreate(&lt) != CUBLAS_STATUS_SUCCESS) return set_error(STCA_ECUDA, "cublasLtCreate failed");
@@ -376,12 +378,23 @@ int gemm_rm(stca_handle* H, bool ta, bool tb, int64_t m, int64_t n, int64_t k, c
   if (rc == STCA_OK) {
     size_t ws = kWs;
     cublasLtMatmulPreferenceSetAttribute(pref, CUBLASLT_MATMUL_PREF_MAX_WORKSPACE_BYTES, &ws, sizeof(ws));
+    // operands may be column slices (one head's columns): tell the heuristic
+    // their true alignment, which is below the 256 bytes it assumes by default
+    auto align = [](const void* p) {
+      uint32_t a = 256;
+      while (a > 4 && reinterpret_cast<uintptr_t>(p) % a) a >>= 1;
+      return a;
+    };
+    const uint32_t aA = align(B), aB = align(A), aC = align(C);
+    cublasLtMatmulPreferenceSetAttribute(pref, CUBLASLT_MATMUL_PREF_MIN_ALIGNMENT_A_BYTES, &aA, sizeof(aA));
+    cublasLtMatmulPreferenceSetAttribute(pref, CUBLASLT_MATMUL_PREF_MIN_ALIGNMENT_B_BYTES, &aB, sizeof(aB));
+    cublasLtMatmulPreferenceSetAttribute(pref, CUBLASLT_MATMUL_PREF_MIN_ALIGNMENT_C_BYTES, &aC, sizeof(aC));
+    cublasLtMatmulPreferenceSetAttribute(pref, CUBLASLT_MATMUL_PREF_MIN_ALIGNMENT_D_BYTES, &aC, sizeof(aC));
     if (cublasLtMatmulAlgoGetHeuristic(lt, op, l1, l2, lc, lc, pref, 1, &heur, &found) !=
             CUBLAS_STATUS_SUCCESS || found < 1)
       rc = set_error(STCA_ECUDA, "cuBLASLt found no algorithm for a backward product");
   }
   if (rc == STCA_OK) {
-    const float alpha = 1.f;
     if (cublasLtMatmul(lt, op, &alpha, B, l1, A, l2, &beta, C, lc, C, lc, &heur.algo, H->lt_ws, kWs, s) !=
         CUBLAS_STATUS_SUCCESS)
       rc = set_error(STCA_ECUDA, "cuBLASLt backward product failed");
@@ -532,6 +545,99 @@ extern "C" int stca_attention_backward(stca_handle* H, int layer, const float* U
   if (d == 64) run(attn_bw_rows_kernel<8>, attn_bw_keys_kernel<8>);
   else if (d == 128) run(attn_bw_rows_kernel<16>, attn_bw_keys_kernel<16>);
   else run(attn_bw_rows_kernel<32>, attn_bw_keys_kernel<32>);
+  STCA_CUDA_TRY(cudaGetLastError());
+  set_error(STCA_OK, "");
+  return STCA_OK;
+}
+
+namespace {
+
+int projection_args(stca_handle* H, int layer, int64_t T, const void* a, const void* b,
+                    const void* c, const void* w1, const void* w2, const char* who) {
+  if (!H) return set_error(STCA_EINVAL, "handle is NULL");
+  if (layer < 0 || layer >= H->M) return set_error(STCA_EINVAL, "layer out of range");
+  if (T < 0 || T > (int64_t(1) << 31)) return set_error(STCA_EINVAL, std::string(who) + ": T out of range");
+  if (!w1 || !w2 || (T > 0 && (!a || !b || !c)))
+    return set_error(STCA_EINVAL, std::string(who) + ": NULL argument");
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev != H->device) cudaSetDevice(H->device);
+  return STCA_OK;
+}
+
+}  // namespace
+
+extern "C" int stca_output_backward(stca_handle* H, int layer, const float* C, int64_t T,
+                                    const float* dZ, float* dC, float* dWv, float* dWo, void* stream) {
+  if (int rc = projection_args(H, layer, T, C, dZ, dC, dWv, dWo, "stca_output_backward")) return rc;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int d = H->d, h = H->h, dh = d / h;
+  const size_t dd = static_cast<size_t>(d) * d;
+  if (T == 0) {
+    STCA_CUDA_TRY(cudaMemsetAsync(dWv, 0, dd * sizeof(float), s));
+    STCA_CUDA_TRY(cudaMemsetAsync(dWo, 0, dd * sizeof(float), s));
+    set_error(STCA_OK, "");
+    return STCA_OK;
+  }
+  const LayerW32& Wl = H->L32[layer];
+  // workspace: Oh = the heads' c_j W_V^j side by side (T x d), dOh = dZ W_O^T (T x d)
+  const size_t td = static_cast<size_t>(T) * d;
+  if (int rc = ensure(&H->bw_ws, &H->bw_ws_cap, 2 * td * sizeof(float))) return rc;
+  float* Oh = static_cast<float*>(H->bw_ws);
+  float* dOh = Oh + td;
+  const int64_t hd = static_cast<int64_t>(h) * d;
+  for (int j = 0; j < h; ++j)     // Oh[:, j] = C_j W_V[:, j]   (T x d_h)
+    if (int rc = gemm_rm(H, false, false, T, dh, d, C + j * d, hd, Wl.Wv + j * dh, d, Oh + j * dh, d, 0.f, s))
+      return rc;
+  // dW_O = Oh^T dZ, dOh = dZ W_O^T
+  if (int rc = gemm_rm(H, true, false, d, d, T, Oh, d, dZ, d, dWo, d, 0.f, s)) return rc;
+  if (int rc = gemm_rm(H, false, true, T, d, d, dZ, d, Wl.Wo, d, dOh, d, 0.f, s)) return rc;
+  for (int j = 0; j < h; ++j) {
+    // dC_j = dOh[:, j] W_V[:, j]^T  (T x d),  dW_V[:, j] = C_j^T dOh[:, j]  (d x d_h)
+    if (int rc = gemm_rm(H, false, true, T, d, dh, dOh + j * dh, d, Wl.Wv + j * dh, d, dC + j * d, hd, 0.f, s))
+      return rc;
+    if (int rc = gemm_rm(H, true, false, d, dh, T, C + j * d, hd, dOh + j * dh, d, dWv + j * dh, d, 0.f, s))
+      return rc;
+  }
+  STCA_CUDA_TRY(cudaGetLastError());
+  set_error(STCA_OK, "");
+  return STCA_OK;
+}
+
+extern "C" int stca_query_backward(stca_handle* H, int layer, const float* Q, int64_t T,
+                                   const float* dU, float* dQ, float* dWq, float* dWk, void* stream) {
+  if (int rc = projection_args(H, layer, T, Q, dU, dQ, dWq, dWk, "stca_query_backward")) return rc;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int d = H->d, h = H->h, dh = d / h;
+  const size_t dd = static_cast<size_t>(d) * d;
+  if (T == 0) {
+    STCA_CUDA_TRY(cudaMemsetAsync(dWq, 0, dd * sizeof(float), s));
+    STCA_CUDA_TRY(cudaMemsetAsync(dWk, 0, dd * sizeof(float), s));
+    set_error(STCA_OK, "");
+    return STCA_OK;
+  }
+  const LayerW32& Wl = H->L32[layer];
+  const float scale = 1.f / std::sqrt(static_cast<float>(dh));
+  // workspace: P = Q W_Q (T x d, head j on columns j d_h ..), dP (T x d)
+  const size_t td = static_cast<size_t>(T) * d;
+  if (int rc = ensure(&H->bw_ws, &H->bw_ws_cap, 2 * td * sizeof(float))) return rc;
+  float* P = static_cast<float*>(H->bw_ws);
+  float* dP = P + td;
+  const int64_t hd = static_cast<int64_t>(h) * d;
+  if (int rc = gemm_rm(H, false, false, T, d, d, Q, d, Wl.Wq, d, P, d, 0.f, s)) return rc;
+  for (int j = 0; j < h; ++j) {
+    // W_K^j is stored transposed: WkT[j] (d_h x d) = W_K[:, j]^T
+    const float* WkTj = Wl.WkT + static_cast<size_t>(j) * dh * d;
+    // dP[:, j] = scale dU_j W_K^j   (T x d_h)
+    if (int rc = gemm_rm(H, false, true, T, dh, d, dU + j * d, hd, WkTj, d, dP + j * dh, d, 0.f, s, scale))
+      return rc;
+    // dW_K[:, j] = scale dU_j^T P[:, j]   (d x d_h)
+    if (int rc = gemm_rm(H, true, false, d, dh, T, dU + j * d, hd, P + j * dh, d, dWk + j * dh, d, 0.f, s, scale))
+      return rc;
+  }
+  // dQ = dP W_Q^T, dW_Q = Q^T dP
+  if (int rc = gemm_rm(H, false, true, T, d, d, dP, d, Wl.Wq, d, dQ, d, 0.f, s)) return rc;
+  if (int rc = gemm_rm(H, true, false, d, d, T, Q, d, dP, d, dWq, d, 0.f, s)) return rc;
   STCA_CUDA_TRY(cudaGetLastError());
   set_error(STCA_OK, "");
   return STCA_OK;

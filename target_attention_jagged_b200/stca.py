@@ -37,7 +37,7 @@ EXPORTS = ("stca_init", "stca_destroy", "stca_encode", "stca_forward", "stca_run
            "stca_get_option", "stca_kernel_times", "stca_get_encoded", "stca_plan_attention",
            "stca_forward_static", "stca_head", "stca_forward_head", "stca_sl_beta", "stca_sl_plan",
            "stca_sl_gather", "stca_encode_backward", "stca_attention_backward",
-           "stca_last_error")
+           "stca_output_backward", "stca_query_backward", "stca_last_error")
 
 
 class StcaError(RuntimeError):
@@ -67,6 +67,8 @@ def _load():
     lib.stca_sl_gather.argtypes = [P, I64, I64, P, P, I64, I64, P, P, P]
     lib.stca_encode_backward.argtypes = [P, I, P, I64, P, P, P, P, P, P, P, P]
     lib.stca_attention_backward.argtypes = [P, I, P, PI64, I64, P, P, P, P]
+    lib.stca_output_backward.argtypes = [P, I, P, I64, P, P, P, P, P]
+    lib.stca_query_backward.argtypes = [P, I, P, I64, P, P, P, P, P]
     lib.stca_run_host.argtypes = [P, P, PI64, I64, I64, P, PI64, I64, P, P]
     lib.stca_validate_offsets.argtypes = [PI64, I64, I64, I]
     lib.stca_device_status.argtypes = [P, P]
@@ -329,6 +331,41 @@ def stca_attention_backward(handle: int, layer: int, U, target_offsets, dC, N: i
                                         dU.data_ptr() if T > 0 else None, dX.data_ptr(),
                                         _stream_ptr(stream)))
     return dU, dX
+
+
+def _f32_out(*shape, device):
+    import torch
+    return torch.empty(shape, dtype=torch.float32, device=device)
+
+
+def stca_output_backward(handle: int, layer: int, C, dZ, h: int, stream=None):
+    """Gradients of o = [c_j W_V^j]_j W_O (Eqs. (6), (13)): C (T, h, d) or (T h, d)
+    and dZ (T, d), fp32 contiguous CUDA.  Returns dC (T h, d), dWv, dWo (d, d)."""
+    import torch
+    T, d = int(dZ.shape[0]), int(dZ.shape[1])
+    assert C.dtype == torch.float32 and dZ.dtype == torch.float32
+    assert C.is_contiguous() and dZ.is_contiguous() and C.numel() == T * h * d
+    dC = _f32_out(T * h, d, device=dZ.device)
+    dWv, dWo = _f32_out(d, d, device=dZ.device), _f32_out(d, d, device=dZ.device)
+    live = lambda t: t.data_ptr() if T > 0 else None  # noqa: E731
+    _check(_lib.stca_output_backward(handle, layer, live(C), T, live(dZ), live(dC), dWv.data_ptr(),
+                                     dWo.data_ptr(), _stream_ptr(stream)))
+    return dC, dWv, dWo
+
+
+def stca_query_backward(handle: int, layer: int, Q, dU, h: int, stream=None):
+    """Gradients of u_j = (q W_Q^j) W_K^j^T / sqrt(d_h) (Eq. (13)): Q (T, d) and
+    dU (T h, d), fp32 contiguous CUDA.  Returns dQ (T, d), dWq, dWk (d, d)."""
+    import torch
+    T, d = int(Q.shape[0]), int(Q.shape[1])
+    assert Q.dtype == torch.float32 and dU.dtype == torch.float32
+    assert Q.is_contiguous() and dU.is_contiguous() and dU.numel() == T * h * d
+    dQ = _f32_out(T, d, device=Q.device)
+    dWq, dWk = _f32_out(d, d, device=Q.device), _f32_out(d, d, device=Q.device)
+    live = lambda t: t.data_ptr() if T > 0 else None  # noqa: E731
+    _check(_lib.stca_query_backward(handle, layer, live(Q), T, live(dU), live(dQ), dWq.data_ptr(),
+                                    dWk.data_ptr(), _stream_ptr(stream)))
+    return dQ, dWq, dWk
 
 
 def stca_forward_head(handle: int, targets, target_offsets, Z, zout, stream=None):
