@@ -615,7 +615,7 @@ def run_ours(args, rank, world, local_rank):
                           "note": "CUDA-core flash-style kernels (softmax recomputed)"},
             "projections": {"ms": proj_ms, "flops": 20 * wl.T * wl.d * wl.d,
                             "note": "output side (W_V, W_O) and query side (W_Q, W_K): "
-                                    "cuBLASLt TF32 products, one per head for the per-head slices"}}
+                                    "cuBLASLt TF32 products, the per-head slices as strided batches"}}
 
     # ---- the sparse-training batch builder and a forward over its packed batch
     train_batch = None

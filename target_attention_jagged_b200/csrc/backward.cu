@@ -340,7 +340,8 @@ unsigned grid_for(int64_t n) { return static_cast<unsigned>(std::min<int64_t>((n
 // column-major view C^T = op(B)^T op(A)^T.  ta / tb: A / B stored transposed.
 int gemm_rm(stca_handle* H, bool ta, bool tb, int64_t m, int64_t n, int64_t k, const float* A,
             int64_t lda, const float* B, int64_t ldb, float* C, int64_t ldc, float beta,
-            cudaStream_t s, float alpha = 1.f) {
+            cudaStream_t s, float alpha = 1.f, int batch = 1, int64_t sA = 0, int64_t sB = 0,
+            int64_t sC = 0) {
   if (!H->lt) {
     cublasLtHandle_t lt = nullptr;
     if (cublasLtCreate(&lt) != CUBLAS_STATUS_SUCCESS) return set_error(STCA_ECUDA, "cublasLtCreate failed");
@@ -373,19 +374,32 @@ int gemm_rm(stca_handle* H, bool ta, bool tb, int64_t m, int64_t n, int64_t k, c
       cublasLtMatrixLayoutCreate(&lc, CUDA_R_32F, n, m, ldc) != CUBLAS_STATUS_SUCCESS ||
       cublasLtMatmulPreferenceCreate(&pref) != CUBLAS_STATUS_SUCCESS)
     rc = set_error(STCA_ECUDA, "cuBLASLt descriptor set-up failed");
+  if (rc == STCA_OK && batch > 1) {
+    // `batch` products, operand i at A + i sA, B + i sB, C + i sC
+    const int64_t strides[3] = {sB, sA, sC};
+    cublasLtMatrixLayout_t lays[3] = {l1, l2, lc};
+    for (int i = 0; i < 3 && rc == STCA_OK; ++i)
+      if (cublasLtMatrixLayoutSetAttribute(lays[i], CUBLASLT_MATRIX_LAYOUT_BATCH_COUNT, &batch, sizeof(batch)) !=
+              CUBLAS_STATUS_SUCCESS ||
+          cublasLtMatrixLayoutSetAttribute(lays[i], CUBLASLT_MATRIX_LAYOUT_STRIDED_BATCH_OFFSET, &strides[i],
+                                           sizeof(strides[i])) != CUBLAS_STATUS_SUCCESS)
+        rc = set_error(STCA_ECUDA, "cuBLASLt batch set-up failed");
+  }
   cublasLtMatmulHeuristicResult_t heur{};
   int found = 0;
   if (rc == STCA_OK) {
     size_t ws = kWs;
     cublasLtMatmulPreferenceSetAttribute(pref, CUBLASLT_MATMUL_PREF_MAX_WORKSPACE_BYTES, &ws, sizeof(ws));
     // operands may be column slices (one head's columns): tell the heuristic
-    // their true alignment, which is below the 256 bytes it assumes by default
-    auto align = [](const void* p) {
+    // their true alignment (of every batch member), which is below the 256
+    // bytes it assumes by default
+    auto align = [batch](const void* p, int64_t stride) {
       uint32_t a = 256;
-      while (a > 4 && reinterpret_cast<uintptr_t>(p) % a) a >>= 1;
+      const uintptr_t step = batch > 1 ? static_cast<uintptr_t>(stride) * sizeof(float) : 0;
+      while (a > 4 && (reinterpret_cast<uintptr_t>(p) % a || step % a)) a >>= 1;
       return a;
     };
-    const uint32_t aA = align(B), aB = align(A), aC = align(C);
+    const uint32_t aA = align(B, sB), aB = align(A, sA), aC = align(C, sC);
     cublasLtMatmulPreferenceSetAttribute(pref, CUBLASLT_MATMUL_PREF_MIN_ALIGNMENT_A_BYTES, &aA, sizeof(aA));
     cublasLtMatmulPreferenceSetAttribute(pref, CUBLASLT_MATMUL_PREF_MIN_ALIGNMENT_B_BYTES, &aB, sizeof(aB));
     cublasLtMatmulPreferenceSetAttribute(pref, CUBLASLT_MATMUL_PREF_MIN_ALIGNMENT_C_BYTES, &aC, sizeof(aC));
@@ -586,19 +600,18 @@ extern "C" int stca_output_backward(stca_handle* H, int layer, const float* C, i
   float* Oh = static_cast<float*>(H->bw_ws);
   float* dOh = Oh + td;
   const int64_t hd = static_cast<int64_t>(h) * d;
-  for (int j = 0; j < h; ++j)     // Oh[:, j] = C_j W_V[:, j]   (T x d_h)
-    if (int rc = gemm_rm(H, false, false, T, dh, d, C + j * d, hd, Wl.Wv + j * dh, d, Oh + j * dh, d, 0.f, s))
-      return rc;
+  // per head j (one batched product each): operands step by d (C_j), d_h (column slices)
+  // Oh[:, j] = C_j W_V[:, j]   (T x d_h)
+  if (int rc = gemm_rm(H, false, false, T, dh, d, C, hd, Wl.Wv, d, Oh, d, 0.f, s, 1.f, h, d, dh, dh))
+    return rc;
   // dW_O = Oh^T dZ, dOh = dZ W_O^T
   if (int rc = gemm_rm(H, true, false, d, d, T, Oh, d, dZ, d, dWo, d, 0.f, s)) return rc;
   if (int rc = gemm_rm(H, false, true, T, d, d, dZ, d, Wl.Wo, d, dOh, d, 0.f, s)) return rc;
-  for (int j = 0; j < h; ++j) {
-    // dC_j = dOh[:, j] W_V[:, j]^T  (T x d),  dW_V[:, j] = C_j^T dOh[:, j]  (d x d_h)
-    if (int rc = gemm_rm(H, false, true, T, d, dh, dOh + j * dh, d, Wl.Wv + j * dh, d, dC + j * d, hd, 0.f, s))
-      return rc;
-    if (int rc = gemm_rm(H, true, false, d, dh, T, C + j * d, hd, dOh + j * dh, d, dWv + j * dh, d, 0.f, s))
-      return rc;
-  }
+  // dC_j = dOh[:, j] W_V[:, j]^T  (T x d),  dW_V[:, j] = C_j^T dOh[:, j]  (d x d_h)
+  if (int rc = gemm_rm(H, false, true, T, d, dh, dOh, d, Wl.Wv, d, dC, hd, 0.f, s, 1.f, h, dh, dh, d))
+    return rc;
+  if (int rc = gemm_rm(H, true, false, d, dh, T, C, hd, dOh, d, dWv, d, 0.f, s, 1.f, h, d, dh, dh))
+    return rc;
   STCA_CUDA_TRY(cudaGetLastError());
   set_error(STCA_OK, "");
   return STCA_OK;
@@ -625,16 +638,14 @@ extern "C" int stca_query_backward(stca_handle* H, int layer, const float* Q, in
   float* dP = P + td;
   const int64_t hd = static_cast<int64_t>(h) * d;
   if (int rc = gemm_rm(H, false, false, T, d, d, Q, d, Wl.Wq, d, P, d, 0.f, s)) return rc;
-  for (int j = 0; j < h; ++j) {
-    // W_K^j is stored transposed: WkT[j] (d_h x d) = W_K[:, j]^T
-    const float* WkTj = Wl.WkT + static_cast<size_t>(j) * dh * d;
-    // dP[:, j] = scale dU_j W_K^j   (T x d_h)
-    if (int rc = gemm_rm(H, false, true, T, dh, d, dU + j * d, hd, WkTj, d, dP + j * dh, d, 0.f, s, scale))
-      return rc;
-    // dW_K[:, j] = scale dU_j^T P[:, j]   (d x d_h)
-    if (int rc = gemm_rm(H, true, false, d, dh, T, dU + j * d, hd, P + j * dh, d, dWk + j * dh, d, 0.f, s, scale))
-      return rc;
-  }
+  // per head j, batched: W_K^j is stored transposed, WkT[j] (d_h x d) = W_K[:, j]^T,
+  // WkT[j] = WkT + j d_h d.  dP[:, j] = scale dU_j W_K^j   (T x d_h)
+  const int64_t wk_step = static_cast<int64_t>(dh) * d;
+  if (int rc = gemm_rm(H, false, true, T, dh, d, dU, hd, Wl.WkT, d, dP, d, 0.f, s, scale, h, d, wk_step, dh))
+    return rc;
+  // dW_K[:, j] = scale dU_j^T P[:, j]   (d x d_h)
+  if (int rc = gemm_rm(H, true, false, d, dh, T, dU, hd, P, d, dWk, d, 0.f, s, scale, h, d, dh, dh))
+    return rc;
   // dQ = dP W_Q^T, dW_Q = Q^T dP
   if (int rc = gemm_rm(H, false, true, T, d, d, dP, d, Wl.Wq, d, dQ, d, 0.f, s)) return rc;
   if (int rc = gemm_rm(H, true, false, d, d, T, Q, d, dP, d, dWq, d, 0.f, s)) return rc;
