@@ -1,4 +1,4 @@
-"""Plain fp64 CPU oracle of the backward pass of two pieces of the STCA forward
+"""Plain fp64 CPU oracle of the backward pass of the pieces of the STCA forward
 -- TEST INFRASTRUCTURE ONLY.
 
 Only tests/, __graft_entry__.smoke() and bench.py's CPU-baseline / reference
@@ -6,8 +6,10 @@ legs may import or run this module.  The product path (the CUDA library and its
 Python binding) never calls it and shares no code with it.
 
 Sources: "Make It Long, Keep It Fast" digest §2.1, Eqs. (1)-(2) (the history
-encoding X~ = LN(SwiGLUFFN(X))) and Eq. (13) (the reordered single-query
-attention, alpha = softmax(u X~^T), c = alpha X~); the STCA blog §2.5 (request-
+encoding X~ = LN(SwiGLUFFN(X))), Eq. (3) (the query init), Eq. (13) (the
+reordered single-query attention, alpha = softmax(u X~^T), c = alpha X~, with
+the projections W_Q, W_K, W_V and W_O of Eq. (6)), Eq. (7) (the W_C fusion) and
+Eq. (9) (the prediction head); the STCA blog §2.5 (request-
 level batching trains with the history encoded once for all of a request's
 targets, so the gradient of X~ sums over every target and head).
 
@@ -131,3 +133,44 @@ def query_backward(Q, Wq, Wk, h, dU):
     dP = np.concatenate([s * dU[:, j, :] @ Wk[:, j * dh:(j + 1) * dh] for j in range(h)], axis=-1)
     dWk = np.concatenate([s * dU[:, j, :].T @ P[:, j * dh:(j + 1) * dh] for j in range(h)], axis=-1)
     return dP @ Wq.T, Q.T @ dP, dWk
+
+
+def ffn_backward(x, Wu, Wg, Wd, dy):
+    """Gradients of <((x W_u) * SiLU(x W_g)) W_d, dy>: the SwiGLU FFN with no
+    LayerNorm (Eq. (1) as Eqs. (7) and (9) use it).  Returns dx, dWu, dWg, dWd."""
+    x, Wu, Wg, Wd, dy = _f64(x), _f64(Wu), _f64(Wg), _f64(Wd), _f64(dy)
+    a = x @ Wu
+    g = x @ Wg
+    sg = sigmoid(g)
+    H = a * (g * sg)
+    dH = dy @ Wd.T
+    da = dH * (g * sg)
+    dg = dH * a * sg * (1.0 + g * (1.0 - sg))
+    return da @ Wu.T + dg @ Wg.T, x.T @ da, x.T @ dg, H.T @ dy
+
+
+def fusion_backward(outs, xt, Wc, Wu, Wg, Wd, dy):
+    """Gradients of <SwiGLUFFN([o^(1) || ... || o^(i) || x_t] W_C), dy>.
+
+    Eq. (7) (W_C of layer i+1 and that layer's query FFN) and Eq. (9) (W_Z
+    and the head's FFN) have this form, x_t the last block (reading O8).
+    Returns (douts: list of (T, d), dxt, dWc, dWu, dWg, dWd)."""
+    outs = [_f64(o) for o in outs]
+    cat = np.concatenate(outs + [_f64(xt)], axis=-1)
+    a = cat @ _f64(Wc)
+    da, dWu, dWg, dWd = ffn_backward(a, Wu, Wg, Wd, dy)
+    dcat = da @ _f64(Wc).T
+    d = outs[0].shape[1] if outs else _f64(xt).shape[1]
+    douts = [dcat[:, k * d:(k + 1) * d] for k in range(len(outs))]
+    return douts, dcat[:, len(outs) * d:], cat.T @ da, dWu, dWg, dWd
+
+
+def query_init_backward(xt, W, dq):
+    """Gradients of <q^(1), dq> with q^(1) = LN(SwiGLUFFN^(1)(x_t)) (Eq. (3),
+    reading O5: the query FFN and query LayerNorm weights, which default to
+    layer 1's).  Returns the encode_history_backward dict (dX is dx_t)."""
+    q = {"Wu": [W["qWu"][0] if W.get("qWu") is not None else W["Wu"][0]],
+         "Wg": [W["qWg"][0] if W.get("qWg") is not None else W["Wg"][0]],
+         "Wd": [W["qWd"][0] if W.get("qWd") is not None else W["Wd"][0]],
+         "ln_g": [W["q_ln_g"] if W.get("q_ln_g") is not None else W["ln_g"][0]]}
+    return encode_history_backward(xt, q, 0, dq)

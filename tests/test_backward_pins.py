@@ -174,6 +174,138 @@ def test_attention_layer_chain_matches_forward_oracle():
     pin_layer_chain()
 
 
+def _fd_check(loss, args, grads, rng, tag):
+    eps = 1e-6
+    for i, g in enumerate(grads):
+        if g is None:
+            continue
+        V = rng.standard_normal(np.shape(g))
+        a1 = list(args); a1[i] = a1[i] + eps * V
+        a2 = list(args); a2[i] = a2[i] - eps * V
+        fd = (loss(a1) - loss(a2)) / (2 * eps)
+        assert abs(fd - float((np.asarray(g) * V).sum())) <= 1e-6 * max(1.0, abs(fd)), (tag, i)
+
+
+def _tiny_weights(rng, d, h, M, r):
+    from gen import make_workload
+    wl = make_workload(lengths=[5], targets=[2], d=d, h=h, M=M, r=r, dtype="f32", seed=int(rng.integers(1 << 30)),
+                       random_ln=True, distinct_query_ffn=True)
+    return {k: (None if v is None else ([None if a is None else np.asarray(a, np.float64) for a in v]
+                                        if isinstance(v, list) else np.asarray(v, np.float64)))
+            for k, v in wl.weights.items()}
+
+
+def pin_fusion_head_query_init():
+    """Eq. (7) fusion, Eq. (9) head and Eq. (3) query init against finite
+    differences of the forward oracle's query_fusion, prediction_head, query_init."""
+    rng = np.random.default_rng(9)
+    T, d, h, M, r = 3, 4, 2, 3, 2
+    W = _tiny_weights(rng, d, h, M, r)
+    outs = [rng.standard_normal((T, d)) for _ in range(M)]
+    xt = rng.standard_normal((T, d))
+    dy = rng.standard_normal((T, d))
+    # fusion into layer 3 (index 2): q^(3) from o^(1), o^(2), x_t
+    i = 2
+    douts, dxt, dWc, dWu, dWg, dWd = B.fusion_backward(outs[:i], xt, W["Wc"][i], W["qWu"][i], W["qWg"][i],
+                                                       W["qWd"][i], dy)
+
+    def fusion_loss(a):
+        Wd_ = dict(W)
+        Wd_["Wc"] = list(W["Wc"]); Wd_["Wc"][i] = a[3]
+        Wd_["qWu"] = list(W["qWu"]); Wd_["qWu"][i] = a[4]
+        return float((O.query_fusion([a[0], a[1]], a[2], Wd_, i) * dy).sum())
+    _fd_check(fusion_loss, [outs[0], outs[1], xt, W["Wc"][i], W["qWu"][i]],
+              [douts[0], douts[1], dxt, dWc, dWu], rng, "fusion")
+    # the prediction head over all M outputs
+    douts, dxt, dWz, dzu, dzg, dzd = B.fusion_backward(outs, xt, W["Wz"], W["zWu"], W["zWg"], W["zWd"], dy)
+
+    def head_loss(a):
+        Wd_ = dict(W, Wz=a[4], zWg=a[5], zWd=a[6])
+        return float((O.prediction_head(a[:3], a[3], Wd_) * dy).sum())
+    _fd_check(head_loss, outs + [xt, W["Wz"], W["zWg"], W["zWd"]], douts + [dxt, dWz, dzg, dzd], rng, "head")
+    # the query init
+    g = B.query_init_backward(xt, W, dy)
+
+    def init_loss(a):
+        Wd_ = dict(W, q_ln_g=a[1])
+        Wd_["qWd"] = list(W["qWd"]); Wd_["qWd"][0] = a[2]
+        return float((O.query_init(a[0], Wd_) * dy).sum())
+    _fd_check(init_loss, [xt, W["q_ln_g"], W["qWd"][0]], [g["dX"], g["dgamma"], g["dWd"]], rng, "init")
+
+
+def request_backward(X, xt, W, h, GZ, Gz):
+    """Gradient of <Z, GZ> + <z, Gz> for one request, Z of Eq. (8) and z of
+    Eq. (9), by chaining the backward pieces from the head down to layer 1.
+    Returns dX, dxt and a few weight gradients."""
+    M = len(W["Wu"])
+    T, d = xt.shape
+    dh = d // h
+    Xts = [O.encode_history(X, W, i) for i in range(M)]
+    qs, Us, Cs, outs = [O.query_init(xt, W)], [], [], []
+    for i in range(M):
+        q = qs[-1]
+        U = np.stack([(q @ W["Wq"][i][:, j * dh:(j + 1) * dh]) @ W["Wk"][i][:, j * dh:(j + 1) * dh].T / np.sqrt(dh)
+                      for j in range(h)], axis=1)
+        C = np.stack([O.softmax(U[:, j] @ Xts[i].T) @ Xts[i] for j in range(h)], axis=1)
+        Us.append(U); Cs.append(C)
+        outs.append(O.attention_reordered(q, Xts[i], W["Wq"][i], W["Wk"][i], W["Wv"][i], W["Wo"][i], h))
+        if i + 1 < M:
+            qs.append(O.query_fusion(outs, xt, W, i + 1))
+    douts, dxt, dWz, _, _, _ = B.fusion_backward(outs, xt, W["Wz"], W["zWu"], W["zWg"], W["zWd"], Gz)
+    dO = [GZ[:, i] + douts[i] for i in range(M)]
+    dX = np.zeros_like(X)
+    grads = {"dWz": dWz}
+    for i in reversed(range(M)):
+        dC, dWv, _ = B.output_backward(Cs[i], W["Wv"][i], W["Wo"][i], h, dO[i])
+        dU, dXt = B.attention_rows_backward(Us[i].reshape(T * h, d), Xts[i], dC.reshape(T * h, d))
+        dX += B.encode_history_backward(X, W, i, dXt)["dX"]
+        dq, dWq, _ = B.query_backward(qs[i], W["Wq"][i], W["Wk"][i], h, dU.reshape(T, h, d))
+        grads[f"dWv{i}"], grads[f"dWq{i}"] = dWv, dWq
+        if i > 0:
+            dprev, dx_i, dWc, _, _, _ = B.fusion_backward(outs[:i], xt, W["Wc"][i], W["qWu"][i], W["qWg"][i],
+                                                          W["qWd"][i], dq)
+            for k in range(i):
+                dO[k] = dO[k] + dprev[k]
+            dxt = dxt + dx_i
+            grads[f"dWc{i}"] = dWc
+        else:
+            dxt = dxt + B.query_init_backward(xt, W, dq)["dX"]
+    grads["dX"], grads["dxt"] = dX, dxt
+    return grads
+
+
+def pin_request_chain():
+    """Every backward piece chained over a whole request (M = 2, with the head)
+    against finite differences of the forward oracle's forward_request and
+    prediction head."""
+    rng = np.random.default_rng(10)
+    L, T, d, h, M, r = 5, 2, 4, 2, 2, 2
+    W = _tiny_weights(rng, d, h, M, r)
+    X = rng.standard_normal((L, d))
+    xt = rng.standard_normal((T, d))
+    GZ = rng.standard_normal((T, M, d))
+    Gz = rng.standard_normal((T, d))
+    g = request_backward(X, xt, W, h, GZ, Gz)
+
+    def loss(a):
+        Wd_ = dict(W, Wz=a[2])
+        for key, idx, pos in (("Wv", 0, 3), ("Wq", 1, 4), ("Wc", 1, 5)):
+            Wd_[key] = list(W[key]); Wd_[key][idx] = a[pos]
+        Z = O.forward_request(a[0], a[1], Wd_, h)
+        z = O.head_from_outputs(Z, a[1], Wd_)
+        return float((Z * GZ).sum() + (z * Gz).sum())
+    _fd_check(loss, [X, xt, W["Wz"], W["Wv"][0], W["Wq"][1], W["Wc"][1]],
+              [g["dX"], g["dxt"], g["dWz"], g["dWv0"], g["dWq1"], g["dWc1"]], rng, "request")
+
+
+def test_fusion_head_query_init_finite_differences():
+    pin_fusion_head_query_init()
+
+
+def test_request_chain_matches_forward_oracle():
+    pin_request_chain()
+
+
 def test_output_and_query_backward_finite_differences():
     pin_output_query_finite_differences()
 
@@ -244,6 +376,26 @@ def _enc_sigmoid_derivative(X, W, i, dXt, eps=1e-5):
 
 _output_backward = B.output_backward
 _query_backward = B.query_backward
+_fusion_backward = B.fusion_backward
+
+
+def _fusion_xt_first(outs, xt, Wc, Wu, Wg, Wd, dy):
+    cat = np.concatenate([np.asarray(xt, np.float64)] + [np.asarray(o, np.float64) for o in outs], axis=-1)
+    a = cat @ np.asarray(Wc, np.float64)
+    da, dWu, dWg, dWd = B.ffn_backward(a, Wu, Wg, Wd, dy)
+    dcat = da @ np.asarray(Wc, np.float64).T
+    d = np.asarray(xt).shape[1]
+    return ([dcat[:, (k + 1) * d:(k + 2) * d] for k in range(len(outs))], dcat[:, :d], cat.T @ da,
+            dWu, dWg, dWd)
+
+
+def _ffn_silu_term_dropped(x, Wu, Wg, Wd, dy):
+    x, Wu, Wg, Wd, dy = (np.asarray(t, np.float64) for t in (x, Wu, Wg, Wd, dy))
+    a, g = x @ Wu, x @ Wg
+    sg = O.sigmoid(g)
+    dH = dy @ Wd.T
+    da, dg = dH * g * sg, dH * a * sg            # the g (1 - sigmoid(g)) term dropped
+    return da @ Wu.T + dg @ Wg.T, x.T @ da, x.T @ dg, (a * g * sg).T @ dy
 
 
 def _out_wrong_transpose(C, Wv, Wo, h, dZ):
@@ -286,6 +438,8 @@ MUTANTS = {
     "query_replaced": ("attention_rows_backward", _attn_transposed),
     "wo_gradient_transposed": ("output_backward", _out_wrong_transpose),
     "query_scale_dropped": ("query_backward", _query_no_scale),
+    "fusion_xt_first": ("fusion_backward", _fusion_xt_first),
+    "ffn_silu_term_dropped": ("ffn_backward", _ffn_silu_term_dropped),
 }
 
 
@@ -295,7 +449,8 @@ def test_pins_reject_mutant(name, monkeypatch):
     monkeypatch.setattr(B, attr, fn)
     failed = 0
     for pin in (pin_encoder_finite_differences, pin_attention_finite_differences, pin_torch_autograd,
-                pin_invariances, pin_output_query_finite_differences, pin_layer_chain):
+                pin_invariances, pin_output_query_finite_differences, pin_layer_chain,
+                pin_fusion_head_query_init, pin_request_chain):
         try:
             pin()
         except AssertionError:
