@@ -596,10 +596,30 @@ def run_ours(args, rank, world, local_rank):
                 S.stca_output_backward(st.handle, 0, dC, dZb, wl.h, stream)
                 S.stca_query_backward(st.handle, 0, Qb, Ub, wl.h, stream)
             b3.record(stream)
+            # the query side of the step: the head (block M), the Eq. (7) fusion blocks
+            # M-1 .. 1 (accumulating into dZ and dx_t), then the Eq. (3) query init
+            dZf = torch.zeros((wl.T, wl.M, wl.d), dtype=torch.float32, device=dev)
+            dxf = torch.zeros((wl.T, wl.d), dtype=torch.float32, device=dev)
+
+            def query_side():
+                for blk in range(wl.M, 0, -1):
+                    S.stca_fusion_backward(st.handle, blk, Z, xt, dZb, wl.r * wl.d, dZ=dZf, dxt=dxf,
+                                           accumulate=True, stream=stream)
+                S.stca_query_init_backward(st.handle, xt, dZb, wl.r * wl.d, stream)
+            query_side()
+            b4 = torch.cuda.Event(enable_timing=True)
+            b5 = torch.cuda.Event(enable_timing=True)
+            b4.record(stream)
+            for _ in range(nrep):
+                query_side()
+            b5.record(stream)
         torch.cuda.synchronize()
         st.status(stream)
         enc_ms, att_ms = b0.elapsed_time(b1) / nrep, b1.elapsed_time(b2) / nrep
         proj_ms = b2.elapsed_time(b3) / nrep
+        qside_ms = b4.elapsed_time(b5) / nrep
+        d_, rd_, T_ = wl.d, wl.r * wl.d, wl.T
+        qside_fl = sum(6 * T_ * (b + 1) * d_ * d_ + 16 * T_ * d_ * rd_ for b in range(1, wl.M + 1)) + 18 * T_ * d_ * rd_
         rd = wl.r * wl.d
         enc_fl = 18 * wl.N * wl.d * rd              # recomputed forward (6 N d rd) + 6 backward products
         att_fl = 18 * wl.d * c["TL"] * wl.h         # per (row, key): 2 passes of 2 dots + dU; 2 dots + dX~
@@ -615,7 +635,10 @@ def run_ours(args, rank, world, local_rank):
                           "note": "CUDA-core flash-style kernels (softmax recomputed)"},
             "projections": {"ms": proj_ms, "flops": 20 * wl.T * wl.d * wl.d,
                             "note": "output side (W_V, W_O) and query side (W_Q, W_K): "
-                                    "cuBLASLt TF32 products, the per-head slices as strided batches"}}
+                                    "cuBLASLt TF32 products, the per-head slices as strided batches"},
+            "query_side": {"ms": qside_ms, "flops": qside_fl,
+                           "note": "the head (Eq. (9)), the M-1 fusion blocks (Eq. (7)) and the query init "
+                                   "(Eq. (3)): cuBLASLt TF32 products + SwiGLU / LayerNorm derivative kernels"}}
 
     # ---- the sparse-training batch builder and a forward over its packed batch
     train_batch = None

@@ -377,6 +377,38 @@ int stca_output_backward(stca_handle* handle, int layer, const float* C, int64_t
 int stca_query_backward(stca_handle* handle, int layer, const float* Q, int64_t T,
                         const float* dU, float* dQ, float* dWq, float* dWk, void* stream);
 
+/*
+ * Query init (digest Eq. (3)): q^(1) = LN(SwiGLUFFN(x_t)) with the query FFN and
+ * query LayerNorm weights (layer 1's unless given separately).  Given the
+ * targets x_t (DEVICE, T x d, handle dtype) and dq (T x d fp32, the gradient of
+ * q^(1)), writes dxt (T x d fp32; may be NULL), dWu, dWg (d x rd), dWd (rd x d),
+ * dgamma, dbeta (d), all DEVICE, caller-owned.  Recomputes the forward in fp32.
+ * Errors: STCA_EINVAL, STCA_ENOMEM, STCA_ECUDA.
+ */
+int stca_query_init_backward(stca_handle* handle, const void* targets, int64_t T, const float* dq,
+                             float* dxt, float* dWu, float* dWg, float* dWd, float* dgamma,
+                             float* dbeta, void* stream);
+
+/*
+ * A fusion block: y = SwiGLUFFN([o^(1) || ... || o^(b) || x_t] W), x_t last.
+ *   block b in [1, M-1]: Eq. (7), the next query q^(b+1), with W = W_C of layer
+ *     b+1 ((b+1) d x d) and that layer's query FFN;
+ *   block b = M: Eq. (9), the prediction-head token z, with W = W_Z
+ *     ((M+1) d x d) and the head's FFN (needs the head weights at stca_init).
+ * Z: (T, M, d) fp32 as stca_forward writes it; only o^(1..b), the first b d
+ * columns of each row, are read.  targets: T x d, handle dtype.  dy: T x d
+ * fp32, the gradient of y.  Writes dZ's first b d columns of each row (row
+ * stride M d; the other columns are not touched) and dxt (T x d), overwriting
+ * them, or adding to them when `accumulate` is nonzero (o^(1) and x_t feed
+ * several blocks).  Writes dW ((b+1) d x d), dWu, dWg (d x rd), dWd (rd x d).
+ * All DEVICE pointers, caller-owned.  T = 0 writes zero weight gradients.
+ * Errors: STCA_EINVAL (bad block, no head weights for block M), STCA_ENOMEM,
+ * STCA_ECUDA.
+ */
+int stca_fusion_backward(stca_handle* handle, int block, const float* Z, const void* targets,
+                         int64_t T, const float* dy, int accumulate, float* dZ, float* dxt,
+                         float* dW, float* dWu, float* dWg, float* dWd, void* stream);
+
 /* Tunables and introspection (STCA_OPT_*).  Values are validated. */
 enum {
   STCA_OPT_ATTN_PATH = 1,     /* 0 auto, 1 CUDA cores, 2 tensor cores (bf16 only) */

@@ -439,20 +439,16 @@ int ensure(void** p, size_t* cap, size_t bytes) {
 
 using namespace stca;
 
-extern "C" int stca_encode_backward(stca_handle* H, int layer, const void* X, int64_t N,
-                                    const float* dXt, float* dX, float* dWu, float* dWg,
-                                    float* dWd, float* dgamma, float* dbeta, void* stream) {
-  if (!H) return set_error(STCA_EINVAL, "handle is NULL");
-  if (layer < 0 || layer >= H->M) return set_error(STCA_EINVAL, "layer out of range");
-  if (N < 1 || N > (int64_t(1) << 31)) return set_error(STCA_EINVAL, "N must be in [1, 2^31]");
-  if (!X || !dXt || !dWu || !dWg || !dWd || !dgamma || !dbeta)
-    return set_error(STCA_EINVAL, "stca_encode_backward: NULL argument");
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev != H->device) cudaSetDevice(H->device);
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
+namespace {
+
+// Backward of Y = LN(((X W_u) * SiLU(X W_g)) W_d) with LN's scale gamma, for N
+// rows of X (handle dtype): the history encoding of Eqs. (1)-(2) and, with the
+// query weights, the query init of Eq. (3).  dX may be NULL.
+int ffn_ln_backward(stca_handle* H, const void* X, int64_t N, const float* dXt, float* dX,
+                    const float* Wu, const float* Wg, const float* Wd, const float* gamma, float* dWu,
+                    float* dWg, float* dWd, float* dgamma, float* dbeta, cudaStream_t s) {
   const int d = H->d, rd = H->rd;
-  const LayerW32& Wl = H->L32[layer];
+  if (d > 32 * kLnMaxCols) return set_error(STCA_EINVAL, "encoder backward needs d <= 256");
   // workspace: Xf (N d), A (N rd), G (N rd), Hh (N rd), Y (N d)
   const size_t nd = static_cast<size_t>(N) * d, nr = static_cast<size_t>(N) * rd;
   if (int rc = ensure(&H->bw_ws, &H->bw_ws_cap, (2 * nd + 3 * nr) * sizeof(float))) return rc;
@@ -467,30 +463,62 @@ extern "C" int stca_encode_backward(stca_handle* H, int layer, const void* X, in
     STCA_CUDA_TRY(cudaMemcpyAsync(Xf, X, nd * sizeof(float), cudaMemcpyDeviceToDevice, s));
   }
   // forward recomputation: A = X W_u, G = X W_g, H = A SiLU(G), Y = H W_d
-  if (int rc = gemm_rm(H, false, false, N, rd, d, Xf, d, Wl.Wu, rd, A, rd, 0.f, s)) return rc;
-  if (int rc = gemm_rm(H, false, false, N, rd, d, Xf, d, Wl.Wg, rd, G, rd, 0.f, s)) return rc;
+  if (int rc = gemm_rm(H, false, false, N, rd, d, Xf, d, Wu, rd, A, rd, 0.f, s)) return rc;
+  if (int rc = gemm_rm(H, false, false, N, rd, d, Xf, d, Wg, rd, G, rd, 0.f, s)) return rc;
   swiglu_fwd_kernel<<<grid_for(nr), 256, 0, s>>>(A, G, Hh, nr);
-  if (int rc = gemm_rm(H, false, false, N, d, rd, Hh, rd, Wl.Wd, d, Y, d, 0.f, s)) return rc;
+  if (int rc = gemm_rm(H, false, false, N, d, rd, Hh, rd, Wd, d, Y, d, 0.f, s)) return rc;
   // LayerNorm: Y <- dy; dgamma, dbeta
   STCA_CUDA_TRY(cudaMemsetAsync(dgamma, 0, d * sizeof(float), s));
   STCA_CUDA_TRY(cudaMemsetAsync(dbeta, 0, d * sizeof(float), s));
-  if (d > 32 * kLnMaxCols) return set_error(STCA_EINVAL, "encoder backward needs d <= 256");
-  ln_bwd_kernel<<<static_cast<unsigned>((N + kLnRows - 1) / kLnRows), 256, 0, s>>>(Y, dXt, Wl.ln_g, dgamma,
+  ln_bwd_kernel<<<static_cast<unsigned>((N + kLnRows - 1) / kLnRows), 256, 0, s>>>(Y, dXt, gamma, dgamma,
                                                                                    dbeta, N, d);
   // dW_d = H^T dy; dH = dy W_d^T (over H)
   if (int rc = gemm_rm(H, true, false, rd, d, N, Hh, rd, Y, d, dWd, d, 0.f, s)) return rc;
-  if (int rc = gemm_rm(H, false, true, N, rd, d, Y, d, Wl.Wd, d, Hh, rd, 0.f, s)) return rc;
+  if (int rc = gemm_rm(H, false, true, N, rd, d, Y, d, Wd, d, Hh, rd, 0.f, s)) return rc;
   swiglu_bwd_kernel<<<grid_for(nr), 256, 0, s>>>(A, G, Hh, nr);
   // dW_u = X^T dA, dW_g = X^T dG; dX = dA W_u^T + dG W_g^T
   if (int rc = gemm_rm(H, true, false, d, rd, N, Xf, d, A, rd, dWu, rd, 0.f, s)) return rc;
   if (int rc = gemm_rm(H, true, false, d, rd, N, Xf, d, G, rd, dWg, rd, 0.f, s)) return rc;
   if (dX) {
-    if (int rc = gemm_rm(H, false, true, N, d, rd, A, rd, Wl.Wu, rd, dX, d, 0.f, s)) return rc;
-    if (int rc = gemm_rm(H, false, true, N, d, rd, G, rd, Wl.Wg, rd, dX, d, 1.f, s)) return rc;
+    if (int rc = gemm_rm(H, false, true, N, d, rd, A, rd, Wu, rd, dX, d, 0.f, s)) return rc;
+    if (int rc = gemm_rm(H, false, true, N, d, rd, G, rd, Wg, rd, dX, d, 1.f, s)) return rc;
   }
   STCA_CUDA_TRY(cudaGetLastError());
   set_error(STCA_OK, "");
   return STCA_OK;
+}
+
+}  // namespace
+
+extern "C" int stca_encode_backward(stca_handle* H, int layer, const void* X, int64_t N,
+                                    const float* dXt, float* dX, float* dWu, float* dWg,
+                                    float* dWd, float* dgamma, float* dbeta, void* stream) {
+  if (!H) return set_error(STCA_EINVAL, "handle is NULL");
+  if (layer < 0 || layer >= H->M) return set_error(STCA_EINVAL, "layer out of range");
+  if (N < 1 || N > (int64_t(1) << 31)) return set_error(STCA_EINVAL, "N must be in [1, 2^31]");
+  if (!X || !dXt || !dWu || !dWg || !dWd || !dgamma || !dbeta)
+    return set_error(STCA_EINVAL, "stca_encode_backward: NULL argument");
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev != H->device) cudaSetDevice(H->device);
+  const LayerW32& Wl = H->L32[layer];
+  return ffn_ln_backward(H, X, N, dXt, dX, Wl.Wu, Wl.Wg, Wl.Wd, Wl.ln_g, dWu, dWg, dWd, dgamma, dbeta,
+                         static_cast<cudaStream_t>(stream));
+}
+
+extern "C" int stca_query_init_backward(stca_handle* H, const void* targets, int64_t T, const float* dq,
+                                        float* dxt, float* dWu, float* dWg, float* dWd, float* dgamma,
+                                        float* dbeta, void* stream) {
+  if (!H) return set_error(STCA_EINVAL, "handle is NULL");
+  if (T < 1 || T > (int64_t(1) << 31)) return set_error(STCA_EINVAL, "T must be in [1, 2^31]");
+  if (!targets || !dq || !dWu || !dWg || !dWd || !dgamma || !dbeta)
+    return set_error(STCA_EINVAL, "stca_query_init_backward: NULL argument");
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev != H->device) cudaSetDevice(H->device);
+  const LayerW32& W0 = H->L32[0];
+  return ffn_ln_backward(H, targets, T, dq, dxt, W0.qWu, W0.qWg, W0.qWd, H->q_ln_g, dWu, dWg, dWd, dgamma,
+                         dbeta, static_cast<cudaStream_t>(stream));
 }
 
 extern "C" int stca_attention_backward(stca_handle* H, int layer, const float* U,
@@ -649,6 +677,80 @@ extern "C" int stca_query_backward(stca_handle* H, int layer, const float* Q, in
   // dQ = dP W_Q^T, dW_Q = Q^T dP
   if (int rc = gemm_rm(H, false, true, T, d, d, dP, d, Wl.Wq, d, dQ, d, 0.f, s)) return rc;
   if (int rc = gemm_rm(H, true, false, d, d, T, Q, d, dP, d, dWq, d, 0.f, s)) return rc;
+  STCA_CUDA_TRY(cudaGetLastError());
+  set_error(STCA_OK, "");
+  return STCA_OK;
+}
+
+extern "C" int stca_fusion_backward(stca_handle* H, int block, const float* Z, const void* targets, int64_t T,
+                                    const float* dy, int accumulate, float* dZ, float* dxt, float* dW,
+                                    float* dWu, float* dWg, float* dWd, void* stream) {
+  if (!H) return set_error(STCA_EINVAL, "handle is NULL");
+  if (block < 1 || block > H->M) return set_error(STCA_EINVAL, "block must be in [1, M]");
+  if (block == H->M && !H->hWz32)
+    return set_error(STCA_EINVAL, "block M is the prediction head: the handle has no head weights");
+  if (T < 0 || T > (int64_t(1) << 31)) return set_error(STCA_EINVAL, "T out of range");
+  if (!dW || !dWu || !dWg || !dWd || (T > 0 && (!Z || !targets || !dy || !dZ || !dxt)))
+    return set_error(STCA_EINVAL, "stca_fusion_backward: NULL argument");
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev != H->device) cudaSetDevice(H->device);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int d = H->d, rd = H->rd, M = H->M;
+  const int64_t bd = static_cast<int64_t>(block) * d, Md = static_cast<int64_t>(M) * d;
+  // block b < M: W_C of layer b+1 (0-based b) with that layer's query FFN (Eq. (7));
+  // block M: W_Z with the head's FFN (Eq. (9))
+  const bool head = block == M;
+  const float* W = head ? H->hWz32 : H->L32[block].Wc;
+  const float* Wu = head ? H->hWu32 : H->L32[block].qWu;
+  const float* Wg = head ? H->hWg32 : H->L32[block].qWg;
+  const float* Wd = head ? H->hWd32 : H->L32[block].qWd;
+  if (T == 0) {
+    STCA_CUDA_TRY(cudaMemsetAsync(dW, 0, static_cast<size_t>(bd + d) * d * sizeof(float), s));
+    STCA_CUDA_TRY(cudaMemsetAsync(dWu, 0, static_cast<size_t>(d) * rd * sizeof(float), s));
+    STCA_CUDA_TRY(cudaMemsetAsync(dWg, 0, static_cast<size_t>(d) * rd * sizeof(float), s));
+    STCA_CUDA_TRY(cudaMemsetAsync(dWd, 0, static_cast<size_t>(rd) * d * sizeof(float), s));
+    set_error(STCA_OK, "");
+    return STCA_OK;
+  }
+  // workspace: xf (T d), a (T d), da (T d), A, G, Hh (T rd each)
+  const size_t nd = static_cast<size_t>(T) * d, nr = static_cast<size_t>(T) * rd;
+  if (int rc = ensure(&H->bw_ws, &H->bw_ws_cap, (3 * nd + 3 * nr) * sizeof(float))) return rc;
+  float* xf = static_cast<float*>(H->bw_ws);
+  float* a = xf + nd;
+  float* da = a + nd;
+  float* A = da + nd;
+  float* G = A + nr;
+  float* Hh = G + nr;
+  if (H->elem == 2) {
+    to_f32_kernel<<<grid_for(nd), 256, 0, s>>>(static_cast<const uint16_t*>(targets), xf, nd);
+  } else {
+    STCA_CUDA_TRY(cudaMemcpyAsync(xf, targets, nd * sizeof(float), cudaMemcpyDeviceToDevice, s));
+  }
+  const float* Wx = W + bd * d;           // the rows of W that multiply x_t (the last block)
+  // a = [o^(1) .. o^(b)] W[:b d] + x_t W[b d:]: the first b d columns of each Z row, then x_t
+  if (int rc = gemm_rm(H, false, false, T, d, bd, Z, Md, W, d, a, d, 0.f, s)) return rc;
+  if (int rc = gemm_rm(H, false, false, T, d, d, xf, d, Wx, d, a, d, 1.f, s)) return rc;
+  // the FFN forward recomputed: A = a W_u, G = a W_g, H = A SiLU(G)
+  if (int rc = gemm_rm(H, false, false, T, rd, d, a, d, Wu, rd, A, rd, 0.f, s)) return rc;
+  if (int rc = gemm_rm(H, false, false, T, rd, d, a, d, Wg, rd, G, rd, 0.f, s)) return rc;
+  swiglu_fwd_kernel<<<grid_for(nr), 256, 0, s>>>(A, G, Hh, nr);
+  // dW_d = H^T dy; dH = dy W_d^T (over H); dA, dG (over A, G)
+  if (int rc = gemm_rm(H, true, false, rd, d, T, Hh, rd, dy, d, dWd, d, 0.f, s)) return rc;
+  if (int rc = gemm_rm(H, false, true, T, rd, d, dy, d, Wd, d, Hh, rd, 0.f, s)) return rc;
+  swiglu_bwd_kernel<<<grid_for(nr), 256, 0, s>>>(A, G, Hh, nr);
+  // dW_u = a^T dA, dW_g = a^T dG, da = dA W_u^T + dG W_g^T
+  if (int rc = gemm_rm(H, true, false, d, rd, T, a, d, A, rd, dWu, rd, 0.f, s)) return rc;
+  if (int rc = gemm_rm(H, true, false, d, rd, T, a, d, G, rd, dWg, rd, 0.f, s)) return rc;
+  if (int rc = gemm_rm(H, false, true, T, d, rd, A, rd, Wu, rd, da, d, 0.f, s)) return rc;
+  if (int rc = gemm_rm(H, false, true, T, d, rd, G, rd, Wg, rd, da, d, 1.f, s)) return rc;
+  // dW = [Z[:, :b d] || x_t]^T da, by its two row blocks
+  if (int rc = gemm_rm(H, true, false, bd, d, T, Z, Md, da, d, dW, d, 0.f, s)) return rc;
+  if (int rc = gemm_rm(H, true, false, d, d, T, xf, d, da, d, dW + bd * d, d, 0.f, s)) return rc;
+  // d[o^(1) .. o^(b)] = da W[:b d]^T into the first b d columns of dZ; dx_t = da W[b d:]^T
+  const float beta = accumulate ? 1.f : 0.f;
+  if (int rc = gemm_rm(H, false, true, T, bd, d, da, d, W, d, dZ, Md, beta, s)) return rc;
+  if (int rc = gemm_rm(H, false, true, T, d, d, da, d, Wx, d, dxt, d, beta, s)) return rc;
   STCA_CUDA_TRY(cudaGetLastError());
   set_error(STCA_OK, "");
   return STCA_OK;

@@ -171,6 +171,7 @@ extern "C" void stca_destroy(stca_handle* H) {
   cudaFree(H->wstep);
   cudaFree(H->wstep_tc);
   cudaFree(H->whead);
+  cudaFree(H->w32head);
   cudaFree(H->wkv);
   cudaFree(H->kv);
   cudaFree(H->lt_ws);
@@ -418,6 +419,29 @@ extern "C" int stca_init(const stca_weights* w, int d, int h, int r, int M, int 
       stca_destroy(H);
       return rc2;
     }
+    // fp32 copies for the backward of Eq. (9): Wz, zWu, zWg, zWd back to back
+    const size_t n[4] = {wz.size(), zu.size(), zg.size(), zd.size()};
+    const float* src[4] = {wz.data(), zu.data(), zg.data(), zd.data()};
+    if (cudaMalloc(&H->w32head, (n[0] + n[1] + n[2] + n[3]) * sizeof(float)) != cudaSuccess) {
+      cudaGetLastError();
+      stca_destroy(H);
+      return set_error(STCA_ENOMEM, "prediction-head weight allocation failed");
+    }
+    const float* part[4];
+    size_t at = 0;
+    for (int k = 0; k < 4; ++k) {
+      part[k] = H->w32head + at;
+      if (cudaMemcpy(H->w32head + at, src[k], n[k] * sizeof(float), cudaMemcpyHostToDevice) != cudaSuccess) {
+        cudaGetLastError();
+        stca_destroy(H);
+        return set_error(STCA_ECUDA, "prediction-head weight upload failed");
+      }
+      at += n[k];
+    }
+    H->hWz32 = part[0];
+    H->hWu32 = part[1];
+    H->hWg32 = part[2];
+    H->hWd32 = part[3];
   }
   if (dtype == STCA_BF16 && encode_tc_supported(d, rd)) {
     std::vector<const float*> Wu(M), Wg(M), Wd(M);

@@ -123,6 +123,8 @@ struct stca_handle {
   bool step_tc_ready = false;
   void* whead = nullptr;                // prediction-head weights (dtype): Wz, [zWu | zWg], zWd
   const void *hWz = nullptr, *hWug = nullptr, *hWd = nullptr;
+  float* w32head = nullptr;             // the same in fp32, for the backward products:
+  const float *hWz32 = nullptr, *hWu32 = nullptr, *hWg32 = nullptr, *hWd32 = nullptr;  // Wz, zWu, zWg, zWd
   int num_sms = 148;
 
   // options

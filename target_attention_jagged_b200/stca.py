@@ -37,7 +37,8 @@ EXPORTS = ("stca_init", "stca_destroy", "stca_encode", "stca_forward", "stca_run
            "stca_get_option", "stca_kernel_times", "stca_get_encoded", "stca_plan_attention",
            "stca_forward_static", "stca_head", "stca_forward_head", "stca_sl_beta", "stca_sl_plan",
            "stca_sl_gather", "stca_encode_backward", "stca_attention_backward",
-           "stca_output_backward", "stca_query_backward", "stca_last_error")
+           "stca_output_backward", "stca_query_backward", "stca_query_init_backward",
+           "stca_fusion_backward", "stca_last_error")
 
 
 class StcaError(RuntimeError):
@@ -69,6 +70,8 @@ def _load():
     lib.stca_attention_backward.argtypes = [P, I, P, PI64, I64, P, P, P, P]
     lib.stca_output_backward.argtypes = [P, I, P, I64, P, P, P, P, P]
     lib.stca_query_backward.argtypes = [P, I, P, I64, P, P, P, P, P]
+    lib.stca_query_init_backward.argtypes = [P, P, I64, P, P, P, P, P, P, P, P]
+    lib.stca_fusion_backward.argtypes = [P, I, P, P, I64, P, I, P, P, P, P, P, P, P]
     lib.stca_run_host.argtypes = [P, P, PI64, I64, I64, P, PI64, I64, P, P]
     lib.stca_validate_offsets.argtypes = [PI64, I64, I64, I]
     lib.stca_device_status.argtypes = [P, P]
@@ -366,6 +369,50 @@ def stca_query_backward(handle: int, layer: int, Q, dU, h: int, stream=None):
     _check(_lib.stca_query_backward(handle, layer, live(Q), T, live(dU), live(dQ), dWq.data_ptr(),
                                     dWk.data_ptr(), _stream_ptr(stream)))
     return dQ, dWq, dWk
+
+
+def stca_query_init_backward(handle: int, targets, dq, rd: int, stream=None):
+    """Gradients of q^(1) = LN(SwiGLUFFN(x_t)) (Eq. (3)) from dq (T x d fp32
+    CUDA); targets: (T, d) CUDA, handle dtype.  Returns a dict of fp32 CUDA
+    tensors dxt, dWu, dWg, dWd, dgamma, dbeta."""
+    import torch
+    T, d = int(targets.shape[0]), int(targets.shape[1])
+    assert dq.dtype == torch.float32 and dq.is_contiguous() and targets.is_contiguous()
+    dev = targets.device
+    out = {"dxt": _f32_out(T, d, device=dev), "dWu": _f32_out(d, rd, device=dev),
+           "dWg": _f32_out(d, rd, device=dev), "dWd": _f32_out(rd, d, device=dev),
+           "dgamma": _f32_out(d, device=dev), "dbeta": _f32_out(d, device=dev)}
+    _check(_lib.stca_query_init_backward(handle, targets.data_ptr(), T, dq.data_ptr(), out["dxt"].data_ptr(),
+                                         out["dWu"].data_ptr(), out["dWg"].data_ptr(), out["dWd"].data_ptr(),
+                                         out["dgamma"].data_ptr(), out["dbeta"].data_ptr(), _stream_ptr(stream)))
+    return out
+
+
+def stca_fusion_backward(handle: int, block: int, Z, targets, dy, rd: int, dZ=None, dxt=None,
+                         accumulate=False, stream=None):
+    """Gradients of the block-`block` fusion (Eq. (7) for block < M, the Eq. (9)
+    head for block = M): Z (T, M, d) fp32, targets (T, d) handle dtype, dy
+    (T, d) fp32, all CUDA.  dZ (T, M, d) / dxt (T, d) are written (or added to,
+    with accumulate) in place when given, else allocated as zeros.  Returns a
+    dict dZ, dxt, dW ((block+1) d, d), dWu, dWg, dWd."""
+    import torch
+    T, M, d = int(Z.shape[0]), int(Z.shape[1]), int(Z.shape[2])
+    assert Z.dtype == torch.float32 and dy.dtype == torch.float32
+    assert Z.is_contiguous() and dy.is_contiguous() and targets.is_contiguous()
+    dev = Z.device
+    if dZ is None:
+        dZ = torch.zeros((T, M, d), dtype=torch.float32, device=dev)
+    if dxt is None:
+        dxt = torch.zeros((T, d), dtype=torch.float32, device=dev)
+    assert dZ.is_contiguous() and dxt.is_contiguous()
+    out = {"dZ": dZ, "dxt": dxt, "dW": _f32_out((block + 1) * d, d, device=dev),
+           "dWu": _f32_out(d, rd, device=dev), "dWg": _f32_out(d, rd, device=dev),
+           "dWd": _f32_out(rd, d, device=dev)}
+    live = lambda t: t.data_ptr() if T > 0 else None  # noqa: E731
+    _check(_lib.stca_fusion_backward(handle, block, live(Z), live(targets), T, live(dy), int(bool(accumulate)),
+                                     live(dZ), live(dxt), out["dW"].data_ptr(), out["dWu"].data_ptr(),
+                                     out["dWg"].data_ptr(), out["dWd"].data_ptr(), _stream_ptr(stream)))
+    return out
 
 
 def stca_forward_head(handle: int, targets, target_offsets, Z, zout, stream=None):
