@@ -106,6 +106,23 @@ def test_null_handle_calls_fail_cleanly():
     assert lib.stca_get_option(None, 1, ctypes.byref(v)) == B.STCA_EINVAL
     assert lib.stca_device_status(None, None) == B.STCA_EINVAL
     assert lib.stca_head(None, None, 4, None, None, None) == B.STCA_EINVAL
+    assert lib.stca_forward_head(None, None, off, 4, None, None, None) == B.STCA_EINVAL
+    assert lib.stca_forward_static(None, None, off, 4, None, None) == B.STCA_EINVAL
+    assert lib.stca_get_encoded(None, 0, None, None) == B.STCA_EINVAL
+    ms = (ctypes.c_double * 4)()
+    n = (ctypes.c_int64 * 4)()
+    assert lib.stca_kernel_times(None, ms, n, 4) == B.STCA_EINVAL
+    # the backward pieces
+    assert lib.stca_encode_backward(None, 0, None, 4, None, None, None, None, None, None, None,
+                                    None) == B.STCA_EINVAL
+    assert lib.stca_attention_backward(None, 0, None, off, 4, None, None, None, None) == B.STCA_EINVAL
+    assert lib.stca_output_backward(None, 0, None, 4, None, None, None, None, None) == B.STCA_EINVAL
+    assert lib.stca_query_backward(None, 0, None, 4, None, None, None, None, None) == B.STCA_EINVAL
+    assert lib.stca_query_init_backward(None, None, 4, None, None, None, None, None, None, None,
+                                        None) == B.STCA_EINVAL
+    assert lib.stca_fusion_backward(None, 1, None, None, 4, None, 0, None, None, None, None, None, None,
+                                    None) == B.STCA_EINVAL
+    assert "NULL" in S.stca_last_error()
     lib.stca_destroy(None)   # accepted
 
 
