@@ -188,6 +188,19 @@ def oracle_sample(wl, budget_s=15.0, seed=0):
                                         f"{tg} targets) of the same workload, {dt:.1f} s"}
 
 
+def oracle_one_thread(wl, budget_s=5.0, seed=1):
+    """The same oracle sample with its BLAS pinned to one thread, or None when
+    the thread count cannot be limited."""
+    try:
+        from threadpoolctl import threadpool_limits
+    except Exception:
+        return None
+    with threadpool_limits(limits=1, user_api="blas"):
+        s = oracle_sample(wl, budget_s=budget_s, seed=seed)
+    return {"value": s["value"], "unit": s["unit"], "targets_per_s": s["targets_per_s"], "cores": 1,
+            "sample": s["sample"]}
+
+
 def run_reference(args, rank):
     """The oracle as the reference arm: each step runs it on a bounded sample."""
     if rank != 0:
@@ -694,6 +707,7 @@ def run_ours(args, rank, world, local_rank):
     }
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = oracle_sample(wl, budget_s=args.cpu_budget)
+        line["cpu_baseline"]["one_thread"] = oracle_one_thread(wl, budget_s=min(5.0, args.cpu_budget))
     print(json.dumps(line), flush=True)
 
 
