@@ -1,13 +1,19 @@
 /*
- * stca.h -- C ABI of the STCA forward library (libstca.so, sm_100a).
+ * stca.h -- C ABI of the STCA library (libstca.so, sm_100a).
  *
  * Stacked Target Cross Attention over jagged user histories with
  * request-level batching.  Sources:
  *   [digest] "Make It Long, Keep It Fast: End-to-End 10k-Sequence Modeling at
- *            Billion Scale on Douyin" (paper digest), §2.1 Eqs. (1)-(8), (13);
- *            §2.2 (request-level batching); §2.3 (ragged target attention).
+ *            Billion Scale on Douyin" (paper digest), §2.1 Eqs. (1)-(9), (12),
+ *            (13); §2.2 (request-level batching); §2.3 (ragged target
+ *            attention; the sparse-training batch builder, Eqs. (15)-(17)).
  *   [blog]   "字节跳动-STCA：抖音 10k 长序列端到端建模的架构、系统与外推三件套"
- *            (STCA blog), §2.2-§2.5.
+ *            (STCA blog), §2.2-§2.6.
+ *
+ * Beyond the forward below: the Eq. (9) prediction-head token (stca_head,
+ * stca_forward_head), the naive Eq. (12) form as an option (STCA_OPT_ATTN_FORM),
+ * the sparse-training batch builder (stca_sl_*), and the backward of every
+ * piece of the step under a given output gradient (stca_*_backward).
  *
  * What the calls compute.  For request r with history X_r (L_r x d, the rows
  * offsets[r] .. offsets[r+1]-1 of X) and targets x_t (rows target_offsets[r]
