@@ -1,8 +1,9 @@
-// Backward pass of two pieces of the STCA forward ("Make It Long, Keep It Fast"
+// Backward pass of the pieces of the STCA step ("Make It Long, Keep It Fast"
 // digest §2.1; training with request-level batching, STCA blog §2.5), under a
 // loss whose gradient is given:
 //
-//  * the history encoding X~ = LN(((X W_u) * SiLU(X W_g)) W_d) (Eqs. (1)-(2)):
+//  * the history encoding X~ = LN(((X W_u) * SiLU(X W_g)) W_d) (Eqs. (1)-(2)),
+//    and with the query weights the query init q(1) of Eq. (3):
 //      dX, dW_u, dW_g, dW_d, dgamma, dbeta from dX~.  The products are plain
 //      fp32 GEMMs run by cuBLASLt (TF32 tensor cores for bf16 handles, exact
 //      fp32 otherwise); the SwiGLU and LayerNorm derivatives are two kernels here.
@@ -15,6 +16,12 @@
 //    Both run on the CUDA cores: a thread holds an eighth of a row's (or key's)
 //    d features, and eight lanes reduce the dot products by shuffles; operands
 //    are staged in shared memory with 16-byte loads.
+//  * the projections around the attention (Eqs. (6), (13)): the output side
+//    (W_V, W_O: dZ -> dC) and the query side (W_Q, W_K: dU -> dQ), plain
+//    products with the per-head slices as strided batches;
+//  * the fusion blocks of Eq. (7) and the head of Eq. (9),
+//    SwiGLUFFN([o(1) || ... || o(b) || x_t] W): d[o(1..b)], dx_t and the weights'
+//    gradients, the FFN forward recomputed.
 #include <cublasLt.h>
 #include <math.h>
 
