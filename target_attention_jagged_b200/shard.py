@@ -62,3 +62,41 @@ def max_over_ranks(value: float, device=None) -> float:
     t = torch.tensor([float(value)], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def gather_outputs(Z_local, t_rows, T_total: int):
+    """The whole batch's output, (T_total, ...) in the batch's target order, on
+    every rank, from each rank's rows Z_local of its targets t_rows.
+
+    Not part of the data path: Z normally stays with the rank that owns the
+    request.  For a caller that wants it everywhere, this is an all-gather of
+    unequal parts -- one all-gather of the row counts, then one of the rows
+    padded to the largest count and one of their target indices -- so every
+    rank takes the same three collectives in the same order.  Without a
+    process group (or with one rank) it only scatters Z_local into place."""
+    import torch
+    import torch.distributed as dist
+    dev = Z_local.device
+    inner = tuple(Z_local.shape[1:])
+    rows = torch.as_tensor(np.asarray(t_rows, dtype=np.int64), device=dev)
+    out = torch.zeros((int(T_total),) + inner, dtype=Z_local.dtype, device=dev)
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        out[rows] = Z_local
+        return out
+    world = dist.get_world_size()
+    n = torch.tensor([Z_local.shape[0]], dtype=torch.int64, device=dev)
+    counts = [torch.zeros_like(n) for _ in range(world)]
+    dist.all_gather(counts, n)
+    counts = [int(c.item()) for c in counts]
+    width = max(1, max(counts))
+    part = torch.zeros((width,) + inner, dtype=Z_local.dtype, device=dev)
+    part[:Z_local.shape[0]] = Z_local
+    idx = torch.full((width,), -1, dtype=torch.int64, device=dev)
+    idx[:rows.shape[0]] = rows
+    parts = [torch.empty_like(part) for _ in range(world)]
+    idxs = [torch.empty_like(idx) for _ in range(world)]
+    dist.all_gather(parts, part)
+    dist.all_gather(idxs, idx)
+    for p, i, c in zip(parts, idxs, counts):
+        out[i[:c]] = p[:c]
+    return out

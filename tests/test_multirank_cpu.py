@@ -13,7 +13,7 @@ import pytest
 import torch.multiprocessing as mp
 
 from gen import make_workload
-from target_attention_jagged_b200.shard import (max_over_ranks, partition_requests,
+from target_attention_jagged_b200.shard import (gather_outputs, max_over_ranks, partition_requests,
                                                 request_work, shard_offsets)
 
 WORLD = 2
@@ -43,6 +43,9 @@ def _worker(rank, world, port, out_dir):
         Z = O.forward(wl.X[x_rows], off, wl.targets[t_rows], toff, wl.weights, wl.h)
         gathered = [None] * world
         dist.all_gather_object(gathered, (mine.tolist(), t_rows.tolist(), Z))
+        # the helper a caller uses to see every target's Z on every rank
+        Z_all = gather_outputs(torch.from_numpy(Z), t_rows, wl.T).numpy()
+        np.save(os.path.join(out_dir, f"gathered{rank}.npy"), Z_all)
         slowest = max_over_ranks(10.0 * (rank + 1))
         if rank == 0:
             full = O.forward_workload(wl)
@@ -69,6 +72,16 @@ def test_sharded_batch_matches_unsharded(tmp_path):
     covered, slowest = open(tmp_path / "meta.txt").read().rsplit(" ", 1)
     assert covered == str(list(range(7)))      # every request exactly once
     assert float(slowest) == 20.0              # max over the two ranks
+    for rank in range(WORLD):                  # gather_outputs: the whole Z on every rank
+        assert np.array_equal(np.load(tmp_path / f"gathered{rank}.npy"), want)
+
+
+def test_gather_outputs_without_a_group():
+    import torch
+    Z = torch.arange(12, dtype=torch.float64).reshape(3, 4)
+    out = gather_outputs(Z, [4, 0, 2], 5)
+    assert out.shape == (5, 4)
+    assert torch.equal(out[[4, 0, 2]], Z) and torch.count_nonzero(out[[1, 3]]) == 0
 
 
 def test_partition_is_balanced_and_complete():
