@@ -100,3 +100,15 @@ def gather_outputs(Z_local, t_rows, T_total: int):
     for p, i, c in zip(parts, idxs, counts):
         out[i[:c]] = p[:c]
     return out
+
+
+def broadcast_weights(weights, src: int = 0):
+    """Rank `src`'s weight dict (numpy arrays, lists of them, None) on every
+    rank: the weights are replicated, sent once before the first stca_init.
+    Other ranks may pass None.  Identity without a process group."""
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return weights
+    box = [weights if dist.get_rank() == src else None]
+    dist.broadcast_object_list(box, src=src)
+    return box[0]

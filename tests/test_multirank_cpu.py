@@ -13,8 +13,8 @@ import pytest
 import torch.multiprocessing as mp
 
 from gen import make_workload
-from target_attention_jagged_b200.shard import (gather_outputs, max_over_ranks, partition_requests,
-                                                request_work, shard_offsets)
+from target_attention_jagged_b200.shard import (broadcast_weights, gather_outputs, max_over_ranks,
+                                                partition_requests, request_work, shard_offsets)
 
 WORLD = 2
 
@@ -37,10 +37,13 @@ def _worker(rank, world, port, out_dir):
     try:
         wl = make_workload(lengths=[40, 7, 63, 1, 25, 90, 3], targets=[2, 1, 0, 3, 1, 2, 1],
                            d=16, h=2, M=2, r=1, dtype="f32", seed=31)
+        # rank 0's weights, replicated once; the others start from nothing
+        W = broadcast_weights(wl.weights if rank == 0 else None)
+        assert all(np.array_equal(W[k][i], wl.weights[k][i]) for k in ("Wu", "Wq") for i in range(wl.M))
         work = request_work(wl.lengths, wl.target_counts, wl.d, wl.h, wl.M, wl.r)
         mine = partition_requests(work, world)[rank]
         x_rows, t_rows, off, toff = shard_offsets(wl.offsets, wl.target_offsets, mine)
-        Z = O.forward(wl.X[x_rows], off, wl.targets[t_rows], toff, wl.weights, wl.h)
+        Z = O.forward(wl.X[x_rows], off, wl.targets[t_rows], toff, W, wl.h)
         gathered = [None] * world
         dist.all_gather_object(gathered, (mine.tolist(), t_rows.tolist(), Z))
         # the helper a caller uses to see every target's Z on every rank
