@@ -294,23 +294,20 @@ def source_hash(kind):
 
 
 def recorded_traffic(kind, config_key):
-    """DRAM bytes per launch from the committed ncu summary, or None when the
-    summary is for another workload or the kernel's sources changed since.
-    The per-target class times combine + step together, so only the encoder
-    and attention classes (one kernel per timed launch) carry a figure."""
-    p = os.path.join(ROOT, "profiles", "traffic.md")
-    if kind not in ("encode", "attention") or config_key != "c3" or not os.path.exists(p):
+    """DRAM bytes per launch from the committed ncu figures (profiles/traffic.json),
+    or None when they are for another workload or the kernel's sources changed
+    since.  The per-target class times combine + step together, so only the
+    encoder and attention classes (one kernel per timed launch) carry a figure."""
+    import json
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if kind not in ("encode", "attention") or not os.path.exists(p):
         return None
     with open(p) as f:
-        for line in f:
-            cells = [x.strip() for x in line.strip().strip("|").split("|")]
-            if len(cells) == 4 and cells[0] == kind:
-                try:
-                    nbytes = int(cells[2])
-                except ValueError:
-                    return None
-                return nbytes if cells[3] == source_hash(kind) else None
-    return None
+        rec = json.load(f)
+    k = rec.get("kernels", {}).get(kind)
+    if rec.get("workload") != config_key or not k:
+        return None
+    return int(k["dram_bytes_per_launch"]) if k.get("source_sha256_16") == source_hash(kind) else None
 
 
 def roofline_of(kind, kt, c, wl, peaks, sustained, steps, config_key=None):

@@ -7,6 +7,7 @@ Compiles every .cu under csrc/ into target_attention_jagged_b200/libstca.so.
 from __future__ import annotations
 
 import argparse
+import concurrent.futures
 import glob
 import os
 import shutil
@@ -55,11 +56,18 @@ def build(debug: bool = False, verbose_ptxas: bool = False, force: bool = False)
     flags += ["-O0", "-G"] if debug else ["-O3"]
     if verbose_ptxas:
         flags += ["-Xptxas", "-v"]
-    objs = []
-    for src in sources():
+    def compile_one(src):
         obj = os.path.join(objdir, os.path.basename(src) + ".o")
         cmd = [nvcc()] + flags + ["-c", src, "-o", obj]
         r = subprocess.run(cmd, capture_output=True, text=True)
+        return src, obj, r
+
+    # the translation units are independent: compile them side by side
+    workers = max(1, min(len(sources()), os.cpu_count() or 1))
+    with concurrent.futures.ThreadPoolExecutor(max_workers=workers) as ex:
+        results = list(ex.map(compile_one, sources()))
+    objs = []
+    for src, obj, r in results:
         if r.returncode != 0 or verbose_ptxas:
             sys.stderr.write(r.stdout + r.stderr)
         if r.returncode != 0:

@@ -78,7 +78,14 @@ def gather_outputs(Z_local, t_rows, T_total: int):
     import torch.distributed as dist
     dev = Z_local.device
     inner = tuple(Z_local.shape[1:])
-    rows = torch.as_tensor(np.asarray(t_rows, dtype=np.int64), device=dev)
+    rows = torch.as_tensor(np.asarray(t_rows, dtype=np.int64).reshape(-1), device=dev)
+    # checked before any collective, so a mismatch fails on its own rank
+    # instead of scattering rows to the wrong targets
+    if rows.shape[0] != Z_local.shape[0]:
+        raise ValueError(f"gather_outputs: {rows.shape[0]} target indices for "
+                         f"{Z_local.shape[0]} rows of Z_local")
+    if rows.numel() and (int(rows.min()) < 0 or int(rows.max()) >= int(T_total)):
+        raise ValueError("gather_outputs: a target index lies outside [0, T_total)")
     out = torch.zeros((int(T_total),) + inner, dtype=Z_local.dtype, device=dev)
     if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
         out[rows] = Z_local

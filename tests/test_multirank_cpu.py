@@ -87,6 +87,15 @@ def test_gather_outputs_without_a_group():
     assert torch.equal(out[[4, 0, 2]], Z) and torch.count_nonzero(out[[1, 3]]) == 0
 
 
+def test_gather_outputs_rejects_mismatched_rows():
+    import torch
+    Z = torch.zeros((3, 4), dtype=torch.float64)
+    with pytest.raises(ValueError):
+        gather_outputs(Z, [4, 0], 5)               # two indices for three rows
+    with pytest.raises(ValueError):
+        gather_outputs(Z, [4, 0, 5], 5)            # index past T_total
+
+
 def test_partition_is_balanced_and_complete():
     rng = np.random.default_rng(0)
     L = rng.integers(100, 10000, size=256)
