@@ -436,6 +436,8 @@ def run_ours(args, rank, world, local_rank):
     st = S.Stca(storage_weights(wl), wl.d, wl.h, wl.r, wl.M, wl.dtype)
     if args.attn_form:
         st.set_option(S.STCA_OPT_ATTN_FORM, args.attn_form)
+    if args.attn_kernel is not None:
+        st.set_option(S.STCA_OPT_ATTN_KERNEL, args.attn_kernel)
     X = to_dev(wl, wl.X, dev)
     xt = to_dev(wl, wl.targets, dev)
     Z = torch.empty((wl.T, wl.M, wl.d), dtype=torch.float32, device=dev)
@@ -719,6 +721,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--attn-form", type=int, default=0, choices=[0, 1, 2],
                     help="attention form: 0 reordered (Eq. 13, default), 1 naive (Eq. 12), 2 auto")
+    ap.add_argument("--attn-kernel", type=int, default=None, choices=[0, 1],
+                    help="tensor-core attention kernel (STCA_OPT_ATTN_KERNEL): 0 two-group, "
+                         "1 split-softmax + combine; default: the library's choice")
     ap.add_argument("--no-backward", action="store_true", help="skip the backward measurement")
     ap.add_argument("--no-train-batch", action="store_true",
                     help="skip the sparse-training batch builder measurement")

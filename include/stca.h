@@ -207,9 +207,14 @@ int stca_get_encoded(stca_handle* handle, int layer, void* dst, void* stream);
  * workspace does not fit returns STCA_EINVAL with the size it needs.  All
  * calls on a device share the array: calls whose work overlaps on the GPU
  * (other streams, other handles) race, so keep them on one stream.  The first
- * call on a device looks up the array's address (cudaGetSymbolAddress); make
- * it before any stream capture.  Nothing a call reads is left over from an
- * earlier call.  stca_init and stca_encode still allocate as documented.
+ * call on a device looks up the array's address (cudaGetSymbolAddress).  A
+ * call uploads its work plan from host memory every time, so it cannot be
+ * captured into a CUDA graph: under an active capture it returns STCA_EINVAL.
+ * Nothing a call reads is left over from an earlier call.  It always runs the
+ * reordered form of Eq. (13): STCA_OPT_ATTN_FORM 1 (the naive form) is
+ * rejected with STCA_EINVAL, and 2 runs the reordered form.  The per-target
+ * step follows STCA_OPT_STEP_PATH as in stca_forward (tensor cores where the
+ * handle has them).  stca_init and stca_encode still allocate as documented.
  */
 int stca_forward_static(stca_handle* handle, const void* targets,
                         const int64_t* target_offsets, int64_t T, float* Z, void* stream);
@@ -431,6 +436,15 @@ enum {
                                  The naive form needs the tensor-core step (see above) and
                                  d_h in {16, 32, 64}; form 1 without them is rejected, form 2
                                  falls back to the reordered form */
+  STCA_OPT_ATTN_KERNEL = 7,   /* tensor-core attention of the reordered form: 0 auto (for
+                                 d <= 128 the two-group kernel, which also merges the split
+                                 partials itself); 1 the split-softmax kernel followed by the
+                                 split combine (the only kernel for d = 256) */
+  STCA_OPT_TEST_STOP_TILES = 8, /* test hook, 0 = off: the tensor-core attention's loader stops
+                                 after this many key tiles per CTA and the kernel takes the exit
+                                 of a bounded wait that ran out (copies and MMAs in flight are
+                                 let finish, TMEM is freed); the next stca_device_status then
+                                 reports STCA_EDEVICE.  The forward's output is not valid then */
   STCA_OPT_LAUNCHES = 100,    /* read-only: kernels launched since the last encode */
   STCA_OPT_LAST_FORM = 101    /* read-only: 1 if the last forward ran the naive form, else 0 */
 };
@@ -448,6 +462,18 @@ enum { STCA_K_ENCODE = 0, STCA_K_ATTN = 1, STCA_K_STEP = 2, STCA_K_HEAD = 3, STC
  * recorded events, then forgets them.
  */
 int stca_kernel_times(stca_handle* handle, double* ms, int64_t* launches, int n);
+
+/*
+ * Device self-test of the attention softmax's exponential 2^x (an addition of
+ * this library, for its own tests; the pages have no counterpart).  For n
+ * fp32 inputs x (DEVICE), writes y (DEVICE) with method 0: the MUFU
+ * ex2.approx; 1: the FMA-pipe form (range reduction to [-1/2, 1/2] and a
+ * degree-3 minimax polynomial; relative error below 1.5e-4 for x in
+ * [-126, 8], 2^-126 below -126); 2: the same two at a time with the packed
+ * fp32 instructions, as the attention evaluates it.  Asynchronous on `stream`.
+ * Errors: STCA_EINVAL, STCA_ECUDA.
+ */
+int stca_selftest_ex2(const float* x, float* y, int64_t n, int method, void* stream);
 
 /* Message of the last error on this host thread ("" if none). */
 const char* stca_last_error(void);

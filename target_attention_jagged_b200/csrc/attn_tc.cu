@@ -38,6 +38,7 @@
 #include <vector>
 
 #include "stca_internal.h"
+#include "softmax_exp.cuh"
 #include "tc_common.cuh"
 
 namespace stca {
@@ -52,6 +53,7 @@ struct AttnParams {
   float* pm;                       // G
   float* pl;                       // G
   int* status;
+  int stop_tiles;                  // > 0: the loader stops after this many key tiles (test hook)
 };
 
 // P_TMEM: P lives in TMEM (packed bf16, 64 columns per buffer) and the P X~
@@ -104,28 +106,8 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, uint6
     if (globaltimer() - t0 > ns) break;
 }
 
-__device__ __forceinline__ float ex2(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
-
-// 2^x on the FMA pipe, for x <= 8 (a score is at most 8 above the row's
-// running max): x = j + f with j = round(x) (magic-number rounding) and
-// f in [-1/2, 1/2]; 2^f by a degree-3 polynomial fitted here to a relative
-// error of 7.5e-5 (1.5e-4 with the fp32 evaluation) on that interval; j is
-// added to the exponent bits.  Below -126 the result is held at 2^-126, which
-// is zero at the precision of P (bf16).  A share of the softmax's
-// exponentials goes this way so that they do not all queue on the MUFU.
-__device__ __forceinline__ float ex2_fma(float x) {
-  x = fmaxf(x, -126.0f);
-  const float t = x + 12582912.0f;                 // 1.5 * 2^23: round(x) in the low bits
-  const float f = x - (t - 12582912.0f);
-  float p = fmaf(f, 0.05517259240150452f, 0.24261370301246643f);
-  p = fmaf(f, p, 0.6932610273361206f);
-  p = fmaf(f, p, 0.9999278783798218f);
-  return __uint_as_float(__float_as_uint(p) + (__float_as_uint(t) << 23));
-}
+using sx::ex2;
+using sx::ex2_fma;
 
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
   asm volatile(
@@ -217,6 +199,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         ++qi;
         const int nt = (item.nkeys + 127) >> 7;
         for (int j = 0; j < nt; ++j) {
+          if (p.stop_tiles > 0 && ki >= static_cast<uint32_t>(p.stop_tiles)) {
+            // test hook: give up here as a wait that ran out would
+            *abort_flag = 1;
+            atomicOr(p.status, kStatusAttnTimeout);
+            ok = false;
+            break;
+          }
           const int s = ki % KS;
           if (!(ok = bwait(&kempty[s], ((ki / KS) & 1) ^ 1, abort_flag, p.status))) break;
           mbar_arrive_expect_tx(&kfull[s], C::kStage);
@@ -232,10 +221,12 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           ++ki;
         }
       }
-      if (!ok) {
-        for (uint32_t c = ki > KS ? ki - KS : 0; c < ki; ++c) drain_wait(&kfull[c % KS], (c / KS) & 1, 100000000ull);
-        for (uint32_t c = qi > QB ? qi - QB : 0; c < qi; ++c) drain_wait(&qfull[c % QB], (c / QB) & 1, 100000000ull);
-      }
+      // Let every copy still in flight land before the CTA can exit: after a
+      // failed wait elsewhere the consumers may have stopped waiting for them.
+      // (On the normal path these phases have completed and the waits return
+      // at once.)
+      for (uint32_t c = ki > KS ? ki - KS : 0; c < ki; ++c) drain_wait(&kfull[c % KS], (c / KS) & 1, 100000000ull);
+      for (uint32_t c = qi > QB ? qi - QB : 0; c < qi; ++c) drain_wait(&qfull[c % QB], (c / QB) & 1, 100000000ull);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ S issuer
@@ -504,6 +495,7 @@ int launch_attn_tc(stca_handle* H, int layer, const AttnItem* items_d, const int
   p.pm = H->part + G * H->d;
   p.pl = p.pm + G;
   p.status = H->status_d;
+  p.stop_tiles = H->opt_stop_tiles;
   const CUtensorMap& tmK = H->tmXt[layer];
   switch (H->d) {
     case 64: return launch_cfg<64, 2, 10, 2>(H, H->tmU, tmK, p, grid, s);
@@ -525,6 +517,7 @@ int launch_attn_tc_naive(stca_handle* H, const AttnItem* items_d, const int32_t*
   p.pm = H->part + G * 64;
   p.pl = p.pm + G;
   p.status = H->status_d;
+  p.stop_tiles = H->opt_stop_tiles;
   return launch_cfg<64, 2, 5, 2, true>(H, H->tmU, H->tmKn, p, grid, s, &H->tmVn);
 }
 

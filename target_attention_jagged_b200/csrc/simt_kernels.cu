@@ -6,6 +6,9 @@
 #include <cuda_bf16.h>
 #include <math.h>
 
+#include <algorithm>
+
+#include "softmax_exp.cuh"
 #include "stca_internal.h"
 
 namespace stca {
@@ -117,77 +120,229 @@ ffn_rows_kernel(const void* __restrict__ X, int64_t nrows, const float* __restri
 }
 
 // ---------------------------------------------------------------- attention
-// One CTA per (work item, target): the target's h scaled query rows u_j
-// (Eq. (13)) against the item's key range, online softmax per head, partial
-// (max, sum, sum p * x~) written for the split combine.
-constexpr int kAttnWarps = 4;
-constexpr int kMaxPerLane = 32;   // d <= 1024
+// CUDA-core split-L single-query attention ("Make It Long, Keep It Fast"
+// digest §2.1, Eq. (13)), for batches whose query rows per request (T_r h) are
+// too few for a tensor-core tile, and for the fp32 configuration.
+//
+// One CTA takes one work item (a request's key range, at most a few thousand
+// keys) and a block of up to kRowsPerCta(NCH) of the request's query rows, so
+// the key range is read once for all of them.  The keys reach shared memory
+// as whole tiles -- a request's history rows are contiguous, so one tile is
+// one cp.async.bulk copy, completed on an mbarrier -- double-buffered so the
+// next tile lands while this one is used.  A warp's lanes form groups of GL
+// lanes (GL a power of two, at most 32); a group takes one key at a time and
+// each lane holds NCH 4-feature chunks of it (16-byte shared loads for fp32,
+// 8-byte for bf16); the dot products with the block's rows (kept in registers)
+// are reduced over the group by warp shuffles.  Each group keeps its own online
+// softmax state per row -- maximum m and sum l in log2 units, accumulator
+// chunks -- rescaled lazily (only when a score exceeds m by more than 8); the
+// groups' states are merged through shared memory at the end and written as
+// the item's partial rows (accumulator, m, l in natural-log units) for the
+// split combine.
+constexpr int kSimtWarps = 4;
+constexpr int kSimtThreads = 32 * kSimtWarps;
+constexpr int kSimtStages = 2;
 
-template <bool XBF>
-__global__ void __launch_bounds__(kAttnWarps * 32)
-attn_simt_kernel(const void* __restrict__ Xt, const float* __restrict__ U,
-                 const AttnItem* __restrict__ items, const int32_t* __restrict__ pairs,
-                 const int64_t* __restrict__ toff, float* __restrict__ pacc,
-                 float* __restrict__ pm, float* __restrict__ pl, int d, int h) {
-  extern __shared__ float sm[];
-  float* us = sm;                                  // h x d
-  float* acc = us + h * d;                         // warps x h x d
-  float* ms = acc + kAttnWarps * h * d;            // warps x h
-  float* ls = ms + kAttnWarps * h;                 // warps x h
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int w_item = pairs[2 * blockIdx.x], tl = pairs[2 * blockIdx.x + 1];
-  const AttnItem it = items[w_item];
-  const int64_t t = toff[it.req] + tl;
-  for (int e = tid; e < h * d; e += blockDim.x) us[e] = U[t * h * d + e];
-  for (int e = tid; e < kAttnWarps * h * d; e += blockDim.x) acc[e] = 0.f;
-  for (int e = tid; e < kAttnWarps * h; e += blockDim.x) { ms[e] = -INFINITY; ls[e] = 0.f; }
-  __syncthreads();
-  const int nper = (d + 31) / 32;
-  float* wacc = acc + warp * h * d;
-  float* wm = ms + warp * h;
-  float* wl = ls + warp * h;
-  for (int key = warp; key < it.nkeys; key += kAttnWarps) {
-    const int64_t row = it.key0 + key;
-    float xv[kMaxPerLane];
-#pragma unroll
-    for (int e = 0; e < kMaxPerLane; ++e)
-      xv[e] = (e < nper && lane + 32 * e < d) ? ld_elem<XBF>(Xt, row * d + lane + 32 * e) : 0.f;
-    for (int j = 0; j < h; ++j) {
-      float s = 0.f;
-#pragma unroll
-      for (int e = 0; e < kMaxPerLane; ++e)
-        if (e < nper && lane + 32 * e < d) s = fmaf(us[j * d + lane + 32 * e], xv[e], s);
-      s = warp_sum(s);
-      const float mo = wm[j];
-      const float mn = fmaxf(mo, s);
-      const float corr = expf(mo - mn);
-      const float p = expf(s - mn);
-#pragma unroll
-      for (int e = 0; e < kMaxPerLane; ++e)
-        if (e < nper && lane + 32 * e < d) {
-          float* a = wacc + j * d + lane + 32 * e;
-          *a = fmaf(*a, corr, p * xv[e]);
-        }
-      __syncwarp();
-      if (lane == 0) { wm[j] = mn; wl[j] = fmaf(wl[j], corr, p); }
-      __syncwarp();
+__host__ __device__ constexpr int simt_rows_per_cta(int nch) { return nch >= 8 ? 1 : 8 / nch; }
+
+__device__ __forceinline__ void load_chunk_f32(const uint8_t* row, int c, float (&x)[4]) {
+  const float4 v = *reinterpret_cast<const float4*>(row + 16 * c);
+  x[0] = v.x; x[1] = v.y; x[2] = v.z; x[3] = v.w;
+}
+
+__device__ __forceinline__ void load_chunk_bf16(const uint8_t* row, int c, float (&x)[4]) {
+  const uint2 v = *reinterpret_cast<const uint2*>(row + 8 * c);
+  x[0] = __uint_as_float(v.x << 16); x[1] = __uint_as_float(v.x & 0xFFFF0000u);
+  x[2] = __uint_as_float(v.y << 16); x[3] = __uint_as_float(v.y & 0xFFFF0000u);
+}
+
+__device__ __forceinline__ bool simt_wait(uint64_t* bar, uint32_t parity, int* status) {
+  uint32_t ok;
+  const long long t0 = clock64();
+  for (;;) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(ok)
+        : "r"(static_cast<uint32_t>(__cvta_generic_to_shared(bar))), "r"(parity)
+        : "memory");
+    if (ok) return true;
+    if (clock64() - t0 > (1ll << 32)) {       // about two seconds
+      atomicOr(status, kStatusAttnTimeout);
+      return false;
     }
   }
+}
+
+template <bool XBF, int NCH>
+__global__ void __launch_bounds__(kSimtThreads, 4)
+attn_simt_kernel(const void* __restrict__ Xt, const float* __restrict__ U,
+                 const AttnItem* __restrict__ items, const int32_t* __restrict__ pairs,
+                 float* __restrict__ pacc, float* __restrict__ pm, float* __restrict__ pl, int d,
+                 int GL, int kt, int us_off, int* status) {
+  constexpr int RB = simt_rows_per_cta(NCH);
+  constexpr float kLog2e = 1.4426950408889634f;
+  extern __shared__ __align__(128) uint8_t smem_simt[];
+  const int es = XBF ? 2 : 4;
+  const int rowb = d * es;                                   // bytes per key row (multiple of 16)
+  const size_t stage_bytes = static_cast<size_t>(kt) * rowb;
+  uint8_t* stages = smem_simt;                                      // later: the merge area
+  float* us = reinterpret_cast<float*>(smem_simt + us_off);                          // RB x d
+  uint64_t* full = reinterpret_cast<uint64_t*>(us + RB * d);                  // kSimtStages
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int item_i = pairs[2 * blockIdx.x], row0 = pairs[2 * blockIdx.x + 1];
+  const AttnItem it = items[item_i];
+  const int nrows = min(RB, it.rows - row0);
+  const int ntiles = (it.nkeys + kt - 1) / kt;
+  const uint8_t* src0 = static_cast<const uint8_t*>(Xt) + it.key0 * rowb;
+  if (tid == 0) {
+    for (int s = 0; s < kSimtStages; ++s)
+      asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(
+          static_cast<uint32_t>(__cvta_generic_to_shared(&full[s]))));
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
   __syncthreads();
-  // merge the warps' states and write this item's partial rows
-  for (int e = tid; e < h * d; e += blockDim.x) {
-    const int j = e / d, k = e - j * d;
-    float mx = -INFINITY;
-    for (int w = 0; w < kAttnWarps; ++w) mx = fmaxf(mx, ms[w * h + j]);
-    float a = 0.f, l = 0.f;
-    for (int w = 0; w < kAttnWarps; ++w) {
-      const float f = expf(ms[w * h + j] - mx);   // warps with no key: exp(-inf) = 0
-      a = fmaf(acc[(w * h + j) * d + k], f, a);
-      l = fmaf(ls[w * h + j], f, l);
+  auto issue = [&](int t) {           // thread 0: tile t into stage t % 2, one bulk copy
+    const int s = t % kSimtStages;
+    const int nk = min(kt, it.nkeys - t * kt);
+    const uint32_t bytes = static_cast<uint32_t>(nk) * rowb;
+    const uint32_t bar = static_cast<uint32_t>(__cvta_generic_to_shared(&full[s]));
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+                 : "memory");
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            static_cast<uint32_t>(__cvta_generic_to_shared(stages + s * stage_bytes))),
+        "l"(src0 + static_cast<int64_t>(t) * stage_bytes), "r"(bytes), "r"(bar)
+        : "memory");
+  };
+  if (tid == 0)
+    for (int t = 0; t < min(ntiles, kSimtStages); ++t) issue(t);
+  // the block's query rows, fp32, into shared memory and then registers
+  for (int e = tid; e < RB * d; e += kSimtThreads) {
+    const int r = e / d;
+    us[e] = r < nrows ? U[(it.qrow0 + row0 + r) * d + (e - r * d)] : 0.f;
+  }
+  __syncthreads();
+  const int gq = lane / GL, li = lane % GL;        // group within the warp, lane within the group
+  const int kpw = 32 / GL;                         // keys per warp step
+  const int nch = d / 4;                           // 4-feature chunks in a row
+  float ur[RB][NCH][4];
+#pragma unroll
+  for (int r = 0; r < RB; ++r)
+#pragma unroll
+    for (int i = 0; i < NCH; ++i) {
+      const int c = li + GL * i;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) ur[r][i][k] = c < nch ? us[r * d + 4 * c + k] : 0.f;
     }
-    const int64_t g = it.row_base + static_cast<int64_t>(tl) * h + j;
-    pacc[g * d + k] = a;
-    if (k == 0) { pm[g] = mx; pl[g] = l; }
+  float m[RB], l[RB], acc[RB][NCH][4];
+#pragma unroll
+  for (int r = 0; r < RB; ++r) {
+    m[r] = -INFINITY;
+    l[r] = 0.f;
+#pragma unroll
+    for (int i = 0; i < NCH; ++i)
+#pragma unroll
+      for (int k = 0; k < 4; ++k) acc[r][i][k] = 0.f;
+  }
+  bool ok = true;
+  for (int t = 0; t < ntiles; ++t) {
+    const int s = t % kSimtStages;
+    if (ok) ok = simt_wait(&full[s], (t / kSimtStages) & 1, status);
+    ok = __syncthreads_and(ok) != 0;      // one decision for the whole CTA (the loop below shuffles)
+    const int nk = min(kt, it.nkeys - t * kt);
+    const uint8_t* tile = stages + s * stage_bytes;
+    if (ok) {
+      // warp-uniform trip count: every lane of the warp takes part in the
+      // shuffles below; a group whose key lies past the tile's end computes on
+      // zeros and leaves its state unchanged
+      for (int kb = warp * kpw; kb < nk; kb += kSimtWarps * kpw) {
+        const int k = kb + gq;
+        const bool valid = k < nk;
+        const uint8_t* xrow = tile + static_cast<size_t>(valid ? k : 0) * rowb;
+        float x[NCH][4];
+#pragma unroll
+        for (int i = 0; i < NCH; ++i) {
+          const int c = li + GL * i;
+          if (valid && c < nch) {
+            if constexpr (XBF) load_chunk_bf16(xrow, c, x[i]);
+            else load_chunk_f32(xrow, c, x[i]);
+          } else {
+            x[i][0] = x[i][1] = x[i][2] = x[i][3] = 0.f;
+          }
+        }
+#pragma unroll
+        for (int r = 0; r < RB; ++r) {
+          float sc = 0.f;
+#pragma unroll
+          for (int i = 0; i < NCH; ++i)
+#pragma unroll
+            for (int q = 0; q < 4; ++q) sc = fmaf(ur[r][i][q], x[i][q], sc);
+          for (int o = GL >> 1; o > 0; o >>= 1) sc += __shfl_xor_sync(0xffffffffu, sc, o);
+          if (!valid) continue;
+          const float s2 = sc * kLog2e;              // log2 units
+          if (s2 > m[r] + 8.0f) {                    // lazy rescale (always on the first key)
+            const float corr = sx::ex2(m[r] - s2);    // 0 from m = -inf
+            l[r] *= corr;
+#pragma unroll
+            for (int i = 0; i < NCH; ++i)
+#pragma unroll
+              for (int q = 0; q < 4; ++q) acc[r][i][q] *= corr;
+            m[r] = s2;
+          }
+          const float p = sx::ex2(s2 - m[r]);
+          l[r] += p;
+#pragma unroll
+          for (int i = 0; i < NCH; ++i)
+#pragma unroll
+            for (int q = 0; q < 4; ++q) acc[r][i][q] = fmaf(p, x[i][q], acc[r][i][q]);
+        }
+      }
+    }
+    __syncthreads();                      // every warp is done with stage s
+    if (tid == 0 && ok && t + kSimtStages < ntiles) issue(t + kSimtStages);
+  }
+  // let copies still in flight (after a failed wait) land before the stages are reused
+  // (on the normal path these phases are complete and the waits return at once)
+  if (tid == 0)
+    for (int t = max(0, ntiles - kSimtStages); t < ntiles; ++t)
+      simt_wait(&full[t % kSimtStages], (t / kSimtStages) & 1, status);
+  __syncthreads();
+  // merge the groups' states: state g = (warp, group) -> [RB rows][d + 2] floats
+  const int ngroups = kSimtWarps * kpw;
+  float* st = reinterpret_cast<float*>(smem_simt);            // the stages are free now
+  const int g = warp * kpw + gq;
+#pragma unroll
+  for (int r = 0; r < RB; ++r) {
+    float* row = st + (static_cast<size_t>(g) * RB + r) * (d + 2);
+#pragma unroll
+    for (int i = 0; i < NCH; ++i) {
+      const int c = li + GL * i;
+      if (c < nch)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) row[4 * c + q] = acc[r][i][q];
+    }
+    if (li == 0) { row[d] = m[r]; row[d + 1] = l[r]; }
+  }
+  __syncthreads();
+  for (int e = tid; e < nrows * d; e += kSimtThreads) {
+    const int r = e / d, f = e - r * d;
+    float mx = -INFINITY;
+    for (int q = 0; q < ngroups; ++q) mx = fmaxf(mx, st[(static_cast<size_t>(q) * RB + r) * (d + 2) + d]);
+    float a = 0.f, lsum = 0.f;
+    for (int q = 0; q < ngroups; ++q) {
+      const float* row = st + (static_cast<size_t>(q) * RB + r) * (d + 2);
+      const float w = row[d + 1] > 0.f ? sx::ex2(row[d] - mx) : 0.f;   // a group with no key: 0
+      a = fmaf(w, row[f], a);
+      lsum = fmaf(w, row[d + 1], lsum);
+    }
+    const int64_t gr = it.row_base + row0 + r;
+    pacc[gr * d + f] = a;
+    if (f == 0) {
+      pm[gr] = mx * 0.6931471805599453f;              // natural-log units for the combine
+      pl[gr] = lsum;
+    }
   }
 }
 
@@ -220,32 +375,65 @@ void launch_ffn_rows(const void* X, int x_is_bf16, int64_t nrows, const LayerW32
 #undef STCA_FFN
 }
 
-size_t attn_simt_smem(const stca_handle* H) {
-  return (static_cast<size_t>(H->h) * H->d * (1 + kAttnWarps) + 2 * kAttnWarps * H->h) *
-         sizeof(float);
+namespace {
+// Launch geometry of the CUDA-core attention for width d: NCH chunks of 4
+// features per lane, GL lanes per key (a power of two), kt keys per tile.
+struct SimtGeom {
+  int nch, gl, kt, rb;
+  size_t us_off, smem;
+};
+
+SimtGeom simt_geom(int d, int elem) {
+  SimtGeom g{};
+  const int chunks = d / 4;
+  g.nch = 1;
+  while (g.nch * 32 < chunks) g.nch *= 2;                  // 1, 2, 4, 8 (d <= 1024)
+  g.gl = 1;
+  while (g.gl * g.nch < chunks && g.gl < 32) g.gl *= 2;
+  g.rb = simt_rows_per_cta(g.nch);
+  const int rowb = d * elem;
+  g.kt = std::max(8, std::min(256, (24 << 10) / rowb) / 8 * 8);   // up to 24 KB per stage
+  const size_t stages = static_cast<size_t>(kSimtStages) * g.kt * rowb;
+  const size_t merge = static_cast<size_t>(kSimtWarps) * (32 / g.gl) * g.rb * (d + 2) * sizeof(float);
+  // the stages, reused as the merge area at the end; then the query rows and
+  // the mbarriers
+  g.us_off = (std::max(stages, merge) + 15) / 16 * 16;
+  g.smem = g.us_off + static_cast<size_t>(g.rb) * d * sizeof(float) + 64;
+  return g;
 }
+}  // namespace
+
+int attn_simt_rows_per_cta(int d) { return simt_geom(d, 4).rb; }
+
+size_t attn_simt_smem(const stca_handle* H) { return simt_geom(H->d, H->elem).smem; }
 
 void launch_attn_simt(const stca_handle* H, int layer, const void* xt_layer,
                       const AttnItem* items_d, const int32_t* pairs_d, int64_t npairs,
                       const int64_t* toff_d, cudaStream_t s) {
   (void)layer;
+  (void)toff_d;
   if (npairs <= 0) return;
-  const size_t smem = attn_simt_smem(H);
+  const SimtGeom g = simt_geom(H->d, H->elem);
   const int64_t G = H->last_G;
   float* pacc = H->part;
   float* pm = pacc + G * H->d;
   float* pl = pm + G;
-  if (H->elem == 2) {
-    cudaFuncSetAttribute(attn_simt_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         (int)smem);
-    attn_simt_kernel<true><<<static_cast<unsigned>(npairs), kAttnWarps * 32, smem, s>>>(
-        xt_layer, H->U, items_d, pairs_d, toff_d, pacc, pm, pl, H->d, H->h);
-  } else {
-    cudaFuncSetAttribute(attn_simt_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         (int)smem);
-    attn_simt_kernel<false><<<static_cast<unsigned>(npairs), kAttnWarps * 32, smem, s>>>(
-        xt_layer, H->U, items_d, pairs_d, toff_d, pacc, pm, pl, H->d, H->h);
+#define STCA_SIMT(XB, NC)                                                                          \
+  do {                                                                                             \
+    auto k = attn_simt_kernel<XB, NC>;                                                             \
+    cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)g.smem);             \
+    k<<<static_cast<unsigned>(npairs), kSimtThreads, g.smem, s>>>(xt_layer, H->U, items_d, pairs_d, \
+                                                                  pacc, pm, pl, H->d, g.gl, g.kt,  \
+                                                                  (int)g.us_off, H->status_d);     \
+  } while (0)
+  const bool bf = H->elem == 2;
+  switch (g.nch) {
+    case 1: if (bf) STCA_SIMT(true, 1); else STCA_SIMT(false, 1); break;
+    case 2: if (bf) STCA_SIMT(true, 2); else STCA_SIMT(false, 2); break;
+    case 4: if (bf) STCA_SIMT(true, 4); else STCA_SIMT(false, 4); break;
+    default: if (bf) STCA_SIMT(true, 8); else STCA_SIMT(false, 8); break;
   }
+#undef STCA_SIMT
 }
 
 }  // namespace stca

@@ -185,6 +185,7 @@ extern "C" void stca_destroy(stca_handle* H) {
   cudaFree(H->Ubf);
   cudaFree(H->part);
   cudaFree(H->cbuf);
+  cudaFree(H->attn_cnt);
   cudaFree(H->plan_d);
   cudaFree(H->status_d);
   cudaFree(H->x_stage);
@@ -392,25 +393,33 @@ extern "C" int stca_init(const stca_weights* w, int d, int h, int r, int M, int 
         stca_destroy(H);
         return rc2;
       }
-      if (naive_layout(dh).G > 0) {
-        // naive form (Eq. (12)): [W_K | W_V] of every layer, d x 2d bf16
-        std::vector<uint16_t> kvw(static_cast<size_t>(M) * d * 2 * d);
+      if (naive_layout(dh).G > 0 && kv_proj_supported(d)) {
+        // naive form (Eq. (12)): [W_K | W_V] of every layer, stored transposed
+        // (2d outputs x d inputs, K-major) as the B operand of the projection
+        std::vector<uint16_t> kvw(static_cast<size_t>(M) * 2 * d * d);
         auto bf = [](float f) {
           uint32_t u;
           memcpy(&u, &f, 4);
           return static_cast<uint16_t>(u >> 16);     // bf16-valued already
         };
         for (int i = 0; i < M; ++i)
-          for (int k = 0; k < d; ++k)
-            for (int m = 0; m < 2 * d; ++m)
-              kvw[(static_cast<size_t>(i) * d + k) * 2 * d + m] =
-                  bf(m < d ? sw[i].Wk[static_cast<size_t>(k) * d + m] : sw[i].Wv[static_cast<size_t>(k) * d + m - d]);
+          for (int o = 0; o < 2 * d; ++o)
+            for (int k = 0; k < d; ++k)
+              kvw[(static_cast<size_t>(i) * 2 * d + o) * d + k] =
+                  bf(o < d ? sw[i].Wk[static_cast<size_t>(k) * d + o] : sw[i].Wv[static_cast<size_t>(k) * d + o - d]);
         if (cudaMalloc(&H->wkv, kvw.size() * 2) != cudaSuccess ||
             cudaMemcpy(H->wkv, kvw.data(), kvw.size() * 2, cudaMemcpyHostToDevice) != cudaSuccess) {
           cudaGetLastError();
           stca_destroy(H);
           return set_error(STCA_ENOMEM, "naive-form weight upload failed");
         }
+        for (int i = 0; i < M; ++i)
+          if (int rc2 = make_tmap_bf16_2d(&H->tmWkv[i],
+                                          static_cast<const uint16_t*>(H->wkv) + static_cast<size_t>(i) * 2 * d * d,
+                                          d, 2 * d, 64, 256)) {
+            stca_destroy(H);
+            return rc2;
+          }
       }
     }
   }
@@ -543,7 +552,7 @@ NaiveLayout stca::naive_layout(int dh) {
 }
 
 void stca::build_plan_host(const int64_t* off, const int64_t* toff, int64_t R, int h, int path,
-                            int num_ctas, int64_t split_keys, PlanHost& P, int dh) {
+                            int num_ctas, int64_t split_keys, PlanHost& P, int dh, int simt_rows) {
   P = PlanHost();
   P.req_pair_begin.assign(R + 1, 0);
   auto& items = P.items;
@@ -571,10 +580,11 @@ void stca::build_plan_host(const int64_t* off, const int64_t* toff, int64_t R, i
         it.qrow0 = toff[r] * h;
         it.mt = 0;
         it.rows = static_cast<int32_t>(Tr * h);
+        it.pair = static_cast<int32_t>(r);
         G += Tr * h;
-        for (int64_t tl = 0; tl < Tr; ++tl) {
+        for (int64_t row0 = 0; row0 < Tr * h; row0 += std::max(simt_rows, 1)) {
           P.pairs_simt.push_back(static_cast<int32_t>(items.size()));
-          P.pairs_simt.push_back(static_cast<int32_t>(tl));
+          P.pairs_simt.push_back(static_cast<int32_t>(row0));
         }
         items.push_back(it);
       }
@@ -614,7 +624,8 @@ void stca::build_plan_host(const int64_t* off, const int64_t* toff, int64_t R, i
   P.cta_begin.assign(P.grid + 1, 0);
   int64_t cursor = 0;     // global key-tile index of the pair's first tile
   int next_cta = 0;
-  for (const Pair& pr : pairs) {
+  for (size_t pi = 0; pi < pairs.size(); ++pi) {
+    const Pair& pr = pairs[pi];
     P.pair_item_begin.push_back(static_cast<int32_t>(items.size()));
     const int64_t L = off[pr.r + 1] - off[pr.r];
     const int64_t rows = path == 3 ? 128
@@ -631,6 +642,7 @@ void stca::build_plan_host(const int64_t* off, const int64_t* toff, int64_t R, i
       it.row_base = G;
       it.mt = static_cast<int32_t>(pr.mt);
       it.rows = static_cast<int32_t>(rows);
+      it.pair = static_cast<int32_t>(pi);
       if (path == 3) {
         const int64_t nslots = (toff[pr.r + 1] - toff[pr.r] + NL.Tq - 1) / NL.Tq;
         it.qrow0 = P.qbase[pr.r] + pr.mt * 128;
@@ -685,6 +697,10 @@ int stca::check_plan(const PlanHost& P, const int64_t* off, const int64_t* toff,
   for (int64_t p = 0; p < npairs; ++p)
     if (P.pair_item_begin[p] > P.pair_item_begin[p + 1]) return bad("pair items");
   if (P.pair_item_begin[npairs] != static_cast<int32_t>(P.items.size())) return bad("pair end");
+  if (path >= 2)
+    for (int64_t p = 0; p < npairs; ++p)
+      for (int32_t w = P.pair_item_begin[p]; w < P.pair_item_begin[p + 1]; ++w)
+        if (P.items[w].pair != p) return bad("item's pair index");
   for (int64_t r = 0; r < R; ++r) {
     const int64_t rows = (toff[r + 1] - toff[r]) * h;
     const int64_t want = path == 2 ? (rows + 127) / 128 : path == 3 ? (P.qbase[r + 1] - P.qbase[r]) / 128 : 1;
@@ -707,10 +723,9 @@ int stca::check_plan(const PlanHost& P, const int64_t* off, const int64_t* toff,
       if (P.cta_begin[c] > P.cta_begin[c + 1]) return bad("CTA ranges order");
   } else {
     for (size_t q = 0; q < P.pairs_simt.size(); q += 2) {
-      const int32_t w = P.pairs_simt[q], tl = P.pairs_simt[q + 1];
-      if (w < 0 || w >= static_cast<int32_t>(P.items.size()) || tl < 0 ||
-          tl >= toff[P.items[w].req + 1] - toff[P.items[w].req])
-        return bad("(item, target) pair");
+      const int32_t w = P.pairs_simt[q], row0 = P.pairs_simt[q + 1];
+      if (w < 0 || w >= static_cast<int32_t>(P.items.size()) || row0 < 0 || row0 >= P.items[w].rows)
+        return bad("(item, query row block) pair");
     }
   }
   (void)N;
@@ -726,7 +741,8 @@ static int build_plan(stca_handle* H, const int64_t* toff, int64_t T, int path, 
     return STCA_OK;   // same layout as the previous forward on this encode: plan is on device
   const int64_t* off = H->offsets_h.data();
   PlanHost P;
-  build_plan_host(off, toff, R, H->h, path, H->num_sms, H->opt_split_keys, P, H->dh);
+  build_plan_host(off, toff, R, H->h, path, H->num_sms, H->opt_split_keys, P, H->dh,
+                  attn_simt_rows_per_cta(H->d));
   if (int rc = check_plan(P, off, toff, R, H->h, path)) return rc;
   const auto& items = P.items;
   const auto& pairs_simt = P.pairs_simt;
@@ -775,6 +791,7 @@ static int build_plan(stca_handle* H, const int64_t* toff, int64_t T, int path, 
   STCA_CUDA_TRY(cudaMemcpyAsync(H->plan_d, H->plan_h, bytes, cudaMemcpyHostToDevice, s));
   STCA_CUDA_TRY(cudaEventRecord(H->plan_evt, s));
   H->last_G = G;
+  H->last_npairs = static_cast<int64_t>(pair_item_begin.size()) - 1;
   H->last_pairs = static_cast<int64_t>(pairs_simt.size() / 2);
   H->last_max_items = 0;
   for (size_t k = 0; k + 1 < pair_item_begin.size(); ++k)
@@ -786,54 +803,11 @@ static int build_plan(stca_handle* H, const int64_t* toff, int64_t T, int path, 
 }
 
 // Naive form, Eq. (12): K = X~(layer+1) W_K and V = X~(layer+1) W_V for every
-// history row at once, into H->kv (row n: [K_n | V_n], bf16).  A plain GEMM,
-// [N x d] x [d x 2d], run by cuBLASLt (bf16 operands, fp32 accumulation).
+// history row at once, into H->kv (row n: [K_n | V_n], bf16), by the
+// tensor-core projection kernel (kv_proj.cu).
 static int kv_project(stca_handle* H, int layer, cudaStream_t s) {
-  const int d = H->d;
-  const int64_t N = H->N;
-  if (!H->lt) {
-    cublasLtHandle_t lt = nullptr;
-    if (cublasLtCreate(&lt) != CUBLAS_STATUS_SUCCESS) return set_error(STCA_ECUDA, "cublasLtCreate failed");
-    H->lt = lt;
-  }
-  constexpr size_t kWs = size_t(32) << 20;
-  if (int rc = ensure_dev(&H->lt_ws, &H->lt_ws_cap, kWs)) return rc;
-  cublasLtHandle_t lt = static_cast<cublasLtHandle_t>(H->lt);
-  cublasLtMatmulDesc_t op = nullptr;
-  cublasLtMatrixLayout_t la = nullptr, lb = nullptr, lc = nullptr;
-  cublasLtMatmulPreference_t pref = nullptr;
-  int rc = STCA_OK;
-  // column-major view: KV^T (2d x N) = W^T (2d x d) * X~^T (d x N)
-  if (cublasLtMatmulDescCreate(&op, CUBLAS_COMPUTE_32F, CUDA_R_32F) != CUBLAS_STATUS_SUCCESS ||
-      cublasLtMatrixLayoutCreate(&la, CUDA_R_16BF, 2 * d, d, 2 * d) != CUBLAS_STATUS_SUCCESS ||
-      cublasLtMatrixLayoutCreate(&lb, CUDA_R_16BF, d, N, d) != CUBLAS_STATUS_SUCCESS ||
-      cublasLtMatrixLayoutCreate(&lc, CUDA_R_16BF, 2 * d, N, 2 * d) != CUBLAS_STATUS_SUCCESS ||
-      cublasLtMatmulPreferenceCreate(&pref) != CUBLAS_STATUS_SUCCESS) {
-    rc = set_error(STCA_ECUDA, "cuBLASLt descriptor set-up failed");
-  }
-  cublasLtMatmulHeuristicResult_t heur{};
-  int found = 0;
-  if (rc == STCA_OK) {
-    size_t ws = kWs;
-    cublasLtMatmulPreferenceSetAttribute(pref, CUBLASLT_MATMUL_PREF_MAX_WORKSPACE_BYTES, &ws, sizeof(ws));
-    if (cublasLtMatmulAlgoGetHeuristic(lt, op, la, lb, lc, lc, pref, 1, &heur, &found) !=
-            CUBLAS_STATUS_SUCCESS || found < 1)
-      rc = set_error(STCA_ECUDA, "cuBLASLt found no algorithm for the K/V projection");
-  }
-  if (rc == STCA_OK) {
-    const float alpha = 1.f, beta = 0.f;
-    const uint16_t* w = static_cast<const uint16_t*>(H->wkv) + static_cast<size_t>(layer) * d * 2 * d;
-    const void* x = static_cast<const char*>(H->xt) + static_cast<size_t>(N) * d * 2 * layer;
-    if (cublasLtMatmul(lt, op, &alpha, w, la, x, lb, &beta, H->kv, lc, H->kv, lc, &heur.algo, H->lt_ws,
-                       kWs, s) != CUBLAS_STATUS_SUCCESS)
-      rc = set_error(STCA_ECUDA, "cuBLASLt K/V projection failed");
-  }
-  if (pref) cublasLtMatmulPreferenceDestroy(pref);
-  if (lc) cublasLtMatrixLayoutDestroy(lc);
-  if (lb) cublasLtMatrixLayoutDestroy(lb);
-  if (la) cublasLtMatrixLayoutDestroy(la);
-  if (op) cublasLtMatmulDescDestroy(op);
-  return rc;
+  return launch_kv_proj(H->d, H->tmXt[layer], H->tmWkv[layer], static_cast<uint16_t*>(H->kv), H->N,
+                        H->num_sms, H->status_d, s);
 }
 
 // FLOPs of one layer's attention in either form: the reordered form contracts
@@ -906,10 +880,20 @@ static int forward_impl(stca_handle* H, const void* targets, const int64_t* targ
     if (int rc = ensure_dev(reinterpret_cast<void**>(&H->Ubf), &H->Ubf_cap, urows * d * 2)) return rc;
     if (int rc = make_tmap_bf16_2d(&H->tmU, H->Ubf, d, urows, 64, 128)) return rc;
   }
+  // the two-group kernel (d <= 128, reordered form) merges the split
+  // partials itself, counting arrivals per pair and layer
+  const bool pp = path == 2 && !naive && attn_pp_supported(d) && H->opt_attn_kernel != 1;
   if (int rc = ensure_dev(reinterpret_cast<void**>(&H->part), &H->part_cap,
-                          static_cast<size_t>(std::max<int64_t>(H->last_G, 1)) * ((naive ? 64 : d) + 2) *
+                          static_cast<size_t>(std::max<int64_t>(H->last_G, 1)) * ((naive ? 64 : d) + 4) *
                               sizeof(float)))
     return rc;
+  const size_t cnt_per_layer = static_cast<size_t>(std::max<int64_t>(H->last_npairs, 1)) * 8;
+  if (pp) {
+    if (int rc = ensure_dev(reinterpret_cast<void**>(&H->attn_cnt), &H->attn_cnt_cap,
+                            cnt_per_layer * H->M * sizeof(int)))
+      return rc;
+    STCA_CUDA_TRY(cudaMemsetAsync(H->attn_cnt, 0, cnt_per_layer * H->M * sizeof(int), s));
+  }
   if (int rc = ensure_dev(reinterpret_cast<void**>(&H->cbuf), &H->cbuf_cap, urows * d * sizeof(float)))
     return rc;
   char* p = static_cast<char*>(H->plan_d);
@@ -932,7 +916,7 @@ static int forward_impl(stca_handle* H, const void* targets, const int64_t* targ
   const bool step_tc = path == 2 && H->step_tc_ready && H->opt_step_path != 1;
   // the tensor-core step merges the split partials itself when every query
   // tile has few enough items; otherwise combine_kernel merges them first
-  const bool fused = !naive && step_tc && H->last_max_items <= step_tc_max_items() &&
+  const bool fused = !naive && !pp && step_tc && H->last_max_items <= step_tc_max_items() &&
                      H->last_G < (int64_t(1) << 31);
   NaiveStep ns{NL.G, NL.Tq, reinterpret_cast<const int64_t*>(p + H->off_qbase), H->Ubf};
   const bool head_in_step = zout && step_tc && H->head_tc;
@@ -958,6 +942,10 @@ static int forward_impl(stca_handle* H, const void* targets, const int64_t* targ
         rc = kv_project(H, i, s);
         if (!rc) rc = launch_attn_tc_naive(H, items_d, cta_d, H->last_grid, s);
         H->launches++;
+      } else if (pp) {
+        rc = launch_attn_pp(d, H->tmU, H->tmXt[i], items_d, cta_d, plan.pair_item_begin,
+                            H->last_grid, H->part, H->last_G, H->cbuf,
+                            H->attn_cnt + cnt_per_layer * i, H->status_d, H->opt_stop_tiles, s);
       } else if (path == 2) {
         rc = launch_attn_tc(H, i, items_d, cta_d, H->last_grid, s);
       } else {
@@ -973,7 +961,7 @@ static int forward_impl(stca_handle* H, const void* targets, const int64_t* targ
       if (naive) {
         launch_combine_naive(H, plan, H->part, H->last_G, T, H->cbuf, s);
         H->launches++;
-      } else if (!fused) {
+      } else if (!fused && !pp) {
         launch_combine(H, plan, H->part, H->last_G, T, H->cbuf, s);
         H->launches++;
       }
@@ -1121,6 +1109,7 @@ extern "C" int stca_device_status(stca_handle* H, void* stream) {
     if (st & kStatusEncodeTimeout) m += " encoder gave up a bounded wait;";
     if (st & kStatusAttnTimeout) m += " attention gave up a bounded wait;";
     if (st & kStatusStepTimeout) m += " per-target step gave up a bounded wait;";
+    if (st & kStatusKvTimeout) m += " K/V projection gave up a bounded wait;";
     return set_error(STCA_EDEVICE, m);
   }
   return ok();
@@ -1149,6 +1138,14 @@ extern "C" int stca_set_option(stca_handle* H, int option, int64_t value) {
       if (value < 0 || value > 2) return set_error(STCA_EINVAL, "attention form must be 0, 1 or 2");
       H->opt_attn_form = static_cast<int>(value);
       return ok();
+    case STCA_OPT_ATTN_KERNEL:
+      if (value < 0 || value > 1) return set_error(STCA_EINVAL, "attention kernel must be 0 or 1");
+      H->opt_attn_kernel = static_cast<int>(value);
+      return ok();
+    case STCA_OPT_TEST_STOP_TILES:
+      if (value < 0 || value > (int64_t(1) << 30)) return set_error(STCA_EINVAL, "stop tiles must be >= 0");
+      H->opt_stop_tiles = static_cast<int>(value);
+      return ok();
     case STCA_OPT_SPLIT_KEYS:
       if (value < 0 || value % 128 || value > (int64_t(1) << 30))
         return set_error(STCA_EINVAL, "split must be 0 or a positive multiple of 128");
@@ -1169,6 +1166,8 @@ extern "C" int stca_get_option(stca_handle* H, int option, int64_t* value) {
     case STCA_OPT_TIMING: *value = H->timing ? 1 : 0; return ok();
     case STCA_OPT_LAUNCHES: *value = H->launches; return ok();
     case STCA_OPT_ATTN_FORM: *value = H->opt_attn_form; return ok();
+    case STCA_OPT_ATTN_KERNEL: *value = H->opt_attn_kernel; return ok();
+    case STCA_OPT_TEST_STOP_TILES: *value = H->opt_stop_tiles; return ok();
     case STCA_OPT_LAST_FORM: *value = H->last_naive ? 1 : 0; return ok();
     default: return set_error(STCA_EINVAL, "unknown option " + std::to_string(option));
   }

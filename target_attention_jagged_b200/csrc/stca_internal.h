@@ -23,7 +23,7 @@ int set_error(int code, const std::string& msg);
   } while (0)
 
 // Device status word bits written by kernels that give up a bounded wait.
-enum : int { kStatusEncodeTimeout = 1, kStatusAttnTimeout = 2, kStatusStepTimeout = 4 };
+enum : int { kStatusEncodeTimeout = 1, kStatusAttnTimeout = 2, kStatusStepTimeout = 4, kStatusKvTimeout = 8 };
 
 // ---------------------------------------------------------------- work plan
 // One attention work item: a contiguous key range of one request's history
@@ -38,7 +38,7 @@ struct AttnItem {
   int32_t mt;         // query tile index within the request
   int32_t rows;       // query rows of this tile that belong to the request
   int32_t kcol;       // naive form: first feature of the tile's head group in K and V
-  int32_t pad_;
+  int32_t pair;       // (request, query tile) pair of the item (tensor-core path)
 };
 
 // Query layout of the naive-form attention (Eq. (12) with K = X~ W_K and
@@ -110,7 +110,8 @@ struct stca_handle {
   int opt_attn_form = 0;                // 0 reordered (Eq. (13)), 1 naive (Eq. (12)), 2 auto
   bool last_naive = false;              // the last forward ran the naive form
   void* kv = nullptr;       size_t kv_cap = 0;     // naive form: N x 2d bf16, [K | V] per row
-  void* wkv = nullptr;                  // naive form: per layer [W_K | W_V], d x 2d bf16
+  void* wkv = nullptr;                  // naive form: per layer [W_K | W_V]^T, 2d x d bf16 (K-major)
+  CUtensorMap tmWkv[16];                // their TMA descriptors (box 64 inputs x 256 outputs)
   void* lt = nullptr;                   // cuBLASLt handle (naive-form projection)
   void* lt_ws = nullptr;    size_t lt_ws_cap = 0;  // its workspace
   void* bw_ws = nullptr;    size_t bw_ws_cap = 0;  // encoder backward workspace (fp32)
@@ -130,6 +131,8 @@ struct stca_handle {
   // options
   int opt_attn_path = 0, opt_encode_path = 0, opt_step_path = 0;
   int64_t opt_split_keys = 0;
+  int opt_attn_kernel = 0;              // 0 auto (two-group kernel for d <= 128), 1 split-softmax kernel
+  int opt_stop_tiles = 0;               // test hook: the attention loader stops after this many tiles
   int64_t launches = 0;
   bool timing = false;
   struct TimedRec { int cls; cudaEvent_t a, b; };
@@ -149,6 +152,7 @@ struct stca_handle {
   uint16_t* Ubf = nullptr;  size_t Ubf_cap = 0;    // bf16 copy for tensor cores
   float* part = nullptr;    size_t part_cap = 0;   // G x (d + 2)
   float* cbuf = nullptr;    size_t cbuf_cap = 0;   // T x h x d: merged alpha X~ rows
+  int* attn_cnt = nullptr;  size_t attn_cnt_cap = 0;  // M x pairs x 8 arrival counters
   void* plan_d = nullptr;   size_t plan_cap = 0;   // uploaded plan arrays
   void* plan_h = nullptr;   size_t plan_h_cap = 0; // pinned staging
   cudaEvent_t plan_evt = nullptr;
@@ -163,6 +167,7 @@ struct stca_handle {
   std::vector<int64_t> last_toff;
   int last_path = 0;                    // 1 CUDA cores, 2 tensor cores
   int64_t last_G = 0, last_pairs = 0;
+  int64_t last_npairs = 0;              // (request, query tile) pairs of the plan
   int last_max_items = 0;               // most items of one (request, query tile) pair
   int last_grid = 0;                    // CTAs of the tensor-core attention
   size_t off_items = 0, off_pairs = 0, off_cta = 0, off_treq = 0, off_toff = 0, off_rpb = 0,
@@ -205,6 +210,9 @@ int head_weights_setup(stca_handle* H, const float* Wz, const float* zWu, const 
 void launch_head(const stca_handle* H, const void* targets, int64_t T, const float* Z, float* zout,
                  cudaStream_t s);
 size_t attn_simt_smem(const stca_handle* H);
+// Query rows per CTA of the CUDA-core attention for width d (its grid is
+// (work item, first row) pairs, one per block of this many rows).
+int attn_simt_rows_per_cta(int d);
 
 // Tensor-core per-target step (step_tc.cu)
 bool step_tc_supported(const stca_handle* H);
@@ -233,7 +241,7 @@ int launch_step_tc(const stca_handle* H, int layer, const void* targets, int64_t
 // Host-side attention work plan (stca_api.cu).
 struct PlanHost {
   std::vector<AttnItem> items;
-  std::vector<int32_t> pairs_simt;       // (item, target) pairs, CUDA-core grid
+  std::vector<int32_t> pairs_simt;       // (item, first query row) pairs, CUDA-core grid
   std::vector<int32_t> cta_begin;        // tensor-core grid + 1
   std::vector<int32_t> req_pair_begin;   // R + 1
   std::vector<int32_t> pair_item_begin;  // pairs + 1
@@ -243,7 +251,7 @@ struct PlanHost {
   int grid = 0;                          // tensor-core CTAs
 };
 void build_plan_host(const int64_t* off, const int64_t* toff, int64_t R, int h, int path,
-                     int num_ctas, int64_t split_keys, PlanHost& P, int dh = 0);
+                     int num_ctas, int64_t split_keys, PlanHost& P, int dh = 0, int simt_rows = 1);
 NaiveLayout naive_layout(int dh);
 int check_plan(const PlanHost& P, const int64_t* off, const int64_t* toff, int64_t R, int h,
                int path);
@@ -252,6 +260,22 @@ void launch_target_step_ws(const stca_handle* H, int layer, const void* targets,
 int launch_attn_tc_ws(int d, const CUtensorMap& tmQ, const CUtensorMap& tmK,
                       const AttnItem* items_d, const int32_t* cta_begin_d, int grid, float* part,
                       int64_t G, int* status, cudaStream_t s);
+
+// Two-group tensor-core attention with the split combine inside (attn_pp.cu):
+// writes the merged rows c (T h x d fp32) to `cout`; part holds G x d partial
+// rows then G x 4 (m, l) values; counters (pairs x 8 ints) must be zero.
+bool attn_pp_supported(int d);
+int launch_attn_pp(int d, const CUtensorMap& tmQ, const CUtensorMap& tmK, const AttnItem* items_d,
+                   const int32_t* cta_begin_d, const int32_t* pair_item_begin_d, int grid,
+                   float* part, int64_t G, float* cout, int* counters, int* status, int stop_tiles,
+                   cudaStream_t s);
+
+// Naive form's K/V projection on the tensor cores (kv_proj.cu): out (N x 2d
+// bf16) = X~ (tmX: N x d, box 64 x 128) times [W_K | W_V] (tmW: its transpose,
+// 2d x d, box 64 x 256).
+bool kv_proj_supported(int d);
+int launch_kv_proj(int d, const CUtensorMap& tmX, const CUtensorMap& tmW, uint16_t* out, int64_t N,
+                   int num_sms, int* status, cudaStream_t s);
 
 // Tensor-core attention (attn_tc.cu)
 bool attn_tc_supported(int d);

@@ -13,7 +13,10 @@
 //
 // Set-up: the first call on each device looks up the array's device address
 // with cudaGetSymbolAddress (with that device current), which also loads the
-// module that holds the array; make that first call before any stream capture.
+// module that holds the array.  No call can be captured into a CUDA graph: the
+// work plan is uploaded from host memory each time, so a call under an active
+// capture is refused.  The attention runs in the reordered form of Eq. (13);
+// the per-target step runs where stca_forward would run it.
 //
 // The array is file-scope device memory of kStaticScratchBytes (32 MiB).
 // Every GPU that loads the library holds it until the process exits, and
@@ -103,6 +106,23 @@ extern "C" int stca_forward_static(stca_handle* H, const void* targets,
   if (H->dtype != STCA_BF16 || !attn_tc_supported(H->d) || H->opt_attn_path == 1)
     return set_error(STCA_EINVAL,
                      "stca_forward_static runs the tensor-core path only: bf16 and d in {64, 128, 256}");
+  if (H->opt_attn_form == 1)
+    return set_error(STCA_EINVAL, "stca_forward_static runs the reordered form (Eq. (13)) only; "
+                                  "STCA_OPT_ATTN_FORM 1 (the naive form) is not available here");
+  if (H->opt_step_path == 2 && !H->step_tc_ready)
+    return set_error(STCA_EINVAL, "tensor-core step needs bf16, d in {128, 256} and r d <= 512");
+  {
+    // the host-side plan is copied from this thread's staging memory on every
+    // call, so a captured call would replay whatever that memory holds later
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(static_cast<cudaStream_t>(stream), &cs) != cudaSuccess) {
+      cudaGetLastError();
+      return set_error(STCA_ECUDA, "stca_forward_static: cannot query the stream's capture state");
+    }
+    if (cs != cudaStreamCaptureStatusNone)
+      return set_error(STCA_EINVAL, "stca_forward_static cannot be captured into a CUDA graph "
+                                    "(its work plan is uploaded from host memory on every call)");
+  }
   int prev = -1;
   if (cudaGetDevice(&prev) != cudaSuccess) return set_error(STCA_ECUDA, "cudaGetDevice failed");
   if (prev != H->device && cudaSetDevice(H->device) != cudaSuccess)
@@ -120,13 +140,18 @@ extern "C" int stca_forward_static(stca_handle* H, const void* targets,
   // runs (fewer CTAs) until they do.
   thread_local PlanHost P;
   thread_local std::vector<unsigned char> staging;
+  // Runs per CTA are equal, so halving the CTAs roughly halves the items that
+  // a pair's keys split into; stop once a halving no longer shrinks the
+  // partials (e.g. when STCA_OPT_SPLIT_KEYS already caps the run length).
   int ctas = H->num_sms;
   StaticLayout L{};
+  int64_t prev_G = -1;
   for (;;) {
     build_plan_host(off, target_offsets, R, h, 2, ctas, H->opt_split_keys, P);
     if (int rc = check_plan(P, off, target_offsets, R, h, 2)) return rc;
     L = layout_for(P, R, T, h, d);
-    if (L.total <= kStaticScratchBytes || ctas == 1) break;
+    if (L.total <= kStaticScratchBytes || ctas == 1 || P.G == prev_G) break;
+    prev_G = P.G;
     ctas = std::max(1, ctas / 2);
   }
   if (L.total > kStaticScratchBytes)
@@ -167,7 +192,21 @@ extern "C" int stca_forward_static(stca_handle* H, const void* targets,
   plan.mtile_rows = 128;
   plan.log2_partials = 1;
 
-  launch_target_step_ws(H, -1, targets, T, nullptr, Z, Ubf, s);
+  // The per-target step runs where stca_forward runs it: on the tensor cores
+  // when the handle has that step (merging the split partials itself when
+  // every query tile has few enough items), else on the CUDA cores.
+  const bool step_tc = H->step_tc_ready && H->opt_step_path != 1;
+  int max_items = 0;
+  for (size_t k = 0; k + 1 < P.pair_item_begin.size(); ++k)
+    max_items = std::max(max_items, P.pair_item_begin[k + 1] - P.pair_item_begin[k]);
+  const bool fused = step_tc && max_items <= step_tc_max_items();
+  auto step = [&](int layer, const float* cm) -> int {
+    if (step_tc)
+      return launch_step_tc(H, layer, targets, T, fused ? nullptr : cm, &plan, part, P.G, Z, Ubf, s);
+    launch_target_step_ws(H, layer, targets, T, cm, Z, Ubf, s);
+    return STCA_OK;
+  };
+  if (int rc = step(-1, nullptr)) return rc;
   if (cudaError_t e = cudaGetLastError())
     return set_error(STCA_ECUDA, std::string("query init: ") + cudaGetErrorString(e));
   for (int i = 0; i < H->M; ++i) {
@@ -176,8 +215,8 @@ extern "C" int stca_forward_static(stca_handle* H, const void* targets,
       return rc;
     if (cudaError_t e = cudaGetLastError())
       return set_error(STCA_ECUDA, std::string("attention: ") + cudaGetErrorString(e));
-    launch_combine(H, plan, part, P.G, T, cbuf, s);
-    launch_target_step_ws(H, i, targets, T, cbuf, Z, Ubf, s);
+    if (!fused) launch_combine(H, plan, part, P.G, T, cbuf, s);
+    if (int rc = step(i, cbuf)) return rc;
     if (cudaError_t e = cudaGetLastError())
       return set_error(STCA_ECUDA, std::string("target step: ") + cudaGetErrorString(e));
   }

@@ -26,6 +26,8 @@ STCA_OK, STCA_EINVAL, STCA_ESTATE, STCA_ENOMEM, STCA_ECUDA, STCA_EDEVICE = 0, -1
 STCA_OPT_ATTN_PATH, STCA_OPT_ENCODE_PATH, STCA_OPT_SPLIT_KEYS, STCA_OPT_TIMING = 1, 2, 3, 4
 STCA_OPT_STEP_PATH = 5
 STCA_OPT_ATTN_FORM = 6
+STCA_OPT_ATTN_KERNEL = 7
+STCA_OPT_TEST_STOP_TILES = 8
 STCA_OPT_LAUNCHES = 100
 STCA_OPT_LAST_FORM = 101
 STCA_K_ENCODE, STCA_K_ATTN, STCA_K_STEP, STCA_K_HEAD, STCA_K_CLASSES = 0, 1, 2, 3, 4
@@ -38,7 +40,7 @@ EXPORTS = ("stca_init", "stca_destroy", "stca_encode", "stca_forward", "stca_run
            "stca_forward_static", "stca_head", "stca_forward_head", "stca_sl_beta", "stca_sl_plan",
            "stca_sl_gather", "stca_encode_backward", "stca_attention_backward",
            "stca_output_backward", "stca_query_backward", "stca_query_init_backward",
-           "stca_fusion_backward", "stca_last_error")
+           "stca_fusion_backward", "stca_selftest_ex2", "stca_last_error")
 
 
 class StcaError(RuntimeError):
@@ -75,6 +77,7 @@ def _load():
     lib.stca_run_host.argtypes = [P, P, PI64, I64, I64, P, PI64, I64, P, P]
     lib.stca_validate_offsets.argtypes = [PI64, I64, I64, I]
     lib.stca_device_status.argtypes = [P, P]
+    lib.stca_selftest_ex2.argtypes = [P, P, I64, I, P]
     lib.stca_set_option.argtypes = [P, I, I64]
     lib.stca_get_option.argtypes = [P, I, PI64]
     lib.stca_get_encoded.argtypes = [P, I, P, P]
@@ -446,6 +449,15 @@ def stca_validate_offsets(offsets, total: int, require_nonempty: bool = True) ->
 
 def stca_device_status(handle: int, stream=None) -> None:
     _check(_lib.stca_device_status(handle, _stream_ptr(stream)))
+
+
+def stca_selftest_ex2(x, y, method: int, stream=None) -> None:
+    """y = 2^x on the device by the attention softmax's exponential: method 0
+    the MUFU, 1 the FMA-pipe polynomial, 2 the same in pairs (packed fp32)."""
+    import torch
+    assert x.dtype == torch.float32 and y.dtype == torch.float32 and x.is_cuda and y.is_cuda
+    assert x.is_contiguous() and y.is_contiguous() and x.numel() == y.numel()
+    _check(_lib.stca_selftest_ex2(x.data_ptr(), y.data_ptr(), x.numel(), method, _stream_ptr(stream)))
 
 
 def stca_set_option(handle: int, option: int, value: int) -> None:

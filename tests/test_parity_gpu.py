@@ -221,3 +221,49 @@ def test_tensor_core_step_rejected_when_unsupported(gpu):
     wl = make_workload(lengths=[50], targets=[2], d=128, h=4, M=1, r=2, dtype="bf16", seed=13)
     with pytest.raises(S.StcaError):
         run_gpu(wl, gpu, step_path=STEP_TC, attn_path=ATTN_SIMT)
+
+
+# ------------------------------------------------------------ the two tensor-core attention kernels
+# 0: the two-group kernel (d <= 128), which merges split partials itself;
+# 1: the split-softmax kernel followed by the split combine.
+
+KERNEL_TWO_GROUP, KERNEL_SPLIT_SOFTMAX = 0, 1
+
+
+@pytest.mark.parametrize("kernel", [KERNEL_TWO_GROUP, KERNEL_SPLIT_SOFTMAX])
+@pytest.mark.parametrize("d,h", [(128, 8), (64, 4), (128, 2)])
+def test_tc_kernels_ragged(gpu, kernel, d, h):
+    wl = make_workload(lengths=EDGE_L, targets=EDGE_T, d=d, h=h, M=2, r=2, dtype="bf16",
+                       seed=400 + d + h)
+    check_full(wl, run_gpu(wl, gpu, attn_path=ATTN_TC, attn_kernel=kernel))
+
+
+@pytest.mark.parametrize("kernel", [KERNEL_TWO_GROUP, KERNEL_SPLIT_SOFTMAX])
+@pytest.mark.parametrize("split", [0, 128, 384])
+def test_tc_kernels_split_merge(gpu, kernel, split):
+    """Pairs cut into many items (one 20k-key request over every CTA, a second
+    with three query tiles, the last one ragged): every split is merged, by the
+    last-arriving warp (two-group kernel) or the combine kernel."""
+    wl = make_workload(lengths=[20000, 3000, 1], targets=[3, 40, 2], d=128, h=8, M=2, r=2,
+                       dtype="bf16", seed=410)
+    check_full(wl, run_gpu(wl, gpu, attn_path=ATTN_TC, split=split, attn_kernel=kernel))
+
+
+@pytest.mark.parametrize("kernel", [KERNEL_TWO_GROUP, KERNEL_SPLIT_SOFTMAX])
+def test_tc_kernels_sharp_softmax(gpu, kernel):
+    wl = make_workload(lengths=[3000, 900, 130], targets=[4, 3, 1], d=128, h=4, M=2, r=2,
+                       dtype="bf16", seed=411)
+    wl.weights["Wq"] = [w * 3.0 for w in wl.weights["Wq"]]
+    for r in range(3):
+        lo = int(wl.offsets[r])
+        n = min(256, int(wl.lengths[r]))
+        wl.X[lo:lo + n] = wl.X[lo]
+    check_full(wl, run_gpu(wl, gpu, attn_path=ATTN_TC, attn_kernel=kernel))
+
+
+def test_tc_kernels_agree_on_c3(gpu):
+    wl = make_config_workload("c3")
+    a = run_gpu(wl, gpu, attn_kernel=KERNEL_TWO_GROUP)
+    check_sampled(wl, a, 2, seed=3)
+    b = run_gpu(wl, gpu, attn_kernel=KERNEL_SPLIT_SOFTMAX)
+    assert normwise_err(a, b) <= 2e-2
