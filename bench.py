@@ -568,15 +568,25 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.synchronize()
     st.status(stream)
     fused_head_ms = (q1.elapsed_time(q2) - q0.elapsed_time(q1)) / args.steps
-    head_peak = 148 * 128 * 2 * 1.965e9 / 1e12
     head_ach = c["head_flops"] / (head_ms / 1e3) / 1e12
+    # bf16 handles with the tensor-core step run the head's products on the
+    # tensor cores (step_tc_kernel, head only); the others on the CUDA cores
+    head_tc = wl.dtype == "bf16" and wl.d in (128, 256) and wl.r * wl.d <= 512 and wl.M <= 8
+    if head_tc:
+        head_peak = peaks["bf16_tflops"]
+        head_roof = {"bound": "tensor", "achieved": head_ach, "peak": head_peak, "unit": "TFLOP/s",
+                     "frac": head_ach / head_peak, "flops_per_launch": c["head_flops"],
+                     "peak_source": f"bf16_tflops ({peak_src})"}
+    else:
+        head_peak = 148 * 128 * 2 * 1.965e9 / 1e12
+        head_roof = {"bound": "alu", "achieved": head_ach, "peak": head_peak, "unit": "TFLOP/s",
+                     "frac": head_ach / head_peak, "flops_per_launch": c["head_flops"],
+                     "peak_source": "nominal FP32 FFMA: 148 SMs x 128 lanes x 2 x 1.965 GHz"}
     head = {"ms_per_head": head_ms, "targets_per_s": world * wl.T / (head_ms / 1e3),
             "fused_in_last_step_ms": fused_head_ms,
-            "kernel": "head_kernel", "inputs": "Z and weights L2-resident (back-to-back calls)",
-            "roofline": {"bound": "alu", "achieved": head_ach, "peak": head_peak,
-                         "unit": "TFLOP/s", "frac": head_ach / head_peak,
-                         "flops_per_launch": c["head_flops"],
-                         "peak_source": "nominal FP32 FFMA: 148 SMs x 128 lanes x 2 x 1.965 GHz"}}
+            "kernel": "step_tc_kernel (head products only)" if head_tc else "head_kernel",
+            "inputs": "Z and weights L2-resident (back-to-back calls)",
+            "roofline": head_roof}
 
     # ---- backward of layer 1 (history encoding and merged attention), synthetic loss
     backward = None
@@ -634,7 +644,13 @@ def run_ours(args, rank, world, local_rank):
         qside_fl = sum(6 * T_ * (b + 1) * d_ * d_ + 16 * T_ * d_ * rd_ for b in range(1, wl.M + 1)) + 18 * T_ * d_ * rd_
         rd = wl.r * wl.d
         enc_fl = 18 * wl.N * wl.d * rd              # recomputed forward (6 N d rd) + 6 backward products
-        att_fl = 18 * wl.d * c["TL"] * wl.h         # per (row, key): 2 passes of 2 dots + dU; 2 dots + dX~
+        att_tc = wl.dtype == "bf16" and wl.d in (64, 128)
+        if att_tc:
+            # tensor cores: the forward attention for c and the row statistics (S, P X~),
+            # then per (row, key) S, dP, P^T dC, dS^T U and dS X~: 14 d FLOPs
+            att_fl = 14 * wl.d * c["TL"] * wl.h
+        else:
+            att_fl = 18 * wl.d * c["TL"] * wl.h     # per (row, key): 2 passes of 2 dots + dU; 2 dots + dX~
         tf32 = 1100.0
         fp32 = 148 * 128 * 2 * 1.965e9 / 1e12
         backward = {
@@ -642,9 +658,14 @@ def run_ours(args, rank, world, local_rank):
             "encode": {"ms": enc_ms, "flops": enc_fl, "tflops": enc_fl / (enc_ms / 1e3) / 1e12,
                        "frac_of_nominal_tf32": enc_fl / (enc_ms / 1e3) / 1e12 / tf32,
                        "note": "cuBLASLt TF32 products + SwiGLU / LayerNorm derivative kernels"},
-            "attention": {"ms": att_ms, "flops": att_fl, "tflops": att_fl / (att_ms / 1e3) / 1e12,
-                          "frac_of_nominal_fp32": att_fl / (att_ms / 1e3) / 1e12 / fp32,
-                          "note": "CUDA-core flash-style kernels (softmax recomputed)"},
+            "attention": ({"ms": att_ms, "flops": att_fl, "tflops": att_fl / (att_ms / 1e3) / 1e12,
+                           "frac_of_measured_bf16": att_fl / (att_ms / 1e3) / 1e12 / peaks["bf16_tflops"],
+                           "note": "tcgen05: the forward attention for c and the row statistics, delta = dC . c, "
+                                   "then S, dP, dX~ = P^T dC + dS^T U and dU = dS X~ per key tile"}
+                          if att_tc else
+                          {"ms": att_ms, "flops": att_fl, "tflops": att_fl / (att_ms / 1e3) / 1e12,
+                           "frac_of_nominal_fp32": att_fl / (att_ms / 1e3) / 1e12 / fp32,
+                           "note": "CUDA-core flash-style kernels (softmax recomputed)"}),
             "projections": {"ms": proj_ms, "flops": 20 * wl.T * wl.d * wl.d,
                             "note": "output side (W_V, W_O) and query side (W_Q, W_K): "
                                     "cuBLASLt TF32 products, the per-head slices as strided batches"},

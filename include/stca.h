@@ -222,9 +222,13 @@ int stca_forward_static(stca_handle* handle, const void* targets,
 /*
  * End-to-end call on HOST buffers: copies X and targets from host memory to
  * device staging buffers the handle owns, encodes, runs the forward, copies
- * Z (T x M x d fp32) back to host memory and waits for the stream.  Host
- * buffers should be page-locked for the copies to overlap; pageable memory
- * works but is slower.  Same argument rules as stca_encode and stca_forward.
+ * Z (T x M x d fp32) back to host memory and waits for the stream.  With the
+ * tensor-core encoder and at least 65536 history rows, X is copied in 8 chunks
+ * of whole 128-row tiles on a second stream the handle owns, and each chunk is
+ * encoded as soon as its copy has landed, so encoding overlaps the copy of the
+ * later chunks.  Host buffers should be page-locked for the copies to overlap;
+ * pageable memory works but is slower.  Same argument rules as stca_encode and
+ * stca_forward.
  */
 int stca_run_host(stca_handle* handle, const void* X_host, const int64_t* offsets,
                   int64_t R, int64_t N, const void* targets_host,
@@ -445,6 +449,9 @@ enum {
                                  of a bounded wait that ran out (copies and MMAs in flight are
                                  let finish, TMEM is freed); the next stca_device_status then
                                  reports STCA_EDEVICE.  The forward's output is not valid then */
+  STCA_OPT_BW_GEMM = 9,       /* products of the backward pieces for bf16 handles: 0 the library's
+                                 tensor-core GEMM with TF32 operands (default); 1 cuBLASLt TF32
+                                 (kept for comparison); fp32 handles always use exact fp32 */
   STCA_OPT_LAUNCHES = 100,    /* read-only: kernels launched since the last encode */
   STCA_OPT_LAST_FORM = 101    /* read-only: 1 if the last forward ran the naive form, else 0 */
 };

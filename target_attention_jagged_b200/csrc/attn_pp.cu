@@ -59,6 +59,7 @@ struct PPParams {
   float* pml;                       // G x 4: m of each column half, then l of each half
   float* cout;                      // T h x D: merged rows c, row = query row
   int* counters;                    // pairs x 8 arrivals, zero at launch
+  float* stats;                     // NULL, or T h x 2: the row's softmax max (log2 units) and sum
   int* status;
   int stop_tiles;                   // > 0: the loader stops after this many key tiles (test hook)
 };
@@ -154,6 +155,10 @@ __device__ __forceinline__ void merge_slot(const PPParams& p, const AttnItem& it
       acc.w = fmaf(f, v.w, acc.w);
     }
     const float inv = 1.f / L;
+    if (p.stats && b == 0 && c4 == 0) {
+      p.stats[(item.qrow0 + row) * 2] = mx;
+      p.stats[(item.qrow0 + row) * 2 + 1] = L;
+    }
     reinterpret_cast<float4*>(p.cout + (item.qrow0 + row) * D + b * (D / 2))[c4] =
         make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
   }
@@ -488,6 +493,10 @@ attn_pp_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         p.pml[(item.row_base + r) * 4 + b] = mx;
         p.pml[(item.row_base + r) * 4 + 2 + b] = Ltot;
       }
+      if (np == 1 && valid && p.stats && b == 0) {
+        p.stats[(item.qrow0 + r) * 2] = mx;
+        p.stats[(item.qrow0 + r) * 2 + 1] = Ltot;
+      }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(oempty);
@@ -533,8 +542,9 @@ bool attn_pp_supported(int d) { return d == 64 || d == 128; }
 int launch_attn_pp(int d, const CUtensorMap& tmQ, const CUtensorMap& tmK, const AttnItem* items_d,
                    const int32_t* cta_begin_d, const int32_t* pair_item_begin_d, int grid,
                    float* part, int64_t G, float* cout, int* counters, int* status, int stop_tiles,
-                   cudaStream_t s) {
+                   cudaStream_t s, float* stats) {
   PPParams p{};
+  p.stats = stats;
   p.items = items_d;
   p.cta_item_begin = cta_begin_d;
   p.pair_item_begin = pair_item_begin_d;

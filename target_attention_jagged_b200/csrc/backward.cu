@@ -349,6 +349,17 @@ int gemm_rm(stca_handle* H, bool ta, bool tb, int64_t m, int64_t n, int64_t k, c
             int64_t lda, const float* B, int64_t ldb, float* C, int64_t ldc, float beta,
             cudaStream_t s, float alpha = 1.f, int batch = 1, int64_t sA = 0, int64_t sB = 0,
             int64_t sC = 0) {
+  // bf16 handles: TF32 products on the tensor cores by the library's own GEMM
+  // (gemm_tc.cu); fp32 handles keep exact fp32 products (cuBLASLt, no TF32),
+  // which the 1e-3 bound of the fp32 configuration needs
+  // (a product whose operands TMA cannot address -- unaligned, or a tensor map
+  // the driver declines -- is refused before anything is launched, and runs on
+  // cuBLASLt instead)
+  if (H->elem == 2 && H->opt_bw_gemm != 1) {
+    const int rc = tc_gemm_tf32(ta, tb, m, n, k, A, lda, B, ldb, C, ldc, beta, alpha, batch, sA, sB, sC,
+                                H->num_sms, H->status_d, s);
+    if (rc != STCA_EINVAL) return rc;
+  }
   if (!H->lt) {
     cublasLtHandle_t lt = nullptr;
     if (cublasLtCreate(&lt) != CUBLAS_STATUS_SUCCESS) return set_error(STCA_ECUDA, "cublasLtCreate failed");
@@ -528,6 +539,87 @@ extern "C" int stca_query_init_backward(stca_handle* H, const void* targets, int
                          dbeta, static_cast<cudaStream_t>(stream));
 }
 
+namespace {
+
+size_t al256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// The tensor-core attention backward (attn_bw_tc.cu): the forward's work plan,
+// bf16 copies of U (log2-scaled) and dC, the forward attention for c and the
+// row statistics, delta = dC . c, then the backward kernel.
+int attention_backward_tc(stca_handle* H, int layer, const float* U, const int64_t* toff, int64_t T,
+                          const float* dC, float* dU, float* dXt, cudaStream_t s) {
+  const int d = H->d, h = H->h;
+  const int64_t R = H->R, N = H->N, rows = T * h;
+  const int64_t* off = H->offsets_h.data();
+  PlanHost P;
+  build_plan_host(off, toff, R, h, 2, H->num_sms, 0, P, H->dh);
+  if (int rc = check_plan(P, off, toff, R, h, 2)) return rc;
+  bool split_pairs = false, shared_rows = false;
+  for (size_t k = 0; k + 1 < P.pair_item_begin.size(); ++k)
+    split_pairs |= P.pair_item_begin[k + 1] - P.pair_item_begin[k] > 1;
+  for (int64_t r = 0; r < R; ++r) shared_rows |= P.req_pair_begin[r + 1] - P.req_pair_begin[r] != 1;
+  const int64_t npairs = static_cast<int64_t>(P.pair_item_begin.size()) - 1;
+  // plan arrays
+  const size_t o_items = 0, o_cta = al256(P.items.size() * sizeof(AttnItem));
+  const size_t o_pib = al256(o_cta + P.cta_begin.size() * sizeof(int32_t));
+  const size_t o_rpb = al256(o_pib + P.pair_item_begin.size() * sizeof(int32_t));
+  const size_t plan_bytes = al256(o_rpb + P.req_pair_begin.size() * sizeof(int32_t));
+  if (int rc = ensure(&H->bw_plan, &H->bw_plan_cap, plan_bytes)) return rc;
+  char* pl = static_cast<char*>(H->bw_plan);
+  STCA_CUDA_TRY(cudaMemcpyAsync(pl + o_items, P.items.data(), P.items.size() * sizeof(AttnItem),
+                                cudaMemcpyHostToDevice, s));
+  STCA_CUDA_TRY(cudaMemcpyAsync(pl + o_cta, P.cta_begin.data(), P.cta_begin.size() * sizeof(int32_t),
+                                cudaMemcpyHostToDevice, s));
+  STCA_CUDA_TRY(cudaMemcpyAsync(pl + o_pib, P.pair_item_begin.data(),
+                                P.pair_item_begin.size() * sizeof(int32_t), cudaMemcpyHostToDevice, s));
+  STCA_CUDA_TRY(cudaMemcpyAsync(pl + o_rpb, P.req_pair_begin.data(),
+                                P.req_pair_begin.size() * sizeof(int32_t), cudaMemcpyHostToDevice, s));
+  // workspace: U', dC' (bf16), c, statistics, delta, the forward's partials and counters
+  const size_t w_ub = 0, w_cb = al256(static_cast<size_t>(rows) * d * 2);
+  const size_t w_c = al256(w_cb + static_cast<size_t>(rows) * d * 2);
+  const size_t w_st = al256(w_c + static_cast<size_t>(rows) * d * 4);
+  const size_t w_dl = al256(w_st + static_cast<size_t>(rows) * 2 * 4);
+  const size_t w_part = al256(w_dl + static_cast<size_t>(rows) * 4);
+  const size_t w_cnt = al256(w_part + static_cast<size_t>(std::max<int64_t>(P.G, 1)) * (d + 4) * 4);
+  const size_t ws_bytes = al256(w_cnt + static_cast<size_t>(std::max<int64_t>(npairs, 1)) * 8 * 4);
+  if (int rc = ensure(&H->bw_ws, &H->bw_ws_cap, ws_bytes)) return rc;
+  char* w = static_cast<char*>(H->bw_ws);
+  uint16_t* Ub = reinterpret_cast<uint16_t*>(w + w_ub);
+  uint16_t* Cb = reinterpret_cast<uint16_t*>(w + w_cb);
+  float* cbuf = reinterpret_cast<float*>(w + w_c);
+  float* stats = reinterpret_cast<float*>(w + w_st);
+  float* delta = reinterpret_cast<float*>(w + w_dl);
+  float* part = reinterpret_cast<float*>(w + w_part);
+  int* cnt = reinterpret_cast<int*>(w + w_cnt);
+  CUtensorMap tmU, tmC;
+  if (int rc = make_tmap_bf16_2d(&tmU, Ub, d, rows, 64, 128)) return rc;
+  if (int rc = make_tmap_bf16_2d(&tmC, Cb, d, rows, 64, 128)) return rc;
+  STCA_CUDA_TRY(cudaMemsetAsync(cnt, 0, static_cast<size_t>(std::max<int64_t>(npairs, 1)) * 8 * 4, s));
+  launch_bw_prep(U, dC, Ub, Cb, rows * d, s);
+  STCA_CUDA_TRY(cudaGetLastError());
+  const AttnItem* items_d = reinterpret_cast<const AttnItem*>(pl + o_items);
+  const int32_t* cta_d = reinterpret_cast<const int32_t*>(pl + o_cta);
+  const int32_t* pib_d = reinterpret_cast<const int32_t*>(pl + o_pib);
+  const int32_t* rpb_d = reinterpret_cast<const int32_t*>(pl + o_rpb);
+  if (int rc = launch_attn_pp(d, tmU, H->tmXt[layer], items_d, cta_d, pib_d, P.grid, part, P.G, cbuf, cnt,
+                              H->status_d, H->opt_stop_tiles, s, stats))
+    return rc;
+  launch_bw_delta(dC, cbuf, delta, rows, d, s);
+  STCA_CUDA_TRY(cudaGetLastError());
+  if (split_pairs) STCA_CUDA_TRY(cudaMemsetAsync(dU, 0, static_cast<size_t>(rows) * d * 4, s));
+  // rows of requests without targets, or with several query tiles adding to them
+  if (shared_rows) STCA_CUDA_TRY(cudaMemsetAsync(dXt, 0, static_cast<size_t>(N) * d * 4, s));
+  if (int rc = launch_attn_bw_tc(d, tmU, tmC, H->tmXt[layer], items_d, cta_d, pib_d, rpb_d, P.grid, stats,
+                                 delta, dU, dXt, H->status_d, H->opt_stop_tiles, s))
+    return rc;
+  // (the plan's copies are from pageable memory, which the runtime has staged
+  // by the time each cudaMemcpyAsync returns)
+  set_error(STCA_OK, "");
+  return STCA_OK;
+}
+
+}  // namespace
+
 extern "C" int stca_attention_backward(stca_handle* H, int layer, const float* U,
                                        const int64_t* target_offsets, int64_t T, const float* dC,
                                        float* dU, float* dXt, void* stream) {
@@ -542,6 +634,8 @@ extern "C" int stca_attention_backward(stca_handle* H, int layer, const float* U
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int d = H->d, h = H->h;
   const int64_t R = H->R, N = H->N;
+  if (H->dtype == STCA_BF16 && attn_bw_tc_supported(d) && attn_pp_supported(d) && H->opt_attn_path != 1)
+    return attention_backward_tc(H, layer, U, target_offsets, T, dC, dU, dXt, s);
   // work units and offsets, uploaded through the handle's backward plan buffer
   std::vector<BwUnit> rows, keys;
   std::vector<int64_t> offs(2 * (R + 1));

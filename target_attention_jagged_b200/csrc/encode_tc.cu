@@ -51,11 +51,12 @@ namespace {
 using namespace tc;
 
 struct EncParams {
-  int64_t N;                 // history rows
+  int64_t N;                 // history rows of this launch
+  int64_t layer_rows;        // rows of one layer's X~ (the whole batch)
   int ntiles;                // ceil(N / 128)
   int M;                     // layers
   int nchunk;                // rd / 64
-  uint8_t* xt;               // X~ base; layer i at xt + i * N * d * 2
+  uint8_t* xt;               // X~ of this launch's first row; layer i at xt + i * layer_rows * d * 2
   const float* ln_g[16];
   const float* ln_b[16];
   int* status;
@@ -438,7 +439,7 @@ encode_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
           const float rstd = rsqrtf(var + 1e-5f);
           const float4* gam = reinterpret_cast<const float4*>(p.ln_g[layer] + hh * DH);
           const float4* bet = reinterpret_cast<const float4*>(p.ln_b[layer] + hh * DH);
-          uint8_t* orow = p.xt + (static_cast<int64_t>(layer) * p.N + row) * (D * 2) + hh * DH * 2;
+          uint8_t* orow = p.xt + (static_cast<int64_t>(layer) * p.layer_rows + row) * (D * 2) + hh * DH * 2;
 #pragma unroll
           for (int cb = 0; cb < DH / 32; ++cb) {
             const uint32_t* vv;
@@ -519,6 +520,22 @@ int launch_cfg(stca_handle* H, const CUtensorMap& tmX, const EncParams& p, cudaS
 
 }  // namespace
 
+int make_tmap_f32_3d(CUtensorMap* m, const void* base, const uint64_t dims[3], const uint64_t strides[2],
+                     const uint32_t box[3]) {
+  auto fn = encode_fn();
+  if (!fn) return set_error(STCA_ECUDA, "cuTensorMapEncodeTiled is unavailable");
+  const cuuint64_t d[3] = {dims[0], dims[1], dims[2]};
+  const cuuint64_t st[2] = {strides[0], strides[1]};
+  const cuuint32_t bx[3] = {box[0], box[1], box[2]};
+  const cuuint32_t es[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void*>(base), d, st, bx, es,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS)
+    return set_error(STCA_ECUDA, "cuTensorMapEncodeTiled (fp32, 3-d) failed (" + std::to_string(int(r)) + ")");
+  return STCA_OK;
+}
+
 int make_tmap_bf16_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer,
                       uint32_t box_inner, uint32_t box_outer) {
   return make_tmap_bf16_2d_strided(m, base, inner, outer, inner * 2, box_inner, box_outer);
@@ -584,15 +601,16 @@ int encode_tc_setup(stca_handle* H, const std::vector<const float*>& Wu,
   return STCA_OK;
 }
 
-int launch_encode_tc(stca_handle* H, const void* X, int64_t N, cudaStream_t s) {
+int launch_encode_tc(stca_handle* H, const void* X, int64_t N, cudaStream_t s, int64_t row0) {
   CUtensorMap tmX;
   if (int rc = make_tmap_bf16_2d(&tmX, X, H->d, N, 64, 128)) return rc;
   EncParams p{};
   p.N = N;
+  p.layer_rows = H->N;
   p.ntiles = static_cast<int>((N + 127) / 128);
   p.M = H->M;
   p.nchunk = H->rd / 64;
-  p.xt = static_cast<uint8_t*>(H->xt);
+  p.xt = static_cast<uint8_t*>(H->xt) + row0 * H->d * 2;
   for (int i = 0; i < H->M; ++i) {
     p.ln_g[i] = H->L32[i].ln_g;
     p.ln_b[i] = H->L32[i].ln_b;

@@ -1,0 +1,336 @@
+// Tensor-core GEMM with TF32 operands and fp32 accumulation, for the backward
+// products of bf16 handles (the products of the history encoding's backward,
+// the attention projections' and the fusion blocks'; "Make It Long, Keep It
+// Fast" digest §2.1, Eqs. (1)-(3), (6), (7), (9), (13)).
+//
+// Row-major C (m x n) = alpha op(A) op(B) + beta C, where op(A) is m x k and
+// op(B) is k x n; A or B may be stored transposed.  Each operand reaches
+// shared memory by TMA in the layout the tensor core reads directly:
+//   * op(A) = A (row-major m x k, k contiguous): K-major A, one [128 x 32] box;
+//   * op(A) = A^T (A stored k x m, m contiguous): MN-major A, four [32 k x 32 m]
+//     boxes side by side (a 128-byte row holds 32 of the 128 m values);
+//   * op(B) = B^T (B stored n x k, k contiguous): K-major B, one [BN x 32] box;
+//   * op(B) = B (B stored k x n, n contiguous): MN-major B, BN / 32 boxes.
+// One tcgen05.mma.kind::tf32 is M = 128 x N = BN x K = 8; a stage holds K = 32.
+// Partial tiles are zero-filled by TMA.  A batch of products is the third
+// tensor-map dimension.  When the output has few tiles and K is long (the
+// weight gradients, whose K is every history row), K is split over CTAs and
+// each adds its part to C atomically (C pre-scaled by the host).
+//
+// Warp roles (192 threads): warp 0 TMA, warp 1 TMEM owner and MMA issuer,
+// warps 2-5 epilogue (warp w reads TMEM lane quarter w % 4, one output row per
+// thread).  Waits are bounded; a failed wait sets the status word, in-flight
+// copies and products are let finish and TMEM is freed.
+#include <cuda.h>
+
+#include <algorithm>
+#include <string>
+
+#include "stca_internal.h"
+#include "tc_common.cuh"
+
+namespace stca {
+namespace {
+
+using namespace tc;
+
+constexpr int kGemmThreads = 192;
+constexpr int kGemmStages = 6;
+constexpr uint32_t kAStage = 128u * 128u;      // [128 x 32] fp32
+
+struct GemmArgs {
+  int64_t m, n, k;
+  int tiles_m, tiles_n, ksplit;
+  int64_t k_per_split;          // multiple of 32
+  float* C;
+  int64_t ldc, sC;
+  float alpha, beta;
+  int atomic;                   // 1: add alpha acc to C atomically (C pre-scaled)
+  int a_bmid, b_bmid;           // the batch is the tensor map's middle dimension (see below)
+  int* status;
+};
+
+__host__ __device__ constexpr uint32_t idesc_tf32(int M, int N, bool a_mn, bool b_mn) {
+  return (1u << 4)                          // D format: f32
+         | (2u << 7)                        // A format: tf32
+         | (2u << 10)                       // B format: tf32
+         | (static_cast<uint32_t>(a_mn) << 15) | (static_cast<uint32_t>(b_mn) << 16) |
+         (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+__device__ __forceinline__ void mma_tf32(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                         uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, int x, int y, int z,
+                                            uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ bool gwait(uint64_t* bar, uint32_t parity, volatile int* abort_flag, int* status) {
+  if (mbar_wait(bar, parity, abort_flag)) return true;
+  *abort_flag = 1;
+  atomicOr(status, kStatusStepTimeout);
+  return false;
+}
+
+__device__ __forceinline__ void gdrain(uint64_t* bar, uint32_t parity, uint64_t ns) {
+  const uint64_t t0 = globaltimer();
+  while (!mbar_try_wait(bar, parity))
+    if (globaltimer() - t0 > ns) break;
+}
+
+template <int BN, bool AMN, bool BMN>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+gemm_tf32_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                 const GemmArgs g) {
+  constexpr uint32_t kBStage = BN * 128u;
+  constexpr uint32_t kStage = kAStage + kBStage;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  if (smem_u32(smem_raw) & 1023u) {
+    if (threadIdx.x == 0) atomicOr(g.status, kStatusStepTimeout);
+    return;
+  }
+  uint8_t* sm = smem_raw;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sm + kGemmStages * kStage);
+  uint64_t* empty = full + kGemmStages;
+  uint64_t* accfull = empty + kGemmStages;
+  uint64_t* mdrain = accfull + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mdrain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  int u = blockIdx.x;
+  const int ks = u % g.ksplit; u /= g.ksplit;
+  const int tn = u % g.tiles_n; u /= g.tiles_n;
+  const int tm = u % g.tiles_m;
+  const int b = u / g.tiles_m;
+  const int64_t m0 = static_cast<int64_t>(tm) * 128, n0 = static_cast<int64_t>(tn) * BN;
+  const int64_t k0 = ks * g.k_per_split, k1 = min(g.k, k0 + g.k_per_split);
+  const int nst = static_cast<int>((k1 - k0 + 31) / 32);
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kGemmStages; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
+    mbar_init(accfull, 1);
+    mbar_init(mdrain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tmA);
+    prefetch_tmap(&tmB);
+  }
+  constexpr uint32_t kCols = BN < 32 ? 32 : BN;
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, kCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t sbase = smem_u32(sm);
+
+  if (warp == 0) {
+    if (lane == 0) {
+      bool ok = true;
+      int st = 0;
+      for (; ok && st < nst; ++st) {
+        const int s = st % kGemmStages;
+        if (!(ok = gwait(&empty[s], ((st / kGemmStages) & 1) ^ 1, abort_flag, g.status))) break;
+        mbar_arrive_expect_tx(&full[s], kStage);
+        uint8_t* a = sm + s * kStage;
+        uint8_t* bb = a + kAStage;
+        const int kk = static_cast<int>(k0 + 32 * st);
+        // (inner, outer) coordinates, with the batch index in the middle or last
+        auto ld = [&](void* dst, const CUtensorMap* map, int x, int y, int bmid) {
+          if (bmid) tma_load_3d(dst, map, x, b, y, &full[s]);
+          else tma_load_3d(dst, map, x, y, b, &full[s]);
+        };
+        if constexpr (AMN) {
+          for (int i = 0; i < 4; ++i) ld(a + i * 4096, &tmA, static_cast<int>(m0) + 32 * i, kk, g.a_bmid);
+        } else {
+          ld(a, &tmA, kk, static_cast<int>(m0), g.a_bmid);
+        }
+        if constexpr (BMN) {
+          for (int i = 0; i < BN / 32; ++i) ld(bb + i * 4096, &tmB, static_cast<int>(n0) + 32 * i, kk, g.b_bmid);
+        } else {
+          ld(bb, &tmB, kk, static_cast<int>(n0), g.b_bmid);
+        }
+      }
+      for (int c = st > kGemmStages ? st - kGemmStages : 0; c < st; ++c)
+        gdrain(&full[c % kGemmStages], (c / kGemmStages) & 1, 100000000ull);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_tf32(128, BN, AMN, BMN);
+      bool ok = true;
+      for (int st = 0; st < nst; ++st) {
+        const int s = st % kGemmStages;
+        if (!(ok = gwait(&full[s], (st / kGemmStages) & 1, abort_flag, g.status))) break;
+        tc_fence_after();
+        const uint32_t a = sbase + s * kStage, bb = a + kAStage;
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {          // K = 8 per MMA
+          const uint64_t ad = AMN ? sdesc_sw128(a + kk * 1024, 4096, 1024) : sdesc_sw128(a + kk * 32, 16, 1024);
+          const uint64_t bd = BMN ? sdesc_sw128(bb + kk * 1024, 4096, 1024) : sdesc_sw128(bb + kk * 32, 16, 1024);
+          mma_tf32(tmem, ad, bd, idesc, (st | kk) != 0);
+        }
+        mma_commit(&empty[s]);
+      }
+      if (ok) mma_commit(accfull);
+      mma_commit(mdrain);
+      gdrain(mdrain, 0, 500000000ull);
+    }
+  } else {
+    const int q = warp & 3;
+    const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
+    const int64_t row = m0 + q * 32 + lane;
+    const bool ok = __all_sync(0xffffffffu, nst == 0 || gwait(accfull, 0, abort_flag, g.status)) != 0;
+    if (ok && nst > 0) {
+      tc_fence_after();
+      float* crow = g.C + static_cast<int64_t>(b) * g.sC + row * g.ldc;
+#pragma unroll 1
+      for (int c = 0; c < (BN + 31) / 32; ++c) {
+        uint32_t v[32];
+        tmem_ld32(tmem + lane_off + 32 * c, v);
+        tmem_ld_wait();
+        if (row < g.m) {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const int64_t col = n0 + 32 * c + j;
+            if (col < g.n) {
+              const float x = g.alpha * __uint_as_float(v[j]);
+              if (g.atomic) atomicAdd(crow + col, x);
+              else crow[col] = g.beta != 0.f ? fmaf(g.beta, crow[col], x) : x;
+            }
+          }
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kCols);
+  }
+}
+
+// 128-bit alignment of an address and of a stride in elements.
+bool al16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool st16(int64_t elems) { return ((elems * 4) & 15) == 0; }
+
+// Tensor map of one operand stored row-major as `rows` x `inner` with row
+// stride ld, the box `bx` inner x `by` rows.  A batch whose members sit side by
+// side along the rows (stride below a whole matrix: one head's columns) is
+// the map's middle dimension, so the strides grow outward; a batch of whole
+// matrices is the outer dimension.  *bmid tells the kernel which.
+int operand_map(CUtensorMap* m, const float* base, int64_t inner, int64_t rows, int64_t ld, int batch,
+                int64_t stride, uint32_t bx, uint32_t by, int* bmid) {
+  *bmid = batch > 1 && stride < ld * rows ? 1 : 0;
+  if (*bmid) {
+    const uint64_t dims[3] = {static_cast<uint64_t>(inner), static_cast<uint64_t>(batch), static_cast<uint64_t>(rows)};
+    const uint64_t str[2] = {static_cast<uint64_t>(stride) * 4, static_cast<uint64_t>(ld) * 4};
+    const uint32_t box[3] = {bx, 1, by};
+    return make_tmap_f32_3d(m, base, dims, str, box);
+  }
+  const uint64_t dims[3] = {static_cast<uint64_t>(inner), static_cast<uint64_t>(rows), static_cast<uint64_t>(batch)};
+  const uint64_t str[2] = {static_cast<uint64_t>(ld) * 4,
+                           static_cast<uint64_t>(batch > 1 ? stride : ld * rows) * 4};
+  const uint32_t box[3] = {bx, by, 1};
+  return make_tmap_f32_3d(m, base, dims, str, box);
+}
+
+template <int BN, bool AMN, bool BMN>
+int launch_gemm(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmArgs& g, int64_t units,
+                cudaStream_t s) {
+  auto k = gemm_tf32_kernel<BN, AMN, BMN>;
+  // the stages, then 2 kGemmStages + 2 mbarriers, the TMEM slot and the abort flag
+  const uint32_t smem = kGemmStages * (kAStage + BN * 128u) + (2 * kGemmStages + 2) * 8 + 16;
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return set_error(STCA_ECUDA, std::string("gemm_tc smem: ") + cudaGetErrorString(e));
+  k<<<static_cast<unsigned>(units), kGemmThreads, smem, s>>>(tmA, tmB, g);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return set_error(STCA_ECUDA, std::string("gemm_tc launch: ") + cudaGetErrorString(e));
+  return STCA_OK;
+}
+
+template <int BN>
+int launch_gemm_bn(bool amn, bool bmn, const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmArgs& g,
+                   int64_t units, cudaStream_t s) {
+  if (amn && bmn) return launch_gemm<BN, true, true>(tmA, tmB, g, units, s);
+  if (amn) return launch_gemm<BN, true, false>(tmA, tmB, g, units, s);
+  if (bmn) return launch_gemm<BN, false, true>(tmA, tmB, g, units, s);
+  return launch_gemm<BN, false, false>(tmA, tmB, g, units, s);
+}
+
+}  // namespace
+
+int tc_gemm_tf32(bool ta, bool tb, int64_t m, int64_t n, int64_t k, const float* A, int64_t lda,
+                 const float* B, int64_t ldb, float* C, int64_t ldc, float beta, float alpha, int batch,
+                 int64_t sA, int64_t sB, int64_t sC, int num_sms, int* status, cudaStream_t s) {
+  if (m <= 0 || n <= 0 || batch <= 0) return STCA_OK;
+  if (!al16(A) || !al16(B) || !st16(lda) || !st16(ldb) || (batch > 1 && (!st16(sA) || !st16(sB))))
+    return set_error(STCA_EINVAL, "tensor-core GEMM: operands not 16-byte aligned");
+  if (m > INT32_MAX || n > INT32_MAX || k > INT32_MAX) return set_error(STCA_EINVAL, "tensor-core GEMM: too large");
+  const bool amn = ta, bmn = !tb;
+  // tile width: 128 columns, or 64 / 32 for narrow outputs
+  int BN = 128;
+  while (BN > 32 && BN / 2 >= n) BN /= 2;
+  GemmArgs g{};
+  g.m = m;
+  g.n = n;
+  g.k = k;
+  g.tiles_m = static_cast<int>((m + 127) / 128);
+  g.tiles_n = static_cast<int>((n + BN - 1) / BN);
+  g.C = C;
+  g.ldc = ldc;
+  g.sC = sC;
+  g.alpha = alpha;
+  g.beta = beta;
+  g.status = status;
+  // split a long K over CTAs when the output tiles alone cannot fill the GPU
+  const int64_t tiles = static_cast<int64_t>(g.tiles_m) * g.tiles_n * batch;
+  int ksplit = 1;
+  if (k >= 4096 && tiles < num_sms) ksplit = static_cast<int>(std::min<int64_t>(num_sms / tiles, (k + 1023) / 1024));
+  ksplit = std::max(ksplit, 1);
+  g.k_per_split = ((k + ksplit - 1) / ksplit + 31) / 32 * 32;
+  g.ksplit = static_cast<int>(std::max<int64_t>(1, (k + g.k_per_split - 1) / g.k_per_split));
+  g.atomic = g.ksplit > 1;
+  CUtensorMap tmA, tmB;
+  // op(A): A^T stored k x m (MN-major) or A stored m x k (K-major);
+  // op(B): B stored k x n (MN-major) or B^T stored n x k (K-major).
+  // A map the driver declines is reported as STCA_EINVAL: nothing has run yet.
+  if (operand_map(&tmA, A, amn ? m : k, amn ? k : m, lda, batch, sA, 32, amn ? 32u : 128u, &g.a_bmid) ||
+      operand_map(&tmB, B, bmn ? n : k, bmn ? k : n, ldb, batch, sB, 32, bmn ? 32u : static_cast<uint32_t>(BN),
+                  &g.b_bmid))
+    return set_error(STCA_EINVAL, "tensor-core GEMM: operand layout not expressible as a tensor map");
+  if (g.atomic) {
+    // every split adds alpha times its part to C, which starts as beta C
+    if (beta == 0.f) {
+      for (int i = 0; i < batch; ++i)
+        STCA_CUDA_TRY(cudaMemset2DAsync(C + i * sC, ldc * 4, 0, n * 4, m, s));
+    } else if (beta != 1.f) {
+      return set_error(STCA_EINVAL, "tensor-core GEMM: split K needs beta 0 or 1");
+    }
+  }
+  const int64_t units = static_cast<int64_t>(g.tiles_m) * g.tiles_n * g.ksplit * batch;
+  if (units > INT32_MAX) return set_error(STCA_EINVAL, "tensor-core GEMM: too many tiles");
+  switch (BN) {
+    case 128: return launch_gemm_bn<128>(amn, bmn, tmA, tmB, g, units, s);
+    case 64: return launch_gemm_bn<64>(amn, bmn, tmA, tmB, g, units, s);
+    default: return launch_gemm_bn<32>(amn, bmn, tmA, tmB, g, units, s);
+  }
+}
+
+}  // namespace stca

@@ -192,6 +192,8 @@ extern "C" void stca_destroy(stca_handle* H) {
   cudaFree(H->t_stage);
   cudaFree(H->z_stage);
   if (H->plan_h) cudaFreeHost(H->plan_h);
+  for (auto e : H->chunk_evt) cudaEventDestroy(e);
+  if (H->copy_stream) cudaStreamDestroy(H->copy_stream);
   if (H->plan_evt) cudaEventDestroy(H->plan_evt);
   for (auto& t : H->timed) { cudaEventDestroy(t.a); cudaEventDestroy(t.b); }
   for (auto e : H->ev_pool) cudaEventDestroy(e);
@@ -470,16 +472,14 @@ extern "C" int stca_init(const stca_weights* w, int d, int h, int r, int M, int 
 
 // ------------------------------------------------------------------ encode
 
-extern "C" int stca_encode(stca_handle* H, const void* X, const int64_t* offsets, int64_t R,
-                           int64_t N, void* stream) {
+// Checks, the handle's encoded-state bookkeeping and the X~ tensor maps of an
+// encode of N rows (the launches follow).
+static int encode_begin(stca_handle* H, const void* X, const int64_t* offsets, int64_t R, int64_t N) {
   if (!H) return set_error(STCA_EINVAL, "handle is NULL");
   if (!X) return set_error(STCA_EINVAL, "X is NULL");
   if (reinterpret_cast<uintptr_t>(X) % 16) return set_error(STCA_EINVAL, "X must be 16-byte aligned");
   if (N < 1) return set_error(STCA_EINVAL, "N must be >= 1");
   if (int rc = validate_offsets(offsets, R, N, true, "offsets")) return rc;
-  DeviceGuard g(H->device);
-  if (!g.ok) return set_error(STCA_ECUDA, "cannot select the handle's device");
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
   const size_t layer_bytes = static_cast<size_t>(N) * H->d * H->elem;
   if (int rc = ensure_dev(&H->xt, &H->xt_cap, layer_bytes * H->M)) return rc;
   H->encoded = false;
@@ -494,10 +494,25 @@ extern "C" int stca_encode(stca_handle* H, const void* X, const int64_t* offsets
                                      H->d, N, 64, 128))
         return rc;
   }
-  const bool bf = H->dtype == STCA_BF16;
   if (H->opt_encode_path == 2 && !H->tc_encode_ready)
     return set_error(STCA_EINVAL, "tensor-core encoder needs bf16 and d in {64,128,256}, rd % 64 == 0");
-  if (H->tc_encode_ready && H->opt_encode_path != 1) {
+  return STCA_OK;
+}
+
+static bool encode_on_tensor_cores(const stca_handle* H) {
+  return H->tc_encode_ready && H->opt_encode_path != 1;
+}
+
+extern "C" int stca_encode(stca_handle* H, const void* X, const int64_t* offsets, int64_t R,
+                           int64_t N, void* stream) {
+  if (!H) return set_error(STCA_EINVAL, "handle is NULL");
+  DeviceGuard g(H->device);
+  if (!g.ok) return set_error(STCA_ECUDA, "cannot select the handle's device");
+  if (int rc = encode_begin(H, X, offsets, R, N)) return rc;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const size_t layer_bytes = static_cast<size_t>(N) * H->d * H->elem;
+  const bool bf = H->dtype == STCA_BF16;
+  if (encode_on_tensor_cores(H)) {
     int rc;
     {
       TimedLaunch tl(H, STCA_K_ENCODE, s);
@@ -766,6 +781,8 @@ static int build_plan(stca_handle* H, const int64_t* toff, int64_t T, int path, 
     return set_error(STCA_ECUDA, "plan event wait failed");
   if (bytes > H->plan_h_cap) {
     if (H->plan_h) cudaFreeHost(H->plan_h);
+  for (auto e : H->chunk_evt) cudaEventDestroy(e);
+  if (H->copy_stream) cudaStreamDestroy(H->copy_stream);
     H->plan_h = nullptr;
     H->plan_h_cap = 0;
     if (cudaMallocHost(&H->plan_h, bytes) != cudaSuccess) {
@@ -1008,7 +1025,14 @@ extern "C" int stca_head(stca_handle* H, const void* targets, int64_t T, const f
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   {
     TimedLaunch tl(H, STCA_K_HEAD, s);
-    launch_head(H, targets, T, Z, zout, s);
+    // bf16 handles with the tensor-core step: its head products, as in the
+    // forward's last step; otherwise the CUDA-core head kernel
+    if (H->step_tc_ready && H->head_tc && H->opt_step_path != 1 &&
+        reinterpret_cast<uintptr_t>(targets) % 16 == 0 && reinterpret_cast<uintptr_t>(Z) % 16 == 0) {
+      if (int rc = launch_step_tc_head(H, targets, T, Z, zout, s)) return rc;
+    } else {
+      launch_head(H, targets, T, Z, zout, s);
+    }
   }
   H->launches++;
   STCA_CUDA_TRY(cudaGetLastError());
@@ -1062,6 +1086,11 @@ extern "C" int stca_plan_attention(const int64_t* offsets, const int64_t* target
 }
 
 // ------------------------------------------------------------------ host entry
+// End to end from host buffers.  With the tensor-core encoder and a large
+// batch, X crosses to the device in chunks of whole 128-row tiles on a second
+// stream, and each chunk is encoded as soon as its copy lands (an event per
+// chunk), so the encoder works while the next chunks are still in flight; the
+// forward follows the last chunk.  One cudaMemcpyAsync per chunk.
 extern "C" int stca_run_host(stca_handle* H, const void* X_host, const int64_t* offsets,
                              int64_t R, int64_t N, const void* targets_host,
                              const int64_t* target_offsets, int64_t T, float* Z_host,
@@ -1076,7 +1105,8 @@ extern "C" int stca_run_host(stca_handle* H, const void* X_host, const int64_t* 
   DeviceGuard g(H->device);
   if (!g.ok) return set_error(STCA_ECUDA, "cannot select the handle's device");
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const size_t xb = static_cast<size_t>(N) * H->d * H->elem;
+  const size_t row_bytes = static_cast<size_t>(H->d) * H->elem;
+  const size_t xb = static_cast<size_t>(N) * row_bytes;
   const size_t tb = static_cast<size_t>(T) * H->d * H->elem;
   const size_t zb = static_cast<size_t>(T) * H->M * H->d * sizeof(float);
   if (int rc = ensure_dev(&H->x_stage, &H->x_stage_cap, xb)) return rc;
@@ -1084,9 +1114,57 @@ extern "C" int stca_run_host(stca_handle* H, const void* X_host, const int64_t* 
     if (int rc = ensure_dev(&H->t_stage, &H->t_stage_cap, tb)) return rc;
     if (int rc = ensure_dev(reinterpret_cast<void**>(&H->z_stage), &H->z_stage_cap, zb)) return rc;
   }
-  STCA_CUDA_TRY(cudaMemcpyAsync(H->x_stage, X_host, xb, cudaMemcpyHostToDevice, s));
+  constexpr int kChunks = 8;
+  constexpr int64_t kMinChunkRows = 8192;
+  const bool chunked = encode_on_tensor_cores(H) && N >= kChunks * kMinChunkRows;
   if (T > 0) STCA_CUDA_TRY(cudaMemcpyAsync(H->t_stage, targets_host, tb, cudaMemcpyHostToDevice, s));
-  if (int rc = stca_encode(H, H->x_stage, offsets, R, N, stream)) return rc;
+  if (!chunked) {
+    STCA_CUDA_TRY(cudaMemcpyAsync(H->x_stage, X_host, xb, cudaMemcpyHostToDevice, s));
+    if (int rc = stca_encode(H, H->x_stage, offsets, R, N, stream)) return rc;
+  } else {
+    if (!H->copy_stream &&
+        cudaStreamCreateWithFlags(&H->copy_stream, cudaStreamNonBlocking) != cudaSuccess) {
+      cudaGetLastError();
+      H->copy_stream = nullptr;
+      return set_error(STCA_ECUDA, "cannot create the copy stream");
+    }
+    while (H->chunk_evt.size() < kChunks + 1) {
+      cudaEvent_t e = nullptr;
+      if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) {
+        cudaGetLastError();
+        return set_error(STCA_ECUDA, "cannot create the chunk events");
+      }
+      H->chunk_evt.push_back(e);
+    }
+    if (int rc = encode_begin(H, H->x_stage, offsets, R, N)) return rc;
+    // the copies overwrite the staging buffer: after everything on `stream` so far
+    STCA_CUDA_TRY(cudaEventRecord(H->chunk_evt[kChunks], s));
+    STCA_CUDA_TRY(cudaStreamWaitEvent(H->copy_stream, H->chunk_evt[kChunks], 0));
+    const int64_t tiles = (N + 127) / 128;
+    const int64_t per = (tiles + kChunks - 1) / kChunks * 128;
+    for (int c = 0; c < kChunks; ++c) {
+      const int64_t r0 = c * per, rows = std::min<int64_t>(per, N - r0);
+      if (rows <= 0) break;
+      STCA_CUDA_TRY(cudaMemcpyAsync(static_cast<char*>(H->x_stage) + r0 * row_bytes,
+                                    static_cast<const char*>(X_host) + r0 * row_bytes, rows * row_bytes,
+                                    cudaMemcpyHostToDevice, H->copy_stream));
+      STCA_CUDA_TRY(cudaEventRecord(H->chunk_evt[c], H->copy_stream));
+    }
+    for (int c = 0; c < kChunks; ++c) {
+      const int64_t r0 = c * per, rows = std::min<int64_t>(per, N - r0);
+      if (rows <= 0) break;
+      STCA_CUDA_TRY(cudaStreamWaitEvent(s, H->chunk_evt[c], 0));
+      int rc;
+      {
+        TimedLaunch tl(H, STCA_K_ENCODE, s);
+        rc = launch_encode_tc(H, static_cast<const char*>(H->x_stage) + r0 * row_bytes, rows, s, r0);
+      }
+      if (rc) return rc;
+      H->launches++;
+      if (int rc2 = check_launch("encode (tensor cores, chunk)")) return rc2;
+    }
+    H->encoded = true;
+  }
   if (T > 0) {
     if (int rc = stca_forward(H, H->t_stage, target_offsets, T, H->z_stage, stream)) return rc;
     STCA_CUDA_TRY(cudaMemcpyAsync(Z_host, H->z_stage, zb, cudaMemcpyDeviceToHost, s));
@@ -1146,6 +1224,10 @@ extern "C" int stca_set_option(stca_handle* H, int option, int64_t value) {
       if (value < 0 || value > (int64_t(1) << 30)) return set_error(STCA_EINVAL, "stop tiles must be >= 0");
       H->opt_stop_tiles = static_cast<int>(value);
       return ok();
+    case STCA_OPT_BW_GEMM:
+      if (value < 0 || value > 1) return set_error(STCA_EINVAL, "backward GEMM must be 0 or 1");
+      H->opt_bw_gemm = static_cast<int>(value);
+      return ok();
     case STCA_OPT_SPLIT_KEYS:
       if (value < 0 || value % 128 || value > (int64_t(1) << 30))
         return set_error(STCA_EINVAL, "split must be 0 or a positive multiple of 128");
@@ -1168,6 +1250,7 @@ extern "C" int stca_get_option(stca_handle* H, int option, int64_t* value) {
     case STCA_OPT_ATTN_FORM: *value = H->opt_attn_form; return ok();
     case STCA_OPT_ATTN_KERNEL: *value = H->opt_attn_kernel; return ok();
     case STCA_OPT_TEST_STOP_TILES: *value = H->opt_stop_tiles; return ok();
+    case STCA_OPT_BW_GEMM: *value = H->opt_bw_gemm; return ok();
     case STCA_OPT_LAST_FORM: *value = H->last_naive ? 1 : 0; return ok();
     default: return set_error(STCA_EINVAL, "unknown option " + std::to_string(option));
   }

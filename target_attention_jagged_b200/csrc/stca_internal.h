@@ -133,6 +133,7 @@ struct stca_handle {
   int64_t opt_split_keys = 0;
   int opt_attn_kernel = 0;              // 0 auto (two-group kernel for d <= 128), 1 split-softmax kernel
   int opt_stop_tiles = 0;               // test hook: the attention loader stops after this many tiles
+  int opt_bw_gemm = 0;                  // backward products of bf16 handles: 0 tensor cores (TF32), 1 cuBLASLt
   int64_t launches = 0;
   bool timing = false;
   struct TimedRec { int cls; cudaEvent_t a, b; };
@@ -159,6 +160,8 @@ struct stca_handle {
   int* status_d = nullptr;
 
   // host-buffer entry point staging
+  cudaStream_t copy_stream = nullptr;   // stca_run_host: the chunks' host-to-device copies
+  std::vector<cudaEvent_t> chunk_evt;   // one per chunk: its copy has landed
   void* x_stage = nullptr;  size_t x_stage_cap = 0;
   void* t_stage = nullptr;  size_t t_stage_cap = 0;
   float* z_stage = nullptr; size_t z_stage_cap = 0;
@@ -225,6 +228,9 @@ int step_tc_setup(stca_handle* H, const std::vector<StepHostW>& layers, const He
 // partials (part: G x d accumulators, then G maxima, G sums) inside the step;
 // that needs at most step_tc_max_items() items per (request, query tile).
 int step_tc_max_items();
+// The prediction head of Eq. (9) alone on the tensor cores, from Z (T x M x d).
+int launch_step_tc_head(const stca_handle* H, const void* targets, int64_t T, const float* Z, float* zout,
+                        cudaStream_t s);
 // Naive form of the step: `naive` not NULL; cmerged then holds o_head (T x d, the
 // per-head outputs of Eq. (12)), and the query rows of the next layer are written
 // into the packed layout (NaiveLayout) at naive->upk, request r from row qbase[r].
@@ -264,11 +270,13 @@ int launch_attn_tc_ws(int d, const CUtensorMap& tmQ, const CUtensorMap& tmK,
 // Two-group tensor-core attention with the split combine inside (attn_pp.cu):
 // writes the merged rows c (T h x d fp32) to `cout`; part holds G x d partial
 // rows then G x 4 (m, l) values; counters (pairs x 8 ints) must be zero.
+// stats, when not NULL: T h x 2 floats, each row's softmax maximum (log2 units
+// of the bf16 query rows' scores) and sum.
 bool attn_pp_supported(int d);
 int launch_attn_pp(int d, const CUtensorMap& tmQ, const CUtensorMap& tmK, const AttnItem* items_d,
                    const int32_t* cta_begin_d, const int32_t* pair_item_begin_d, int grid,
                    float* part, int64_t G, float* cout, int* counters, int* status, int stop_tiles,
-                   cudaStream_t s);
+                   cudaStream_t s, float* stats = nullptr);
 
 // Naive form's K/V projection on the tensor cores (kv_proj.cu): out (N x 2d
 // bf16) = X~ (tmX: N x d, box 64 x 128) times [W_K | W_V] (tmW: its transpose,
@@ -276,6 +284,15 @@ int launch_attn_pp(int d, const CUtensorMap& tmQ, const CUtensorMap& tmK, const 
 bool kv_proj_supported(int d);
 int launch_kv_proj(int d, const CUtensorMap& tmX, const CUtensorMap& tmW, uint16_t* out, int64_t N,
                    int num_sms, int* status, cudaStream_t s);
+
+// Attention backward on the tensor cores (attn_bw_tc.cu), d in {64, 128}.
+bool attn_bw_tc_supported(int d);
+void launch_bw_prep(const float* U, const float* dC, uint16_t* Ub, uint16_t* dCb, int64_t n, cudaStream_t s);
+void launch_bw_delta(const float* dC, const float* c, float* delta, int64_t rows, int d, cudaStream_t s);
+int launch_attn_bw_tc(int d, const CUtensorMap& tmQ, const CUtensorMap& tmC, const CUtensorMap& tmK,
+                      const AttnItem* items, const int32_t* cta_begin, const int32_t* pair_item_begin,
+                      const int32_t* req_pair_begin, int grid, const float* stats, const float* delta,
+                      float* dU, float* dX, int* status, int stop_tiles, cudaStream_t s);
 
 // Tensor-core attention (attn_tc.cu)
 bool attn_tc_supported(int d);
@@ -288,9 +305,23 @@ int launch_attn_tc_naive(stca_handle* H, const AttnItem* items_d, const int32_t*
 bool encode_tc_supported(int d, int rd);
 int encode_tc_setup(stca_handle* H, const std::vector<const float*>& Wu,
                     const std::vector<const float*>& Wg, const std::vector<const float*>& Wd);
-int launch_encode_tc(stca_handle* H, const void* X, int64_t N, cudaStream_t s);
+// Encodes the N rows at X into rows row0 .. row0 + N - 1 of every layer's X~
+// (H->N rows per layer).
+int launch_encode_tc(stca_handle* H, const void* X, int64_t N, cudaStream_t s, int64_t row0 = 0);
 int make_tmap_bf16_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer,
                       uint32_t box_inner, uint32_t box_outer);
+// fp32 tensor map of three dimensions (innermost first; strides of the outer
+// two in bytes, multiples of 16), 128-byte swizzle.
+int make_tmap_f32_3d(CUtensorMap* m, const void* base, const uint64_t dims[3], const uint64_t strides[2],
+                     const uint32_t box[3]);
+// Hand-written tensor-core GEMM with TF32 operands (gemm_tc.cu), row-major:
+// C (m x n) = alpha op(A) op(B) + beta C, ta / tb: A / B stored transposed;
+// `batch` products with operand strides sA, sB, sC (elements).  Returns
+// STCA_EINVAL without launching when the operands' alignment does not allow
+// TMA (addresses and row strides multiples of 16 bytes).
+int tc_gemm_tf32(bool ta, bool tb, int64_t m, int64_t n, int64_t k, const float* A, int64_t lda,
+                 const float* B, int64_t ldb, float* C, int64_t ldc, float beta, float alpha, int batch,
+                 int64_t sA, int64_t sB, int64_t sC, int num_sms, int* status, cudaStream_t s);
 // The same with rows `row_bytes` apart (a multiple of 16).
 int make_tmap_bf16_2d_strided(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer,
                               uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer);

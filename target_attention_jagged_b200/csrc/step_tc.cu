@@ -179,6 +179,7 @@ struct StepTcArgs {
   const int64_t* qbase;         // first packed row of each request
   uint16_t* upk;                // packed query rows [rows x 64] bf16
   float* zout;                  // prediction head z (T x d) when the last layer runs it, or NULL
+  int head_only;                // the head alone: its operand [o(1) .. o(M) | x_t] all from Z
 };
 
 // Shared memory, in bytes (1024-aligned base): the A-tile ring, then the
@@ -365,7 +366,7 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_tc_kernel(const StepTcAr
     int32_t* cw_g = reinterpret_cast<int32_t*>(sm + Y.cw);
     float* cw_f = reinterpret_cast<float*>(cw_g + nq * kMaxItems);
     int32_t* cw_n = reinterpret_cast<int32_t*>(cw_f + nq * kMaxItems);
-    if (L >= 0 && a.cmerged == nullptr) {
+    if (L >= 0 && a.cmerged == nullptr && !a.head_only) {
       // split combine of Eq. (13)'s alpha_j X~: c_j = sum_w 2^(m_w - m) acc_w / L,
       // L = sum_w 2^(m_w - m) l_w, over the items w that cover query row (t, j)
       for (int qi = tid; qi < nq; qi += 32 * kWorkers) {
@@ -419,10 +420,10 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_tc_kernel(const StepTcAr
         for (int e = tid; e < kTgt * wcat8; e += 32 * kWorkers) {
           const int t = e / wcat8, k8 = e - t * wcat8;
           const int blk = k8 / d8, kk = 8 * (k8 - blk * d8);
-          if (blk == L) continue;
+          if (blk == L && !a.head_only) continue;
           uint4 v = make_uint4(0u, 0u, 0u, 0u);
           if (t < nb) {
-            if (blk < L) {
+            if (blk < L || (blk == L && a.head_only)) {
               const float4* z = reinterpret_cast<const float4*>(a.Z + ((t0 + t) * M + blk) * d + kk);
               const float4 z0 = z[0], z1 = z[1];
               v = make_uint4(pack_bf16x2(z0.x, z0.y), pack_bf16x2(z0.z, z0.w),
@@ -434,7 +435,9 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_tc_kernel(const StepTcAr
           *reinterpret_cast<uint4*>(bufs[kC] + (8 * k8 >> 6) * kBTile + sw128_off(t, (8 * k8) & 63)) = v;
         }
       }
-      if (a.naive) {
+      if (a.head_only) {
+        // nothing more: the head's operand is complete
+      } else if (a.naive) {
         // naive form: the per-head outputs o_head[t] (already alpha V per head)
         // are the B operand of W_O as they are
         const int d8 = d / 8;
@@ -767,6 +770,45 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_tc_kernel(const StepTcAr
 // q(layer+2) and its u; layer = M-1: output only.  Writes the bf16 query rows
 // scaled by log2(e) / sqrt(d_h) (the tensor-core attention's units).
 int step_tc_max_items() { return kMaxItems; }
+
+// The prediction head of Eq. (9) alone, for T targets whose Z (T x M x d) is
+// given: one launch of the step kernel with the head's three products.
+int launch_step_tc_head(const stca_handle* H, const void* targets, int64_t T, const float* Z, float* zout,
+                        cudaStream_t s) {
+  if (T <= 0) return STCA_OK;
+  if (!H->step_tc_ready || !H->head_tc) return set_error(STCA_ESTATE, "tensor-core head weights are not set up");
+  const int M = H->M;
+  StepTcArgs a{};
+  a.layer = M - 1;
+  a.M = M; a.d = H->d; a.h = H->h; a.dh = H->dh; a.rd = H->rd;
+  a.T = T;
+  a.targets = static_cast<const uint16_t*>(targets);
+  a.Z = const_cast<float*>(Z);     // read only: the head writes zout
+  a.tiles = H->wstep_tc;
+  a.q_ln_g = H->q_ln_g;
+  a.q_ln_b = H->q_ln_b;
+  a.status = H->status_d;
+  a.zout = zout;
+  a.head_only = 1;
+  a.kind[0] = kC; a.g[0] = H->tcZC;
+  a.kind[1] = kUG; a.g[1] = H->tcZUG;
+  a.kind[2] = kZ; a.g[2] = H->tcZD;
+  a.ng = 3;
+  int nring = kMaxRing;
+  while (nring > 2 && step_layout(H->d, H->rd, M, H->h, nring).total + 1024 > 227u * 1024) --nring;
+  const StepLayout Y = step_layout(H->d, H->rd, M, H->h, nring);
+  if (Y.total + 1024 > 227u * 1024) return set_error(STCA_EINVAL, "tensor-core head: shared memory");
+  a.nring = nring;
+  a.kch = 4;
+  const size_t smem = Y.total + 1024;
+  cudaError_t e = cudaFuncSetAttribute(step_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return set_error(STCA_ECUDA, std::string("step_tc smem: ") + cudaGetErrorString(e));
+  const unsigned grid = static_cast<unsigned>((T + kTgt - 1) / kTgt);
+  e = launch_pdl(step_tc_kernel, dim3(grid), dim3(kStepThreads), smem, s, a);
+  if (e != cudaSuccess) return set_error(STCA_ECUDA, std::string("step_tc launch: ") + cudaGetErrorString(e));
+  return STCA_OK;
+}
 
 int launch_step_tc(const stca_handle* H, int layer, const void* targets, int64_t T,
                    const float* cmerged, const StepPlan* plan, const float* part, int64_t G,

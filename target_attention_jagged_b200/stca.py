@@ -28,6 +28,7 @@ STCA_OPT_STEP_PATH = 5
 STCA_OPT_ATTN_FORM = 6
 STCA_OPT_ATTN_KERNEL = 7
 STCA_OPT_TEST_STOP_TILES = 8
+STCA_OPT_BW_GEMM = 9
 STCA_OPT_LAUNCHES = 100
 STCA_OPT_LAST_FORM = 101
 STCA_K_ENCODE, STCA_K_ATTN, STCA_K_STEP, STCA_K_HEAD, STCA_K_CLASSES = 0, 1, 2, 3, 4

@@ -39,25 +39,63 @@ def test_encode_backward_matches_oracle(gpu, dtype, d, r, layer):
         assert _rel(got[k], want[k]) <= tol, (k, _rel(got[k], want[k]))
 
 
-@pytest.mark.parametrize("dtype,d,h,layer", [("bf16", 128, 8, 0), ("f32", 64, 2, 1),
-                                             ("bf16", 256, 16, 1)])
-def test_attention_backward_matches_oracle(gpu, dtype, d, h, layer):
+@pytest.mark.parametrize("d,r,lengths", [(128, 4, [5000, 1200, 3]), (64, 2, [4100, 1])])
+def test_encode_backward_gemm_paths(gpu, d, r, lengths):
+    """bf16 handle: the library's tensor-core TF32 GEMM (default) and cuBLASLt
+    (STCA_OPT_BW_GEMM = 1) against the oracle, on enough rows (N > 4096) that the
+    weight gradients' long K is split over CTAs and added atomically."""
     import torch
     import target_attention_jagged_b200 as S
-    lengths, targets = [700, 1, 129, 300, 64], [3, 2, 0, 5, 1]
+    wl = make_workload(lengths=lengths, targets=[1] * len(lengths), d=d, h=4, M=1, r=r, dtype="bf16",
+                       seed=950 + d, random_ln=True)
+    G = np.random.default_rng(d).standard_normal((wl.N, d)).astype(np.float32)
+    want = B.encode_history_backward(wl.X, wl.weights, 0, G)
+    for gemm in (0, 1):
+        with S.Stca(storage_weights(wl), d, 4, r, 1, "bf16") as st:
+            st.set_option(S.STCA_OPT_BW_GEMM, gemm)
+            X = to_device(wl, wl.X, gpu)
+            g = S.stca_encode_backward(st.handle, 0, X, torch.from_numpy(G).to(gpu), d, r * d)
+            torch.cuda.synchronize()
+            st.status()
+            got = {k: v.cpu().numpy() for k, v in g.items()}
+        assert normwise_err(got["dX"], want["dX"]) <= TOL["bf16"], gemm
+        for k in ("dWu", "dWg", "dWd", "dgamma", "dbeta"):
+            assert _rel(got[k], want[k]) <= TOL["bf16"], (gemm, k, _rel(got[k], want[k]))
+
+
+# path 0: the library's choice (tensor cores for bf16 and d in {64, 128}, else
+# CUDA cores); path 1: the CUDA-core kernels forced (STCA_OPT_ATTN_PATH).
+# The last cases give requests several 128-row query tiles (several tiles add
+# to the same history rows) and a 6000-key history (its query tile's keys are
+# split over several CTAs, whose dU parts add up).
+@pytest.mark.parametrize("dtype,d,h,layer,lengths,targets,path", [
+    ("bf16", 128, 8, 0, [700, 1, 129, 300, 64], [3, 2, 0, 5, 1], 0),
+    ("bf16", 128, 8, 0, [700, 1, 129, 300, 64], [3, 2, 0, 5, 1], 1),
+    ("f32", 64, 2, 1, [700, 1, 129, 300, 64], [3, 2, 0, 5, 1], 0),
+    ("bf16", 256, 16, 1, [700, 1, 129, 300, 64], [3, 2, 0, 5, 1], 0),
+    ("bf16", 64, 4, 1, [700, 1, 129, 300, 64], [3, 2, 0, 5, 1], 0),
+    ("bf16", 128, 8, 1, [6000, 333, 1, 900], [20, 17, 1, 0], 0),
+    ("bf16", 64, 8, 0, [6000, 333, 1, 900], [20, 17, 1, 0], 0),
+])
+def test_attention_backward_matches_oracle(gpu, dtype, d, h, layer, lengths, targets, path):
+    import torch
+    import target_attention_jagged_b200 as S
     wl = make_workload(lengths=lengths, targets=targets, d=d, h=h, M=2, r=2, dtype=dtype, seed=77 + d)
     rng = np.random.default_rng(d + h)
     rows = wl.T * h
     U = (rng.standard_normal((rows, d)) * (2.0 / np.sqrt(d))).astype(np.float32)
     dC = rng.standard_normal((rows, d)).astype(np.float32)
     with S.Stca(storage_weights(wl), d, h, 2, 2, dtype) as st:
+        if path:
+            st.set_option(S.STCA_OPT_ATTN_PATH, path)
         st.encode(to_device(wl, wl.X, gpu), wl.offsets)
         xt = torch.empty((wl.N, d), dtype=torch.bfloat16 if dtype == "bf16" else torch.float32, device=gpu)
         S.stca_get_encoded(st.handle, layer, xt)
-        dU, dX = S.stca_attention_backward(st.handle, layer, torch.from_numpy(U).to(gpu),
-                                           wl.target_offsets, torch.from_numpy(dC).to(gpu), wl.N)
-        torch.cuda.synchronize()
-        st.status()
+        for _ in range(2):          # a second call reuses the workspace
+            dU, dX = S.stca_attention_backward(st.handle, layer, torch.from_numpy(U).to(gpu),
+                                               wl.target_offsets, torch.from_numpy(dC).to(gpu), wl.N)
+            torch.cuda.synchronize()
+            st.status()
         Xt = xt.float().cpu().numpy()
         got_u, got_x = dU.cpu().numpy(), dX.cpu().numpy()
     want_u, want_x = B.attention_backward_batch(U, Xt, wl.offsets, wl.target_offsets, h, dC)

@@ -53,6 +53,26 @@ def test_head_on_given_outputs(gpu, dtype, d, h, M, r, T):
     assert err <= TOL[dtype], f"head normwise error {err:.3e}"
 
 
+@pytest.mark.parametrize("step_path", [1, 2])
+def test_head_paths_bf16(gpu, step_path):
+    """stca_head on a bf16 handle: the tensor-core head products (step path 2,
+    the default where the handle has them) and the CUDA-core head kernel
+    (step path 1), 1000 targets with a ragged last CTA."""
+    import target_attention_jagged_b200 as S
+    T, d, h, M, r = 1000, 128, 8, 3, 4
+    wl = make_workload(lengths=[5], targets=[T], d=d, h=h, M=M, r=r, dtype="bf16", seed=350 + step_path)
+    Z = np.random.default_rng([T, d]).standard_normal((T, M, d)).astype(np.float32)
+    st = S.Stca(storage_weights(wl), d, h, r, M, "bf16")
+    try:
+        st.set_option(S.STCA_OPT_STEP_PATH, step_path)
+        z = _head_gpu(st, wl, Z, gpu)
+    finally:
+        st.close()
+    want = O.head_from_outputs(Z, wl.targets, wl.weights)
+    err = normwise_err(z, want)
+    assert err <= TOL["bf16"], f"head (step path {step_path}) normwise error {err:.3e}"
+
+
 def test_head_after_forward_c2(gpu):
     import target_attention_jagged_b200 as S
     wl = make_config_workload("c2")

@@ -171,6 +171,25 @@ def test_run_host_matches_device(gpu):
         assert np.array_equal(Zh.numpy(), Zd)
 
 
+def test_run_host_chunked_matches_device(gpu):
+    """72,000 history rows: stca_run_host copies X in chunks on its own stream and
+    encodes each chunk as it lands; the result is bit for bit the device path's."""
+    import torch
+    import target_attention_jagged_b200 as S
+    from tests.gpu_helpers import storage_weights
+    wl = make_workload(lengths=[9000] * 8, targets=[2, 1, 3, 1, 2, 1, 1, 4], d=128, h=8, M=2, r=2,
+                       dtype="bf16", seed=17)
+    Zd = run_gpu(wl, gpu)
+    with S.Stca(storage_weights(wl), wl.d, wl.h, wl.r, wl.M, wl.dtype) as st:
+        Xh = torch.from_numpy(wl.storage(wl.X)).pin_memory()
+        th = torch.from_numpy(wl.storage(wl.targets)).pin_memory()
+        for _ in range(2):
+            Zh = torch.full((wl.T, wl.M, wl.d), float("nan"), dtype=torch.float32).pin_memory()
+            S.stca_run_host(st.handle, Xh, wl.offsets, th, wl.target_offsets, Zh)
+            assert np.array_equal(Zh.numpy(), Zd)
+        st.status()
+
+
 def test_forward_before_encode_and_bad_offsets(gpu):
     import torch
     import target_attention_jagged_b200 as S
