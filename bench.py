@@ -421,6 +421,22 @@ def measure_train_batch(S, torch, dev, stream, peaks, steps):
                                       "targets_per_s": wl.T / (step_ms / 1e3)}}
 
 
+def shard_workload(full, rank, world):
+    """Rank `rank`'s part of the batch `full`: whole requests, balanced by work
+    with the library's partitioner (target_attention_jagged_b200.shard)."""
+    import copy
+    from target_attention_jagged_b200.shard import partition_requests, request_work, shard_offsets
+    work = request_work(full.lengths, full.target_counts, full.d, full.h, full.M, full.r)
+    reqs = partition_requests(work, world)[rank]
+    x_rows, t_rows, off, toff = shard_offsets(full.offsets, full.target_offsets, reqs)
+    wl = copy.copy(full)
+    wl.lengths = full.lengths[reqs]
+    wl.target_counts = full.target_counts[reqs]
+    wl.offsets, wl.target_offsets = off, toff
+    wl.X, wl.targets = full.X[x_rows], full.targets[t_rows]
+    return wl
+
+
 def run_ours(args, rank, world, local_rank):
     import torch
     import torch.distributed as dist
@@ -429,7 +445,17 @@ def run_ours(args, rank, world, local_rank):
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
-    wl = make_config_workload(args.config, seed=CONFIGS[args.config]["seed"] + 1000 * rank)
+    if args.strong:
+        # strong scaling: every rank draws the same batch and keeps the requests
+        # the longest-processing-time partition gives it (no data-path collective)
+        full = make_config_workload(args.config, seed=CONFIGS[args.config]["seed"])
+        wl = shard_workload(full, rank, world)
+        batch_N, batch_T = full.N, full.T
+        cfg_wl = full
+    else:
+        wl = make_config_workload(args.config, seed=CONFIGS[args.config]["seed"] + 1000 * rank)
+        batch_N, batch_T = world * wl.N, world * wl.T
+        cfg_wl = wl
     c = counts(wl)
     peaks, peak_src = load_peaks()
     stream = torch.cuda.Stream(device=dev)
@@ -505,8 +531,8 @@ def run_ours(args, rank, world, local_rank):
     st.status(stream)
     elapsed_ms = max_over_ranks(local_ms, dev)
     sec = elapsed_ms / 1e3
-    value = world * wl.N * args.steps / sec
-    targets_per_s = world * wl.T * args.steps / sec
+    value = batch_N * args.steps / sec
+    targets_per_s = batch_T * args.steps / sec
     sustained = sec > 1.0
     rooflines = {k: roofline_of(k, kt, c, wl, peaks, sustained, args.steps, args.config) for k in kt}
     for r_ in rooflines.values():
@@ -582,7 +608,7 @@ def run_ours(args, rank, world, local_rank):
         head_roof = {"bound": "alu", "achieved": head_ach, "peak": head_peak, "unit": "TFLOP/s",
                      "frac": head_ach / head_peak, "flops_per_launch": c["head_flops"],
                      "peak_source": "nominal FP32 FFMA: 148 SMs x 128 lanes x 2 x 1.965 GHz"}
-    head = {"ms_per_head": head_ms, "targets_per_s": world * wl.T / (head_ms / 1e3),
+    head = {"ms_per_head": head_ms, "targets_per_s": batch_T / (head_ms / 1e3),
             "fused_in_last_step_ms": fused_head_ms,
             "kernel": "step_tc_kernel (head products only)" if head_tc else "head_kernel",
             "inputs": "Z and weights L2-resident (back-to-back calls)",
@@ -694,11 +720,11 @@ def run_ours(args, rank, world, local_rank):
     g1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(g0.elapsed_time(g1), dev)
-    e2e = {"value": world * wl.N * args.steps / (e2e_ms / 1e3), "unit": UNIT,
+    e2e = {"value": batch_N * args.steps / (e2e_ms / 1e3), "unit": UNIT,
            "h2d_bytes_per_step": int(Xh.numel() * Xh.element_size() + th.numel() * th.element_size()
                                      + 2 * 8 * (wl.R + 1)),
            "d2h_bytes_per_step": int(Zh.numel() * Zh.element_size()),
-           "targets_per_s": world * wl.T * args.steps / (e2e_ms / 1e3)}
+           "targets_per_s": batch_T * args.steps / (e2e_ms / 1e3)}
     st.close()
 
     if rank != 0:
@@ -706,17 +732,17 @@ def run_ours(args, rank, world, local_rank):
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": wl.dtype,
+        "scaling": "strong" if args.strong else "weak", "vs_baseline": None, "dtype": wl.dtype,
         "data": "synthetic (seeded N(0,1) embeddings, Xavier-uniform weights)",
-        "config": dict(workload_config(wl, world),
+        "config": dict(workload_config(cfg_wl, world),
                        attn_form="naive (Eq. 12)" if naive_used else "reordered (Eq. 13)"),
         "targets_per_s": targets_per_s,
         "roofline": roof, "roofline_step": step_roof,
         "kernels": {k: {"ms_total": v[0], "launches": v[1]} for k, v in kt.items()},
         "kernel_timing": "second pass of the same steps with CUDA events around every launch",
         "forward_only": {"ms_per_forward": fwd_ms,
-                         "targets_per_s": world * wl.T / (fwd_ms / 1e3),
-                         "history_tokens_per_s": world * wl.N / (fwd_ms / 1e3)},
+                         "targets_per_s": batch_T / (fwd_ms / 1e3),
+                         "history_tokens_per_s": batch_N / (fwd_ms / 1e3)},
         "head": head,
         "train_batch": train_batch,
         "backward": backward,
@@ -745,6 +771,9 @@ def main():
     ap.add_argument("--attn-kernel", type=int, default=None, choices=[0, 1],
                     help="tensor-core attention kernel (STCA_OPT_ATTN_KERNEL): 0 two-group, "
                          "1 split-softmax + combine; default: the library's choice")
+    ap.add_argument("--strong", action="store_true",
+                    help="strong scaling: one batch partitioned over the ranks by request "
+                         "(shard.partition_requests); default: weak, a full batch per rank")
     ap.add_argument("--no-backward", action="store_true", help="skip the backward measurement")
     ap.add_argument("--no-train-batch", action="store_true",
                     help="skip the sparse-training batch builder measurement")

@@ -781,8 +781,6 @@ static int build_plan(stca_handle* H, const int64_t* toff, int64_t T, int path, 
     return set_error(STCA_ECUDA, "plan event wait failed");
   if (bytes > H->plan_h_cap) {
     if (H->plan_h) cudaFreeHost(H->plan_h);
-  for (auto e : H->chunk_evt) cudaEventDestroy(e);
-  if (H->copy_stream) cudaStreamDestroy(H->copy_stream);
     H->plan_h = nullptr;
     H->plan_h_cap = 0;
     if (cudaMallocHost(&H->plan_h, bytes) != cudaSuccess) {
