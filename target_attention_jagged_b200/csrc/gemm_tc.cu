@@ -280,6 +280,9 @@ int tc_gemm_tf32(bool ta, bool tb, int64_t m, int64_t n, int64_t k, const float*
                  const float* B, int64_t ldb, float* C, int64_t ldc, float beta, float alpha, int batch,
                  int64_t sA, int64_t sB, int64_t sC, int num_sms, int* status, cudaStream_t s) {
   if (m <= 0 || n <= 0 || batch <= 0) return STCA_OK;
+  // TF32 operands must be K-major: the tensor core reads 32-bit types only in
+  // that layout (a transposed operand is declined here and runs elsewhere)
+  if (ta || !tb) return set_error(STCA_EINVAL, "tensor-core TF32 GEMM: operands must be K-major");
   if (!al16(A) || !al16(B) || !st16(lda) || !st16(ldb) || (batch > 1 && (!st16(sA) || !st16(sB))))
     return set_error(STCA_EINVAL, "tensor-core GEMM: operands not 16-byte aligned");
   if (m > INT32_MAX || n > INT32_MAX || k > INT32_MAX) return set_error(STCA_EINVAL, "tensor-core GEMM: too large");

@@ -100,7 +100,12 @@ def test_attention_backward_matches_oracle(gpu, dtype, d, h, layer, lengths, tar
         got_u, got_x = dU.cpu().numpy(), dX.cpu().numpy()
     want_u, want_x = B.attention_backward_batch(U, Xt, wl.offsets, wl.target_offsets, h, dC)
     tol = TOL[dtype]
-    assert normwise_err(got_u, want_u) <= tol, normwise_err(got_u, want_u)
+    # A request with a one-key history has dU = 0 exactly (a softmax over one key
+    # does not depend on u): those rows are held to the tensor's scale, since a
+    # rounding residue has no row scale to be relative to.
+    live = np.abs(want_u).max(axis=1) > 0
+    assert normwise_err(got_u[live], want_u[live]) <= tol, normwise_err(got_u[live], want_u[live])
+    assert np.abs(got_u[~live]).max(initial=0.0) <= tol * np.abs(want_u).max()
     keyrows = np.abs(want_x).max(axis=1) > 0               # rows of requests with targets
     assert normwise_err(got_x[keyrows], want_x[keyrows]) <= tol
     assert np.all(got_x[~keyrows] == 0)
