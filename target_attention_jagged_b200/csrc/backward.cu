@@ -23,6 +23,7 @@
 //    SwiGLUFFN([o(1) || ... || o(b) || x_t] W): d[o(1..b)], dx_t and the weights'
 //    gradients, the FFN forward recomputed.
 #include <cublasLt.h>
+#include <cuda_bf16.h>
 #include <math.h>
 
 #include <cmath>
@@ -266,7 +267,8 @@ constexpr int kLnMaxCols = 8;                  // d / 32, d <= 256
 
 __global__ void __launch_bounds__(256) ln_bwd_kernel(float* __restrict__ Y, const float* __restrict__ dXt,
                                                      const float* __restrict__ gamma, float* __restrict__ dgamma,
-                                                     float* __restrict__ dbeta, int64_t N, int d) {
+                                                     float* __restrict__ dbeta, int64_t N, int d,
+                                                     uint16_t* __restrict__ dy16 = nullptr) {
   __shared__ float sg[256], sb[256];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   for (int c = threadIdx.x; c < d; c += 256) sg[c] = sb[c] = 0.f;
@@ -317,7 +319,9 @@ __global__ void __launch_bounds__(256) ln_bwd_kernel(float* __restrict__ Y, cons
       const int c = lane + 32 * j;
       if (c >= d) continue;
       const float yh = (yv[j] - mu) * rstd, dyh = gv[j] * gamma[c];
-      y[c] = rstd * (dyh - m1 - yh * m2);
+      const float dy = rstd * (dyh - m1 - yh * m2);
+      y[c] = dy;
+      if (dy16) dy16[row * d + c] = __bfloat16_as_ushort(__float2bfloat16_rn(dy));
     }
   }
 #pragma unroll
@@ -332,6 +336,33 @@ __global__ void __launch_bounds__(256) ln_bwd_kernel(float* __restrict__ Y, cons
   for (int c = threadIdx.x; c < d; c += 256) {
     atomicAdd(&dgamma[c], sg[c]);
     atomicAdd(&dbeta[c], sb[c]);
+  }
+}
+
+// bf16 layouts of one SwiGLU FFN's weights for the tensor-core backward:
+//   W1i (2rd x d): rows 128 c + j hold column 64 c + j of W_u (j < 64) or
+//                  column 64 c + j - 64 of W_g: up and gate of 64 hidden units
+//                  per 128-row tile (the recomputation's B operand, K-major);
+//   WdT (d x rd) = W_d^T;  Wd16 (rd x d), Wu16, Wg16 (d x rd): row-major copies.
+__global__ void ffn_weights16_kernel(const float* __restrict__ Wu, const float* __restrict__ Wg,
+                                     const float* __restrict__ Wd, uint16_t* __restrict__ W1i,
+                                     uint16_t* __restrict__ WdT, uint16_t* __restrict__ Wd16,
+                                     uint16_t* __restrict__ Wu16, uint16_t* __restrict__ Wg16, int d, int rd) {
+  const int64_t n = static_cast<int64_t>(d) * rd;
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    auto bf = [](float f) { return __bfloat16_as_ushort(__float2bfloat16_rn(f)); };
+    // i = k * rd + hcol (row-major d x rd index of W_u / W_g)
+    const int64_t k = i / rd, hcol = i - k * rd;
+    const int64_t c = hcol / 64, j = hcol - c * 64;
+    W1i[(128 * c + j) * d + k] = bf(Wu[i]);
+    W1i[(128 * c + 64 + j) * d + k] = bf(Wg[i]);
+    Wu16[i] = bf(Wu[i]);
+    Wg16[i] = bf(Wg[i]);
+    // i as a row-major rd x d index of W_d: (h, nn)
+    const int64_t h = i / d, nn = i - h * d;
+    Wd16[i] = bf(Wd[i]);
+    WdT[nn * rd + h] = bf(Wd[i]);
   }
 }
 
@@ -459,6 +490,76 @@ using namespace stca;
 
 namespace {
 
+// The same backward for bf16 handles on the library's tensor-core GEMM, with
+// bf16 intermediates: [A | G] = X [W_u | W_g] with H = A SiLU(G) formed in the
+// GEMM's epilogue; Y = H W_d; the LayerNorm derivative (dy, also as bf16);
+// dW_d = H^T dy; dH = dy W_d^T with the SwiGLU derivative in the epilogue
+// (dA, dG over A, G); dW_u = X^T dA, dW_g = X^T dG; dX = dA W_u^T + dG W_g^T.
+// Products with K = N (the weight gradients) split K over CTAs.
+int ffn_ln_backward16(stca_handle* H, const uint16_t* X, int64_t N, const float* dXt, float* dX,
+                      const float* Wu, const float* Wg, const float* Wd, const float* gamma, float* dWu,
+                      float* dWg, float* dWd, float* dgamma, float* dbeta, cudaStream_t s) {
+  const int d = H->d, rd = H->rd;
+  const size_t nd = static_cast<size_t>(N) * d, nr = static_cast<size_t>(N) * rd;
+  const size_t wn = static_cast<size_t>(d) * rd;
+  // workspace: A16, G16, H16 (N rd bf16), dy16 (N d bf16), Y (N d fp32), weights (5 d rd bf16)
+  auto a256 = [](size_t x) { return (x + 255) & ~size_t(255); };
+  const size_t oA = 0, oG = a256(oA + nr * 2), oH = a256(oG + nr * 2), oDy = a256(oH + nr * 2);
+  const size_t oY = a256(oDy + nd * 2), oW = a256(oY + nd * 4), total = a256(oW + 6 * wn * 2);
+  if (int rc = ensure(&H->bw_ws, &H->bw_ws_cap, total)) return rc;
+  char* w = static_cast<char*>(H->bw_ws);
+  uint16_t* A16 = reinterpret_cast<uint16_t*>(w + oA);
+  uint16_t* G16 = reinterpret_cast<uint16_t*>(w + oG);
+  uint16_t* H16 = reinterpret_cast<uint16_t*>(w + oH);
+  uint16_t* dy16 = reinterpret_cast<uint16_t*>(w + oDy);
+  float* Y = reinterpret_cast<float*>(w + oY);
+  uint16_t* W1i = reinterpret_cast<uint16_t*>(w + oW);      // 2 wn
+  uint16_t* WdT = W1i + 2 * wn;
+  uint16_t* Wd16 = WdT + wn;
+  uint16_t* Wu16 = Wd16 + wn;
+  uint16_t* Wg16 = Wu16 + wn;
+  ffn_weights16_kernel<<<grid_for(static_cast<int64_t>(wn)), 256, 0, s>>>(Wu, Wg, Wd, W1i, WdT, Wd16, Wu16, Wg16, d, rd);
+  STCA_CUDA_TRY(cudaGetLastError());
+  const int ns = H->num_sms;
+  int* st = H->status_d;
+  // forward recomputation
+  if (int rc = tc_gemm_bf16(false, true, N, 2 * rd, d, X, d, W1i, d, nullptr, 0, 0.f, 1, A16, G16, H16, rd, ns, st, s))
+    return rc;
+  if (int rc = tc_gemm_bf16(false, true, N, d, rd, H16, rd, WdT, rd, Y, d, 0.f, 0, nullptr, nullptr, nullptr, 0, ns, st, s))
+    return rc;
+  // LayerNorm: Y <- dy (also dy16); dgamma, dbeta
+  STCA_CUDA_TRY(cudaMemsetAsync(dgamma, 0, d * sizeof(float), s));
+  STCA_CUDA_TRY(cudaMemsetAsync(dbeta, 0, d * sizeof(float), s));
+  ln_bwd_kernel<<<static_cast<unsigned>((N + kLnRows - 1) / kLnRows), 256, 0, s>>>(Y, dXt, gamma, dgamma,
+                                                                                   dbeta, N, d, dy16);
+  STCA_CUDA_TRY(cudaGetLastError());
+  // dW_d = H^T dy
+  if (int rc = tc_gemm_bf16(true, false, rd, d, N, H16, rd, dy16, d, dWd, d, 0.f, 0, nullptr, nullptr, nullptr, 0,
+                            ns, st, s))
+    return rc;
+  // dH = dy W_d^T, then dA, dG over A16, G16
+  if (int rc = tc_gemm_bf16(false, true, N, rd, d, dy16, d, Wd16, d, nullptr, 0, 0.f, 2, A16, G16, nullptr, rd,
+                            ns, st, s))
+    return rc;
+  // dW_u = X^T dA, dW_g = X^T dG
+  if (int rc = tc_gemm_bf16(true, false, d, rd, N, X, d, A16, rd, dWu, rd, 0.f, 0, nullptr, nullptr, nullptr, 0,
+                            ns, st, s))
+    return rc;
+  if (int rc = tc_gemm_bf16(true, false, d, rd, N, X, d, G16, rd, dWg, rd, 0.f, 0, nullptr, nullptr, nullptr, 0,
+                            ns, st, s))
+    return rc;
+  if (dX) {
+    if (int rc = tc_gemm_bf16(false, true, N, d, rd, A16, rd, Wu16, rd, dX, d, 0.f, 0, nullptr, nullptr, nullptr,
+                              0, ns, st, s))
+      return rc;
+    if (int rc = tc_gemm_bf16(false, true, N, d, rd, G16, rd, Wg16, rd, dX, d, 1.f, 0, nullptr, nullptr, nullptr,
+                              0, ns, st, s))
+      return rc;
+  }
+  set_error(STCA_OK, "");
+  return STCA_OK;
+}
+
 // Backward of Y = LN(((X W_u) * SiLU(X W_g)) W_d) with LN's scale gamma, for N
 // rows of X (handle dtype): the history encoding of Eqs. (1)-(2) and, with the
 // query weights, the query init of Eq. (3).  dX may be NULL.
@@ -467,6 +568,10 @@ int ffn_ln_backward(stca_handle* H, const void* X, int64_t N, const float* dXt, 
                     float* dWg, float* dWd, float* dgamma, float* dbeta, cudaStream_t s) {
   const int d = H->d, rd = H->rd;
   if (d > 32 * kLnMaxCols) return set_error(STCA_EINVAL, "encoder backward needs d <= 256");
+  // bf16 handles: the tensor-core pipeline, where its tiles fit the sizes
+  if (H->elem == 2 && H->opt_bw_gemm != 1 && d % 64 == 0 && rd % 128 == 0 && N <= INT32_MAX)
+    return ffn_ln_backward16(H, static_cast<const uint16_t*>(X), N, dXt, dX, Wu, Wg, Wd, gamma, dWu, dWg, dWd,
+                             dgamma, dbeta, s);
   // workspace: Xf (N d), A (N rd), G (N rd), Hh (N rd), Y (N d)
   const size_t nd = static_cast<size_t>(N) * d, nr = static_cast<size_t>(N) * rd;
   if (int rc = ensure(&H->bw_ws, &H->bw_ws_cap, (2 * nd + 3 * nr) * sizeof(float))) return rc;

@@ -226,6 +226,235 @@ gemm_tf32_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
   }
 }
 
+// ---------------------------------------------------------------- bf16 operands
+// The same GEMM with bf16 operands (tcgen05.mma.kind::f16), which the tensor
+// core reads K-major or MN-major alike: a stage holds K = 64 (one 128-byte row
+// of 64 bf16), one MMA is K = 16.  MN-major operands arrive as [64 k x 64 mn]
+// boxes (8 KB) side by side.  Three epilogues:
+//   kEpiStore   C (fp32) = alpha acc + beta C, or atomic adds under split K;
+//   kEpiSwigluF the 128 columns of a tile are the up and gate projections of
+//               64 hidden units (the weight's rows interleaved per 64): writes
+//               A, G and H = A SiLU(G) as bf16 at hidden columns 64 tn ..;
+//   kEpiSwigluB acc is dH for hidden columns 128 tn ..: reads A and G there
+//               (bf16) and writes dA = dH SiLU(G) over A and
+//               dG = dH A SiLU'(G) over G.
+enum : int { kEpiStore = 0, kEpiSwigluF = 1, kEpiSwigluB = 2 };
+
+struct Gemm16Args {
+  int64_t m, n, k;
+  int tiles_m, tiles_n, ksplit;
+  int64_t k_per_split;          // multiple of 64
+  float* C;
+  int64_t ldc;
+  float alpha, beta;
+  int atomic;
+  uint16_t *A16, *G16, *H16;    // SwiGLU epilogues: N x rd bf16 (ld = ld16)
+  int64_t ld16;
+  int* status;
+};
+
+constexpr uint32_t kA16Stage = 128u * 128u;     // [128 x 64] bf16
+
+__device__ __forceinline__ float sigmoid_f(float z) { return 1.0f / (1.0f + __expf(-z)); }
+
+template <int BN, bool AMN, bool BMN, int EPI>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                 const Gemm16Args g) {
+  constexpr uint32_t kBStage = BN * 128u;
+  constexpr uint32_t kStage = kA16Stage + kBStage;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  if (smem_u32(smem_raw) & 1023u) {
+    if (threadIdx.x == 0) atomicOr(g.status, kStatusStepTimeout);
+    return;
+  }
+  uint8_t* sm = smem_raw;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sm + kGemmStages * kStage);
+  uint64_t* empty = full + kGemmStages;
+  uint64_t* accfull = empty + kGemmStages;
+  uint64_t* mdrain = accfull + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mdrain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  int u = blockIdx.x;
+  const int ks = u % g.ksplit; u /= g.ksplit;
+  const int tn = u % g.tiles_n; u /= g.tiles_n;
+  const int tm = u;
+  const int64_t m0 = static_cast<int64_t>(tm) * 128, n0 = static_cast<int64_t>(tn) * BN;
+  const int64_t k0 = ks * g.k_per_split, k1 = min(g.k, k0 + g.k_per_split);
+  const int nst = static_cast<int>((k1 - k0 + 63) / 64);
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kGemmStages; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
+    mbar_init(accfull, 1);
+    mbar_init(mdrain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tmA);
+    prefetch_tmap(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, BN);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t sbase = smem_u32(sm);
+
+  if (warp == 0) {
+    if (lane == 0) {
+      bool ok = true;
+      int st = 0;
+      for (; ok && st < nst; ++st) {
+        const int s = st % kGemmStages;
+        if (!(ok = gwait(&empty[s], ((st / kGemmStages) & 1) ^ 1, abort_flag, g.status))) break;
+        mbar_arrive_expect_tx(&full[s], kStage);
+        uint8_t* a = sm + s * kStage;
+        uint8_t* bb = a + kA16Stage;
+        const int kk = static_cast<int>(k0 + 64 * st);
+        if constexpr (AMN) {
+          for (int i = 0; i < 2; ++i) tma_load_2d(a + i * 8192, &tmA, static_cast<int>(m0) + 64 * i, kk, &full[s]);
+        } else {
+          tma_load_2d(a, &tmA, kk, static_cast<int>(m0), &full[s]);
+        }
+        if constexpr (BMN) {
+          for (int i = 0; i < BN / 64; ++i)
+            tma_load_2d(bb + i * 8192, &tmB, static_cast<int>(n0) + 64 * i, kk, &full[s]);
+        } else {
+          tma_load_2d(bb, &tmB, kk, static_cast<int>(n0), &full[s]);
+        }
+      }
+      for (int c = st > kGemmStages ? st - kGemmStages : 0; c < st; ++c)
+        gdrain(&full[c % kGemmStages], (c / kGemmStages) & 1, 100000000ull);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16(128, BN, AMN, BMN);
+      bool ok = true;
+      for (int st = 0; st < nst; ++st) {
+        const int s = st % kGemmStages;
+        if (!(ok = gwait(&full[s], (st / kGemmStages) & 1, abort_flag, g.status))) break;
+        tc_fence_after();
+        const uint32_t a = sbase + s * kStage, bb = a + kA16Stage;
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {          // K = 16 per MMA
+          const uint64_t ad = AMN ? sdesc_sw128(a + kk * 2048, 8192, 1024) : sdesc_sw128(a + kk * 32, 16, 1024);
+          const uint64_t bd = BMN ? sdesc_sw128(bb + kk * 2048, 8192, 1024) : sdesc_sw128(bb + kk * 32, 16, 1024);
+          mma_bf16_ss(tmem, ad, bd, idesc, (st | kk) != 0);
+        }
+        mma_commit(&empty[s]);
+      }
+      if (ok) mma_commit(accfull);
+      mma_commit(mdrain);
+      gdrain(mdrain, 0, 500000000ull);
+    }
+  } else {
+    const int q = warp & 3;
+    const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
+    const int64_t row = m0 + q * 32 + lane;
+    const bool ok = __all_sync(0xffffffffu, nst == 0 || gwait(accfull, 0, abort_flag, g.status)) != 0;
+    if (ok && nst > 0) {
+      tc_fence_after();
+      if constexpr (EPI == kEpiStore) {
+        float* crow = g.C + row * g.ldc;
+#pragma unroll 1
+        for (int c = 0; c < BN / 32; ++c) {
+          uint32_t v[32];
+          tmem_ld32(tmem + lane_off + 32 * c, v);
+          tmem_ld_wait();
+          if (row < g.m) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              const int64_t col = n0 + 32 * c + j;
+              if (col < g.n) {
+                const float x = g.alpha * __uint_as_float(v[j]);
+                if (g.atomic) atomicAdd(crow + col, x);
+                else crow[col] = g.beta != 0.f ? fmaf(g.beta, crow[col], x) : x;
+              }
+            }
+          }
+        }
+      } else if constexpr (EPI == kEpiSwigluF) {
+        // columns 0..63: up projection of hidden units 64 tn .. +63; 64..127: gate
+#pragma unroll 1
+        for (int c = 0; c < 2; ++c) {
+          uint32_t va[32], vg[32];
+          tmem_ld32(tmem + lane_off + 32 * c, va);
+          tmem_ld32(tmem + lane_off + 64 + 32 * c, vg);
+          tmem_ld_wait();
+          if (row < g.m) {
+            const int64_t col = static_cast<int64_t>(tn) * 64 + 32 * c;
+            uint4* pa = reinterpret_cast<uint4*>(g.A16 + row * g.ld16 + col);
+            uint4* pg = reinterpret_cast<uint4*>(g.G16 + row * g.ld16 + col);
+            uint4* ph = reinterpret_cast<uint4*>(g.H16 + row * g.ld16 + col);
+#pragma unroll
+            for (int j8 = 0; j8 < 4; ++j8) {
+              uint32_t wa[4], wg[4], wh[4];
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const float a0 = __uint_as_float(va[8 * j8 + 2 * e]), a1 = __uint_as_float(va[8 * j8 + 2 * e + 1]);
+                const float g0 = __uint_as_float(vg[8 * j8 + 2 * e]), g1 = __uint_as_float(vg[8 * j8 + 2 * e + 1]);
+                wa[e] = pack_bf16x2(a0, a1);
+                wg[e] = pack_bf16x2(g0, g1);
+                wh[e] = pack_bf16x2(a0 * g0 * sigmoid_f(g0), a1 * g1 * sigmoid_f(g1));
+              }
+              pa[j8] = make_uint4(wa[0], wa[1], wa[2], wa[3]);
+              pg[j8] = make_uint4(wg[0], wg[1], wg[2], wg[3]);
+              ph[j8] = make_uint4(wh[0], wh[1], wh[2], wh[3]);
+            }
+          }
+        }
+      } else {
+        // dH of hidden columns n0 .. n0 + BN - 1
+#pragma unroll 1
+        for (int c = 0; c < BN / 32; ++c) {
+          uint32_t v[32];
+          tmem_ld32(tmem + lane_off + 32 * c, v);
+          tmem_ld_wait();
+          if (row < g.m) {
+            const int64_t col = n0 + 32 * c;
+            uint4* pa = reinterpret_cast<uint4*>(g.A16 + row * g.ld16 + col);
+            uint4* pg = reinterpret_cast<uint4*>(g.G16 + row * g.ld16 + col);
+#pragma unroll
+            for (int j8 = 0; j8 < 4; ++j8) {
+              const uint4 av = pa[j8], gv = pg[j8];
+              const uint32_t aw[4] = {av.x, av.y, av.z, av.w}, gw[4] = {gv.x, gv.y, gv.z, gv.w};
+              uint32_t da[4], dg[4];
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                float outa[2], outg[2];
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                  const float a = __uint_as_float(hh ? (aw[e] & 0xFFFF0000u) : (aw[e] << 16));
+                  const float gg = __uint_as_float(hh ? (gw[e] & 0xFFFF0000u) : (gw[e] << 16));
+                  const float dh = __uint_as_float(v[8 * j8 + 2 * e + hh]);
+                  const float sg = sigmoid_f(gg);
+                  outa[hh] = dh * gg * sg;
+                  outg[hh] = dh * a * sg * (1.f + gg * (1.f - sg));
+                }
+                da[e] = pack_bf16x2(outa[0], outa[1]);
+                dg[e] = pack_bf16x2(outg[0], outg[1]);
+              }
+              pa[j8] = make_uint4(da[0], da[1], da[2], da[3]);
+              pg[j8] = make_uint4(dg[0], dg[1], dg[2], dg[3]);
+            }
+          }
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, BN);
+  }
+}
+
 // 128-bit alignment of an address and of a stride in elements.
 bool al16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 bool st16(int64_t elems) { return ((elems * 4) & 15) == 0; }
@@ -333,6 +562,86 @@ int tc_gemm_tf32(bool ta, bool tb, int64_t m, int64_t n, int64_t k, const float*
     case 128: return launch_gemm_bn<128>(amn, bmn, tmA, tmB, g, units, s);
     case 64: return launch_gemm_bn<64>(amn, bmn, tmA, tmB, g, units, s);
     default: return launch_gemm_bn<32>(amn, bmn, tmA, tmB, g, units, s);
+  }
+}
+
+
+namespace {
+// bf16 operand map: stored row-major `rows` x `inner` with row stride ld
+// (elements), box bx x by.
+int map16(CUtensorMap* m, const uint16_t* base, int64_t inner, int64_t rows, int64_t ld, uint32_t bx, uint32_t by) {
+  return make_tmap_bf16_2d_strided(m, base, static_cast<uint64_t>(inner), static_cast<uint64_t>(rows),
+                                   static_cast<uint64_t>(ld) * 2, bx, by);
+}
+
+template <int BN, int EPI>
+int launch16(bool amn, bool bmn, const CUtensorMap& tmA, const CUtensorMap& tmB, const Gemm16Args& g,
+             int64_t units, cudaStream_t s) {
+  const uint32_t smem = kGemmStages * (kA16Stage + BN * 128u) + (2 * kGemmStages + 2) * 8 + 16;
+  auto go = [&](auto kf) -> int {
+    cudaError_t e = cudaFuncSetAttribute(kf, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return set_error(STCA_ECUDA, std::string("gemm_bf16 smem: ") + cudaGetErrorString(e));
+    kf<<<static_cast<unsigned>(units), kGemmThreads, smem, s>>>(tmA, tmB, g);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return set_error(STCA_ECUDA, std::string("gemm_bf16 launch: ") + cudaGetErrorString(e));
+    return STCA_OK;
+  };
+  if (amn && bmn) return go(gemm_bf16_kernel<BN, true, true, EPI>);
+  if (amn) return go(gemm_bf16_kernel<BN, true, false, EPI>);
+  if (bmn) return go(gemm_bf16_kernel<BN, false, true, EPI>);
+  return go(gemm_bf16_kernel<BN, false, false, EPI>);
+}
+}  // namespace
+
+int tc_gemm_bf16(bool ta, bool tb, int64_t m, int64_t n, int64_t k, const uint16_t* A, int64_t lda,
+                 const uint16_t* B, int64_t ldb, float* C, int64_t ldc, float beta, int epi, uint16_t* A16,
+                 uint16_t* G16, uint16_t* H16, int64_t ld16, int num_sms, int* status, cudaStream_t s) {
+  if (m <= 0 || n <= 0) return STCA_OK;
+  auto al = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; };
+  if (!al(A) || !al(B) || (lda * 2) % 16 || (ldb * 2) % 16)
+    return set_error(STCA_EINVAL, "bf16 tensor-core GEMM: operands not 16-byte aligned");
+  const bool amn = ta, bmn = !tb;
+  const int BN = (epi != kEpiStore || n > 64) ? 128 : 64;
+  if (epi != kEpiStore && (n % 128 || !A16 || !G16 || (epi == kEpiSwigluF && !H16)))
+    return set_error(STCA_EINVAL, "bf16 tensor-core GEMM: SwiGLU epilogue needs whole 128-column tiles");
+  Gemm16Args g{};
+  g.m = m;
+  g.n = n;
+  g.k = k;
+  g.tiles_m = static_cast<int>((m + 127) / 128);
+  g.tiles_n = static_cast<int>((n + BN - 1) / BN);
+  g.C = C;
+  g.ldc = ldc;
+  g.alpha = 1.f;
+  g.beta = beta;
+  g.A16 = A16;
+  g.G16 = G16;
+  g.H16 = H16;
+  g.ld16 = ld16;
+  g.status = status;
+  const int64_t tiles = static_cast<int64_t>(g.tiles_m) * g.tiles_n;
+  int ksplit = 1;
+  if (epi == kEpiStore && k >= 4096 && tiles < num_sms)
+    ksplit = static_cast<int>(std::min<int64_t>(num_sms / tiles, (k + 2047) / 2048));
+  ksplit = std::max(ksplit, 1);
+  g.k_per_split = ((k + ksplit - 1) / ksplit + 63) / 64 * 64;
+  g.ksplit = static_cast<int>(std::max<int64_t>(1, (k + g.k_per_split - 1) / g.k_per_split));
+  g.atomic = g.ksplit > 1;
+  CUtensorMap tmA, tmB;
+  if (map16(&tmA, A, amn ? m : k, amn ? k : m, lda, 64, amn ? 64u : 128u) ||
+      map16(&tmB, B, bmn ? n : k, bmn ? k : n, ldb, 64, bmn ? 64u : static_cast<uint32_t>(BN)))
+    return set_error(STCA_EINVAL, "bf16 tensor-core GEMM: operand layout not expressible as a tensor map");
+  if (g.atomic) {
+    if (beta == 0.f) STCA_CUDA_TRY(cudaMemset2DAsync(C, ldc * 4, 0, n * 4, m, s));
+    else if (beta != 1.f) return set_error(STCA_EINVAL, "bf16 tensor-core GEMM: split K needs beta 0 or 1");
+  }
+  const int64_t units = tiles * g.ksplit;
+  if (units > INT32_MAX) return set_error(STCA_EINVAL, "bf16 tensor-core GEMM: too many tiles");
+  if (BN == 64) return launch16<64, kEpiStore>(amn, bmn, tmA, tmB, g, units, s);
+  switch (epi) {
+    case kEpiSwigluF: return launch16<128, kEpiSwigluF>(amn, bmn, tmA, tmB, g, units, s);
+    case kEpiSwigluB: return launch16<128, kEpiSwigluB>(amn, bmn, tmA, tmB, g, units, s);
+    default: return launch16<128, kEpiStore>(amn, bmn, tmA, tmB, g, units, s);
   }
 }
 

@@ -134,7 +134,11 @@ def test_attention_layer_chain(gpu, dtype, d, h, layer):
     tol = TOL[dtype]
     for k, want in (("dWv", w_dWv), ("dWo", w_dWo), ("dWq", w_dWq), ("dWk", w_dWk)):
         assert _rel(got[k], want) <= tol, (k, _rel(got[k], want))
-    assert normwise_err(got["dQ"], w_dQ) <= tol
+    # targets of the one-key request have dQ = 0 exactly (their dU is zero): those
+    # rows are held to the tensor's scale, the others per row
+    live = np.abs(w_dQ).max(axis=1) > 0
+    assert normwise_err(got["dQ"][live], w_dQ[live]) <= tol
+    assert np.abs(got["dQ"][~live]).max(initial=0.0) <= tol * np.abs(w_dQ).max()
     keyrows = np.abs(w_dX).max(axis=1) > 0
     assert normwise_err(got["dX"][keyrows], w_dX[keyrows]) <= tol
     assert np.all(got["dX"][~keyrows] == 0)
