@@ -126,42 +126,57 @@ __device__ __forceinline__ void st_tmem32(uint32_t taddr, const uint32_t (&r)[32
 
 // The last warp to arrive on a split pair's slot merges the slot's rows (lane
 // quarter q: rows 32 q .. 32 q + 31; column half b) of all the pair's items:
-// c = sum_w 2^(m_w - m) acc_w / sum_w 2^(m_w - m) l_w, m = max_w m_w.  Lanes
-// cover float4 columns of one or more rows at a time, so the partial rows are
-// read coalesced (from L2: other CTAs wrote them).
+// c = sum_w 2^(m_w - m) acc_w / sum_w 2^(m_w - m) l_w, m = max_w m_w.  Lane r
+// takes row 32 q + r: first the items' (m, l) -- a running maximum and sum --
+// then, item by item, all D / 8 float4 of its half row at once, so each item
+// costs one round trip to L2 (other CTAs wrote the partials; the merge runs
+// at the tail of the kernel, where latency is what counts).
 template <int D>
 __device__ __forceinline__ void merge_slot(const PPParams& p, const AttnItem& item, int b, int q,
                                            int lane) {
-  constexpr int kChunks = D / 8;              // float4 chunks in a half row
-  constexpr int kRowsPer = 32 / kChunks;      // rows per warp step
+  constexpr int kC4 = D / 8;                  // float4 of a half row
+  const int row = q * 32 + lane;
+  if (row >= item.rows) return;               // the items of a pair share its rows
   const int w0 = p.pair_item_begin[item.pair], w1 = p.pair_item_begin[item.pair + 1];
-  const int c4 = lane % kChunks, rsub = lane / kChunks;
-  for (int rr = 0; rr < 32; rr += kRowsPer) {
-    const int row = q * 32 + rr + rsub;
-    if (row >= item.rows) break;             // the items of a pair share its rows
-    float mx = -INFINITY;
-    for (int w = w0; w < w1; ++w)
-      mx = fmaxf(mx, __ldcg(p.pml + (p.items[w].row_base + row) * 4 + b));
-    float L = 0.f;
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int w = w0; w < w1; ++w) {
-      const int64_t g = p.items[w].row_base + row;
-      const float f = sx::ex2(__ldcg(p.pml + g * 4 + b) - mx);
-      L = fmaf(f, __ldcg(p.pml + g * 4 + 2 + b), L);
-      const float4 v = __ldcg(reinterpret_cast<const float4*>(p.pacc + g * D + b * (D / 2)) + c4);
-      acc.x = fmaf(f, v.x, acc.x);
-      acc.y = fmaf(f, v.y, acc.y);
-      acc.z = fmaf(f, v.z, acc.z);
-      acc.w = fmaf(f, v.w, acc.w);
+  float mx = -INFINITY, L = 0.f;
+#pragma unroll 4
+  for (int w = w0; w < w1; ++w) {
+    const int64_t g = p.items[w].row_base + row;
+    const float mw = __ldcg(p.pml + g * 4 + b), lw = __ldcg(p.pml + g * 4 + 2 + b);
+    if (mw > mx) {
+      L = L * sx::ex2(mx - mw) + lw;           // 0 from mx = -inf
+      mx = mw;
+    } else {
+      L = fmaf(lw, sx::ex2(mw - mx), L);
     }
-    const float inv = 1.f / L;
-    if (p.stats && b == 0 && c4 == 0) {
-      p.stats[(item.qrow0 + row) * 2] = mx;
-      p.stats[(item.qrow0 + row) * 2 + 1] = L;
-    }
-    reinterpret_cast<float4*>(p.cout + (item.qrow0 + row) * D + b * (D / 2))[c4] =
-        make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
   }
+  const float inv = 1.f / L;
+  if (p.stats && b == 0) {
+    p.stats[(item.qrow0 + row) * 2] = mx;
+    p.stats[(item.qrow0 + row) * 2 + 1] = L;
+  }
+  float4 acc[kC4];
+#pragma unroll
+  for (int c = 0; c < kC4; ++c) acc[c] = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 1
+  for (int w = w0; w < w1; ++w) {
+    const int64_t g = p.items[w].row_base + row;
+    const float f = sx::ex2(__ldcg(p.pml + g * 4 + b) - mx) * inv;
+    const float4* src = reinterpret_cast<const float4*>(p.pacc + g * D + b * (D / 2));
+    float4 v[kC4];
+#pragma unroll
+    for (int c = 0; c < kC4; ++c) v[c] = __ldcg(src + c);
+#pragma unroll
+    for (int c = 0; c < kC4; ++c) {
+      acc[c].x = fmaf(f, v[c].x, acc[c].x);
+      acc[c].y = fmaf(f, v[c].y, acc[c].y);
+      acc[c].z = fmaf(f, v[c].z, acc[c].z);
+      acc[c].w = fmaf(f, v[c].w, acc[c].w);
+    }
+  }
+  float4* dst = reinterpret_cast<float4*>(p.cout + (item.qrow0 + row) * D + b * (D / 2));
+#pragma unroll
+  for (int c = 0; c < kC4; ++c) dst[c] = acc[c];
 }
 
 // FMA_PAIRS of every 4 consecutive pairs of a row's exponentials go to the

@@ -192,27 +192,37 @@ gemm_tf32_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
       gdrain(mdrain, 0, 500000000ull);
     }
   } else {
+    // epilogue: rows staged in the pipeline's (now free) shared memory, lane =
+    // row, then written row by row with the whole warp (coalesced)
     const int q = warp & 3;
     const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
-    const int64_t row = m0 + q * 32 + lane;
     const bool ok = __all_sync(0xffffffffu, nst == 0 || gwait(accfull, 0, abort_flag, g.status)) != 0;
     if (ok && nst > 0) {
       tc_fence_after();
-      float* crow = g.C + static_cast<int64_t>(b) * g.sC + row * g.ldc;
+      constexpr int kLd = BN + 4;
+      float* stg = reinterpret_cast<float*>(sm) + q * 32 * kLd;
 #pragma unroll 1
-      for (int c = 0; c < (BN + 31) / 32; ++c) {
+      for (int c = 0; c < BN / 32; ++c) {
         uint32_t v[32];
         tmem_ld32(tmem + lane_off + 32 * c, v);
         tmem_ld_wait();
-        if (row < g.m) {
+        float4* d4 = reinterpret_cast<float4*>(stg + lane * kLd + 32 * c);
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const int64_t col = n0 + 32 * c + j;
-            if (col < g.n) {
-              const float x = g.alpha * __uint_as_float(v[j]);
-              if (g.atomic) atomicAdd(crow + col, x);
-              else crow[col] = g.beta != 0.f ? fmaf(g.beta, crow[col], x) : x;
-            }
+        for (int j = 0; j < 8; ++j)
+          d4[j] = make_float4(g.alpha * __uint_as_float(v[4 * j]), g.alpha * __uint_as_float(v[4 * j + 1]),
+                              g.alpha * __uint_as_float(v[4 * j + 2]), g.alpha * __uint_as_float(v[4 * j + 3]));
+      }
+      __syncwarp();
+      for (int rr = 0; rr < 32; ++rr) {
+        const int64_t row = m0 + q * 32 + rr;
+        if (row >= g.m) break;
+        float* crow = g.C + static_cast<int64_t>(b) * g.sC + row * g.ldc;
+        for (int cc = lane; cc < BN; cc += 32) {
+          const int64_t col = n0 + cc;
+          if (col < g.n) {
+            const float x = stg[rr * kLd + cc];
+            if (g.atomic) atomicAdd(crow + col, x);
+            else crow[col] = g.beta != 0.f ? fmaf(g.beta, crow[col], x) : x;
           }
         }
       }
@@ -353,95 +363,167 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
       gdrain(mdrain, 0, 500000000ull);
     }
   } else {
+    // Epilogue: each warp takes TMEM lane quarter q, rows m0 + 32 q .. + 31.  The
+    // pipeline's shared memory is free once every product is done; a warp stages
+    // its 32 rows there (lane = row) and then writes them row by row with the
+    // whole warp, so global accesses are coalesced.
     const int q = warp & 3;
     const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
-    const int64_t row = m0 + q * 32 + lane;
     const bool ok = __all_sync(0xffffffffu, nst == 0 || gwait(accfull, 0, abort_flag, g.status)) != 0;
     if (ok && nst > 0) {
       tc_fence_after();
+      const int64_t rbase = m0 + q * 32;
       if constexpr (EPI == kEpiStore) {
-        float* crow = g.C + row * g.ldc;
+        constexpr int kLd = BN + 4;                       // floats per staged row
+        float* stg = reinterpret_cast<float*>(sm) + q * 32 * kLd;
 #pragma unroll 1
         for (int c = 0; c < BN / 32; ++c) {
           uint32_t v[32];
           tmem_ld32(tmem + lane_off + 32 * c, v);
           tmem_ld_wait();
-          if (row < g.m) {
+          float4* d4 = reinterpret_cast<float4*>(stg + lane * kLd + 32 * c);
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              const int64_t col = n0 + 32 * c + j;
-              if (col < g.n) {
-                const float x = g.alpha * __uint_as_float(v[j]);
-                if (g.atomic) atomicAdd(crow + col, x);
-                else crow[col] = g.beta != 0.f ? fmaf(g.beta, crow[col], x) : x;
+          for (int j = 0; j < 8; ++j)
+            d4[j] = make_float4(g.alpha * __uint_as_float(v[4 * j]), g.alpha * __uint_as_float(v[4 * j + 1]),
+                                g.alpha * __uint_as_float(v[4 * j + 2]), g.alpha * __uint_as_float(v[4 * j + 3]));
+        }
+        __syncwarp();
+        const bool vec = (g.ldc & 3) == 0 && (reinterpret_cast<uintptr_t>(g.C) & 15) == 0;
+        for (int rr = 0; rr < 32; ++rr) {
+          const int64_t row = rbase + rr;
+          if (row >= g.m) break;
+          float* crow = g.C + row * g.ldc;
+          for (int c4 = lane; c4 < BN / 4; c4 += 32) {
+            const int64_t col = n0 + 4 * c4;
+            const float4 x = reinterpret_cast<const float4*>(stg + rr * kLd)[c4];
+            if (vec && col + 3 < g.n) {
+              if (g.atomic) {
+                asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(crow + col), "f"(x.x),
+                             "f"(x.y), "f"(x.z), "f"(x.w)
+                             : "memory");
+              } else {
+                float4 y = x;
+                if (g.beta != 0.f) {
+                  const float4 o = *reinterpret_cast<const float4*>(crow + col);
+                  y = make_float4(fmaf(g.beta, o.x, x.x), fmaf(g.beta, o.y, x.y), fmaf(g.beta, o.z, x.z),
+                                  fmaf(g.beta, o.w, x.w));
+                }
+                *reinterpret_cast<float4*>(crow + col) = y;
               }
+            } else {
+              const float xs[4] = {x.x, x.y, x.z, x.w};
+              for (int e = 0; e < 4; ++e)
+                if (col + e < g.n) {
+                  if (g.atomic) atomicAdd(crow + col + e, xs[e]);
+                  else crow[col + e] = g.beta != 0.f ? fmaf(g.beta, crow[col + e], xs[e]) : xs[e];
+                }
             }
           }
         }
       } else if constexpr (EPI == kEpiSwigluF) {
-        // columns 0..63: up projection of hidden units 64 tn .. +63; 64..127: gate
+        // columns 0..63: up projection of hidden units 64 tn .. +63; 64..127: gate.
+        // Staged rows: A, G, H of this warp's rows, 64 bf16 (+ 8 pad) each.
+        constexpr int kLd = 72;
+        uint16_t* sA = reinterpret_cast<uint16_t*>(sm) + q * 3 * 32 * kLd;
+        uint16_t* sG = sA + 32 * kLd;
+        uint16_t* sH = sG + 32 * kLd;
 #pragma unroll 1
         for (int c = 0; c < 2; ++c) {
           uint32_t va[32], vg[32];
           tmem_ld32(tmem + lane_off + 32 * c, va);
           tmem_ld32(tmem + lane_off + 64 + 32 * c, vg);
           tmem_ld_wait();
-          if (row < g.m) {
-            const int64_t col = static_cast<int64_t>(tn) * 64 + 32 * c;
-            uint4* pa = reinterpret_cast<uint4*>(g.A16 + row * g.ld16 + col);
-            uint4* pg = reinterpret_cast<uint4*>(g.G16 + row * g.ld16 + col);
-            uint4* ph = reinterpret_cast<uint4*>(g.H16 + row * g.ld16 + col);
 #pragma unroll
-            for (int j8 = 0; j8 < 4; ++j8) {
-              uint32_t wa[4], wg[4], wh[4];
+          for (int j8 = 0; j8 < 4; ++j8) {
+            uint32_t wa[4], wg[4], wh[4];
 #pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                const float a0 = __uint_as_float(va[8 * j8 + 2 * e]), a1 = __uint_as_float(va[8 * j8 + 2 * e + 1]);
-                const float g0 = __uint_as_float(vg[8 * j8 + 2 * e]), g1 = __uint_as_float(vg[8 * j8 + 2 * e + 1]);
-                wa[e] = pack_bf16x2(a0, a1);
-                wg[e] = pack_bf16x2(g0, g1);
-                wh[e] = pack_bf16x2(a0 * g0 * sigmoid_f(g0), a1 * g1 * sigmoid_f(g1));
-              }
-              pa[j8] = make_uint4(wa[0], wa[1], wa[2], wa[3]);
-              pg[j8] = make_uint4(wg[0], wg[1], wg[2], wg[3]);
-              ph[j8] = make_uint4(wh[0], wh[1], wh[2], wh[3]);
+            for (int e = 0; e < 4; ++e) {
+              const float a0 = __uint_as_float(va[8 * j8 + 2 * e]), a1 = __uint_as_float(va[8 * j8 + 2 * e + 1]);
+              const float g0 = __uint_as_float(vg[8 * j8 + 2 * e]), g1 = __uint_as_float(vg[8 * j8 + 2 * e + 1]);
+              wa[e] = pack_bf16x2(a0, a1);
+              wg[e] = pack_bf16x2(g0, g1);
+              wh[e] = pack_bf16x2(a0 * g0 * sigmoid_f(g0), a1 * g1 * sigmoid_f(g1));
             }
+            const int off = lane * kLd + 32 * c + 8 * j8;
+            *reinterpret_cast<uint4*>(sA + off) = make_uint4(wa[0], wa[1], wa[2], wa[3]);
+            *reinterpret_cast<uint4*>(sG + off) = make_uint4(wg[0], wg[1], wg[2], wg[3]);
+            *reinterpret_cast<uint4*>(sH + off) = make_uint4(wh[0], wh[1], wh[2], wh[3]);
+          }
+        }
+        __syncwarp();
+        // 4 rows per warp instruction: lanes 8 i .. 8 i + 7 write row rr + i (128 bytes)
+        const int64_t col = static_cast<int64_t>(tn) * 64 + 8 * (lane & 7);
+        for (int rr = 0; rr < 32; rr += 4) {
+          const int r = rr + (lane >> 3);
+          const int64_t row = rbase + r;
+          if (row < g.m) {
+            const int off = r * kLd + 8 * (lane & 7);
+            *reinterpret_cast<uint4*>(g.A16 + row * g.ld16 + col) = *reinterpret_cast<const uint4*>(sA + off);
+            *reinterpret_cast<uint4*>(g.G16 + row * g.ld16 + col) = *reinterpret_cast<const uint4*>(sG + off);
+            *reinterpret_cast<uint4*>(g.H16 + row * g.ld16 + col) = *reinterpret_cast<const uint4*>(sH + off);
           }
         }
       } else {
-        // dH of hidden columns n0 .. n0 + BN - 1
+        // dH of hidden columns n0 .. n0 + 127: the A and G tiles of this warp's
+        // rows come in coalesced (2 rows per instruction), dA and dG go back the
+        // same way over them
+        constexpr int kLd = 136;                          // 128 bf16 + 8 pad per staged row
+        uint16_t* sA = reinterpret_cast<uint16_t*>(sm) + q * 2 * 32 * kLd;
+        uint16_t* sG = sA + 32 * kLd;
+        for (int rr = 0; rr < 32; rr += 2) {
+          const int r = rr + (lane >> 4);
+          const int64_t row = rbase + r;
+          const int off = r * kLd + 8 * (lane & 15);
+          uint4 av = make_uint4(0u, 0u, 0u, 0u), gv = av;
+          if (row < g.m) {
+            av = *reinterpret_cast<const uint4*>(g.A16 + row * g.ld16 + n0 + 8 * (lane & 15));
+            gv = *reinterpret_cast<const uint4*>(g.G16 + row * g.ld16 + n0 + 8 * (lane & 15));
+          }
+          *reinterpret_cast<uint4*>(sA + off) = av;
+          *reinterpret_cast<uint4*>(sG + off) = gv;
+        }
+        __syncwarp();
 #pragma unroll 1
         for (int c = 0; c < BN / 32; ++c) {
           uint32_t v[32];
           tmem_ld32(tmem + lane_off + 32 * c, v);
           tmem_ld_wait();
-          if (row < g.m) {
-            const int64_t col = n0 + 32 * c;
-            uint4* pa = reinterpret_cast<uint4*>(g.A16 + row * g.ld16 + col);
-            uint4* pg = reinterpret_cast<uint4*>(g.G16 + row * g.ld16 + col);
 #pragma unroll
-            for (int j8 = 0; j8 < 4; ++j8) {
-              const uint4 av = pa[j8], gv = pg[j8];
-              const uint32_t aw[4] = {av.x, av.y, av.z, av.w}, gw[4] = {gv.x, gv.y, gv.z, gv.w};
-              uint32_t da[4], dg[4];
+          for (int j8 = 0; j8 < 4; ++j8) {
+            const int off = lane * kLd + 32 * c + 8 * j8;
+            const uint4 av = *reinterpret_cast<const uint4*>(sA + off);
+            const uint4 gv = *reinterpret_cast<const uint4*>(sG + off);
+            const uint32_t aw[4] = {av.x, av.y, av.z, av.w}, gw[4] = {gv.x, gv.y, gv.z, gv.w};
+            uint32_t da[4], dg[4];
 #pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                float outa[2], outg[2];
+            for (int e = 0; e < 4; ++e) {
+              float outa[2], outg[2];
 #pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {
-                  const float a = __uint_as_float(hh ? (aw[e] & 0xFFFF0000u) : (aw[e] << 16));
-                  const float gg = __uint_as_float(hh ? (gw[e] & 0xFFFF0000u) : (gw[e] << 16));
-                  const float dh = __uint_as_float(v[8 * j8 + 2 * e + hh]);
-                  const float sg = sigmoid_f(gg);
-                  outa[hh] = dh * gg * sg;
-                  outg[hh] = dh * a * sg * (1.f + gg * (1.f - sg));
-                }
-                da[e] = pack_bf16x2(outa[0], outa[1]);
-                dg[e] = pack_bf16x2(outg[0], outg[1]);
+              for (int hh = 0; hh < 2; ++hh) {
+                const float aa = __uint_as_float(hh ? (aw[e] & 0xFFFF0000u) : (aw[e] << 16));
+                const float gg = __uint_as_float(hh ? (gw[e] & 0xFFFF0000u) : (gw[e] << 16));
+                const float dh = __uint_as_float(v[8 * j8 + 2 * e + hh]);
+                const float sg = sigmoid_f(gg);
+                outa[hh] = dh * gg * sg;
+                outg[hh] = dh * aa * sg * (1.f + gg * (1.f - sg));
               }
-              pa[j8] = make_uint4(da[0], da[1], da[2], da[3]);
-              pg[j8] = make_uint4(dg[0], dg[1], dg[2], dg[3]);
+              da[e] = pack_bf16x2(outa[0], outa[1]);
+              dg[e] = pack_bf16x2(outg[0], outg[1]);
             }
+            *reinterpret_cast<uint4*>(sA + off) = make_uint4(da[0], da[1], da[2], da[3]);
+            *reinterpret_cast<uint4*>(sG + off) = make_uint4(dg[0], dg[1], dg[2], dg[3]);
+          }
+        }
+        __syncwarp();
+        for (int rr = 0; rr < 32; rr += 2) {
+          const int r = rr + (lane >> 4);
+          const int64_t row = rbase + r;
+          if (row < g.m) {
+            const int off = r * kLd + 8 * (lane & 15);
+            *reinterpret_cast<uint4*>(g.A16 + row * g.ld16 + n0 + 8 * (lane & 15)) =
+                *reinterpret_cast<const uint4*>(sA + off);
+            *reinterpret_cast<uint4*>(g.G16 + row * g.ld16 + n0 + 8 * (lane & 15)) =
+                *reinterpret_cast<const uint4*>(sG + off);
           }
         }
       }

@@ -38,7 +38,7 @@ namespace {
 using namespace tc;
 
 constexpr int kKvThreads = 192;
-constexpr int kAS = 6;                        // A ring stages ([128 x 64] bf16 each)
+constexpr int kAS = 5;                        // A ring stages ([128 x 64] bf16 each)
 constexpr uint32_t kABlock = 128u * 128u;     // 16 KB
 constexpr uint32_t kBBlock = 256u * 128u;     // [256 outputs x 64 inputs]: 32 KB
 
@@ -48,7 +48,8 @@ struct KvCfg {
   static constexpr int NS = 2 * D / 256;                  // 256-output slices
   static constexpr uint32_t oB = 0;
   static constexpr uint32_t oA = oB + KB * kBBlock;
-  static constexpr uint32_t oBar = oA + kAS * kABlock;
+  static constexpr uint32_t oStg = oA + kAS * kABlock;     // epilogue staging: 4 warps x 32 rows x 72 bf16
+  static constexpr uint32_t oBar = oStg + 4 * 32 * 72 * 2;
   // bfull; afull, aempty [kAS]; accfull, accempty [2]; mdrain
   static constexpr int kBars = 1 + 2 * kAS + 4 + 1;
   static constexpr uint32_t oMisc = oBar + kBars * 8;
@@ -185,24 +186,28 @@ kv_proj_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ 
   } else {
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;
-    const int r = q * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
     const int ld_out = 2 * D;
     uint32_t u = 0;
     for (int64_t t = tile0; t < ntiles; t += tstep, ++u) {
       const int buf = u & 1;
-      if (!kwait(&accfull[buf], (u >> 1) & 1, abort_flag, p.status)) break;
+      // one answer for the warp: the TMEM loads below are warp-collective
+      if (!__all_sync(0xffffffffu, kwait(&accfull[buf], (u >> 1) & 1, abort_flag, p.status))) break;
       __syncwarp();
       tc_fence_after();
-      const int64_t row = t * 128 + r;
-      uint16_t* dst = p.out + row * ld_out + slice * 256;
+      // 64 outputs at a time: each thread stages its row's 64 bf16, then the
+      // warp writes its 32 rows coalesced (8 lanes x 16 bytes per row, 4 rows
+      // per instruction)
+      uint16_t* stg = reinterpret_cast<uint16_t*>(sm + C::oStg) + q * 32 * 72;
+      const int64_t row0 = t * 128 + q * 32;
 #pragma unroll 1
-      for (int c = 0; c < 8; ++c) {              // 256 outputs, 32 at a time
-        uint32_t v[32];
-        tmem_ld32(tmem + lane_off + buf * 256 + c * 32, v);
-        tmem_ld_wait();
-        if (row < p.N) {
-          uint4* d4 = reinterpret_cast<uint4*>(dst + c * 32);
+      for (int c64 = 0; c64 < 4; ++c64) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          uint32_t v[32];
+          tmem_ld32(tmem + lane_off + buf * 256 + c64 * 64 + h * 32, v);
+          tmem_ld_wait();
+          uint4* d4 = reinterpret_cast<uint4*>(stg + lane * 72 + 32 * h);
 #pragma unroll
           for (int k = 0; k < 4; ++k)
             d4[k] = make_uint4(pack_bf16x2(__uint_as_float(v[8 * k]), __uint_as_float(v[8 * k + 1])),
@@ -210,6 +215,16 @@ kv_proj_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ 
                                pack_bf16x2(__uint_as_float(v[8 * k + 4]), __uint_as_float(v[8 * k + 5])),
                                pack_bf16x2(__uint_as_float(v[8 * k + 6]), __uint_as_float(v[8 * k + 7])));
         }
+        __syncwarp();
+#pragma unroll
+        for (int rr = 0; rr < 32; rr += 4) {
+          const int rl = rr + (lane >> 3);
+          const int64_t row = row0 + rl;
+          if (row < p.N)
+            *reinterpret_cast<uint4*>(p.out + row * ld_out + slice * 256 + c64 * 64 + 8 * (lane & 7)) =
+                *reinterpret_cast<const uint4*>(stg + rl * 72 + 8 * (lane & 7));
+        }
+        __syncwarp();
       }
       tc_fence_before();
       __syncwarp();
