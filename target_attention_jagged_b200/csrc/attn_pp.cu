@@ -33,9 +33,9 @@
 // never a wait -- and the warp that arrives last merges the slot's rows of all
 // the pair's items into c.  The counters must be zero when the kernel starts.
 //
-// Warp roles (320 threads): warp 0 loads Q and X~ tiles (TMA), warp 1 owns
-// TMEM and issues all MMAs, warps 2-5 are softmax group 0, warps 6-9 group 1
-// (warp w reads TMEM lane quarter w % 4).  Every wait is a bounded mbarrier
+// Warp roles (384 threads): warp 0 loads Q and X~ tiles (TMA), warp 1 owns
+// TMEM and issues all MMAs, warps 2-3 idle, warps 4-7 are softmax group 0,
+// warps 8-11 group 1 (warp w reads TMEM lane quarter w % 4).  Every wait is a bounded mbarrier
 // wait; a wait that gives up sets the device status and stops the CTA's other
 // roles, and the CTA lets its copies and MMAs in flight finish before it exits.
 #include <cuda.h>
@@ -85,7 +85,13 @@ struct PPCfg {
   static_assert(kSmem <= 227 * 1024, "shared memory overflow");
 };
 
-constexpr int kPPThreads = 320;
+// Three warpgroups: warps 0-3 (loader, MMA issuer, two idle) hand registers
+// to the two softmax warpgroups, so a softmax thread can hold its whole row of
+// a key tile.  Launched at 168 per thread (65536 / 384, rounded down to the
+// allocation unit); 128 x 48 + 256 x 224 = 63488 <= 384 x 168 = 64512.
+constexpr int kPPThreads = 384;
+constexpr int kPPRegsLow = 48, kPPRegsHigh = 224;
+static_assert(128 * kPPRegsLow + 256 * kPPRegsHigh <= kPPThreads * 168, "register split");
 constexpr float kRescale = 8.0f;                 // log2 units
 
 __device__ __forceinline__ bool pwait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
@@ -238,6 +244,8 @@ attn_pp_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   pdl_wait();                          // the predecessor's results are visible from here on
   const uint32_t sbase = smem_u32(sm);
 
+  if (warp < 4) {
+  regs_dec<kPPRegsLow>();
   if (warp == 0) {
     // ------------------------------------------------------------ TMA loader
     if (lane == 0) {
@@ -344,9 +352,11 @@ attn_pp_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       mma_commit(mdrain);
       pdrain(mdrain, 0, 500000000ull);
     }
+  }
   } else {
+    regs_inc<kPPRegsHigh>();
     // ------------------------------------------------------------ softmax groups
-    const int b = (warp - 2) >> 2;           // group: tiles g with g % 2 == b
+    const int b = (warp - 4) >> 2;           // group: tiles g with g % 2 == b
     const int q = warp & 3;                  // TMEM lane quarter
     const int r = q * 32 + lane;             // query row of the tile
     const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
@@ -363,33 +373,33 @@ attn_pp_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         if (!(ok = pwait_warp(&sfull[b], cb & 1, abort_flag, p.status))) break;
         __syncwarp();
         tc_fence_after();
-        // two passes over the tile's S columns, 64 at a time (registers: a
-        // thread holds half of its row at once): the row maximum, then the
-        // exponentials, written back as packed bf16 P over the first 64 columns
+        // the thread's whole row of the tile's S (128 columns) in one TMEM
+        // round trip: the row maximum, then the exponentials, written back as
+        // packed bf16 P over the first 64 columns
         const int nvalid = min(128, item.nkeys - j * 128);
         const uint32_t srow = tmem + lane_off + C::kS + b * 128;
-        float mx = -INFINITY;
+        uint32_t sv[4][32];
 #pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-          uint32_t sv[2][32];
-          tmem_ld32(srow + hh * 64, sv[0]);
-          tmem_ld32(srow + hh * 64 + 32, sv[1]);
-          tmem_ld_wait();
-          if (nvalid < 128) {   // the item's last tile: keys past its end take no weight
+        for (int c = 0; c < 4; ++c) tmem_ld32(srow + 32 * c, sv[c]);
+        tmem_ld_wait();
+        if (nvalid < 128) {     // the item's last tile: keys past its end take no weight
 #pragma unroll
-            for (int c = 0; c < 2; ++c)
+          for (int c = 0; c < 4; ++c)
 #pragma unroll
-              for (int k = 0; k < 32; ++k)
-                if (hh * 64 + c * 32 + k >= nvalid) sv[c][k] = __float_as_uint(-INFINITY);
-          }
+            for (int k = 0; k < 32; ++k)
+              if (c * 32 + k >= nvalid) sv[c][k] = __float_as_uint(-INFINITY);
+        }
+        float mx;
+        {
+          float m4[4];
 #pragma unroll
-          for (int c = 0; c < 2; ++c) {
-            float m = fmaxf(__uint_as_float(sv[c][0]), __uint_as_float(sv[c][1]));
+          for (int c = 0; c < 4; ++c) {
+            m4[c] = fmaxf(__uint_as_float(sv[c][0]), __uint_as_float(sv[c][1]));
 #pragma unroll
             for (int k = 2; k < 32; k += 2)
-              m = sx::max3(m, __uint_as_float(sv[c][k]), __uint_as_float(sv[c][k + 1]));
-            mx = fmaxf(mx, m);
+              m4[c] = sx::max3(m4[c], __uint_as_float(sv[c][k]), __uint_as_float(sv[c][k + 1]));
           }
+          mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
         }
         const bool resc = mx > m_run + kRescale;          // always on the item's first tile
         const float m_new = resc ? mx : m_run;
@@ -399,21 +409,10 @@ attn_pp_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         uint64_t ls[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {
-          uint32_t sv[2][32];
-          tmem_ld32(srow + hh * 64, sv[0]);
-          tmem_ld32(srow + hh * 64 + 32, sv[1]);
-          tmem_ld_wait();
-          if (nvalid < 128) {
-#pragma unroll
-            for (int c = 0; c < 2; ++c)
-#pragma unroll
-              for (int k = 0; k < 32; ++k)
-                if (hh * 64 + c * 32 + k >= nvalid) sv[c][k] = __float_as_uint(-INFINITY);
-          }
           uint32_t pk[32];
 #pragma unroll
           for (int k = 0; k < 64; k += 2) {
-            const int c = k >> 5, e = k & 31;
+            const int c = 2 * hh + (k >> 5), e = k & 31;
             const uint64_t x = sx::f2_add(sx::f2(__uint_as_float(sv[c][e]), __uint_as_float(sv[c][e + 1])), negm);
             float x0, x1, p0, p1;
             sx::f2_split(x, x0, x1);
@@ -426,8 +425,8 @@ attn_pp_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
             ls[(k >> 1) & 3] = sx::f2_add(ls[(k >> 1) & 3], sx::f2(p0, p1));
             pk[k >> 1] = pack_bf16x2(p0, p1);
           }
-          // P of keys 64 hh .. 64 hh + 63: columns 32 hh .. 32 hh + 31, S
-          // columns this row has already read
+          // P of keys 64 hh .. 64 hh + 63: columns 32 hh .. 32 hh + 31 (the
+          // whole row is already in registers)
           st_tmem32(srow + hh * 32, pk);
         }
         tmem_st_wait();
@@ -543,7 +542,14 @@ int launch_pp(const CUtensorMap& tmQ, const CUtensorMap& tmK, const PPParams& p,
               cudaStream_t s) {
   using C = PPCfg<D>;
   auto k = attn_pp_kernel<D, FMA_PAIRS>;
-  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+  cudaFuncAttributes fa{};
+  cudaError_t e = cudaFuncGetAttributes(&fa, k);
+  if (e != cudaSuccess) return set_error(STCA_ECUDA, std::string("attn_pp attributes: ") + cudaGetErrorString(e));
+  // the warpgroups' register split must fit what the block is launched with,
+  // or the raising warpgroups would wait for registers that never come
+  if (fa.numRegs * kPPThreads < 128 * kPPRegsLow + 256 * kPPRegsHigh)
+    return set_error(STCA_ECUDA, "attn_pp: built with too few registers per thread for its register split");
+  e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
   if (e != cudaSuccess) return set_error(STCA_ECUDA, std::string("attn_pp smem: ") + cudaGetErrorString(e));
   e = launch_pdl(k, dim3(grid), dim3(kPPThreads), C::kSmem, s, tmQ, tmK, p);
   if (e != cudaSuccess) return set_error(STCA_ECUDA, std::string("attn_pp launch: ") + cudaGetErrorString(e));

@@ -357,8 +357,9 @@ __global__ void ffn_weights16_kernel(const float* __restrict__ Wu, const float* 
     const int64_t c = hcol / 64, j = hcol - c * 64;
     W1i[(128 * c + j) * d + k] = bf(Wu[i]);
     W1i[(128 * c + 64 + j) * d + k] = bf(Wg[i]);
-    Wu16[i] = bf(Wu[i]);
-    Wg16[i] = bf(Wg[i]);
+    // [W_u | W_g] side by side: row k of a d x 2 rd matrix
+    Wu16[k * 2 * rd + hcol] = bf(Wu[i]);
+    Wg16[k * 2 * rd + hcol] = bf(Wg[i]);
     // i as a row-major rd x d index of W_d: (h, nn)
     const int64_t h = i / d, nn = i - h * d;
     Wd16[i] = bf(Wd[i]);
@@ -494,38 +495,42 @@ namespace {
 // bf16 intermediates: [A | G] = X [W_u | W_g] with H = A SiLU(G) formed in the
 // GEMM's epilogue; Y = H W_d; the LayerNorm derivative (dy, also as bf16);
 // dW_d = H^T dy; dH = dy W_d^T with the SwiGLU derivative in the epilogue
-// (dA, dG over A, G); dW_u = X^T dA, dW_g = X^T dG; dX = dA W_u^T + dG W_g^T.
-// Products with K = N (the weight gradients) split K over CTAs.
+// (dA, dG over A, G); dW_u = X^T dA, dW_g = X^T dG; dX = [dA | dG] [W_u | W_g]^T,
+// one product over K = 2 rd.  A and G share the rows of one N x 2 rd buffer
+// (A in the first rd columns), so dA and dG are that product's left operand
+// as they lie.  Products with K = N (the weight gradients) split K over CTAs.
 int ffn_ln_backward16(stca_handle* H, const uint16_t* X, int64_t N, const float* dXt, float* dX,
                       const float* Wu, const float* Wg, const float* Wd, const float* gamma, float* dWu,
                       float* dWg, float* dWd, float* dgamma, float* dbeta, cudaStream_t s) {
   const int d = H->d, rd = H->rd;
   const size_t nd = static_cast<size_t>(N) * d, nr = static_cast<size_t>(N) * rd;
   const size_t wn = static_cast<size_t>(d) * rd;
-  // workspace: A16, G16, H16 (N rd bf16), dy16 (N d bf16), Y (N d fp32), weights (5 d rd bf16)
+  // workspace: AG (N x 2 rd bf16), H16 (N rd bf16), dy16 (N d bf16), Y (N d fp32), weights (6 d rd bf16)
   auto a256 = [](size_t x) { return (x + 255) & ~size_t(255); };
-  const size_t oA = 0, oG = a256(oA + nr * 2), oH = a256(oG + nr * 2), oDy = a256(oH + nr * 2);
+  const size_t oAG = 0, oH = a256(oAG + 2 * nr * 2), oDy = a256(oH + nr * 2);
   const size_t oY = a256(oDy + nd * 2), oW = a256(oY + nd * 4), total = a256(oW + 6 * wn * 2);
   if (int rc = ensure(&H->bw_ws, &H->bw_ws_cap, total)) return rc;
   char* w = static_cast<char*>(H->bw_ws);
-  uint16_t* A16 = reinterpret_cast<uint16_t*>(w + oA);
-  uint16_t* G16 = reinterpret_cast<uint16_t*>(w + oG);
+  uint16_t* AG = reinterpret_cast<uint16_t*>(w + oAG);
   uint16_t* H16 = reinterpret_cast<uint16_t*>(w + oH);
   uint16_t* dy16 = reinterpret_cast<uint16_t*>(w + oDy);
   float* Y = reinterpret_cast<float*>(w + oY);
   uint16_t* W1i = reinterpret_cast<uint16_t*>(w + oW);      // 2 wn
   uint16_t* WdT = W1i + 2 * wn;
   uint16_t* Wd16 = WdT + wn;
-  uint16_t* Wu16 = Wd16 + wn;
-  uint16_t* Wg16 = Wu16 + wn;
-  ffn_weights16_kernel<<<grid_for(static_cast<int64_t>(wn)), 256, 0, s>>>(Wu, Wg, Wd, W1i, WdT, Wd16, Wu16, Wg16, d, rd);
+  uint16_t* Wug = Wd16 + wn;                                  // d x 2 rd: [W_u | W_g]
+  ffn_weights16_kernel<<<grid_for(static_cast<int64_t>(wn)), 256, 0, s>>>(Wu, Wg, Wd, W1i, WdT, Wd16, Wug,
+                                                                          Wug + rd, d, rd);
   STCA_CUDA_TRY(cudaGetLastError());
   const int ns = H->num_sms;
   int* st = H->status_d;
+  const int64_t ldag = 2 * static_cast<int64_t>(rd);
   // forward recomputation
-  if (int rc = tc_gemm_bf16(false, true, N, 2 * rd, d, X, d, W1i, d, nullptr, 0, 0.f, 1, A16, G16, H16, rd, ns, st, s))
+  if (int rc = tc_gemm_bf16(false, true, N, 2 * rd, d, X, d, W1i, d, nullptr, 0, 0.f, 1, AG, AG + rd, H16, ldag,
+                            rd, ns, st, s))
     return rc;
-  if (int rc = tc_gemm_bf16(false, true, N, d, rd, H16, rd, WdT, rd, Y, d, 0.f, 0, nullptr, nullptr, nullptr, 0, ns, st, s))
+  if (int rc = tc_gemm_bf16(false, true, N, d, rd, H16, rd, WdT, rd, Y, d, 0.f, 0, nullptr, nullptr, nullptr, 0, 0,
+                            ns, st, s))
     return rc;
   // LayerNorm: Y <- dy (also dy16); dgamma, dbeta
   STCA_CUDA_TRY(cudaMemsetAsync(dgamma, 0, d * sizeof(float), s));
@@ -535,25 +540,23 @@ int ffn_ln_backward16(stca_handle* H, const uint16_t* X, int64_t N, const float*
   STCA_CUDA_TRY(cudaGetLastError());
   // dW_d = H^T dy
   if (int rc = tc_gemm_bf16(true, false, rd, d, N, H16, rd, dy16, d, dWd, d, 0.f, 0, nullptr, nullptr, nullptr, 0,
-                            ns, st, s))
+                            0, ns, st, s))
     return rc;
-  // dH = dy W_d^T, then dA, dG over A16, G16
-  if (int rc = tc_gemm_bf16(false, true, N, rd, d, dy16, d, Wd16, d, nullptr, 0, 0.f, 2, A16, G16, nullptr, rd,
-                            ns, st, s))
+  // dH = dy W_d^T, then dA, dG over A, G
+  if (int rc = tc_gemm_bf16(false, true, N, rd, d, dy16, d, Wd16, d, nullptr, 0, 0.f, 2, AG, AG + rd, nullptr,
+                            ldag, 0, ns, st, s))
     return rc;
   // dW_u = X^T dA, dW_g = X^T dG
-  if (int rc = tc_gemm_bf16(true, false, d, rd, N, X, d, A16, rd, dWu, rd, 0.f, 0, nullptr, nullptr, nullptr, 0,
-                            ns, st, s))
+  if (int rc = tc_gemm_bf16(true, false, d, rd, N, X, d, AG, ldag, dWu, rd, 0.f, 0, nullptr, nullptr, nullptr, 0,
+                            0, ns, st, s))
     return rc;
-  if (int rc = tc_gemm_bf16(true, false, d, rd, N, X, d, G16, rd, dWg, rd, 0.f, 0, nullptr, nullptr, nullptr, 0,
-                            ns, st, s))
+  if (int rc = tc_gemm_bf16(true, false, d, rd, N, X, d, AG + rd, ldag, dWg, rd, 0.f, 0, nullptr, nullptr, nullptr,
+                            0, 0, ns, st, s))
     return rc;
+  // dX = [dA | dG] [W_u | W_g]^T
   if (dX) {
-    if (int rc = tc_gemm_bf16(false, true, N, d, rd, A16, rd, Wu16, rd, dX, d, 0.f, 0, nullptr, nullptr, nullptr,
-                              0, ns, st, s))
-      return rc;
-    if (int rc = tc_gemm_bf16(false, true, N, d, rd, G16, rd, Wg16, rd, dX, d, 1.f, 0, nullptr, nullptr, nullptr,
-                              0, ns, st, s))
+    if (int rc = tc_gemm_bf16(false, true, N, d, 2 * rd, AG, ldag, Wug, ldag, dX, d, 0.f, 0, nullptr, nullptr,
+                              nullptr, 0, 0, ns, st, s))
       return rc;
   }
   set_error(STCA_OK, "");

@@ -258,45 +258,51 @@ struct Gemm16Args {
   int64_t ldc;
   float alpha, beta;
   int atomic;
-  uint16_t *A16, *G16, *H16;    // SwiGLU epilogues: N x rd bf16 (ld = ld16)
-  int64_t ld16;
+  uint16_t *A16, *G16, *H16;    // SwiGLU epilogues: N x rd bf16 (A, G: ld = ld16; H: ld = ldh)
+  int64_t ld16, ldh;
   int* status;
 };
 
 constexpr uint32_t kA16Stage = 128u * 128u;     // [128 x 64] bf16
+constexpr int kGemm16Stages = 4;
+constexpr int kGemm16Threads = 320;             // loader, MMA issuer, eight epilogue warps
+// eight warps' staged rows; the largest is the SwiGLU backward's (A and G,
+// 32 rows x 72 bf16 each); the plain store's is 32 x 68 floats
+constexpr uint32_t kGemm16Staging = 8u * 2 * 32 * 72 * 2;
 
-__device__ __forceinline__ float sigmoid_f(float z) { return 1.0f / (1.0f + __expf(-z)); }
+__device__ __forceinline__ float sigmoid_f(float z) { return __fdividef(1.0f, 1.0f + __expf(-z)); }
 
 template <int BN, bool AMN, bool BMN, int EPI>
-__global__ void __launch_bounds__(kGemmThreads, 1)
+__global__ void __launch_bounds__(kGemm16Threads, 1)
 gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                  const Gemm16Args g) {
+  // Persistent: CTA c takes units c, c + gridDim.x, ... (unit = (row tile,
+  // column tile, K split)); two TMEM accumulators let the epilogue of one unit
+  // run while the next unit's stages load and multiply.
+  constexpr int kStages = kGemm16Stages;
   constexpr uint32_t kBStage = BN * 128u;
   constexpr uint32_t kStage = kA16Stage + kBStage;
+  constexpr uint32_t kStgOff = kStages * kStage;           // epilogue staging
+  constexpr uint32_t kBarOff = kStgOff + kGemm16Staging;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   if (smem_u32(smem_raw) & 1023u) {
     if (threadIdx.x == 0) atomicOr(g.status, kStatusStepTimeout);
     return;
   }
   uint8_t* sm = smem_raw;
-  uint64_t* full = reinterpret_cast<uint64_t*>(sm + kGemmStages * kStage);
-  uint64_t* empty = full + kGemmStages;
-  uint64_t* accfull = empty + kGemmStages;
-  uint64_t* mdrain = accfull + 1;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sm + kBarOff);
+  uint64_t* empty = full + kStages;
+  uint64_t* accfull = empty + kStages;       // [2]
+  uint64_t* accempty = accfull + 2;          // [2]
+  uint64_t* mdrain = accempty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mdrain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  int u = blockIdx.x;
-  const int ks = u % g.ksplit; u /= g.ksplit;
-  const int tn = u % g.tiles_n; u /= g.tiles_n;
-  const int tm = u;
-  const int64_t m0 = static_cast<int64_t>(tm) * 128, n0 = static_cast<int64_t>(tn) * BN;
-  const int64_t k0 = ks * g.k_per_split, k1 = min(g.k, k0 + g.k_per_split);
-  const int nst = static_cast<int>((k1 - k0 + 63) / 64);
+  const int64_t units = static_cast<int64_t>(g.tiles_m) * g.tiles_n * g.ksplit;
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kGemmStages; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
-    mbar_init(accfull, 1);
+    for (int i = 0; i < kStages; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
+    for (int i = 0; i < 2; ++i) { mbar_init(&accfull[i], 1); mbar_init(&accempty[i], 8); }
     mbar_init(mdrain, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -306,7 +312,7 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     prefetch_tmap(&tmB);
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, BN);
+    tmem_alloc(tmem_slot, 2 * BN);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -314,72 +320,128 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const uint32_t sbase = smem_u32(sm);
+  // unit -> (row tile, column tile, K range)
+  auto decode = [&](int64_t u, int64_t& m0, int64_t& n0, int& tn, int64_t& k0, int& nst) {
+    const int ks = static_cast<int>(u % g.ksplit);
+    const int64_t r = u / g.ksplit;
+    tn = static_cast<int>(r % g.tiles_n);
+    const int64_t tm = r / g.tiles_n;
+    m0 = tm * 128;
+    n0 = static_cast<int64_t>(tn) * BN;
+    k0 = ks * g.k_per_split;
+    const int64_t k1 = min(g.k, k0 + g.k_per_split);
+    nst = static_cast<int>((k1 - k0 + 63) / 64);
+  };
 
   if (warp == 0) {
     if (lane == 0) {
       bool ok = true;
-      int st = 0;
-      for (; ok && st < nst; ++st) {
-        const int s = st % kGemmStages;
-        if (!(ok = gwait(&empty[s], ((st / kGemmStages) & 1) ^ 1, abort_flag, g.status))) break;
-        mbar_arrive_expect_tx(&full[s], kStage);
-        uint8_t* a = sm + s * kStage;
-        uint8_t* bb = a + kA16Stage;
-        const int kk = static_cast<int>(k0 + 64 * st);
-        if constexpr (AMN) {
-          for (int i = 0; i < 2; ++i) tma_load_2d(a + i * 8192, &tmA, static_cast<int>(m0) + 64 * i, kk, &full[s]);
-        } else {
-          tma_load_2d(a, &tmA, kk, static_cast<int>(m0), &full[s]);
-        }
-        if constexpr (BMN) {
-          for (int i = 0; i < BN / 64; ++i)
-            tma_load_2d(bb + i * 8192, &tmB, static_cast<int>(n0) + 64 * i, kk, &full[s]);
-        } else {
-          tma_load_2d(bb, &tmB, kk, static_cast<int>(n0), &full[s]);
+      uint32_t st = 0;
+      for (int64_t u = blockIdx.x; ok && u < units; u += gridDim.x) {
+        int64_t m0, n0, k0;
+        int tn, nst;
+        decode(u, m0, n0, tn, k0, nst);
+        for (int j = 0; j < nst; ++j, ++st) {
+          const int s = st % kStages;
+          if (!(ok = gwait(&empty[s], ((st / kStages) & 1) ^ 1, abort_flag, g.status))) break;
+          mbar_arrive_expect_tx(&full[s], kStage);
+          uint8_t* a = sm + s * kStage;
+          uint8_t* bb = a + kA16Stage;
+          const int kk = static_cast<int>(k0 + 64 * j);
+          if constexpr (AMN) {
+            for (int i = 0; i < 2; ++i) tma_load_2d(a + i * 8192, &tmA, static_cast<int>(m0) + 64 * i, kk, &full[s]);
+          } else {
+            tma_load_2d(a, &tmA, kk, static_cast<int>(m0), &full[s]);
+          }
+          if constexpr (BMN) {
+            for (int i = 0; i < BN / 64; ++i)
+              tma_load_2d(bb + i * 8192, &tmB, static_cast<int>(n0) + 64 * i, kk, &full[s]);
+          } else {
+            tma_load_2d(bb, &tmB, kk, static_cast<int>(n0), &full[s]);
+          }
         }
       }
-      for (int c = st > kGemmStages ? st - kGemmStages : 0; c < st; ++c)
-        gdrain(&full[c % kGemmStages], (c / kGemmStages) & 1, 100000000ull);
+      for (uint32_t c = st > kStages ? st - kStages : 0; c < st; ++c)
+        gdrain(&full[c % kStages], (c / kStages) & 1, 100000000ull);
     }
   } else if (warp == 1) {
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_bf16(128, BN, AMN, BMN);
       bool ok = true;
-      for (int st = 0; st < nst; ++st) {
-        const int s = st % kGemmStages;
-        if (!(ok = gwait(&full[s], (st / kGemmStages) & 1, abort_flag, g.status))) break;
+      uint32_t st = 0, uc = 0;
+      for (int64_t u = blockIdx.x; ok && u < units; u += gridDim.x, ++uc) {
+        int64_t m0, n0, k0;
+        int tn, nst;
+        decode(u, m0, n0, tn, k0, nst);
+        const int buf = uc & 1;
+        if (!(ok = gwait(&accempty[buf], ((uc >> 1) & 1) ^ 1, abort_flag, g.status))) break;
         tc_fence_after();
-        const uint32_t a = sbase + s * kStage, bb = a + kA16Stage;
+        for (int j = 0; j < nst; ++j, ++st) {
+          const int s = st % kStages;
+          if (!(ok = gwait(&full[s], (st / kStages) & 1, abort_flag, g.status))) break;
+          tc_fence_after();
+          const uint32_t a = sbase + s * kStage, bb = a + kA16Stage;
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {          // K = 16 per MMA
-          const uint64_t ad = AMN ? sdesc_sw128(a + kk * 2048, 8192, 1024) : sdesc_sw128(a + kk * 32, 16, 1024);
-          const uint64_t bd = BMN ? sdesc_sw128(bb + kk * 2048, 8192, 1024) : sdesc_sw128(bb + kk * 32, 16, 1024);
-          mma_bf16_ss(tmem, ad, bd, idesc, (st | kk) != 0);
+          for (int kk = 0; kk < 4; ++kk) {          // K = 16 per MMA
+            const uint64_t ad = AMN ? sdesc_sw128(a + kk * 2048, 8192, 1024) : sdesc_sw128(a + kk * 32, 16, 1024);
+            const uint64_t bd = BMN ? sdesc_sw128(bb + kk * 2048, 8192, 1024) : sdesc_sw128(bb + kk * 32, 16, 1024);
+            mma_bf16_ss(tmem + buf * BN, ad, bd, idesc, (j | kk) != 0);
+          }
+          mma_commit(&empty[s]);
         }
-        mma_commit(&empty[s]);
+        if (!ok) break;
+        mma_commit(&accfull[buf]);
       }
-      if (ok) mma_commit(accfull);
       mma_commit(mdrain);
       gdrain(mdrain, 0, 500000000ull);
     }
   } else {
-    // Epilogue: each warp takes TMEM lane quarter q, rows m0 + 32 q .. + 31.  The
-    // pipeline's shared memory is free once every product is done; a warp stages
-    // its 32 rows there (lane = row) and then writes them row by row with the
-    // whole warp, so global accesses are coalesced.
-    const int q = warp & 3;
+    // Epilogue, eight warps: warp w takes TMEM lane quarter q = w % 4 (rows
+    // m0 + 32 q .. + 31 of a unit) and column half hf; it stages its rows in
+    // its own shared-memory area (lane = row), frees the accumulator once all
+    // eight have read it, and writes the rows with the whole warp (coalesced).
+    const int q = warp & 3, hf = (warp - 2) >> 2;
     const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
-    const bool ok = __all_sync(0xffffffffu, nst == 0 || gwait(accfull, 0, abort_flag, g.status)) != 0;
-    if (ok && nst > 0) {
-      tc_fence_after();
+    uint8_t* stg_base = sm + kStgOff + (warp - 2) * (kGemm16Staging / 8);
+    uint32_t uc = 0;
+    for (int64_t u = blockIdx.x; u < units; u += gridDim.x, ++uc) {
+      int64_t m0, n0, k0;
+      int tn, nst;
+      decode(u, m0, n0, tn, k0, nst);
+      const int buf = uc & 1;
       const int64_t rbase = m0 + q * 32;
+      if constexpr (EPI == kEpiSwigluB) {
+        // dH of hidden columns n0 + 64 hf .. + 63: the A and G rows come in
+        // coalesced (4 rows per instruction) before the accumulator is ready
+        constexpr int kLd = 72;                           // 64 bf16 + 8 pad per staged row
+        uint16_t* sA = reinterpret_cast<uint16_t*>(stg_base);
+        uint16_t* sG = sA + 32 * kLd;
+        const int64_t col = n0 + 64 * hf + 8 * (lane & 7);
+        for (int rr = 0; rr < 32; rr += 4) {
+          const int r = rr + (lane >> 3);
+          const int64_t row = rbase + r;
+          const int off = r * kLd + 8 * (lane & 7);
+          uint4 av = make_uint4(0u, 0u, 0u, 0u), gv = av;
+          if (row < g.m) {
+            av = *reinterpret_cast<const uint4*>(g.A16 + row * g.ld16 + col);
+            gv = *reinterpret_cast<const uint4*>(g.G16 + row * g.ld16 + col);
+          }
+          *reinterpret_cast<uint4*>(sA + off) = av;
+          *reinterpret_cast<uint4*>(sG + off) = gv;
+        }
+        __syncwarp();
+      }
+      if (!__all_sync(0xffffffffu, gwait(&accfull[buf], (uc >> 1) & 1, abort_flag, g.status))) break;
+      tc_fence_after();
+      const uint32_t tacc = tmem + buf * BN;
       if constexpr (EPI == kEpiStore) {
-        constexpr int kLd = BN + 4;                       // floats per staged row
-        float* stg = reinterpret_cast<float*>(sm) + q * 32 * kLd;
+        constexpr int kHalf = BN / 2;                     // columns per warp
+        constexpr int kLd = kHalf + 4;                    // floats per staged row
+        float* stg = reinterpret_cast<float*>(stg_base);
 #pragma unroll 1
-        for (int c = 0; c < BN / 32; ++c) {
+        for (int c = 0; c < kHalf / 32; ++c) {
           uint32_t v[32];
-          tmem_ld32(tmem + lane_off + 32 * c, v);
+          tmem_ld32(tacc + lane_off + kHalf * hf + 32 * c, v);
           tmem_ld_wait();
           float4* d4 = reinterpret_cast<float4*>(stg + lane * kLd + 32 * c);
 #pragma unroll
@@ -387,52 +449,58 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
             d4[j] = make_float4(g.alpha * __uint_as_float(v[4 * j]), g.alpha * __uint_as_float(v[4 * j + 1]),
                                 g.alpha * __uint_as_float(v[4 * j + 2]), g.alpha * __uint_as_float(v[4 * j + 3]));
         }
+        tc_fence_before();
         __syncwarp();
+        if (lane == 0) mbar_arrive(&accempty[buf]);
+        // kHalf / 4 float4 per row: 32 / (kHalf / 4) rows per warp instruction
+        constexpr int kC4 = kHalf / 4, kRows = 32 / kC4;
         const bool vec = (g.ldc & 3) == 0 && (reinterpret_cast<uintptr_t>(g.C) & 15) == 0;
-        for (int rr = 0; rr < 32; ++rr) {
-          const int64_t row = rbase + rr;
-          if (row >= g.m) break;
+        const int c4 = lane % kC4;
+        const int64_t col = n0 + kHalf * hf + 4 * c4;
+        for (int rr = 0; rr < 32; rr += kRows) {
+          const int r = rr + lane / kC4;
+          const int64_t row = rbase + r;
+          if (row >= g.m) continue;
           float* crow = g.C + row * g.ldc;
-          for (int c4 = lane; c4 < BN / 4; c4 += 32) {
-            const int64_t col = n0 + 4 * c4;
-            const float4 x = reinterpret_cast<const float4*>(stg + rr * kLd)[c4];
-            if (vec && col + 3 < g.n) {
-              if (g.atomic) {
-                asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(crow + col), "f"(x.x),
-                             "f"(x.y), "f"(x.z), "f"(x.w)
-                             : "memory");
-              } else {
-                float4 y = x;
-                if (g.beta != 0.f) {
-                  const float4 o = *reinterpret_cast<const float4*>(crow + col);
-                  y = make_float4(fmaf(g.beta, o.x, x.x), fmaf(g.beta, o.y, x.y), fmaf(g.beta, o.z, x.z),
-                                  fmaf(g.beta, o.w, x.w));
-                }
-                *reinterpret_cast<float4*>(crow + col) = y;
-              }
+          const float4 x = reinterpret_cast<const float4*>(stg + r * kLd)[c4];
+          if (vec && col + 3 < g.n) {
+            if (g.atomic) {
+              asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(crow + col), "f"(x.x),
+                           "f"(x.y), "f"(x.z), "f"(x.w)
+                           : "memory");
             } else {
-              const float xs[4] = {x.x, x.y, x.z, x.w};
-              for (int e = 0; e < 4; ++e)
-                if (col + e < g.n) {
-                  if (g.atomic) atomicAdd(crow + col + e, xs[e]);
-                  else crow[col + e] = g.beta != 0.f ? fmaf(g.beta, crow[col + e], xs[e]) : xs[e];
-                }
+              float4 y = x;
+              if (g.beta != 0.f) {
+                const float4 o = *reinterpret_cast<const float4*>(crow + col);
+                y = make_float4(fmaf(g.beta, o.x, x.x), fmaf(g.beta, o.y, x.y), fmaf(g.beta, o.z, x.z),
+                                fmaf(g.beta, o.w, x.w));
+              }
+              *reinterpret_cast<float4*>(crow + col) = y;
             }
+          } else {
+            const float xs[4] = {x.x, x.y, x.z, x.w};
+            for (int e = 0; e < 4; ++e)
+              if (col + e < g.n) {
+                if (g.atomic) atomicAdd(crow + col + e, xs[e]);
+                else crow[col + e] = g.beta != 0.f ? fmaf(g.beta, crow[col + e], xs[e]) : xs[e];
+              }
           }
         }
       } else if constexpr (EPI == kEpiSwigluF) {
-        // columns 0..63: up projection of hidden units 64 tn .. +63; 64..127: gate.
-        // Staged rows: A, G, H of this warp's rows, 64 bf16 (+ 8 pad) each.
-        constexpr int kLd = 72;
-        uint16_t* sA = reinterpret_cast<uint16_t*>(sm) + q * 3 * 32 * kLd;
+        // columns 0..63: up projection of hidden units 64 tn .. +63; 64..127:
+        // gate.  Half hf takes hidden units 32 hf .. 32 hf + 31 of the tile.
+        constexpr int kLd = 40;                           // 32 bf16 + 8 pad per staged row
+        uint16_t* sA = reinterpret_cast<uint16_t*>(stg_base);
         uint16_t* sG = sA + 32 * kLd;
         uint16_t* sH = sG + 32 * kLd;
-#pragma unroll 1
-        for (int c = 0; c < 2; ++c) {
+        {
           uint32_t va[32], vg[32];
-          tmem_ld32(tmem + lane_off + 32 * c, va);
-          tmem_ld32(tmem + lane_off + 64 + 32 * c, vg);
+          tmem_ld32(tacc + lane_off + 32 * hf, va);
+          tmem_ld32(tacc + lane_off + 64 + 32 * hf, vg);
           tmem_ld_wait();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&accempty[buf]);
 #pragma unroll
           for (int j8 = 0; j8 < 4; ++j8) {
             uint32_t wa[4], wg[4], wh[4];
@@ -444,49 +512,33 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
               wg[e] = pack_bf16x2(g0, g1);
               wh[e] = pack_bf16x2(a0 * g0 * sigmoid_f(g0), a1 * g1 * sigmoid_f(g1));
             }
-            const int off = lane * kLd + 32 * c + 8 * j8;
+            const int off = lane * kLd + 8 * j8;
             *reinterpret_cast<uint4*>(sA + off) = make_uint4(wa[0], wa[1], wa[2], wa[3]);
             *reinterpret_cast<uint4*>(sG + off) = make_uint4(wg[0], wg[1], wg[2], wg[3]);
             *reinterpret_cast<uint4*>(sH + off) = make_uint4(wh[0], wh[1], wh[2], wh[3]);
           }
         }
         __syncwarp();
-        // 4 rows per warp instruction: lanes 8 i .. 8 i + 7 write row rr + i (128 bytes)
-        const int64_t col = static_cast<int64_t>(tn) * 64 + 8 * (lane & 7);
-        for (int rr = 0; rr < 32; rr += 4) {
-          const int r = rr + (lane >> 3);
+        // 8 rows per warp instruction: lanes 4 i .. 4 i + 3 write row rr + i (64 bytes)
+        const int64_t col = static_cast<int64_t>(tn) * 64 + 32 * hf + 8 * (lane & 3);
+        for (int rr = 0; rr < 32; rr += 8) {
+          const int r = rr + (lane >> 2);
           const int64_t row = rbase + r;
           if (row < g.m) {
-            const int off = r * kLd + 8 * (lane & 7);
+            const int off = r * kLd + 8 * (lane & 3);
             *reinterpret_cast<uint4*>(g.A16 + row * g.ld16 + col) = *reinterpret_cast<const uint4*>(sA + off);
             *reinterpret_cast<uint4*>(g.G16 + row * g.ld16 + col) = *reinterpret_cast<const uint4*>(sG + off);
-            *reinterpret_cast<uint4*>(g.H16 + row * g.ld16 + col) = *reinterpret_cast<const uint4*>(sH + off);
+            *reinterpret_cast<uint4*>(g.H16 + row * g.ldh + col) = *reinterpret_cast<const uint4*>(sH + off);
           }
         }
       } else {
-        // dH of hidden columns n0 .. n0 + 127: the A and G tiles of this warp's
-        // rows come in coalesced (2 rows per instruction), dA and dG go back the
-        // same way over them
-        constexpr int kLd = 136;                          // 128 bf16 + 8 pad per staged row
-        uint16_t* sA = reinterpret_cast<uint16_t*>(sm) + q * 2 * 32 * kLd;
+        constexpr int kLd = 72;
+        uint16_t* sA = reinterpret_cast<uint16_t*>(stg_base);
         uint16_t* sG = sA + 32 * kLd;
-        for (int rr = 0; rr < 32; rr += 2) {
-          const int r = rr + (lane >> 4);
-          const int64_t row = rbase + r;
-          const int off = r * kLd + 8 * (lane & 15);
-          uint4 av = make_uint4(0u, 0u, 0u, 0u), gv = av;
-          if (row < g.m) {
-            av = *reinterpret_cast<const uint4*>(g.A16 + row * g.ld16 + n0 + 8 * (lane & 15));
-            gv = *reinterpret_cast<const uint4*>(g.G16 + row * g.ld16 + n0 + 8 * (lane & 15));
-          }
-          *reinterpret_cast<uint4*>(sA + off) = av;
-          *reinterpret_cast<uint4*>(sG + off) = gv;
-        }
-        __syncwarp();
 #pragma unroll 1
-        for (int c = 0; c < BN / 32; ++c) {
+        for (int c = 0; c < 2; ++c) {
           uint32_t v[32];
-          tmem_ld32(tmem + lane_off + 32 * c, v);
+          tmem_ld32(tacc + lane_off + 64 * hf + 32 * c, v);
           tmem_ld_wait();
 #pragma unroll
           for (int j8 = 0; j8 < 4; ++j8) {
@@ -514,26 +566,28 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
             *reinterpret_cast<uint4*>(sG + off) = make_uint4(dg[0], dg[1], dg[2], dg[3]);
           }
         }
+        tc_fence_before();
         __syncwarp();
-        for (int rr = 0; rr < 32; rr += 2) {
-          const int r = rr + (lane >> 4);
+        if (lane == 0) mbar_arrive(&accempty[buf]);
+        const int64_t col = n0 + 64 * hf + 8 * (lane & 7);
+        for (int rr = 0; rr < 32; rr += 4) {
+          const int r = rr + (lane >> 3);
           const int64_t row = rbase + r;
           if (row < g.m) {
-            const int off = r * kLd + 8 * (lane & 15);
-            *reinterpret_cast<uint4*>(g.A16 + row * g.ld16 + n0 + 8 * (lane & 15)) =
-                *reinterpret_cast<const uint4*>(sA + off);
-            *reinterpret_cast<uint4*>(g.G16 + row * g.ld16 + n0 + 8 * (lane & 15)) =
-                *reinterpret_cast<const uint4*>(sG + off);
+            const int off = r * kLd + 8 * (lane & 7);
+            *reinterpret_cast<uint4*>(g.A16 + row * g.ld16 + col) = *reinterpret_cast<const uint4*>(sA + off);
+            *reinterpret_cast<uint4*>(g.G16 + row * g.ld16 + col) = *reinterpret_cast<const uint4*>(sG + off);
           }
         }
       }
+      __syncwarp();                                     // staging rows are reused by the next unit
     }
   }
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, BN);
+    tmem_dealloc(tmem, 2 * BN);
   }
 }
 
@@ -658,12 +712,15 @@ int map16(CUtensorMap* m, const uint16_t* base, int64_t inner, int64_t rows, int
 
 template <int BN, int EPI>
 int launch16(bool amn, bool bmn, const CUtensorMap& tmA, const CUtensorMap& tmB, const Gemm16Args& g,
-             int64_t units, cudaStream_t s) {
-  const uint32_t smem = kGemmStages * (kA16Stage + BN * 128u) + (2 * kGemmStages + 2) * 8 + 16;
+             int64_t units, int num_sms, cudaStream_t s) {
+  const uint32_t smem = kGemm16Stages * (kA16Stage + BN * 128u) + kGemm16Staging + (2 * kGemm16Stages + 5) * 8 + 16;
+  static_assert(kGemm16Stages * (kA16Stage + 128u * 128u) + kGemm16Staging + (2 * kGemm16Stages + 5) * 8 + 16 <=
+                    227u * 1024u, "bf16 GEMM shared memory");
+  const unsigned grid = static_cast<unsigned>(std::min<int64_t>(units, std::max(num_sms, 1)));
   auto go = [&](auto kf) -> int {
     cudaError_t e = cudaFuncSetAttribute(kf, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return set_error(STCA_ECUDA, std::string("gemm_bf16 smem: ") + cudaGetErrorString(e));
-    kf<<<static_cast<unsigned>(units), kGemmThreads, smem, s>>>(tmA, tmB, g);
+    kf<<<grid, kGemm16Threads, smem, s>>>(tmA, tmB, g);
     e = cudaGetLastError();
     if (e != cudaSuccess) return set_error(STCA_ECUDA, std::string("gemm_bf16 launch: ") + cudaGetErrorString(e));
     return STCA_OK;
@@ -677,8 +734,9 @@ int launch16(bool amn, bool bmn, const CUtensorMap& tmA, const CUtensorMap& tmB,
 
 int tc_gemm_bf16(bool ta, bool tb, int64_t m, int64_t n, int64_t k, const uint16_t* A, int64_t lda,
                  const uint16_t* B, int64_t ldb, float* C, int64_t ldc, float beta, int epi, uint16_t* A16,
-                 uint16_t* G16, uint16_t* H16, int64_t ld16, int num_sms, int* status, cudaStream_t s) {
+                 uint16_t* G16, uint16_t* H16, int64_t ld16, int64_t ldh, int num_sms, int* status, cudaStream_t s) {
   if (m <= 0 || n <= 0) return STCA_OK;
+  if (k <= 0) return set_error(STCA_EINVAL, "bf16 tensor-core GEMM: empty inner dimension");
   auto al = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; };
   if (!al(A) || !al(B) || (lda * 2) % 16 || (ldb * 2) % 16)
     return set_error(STCA_EINVAL, "bf16 tensor-core GEMM: operands not 16-byte aligned");
@@ -700,6 +758,7 @@ int tc_gemm_bf16(bool ta, bool tb, int64_t m, int64_t n, int64_t k, const uint16
   g.G16 = G16;
   g.H16 = H16;
   g.ld16 = ld16;
+  g.ldh = ldh;
   g.status = status;
   const int64_t tiles = static_cast<int64_t>(g.tiles_m) * g.tiles_n;
   int ksplit = 1;
@@ -719,11 +778,11 @@ int tc_gemm_bf16(bool ta, bool tb, int64_t m, int64_t n, int64_t k, const uint16
   }
   const int64_t units = tiles * g.ksplit;
   if (units > INT32_MAX) return set_error(STCA_EINVAL, "bf16 tensor-core GEMM: too many tiles");
-  if (BN == 64) return launch16<64, kEpiStore>(amn, bmn, tmA, tmB, g, units, s);
+  if (BN == 64) return launch16<64, kEpiStore>(amn, bmn, tmA, tmB, g, units, num_sms, s);
   switch (epi) {
-    case kEpiSwigluF: return launch16<128, kEpiSwigluF>(amn, bmn, tmA, tmB, g, units, s);
-    case kEpiSwigluB: return launch16<128, kEpiSwigluB>(amn, bmn, tmA, tmB, g, units, s);
-    default: return launch16<128, kEpiStore>(amn, bmn, tmA, tmB, g, units, s);
+    case kEpiSwigluF: return launch16<128, kEpiSwigluF>(amn, bmn, tmA, tmB, g, units, num_sms, s);
+    case kEpiSwigluB: return launch16<128, kEpiSwigluB>(amn, bmn, tmA, tmB, g, units, num_sms, s);
+    default: return launch16<128, kEpiStore>(amn, bmn, tmA, tmB, g, units, num_sms, s);
   }
 }
 

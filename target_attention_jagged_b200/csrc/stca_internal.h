@@ -324,12 +324,13 @@ int tc_gemm_tf32(bool ta, bool tb, int64_t m, int64_t n, int64_t k, const float*
                  int64_t sA, int64_t sB, int64_t sC, int num_sms, int* status, cudaStream_t s);
 // The same GEMM with bf16 operands (any layout), fp32 C; epi 0 stores C,
 // epi 1 (SwiGLU forward: the weight's 128-row tiles interleave 64 up and 64
-// gate rows) writes A16, G16 and H16 = A SiLU(G) (bf16, row stride ld16) at
-// hidden columns 64 tn; epi 2 (SwiGLU backward: acc = dH) reads A16 and G16
-// and overwrites them with dA and dG.
+// gate rows) writes A16, G16 (row stride ld16) and H16 = A SiLU(G) (row
+// stride ldh), all bf16, at hidden columns 64 tn; epi 2 (SwiGLU backward:
+// acc = dH) reads A16 and G16 and overwrites them with dA and dG.
 int tc_gemm_bf16(bool ta, bool tb, int64_t m, int64_t n, int64_t k, const uint16_t* A, int64_t lda,
                  const uint16_t* B, int64_t ldb, float* C, int64_t ldc, float beta, int epi, uint16_t* A16,
-                 uint16_t* G16, uint16_t* H16, int64_t ld16, int num_sms, int* status, cudaStream_t s);
+                 uint16_t* G16, uint16_t* H16, int64_t ld16, int64_t ldh, int num_sms, int* status,
+                 cudaStream_t s);
 // The same with rows `row_bytes` apart (a multiple of 16).
 int make_tmap_bf16_2d_strided(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer,
                               uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer);
