@@ -768,9 +768,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--attn-form", type=int, default=0, choices=[0, 1, 2],
                     help="attention form: 0 reordered (Eq. 13, default), 1 naive (Eq. 12), 2 auto")
-    ap.add_argument("--attn-kernel", type=int, default=None, choices=[0, 1],
-                    help="tensor-core attention kernel (STCA_OPT_ATTN_KERNEL): 0 two-group, "
-                         "1 split-softmax + combine; default: the library's choice")
+    ap.add_argument("--attn-kernel", type=int, default=None, choices=[0, 1, 2],
+                    help="tensor-core attention kernel (STCA_OPT_ATTN_KERNEL): 0 auto, "
+                         "1 split-softmax + combine, 2 two-group; default: the library's choice")
     ap.add_argument("--strong", action="store_true",
                     help="strong scaling: one batch partitioned over the ranks by request "
                          "(shard.partition_requests); default: weak, a full batch per rank")

@@ -440,10 +440,12 @@ enum {
                                  The naive form needs the tensor-core step (see above) and
                                  d_h in {16, 32, 64}; form 1 without them is rejected, form 2
                                  falls back to the reordered form */
-  STCA_OPT_ATTN_KERNEL = 7,   /* tensor-core attention of the reordered form: 0 auto (for
-                                 d <= 128 the two-group kernel, which also merges the split
-                                 partials itself); 1 the split-softmax kernel followed by the
-                                 split combine (the only kernel for d = 256) */
+  STCA_OPT_ATTN_KERNEL = 7,   /* tensor-core attention of the reordered form: 0 auto (the
+                                 split-softmax kernel, with its query tile in TMEM for
+                                 d <= 128); 1 the split-softmax kernel; both are followed by
+                                 the split combine (in the next per-target step, or its own
+                                 launch); 2 the two-group kernel (d <= 128), which merges the
+                                 split partials itself */
   STCA_OPT_TEST_STOP_TILES = 8, /* test hook, 0 = off: the tensor-core attention's loader stops
                                  after this many key tiles per CTA and the kernel takes the exit
                                  of a bounded wait that ran out (copies and MMAs in flight are

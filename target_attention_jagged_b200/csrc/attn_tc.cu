@@ -49,11 +49,12 @@ using namespace tc;
 struct AttnParams {
   const AttnItem* items;
   const int32_t* cta_item_begin;   // gridDim.x + 1
-  float* pacc;                     // G x d
+  float* pacc;                     // G x d (PROJ: G x d_h, the projected rows)
   float* pm;                       // G
   float* pl;                       // G
   int* status;
   int stop_tiles;                  // > 0: the loader stops after this many key tiles (test hook)
+  int h, dh;                       // PROJ: heads and head width (query row r is head r % h)
 };
 
 // P_TMEM: P lives in TMEM (packed bf16, 64 columns per buffer) and the P X~
@@ -61,7 +62,18 @@ struct AttnParams {
 // through shared memory.  Keeping P out of shared memory matters: the MMAs'
 // operand reads, the TMA writes of X~ and the P writes would otherwise all
 // share its bandwidth.
-template <int D, int QB, int KS, int PB, bool SEPV>
+// QT: the query tile is copied from shared memory into TMEM once per item and
+// S = U X~^T takes it from there (a TMEM A operand), so the key tiles' S
+// products read only X~ from shared memory.
+// PROJ (with QT, d = 128): the item's output rows are projected by W_V in the
+// kernel (Eqs. (6), (13): o_j = alpha_j X~ W_V^j, and the split combine is
+// linear, so the unnormalised partials may be projected before it): O is
+// rounded to bf16 into the P columns of TMEM, one more product O W_V (all
+// heads' W_V^j side by side, B = [W_V]^T from shared memory, loaded once per
+// CTA) overwrites the O accumulator, and each row keeps only its head's d_h
+// columns.  Partials shrink from d to d_h floats per row, and the per-target
+// step starts from o_j directly.
+template <int D, int QB, int KS, int PB, bool SEPV, bool QT = false, bool PROJ = false>
 struct AttnCfg {
   static constexpr bool P_TMEM = D <= 128;
   static constexpr int KB = D / 64;
@@ -72,9 +84,10 @@ struct AttnCfg {
   static constexpr uint32_t oQ = 0;
   static constexpr uint32_t oK = oQ + QB * kTile;
   static constexpr uint32_t oP = oK + KS * kStage;
-  static constexpr uint32_t oX = oP + (P_TMEM ? 0 : PB * kPBytes);   // pair exchange: 2 x 2 x 128 floats
+  static constexpr uint32_t oWv = oP + (P_TMEM ? 0 : PB * kPBytes);  // PROJ: [W_V]^T, d x d
+  static constexpr uint32_t oX = oWv + (PROJ ? kTile : 0);   // pair exchange: 2 x 2 x 128 floats
   static constexpr uint32_t oBar = oX + 2 * 2 * 128 * 4;
-  static constexpr int kBars = 2 * QB + 2 * KS + 4 + 2 * PB + 3 + 1 + 8;
+  static constexpr int kBars = 2 * QB + 2 * KS + 4 + 2 * PB + 3 + 1 + 8 + 1 + 3;
   static constexpr uint32_t oMisc = oBar + kBars * 8;
   // No alignment slack: the dynamic shared memory of a block starts at a
   // 1024-byte boundary (after the 1 KB the system reserves), and the kernel
@@ -83,7 +96,10 @@ struct AttnCfg {
   static constexpr uint32_t kS = 0;        // 2 x 128 TMEM columns of scores
   static constexpr uint32_t kO = 256;      // D columns of the output accumulator
   static constexpr uint32_t kPt = kO + D;  // P_TMEM: PB x 64 columns of P
-  static_assert(kO + D + (P_TMEM ? PB * 64 : 0) <= 512, "TMEM overflow");
+  static constexpr uint32_t kQt = kPt + (P_TMEM ? PB * 64 : 0);   // QT: D / 2 columns of U
+  static_assert(kQt + (QT ? D / 2 : 0) <= 512, "TMEM overflow");
+  static_assert(!QT || (P_TMEM && !SEPV), "the TMEM query tile is for the reordered form, d <= 128");
+  static_assert(!PROJ || (QT && D == 128 && PB == 1), "the in-kernel projection reuses the P columns");
   static_assert(kSmem <= 227 * 1024, "shared memory overflow");
 };
 
@@ -124,11 +140,12 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
 }
 
 
-template <int D, int QB, int KS, int PB, bool SEPV>
+// tmV: the value tiles (SEPV) or the [W_V]^T tile (PROJ); otherwise unused.
+template <int D, int QB, int KS, int PB, bool SEPV, bool QT, bool PROJ>
 __global__ void __launch_bounds__(kAttnThreads, 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
-  using C = AttnCfg<D, QB, KS, PB, SEPV>;
+  using C = AttnCfg<D, QB, KS, PB, SEPV, QT, PROJ>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   if (smem_u32(smem_raw) & 1023u) {      // the swizzled tiles need 1024-byte alignment
     if (threadIdx.x == 0) atomicOr(p.status, kStatusAttnTimeout);
@@ -148,6 +165,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   uint64_t* oempty = ofinal + 1;      // one phase per item (partial stored)
   uint64_t* mdrain = oempty + 1;
   uint64_t* xmax = mdrain + 1;        // [quarter][parity]: the pair's exchange
+  uint64_t* qtdone = xmax + 8;        // QT: one phase per item (its S products are done)
+  uint64_t* wvfull = qtdone + 1;      // PROJ: the [W_V]^T tile has landed
+  uint64_t* obready = wvfull + 1;     // PROJ: one phase per item (O as bf16 is in TMEM)
+  uint64_t* vdone = obready + 1;      // PROJ: one phase per item (O W_V is done)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + C::oMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + C::oMisc + 4);
 
@@ -163,13 +184,17 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     mbar_init(oempty, kSoftWarps);
     mbar_init(mdrain, 2);
     for (int i = 0; i < 8; ++i) mbar_init(&xmax[i], 2);
+    mbar_init(qtdone, 1);
+    mbar_init(wvfull, 1);
+    mbar_init(obready, kSoftWarps);
+    mbar_init(vdone, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
     prefetch_tmap(&tmQ);
     prefetch_tmap(&tmK);
-    if constexpr (SEPV) prefetch_tmap(&tmV);
+    if constexpr (SEPV || PROJ) prefetch_tmap(&tmV);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, 512);
@@ -188,6 +213,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       const uint64_t stream_policy = policy_evict_first();   // X~ is read once per layer
       uint32_t qi = 0, ki = 0;
       bool ok = true;
+      if constexpr (PROJ) {
+        if (it0 < it1) {
+          mbar_arrive_expect_tx(wvfull, C::kTile);
+          for (int kb = 0; kb < C::KB; ++kb)
+            tma_load_2d(sm + C::oWv + kb * C::kBlock, &tmV, kb * 64, 0, wvfull);
+        }
+      }
       for (int it = it0; ok && it < it1; ++it) {
         const AttnItem item = p.items[it];
         const int qb = qi % QB;
@@ -227,6 +259,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       // at once.)
       for (uint32_t c = ki > KS ? ki - KS : 0; c < ki; ++c) drain_wait(&kfull[c % KS], (c / KS) & 1, 100000000ull);
       for (uint32_t c = qi > QB ? qi - QB : 0; c < qi; ++c) drain_wait(&qfull[c % QB], (c / QB) & 1, 100000000ull);
+      if (PROJ && it0 < it1) drain_wait(wvfull, 0, 100000000ull);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ S issuer
@@ -240,9 +273,22 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         const AttnItem item = p.items[it];
         const int nt = (item.nkeys + 127) >> 7;
         const int qb = qi % QB;
+        if constexpr (QT) {
+          // the previous item's S products read the TMEM copy of its query tile
+          if (qi > 0 && !(ok = bwait(qtdone, (qi - 1) & 1, abort_flag, p.status))) break;
+        }
         if (!(ok = bwait(&qfull[qb], (qi / QB) & 1, abort_flag, p.status))) break;
         tc_fence_after();
         const uint32_t qaddr = sbase + C::oQ + qb * C::kTile;
+        if constexpr (QT) {
+          // 16 features of the 128 rows per copy, into the columns the S
+          // products read as their A operand (2 bf16 per column)
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk)
+            tmem_cp_128x256b(tmem + C::kQt + kk * 8,
+                             sdesc_sw128(qaddr + (kk >> 2) * C::kBlock + (kk & 3) * 32, 16, 1024));
+          mma_commit(&qempty[qb]);           // the shared-memory tile is free once copied
+        }
         for (int j = 0; ok && j < nt; ++j, ++sc, ++ki) {
           const int sb = sc & 1;
           if (!(ok = bwait(&sempty[sb], ((sc >> 1) & 1) ^ 1, abort_flag, p.status))) break;
@@ -251,13 +297,17 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           tc_fence_after();
           const uint32_t kaddr = sbase + C::oK + s * C::kStage;
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk)
-            mma_bf16_ss(tmem + C::kS + sb * 128,
-                        sdesc_sw128(qaddr + (kk >> 2) * C::kBlock + (kk & 3) * 32, 16, 1024),
-                        sdesc_sw128(kaddr + (kk >> 2) * C::kBlock + (kk & 3) * 32, 16, 1024),
-                        idS, kk != 0);
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint64_t kd = sdesc_sw128(kaddr + (kk >> 2) * C::kBlock + (kk & 3) * 32, 16, 1024);
+            if constexpr (QT)
+              mma_bf16_ts(tmem + C::kS + sb * 128, tmem + C::kQt + kk * 8, kd, idS, kk != 0);
+            else
+              mma_bf16_ss(tmem + C::kS + sb * 128,
+                          sdesc_sw128(qaddr + (kk >> 2) * C::kBlock + (kk & 3) * 32, 16, 1024), kd,
+                          idS, kk != 0);
+          }
           mma_commit(&sfull[sb]);
-          if (j + 1 == nt) mma_commit(&qempty[qb]);
+          if (j + 1 == nt) mma_commit(QT ? qtdone : &qempty[qb]);
         }
         ++qi;
       }
@@ -304,6 +354,20 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         }
         if (!ok) break;
         mma_commit(ofinal);
+        if constexpr (PROJ) {
+          // O W_V: A = O as bf16 (written by the softmax warps into the P
+          // columns), B = [W_V]^T K-major; the result overwrites O
+          constexpr uint32_t idV = idesc_bf16(128, D);
+          if (ic == 0 && !(ok = bwait(wvfull, 0, abort_flag, p.status))) break;
+          if (!(ok = bwait(obready, ic & 1, abort_flag, p.status))) break;
+          tc_fence_after();
+          const uint32_t waddr = sbase + C::oWv;
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk)
+            mma_bf16_ts(tmem + C::kO, tmem + C::kPt + kk * 8,
+                        sdesc_sw128(waddr + (kk >> 2) * C::kBlock + (kk & 3) * 32, 16, 1024), idV, kk != 0);
+          mma_commit(vdone);
+        }
       }
       mma_commit(mdrain);
       drain_wait(mdrain, 0, 500000000ull);
@@ -437,6 +501,47 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       tc_fence_after();
       const bool valid = r < item.rows;
       const int64_t g = item.row_base + r;
+      if constexpr (PROJ) {
+        // O (this half's D / 2 features) as bf16 into the P columns: column c
+        // holds features 2c, 2c + 1, the A operand of O W_V
+        {
+          uint32_t pk[32];
+#pragma unroll
+          for (int c = 0; c < 2; ++c) {
+            uint32_t ov[32];
+            tmem_ld32(tmem + lane_off + C::kO + hf * 64 + c * 32, ov);
+            tmem_ld_wait();
+#pragma unroll
+            for (int k = 0; k < 16; ++k)
+              pk[c * 16 + k] = pack_bf16x2(__uint_as_float(ov[2 * k]), __uint_as_float(ov[2 * k + 1]));
+          }
+          tmem_st32(tmem + lane_off + C::kPt + hf * 32, pk);
+          tmem_st_wait();
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(obready);
+        if (!(ok = bwait(vdone, ic & 1, abort_flag, p.status))) break;
+        __syncwarp();
+        tc_fence_after();
+        // the row's head j = r % h keeps columns [j d_h, (j + 1) d_h) of O W_V;
+        // this half holds columns [64 hf, 64 hf + 64)
+        const int j0 = (r % p.h) * p.dh - 64 * hf;     // the head's first column, in this half's terms
+        float* dst = p.pacc + g * p.dh;                // column j0 + c of this half -> dst[c]
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          uint32_t ov[32];
+          tmem_ld32(tmem + lane_off + C::kO + hf * 64 + c * 32, ov);
+          tmem_ld_wait();
+          if (valid) {
+#pragma unroll
+            for (int k = 0; k < 32; ++k) {
+              const int col = c * 32 + k;
+              if (col >= j0 && col < j0 + p.dh) dst[col - j0] = __uint_as_float(ov[k]);
+            }
+          }
+        }
+      } else {
       float* dst = p.pacc + g * D;
 #pragma unroll 1
       for (int cb = hf * (D / 64); cb < (hf + 1) * (D / 64); ++cb) {
@@ -451,6 +556,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                                 __uint_as_float(ov[4 * k + 2]), __uint_as_float(ov[4 * k + 3]));
         }
       }
+      }   // PROJ
       if (valid && hf == 0) {
         p.pm[g] = m_used;
         p.pl[g] = l;
@@ -469,11 +575,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   }
 }
 
-template <int D, int QB, int KS, int PB, bool SEPV = false>
+template <int D, int QB, int KS, int PB, bool SEPV = false, bool QT = false, bool PROJ = false>
 int launch_cfg(stca_handle* H, const CUtensorMap& tmQ, const CUtensorMap& tmK, const AttnParams& p,
                int grid, cudaStream_t s, const CUtensorMap* tmV = nullptr) {
-  using C = AttnCfg<D, QB, KS, PB, SEPV>;
-  auto k = attn_tc_kernel<D, QB, KS, PB, SEPV>;
+  using C = AttnCfg<D, QB, KS, PB, SEPV, QT, PROJ>;
+  auto k = attn_tc_kernel<D, QB, KS, PB, SEPV, QT, PROJ>;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
   if (e != cudaSuccess) return set_error(STCA_ECUDA, std::string("attn_tc smem: ") + cudaGetErrorString(e));
   e = launch_pdl(k, dim3(grid), dim3(kAttnThreads), C::kSmem, s, tmQ, tmK, tmV ? *tmV : tmK, p);
@@ -485,8 +591,12 @@ int launch_cfg(stca_handle* H, const CUtensorMap& tmQ, const CUtensorMap& tmK, c
 
 bool attn_tc_supported(int d) { return d == 64 || d == 128 || d == 256; }
 
+bool attn_tc_proj_supported(const stca_handle* H) {
+  return H->d == 128 && H->wvt != nullptr && H->dh % 4 == 0;
+}
+
 int launch_attn_tc(stca_handle* H, int layer, const AttnItem* items_d, const int32_t* cta_begin_d,
-                   int grid, cudaStream_t s) {
+                   int grid, cudaStream_t s, bool proj) {
   AttnParams p{};
   p.items = items_d;
   p.cta_item_begin = cta_begin_d;
@@ -496,10 +606,16 @@ int launch_attn_tc(stca_handle* H, int layer, const AttnItem* items_d, const int
   p.pl = p.pm + G;
   p.status = H->status_d;
   p.stop_tiles = H->opt_stop_tiles;
+  p.h = H->h;
+  p.dh = H->dh;
   const CUtensorMap& tmK = H->tmXt[layer];
+  if (proj) {
+    if (!attn_tc_proj_supported(H)) return set_error(STCA_EINVAL, "in-kernel W_V projection needs d = 128");
+    return launch_cfg<128, 1, 5, 1, false, true, true>(H, H->tmU, tmK, p, grid, s, &H->tmWvT[layer]);
+  }
   switch (H->d) {
-    case 64: return launch_cfg<64, 2, 10, 2>(H, H->tmU, tmK, p, grid, s);
-    case 128: return launch_cfg<128, 2, 5, 2>(H, H->tmU, tmK, p, grid, s);
+    case 64: return launch_cfg<64, 2, 10, 2, false, true>(H, H->tmU, tmK, p, grid, s);
+    case 128: return launch_cfg<128, 2, 5, 1, false, true>(H, H->tmU, tmK, p, grid, s);
     case 256: return launch_cfg<256, 1, 2, 1>(H, H->tmU, tmK, p, grid, s);
     default: return set_error(STCA_EINVAL, "tensor-core attention needs d in {64, 128, 256}");
   }
@@ -533,8 +649,8 @@ int launch_attn_tc_ws(int d, const CUtensorMap& tmQ, const CUtensorMap& tmK,
   p.pl = p.pm + G;
   p.status = status;
   switch (d) {
-    case 64: return launch_cfg<64, 2, 10, 2>(nullptr, tmQ, tmK, p, grid, s);
-    case 128: return launch_cfg<128, 2, 5, 2>(nullptr, tmQ, tmK, p, grid, s);
+    case 64: return launch_cfg<64, 2, 10, 2, false, true>(nullptr, tmQ, tmK, p, grid, s);
+    case 128: return launch_cfg<128, 2, 5, 1, false, true>(nullptr, tmQ, tmK, p, grid, s);
     case 256: return launch_cfg<256, 1, 2, 1>(nullptr, tmQ, tmK, p, grid, s);
     default: return set_error(STCA_EINVAL, "tensor-core attention needs d in {64, 128, 256}");
   }

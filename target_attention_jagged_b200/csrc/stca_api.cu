@@ -173,6 +173,7 @@ extern "C" void stca_destroy(stca_handle* H) {
   cudaFree(H->whead);
   cudaFree(H->w32head);
   cudaFree(H->wkv);
+  cudaFree(H->wvt);
   cudaFree(H->kv);
   cudaFree(H->lt_ws);
   cudaFree(H->bw_ws);
@@ -394,6 +395,31 @@ extern "C" int stca_init(const stca_weights* w, int d, int h, int r, int M, int 
       if (int rc2 = step_tc_setup(H, sw, hw)) {
         stca_destroy(H);
         return rc2;
+      }
+      if (d == 128) {
+        // [W_V]^T of every layer (output n = j d_h + c of head j, input k):
+        // the B operand of the attention kernel's in-kernel projection
+        std::vector<uint16_t> vt(static_cast<size_t>(M) * d * d);
+        for (int i = 0; i < M; ++i)
+          for (int o = 0; o < d; ++o)
+            for (int k = 0; k < d; ++k) {
+              uint32_t u;
+              memcpy(&u, &sw[i].Wv[static_cast<size_t>(k) * d + o], 4);
+              vt[(static_cast<size_t>(i) * d + o) * d + k] = static_cast<uint16_t>(u >> 16);   // bf16-valued
+            }
+        if (cudaMalloc(&H->wvt, vt.size() * 2) != cudaSuccess ||
+            cudaMemcpy(H->wvt, vt.data(), vt.size() * 2, cudaMemcpyHostToDevice) != cudaSuccess) {
+          cudaGetLastError();
+          stca_destroy(H);
+          return set_error(STCA_ENOMEM, "W_V upload failed");
+        }
+        for (int i = 0; i < M; ++i)
+          if (int rc2 = make_tmap_bf16_2d(&H->tmWvT[i],
+                                          static_cast<const uint16_t*>(H->wvt) + static_cast<size_t>(i) * d * d,
+                                          d, d, 64, 128)) {
+            stca_destroy(H);
+            return rc2;
+          }
       }
       if (naive_layout(dh).G > 0 && kv_proj_supported(d)) {
         // naive form (Eq. (12)): [W_K | W_V] of every layer, stored transposed
@@ -897,7 +923,7 @@ static int forward_impl(stca_handle* H, const void* targets, const int64_t* targ
   }
   // the two-group kernel (d <= 128, reordered form) merges the split
   // partials itself, counting arrivals per pair and layer
-  const bool pp = path == 2 && !naive && attn_pp_supported(d) && H->opt_attn_kernel != 1;
+  const bool pp = path == 2 && !naive && attn_pp_supported(d) && H->opt_attn_kernel == 2;
   if (int rc = ensure_dev(reinterpret_cast<void**>(&H->part), &H->part_cap,
                           static_cast<size_t>(std::max<int64_t>(H->last_G, 1)) * ((naive ? 64 : d) + 4) *
                               sizeof(float)))
@@ -929,17 +955,24 @@ static int forward_impl(stca_handle* H, const void* targets, const int64_t* targ
     return set_error(STCA_EINVAL, "tensor-core step needs the tensor-core attention, bf16, "
                                   "d in {128, 256} and r d <= 512");
   const bool step_tc = path == 2 && H->step_tc_ready && H->opt_step_path != 1;
+  // proj: the attention kernel projects its rows by W_V itself (o_j = alpha_j
+  // X~ W_V^j, Eqs. (6), (13)), so partials are d_h wide and the step starts
+  // from o_head; STCA_OPT_ATTN_KERNEL = 1 keeps the unprojected rows c_j
+  const bool proj = path == 2 && !naive && !pp && step_tc && H->opt_attn_kernel == 0 &&
+                    attn_tc_proj_supported(H);
   // the tensor-core step merges the split partials itself when every query
   // tile has few enough items; otherwise combine_kernel merges them first
-  const bool fused = !naive && !pp && step_tc && H->last_max_items <= step_tc_max_items() &&
+  const bool fused = !naive && !pp && step_tc &&
+                     H->last_max_items <= (proj ? step_tc_max_items_proj() : step_tc_max_items()) &&
                      H->last_G < (int64_t(1) << 31);
+  const int proj_mode = proj ? (fused ? 2 : 1) : 0;
   NaiveStep ns{NL.G, NL.Tq, reinterpret_cast<const int64_t*>(p + H->off_qbase), H->Ubf};
   const bool head_in_step = zout && step_tc && H->head_tc;
   auto step = [&](int layer, const float* cm) {
     if (step_tc)
       return launch_step_tc(H, layer, targets, T, fused ? nullptr : cm, &plan, H->part, H->last_G,
                             Z, H->Ubf, s, naive ? &ns : nullptr,
-                            head_in_step && layer == H->M - 1 ? zout : nullptr);
+                            head_in_step && layer == H->M - 1 ? zout : nullptr, layer >= 0 ? proj_mode : 0);
     launch_target_step(H, layer, targets, T, plan, cm, Z, s);
     return static_cast<int>(STCA_OK);
   };
@@ -962,7 +995,7 @@ static int forward_impl(stca_handle* H, const void* targets, const int64_t* targ
                             H->last_grid, H->part, H->last_G, H->cbuf,
                             H->attn_cnt + cnt_per_layer * i, H->status_d, H->opt_stop_tiles, s);
       } else if (path == 2) {
-        rc = launch_attn_tc(H, i, items_d, cta_d, H->last_grid, s);
+        rc = launch_attn_tc(H, i, items_d, cta_d, H->last_grid, s, proj);
       } else {
         const void* xti = static_cast<const char*>(H->xt) + layer_bytes * i;
         launch_attn_simt(H, i, xti, items_d, pairs_d, H->last_pairs, plan.toff, s);
@@ -977,7 +1010,8 @@ static int forward_impl(stca_handle* H, const void* targets, const int64_t* targ
         launch_combine_naive(H, plan, H->part, H->last_G, T, H->cbuf, s);
         H->launches++;
       } else if (!fused && !pp) {
-        launch_combine(H, plan, H->part, H->last_G, T, H->cbuf, s);
+        if (proj) launch_combine_proj(H, plan, H->part, H->last_G, T, H->cbuf, s);
+        else launch_combine(H, plan, H->part, H->last_G, T, H->cbuf, s);
         H->launches++;
       }
       rc = step(i, H->cbuf);
@@ -1215,7 +1249,7 @@ extern "C" int stca_set_option(stca_handle* H, int option, int64_t value) {
       H->opt_attn_form = static_cast<int>(value);
       return ok();
     case STCA_OPT_ATTN_KERNEL:
-      if (value < 0 || value > 1) return set_error(STCA_EINVAL, "attention kernel must be 0 or 1");
+      if (value < 0 || value > 2) return set_error(STCA_EINVAL, "attention kernel must be 0, 1 or 2");
       H->opt_attn_kernel = static_cast<int>(value);
       return ok();
     case STCA_OPT_TEST_STOP_TILES:

@@ -110,6 +110,8 @@ struct stca_handle {
   int opt_attn_form = 0;                // 0 reordered (Eq. (13)), 1 naive (Eq. (12)), 2 auto
   bool last_naive = false;              // the last forward ran the naive form
   void* kv = nullptr;       size_t kv_cap = 0;     // naive form: N x 2d bf16, [K | V] per row
+  void* wvt = nullptr;                  // per layer [W_V]^T (all heads), d x d bf16 (K-major), d = 128
+  CUtensorMap tmWvT[16];                // their TMA descriptors (box 64 x 128)
   void* wkv = nullptr;                  // naive form: per layer [W_K | W_V]^T, 2d x d bf16 (K-major)
   CUtensorMap tmWkv[16];                // their TMA descriptors (box 64 inputs x 256 outputs)
   void* lt = nullptr;                   // cuBLASLt handle (naive-form projection)
@@ -200,6 +202,10 @@ struct StepPlan {
 // Per-target step (target_step.cu)
 void launch_combine(const stca_handle* H, const StepPlan& plan, const float* part, int64_t G,
                     int64_t T, float* out, cudaStream_t s);
+// The same merge of d_h-wide partials already projected by W_V (the attention
+// kernel's in-kernel projection): out = o_head, T x d.
+void launch_combine_proj(const stca_handle* H, const StepPlan& plan, const float* part, int64_t G,
+                         int64_t T, float* out, cudaStream_t s);
 // Naive form: per-head outputs o_head (T x d fp32) from 64-wide partials.
 void launch_combine_naive(const stca_handle* H, const StepPlan& plan, const float* part, int64_t G,
                           int64_t T, float* out, cudaStream_t s);
@@ -228,6 +234,7 @@ int step_tc_setup(stca_handle* H, const std::vector<StepHostW>& layers, const He
 // partials (part: G x d accumulators, then G maxima, G sums) inside the step;
 // that needs at most step_tc_max_items() items per (request, query tile).
 int step_tc_max_items();
+int step_tc_max_items_proj();
 // The prediction head of Eq. (9) alone on the tensor cores, from Z (T x M x d).
 int launch_step_tc_head(const stca_handle* H, const void* targets, int64_t T, const float* Z, float* zout,
                         cudaStream_t s);
@@ -239,10 +246,14 @@ struct NaiveStep {
   const int64_t* qbase;     // device, R + 1
   uint16_t* upk;            // device, [rows x 64] bf16
 };
+// proj: the attention already projected its rows by W_V (d_h-wide partials of
+// o_j): 1 cmerged holds the merged o_head (T x d); 2 cmerged is NULL and the
+// step merges the partials (part) itself, at most step_tc_max_items_proj()
+// items per query row.
 int launch_step_tc(const stca_handle* H, int layer, const void* targets, int64_t T,
                    const float* cmerged, const StepPlan* plan, const float* part, int64_t G,
                    float* Z, uint16_t* Ubf, cudaStream_t s, const NaiveStep* naive = nullptr,
-                   float* zout = nullptr);
+                   float* zout = nullptr, int proj = 0);
 
 // Host-side attention work plan (stca_api.cu).
 struct PlanHost {
@@ -296,8 +307,11 @@ int launch_attn_bw_tc(int d, const CUtensorMap& tmQ, const CUtensorMap& tmC, con
 
 // Tensor-core attention (attn_tc.cu)
 bool attn_tc_supported(int d);
+// proj: the kernel also projects each item's rows by W_V (d = 128; [W_V]^T
+// of the layer from H->tmWvT) and writes d_h-wide partials of o_j.
+bool attn_tc_proj_supported(const stca_handle* H);
 int launch_attn_tc(stca_handle* H, int layer, const AttnItem* items_d, const int32_t* cta_begin_d,
-                   int grid, cudaStream_t s);
+                   int grid, cudaStream_t s, bool proj = false);
 int launch_attn_tc_naive(stca_handle* H, const AttnItem* items_d, const int32_t* cta_begin_d,
                          int grid, cudaStream_t s);
 

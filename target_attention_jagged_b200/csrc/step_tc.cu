@@ -180,6 +180,8 @@ struct StepTcArgs {
   uint16_t* upk;                // packed query rows [rows x 64] bf16
   float* zout;                  // prediction head z (T x d) when the last layer runs it, or NULL
   int head_only;                // the head alone: its operand [o(1) .. o(M) | x_t] all from Z
+  int proj;                     // the attention projected its rows by W_V already: 1 cmerged
+                                // is o_head (T x d, merged); 2 merge the d_h-wide partials here
 };
 
 // Shared memory, in bytes (1024-aligned base): the A-tile ring, then the
@@ -198,6 +200,9 @@ struct StepLayout {
 // combine kernel (spread over every SM) takes to read and merge them, so the
 // host keeps that kernel then.
 constexpr int kMaxItems = 2;
+// With partials already projected by W_V (d_h floats per row) the merge reads
+// d / d_h times less, and up to kCwItems items per row are merged here.
+constexpr int kCwItems = 8;
 
 __host__ __device__ inline StepLayout step_layout(int d, int rd, int M, int h, int nring) {
   StepLayout L;
@@ -210,7 +215,7 @@ __host__ __device__ inline StepLayout step_layout(int d, int rd, int M, int h, i
   L.scr = L.bQ + (d / 64) * kBTile;
   L.red = L.scr + kTgt * d * 4;
   L.cw = L.red + 2 * 2 * 4 * 8 * 4;              // [2 stats][2 halves][4 quarters][8 targets]
-  L.bar = L.cw + kTgt * h * (kMaxItems * 8 + 4);
+  L.bar = L.cw + kTgt * h * (kCwItems * 8 + 4);
   L.bar = (L.bar + 7) & ~7u;
   L.total = L.bar + (2 * kMaxRing + 4) * 8 + 16;
   return L;
@@ -364,8 +369,8 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_tc_kernel(const StepTcAr
     bool ok = true;
     const int nq = kTgt * h;                  // query rows of this CTA
     int32_t* cw_g = reinterpret_cast<int32_t*>(sm + Y.cw);
-    float* cw_f = reinterpret_cast<float*>(cw_g + nq * kMaxItems);
-    int32_t* cw_n = reinterpret_cast<int32_t*>(cw_f + nq * kMaxItems);
+    float* cw_f = reinterpret_cast<float*>(cw_g + nq * kCwItems);
+    int32_t* cw_n = reinterpret_cast<int32_t*>(cw_f + nq * kCwItems);
     if (L >= 0 && a.cmerged == nullptr && !a.head_only) {
       // split combine of Eq. (13)'s alpha_j X~: c_j = sum_w 2^(m_w - m) acc_w / L,
       // L = sum_w 2^(m_w - m) l_w, over the items w that cover query row (t, j)
@@ -379,27 +384,27 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_tc_kernel(const StepTcAr
           const int64_t mt = qrow / P.mtile_rows, row = qrow - mt * P.mtile_rows;
           const int pair = P.req_pair_begin[r] + static_cast<int>(mt);
           const int w0 = P.pair_item_begin[pair];
-          n = P.pair_item_begin[pair + 1] - w0;
-          float mw[kMaxItems], lw[kMaxItems], mx = -INFINITY;
+          n = min(P.pair_item_begin[pair + 1] - w0, kCwItems);   // the host keeps n <= kCwItems
+          float mw[kCwItems], lw[kCwItems], mx = -INFINITY;
 #pragma unroll
-          for (int w = 0; w < kMaxItems; ++w)
+          for (int w = 0; w < kCwItems; ++w)
             if (w < n) {
               const int64_t g = P.items[w0 + w].row_base + row;
-              cw_g[qi * kMaxItems + w] = static_cast<int32_t>(g);
+              cw_g[qi * kCwItems + w] = static_cast<int32_t>(g);
               mw[w] = a.pm[g];
               lw[w] = a.pl[g];
               mx = fmaxf(mx, mw[w]);
             }
           float ls = 0.f;
 #pragma unroll
-          for (int w = 0; w < kMaxItems; ++w)
+          for (int w = 0; w < kCwItems; ++w)
             if (w < n) {
               mw[w] = exp2f(mw[w] - mx);
               ls = fmaf(lw[w], mw[w], ls);
             }
 #pragma unroll
-          for (int w = 0; w < kMaxItems; ++w)
-            if (w < n) cw_f[qi * kMaxItems + w] = mw[w] / ls;
+          for (int w = 0; w < kCwItems; ++w)
+            if (w < n) cw_f[qi * kCwItems + w] = mw[w] / ls;
         }
         cw_n[qi] = n;
       }
@@ -437,7 +442,21 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_tc_kernel(const StepTcAr
       }
       if (a.head_only) {
         // nothing more: the head's operand is complete
-      } else if (a.naive) {
+      } else if (a.proj == 2) {
+        // o_head[t][j d_h + c] = sum_w f_w po_w[c]: the items' rows, already
+        // projected by W_V^j in the attention, merged into the B operand of W_O
+        const int dhh = a.dh, nqd = nq * dhh;
+        for (int e = tid; e < nqd; e += 32 * kWorkers) {
+          const int qi = e / dhh, c = e - qi * dhh;
+          const int t = qi / h, j = qi - t * h;
+          const int n = cw_n[qi];
+          float acc = 0.f;
+          for (int w = 0; w < n; ++w)
+            acc = fmaf(cw_f[qi * kCwItems + w],
+                       __ldg(a.pacc + static_cast<int64_t>(cw_g[qi * kCwItems + w]) * dhh + c), acc);
+          put_b1(bufs[kO], t, j * dhh + c, acc);           // targets past nb: n = 0
+        }
+      } else if (a.naive || a.proj == 1) {
         // naive form: the per-head outputs o_head[t] (already alpha V per head)
         // are the B operand of W_O as they are
         const int d8 = d / 8;
@@ -512,9 +531,9 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_tc_kernel(const StepTcAr
 #pragma unroll
             for (int w = 0; w < kMaxItems; ++w)
               if (w < n) {
-                const float f = cw_f[q * kMaxItems + w];
+                const float f = cw_f[q * kCwItems + w];
                 const float4 v = __ldg(reinterpret_cast<const float4*>(
-                    a.pacc + static_cast<int64_t>(cw_g[q * kMaxItems + w]) * d + koff));
+                    a.pacc + static_cast<int64_t>(cw_g[q * kCwItems + w]) * d + koff));
                 cv[i].x = fmaf(f, v.x, cv[i].x);
                 cv[i].y = fmaf(f, v.y, cv[i].y);
                 cv[i].z = fmaf(f, v.z, cv[i].z);
@@ -602,21 +621,35 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_tc_kernel(const StepTcAr
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
             const float gg = __uint_as_float(g[j]);
-            hv[j] = __uint_as_float(u[j]) * gg / (1.0f + __expf(-gg));
+            hv[j] = __uint_as_float(u[j]) * __fdividef(gg, 1.0f + __expf(-gg));
           }
           put_b8(bufs[kD], 128 * p + 32 * q4 + lane, t8, hv, lane);
         }
       } else {
-        for (int m = 0; m < G.mb; ++m) {
-          uint32_t r[8];
-          tmem_ld8(tmem + lane_base + m * kTgt + t8, r);
-          tmem_ld_wait();
+        // at most two blocks: the loops over m are unrolled so that vals stays in registers
 #pragma unroll
-          for (int j = 0; j < 8; ++j) vals[m][j] = __uint_as_float(r[j]);
+        for (int m = 0; m < 2; ++m) {
+          if (m < G.mb) {
+            uint32_t r[8];
+            tmem_ld8(tmem + lane_base + m * kTgt + t8, r);
+            tmem_ld_wait();
+#pragma unroll
+            for (int j = 0; j < 8; ++j) vals[m][j] = __uint_as_float(r[j]);
+          }
         }
         if (kind == kD && L < 0) {
           // LayerNorm of Eq. (3) over the d features of each target column:
-          // features are spread over lanes, lane quarters and blocks
+          // features are spread over lanes, lane quarters and blocks; the
+          // scale and shift of this thread's features are loaded first, so
+          // they are in flight during the reductions
+          float lg[2], lb[2];
+#pragma unroll
+          for (int m = 0; m < 2; ++m) {
+            const int f = 128 * m + 32 * q4 + lane;
+            lg[m] = m < G.mb ? __ldg(a.q_ln_g + f) : 0.f;
+            lb[m] = m < G.mb ? __ldg(a.q_ln_b + f) : 0.f;
+          }
+          const float inv_d = 1.0f / d;
           float s[8];
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
@@ -631,7 +664,7 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_tc_kernel(const StepTcAr
           for (int j = 0; j < 8; ++j) {
             float tot = 0.f;
             for (int qq = 0; qq < 4; ++qq) tot += red[((0 * 2 + (wid >> 2)) * 4 + qq) * 8 + j];
-            mean[j] = tot / d;
+            mean[j] = tot * inv_d;
             float e0 = vals[0][j] - mean[j];
             s2[j] = e0 * e0;
             if (G.mb > 1) { const float e1 = vals[1][j] - mean[j]; s2[j] = fmaf(e1, e1, s2[j]); }
@@ -644,11 +677,10 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_tc_kernel(const StepTcAr
           for (int j = 0; j < 8; ++j) {
             float tot = 0.f;
             for (int qq = 0; qq < 4; ++qq) tot += red[((1 * 2 + (wid >> 2)) * 4 + qq) * 8 + j];
-            const float rstd = rsqrtf(tot / d + 1e-5f);
-            for (int m = 0; m < G.mb; ++m) {
-              const int f = 128 * m + 32 * q4 + lane;
-              vals[m][j] = (vals[m][j] - mean[j]) * rstd * a.q_ln_g[f] + a.q_ln_b[f];
-            }
+            const float rstd = rsqrtf(tot * inv_d + 1e-5f);
+#pragma unroll
+            for (int m = 0; m < 2; ++m)
+              if (m < G.mb) vals[m][j] = (vals[m][j] - mean[j]) * rstd * lg[m] + lb[m];
           }
         }
         for (int m = 0; m < G.mb; ++m) {
@@ -770,6 +802,7 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_tc_kernel(const StepTcAr
 // q(layer+2) and its u; layer = M-1: output only.  Writes the bf16 query rows
 // scaled by log2(e) / sqrt(d_h) (the tensor-core attention's units).
 int step_tc_max_items() { return kMaxItems; }
+int step_tc_max_items_proj() { return kCwItems; }
 
 // The prediction head of Eq. (9) alone, for T targets whose Z (T x M x d) is
 // given: one launch of the step kernel with the head's three products.
@@ -812,7 +845,8 @@ int launch_step_tc_head(const stca_handle* H, const void* targets, int64_t T, co
 
 int launch_step_tc(const stca_handle* H, int layer, const void* targets, int64_t T,
                    const float* cmerged, const StepPlan* plan, const float* part, int64_t G,
-                   float* Z, uint16_t* Ubf, cudaStream_t s, const NaiveStep* naive, float* zout) {
+                   float* Z, uint16_t* Ubf, cudaStream_t s, const NaiveStep* naive, float* zout,
+                   int proj) {
   if (T <= 0) return STCA_OK;
   if (!H->step_tc_ready) return set_error(STCA_ESTATE, "tensor-core step weights are not set up");
   const int M = H->M;
@@ -831,6 +865,9 @@ int launch_step_tc(const stca_handle* H, int layer, const void* targets, int64_t
     a.pl = a.pm + G;
   }
   if (plan) a.plan = *plan;
+  if (proj < 0 || proj > 2 || (proj && (naive || (proj == 1) != (cmerged != nullptr))))
+    return set_error(STCA_EINVAL, "tensor-core step: bad projected-input mode");
+  a.proj = layer >= 0 ? proj : 0;
   if (naive) {
     if (!plan || (layer >= 0 && !cmerged))
       return set_error(STCA_EINVAL, "tensor-core step: the naive form needs o_head and the plan");

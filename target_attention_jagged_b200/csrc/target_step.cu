@@ -642,6 +642,18 @@ void launch_combine(const stca_handle* H, const StepPlan& plan, const float* par
                  dim3(kCombineThreads), 0, s, plan, pacc, pm, pl, out, H->d, H->h, nq);
 }
 
+void launch_combine_proj(const stca_handle* H, const StepPlan& plan, const float* part, int64_t G,
+                         int64_t T, float* out, cudaStream_t s) {
+  if (T <= 0) return;
+  // rows d_h wide: row t h + j of the merged output is o_head[t][j d_h ..]
+  const float* pacc = part;
+  const float* pm = part + G * H->d;
+  const float* pl = pm + G;
+  const int64_t nq = T * H->h;
+  tc::launch_pdl(combine_kernel, dim3(static_cast<unsigned>((nq + kCombineRows - 1) / kCombineRows)),
+                 dim3(kCombineThreads), 0, s, plan, pacc, pm, pl, out, H->dh, H->h, nq);
+}
+
 void launch_combine_naive(const stca_handle* H, const StepPlan& plan, const float* part, int64_t G,
                           int64_t T, float* out, cudaStream_t s) {
   if (T <= 0) return;

@@ -234,6 +234,13 @@ __device__ __forceinline__ void tmem_st_wait() {
 }
 
 // Arrive once on `bar` when every MMA this thread issued so far has completed.
+// Copy 128 rows x 256 bits (16 bf16 per row) from a shared-memory matrix, as
+// described by a matrix descriptor, to TMEM: row r to lane r, 8 columns from
+// taddr.  Ordered with the thread's later MMAs (one pipeline, issue order).
+__device__ __forceinline__ void tmem_cp_128x256b(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.128x256b [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
 __device__ __forceinline__ void mma_commit(uint64_t* bar) {
   asm volatile(
       "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(

@@ -15,7 +15,7 @@ from tests.gpu_helpers import TOL, normwise_err, storage_weights, to_device
 pytestmark = pytest.mark.gpu
 
 
-@pytest.mark.parametrize("kernel,d,h", [(0, 128, 8), (1, 128, 8), (1, 256, 8), (0, 64, 4)])
+@pytest.mark.parametrize("kernel,d,h", [(0, 128, 8), (2, 128, 8), (1, 256, 8), (0, 64, 4), (2, 64, 4)])
 def test_attention_gives_up_and_recovers(gpu, kernel, d, h):
     import torch
     import target_attention_jagged_b200 as S

@@ -243,21 +243,25 @@ def test_tensor_core_step_rejected_when_unsupported(gpu):
 
 
 # ------------------------------------------------------------ the two tensor-core attention kernels
-# 0: the two-group kernel (d <= 128), which merges split partials itself;
-# 1: the split-softmax kernel followed by the split combine.
+# 0: the library's choice: for d = 128 the split-softmax kernel projects its
+#    rows by W_V itself, and the step (or, with many items per row, the
+#    combine kernel) merges the d_h-wide partials;
+# 1: the split-softmax kernel followed by the split combine of the rows c_j;
+# 2: the two-group kernel (d <= 128), which merges split partials itself.
 
-KERNEL_TWO_GROUP, KERNEL_SPLIT_SOFTMAX = 0, 1
+KERNEL_AUTO, KERNEL_SPLIT_SOFTMAX, KERNEL_TWO_GROUP = 0, 1, 2
+ALL_KERNELS = [KERNEL_AUTO, KERNEL_SPLIT_SOFTMAX, KERNEL_TWO_GROUP]
 
 
-@pytest.mark.parametrize("kernel", [KERNEL_TWO_GROUP, KERNEL_SPLIT_SOFTMAX])
-@pytest.mark.parametrize("d,h", [(128, 8), (64, 4), (128, 2)])
+@pytest.mark.parametrize("kernel", ALL_KERNELS)
+@pytest.mark.parametrize("d,h", [(128, 8), (64, 4), (128, 2), (128, 1)])
 def test_tc_kernels_ragged(gpu, kernel, d, h):
     wl = make_workload(lengths=EDGE_L, targets=EDGE_T, d=d, h=h, M=2, r=2, dtype="bf16",
                        seed=400 + d + h)
     check_full(wl, run_gpu(wl, gpu, attn_path=ATTN_TC, attn_kernel=kernel))
 
 
-@pytest.mark.parametrize("kernel", [KERNEL_TWO_GROUP, KERNEL_SPLIT_SOFTMAX])
+@pytest.mark.parametrize("kernel", ALL_KERNELS)
 @pytest.mark.parametrize("split", [0, 128, 384])
 def test_tc_kernels_split_merge(gpu, kernel, split):
     """Pairs cut into many items (one 20k-key request over every CTA, a second
@@ -268,7 +272,7 @@ def test_tc_kernels_split_merge(gpu, kernel, split):
     check_full(wl, run_gpu(wl, gpu, attn_path=ATTN_TC, split=split, attn_kernel=kernel))
 
 
-@pytest.mark.parametrize("kernel", [KERNEL_TWO_GROUP, KERNEL_SPLIT_SOFTMAX])
+@pytest.mark.parametrize("kernel", ALL_KERNELS)
 def test_tc_kernels_sharp_softmax(gpu, kernel):
     wl = make_workload(lengths=[3000, 900, 130], targets=[4, 3, 1], d=128, h=4, M=2, r=2,
                        dtype="bf16", seed=411)
@@ -286,3 +290,6 @@ def test_tc_kernels_agree_on_c3(gpu):
     check_sampled(wl, a, 2, seed=3)
     b = run_gpu(wl, gpu, attn_kernel=KERNEL_SPLIT_SOFTMAX)
     assert normwise_err(a, b) <= 2e-2
+    c = run_gpu(wl, gpu, attn_kernel=KERNEL_AUTO)
+    check_sampled(wl, c, 2, seed=4)
+    assert normwise_err(c, b) <= 2e-2
