@@ -55,6 +55,13 @@ struct AttnParams {
   int* status;
   int stop_tiles;                  // > 0: the loader stops after this many key tiles (test hook)
   int h, dh;                       // PROJ: heads and head width (query row r is head r % h)
+  // PROJ with qslot: partials are kept per (query row, item of its pair), at
+  // most kQslots items per pair: row q's item w at pacc[(q kQslots + w) d_h],
+  // its (m, l) at qml[(q kQslots + w) 2], and the pair's item count at qn[q]
+  int qslot;
+  const int32_t* pair_item_begin;  // pairs + 1
+  float* qml;
+  int* qn;
 };
 
 // P_TMEM: P lives in TMEM (packed bf16, 64 columns per buffer) and the P X~
@@ -107,6 +114,13 @@ constexpr int kSoftWarps = 8;               // two per TMEM lane quarter
 constexpr int kPvWarp = 2 + kSoftWarps;     // issues the P X~ products
 constexpr int kAttnThreads = 32 * (kPvWarp + 1);
 constexpr float kRescaleThreshold = 8.0f;   // log2 units
+#ifndef STCA_TC_FMA_PAIRS
+#define STCA_TC_FMA_PAIRS 1
+#endif
+// Of every 4 key pairs, this many take exp2 on the FMA pipe (the degree-3
+// polynomial) and the rest the MUFU; at c3 one in four measured best (forward
+// 0.232 ms, against 0.243 with none and 0.234 with two).
+constexpr int kFmaPairs = STCA_TC_FMA_PAIRS;
 
 __device__ __forceinline__ bool bwait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
                                       int* status) {
@@ -425,11 +439,14 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
             for (int k = 0; k < 32; ++k)
               if (cb * 32 + k >= nvalid) sv[cb][k] = __float_as_uint(-INFINITY);
         }
-        float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+        float m4[4];
 #pragma unroll
-        for (int cb = 0; cb < 2; ++cb)
+        for (int c = 0; c < 4; ++c) {            // 4 chains of 16 keys, two keys per 3-input max
+          const uint32_t* v = &sv[c >> 1][(c & 1) * 16];
+          m4[c] = fmaxf(__uint_as_float(v[0]), __uint_as_float(v[1]));
 #pragma unroll
-          for (int k = 0; k < 32; ++k) m4[k & 3] = fmaxf(m4[k & 3], __uint_as_float(sv[cb][k]));
+          for (int k = 2; k < 16; k += 2) m4[c] = sx::max3(m4[c], __uint_as_float(v[k]), __uint_as_float(v[k + 1]));
+        }
         const float mloc = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
         const float mx = fmaxf(mloc, swap_with_pair(mloc, ok));
         if (!ok) break;
@@ -438,22 +455,32 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         const float corr = resc ? ex2(m_used - m_new) : 1.f;
         l *= corr;
         m_used = m_new;
+        // pairs of keys: the subtraction and the sums in packed f32x2 form;
+        // kFmaPairs of every 4 pairs take exp2 on the FMA pipe (d <= 128)
         uint32_t pk[32];
-        float ls[4] = {0.f, 0.f, 0.f, 0.f};
+        const uint64_t negm = sx::f2(-m_new, -m_new);
+        uint64_t ls2[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
         for (int cb = 0; cb < 2; ++cb)
 #pragma unroll
           for (int k = 0; k < 32; k += 2) {
-            const float p0 = ex2(__uint_as_float(sv[cb][k]) - m_new);      // exp2(-inf) = 0
-            const float x1 = __uint_as_float(sv[cb][k + 1]) - m_new;
-            // with d <= 128, 3 in 8 on the FMA pipe (MUFU-bound; 1 in 4 and 1 in 2
-            // measured slower); with d = 256 the softmax is bound by instruction
-            // issue, and all go to the MUFU
-            const float p1 = (C::P_TMEM && (k & 6) != 0) ? ex2_fma(x1) : ex2(x1);
-            ls[(k >> 1) & 3] += p0 + p1;
+            const uint64_t x = sx::f2_add(sx::f2(__uint_as_float(sv[cb][k]), __uint_as_float(sv[cb][k + 1])), negm);
+            float x0, x1, p0, p1;
+            sx::f2_split(x, x0, x1);
+            if (C::P_TMEM && ((k >> 1) & 3) < kFmaPairs) {
+              sx::ex2_fma2(x0, x1, p0, p1);
+            } else {
+              p0 = ex2(x0);                      // exp2(-inf) = 0
+              p1 = ex2(x1);
+            }
+            ls2[(k >> 1) & 3] = sx::f2_add(ls2[(k >> 1) & 3], sx::f2(p0, p1));
             pk[(cb * 32 + k) >> 1] = pack_bf16x2(p0, p1);
           }
-        l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+        {
+          float a0, a1;
+          sx::f2_split(sx::f2_add(sx::f2_add(ls2[0], ls2[1]), sx::f2_add(ls2[2], ls2[3])), a0, a1);
+          l += a0 + a1;
+        }
         const int pb = pc % PB;
         if (!(ok = bwait(&pempty[pb], ((pc / PB) & 1) ^ 1, abort_flag, p.status))) break;
         __syncwarp();
@@ -527,7 +554,18 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         // the row's head j = r % h keeps columns [j d_h, (j + 1) d_h) of O W_V;
         // this half holds columns [64 hf, 64 hf + 64)
         const int j0 = (r % p.h) * p.dh - 64 * hf;     // the head's first column, in this half's terms
-        float* dst = p.pacc + g * p.dh;                // column j0 + c of this half -> dst[c]
+        int64_t slot = g;
+        if (p.qslot) {
+          const int w0 = p.pair_item_begin[item.pair];
+          const int64_t qrow = item.qrow0 + r;
+          slot = qrow * kQslots + (it - w0);
+          if (valid && hf == 0) {
+            p.qn[qrow] = p.pair_item_begin[item.pair + 1] - w0;
+            p.qml[slot * 2] = m_used;
+            p.qml[slot * 2 + 1] = l;
+          }
+        }
+        float* dst = p.pacc + slot * p.dh;             // column j0 + c of this half -> dst[c]
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
           uint32_t ov[32];
@@ -557,7 +595,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         }
       }
       }   // PROJ
-      if (valid && hf == 0) {
+      if (valid && hf == 0 && !(PROJ && p.qslot)) {
         p.pm[g] = m_used;
         p.pl[g] = l;
       }
@@ -596,7 +634,7 @@ bool attn_tc_proj_supported(const stca_handle* H) {
 }
 
 int launch_attn_tc(stca_handle* H, int layer, const AttnItem* items_d, const int32_t* cta_begin_d,
-                   int grid, cudaStream_t s, bool proj) {
+                   int grid, cudaStream_t s, bool proj, const QslotBufs* qs) {
   AttnParams p{};
   p.items = items_d;
   p.cta_item_begin = cta_begin_d;
@@ -608,6 +646,14 @@ int launch_attn_tc(stca_handle* H, int layer, const AttnItem* items_d, const int
   p.stop_tiles = H->opt_stop_tiles;
   p.h = H->h;
   p.dh = H->dh;
+  if (qs) {
+    if (!proj) return set_error(STCA_EINVAL, "per-row partial slots need the in-kernel projection");
+    p.qslot = 1;
+    p.pair_item_begin = qs->pair_item_begin;
+    p.pacc = qs->pacc;
+    p.qml = qs->qml;
+    p.qn = qs->qn;
+  }
   const CUtensorMap& tmK = H->tmXt[layer];
   if (proj) {
     if (!attn_tc_proj_supported(H)) return set_error(STCA_EINVAL, "in-kernel W_V projection needs d = 128");

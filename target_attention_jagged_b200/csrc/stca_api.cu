@@ -924,9 +924,13 @@ static int forward_impl(stca_handle* H, const void* targets, const int64_t* targ
   // the two-group kernel (d <= 128, reordered form) merges the split
   // partials itself, counting arrivals per pair and layer
   const bool pp = path == 2 && !naive && attn_pp_supported(d) && H->opt_attn_kernel == 2;
-  if (int rc = ensure_dev(reinterpret_cast<void**>(&H->part), &H->part_cap,
-                          static_cast<size_t>(std::max<int64_t>(H->last_G, 1)) * ((naive ? 64 : d) + 4) *
-                              sizeof(float)))
+  // the split partials: G item rows of d (naive form: 64) floats plus (m, l);
+  // or, with the in-kernel projection, kQslots slots of d_h + 2 floats per
+  // query row plus its item count
+  const size_t part_floats =
+      std::max(static_cast<size_t>(std::max<int64_t>(H->last_G, 1)) * ((naive ? 64 : d) + 4),
+               urows * (kQslots * (static_cast<size_t>(H->dh) + 2) + 1));
+  if (int rc = ensure_dev(reinterpret_cast<void**>(&H->part), &H->part_cap, part_floats * sizeof(float)))
     return rc;
   const size_t cnt_per_layer = static_cast<size_t>(std::max<int64_t>(H->last_npairs, 1)) * 8;
   if (pp) {
@@ -966,13 +970,23 @@ static int forward_impl(stca_handle* H, const void* targets, const int64_t* targ
                      H->last_max_items <= (proj ? step_tc_max_items_proj() : step_tc_max_items()) &&
                      H->last_G < (int64_t(1) << 31);
   const int proj_mode = proj ? (fused ? 2 : 1) : 0;
+  // proj with the step's merge: partials in per-row slots (fused implies at
+  // most step_tc_max_items_proj() = kQslots items per pair)
+  QslotBufs qs{};
+  if (proj_mode == 2) {
+    qs.pair_item_begin = plan.pair_item_begin;
+    qs.pacc = H->part;
+    qs.qml = H->part + urows * kQslots * H->dh;
+    qs.qn = reinterpret_cast<int*>(qs.qml + urows * kQslots * 2);
+  }
   NaiveStep ns{NL.G, NL.Tq, reinterpret_cast<const int64_t*>(p + H->off_qbase), H->Ubf};
   const bool head_in_step = zout && step_tc && H->head_tc;
   auto step = [&](int layer, const float* cm) {
     if (step_tc)
       return launch_step_tc(H, layer, targets, T, fused ? nullptr : cm, &plan, H->part, H->last_G,
                             Z, H->Ubf, s, naive ? &ns : nullptr,
-                            head_in_step && layer == H->M - 1 ? zout : nullptr, layer >= 0 ? proj_mode : 0);
+                            head_in_step && layer == H->M - 1 ? zout : nullptr, layer >= 0 ? proj_mode : 0,
+                            proj_mode == 2 ? &qs : nullptr);
     launch_target_step(H, layer, targets, T, plan, cm, Z, s);
     return static_cast<int>(STCA_OK);
   };
@@ -995,7 +1009,7 @@ static int forward_impl(stca_handle* H, const void* targets, const int64_t* targ
                             H->last_grid, H->part, H->last_G, H->cbuf,
                             H->attn_cnt + cnt_per_layer * i, H->status_d, H->opt_stop_tiles, s);
       } else if (path == 2) {
-        rc = launch_attn_tc(H, i, items_d, cta_d, H->last_grid, s, proj);
+        rc = launch_attn_tc(H, i, items_d, cta_d, H->last_grid, s, proj, proj_mode == 2 ? &qs : nullptr);
       } else {
         const void* xti = static_cast<const char*>(H->xt) + layer_bytes * i;
         launch_attn_simt(H, i, xti, items_d, pairs_d, H->last_pairs, plan.toff, s);

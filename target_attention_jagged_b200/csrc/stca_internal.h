@@ -120,7 +120,7 @@ struct stca_handle {
   void* bw_plan = nullptr;  size_t bw_plan_cap = 0;  // attention backward units and statistics
   bool tc_encode_ready = false;
   uint16_t* wstep_tc = nullptr;         // A-tile stream of the tensor-core per-target step
-  std::vector<stca::TcGemm> tcO, tcC, tcUG, tcD, tcQ;   // per layer
+  std::vector<stca::TcGemm> tcO, tcC, tcUG, tcD, tcQ, tcK;   // per layer (tcK: d = 128, h <= 8)
   stca::TcGemm tcZC, tcZUG, tcZD;       // prediction head (Eq. (9)): W_Z, [zW_u | zW_g], zW_d
   bool head_tc = false;
   bool step_tc_ready = false;
@@ -238,6 +238,17 @@ int step_tc_max_items_proj();
 // The prediction head of Eq. (9) alone on the tensor cores, from Z (T x M x d).
 int launch_step_tc_head(const stca_handle* H, const void* targets, int64_t T, const float* Z, float* zout,
                         cudaStream_t s);
+// Partials of the in-kernel projection kept per (query row, item of its pair)
+// (at most kQslots items per pair): row q's item w at pacc[(q kQslots + w) d_h],
+// its (m, l) at qml[(q kQslots + w) 2], the pair's item count at qn[q].  The
+// per-target step then finds a row's partials without the work plan.
+constexpr int kQslots = 8;
+struct QslotBufs {
+  const int32_t* pair_item_begin;
+  float* pacc;
+  float* qml;
+  int* qn;
+};
 // Naive form of the step: `naive` not NULL; cmerged then holds o_head (T x d, the
 // per-head outputs of Eq. (12)), and the query rows of the next layer are written
 // into the packed layout (NaiveLayout) at naive->upk, request r from row qbase[r].
@@ -253,7 +264,7 @@ struct NaiveStep {
 int launch_step_tc(const stca_handle* H, int layer, const void* targets, int64_t T,
                    const float* cmerged, const StepPlan* plan, const float* part, int64_t G,
                    float* Z, uint16_t* Ubf, cudaStream_t s, const NaiveStep* naive = nullptr,
-                   float* zout = nullptr, int proj = 0);
+                   float* zout = nullptr, int proj = 0, const QslotBufs* qs = nullptr);
 
 // Host-side attention work plan (stca_api.cu).
 struct PlanHost {
@@ -311,7 +322,7 @@ bool attn_tc_supported(int d);
 // of the layer from H->tmWvT) and writes d_h-wide partials of o_j.
 bool attn_tc_proj_supported(const stca_handle* H);
 int launch_attn_tc(stca_handle* H, int layer, const AttnItem* items_d, const int32_t* cta_begin_d,
-                   int grid, cudaStream_t s, bool proj = false);
+                   int grid, cudaStream_t s, bool proj = false, const QslotBufs* qs = nullptr);
 int launch_attn_tc_naive(stca_handle* H, const AttnItem* items_d, const int32_t* cta_begin_d,
                          int grid, cudaStream_t s);
 

@@ -42,7 +42,7 @@ constexpr int kWorkers = 8;               // worker warps
 constexpr int kStepThreads = 32 * (2 + kWorkers);
 constexpr uint32_t kATile = 128u * 128u;  // A tile: 128 rows x 64 bf16
 constexpr uint32_t kBTile = kTgt * 128u;  // B tile: 16 rows x 64 bf16
-constexpr int kMaxRing = 8;               // A tiles in flight, at most
+constexpr int kMaxRing = 10;              // A tiles in flight, at most (what fits is used)
 
 // Byte offset of element (row r, column c) of a K-major tile whose rows hold
 // 64 bf16 (128 B) with the 128-byte swizzle: 8-row atoms of 1024 B, the
@@ -112,6 +112,11 @@ int step_tc_setup(stca_handle* H, const std::vector<StepHostW>& layers, const He
   H->tcUG.assign(M, TcGemm());
   H->tcD.assign(M, TcGemm());
   H->tcQ.assign(M, TcGemm());
+  H->tcK.assign(M, TcGemm());
+  // u_j = P_j W_K^j^T on the tensor cores: d = 128 (one feature block) and
+  // 16 h <= 128 (the (target, head) columns of one accumulator)
+  const bool wk_tc = d == 128 && H->h <= 8;
+  std::vector<float> wkt(wk_tc ? static_cast<size_t>(d) * d : 0);
   for (int i = 0; i < M; ++i) {
     const StepHostW& L = layers[i];
     H->tcO[i] = put_tiles(tiles, d, col_blocks(L.Wo, d));
@@ -124,6 +129,12 @@ int step_tc_setup(stca_handle* H, const std::vector<StepHostW>& layers, const He
     H->tcUG[i] = put_tiles(tiles, d, ug);
     H->tcD[i] = put_tiles(tiles, rd, col_blocks(L.qWd, d));
     H->tcQ[i] = put_tiles(tiles, d, col_blocks(L.Wq, d));
+    if (wk_tc) {
+      // as a [inputs x outputs] matrix: input (j, c) = column j d_h + c of W_K, output feature f
+      for (int f = 0; f < d; ++f)
+        for (int k = 0; k < d; ++k) wkt[static_cast<size_t>(k) * d + f] = L.Wk[static_cast<size_t>(f) * d + k];
+      H->tcK[i] = put_tiles(tiles, d, {ColBlock{wkt.data(), d, 0}});
+    }
   }
   if (head.Wz) {
     // prediction head of Eq. (9), run by the last layer's step: W_Z over the
@@ -151,7 +162,10 @@ int step_tc_setup(stca_handle* H, const std::vector<StepHostW>& layers, const He
 // ------------------------------------------------------------------ kernel
 namespace {
 
-enum : int { kO = 0, kC = 1, kUG = 2, kD = 3, kQ = 4, kZ = 5 };   // kZ: the head's down product
+// kZ: the head's down product; kK: u_j = P_j W_K^j^T on the tensor cores,
+// U^T[d features x (target, head)] = [W_K] Pblk, where Pblk (16 h rows x d) holds
+// row (t, j) = P[t] on head j's d_h inputs and zeros elsewhere (Eq. (13))
+enum : int { kO = 0, kC = 1, kUG = 2, kD = 3, kQ = 4, kZ = 5, kK = 6 };
 
 struct StepTcArgs {
   int layer, M, d, h, dh, rd;
@@ -182,6 +196,10 @@ struct StepTcArgs {
   int head_only;                // the head alone: its operand [o(1) .. o(M) | x_t] all from Z
   int proj;                     // the attention projected its rows by W_V already: 1 cmerged
                                 // is o_head (T x d, merged); 2 merge the d_h-wide partials here
+  const float* qml;             // proj 2: the attention's per-row slots (QslotBufs; pacc too)
+  const int* qn;
+  int wk_tc;                    // the W_K products run on the tensor cores (product kind kK)
+  int qtot;                     // A tiles of this launch (kK's Pblk takes the next two ring slots)
 };
 
 // Shared memory, in bytes (1024-aligned base): the A-tile ring, then the
@@ -334,7 +352,9 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_tc_kernel(const StepTcAr
         const TcGemm G = a.g[gi];
         if (!(ok = step_wait(bready, gi & 1, a.status))) break;
         tc_fence_after();
-        const uint32_t bbase = smem_u32(bufs[a.kind[gi]]);
+        const bool wk = a.kind[gi] == kK;
+        const uint32_t bbase = wk ? 0u : smem_u32(bufs[a.kind[gi]]);
+        const uint32_t id = wk ? idesc_bf16(128, kTgt * h) : idesc;
         for (int m = 0; ok && m < G.mb; ++m) {
           const uint32_t acc = tmem + m * kTgt;
           for (int kc = 0; kc < G.kc; ++kc, ++q) {
@@ -342,11 +362,12 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_tc_kernel(const StepTcAr
             if (!(ok = step_wait(&full[s], (q / R) & 1, a.status))) break;
             tc_fence_after();
             const uint32_t aaddr = smem_u32(sm + Y.ring + s * kATile);
-            const uint32_t baddr = bbase + kc * kBTile;
+            // kK: K tile kc of Pblk sits in ring slot (qtot + kc) % R
+            const uint32_t baddr = wk ? smem_u32(sm + Y.ring + ((a.qtot + kc) % R) * kATile) : bbase + kc * kBTile;
 #pragma unroll
             for (int k4 = 0; k4 < 4; ++k4)
               mma_bf16_ss(acc, sdesc_sw128(aaddr + k4 * 32, 16, 1024),
-                          sdesc_sw128(baddr + k4 * 32, 16, 1024), idesc, (kc | k4) != 0);
+                          sdesc_sw128(baddr + k4 * 32, 16, 1024), id, (kc | k4) != 0);
             mma_commit(&empty[s]);
           }
         }
@@ -371,7 +392,54 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_tc_kernel(const StepTcAr
     int32_t* cw_g = reinterpret_cast<int32_t*>(sm + Y.cw);
     float* cw_f = reinterpret_cast<float*>(cw_g + nq * kCwItems);
     int32_t* cw_n = reinterpret_cast<int32_t*>(cw_f + nq * kCwItems);
-    if (L >= 0 && a.cmerged == nullptr && !a.head_only) {
+    // [o(1) .. o(L) | o(L+1): by the output epilogue | x_t] of Eq. (7), or of
+    // the head's Eq. (9) after the last layer: the B operand of W_C (W_Z).
+    // 8 inputs (one 16-byte chunk of a B row) per item, 4 items per thread and
+    // batch.  The first batch's loads are issued before the combine tables are
+    // built and stored after the first product has been released (unless this
+    // operand is the first one, the head alone), so they overlap the tables
+    // and W_O; the output epilogue fills block L.
+    const int wcat8 = (L + 2) * d / 8, d8 = d / 8, ne_cat = L >= 0 ? kTgt * wcat8 : 0;
+    auto concat_load = [&](int e0, uint4 (&v)[4]) {
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int e = e0 + u * 32 * kWorkers;
+        v[u] = make_uint4(0u, 0u, 0u, 0u);
+        if (e >= ne_cat) continue;
+        const int t = e / wcat8, k8 = e - t * wcat8;
+        const int blk = k8 / d8, kk = 8 * (k8 - blk * d8);
+        if (t >= nb || (blk == L && !a.head_only)) continue;
+        if (blk < L || (blk == L && a.head_only)) {
+          const float4* z = reinterpret_cast<const float4*>(a.Z + ((t0 + t) * M + blk) * d + kk);
+          const float4 z0 = z[0], z1 = z[1];
+          v[u] = make_uint4(pack_bf16x2(z0.x, z0.y), pack_bf16x2(z0.z, z0.w),
+                            pack_bf16x2(z1.x, z1.y), pack_bf16x2(z1.z, z1.w));
+        } else {
+          v[u] = *reinterpret_cast<const uint4*>(a.targets + (t0 + t) * d + kk);
+        }
+      }
+    };
+    auto concat_store = [&](int e0, const uint4 (&v)[4]) {
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int e = e0 + u * 32 * kWorkers;
+        if (e >= ne_cat) break;
+        const int t = e / wcat8, k8 = e - t * wcat8;
+        if (k8 / d8 == L && !a.head_only) continue;
+        *reinterpret_cast<uint4*>(bufs[kC] + (8 * k8 >> 6) * kBTile + sw128_off(t, (8 * k8) & 63)) = v[u];
+      }
+    };
+    auto build_concat_rest = [&]() {       // batches after the first
+      for (int e0 = tid + 4 * 32 * kWorkers; e0 < ne_cat; e0 += 4 * 32 * kWorkers) {
+        uint4 v[4];
+        concat_load(e0, v);
+        concat_store(e0, v);
+      }
+    };
+    const bool concat = L >= 0 && (L + 1 < M || a.zout);
+    uint4 cat0[4];
+    if (concat) concat_load(tid, cat0);
+    if (L >= 0 && a.cmerged == nullptr && !a.head_only && a.proj != 2) {
       // split combine of Eq. (13)'s alpha_j X~: c_j = sum_w 2^(m_w - m) acc_w / L,
       // L = sum_w 2^(m_w - m) l_w, over the items w that cover query row (t, j)
       for (int qi = tid; qi < nq; qi += 32 * kWorkers) {
@@ -417,44 +485,72 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_tc_kernel(const StepTcAr
         put_b1(bufs[kUG], t, k, t < nb ? bf2f(a.targets[(t0 + t) * d + k]) : 0.f);
       }
     } else {
-      if (L + 1 < M || a.zout) {
-        // [o(1) .. o(L) | o(L+1): by the output epilogue | x_t] of Eq. (7), or of
-        // the head's Eq. (9) after the last layer
-        // 8 inputs (one 16-byte chunk of a B row) per item
-        const int wcat8 = (L + 2) * d / 8, d8 = d / 8;
-        for (int e = tid; e < kTgt * wcat8; e += 32 * kWorkers) {
-          const int t = e / wcat8, k8 = e - t * wcat8;
-          const int blk = k8 / d8, kk = 8 * (k8 - blk * d8);
-          if (blk == L && !a.head_only) continue;
-          uint4 v = make_uint4(0u, 0u, 0u, 0u);
-          if (t < nb) {
-            if (blk < L || (blk == L && a.head_only)) {
-              const float4* z = reinterpret_cast<const float4*>(a.Z + ((t0 + t) * M + blk) * d + kk);
-              const float4 z0 = z[0], z1 = z[1];
-              v = make_uint4(pack_bf16x2(z0.x, z0.y), pack_bf16x2(z0.z, z0.w),
-                             pack_bf16x2(z1.x, z1.y), pack_bf16x2(z1.z, z1.w));
-            } else {
-              v = *reinterpret_cast<const uint4*>(a.targets + (t0 + t) * d + kk);
-            }
-          }
-          *reinterpret_cast<uint4*>(bufs[kC] + (8 * k8 >> 6) * kBTile + sw128_off(t, (8 * k8) & 63)) = v;
-        }
+      if (concat && a.head_only) {
+        concat_store(tid, cat0);
+        build_concat_rest();
       }
       if (a.head_only) {
         // nothing more: the head's operand is complete
       } else if (a.proj == 2) {
         // o_head[t][j d_h + c] = sum_w f_w po_w[c]: the items' rows, already
         // projected by W_V^j in the attention, merged into the B operand of W_O
-        const int dhh = a.dh, nqd = nq * dhh;
-        for (int e = tid; e < nqd; e += 32 * kWorkers) {
-          const int qi = e / dhh, c = e - qi * dhh;
-          const int t = qi / h, j = qi - t * h;
-          const int n = cw_n[qi];
-          float acc = 0.f;
-          for (int w = 0; w < n; ++w)
-            acc = fmaf(cw_f[qi * kCwItems + w],
-                       __ldg(a.pacc + static_cast<int64_t>(cw_g[qi * kCwItems + w]) * dhh + c), acc);
-          put_b1(bufs[kO], t, j * dhh + c, acc);           // targets past nb: n = 0
+        // a task is 4 columns of one query row (t, j), global row q = (t0 + t) h + j
+        // of the attention's per-row slots: the row's item count, then every
+        // item's (m, l) and 16 bytes of its projected partial, all in flight
+        // at once; the weights 2^(m_w - m) / L are formed here
+        const int dhh = a.dh, c4n = dhh / 4, ntask = nq * c4n;
+        constexpr int kU = 2;
+        for (int e0 = tid; e0 < ntask; e0 += kU * 32 * kWorkers) {
+          int n[kU];
+          int64_t qrow[kU];
+#pragma unroll
+          for (int u = 0; u < kU; ++u) {
+            const int e = e0 + u * 32 * kWorkers;
+            const int qi = e / c4n, t = qi / h;
+            qrow[u] = (t0 + t) * h + (qi - t * h);
+            n[u] = e < ntask && t < nb ? min(a.qn[qrow[u]], kQslots) : 0;
+          }
+          float4 v[kU][kQslots];
+          float2 ml[kU][kQslots];
+#pragma unroll
+          for (int u = 0; u < kU; ++u) {
+            const int e = e0 + u * 32 * kWorkers;
+            const int c4 = e % c4n;
+#pragma unroll
+            for (int w = 0; w < kQslots; ++w) {
+              const int64_t slot = qrow[u] * kQslots + w;
+              v[u][w] = w < n[u] ? __ldg(reinterpret_cast<const float4*>(a.pacc + slot * dhh) + c4)
+                                 : make_float4(0.f, 0.f, 0.f, 0.f);
+              ml[u][w] = w < n[u] ? __ldg(reinterpret_cast<const float2*>(a.qml) + slot) : make_float2(-INFINITY, 0.f);
+            }
+          }
+#pragma unroll
+          for (int u = 0; u < kU; ++u) {
+            const int e = e0 + u * 32 * kWorkers;
+            if (e >= ntask) break;
+            const int qi = e / c4n, c4 = e - qi * c4n;
+            const int t = qi / h, j = qi - t * h;
+            float mx = -INFINITY;
+#pragma unroll
+            for (int w = 0; w < kQslots; ++w) mx = fmaxf(mx, ml[u][w].x);
+            float ls = 0.f;
+            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+            for (int w = 0; w < kQslots; ++w)
+              if (w < n[u]) {
+                const float f = exp2f(ml[u][w].x - mx);
+                ls = fmaf(ml[u][w].y, f, ls);
+                acc.x = fmaf(f, v[u][w].x, acc.x);
+                acc.y = fmaf(f, v[u][w].y, acc.y);
+                acc.z = fmaf(f, v[u][w].z, acc.z);
+                acc.w = fmaf(f, v[u][w].w, acc.w);
+              }
+            const float inv = n[u] > 0 ? 1.0f / ls : 0.f;
+            // 4 bf16 of row t, inputs j d_h + 4 c4 .. + 3 (8 bytes inside one 16-byte chunk)
+            const int k = j * dhh + 4 * c4;
+            *reinterpret_cast<uint2*>(bufs[kO] + (k >> 6) * kBTile + sw128_off(t, k & 63)) =
+                make_uint2(pack_bf16x2(acc.x * inv, acc.y * inv), pack_bf16x2(acc.z * inv, acc.w * inv));
+          }
         }
       } else if (a.naive || a.proj == 1) {
         // naive form: the per-head outputs o_head[t] (already alpha V per head)
@@ -602,16 +698,58 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_tc_kernel(const StepTcAr
     fence_proxy_async_smem();
     __syncwarp();
     if (lane == 0) mbar_arrive(bready);
+    // the W_C operand, while W_O runs (its epilogue's fence covers these stores)
+    if (concat && !a.head_only) {
+      concat_store(tid, cat0);
+      build_concat_rest();
+    }
 
     // ---- epilogues
     for (int gi = 0; gi < a.ng; ++gi) {
       const int kind = a.kind[gi];
       const TcGemm G = a.g[gi];
       if (ok) ok = step_wait(aready, gi & 1, a.status);
+      if (kind == kQ && a.wk_tc) {
+        // Pblk's two ring slots (their last tiles' MMAs are complete): zero
+        // them, then the epilogue below scatters P into its blocks
+        for (int e = tid; e < 2 * static_cast<int>(kATile / 16); e += 32 * kWorkers)
+          *reinterpret_cast<uint4*>(sm + Y.ring + ((a.qtot + e / (kATile / 16)) % R) * kATile +
+                                    (e % (kATile / 16)) * 16) = make_uint4(0u, 0u, 0u, 0u);
+        workers_sync();
+      }
       __syncwarp();
       tc_fence_after();
       float vals[2][8];                       // up to two blocks of 128 features (d <= 256)
-      if (kind == kUG) {
+      if (kind == kK) {
+        // U^T: lane = feature f, column n = t h + j; this warp takes columns
+        // [64 hf, 64 hf + 64) (the rows (t, j) of U for targets t < nb).  The
+        // warp's 64 x 32 block goes through shared memory (Pblk's ring slots,
+        // free once these products are done) so that U's rows are written in
+        // 16-byte pieces
+        const int ncol = kTgt * h, hf = wid >> 2;
+        uint16_t* stg = reinterpret_cast<uint16_t*>(sm + Y.ring + ((a.qtot + (wid >> 2)) % R) * kATile) +
+                        q4 * 64 * 32;                            // [64 rows n][32 features] bf16
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          const int c0 = 64 * hf + 32 * c;
+          if (c0 >= ncol) break;
+          uint32_t v[32];
+          tmem_ld32(tmem + lane_base + c0, v);
+          tmem_ld_wait();
+#pragma unroll
+          for (int k = 0; k < 32; ++k)
+            stg[(32 * c + k) * 32 + lane] = __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(v[k]) * a.uscale));
+        }
+        __syncwarp();
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int ch = lane + 32 * i, row = ch >> 2, part = ch & 3;
+          const int n = 64 * hf + row;
+          if (n < ncol && n / h < nb)
+            *reinterpret_cast<uint4*>(a.Ubf + (t0 * h + n) * static_cast<int64_t>(d) + 32 * q4 + 8 * part) =
+                *reinterpret_cast<const uint4*>(stg + row * 32 + 8 * part);
+        }
+      } else if (kind == kUG) {
         for (int p = 0; p < G.mb / 2; ++p) {
           uint32_t u[8], g[8];
           tmem_ld8(tmem + lane_base + (2 * p) * kTgt + t8, u);
@@ -696,6 +834,12 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_tc_kernel(const StepTcAr
           } else if (kind == kZ) {   // the head's token z of Eq. (9)
             for (int j = 0; j < 8; ++j)
               if (t8 + j < nb) a.zout[(t0 + t8 + j) * d + f] = vals[m][j];
+          } else if (a.wk_tc) {   // kQ: P = q W_Q into Pblk, row t h + f / d_h, column f
+            uint8_t* blk = sm + Y.ring + ((a.qtot + (f >> 6)) % R) * kATile;
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+              *reinterpret_cast<__nv_bfloat16*>(blk + sw128_off((t8 + j) * h + f / dh, f & 63)) =
+                  __float2bfloat16_rn(vals[m][j]);
           } else {   // kQ: P = q W_Q in fp32, as P^T[feature][target] for the W_K products
             float4* dst = reinterpret_cast<float4*>(scr + f * kTgt + t8);
             dst[0] = make_float4(vals[m][0], vals[m][1], vals[m][2], vals[m][3]);
@@ -739,7 +883,7 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_tc_kernel(const StepTcAr
             make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
                        pack_bf16x2(v[6], v[7]));
       }
-    } else if (L + 1 < M) {
+    } else if (L + 1 < M && !a.wk_tc) {
       workers_sync();
       const int hd = h * d;
       for (int b = tid; b < hd / 4; b += 32 * kWorkers) {
@@ -802,7 +946,16 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_tc_kernel(const StepTcAr
 // q(layer+2) and its u; layer = M-1: output only.  Writes the bf16 query rows
 // scaled by log2(e) / sqrt(d_h) (the tensor-core attention's units).
 int step_tc_max_items() { return kMaxItems; }
-int step_tc_max_items_proj() { return kCwItems; }
+
+namespace {
+// the deepest weight ring that fits in shared memory
+int ring_stages(const stca_handle* H, int M) {
+  int nring = kMaxRing;
+  while (nring > 2 && step_layout(H->d, H->rd, M, H->h, nring).total + 1024 > 227u * 1024) --nring;
+  return nring;
+}
+}  // namespace
+int step_tc_max_items_proj() { return kQslots; }
 
 // The prediction head of Eq. (9) alone, for T targets whose Z (T x M x d) is
 // given: one launch of the step kernel with the head's three products.
@@ -846,7 +999,7 @@ int launch_step_tc_head(const stca_handle* H, const void* targets, int64_t T, co
 int launch_step_tc(const stca_handle* H, int layer, const void* targets, int64_t T,
                    const float* cmerged, const StepPlan* plan, const float* part, int64_t G,
                    float* Z, uint16_t* Ubf, cudaStream_t s, const NaiveStep* naive, float* zout,
-                   int proj) {
+                   int proj, const QslotBufs* qs) {
   if (T <= 0) return STCA_OK;
   if (!H->step_tc_ready) return set_error(STCA_ESTATE, "tensor-core step weights are not set up");
   const int M = H->M;
@@ -868,6 +1021,12 @@ int launch_step_tc(const stca_handle* H, int layer, const void* targets, int64_t
   if (proj < 0 || proj > 2 || (proj && (naive || (proj == 1) != (cmerged != nullptr))))
     return set_error(STCA_EINVAL, "tensor-core step: bad projected-input mode");
   a.proj = layer >= 0 ? proj : 0;
+  if (a.proj == 2) {
+    if (!qs) return set_error(STCA_EINVAL, "tensor-core step: merging projected partials needs their row slots");
+    a.pacc = qs->pacc;
+    a.qml = qs->qml;
+    a.qn = qs->qn;
+  }
   if (naive) {
     if (!plan || (layer >= 0 && !cmerged))
       return set_error(STCA_EINVAL, "tensor-core step: the naive form needs o_head and the plan");
@@ -906,7 +1065,15 @@ int launch_step_tc(const stca_handle* H, int layer, const void* targets, int64_t
     add(kUG, H->tcUG[n]);
     add(kD, H->tcD[n]);
     add(kQ, H->tcQ[n]);
+    // the W_K products on the tensor cores: their operand Pblk takes the two
+    // ring slots after the launch's last A tiles, so the ring needs 4 slots
+    if (!naive && H->tcK.size() == static_cast<size_t>(M) && H->tcK[n].tile0 >= 0 &&
+        ring_stages(H, M) >= 4) {
+      add(kK, H->tcK[n]);
+      a.wk_tc = 1;
+    }
   }
+  for (int gi = 0; gi < a.ng; ++gi) a.qtot += a.g[gi].mb * a.g[gi].kc;
   // the deepest ring that fits, and the widest W_V staging chunk that fits
   // in the buffers it borrows
   int nring = kMaxRing;
