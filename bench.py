@@ -95,7 +95,7 @@ _REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_
 class ClockSampler:
     """Samples SM clock, power and clock-event reasons through NVML (read only)."""
 
-    def __init__(self, torch_device_index=0, period_s=0.02):
+    def __init__(self, torch_device_index=0, period_s=0.01):
         self.samples, self.max_mhz, self.ok = [], None, False
         self.period = period_s
         try:
@@ -679,11 +679,18 @@ def run_ours(args, rank, world, local_rank):
             att_fl = 18 * wl.d * c["TL"] * wl.h     # per (row, key): 2 passes of 2 dots + dU; 2 dots + dX~
         tf32 = 1100.0
         fp32 = 148 * 128 * 2 * 1.965e9 / 1e12
+        enc_bf16 = wl.dtype == "bf16" and wl.d % 64 == 0 and rd % 128 == 0
         backward = {
             "layer": 1, "loss": "synthetic <output, G>, G ~ N(0, 1)",
-            "encode": {"ms": enc_ms, "flops": enc_fl, "tflops": enc_fl / (enc_ms / 1e3) / 1e12,
-                       "frac_of_nominal_tf32": enc_fl / (enc_ms / 1e3) / 1e12 / tf32,
-                       "note": "cuBLASLt TF32 products + SwiGLU / LayerNorm derivative kernels"},
+            "encode": ({"ms": enc_ms, "flops": enc_fl, "tflops": enc_fl / (enc_ms / 1e3) / 1e12,
+                        "frac_of_measured_bf16": enc_fl / (enc_ms / 1e3) / 1e12 / peaks["bf16_tflops"],
+                        "note": "tcgen05 bf16 GEMM (gemm_bf16_kernel, persistent, SwiGLU forward and "
+                                "derivative in its epilogues) + the LayerNorm derivative kernel; "
+                                "bf16 intermediates"}
+                       if enc_bf16 else
+                       {"ms": enc_ms, "flops": enc_fl, "tflops": enc_fl / (enc_ms / 1e3) / 1e12,
+                        "frac_of_nominal_tf32": enc_fl / (enc_ms / 1e3) / 1e12 / tf32,
+                        "note": "cuBLASLt products + SwiGLU / LayerNorm derivative kernels"}),
             "attention": ({"ms": att_ms, "flops": att_fl, "tflops": att_fl / (att_ms / 1e3) / 1e12,
                            "frac_of_measured_bf16": att_fl / (att_ms / 1e3) / 1e12 / peaks["bf16_tflops"],
                            "note": "tcgen05: the forward attention for c and the row statistics, delta = dC . c, "
@@ -693,11 +700,13 @@ def run_ours(args, rank, world, local_rank):
                            "frac_of_nominal_fp32": att_fl / (att_ms / 1e3) / 1e12 / fp32,
                            "note": "CUDA-core flash-style kernels (softmax recomputed)"}),
             "projections": {"ms": proj_ms, "flops": 20 * wl.T * wl.d * wl.d,
-                            "note": "output side (W_V, W_O) and query side (W_Q, W_K): "
-                                    "cuBLASLt TF32 products, the per-head slices as strided batches"},
+                            "note": "output side (W_V, W_O) and query side (W_Q, W_K): TF32 products on "
+                                    "tcgen05 (gemm_tf32_kernel) where both operands are K-major, cuBLASLt "
+                                    "TF32 otherwise; the per-head slices as batches"},
             "query_side": {"ms": qside_ms, "flops": qside_fl,
                            "note": "the head (Eq. (9)), the M-1 fusion blocks (Eq. (7)) and the query init "
-                                   "(Eq. (3)): cuBLASLt TF32 products + SwiGLU / LayerNorm derivative kernels"}}
+                                   "(Eq. (3)): TF32 products (gemm_tf32_kernel / cuBLASLt) + SwiGLU / "
+                                   "LayerNorm derivative kernels; the query init on the bf16 GEMM"}}
 
     # ---- the sparse-training batch builder and a forward over its packed batch
     train_batch = None
@@ -760,7 +769,7 @@ def run_ours(args, rank, world, local_rank):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--config", default="c3", choices=sorted(CONFIGS))
