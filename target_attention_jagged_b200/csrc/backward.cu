@@ -258,7 +258,8 @@ __global__ void swiglu_bwd_kernel(float* __restrict__ A, float* __restrict__ G,
 }
 
 // LayerNorm backward: a CTA of 8 warps takes kLnRows consecutive rows, one warp
-// per row at a time.  Y holds y on entry and dy on exit.  Each lane keeps its
+// per row at a time.  Y holds y on entry and dy on exit (or, given dy16, dy goes
+// there as bf16 and Y is left as it was).  Each lane keeps its
 // columns' sums of dX~ * yhat and dX~ in registers over the CTA's rows, the
 // warps add them in shared memory, and the CTA adds its totals to dgamma and
 // dbeta with one atomic per column.
@@ -320,8 +321,9 @@ __global__ void __launch_bounds__(256) ln_bwd_kernel(float* __restrict__ Y, cons
       if (c >= d) continue;
       const float yh = (yv[j] - mu) * rstd, dyh = gv[j] * gamma[c];
       const float dy = rstd * (dyh - m1 - yh * m2);
-      y[c] = dy;
+      // the bf16 pipeline reads dy only as bf16: the fp32 copy is then not written
       if (dy16) dy16[row * d + c] = __bfloat16_as_ushort(__float2bfloat16_rn(dy));
+      else y[c] = dy;
     }
   }
 #pragma unroll
@@ -532,7 +534,7 @@ int ffn_ln_backward16(stca_handle* H, const uint16_t* X, int64_t N, const float*
   if (int rc = tc_gemm_bf16(false, true, N, d, rd, H16, rd, WdT, rd, Y, d, 0.f, 0, nullptr, nullptr, nullptr, 0, 0,
                             ns, st, s))
     return rc;
-  // LayerNorm: Y <- dy (also dy16); dgamma, dbeta
+  // LayerNorm: dy as bf16 (dy16); dgamma, dbeta
   STCA_CUDA_TRY(cudaMemsetAsync(dgamma, 0, d * sizeof(float), s));
   STCA_CUDA_TRY(cudaMemsetAsync(dbeta, 0, d * sizeof(float), s));
   ln_bwd_kernel<<<static_cast<unsigned>((N + kLnRows - 1) / kLnRows), 256, 0, s>>>(Y, dXt, gamma, dgamma,
