@@ -279,15 +279,16 @@ def storage_weights(wl):
     return out
 
 
-KERNEL_SOURCES = {"encode": "encode_tc.cu", "attention": "attn_tc.cu", "target_step": "target_step.cu"}
+KERNEL_SOURCES = {"encode": ("encode_tc.cu",), "attention": ("attn_tc_dev.cuh", "attn_tc.cu"),
+                  "target_step": ("step_tc.cu", "target_step.cu")}
 
 
 def source_hash(kind):
-    """sha256 (first 16 hex digits) of a kernel class's sources: its .cu file
-    followed by the shared tcgen05/TMA helper header."""
+    """sha256 (first 16 hex digits) of a kernel class's sources: its files
+    (KERNEL_SOURCES) followed by the shared tcgen05/TMA helper header."""
     import hashlib
     h = hashlib.sha256()
-    for f in (KERNEL_SOURCES[kind], "tc_common.cuh"):
+    for f in KERNEL_SOURCES[kind] + ("tc_common.cuh",):
         with open(os.path.join(ROOT, "target_attention_jagged_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
@@ -331,6 +332,11 @@ def roofline_of(kind, kt, c, wl, peaks, sustained, steps, config_key=None):
     elif kind == "attention":
         fl = c["attn_flops_naive"] if c.get("naive") else c["attn_flops"]
         flops, bytes_ = fl / per_step, c["attn_bytes_per_layer"] * wl.M / per_step
+    elif kind == "pipe":
+        # the two-half pipeline's launches: every attention layer of both halves,
+        # beside most of the per-target steps
+        flops = (c["attn_flops"] + c["tgt_flops"]) / per_step
+        bytes_ = c["attn_bytes_per_layer"] * wl.M / per_step
     else:
         flops, bytes_ = c["tgt_flops"] / per_step, c["io_bytes"] / per_step
     traffic = recorded_traffic(kind, config_key) if wl.dtype == "bf16" else None

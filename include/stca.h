@@ -454,6 +454,13 @@ enum {
   STCA_OPT_BW_GEMM = 9,       /* products of the backward pieces for bf16 handles: 0 the library's
                                  tensor-core GEMM with TF32 operands (default); 1 cuBLASLt TF32
                                  (kept for comparison); fp32 handles always use exact fp32 */
+  STCA_OPT_PIPELINE = 10,     /* 1 (default): when the forward runs the tensor-core attention
+                                 with its in-kernel W_V projection (d = 128), stca_forward (not
+                                 stca_forward_head) splits the requests into two halves of
+                                 about equal attention work and runs one half's per-target step
+                                 beside the other half's attention, in one launch per phase;
+                                 0: one batch, attention and step in turn.  Results are the same
+                                 up to the split partials' rounding order. */
   STCA_OPT_LAUNCHES = 100,    /* read-only: kernels launched since the last encode */
   STCA_OPT_LAST_FORM = 101    /* read-only: 1 if the last forward ran the naive form, else 0 */
 };
@@ -461,7 +468,9 @@ int stca_set_option(stca_handle* handle, int option, int64_t value);
 int stca_get_option(stca_handle* handle, int option, int64_t* value);
 
 /* Kernel classes reported by stca_kernel_times. */
-enum { STCA_K_ENCODE = 0, STCA_K_ATTN = 1, STCA_K_STEP = 2, STCA_K_HEAD = 3, STCA_K_CLASSES = 4 };
+enum { STCA_K_ENCODE = 0, STCA_K_ATTN = 1, STCA_K_STEP = 2, STCA_K_HEAD = 3,
+       STCA_K_PIPE = 4,   /* a pipeline launch: one half's step beside the other half's attention */
+       STCA_K_CLASSES = 5 };
 
 /*
  * Device time of each kernel class since the previous call, from the CUDA

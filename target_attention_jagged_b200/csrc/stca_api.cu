@@ -773,18 +773,78 @@ int stca::check_plan(const PlanHost& P, const int64_t* off, const int64_t* toff,
   return STCA_OK;
 }
 
-// Build (or reuse) the plan for the targets layout `toff` and upload it.
-static int build_plan(stca_handle* H, const int64_t* toff, int64_t T, int path, cudaStream_t s) {
+// The two-half pipeline's plan: requests [0, RA) and [RA, R) split at about
+// half of the attention work (key tiles x query tiles), each half planned for
+// the SMs its attention leaves to the other half's per-target step (16
+// targets per CTA), both checked, then joined into one plan: half B's items,
+// pairs and partial rows follow half A's, and its CTA runs follow A's
+// grid + 1 entries of cta_begin.  False when it does not apply (a half would
+// be empty, or a pair would have more items than the step merges).
+static bool build_pipe_plan(stca_handle* H, const int64_t* off, const int64_t* toff, int64_t R,
+                            PlanHost& P) {
+  const int h = H->h;
+  if (R < 2) return false;
+  std::vector<int64_t> work(R + 1, 0);
+  for (int64_t r = 0; r < R; ++r)
+    work[r + 1] = work[r] + ((toff[r + 1] - toff[r]) * h + 127) / 128 * ((off[r + 1] - off[r] + 127) / 128);
+  int64_t RA = 1;
+  while (RA < R - 1 && 2 * work[RA] < work[R]) ++RA;
+  const int64_t TA = toff[RA], T = toff[R];
+  if (TA <= 0 || TA >= T) return false;
+  const int nstepA = static_cast<int>((TA + 15) / 16), nstepB = static_cast<int>((T - TA + 15) / 16);
+  const int ctasA = H->num_sms - nstepB, ctasB = H->num_sms - nstepA;
+  if (ctasA < H->num_sms / 4 || ctasB < H->num_sms / 4) return false;
+  PlanHost A, B;
+  build_plan_host(off, toff, RA, h, 2, ctasA, H->opt_split_keys, A, H->dh, 0);
+  build_plan_host(off + RA, toff + RA, R - RA, h, 2, ctasB, H->opt_split_keys, B, H->dh, 0);
+  if (check_plan(A, off, toff, RA, h, 2) || check_plan(B, off + RA, toff + RA, R - RA, h, 2)) {
+    set_error(STCA_OK, "");
+    return false;
+  }
+  for (const PlanHost* X : {&A, &B})
+    for (size_t k = 0; k + 1 < X->pair_item_begin.size(); ++k)
+      if (X->pair_item_begin[k + 1] - X->pair_item_begin[k] > kQslots) return false;
+  const int32_t nA = static_cast<int32_t>(A.items.size()), pA = static_cast<int32_t>(A.req_pair_begin[RA]);
+  P = PlanHost();
+  P.items = A.items;
+  for (AttnItem it : B.items) {
+    it.req += static_cast<int32_t>(RA);
+    it.pair += pA;
+    it.row_base += A.G;
+    P.items.push_back(it);
+  }
+  P.cta_begin = A.cta_begin;
+  for (int32_t c : B.cta_begin) P.cta_begin.push_back(c + nA);
+  P.req_pair_begin.assign(A.req_pair_begin.begin(), A.req_pair_begin.end());
+  for (int64_t r = 1; r <= R - RA; ++r) P.req_pair_begin.push_back(B.req_pair_begin[r] + pA);
+  P.pair_item_begin = A.pair_item_begin;
+  for (size_t k = 1; k < B.pair_item_begin.size(); ++k) P.pair_item_begin.push_back(B.pair_item_begin[k] + nA);
+  P.G = A.G + B.G;
+  P.grid = A.grid + B.grid;
+  H->pipe_RA = RA;
+  H->pipe_TA = TA;
+  H->pipe_gridA = A.grid;
+  H->pipe_gridB = B.grid;
+  return true;
+}
+
+// Build (or reuse) the plan for the targets layout `toff` and upload it; with
+// pipe, the two-half pipeline's plan where it applies (H->last_pipe says).
+static int build_plan(stca_handle* H, const int64_t* toff, int64_t T, int path, cudaStream_t s,
+                      bool pipe = false) {
   const int64_t R = H->R;
-  if (path == H->last_path && !H->last_toff.empty() &&
+  if (path == H->last_path && pipe == H->last_pipe_asked && !H->last_toff.empty() &&
       static_cast<int64_t>(H->last_toff.size()) == R + 1 &&
       std::equal(H->last_toff.begin(), H->last_toff.end(), toff))
     return STCA_OK;   // same layout as the previous forward on this encode: plan is on device
   const int64_t* off = H->offsets_h.data();
   PlanHost P;
-  build_plan_host(off, toff, R, H->h, path, H->num_sms, H->opt_split_keys, P, H->dh,
-                  attn_simt_rows_per_cta(H->d));
-  if (int rc = check_plan(P, off, toff, R, H->h, path)) return rc;
+  H->last_pipe = pipe && path == 2 && build_pipe_plan(H, off, toff, R, P);
+  if (!H->last_pipe) {
+    build_plan_host(off, toff, R, H->h, path, H->num_sms, H->opt_split_keys, P, H->dh,
+                    attn_simt_rows_per_cta(H->d));
+    if (int rc = check_plan(P, off, toff, R, H->h, path)) return rc;
+  }
   const auto& items = P.items;
   const auto& pairs_simt = P.pairs_simt;
   const auto& cta_begin = P.cta_begin;
@@ -839,6 +899,7 @@ static int build_plan(stca_handle* H, const int64_t* toff, int64_t T, int path, 
     H->last_max_items = std::max(H->last_max_items, pair_item_begin[k + 1] - pair_item_begin[k]);
   H->last_grid = grid;
   H->last_path = path;
+  H->last_pipe_asked = pipe;
   H->last_toff.assign(toff, toff + R + 1);
   return STCA_OK;
 }
@@ -900,7 +961,12 @@ static int forward_impl(stca_handle* H, const void* targets, const int64_t* targ
   const bool naive = naive_ok && (H->opt_attn_form == 1 ||
                                   (H->opt_attn_form == 2 && naive_cheaper(H, target_offsets)));
   H->last_naive = naive;
-  if (int rc = build_plan(H, target_offsets, T, naive ? 3 : path, s)) return rc;
+  // the two-half pipeline (STCA_OPT_PIPELINE): the reordered form on the
+  // tensor cores with the in-kernel W_V projection and the step's merge
+  const bool want_pipe = !naive && path == 2 && H->opt_pipeline == 1 && zout == nullptr &&
+                         H->step_tc_ready && H->opt_step_path != 1 && H->opt_attn_kernel == 0 &&
+                         attn_tc_proj_supported(H);
+  if (int rc = build_plan(H, target_offsets, T, naive ? 3 : path, s, want_pipe)) return rc;
   const int d = H->d, h = H->h;
   const size_t urows = static_cast<size_t>(T) * h;
   if (naive) {
@@ -990,6 +1056,58 @@ static int forward_impl(stca_handle* H, const void* targets, const int64_t* targ
     launch_target_step(H, layer, targets, T, plan, cm, Z, s);
     return static_cast<int>(STCA_OK);
   };
+  if (H->last_pipe) {
+    // Two halves, A = targets [0, TA), B = [TA, T): A's query init alone, then
+    // per layer i one launch of A's attention beside B's step i - 1 (the query
+    // init for i = 0) and one of B's attention beside A's step i, then B's
+    // last step alone.  Each launch's two parts are independent; each part
+    // depends only on the previous launch.
+    if (proj_mode != 2) return set_error(STCA_EINVAL, "internal: pipeline plan without the projected merge");
+    const int64_t TA = H->pipe_TA, TB = T - TA, M = H->M, dh = H->dh;
+    const uint16_t* tg = static_cast<const uint16_t*>(targets);
+    auto half_qs = [&](int64_t t0) {
+      QslotBufs q = qs;
+      q.pacc += t0 * h * kQslots * dh;
+      q.qml += t0 * h * kQslots * 2;
+      q.qn += t0 * h;
+      return q;
+    };
+    PipeStep sA{0, tg, TA, Z, H->Ubf, half_qs(0)};
+    PipeStep sB{0, tg + TA * d, TB, Z + TA * M * d, H->Ubf + TA * h * d, half_qs(TA)};
+    PipeAttn aA{0, items_d, cta_d, H->pipe_gridA, qs};
+    PipeAttn aB{0, items_d, cta_d + H->pipe_gridA + 1, H->pipe_gridB, qs};
+    {
+      TimedLaunch tl(H, STCA_K_STEP, s);
+      if (int rc = launch_step_tc(H, -1, tg, TA, nullptr, &plan, H->part, H->last_G, Z, H->Ubf, s)) return rc;
+    }
+    if (int rc2 = check_launch("query init")) return rc2;
+    for (int i = 0; i < M; ++i) {
+      sB.layer = i - 1;
+      aA.layer = i;
+      {
+        TimedLaunch tl(H, STCA_K_PIPE, s);
+        if (int rc = launch_step_attn_pipe(H, sB, aA, s)) return rc;
+      }
+      if (int rc2 = check_launch("pipeline")) return rc2;
+      sA.layer = i;
+      aB.layer = i;
+      {
+        TimedLaunch tl(H, STCA_K_PIPE, s);
+        if (int rc = launch_step_attn_pipe(H, sA, aB, s)) return rc;
+      }
+      if (int rc2 = check_launch("pipeline")) return rc2;
+    }
+    {
+      TimedLaunch tl(H, STCA_K_STEP, s);
+      QslotBufs qB = half_qs(TA);
+      if (int rc = launch_step_tc(H, static_cast<int>(M - 1), sB.targets, TB, nullptr, nullptr, nullptr, 0,
+                                  sB.Z, sB.Ubf, s, nullptr, nullptr, 2, &qB))
+        return rc;
+    }
+    if (int rc2 = check_launch("target step")) return rc2;
+    H->launches += 2 * M + 2;
+    return ok();
+  }
   {
     TimedLaunch tl(H, STCA_K_STEP, s);
     if (int rc = step(-1, nullptr)) return rc;
@@ -1274,6 +1392,10 @@ extern "C" int stca_set_option(stca_handle* H, int option, int64_t value) {
       if (value < 0 || value > 1) return set_error(STCA_EINVAL, "backward GEMM must be 0 or 1");
       H->opt_bw_gemm = static_cast<int>(value);
       return ok();
+    case STCA_OPT_PIPELINE:
+      if (value < 0 || value > 1) return set_error(STCA_EINVAL, "pipeline must be 0 or 1");
+      H->opt_pipeline = static_cast<int>(value);
+      return ok();
     case STCA_OPT_SPLIT_KEYS:
       if (value < 0 || value % 128 || value > (int64_t(1) << 30))
         return set_error(STCA_EINVAL, "split must be 0 or a positive multiple of 128");
@@ -1297,6 +1419,7 @@ extern "C" int stca_get_option(stca_handle* H, int option, int64_t* value) {
     case STCA_OPT_ATTN_KERNEL: *value = H->opt_attn_kernel; return ok();
     case STCA_OPT_TEST_STOP_TILES: *value = H->opt_stop_tiles; return ok();
     case STCA_OPT_BW_GEMM: *value = H->opt_bw_gemm; return ok();
+    case STCA_OPT_PIPELINE: *value = H->opt_pipeline; return ok();
     case STCA_OPT_LAST_FORM: *value = H->last_naive ? 1 : 0; return ok();
     default: return set_error(STCA_EINVAL, "unknown option " + std::to_string(option));
   }

@@ -136,6 +136,7 @@ struct stca_handle {
   int opt_attn_kernel = 0;              // 0 auto (two-group kernel for d <= 128), 1 split-softmax kernel
   int opt_stop_tiles = 0;               // test hook: the attention loader stops after this many tiles
   int opt_bw_gemm = 0;                  // backward products of bf16 handles: 0 tensor cores (TF32), 1 cuBLASLt
+  int opt_pipeline = 1;                 // 1: two-half pipeline where it applies (STCA_OPT_PIPELINE)
   int64_t launches = 0;
   bool timing = false;
   struct TimedRec { int cls; cudaEvent_t a, b; };
@@ -175,6 +176,10 @@ struct stca_handle {
   int64_t last_npairs = 0;              // (request, query tile) pairs of the plan
   int last_max_items = 0;               // most items of one (request, query tile) pair
   int last_grid = 0;                    // CTAs of the tensor-core attention
+  bool last_pipe = false;               // the plan is the two-half pipeline's
+  bool last_pipe_asked = false;         // ... was asked for (part of the plan cache's key)
+  int64_t pipe_RA = 0, pipe_TA = 0;     // its split: first request and first target of half B
+  int pipe_gridA = 0, pipe_gridB = 0;   // its halves' attention CTAs (B's runs follow A's in cta_begin)
   size_t off_items = 0, off_pairs = 0, off_cta = 0, off_treq = 0, off_toff = 0, off_rpb = 0,
          off_pib = 0, off_qbase = 0;
   int64_t last_qrows = 0;               // naive form: rows of the packed query layout
@@ -265,6 +270,28 @@ int launch_step_tc(const stca_handle* H, int layer, const void* targets, int64_t
                    const float* cmerged, const StepPlan* plan, const float* part, int64_t G,
                    float* Z, uint16_t* Ubf, cudaStream_t s, const NaiveStep* naive = nullptr,
                    float* zout = nullptr, int proj = 0, const QslotBufs* qs = nullptr);
+
+// One phase of the two-half pipeline (stca_forward at d = 128 with the
+// in-kernel projection): one launch runs the per-target step of one half of
+// the batch (layer, its targets, Z and U rows, the row slots of its query
+// rows; T = 0: none) beside the attention of the other half (its plan's
+// items and CTA runs; grid = 0: none).
+struct PipeStep {
+  int layer;
+  const void* targets;
+  int64_t T;
+  float* Z;
+  uint16_t* Ubf;
+  QslotBufs qs;
+};
+struct PipeAttn {
+  int layer;
+  const AttnItem* items;
+  const int32_t* cta_begin;
+  int grid;
+  QslotBufs qs;
+};
+int launch_step_attn_pipe(const stca_handle* H, const PipeStep& st, const PipeAttn& at, cudaStream_t s);
 
 // Host-side attention work plan (stca_api.cu).
 struct PlanHost {

@@ -29,6 +29,7 @@
 #include <cstring>
 #include <vector>
 
+#include "attn_tc_dev.cuh"
 #include "stca_internal.h"
 #include "tc_common.cuh"
 
@@ -283,8 +284,11 @@ __device__ __forceinline__ bool step_wait(uint64_t* bar, uint32_t parity, int* s
   return true;
 }
 
-__global__ void __launch_bounds__(kStepThreads, 1) step_tc_kernel(const StepTcArgs a) {
-  extern __shared__ uint8_t smem_raw[];
+// The kernel's body for CTA `cta` of its grid (targets 16 cta ..), on dynamic
+// shared memory smem_raw (its layout plus 1024 bytes of alignment slack).  The
+// calling kernel may have more than kStepThreads threads: the extra warps
+// take no part but the CTA-wide barriers.
+__device__ __forceinline__ void step_tc_body(const StepTcArgs& a, uint8_t* smem_raw, int cta) {
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                            ~static_cast<uintptr_t>(1023));
   const int d = a.d, h = a.h, dh = a.dh, rd = a.rd, L = a.layer;
@@ -297,7 +301,7 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_tc_kernel(const StepTcAr
   uint64_t* mdrain = aready + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mdrain + 2);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t t0 = static_cast<int64_t>(blockIdx.x) * kTgt;
+  const int64_t t0 = static_cast<int64_t>(cta) * kTgt;
   const int nb = a.T - t0 < kTgt ? static_cast<int>(a.T - t0) : kTgt;
   uint8_t* bufs[6] = {sm + Y.bO, sm + Y.bC, sm + Y.bU, sm + Y.bH, sm + Y.bQ, sm + Y.bH};
 
@@ -377,7 +381,7 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_tc_kernel(const StepTcAr
       mma_commit(mdrain);
       step_wait(mdrain, 0, a.status);
     }
-  } else {
+  } else if (warp < 2 + kWorkers) {
     // ------------------------------------------------------------ workers
     const int wid = warp - 2;                 // 0..7
     const int tid = threadIdx.x - 64;         // 0..255
@@ -939,6 +943,11 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_tc_kernel(const StepTcAr
   }
 }
 
+__global__ void __launch_bounds__(kStepThreads, 1) step_tc_kernel(const StepTcArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  step_tc_body(a, smem_raw, static_cast<int>(blockIdx.x));
+}
+
 }  // namespace
 
 // ------------------------------------------------------------------ launch
@@ -996,20 +1005,21 @@ int launch_step_tc_head(const stca_handle* H, const void* targets, int64_t T, co
   return STCA_OK;
 }
 
-int launch_step_tc(const stca_handle* H, int layer, const void* targets, int64_t T,
+namespace {
+// The step kernel's arguments, shared memory and grid for one launch (T > 0).
+int make_step_args(const stca_handle* H, int layer, const void* targets, int64_t T,
                    const float* cmerged, const StepPlan* plan, const float* part, int64_t G,
-                   float* Z, uint16_t* Ubf, cudaStream_t s, const NaiveStep* naive, float* zout,
-                   int proj, const QslotBufs* qs) {
-  if (T <= 0) return STCA_OK;
+                   float* Z, uint16_t* Ubf, const NaiveStep* naive, float* zout, int proj,
+                   const QslotBufs* qs, StepTcArgs& a, size_t& smem, unsigned& grid) {
   if (!H->step_tc_ready) return set_error(STCA_ESTATE, "tensor-core step weights are not set up");
   const int M = H->M;
-  StepTcArgs a{};
+  a = StepTcArgs{};
   a.layer = layer;
   a.M = M; a.d = H->d; a.h = H->h; a.dh = H->dh; a.rd = H->rd;
   a.T = T;
   a.targets = static_cast<const uint16_t*>(targets);
   a.cmerged = cmerged;
-  if (layer >= 0 && cmerged == nullptr) {
+  if (layer >= 0 && cmerged == nullptr && proj != 2) {
     if (!plan || !part || G >= (int64_t(1) << 31))
       return set_error(STCA_EINVAL, "tensor-core step: no split partials to merge");
     a.plan = *plan;
@@ -1092,13 +1102,79 @@ int launch_step_tc(const stca_handle* H, int layer, const void* targets, int64_t
     return set_error(STCA_EINVAL, "tensor-core step: too many heads for the W_V staging");
   a.nring = nring;
   a.kch = kch;
-  const size_t smem = Y.total + 1024;
+  smem = Y.total + 1024;
+  grid = static_cast<unsigned>((T + kTgt - 1) / kTgt);
+  return STCA_OK;
+}
+
+// One launch of the two independent halves of a pipeline phase: CTAs
+// 0 .. nstep - 1 run a per-target step (one half of the batch), the others the
+// next attention layer (the other half; the split-softmax kernel with its
+// query tile in TMEM and W_V in the epilogue, d = 128).
+__global__ void __launch_bounds__(kAttnThreads, 1)
+pipe_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+            const __grid_constant__ CUtensorMap tmV, const AttnParams p, const StepTcArgs a, int nstep) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  const int b = static_cast<int>(blockIdx.x);
+  if (b < nstep) step_tc_body(a, smem_raw, b);
+  else attn_tc_body<128, 1, 5, 1, false, true, true>(tmQ, tmK, tmV, p, smem_raw, b - nstep);
+}
+using PipeAttnCfg = AttnCfg<128, 1, 5, 1, false, true, true>;
+static_assert(kStepThreads <= kAttnThreads, "the pipeline kernel runs both bodies");
+}  // namespace
+
+int launch_step_tc(const stca_handle* H, int layer, const void* targets, int64_t T,
+                   const float* cmerged, const StepPlan* plan, const float* part, int64_t G,
+                   float* Z, uint16_t* Ubf, cudaStream_t s, const NaiveStep* naive, float* zout,
+                   int proj, const QslotBufs* qs) {
+  if (T <= 0) return STCA_OK;
+  StepTcArgs a;
+  size_t smem;
+  unsigned grid;
+  if (int rc = make_step_args(H, layer, targets, T, cmerged, plan, part, G, Z, Ubf, naive, zout, proj, qs, a,
+                              smem, grid))
+    return rc;
   cudaError_t e = cudaFuncSetAttribute(step_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return set_error(STCA_ECUDA, std::string("step_tc smem: ") + cudaGetErrorString(e));
-  const unsigned grid = static_cast<unsigned>((T + kTgt - 1) / kTgt);
   e = launch_pdl(step_tc_kernel, dim3(grid), dim3(kStepThreads), smem, s, a);
   if (e != cudaSuccess) return set_error(STCA_ECUDA, std::string("step_tc launch: ") + cudaGetErrorString(e));
+  return STCA_OK;
+}
+
+int launch_step_attn_pipe(const stca_handle* H, const PipeStep& st, const PipeAttn& at, cudaStream_t s) {
+  if (!attn_tc_proj_supported(H)) return set_error(STCA_EINVAL, "pipelined step: needs the in-kernel projection");
+  StepTcArgs a{};
+  size_t smem_s = 0;
+  unsigned nstep = 0;
+  if (st.T > 0)
+    if (int rc = make_step_args(H, st.layer, st.targets, st.T, nullptr, nullptr, nullptr, 0, st.Z, st.Ubf,
+                                nullptr, nullptr, 2, &st.qs, a, smem_s, nstep))
+      return rc;
+  AttnParams p{};
+  p.items = at.items;
+  p.cta_item_begin = at.cta_begin;
+  p.pacc = at.qs.pacc;
+  p.pm = p.pl = nullptr;               // per-row slots only
+  p.status = H->status_d;
+  p.stop_tiles = H->opt_stop_tiles;
+  p.h = H->h;
+  p.dh = H->dh;
+  p.qslot = 1;
+  p.pair_item_begin = at.qs.pair_item_begin;
+  p.qml = at.qs.qml;
+  p.qn = at.qs.qn;
+  const unsigned agrid = at.grid > 0 ? static_cast<unsigned>(at.grid) : 0u;
+  if (nstep + agrid == 0) return STCA_OK;
+  const size_t smem = std::max<size_t>(smem_s, PipeAttnCfg::kSmem);
+  cudaError_t e = cudaFuncSetAttribute(pipe_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return set_error(STCA_ECUDA, std::string("pipe smem: ") + cudaGetErrorString(e));
+  const CUtensorMap& tmK = H->tmXt[at.grid > 0 ? at.layer : 0];
+  const CUtensorMap& tmV = H->tmWvT[at.grid > 0 ? at.layer : 0];
+  e = launch_pdl(pipe_kernel, dim3(nstep + agrid), dim3(kAttnThreads), smem, s, H->tmU, tmK, tmV, p, a,
+                 static_cast<int>(nstep));
+  if (e != cudaSuccess) return set_error(STCA_ECUDA, std::string("pipe launch: ") + cudaGetErrorString(e));
   return STCA_OK;
 }
 

@@ -29,9 +29,10 @@ STCA_OPT_ATTN_FORM = 6
 STCA_OPT_ATTN_KERNEL = 7
 STCA_OPT_TEST_STOP_TILES = 8
 STCA_OPT_BW_GEMM = 9
+STCA_OPT_PIPELINE = 10
 STCA_OPT_LAUNCHES = 100
 STCA_OPT_LAST_FORM = 101
-STCA_K_ENCODE, STCA_K_ATTN, STCA_K_STEP, STCA_K_HEAD, STCA_K_CLASSES = 0, 1, 2, 3, 4
+STCA_K_ENCODE, STCA_K_ATTN, STCA_K_STEP, STCA_K_HEAD, STCA_K_PIPE, STCA_K_CLASSES = 0, 1, 2, 3, 4, 5
 _NAMES = {STCA_EINVAL: "EINVAL", STCA_ESTATE: "ESTATE", STCA_ENOMEM: "ENOMEM",
           STCA_ECUDA: "ECUDA", STCA_EDEVICE: "EDEVICE"}
 
@@ -503,7 +504,7 @@ def stca_kernel_times(handle: int):
     ms = (ctypes.c_double * STCA_K_CLASSES)()
     n = (ctypes.c_int64 * STCA_K_CLASSES)()
     _check(_lib.stca_kernel_times(handle, ms, n, STCA_K_CLASSES))
-    names = ("encode", "attention", "target_step", "head")
+    names = ("encode", "attention", "target_step", "head", "pipe")
     return {names[c]: (ms[c], n[c]) for c in range(STCA_K_CLASSES)}
 
 

@@ -32,7 +32,7 @@ def to_device(wl, a, device):
 
 
 def run_gpu(wl, device, attn_path=0, encode_path=0, split=0, handle=None, keep=False, step_path=0,
-            attn_form=None, attn_kernel=None):
+            attn_form=None, attn_kernel=None, pipeline=None):
     """Z (T x M x d, numpy fp32) from the CUDA path through the C ABI."""
     import torch
     import target_attention_jagged_b200 as S
@@ -48,6 +48,8 @@ def run_gpu(wl, device, attn_path=0, encode_path=0, split=0, handle=None, keep=F
             st.set_option(S.STCA_OPT_STEP_PATH, step_path)
         if attn_form is not None:
             st.set_option(S.STCA_OPT_ATTN_FORM, attn_form)
+        if pipeline is not None:
+            st.set_option(S.STCA_OPT_PIPELINE, pipeline)
         if attn_kernel is not None:
             st.set_option(S.STCA_OPT_ATTN_KERNEL, attn_kernel)
         X = to_device(wl, wl.X, device)

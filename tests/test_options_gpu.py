@@ -14,6 +14,7 @@ pytestmark = pytest.mark.gpu
     ("STCA_OPT_STEP_PATH", [0, 1, 2], [-1, 3]),
     ("STCA_OPT_ATTN_FORM", [0, 1, 2], [-1, 3]),
     ("STCA_OPT_ATTN_KERNEL", [0, 1, 2], [-1, 3]),
+    ("STCA_OPT_PIPELINE", [0, 1], [-1, 2]),
     ("STCA_OPT_TEST_STOP_TILES", [0, 1, 1000], [-1]),
     ("STCA_OPT_BW_GEMM", [0, 1], [-1, 2]),
     ("STCA_OPT_SPLIT_KEYS", [0, 128, 4096], [-128, 100]),

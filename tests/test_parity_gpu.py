@@ -284,6 +284,57 @@ def test_tc_kernels_sharp_softmax(gpu, kernel):
     check_full(wl, run_gpu(wl, gpu, attn_path=ATTN_TC, attn_kernel=kernel))
 
 
+# The two-half pipeline (STCA_OPT_PIPELINE, on by default where it applies):
+# the halves split the requests by attention work, and one launch runs one
+# half's per-target step beside the other half's attention.  It applies when
+# each pair (request, query tile) of the halves' plans has at most 8 items,
+# i.e. with enough pairs per half; otherwise the forward runs in one piece.
+def _forward_launches(wl, gpu, pipeline):
+    """Z and the number of kernels one forward launched."""
+    import torch
+    import target_attention_jagged_b200 as S
+    from tests.gpu_helpers import storage_weights, to_device
+    with S.Stca(storage_weights(wl), wl.d, wl.h, wl.r, wl.M, wl.dtype) as st:
+        st.set_option(S.STCA_OPT_PIPELINE, pipeline)
+        st.encode(to_device(wl, wl.X, gpu), wl.offsets)
+        n0 = st.get_option(S.STCA_OPT_LAUNCHES)
+        Z = torch.zeros((wl.T, wl.M, wl.d), dtype=torch.float32, device=gpu)
+        st.forward(to_device(wl, wl.targets, gpu), wl.target_offsets, Z)
+        torch.cuda.synchronize()
+        st.status()
+        return Z.cpu().numpy(), st.get_option(S.STCA_OPT_LAUNCHES) - n0
+
+
+@pytest.mark.parametrize("seed", [0, 1])
+def test_pipeline_matches_oracle(gpu, seed):
+    """80 requests of 600..2000 keys: the pipeline engages (2M + 2 launches
+    against 2M + 1), matches the oracle on sampled requests and the one-piece
+    forward on the whole batch.  Seed 1 has ragged targets (0 to 40 per
+    request: several query tiles, empty requests)."""
+    rng = np.random.default_rng(seed)
+    R = 80
+    lengths = rng.integers(600, 2001, R).tolist()
+    targets = [16] * R if seed == 0 else rng.integers(0, 41, R).tolist()
+    wl = make_workload(lengths=lengths, targets=targets, d=128, h=8, M=3, r=2, dtype="bf16", seed=430 + seed)
+    a, na = _forward_launches(wl, gpu, 1)
+    b, nb = _forward_launches(wl, gpu, 0)
+    assert na == 2 * wl.M + 2 and nb == 2 * wl.M + 1, (na, nb)
+    check_sampled(wl, a, 4, seed=seed)
+    assert normwise_err(a, b) <= 2e-2
+
+
+def test_pipeline_falls_back(gpu):
+    """Two requests whose pairs would need far more than 8 items each: the
+    forward runs in one piece (the same launches as with the pipeline off:
+    here with the separate merge of the partials) and matches the oracle."""
+    wl = make_workload(lengths=[20000, 300], targets=[3, 17], d=128, h=8, M=3, r=2, dtype="bf16", seed=441)
+    a, na = _forward_launches(wl, gpu, 1)
+    b, nb = _forward_launches(wl, gpu, 0)
+    assert na == nb, (na, nb)
+    check_full(wl, a)
+    assert normwise_err(a, b) == 0.0
+
+
 def test_tc_kernels_agree_on_c3(gpu):
     wl = make_config_workload("c3")
     a = run_gpu(wl, gpu, attn_kernel=KERNEL_TWO_GROUP)
@@ -293,3 +344,5 @@ def test_tc_kernels_agree_on_c3(gpu):
     c = run_gpu(wl, gpu, attn_kernel=KERNEL_AUTO)
     check_sampled(wl, c, 2, seed=4)
     assert normwise_err(c, b) <= 2e-2
+    e = run_gpu(wl, gpu, attn_kernel=KERNEL_AUTO, pipeline=0)
+    assert normwise_err(c, e) <= 2e-2
