@@ -470,6 +470,8 @@ def run_ours(args, rank, world, local_rank):
         st.set_option(S.STCA_OPT_ATTN_FORM, args.attn_form)
     if args.attn_kernel is not None:
         st.set_option(S.STCA_OPT_ATTN_KERNEL, args.attn_kernel)
+    if args.pipeline is not None:
+        st.set_option(S.STCA_OPT_PIPELINE, args.pipeline)
     X = to_dev(wl, wl.X, dev)
     xt = to_dev(wl, wl.targets, dev)
     Z = torch.empty((wl.T, wl.M, wl.d), dtype=torch.float32, device=dev)
@@ -772,6 +774,75 @@ def run_ours(args, rank, world, local_rank):
     print(json.dumps(line), flush=True)
 
 
+def _pipe_used(S, st, xt, wl, Z):
+    """Whether one forward of this batch ran the two-half pipeline."""
+    st.set_option(S.STCA_OPT_TIMING, 1)
+    S.stca_kernel_times(st.handle)
+    st.forward(xt, wl.target_offsets, Z)
+    n = S.stca_kernel_times(st.handle)["pipe"][1]
+    st.set_option(S.STCA_OPT_TIMING, 0)
+    return n > 0
+
+
+def attn_paths_sweep():
+    """Forward time with the CUDA-core attention path (STCA_OPT_ATTN_PATH 1,
+    which also takes the CUDA-core per-target step) against the tensor-core
+    path (2), over T_r * h, on bf16 batches shaped like the ragged 32-request
+    config (L ~ U[200, 2000]) and like the serving config (L = 10000, 16
+    requests); d 128, M 2, r 2.  Prints one JSON line per shape: the whole
+    forward (min of 3 x 20 calls) and the attention launches alone (events
+    around each launch), in ms, and the normwise difference of the two Z."""
+    import torch
+    import target_attention_jagged_b200 as S
+    from gen import make_workload
+    dev = torch.device("cuda:0")
+    for shape, R, lengths in (("ragged-L200-2000", 32, ("uniform", 200, 2000)),
+                              ("L10000", 16, ("fixed", 10000))):
+        for h in (4, 8):
+            for Tr in (1, 2, 4, 8, 16, 32):
+                wl = make_workload(lengths=lengths, targets=("fixed", Tr), d=128, h=h, M=2, r=2,
+                                   dtype="bf16", seed=11, R=R)
+                rec = {"shape": shape, "R": R, "h": h, "T_r": Tr, "T_r_h": Tr * h, "N": wl.N}
+                zs = {}
+                with S.Stca(storage_weights(wl), wl.d, wl.h, wl.r, wl.M, wl.dtype) as st:
+                    X, xt = to_dev(wl, wl.X, dev), to_dev(wl, wl.targets, dev)
+                    st.encode(X, wl.offsets)
+                    Z = torch.empty((wl.T, wl.M, wl.d), dtype=torch.float32, device=dev)
+                    for path, name in ((1, "cuda_cores"), (2, "tensor_cores")):
+                        st.set_option(S.STCA_OPT_ATTN_PATH, path)
+                        for _ in range(5):
+                            st.forward(xt, wl.target_offsets, Z)
+                        torch.cuda.synchronize()
+                        ts = []
+                        for _ in range(3):
+                            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                            a.record()
+                            for _ in range(20):
+                                st.forward(xt, wl.target_offsets, Z)
+                            b.record()
+                            torch.cuda.synchronize()
+                            ts.append(a.elapsed_time(b) / 20)
+                        pipelined = _pipe_used(S, st, xt, wl, Z)
+                        # the attention launches alone, from a pass with the
+                        # two-half pipeline off (its launches mix in the step)
+                        st.set_option(S.STCA_OPT_PIPELINE, 0)
+                        st.set_option(S.STCA_OPT_TIMING, 1)
+                        S.stca_kernel_times(st.handle)
+                        for _ in range(20):
+                            st.forward(xt, wl.target_offsets, Z)
+                        torch.cuda.synchronize()
+                        kt = S.stca_kernel_times(st.handle)
+                        st.set_option(S.STCA_OPT_TIMING, 0)
+                        st.set_option(S.STCA_OPT_PIPELINE, 1)
+                        st.status()
+                        rec[name] = {"forward_ms": round(min(ts), 4),
+                                     "attention_ms": round(kt["attention"][0] / 20, 4),
+                                     "pipeline": pipelined}
+                        zs[path] = Z.cpu().numpy()
+                rec["z_rel_diff"] = float(np.linalg.norm(zs[1] - zs[2]) / np.linalg.norm(zs[2]))
+                print(json.dumps(rec), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -789,6 +860,12 @@ def main():
     ap.add_argument("--strong", action="store_true",
                     help="strong scaling: one batch partitioned over the ranks by request "
                          "(shard.partition_requests); default: weak, a full batch per rank")
+    ap.add_argument("--pipeline", type=int, default=None, choices=[0, 1],
+                    help="STCA_OPT_PIPELINE: 1 two-half pipeline where it applies, 0 off; "
+                         "default: the library's choice")
+    ap.add_argument("--attn-paths", action="store_true",
+                    help="only sweep the CUDA-core against the tensor-core attention path over "
+                         "T_r * h (one GPU; JSON lines) and exit")
     ap.add_argument("--no-backward", action="store_true", help="skip the backward measurement")
     ap.add_argument("--no-train-batch", action="store_true",
                     help="skip the sparse-training batch builder measurement")
@@ -802,6 +879,9 @@ def main():
         log(f"note: WORLD_SIZE={world} but --gpus={args.gpus}; using WORLD_SIZE")
     if args.impl == "reference":
         run_reference(args, rank)
+        return
+    if args.attn_paths:
+        attn_paths_sweep()
         return
     if world > 1:
         import torch
