@@ -458,9 +458,11 @@ enum {
                                  with its in-kernel W_V projection (d = 128), stca_forward (not
                                  stca_forward_head) splits the requests into two halves of
                                  about equal attention work and runs one half's per-target step
-                                 beside the other half's attention, in one launch per phase;
-                                 0: one batch, attention and step in turn.  Results are the same
-                                 up to the split partials' rounding order. */
+                                 beside the other half's attention, in one launch per phase,
+                                 when the batch has at least 24 (128-key tile x 128-row query
+                                 tile) pairs of attention work per SM; 0: one batch, attention
+                                 and step in turn.  Results are the same up to the split
+                                 partials' rounding order. */
   STCA_OPT_LAUNCHES = 100,    /* read-only: kernels launched since the last encode */
   STCA_OPT_LAST_FORM = 101    /* read-only: 1 if the last forward ran the naive form, else 0 */
 };

@@ -122,7 +122,9 @@ ffn_rows_kernel(const void* __restrict__ X, int64_t nrows, const float* __restri
 // ---------------------------------------------------------------- attention
 // CUDA-core split-L single-query attention ("Make It Long, Keep It Fast"
 // digest §2.1, Eq. (13)), for batches whose query rows per request (T_r h) are
-// too few for a tensor-core tile, and for the fp32 configuration.
+// too few for a tensor-core tile, and for the fp32 configuration.  This
+// key-per-group form serves the widths that the feature-per-lane kernel
+// further down does not (d outside {32, 64, 128, 256}).
 //
 // One CTA takes one work item (a request's key range, at most a few thousand
 // keys) and a block of up to kRowsPerCta(NCH) of the request's query rows, so
@@ -346,6 +348,249 @@ attn_simt_kernel(const void* __restrict__ Xt, const float* __restrict__ U,
   }
 }
 
+// ---------------------------------------------------------------------------
+// The same attention for d in {32, 64, 128, 256} (F = d / 32 features per
+// lane), built so that the history is read at close to HBM speed when a
+// request has few query rows.
+//
+// One CTA of 8 warps takes a work item and a block of up to 16 of the
+// request's query rows (QB, the smallest of 4, 8, 16 that holds the batch's
+// largest block).  Key tiles arrive as before, one bulk copy per tile into a
+// double-buffered ring.  A warp takes KG keys at a time (16; 8 for d = 256)
+// and keeps them in registers, F features per lane: lane l holds features
+// l F .. l F + F - 1 of every key, read as one contiguous shared-memory row
+// per key.  Per query row it forms the KG partial dot products of its lane's
+// features, and a reduce-scatter over the lanes (KG - 1 shuffles, then one
+// per remaining lane bit) leaves lane l with the whole score of key
+// l mod KG.  The online softmax (maximum m and sum in log2 units) then needs
+// one max-reduction per group, and the P-weighted sum over the group's keys
+// broadcasts each key's weight from the lane that holds it.  The warps'
+// states are merged through shared memory at the end and written as the
+// item's partial rows, as above.
+constexpr int kS2Warps = 8;
+constexpr int kS2Threads = 32 * kS2Warps;
+constexpr int kS2Stages = 2;
+constexpr int kS2MaxRows = 16;
+
+template <bool XBF, int F>
+__device__ __forceinline__ void s2_load_key(const uint8_t* row, int lane, float (&x)[F]) {
+  if constexpr (XBF) {
+    const uint8_t* p = row + lane * (2 * F);
+    if constexpr (F == 1) {
+      x[0] = __uint_as_float(static_cast<uint32_t>(*reinterpret_cast<const uint16_t*>(p)) << 16);
+    } else if constexpr (F == 2) {
+      const uint32_t v = *reinterpret_cast<const uint32_t*>(p);
+      x[0] = __uint_as_float(v << 16); x[1] = __uint_as_float(v & 0xFFFF0000u);
+    } else if constexpr (F == 4) {
+      const uint2 v = *reinterpret_cast<const uint2*>(p);
+      x[0] = __uint_as_float(v.x << 16); x[1] = __uint_as_float(v.x & 0xFFFF0000u);
+      x[2] = __uint_as_float(v.y << 16); x[3] = __uint_as_float(v.y & 0xFFFF0000u);
+    } else {
+      const uint4 v = *reinterpret_cast<const uint4*>(p);
+      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        x[2 * i] = __uint_as_float(w[i] << 16);
+        x[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+      }
+    }
+  } else {
+    const float* p = reinterpret_cast<const float*>(row) + lane * F;
+    if constexpr (F == 1) {
+      x[0] = p[0];
+    } else if constexpr (F == 2) {
+      const float2 v = *reinterpret_cast<const float2*>(p);
+      x[0] = v.x; x[1] = v.y;
+    } else {
+#pragma unroll
+      for (int i = 0; i < F / 4; ++i) {
+        const float4 v = reinterpret_cast<const float4*>(p)[i];
+        x[4 * i] = v.x; x[4 * i + 1] = v.y; x[4 * i + 2] = v.z; x[4 * i + 3] = v.w;
+      }
+    }
+  }
+}
+
+// v[k] holds this lane's partial sum for key k of the group (k < KG).  Returns
+// the sum over all 32 lanes for key (lane mod KG).  Round b (KG/2, ..., 1):
+// the lane keeps the half of its values whose key bit b equals its own lane
+// bit b, and adds the partner's (lane ^ b) copy of that half; after the
+// rounds, the lanes of an aligned group of KG hold the group's sums, and the
+// remaining lane bits are summed by plain butterflies.
+template <int KG>
+__device__ __forceinline__ float s2_reduce_scatter(float (&v)[KG], int lane) {
+#pragma unroll
+  for (int b = KG / 2; b >= 1; b >>= 1) {
+    const bool hi = (lane & b) != 0;
+#pragma unroll
+    for (int j = 0; j < b; ++j) {
+      const float keep = hi ? v[j + b] : v[j];
+      const float send = hi ? v[j] : v[j + b];
+      v[j] = keep + __shfl_xor_sync(0xffffffffu, send, b);
+    }
+  }
+  float s = v[0];
+#pragma unroll
+  for (int o = KG; o < 32; o <<= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  return s;
+}
+
+template <bool XBF, int F, int QB>
+__global__ void __launch_bounds__(kS2Threads, 1)
+attn_simt2_kernel(const void* __restrict__ Xt, const float* __restrict__ U,
+                  const AttnItem* __restrict__ items, const int32_t* __restrict__ pairs,
+                  float* __restrict__ pacc, float* __restrict__ pm, float* __restrict__ pl, int kt,
+                  int us_off, int* status) {
+  constexpr int D = 32 * F;
+  constexpr int KG = F >= 8 ? 8 : 16;                  // keys per warp step
+  constexpr int ROWB = D * (XBF ? 2 : 4);              // bytes per key row (a multiple of 16)
+  constexpr float kLog2e = 1.4426950408889634f;
+  extern __shared__ __align__(128) uint8_t smem_s2[];
+  const size_t stage_bytes = static_cast<size_t>(kt) * ROWB;
+  uint8_t* stages = smem_s2;                                        // later: the merge area
+  float* us = reinterpret_cast<float*>(smem_s2 + us_off);           // QB x D query rows
+  uint64_t* full = reinterpret_cast<uint64_t*>(us + QB * D);        // kS2Stages
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int item_i = pairs[2 * blockIdx.x], row0 = pairs[2 * blockIdx.x + 1];
+  const AttnItem it = items[item_i];
+  const int nrows = min(QB, it.rows - row0);
+  const int ntiles = (it.nkeys + kt - 1) / kt;
+  const uint8_t* src0 = static_cast<const uint8_t*>(Xt) + it.key0 * ROWB;
+  if (tid == 0) {
+    for (int s = 0; s < kS2Stages; ++s)
+      asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(
+          static_cast<uint32_t>(__cvta_generic_to_shared(&full[s]))));
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+  auto issue = [&](int t) {           // thread 0: tile t into stage t % 2, one bulk copy
+    const int s = t % kS2Stages;
+    const int nk = min(kt, it.nkeys - t * kt);
+    const uint32_t bytes = static_cast<uint32_t>(nk) * ROWB;
+    const uint32_t bar = static_cast<uint32_t>(__cvta_generic_to_shared(&full[s]));
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+                 : "memory");
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            static_cast<uint32_t>(__cvta_generic_to_shared(stages + s * stage_bytes))),
+        "l"(src0 + static_cast<int64_t>(t) * stage_bytes), "r"(bytes), "r"(bar)
+        : "memory");
+  };
+  if (tid == 0)
+    for (int t = 0; t < min(ntiles, kS2Stages); ++t) issue(t);
+  for (int e = tid; e < QB * D; e += kS2Threads) {
+    const int r = e / D;
+    us[e] = r < nrows ? U[(it.qrow0 + row0 + r) * D + (e - r * D)] : 0.f;
+  }
+  __syncthreads();
+  float m[QB], lsum[QB], acc[QB][F];
+#pragma unroll
+  for (int q = 0; q < QB; ++q) {
+    m[q] = -INFINITY;
+    lsum[q] = 0.f;
+#pragma unroll
+    for (int f = 0; f < F; ++f) acc[q][f] = 0.f;
+  }
+  const int myk = lane & (KG - 1);      // the key of the group whose score this lane ends with
+  bool ok = true;
+  for (int t = 0; t < ntiles; ++t) {
+    const int s = t % kS2Stages;
+    if (ok) ok = simt_wait(&full[s], (t / kS2Stages) & 1, status);
+    ok = __syncthreads_and(ok) != 0;      // one decision for the whole CTA (the loop below shuffles)
+    const int nk = min(kt, it.nkeys - t * kt);
+    const uint8_t* tile = stages + s * stage_bytes;
+    if (ok) {
+      for (int g0 = warp * KG; g0 < nk; g0 += kS2Warps * KG) {   // warp-uniform trip count
+        float x[KG][F];
+#pragma unroll
+        for (int k = 0; k < KG; ++k) {
+          if (g0 + k < nk) {
+            s2_load_key<XBF, F>(tile + static_cast<size_t>(g0 + k) * ROWB, lane, x[k]);
+          } else {
+#pragma unroll
+            for (int f = 0; f < F; ++f) x[k][f] = 0.f;
+          }
+        }
+        const bool kvalid = g0 + myk < nk;
+#pragma unroll
+        for (int q = 0; q < QB; ++q) {
+          if (q >= nrows) break;                              // CTA-uniform
+          float uq[F];
+#pragma unroll
+          for (int f = 0; f < F; ++f) uq[f] = us[q * D + lane * F + f];
+          float v[KG];
+#pragma unroll
+          for (int k = 0; k < KG; ++k) {
+            float a = 0.f;
+#pragma unroll
+            for (int f = 0; f < F; ++f) a = fmaf(uq[f], x[k][f], a);
+            v[k] = a;
+          }
+          const float sc = s2_reduce_scatter<KG>(v, lane);
+          const float s2 = kvalid ? sc * kLog2e : -INFINITY;   // log2 units
+          float gm = s2;
+#pragma unroll
+          for (int o = 1; o < KG; o <<= 1) gm = fmaxf(gm, __shfl_xor_sync(0xffffffffu, gm, o));
+          if (gm > m[q]) {                                      // warp-uniform
+            const float corr = sx::ex2(m[q] - gm);              // 0 from m = -inf
+            lsum[q] *= corr;
+#pragma unroll
+            for (int f = 0; f < F; ++f) acc[q][f] *= corr;
+            m[q] = gm;
+          }
+          const float p = kvalid ? sx::ex2(s2 - m[q]) : 0.f;
+          if (lane < KG) lsum[q] += p;                          // one copy of each key's weight
+#pragma unroll
+          for (int k = 0; k < KG; ++k) {
+            const float pk = __shfl_sync(0xffffffffu, p, k);
+#pragma unroll
+            for (int f = 0; f < F; ++f) acc[q][f] = fmaf(pk, x[k][f], acc[q][f]);
+          }
+        }
+      }
+    }
+    __syncthreads();                      // every warp is done with stage s
+    if (tid == 0 && ok && t + kS2Stages < ntiles) issue(t + kS2Stages);
+  }
+  // let copies still in flight (after a failed wait) land before the stages are reused
+  if (tid == 0)
+    for (int t = max(0, ntiles - kS2Stages); t < ntiles; ++t)
+      simt_wait(&full[t % kS2Stages], (t / kS2Stages) & 1, status);
+  __syncthreads();
+  // merge the warps' states: warp w, row q -> [D + 2] floats (accumulator, m, l)
+  float* st = reinterpret_cast<float*>(smem_s2);              // the stages are free now
+#pragma unroll
+  for (int q = 0; q < QB; ++q) {
+    if (q >= nrows) break;
+    float* row = st + (static_cast<size_t>(warp) * QB + q) * (D + 2);
+#pragma unroll
+    for (int f = 0; f < F; ++f) row[lane * F + f] = acc[q][f];
+    float ls = lsum[q];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ls += __shfl_xor_sync(0xffffffffu, ls, o);
+    if (lane == 0) { row[D] = m[q]; row[D + 1] = ls; }
+  }
+  __syncthreads();
+  for (int e = tid; e < nrows * D; e += kS2Threads) {
+    const int r = e / D, f = e - r * D;
+    float mx = -INFINITY;
+    for (int w = 0; w < kS2Warps; ++w) mx = fmaxf(mx, st[(static_cast<size_t>(w) * QB + r) * (D + 2) + D]);
+    float a = 0.f, lt = 0.f;
+    for (int w = 0; w < kS2Warps; ++w) {
+      const float* row = st + (static_cast<size_t>(w) * QB + r) * (D + 2);
+      const float wt = row[D + 1] > 0.f ? sx::ex2(row[D] - mx) : 0.f;   // a warp with no key: 0
+      a = fmaf(wt, row[f], a);
+      lt = fmaf(wt, row[D + 1], lt);
+    }
+    const int64_t gr = it.row_base + row0 + r;
+    pacc[gr * D + f] = a;
+    if (f == 0) {
+      pm[gr] = mx * 0.6931471805599453f;              // natural-log units for the combine
+      pl[gr] = lt;
+    }
+  }
+}
+
 }  // namespace
 
 // ------------------------------------------------------------------ launchers
@@ -403,9 +648,35 @@ SimtGeom simt_geom(int d, int elem) {
 }
 }  // namespace
 
-int attn_simt_rows_per_cta(int d) { return simt_geom(d, 4).rb; }
+namespace {
+// The feature-per-lane kernel covers d in {32, 64, 128, 256}; other widths
+// take the key-per-group kernel above.
+bool simt2_supported(int d) { return d == 32 || d == 64 || d == 128 || d == 256; }
 
-size_t attn_simt_smem(const stca_handle* H) { return simt_geom(H->d, H->elem).smem; }
+struct Simt2Geom {
+  int kt;
+  size_t us_off, smem;
+};
+
+// kt keys per tile (at most 32 KB a stage); shared memory for QB rows: the
+// stages (reused as the warps' merge area), the query rows, the mbarriers
+Simt2Geom simt2_geom(int d, int elem, int qb) {
+  Simt2Geom g{};
+  const int rowb = d * elem;
+  g.kt = std::max(8, std::min(256, (32 << 10) / rowb) / 8 * 8);
+  const size_t stages = static_cast<size_t>(kS2Stages) * g.kt * rowb;
+  const size_t merge = static_cast<size_t>(kS2Warps) * qb * (d + 2) * sizeof(float);
+  g.us_off = (std::max(stages, merge) + 15) / 16 * 16;
+  g.smem = g.us_off + static_cast<size_t>(qb) * d * sizeof(float) + 64;
+  return g;
+}
+}  // namespace
+
+int attn_simt_rows_per_cta(int d) { return simt2_supported(d) ? kS2MaxRows : simt_geom(d, 4).rb; }
+
+size_t attn_simt_smem(const stca_handle* H) {
+  return simt2_supported(H->d) ? simt2_geom(H->d, H->elem, kS2MaxRows).smem : simt_geom(H->d, H->elem).smem;
+}
 
 void launch_attn_simt(const stca_handle* H, int layer, const void* xt_layer,
                       const AttnItem* items_d, const int32_t* pairs_d, int64_t npairs,
@@ -413,11 +684,43 @@ void launch_attn_simt(const stca_handle* H, int layer, const void* xt_layer,
   (void)layer;
   (void)toff_d;
   if (npairs <= 0) return;
-  const SimtGeom g = simt_geom(H->d, H->elem);
   const int64_t G = H->last_G;
   float* pacc = H->part;
   float* pm = pacc + G * H->d;
   float* pl = pm + G;
+  if (simt2_supported(H->d)) {
+    // QB: the smallest of 4, 8, 16 rows that holds every (item, row block)
+    int64_t most = 1;
+    for (size_t r = 0; r + 1 < H->last_toff.size(); ++r)
+      most = std::max<int64_t>(most, (H->last_toff[r + 1] - H->last_toff[r]) * H->h);
+    const int qb = most <= 4 ? 4 : most <= 8 ? 8 : kS2MaxRows;
+    const Simt2Geom g = simt2_geom(H->d, H->elem, qb);
+#define STCA_SIMT2(XB, FF, QQ)                                                                      \
+  do {                                                                                              \
+    auto k = attn_simt2_kernel<XB, FF, QQ>;                                                         \
+    cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)g.smem);              \
+    k<<<static_cast<unsigned>(npairs), kS2Threads, g.smem, s>>>(xt_layer, H->U, items_d, pairs_d,   \
+                                                                pacc, pm, pl, g.kt, (int)g.us_off,  \
+                                                                H->status_d);                       \
+  } while (0)
+#define STCA_SIMT2_Q(XB, FF)                        \
+  do {                                              \
+    if (qb == 4) STCA_SIMT2(XB, FF, 4);             \
+    else if (qb == 8) STCA_SIMT2(XB, FF, 8);        \
+    else STCA_SIMT2(XB, FF, kS2MaxRows);            \
+  } while (0)
+    const bool bf = H->elem == 2;
+    switch (H->d) {
+      case 32: if (bf) STCA_SIMT2_Q(true, 1); else STCA_SIMT2_Q(false, 1); break;
+      case 64: if (bf) STCA_SIMT2_Q(true, 2); else STCA_SIMT2_Q(false, 2); break;
+      case 128: if (bf) STCA_SIMT2_Q(true, 4); else STCA_SIMT2_Q(false, 4); break;
+      default: if (bf) STCA_SIMT2_Q(true, 8); else STCA_SIMT2_Q(false, 8); break;
+    }
+#undef STCA_SIMT2_Q
+#undef STCA_SIMT2
+    return;
+  }
+  const SimtGeom g = simt_geom(H->d, H->elem);
 #define STCA_SIMT(XB, NC)                                                                          \
   do {                                                                                             \
     auto k = attn_simt_kernel<XB, NC>;                                                             \

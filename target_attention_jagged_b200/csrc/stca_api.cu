@@ -779,7 +779,13 @@ int stca::check_plan(const PlanHost& P, const int64_t* off, const int64_t* toff,
 // targets per CTA), both checked, then joined into one plan: half B's items,
 // pairs and partial rows follow half A's, and its CTA runs follow A's
 // grid + 1 entries of cta_begin.  False when it does not apply (a half would
-// be empty, or a pair would have more items than the step merges).
+// be empty, or a pair would have more items than the step merges) or does not
+// pay: every pipelined launch holds a per-target step, whose latency (about
+// 20 key tiles of attention per SM) the other half's attention must cover, so
+// a batch with less than kPipeMinWork key tiles x query tiles per SM runs in
+// one piece (measured: the pipeline slowed a 32-request batch of 200..2000 keys
+// by half, and left the 64 x 10000-key serving batch, 34 per SM, even).
+constexpr int64_t kPipeMinWork = 24;
 static bool build_pipe_plan(stca_handle* H, const int64_t* off, const int64_t* toff, int64_t R,
                             PlanHost& P) {
   const int h = H->h;
@@ -787,6 +793,7 @@ static bool build_pipe_plan(stca_handle* H, const int64_t* off, const int64_t* t
   std::vector<int64_t> work(R + 1, 0);
   for (int64_t r = 0; r < R; ++r)
     work[r + 1] = work[r] + ((toff[r + 1] - toff[r]) * h + 127) / 128 * ((off[r + 1] - off[r] + 127) / 128);
+  if (work[R] < kPipeMinWork * H->num_sms) return false;
   int64_t RA = 1;
   while (RA < R - 1 && 2 * work[RA] < work[R]) ++RA;
   const int64_t TA = toff[RA], T = toff[R];

@@ -288,7 +288,9 @@ def test_tc_kernels_sharp_softmax(gpu, kernel):
 # the halves split the requests by attention work, and one launch runs one
 # half's per-target step beside the other half's attention.  It applies when
 # each pair (request, query tile) of the halves' plans has at most 8 items,
-# i.e. with enough pairs per half; otherwise the forward runs in one piece.
+# i.e. with enough pairs per half, and when the batch holds at least 24 pairs
+# (key tile, query tile) of attention work per SM; otherwise the forward runs
+# in one piece.
 def _forward_launches(wl, gpu, pipeline):
     """Z and the number of kernels one forward launched."""
     import torch
@@ -307,13 +309,14 @@ def _forward_launches(wl, gpu, pipeline):
 
 @pytest.mark.parametrize("seed", [0, 1])
 def test_pipeline_matches_oracle(gpu, seed):
-    """80 requests of 600..2000 keys: the pipeline engages (2M + 2 launches
-    against 2M + 1), matches the oracle on sampled requests and the one-piece
-    forward on the whole batch.  Seed 1 has ragged targets (0 to 40 per
-    request: several query tiles, empty requests)."""
+    """80 requests of 4000..8000 keys (about 3700 pairs of attention work, 25
+    per SM): the pipeline engages (2M + 2 launches against 2M + 1), matches
+    the oracle on sampled requests and the one-piece forward on the whole
+    batch.  Seed 1 has ragged targets (0 to 40 per request: several query
+    tiles, empty requests)."""
     rng = np.random.default_rng(seed)
     R = 80
-    lengths = rng.integers(600, 2001, R).tolist()
+    lengths = rng.integers(4000, 8001, R).tolist()
     targets = [16] * R if seed == 0 else rng.integers(0, 41, R).tolist()
     wl = make_workload(lengths=lengths, targets=targets, d=128, h=8, M=3, r=2, dtype="bf16", seed=430 + seed)
     a, na = _forward_launches(wl, gpu, 1)
@@ -321,6 +324,19 @@ def test_pipeline_matches_oracle(gpu, seed):
     assert na == 2 * wl.M + 2 and nb == 2 * wl.M + 1, (na, nb)
     check_sampled(wl, a, 4, seed=seed)
     assert normwise_err(a, b) <= 2e-2
+
+
+def test_pipeline_skips_small_batches(gpu):
+    """32 requests of 200..2000 keys, 8 targets each: too little attention
+    work per SM for the pipeline to pay, so the forward runs in one piece (the
+    launches of the pipeline-off forward) and gives the same Z."""
+    wl = make_workload(lengths=("uniform", 200, 2000), targets=("fixed", 8), d=128, h=4, M=2, r=2,
+                       dtype="bf16", seed=442, R=32)
+    a, na = _forward_launches(wl, gpu, 1)
+    b, nb = _forward_launches(wl, gpu, 0)
+    assert na == nb, (na, nb)
+    assert normwise_err(a, b) == 0.0
+    check_sampled(wl, a, 4, seed=5)
 
 
 def test_pipeline_falls_back(gpu):
