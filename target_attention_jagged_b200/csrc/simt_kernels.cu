@@ -362,7 +362,8 @@ attn_simt_kernel(const void* __restrict__ Xt, const float* __restrict__ U,
 // per key.  Per query row it forms the KG partial dot products of its lane's
 // features, and a reduce-scatter over the lanes (KG - 1 shuffles, then one
 // per remaining lane bit) leaves lane l with the whole score of key
-// l mod KG.  The online softmax (maximum m and sum in log2 units) then needs
+// l mod KG.  With QB = 4 the kernel is held to 128 registers, so two CTAs
+// share an SM.  The online softmax (maximum m and sum in log2 units) then needs
 // one max-reduction per group, and the P-weighted sum over the group's keys
 // broadcasts each key's weight from the lane that holds it.  The warps'
 // states are merged through shared memory at the end and written as the
@@ -436,7 +437,7 @@ __device__ __forceinline__ float s2_reduce_scatter(float (&v)[KG], int lane) {
 }
 
 template <bool XBF, int F, int QB>
-__global__ void __launch_bounds__(kS2Threads, 1)
+__global__ void __launch_bounds__(kS2Threads, QB <= 4 ? 2 : 1)
 attn_simt2_kernel(const void* __restrict__ Xt, const float* __restrict__ U,
                   const AttnItem* __restrict__ items, const int32_t* __restrict__ pairs,
                   float* __restrict__ pacc, float* __restrict__ pm, float* __restrict__ pl, int kt,

@@ -71,6 +71,18 @@ def test_ragged_edges(gpu, dtype, d, h, M, r, attn):
     check_full(wl, run_gpu(wl, gpu, attn_path=attn))
 
 
+# The CUDA-core attention's row blocks: its launch picks the block height QB
+# (4, 8 or 16 rows) from the batch's largest T_r h, so these target mixes reach
+# each QB, and the 24- and 48-row requests need more than one block; the key
+# counts leave partial groups of 16 (8 at d = 256) and a partial tile.
+@pytest.mark.parametrize("targets", [[1, 2, 1, 2, 1], [4, 1, 3, 2, 4], [12, 1, 5, 9, 3]])
+@pytest.mark.parametrize("dtype,d,h", [("f32", 32, 2), ("bf16", 32, 2), ("f32", 256, 4), ("bf16", 128, 2)])
+def test_simt_row_blocks(gpu, dtype, d, h, targets):
+    wl = make_workload(lengths=[1, 15, 130, 515, 1021], targets=targets, d=d, h=h, M=2, r=2,
+                       dtype=dtype, seed=200 + d + sum(targets))
+    check_full(wl, run_gpu(wl, gpu, attn_path=ATTN_SIMT))
+
+
 @pytest.mark.parametrize("attn", [ATTN_TC, ATTN_SIMT])
 def test_many_targets_per_request(gpu, attn):
     # T_r * h = 40 * 8 = 320 query rows: three 128-row tiles, the last ragged
