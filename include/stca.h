@@ -158,6 +158,25 @@ int stca_forward(stca_handle* handle, const void* targets, const int64_t* target
                  int64_t T, float* Z, void* stream);
 
 /*
+ * stca_encode followed by stca_forward on the same stream, in one call: the
+ * serving step of request-level batching ("Make It Long, Keep It Fast"
+ * digest, §2.2: encode each request's history once, then attend to it for all
+ * of its targets; Eqs. (2)-(8)).  Arguments, results and errors are those of
+ * the two calls: X, offsets, R, N as for stca_encode; targets,
+ * target_offsets, T, Z as for stca_forward (T == 0 encodes only).  The
+ * encoded histories stay valid for later stca_forward calls.
+ * Because nothing can be enqueued between the two parts, the first per-target
+ * launch of the two-half pipeline (the query initialisation of the first
+ * half, which reads only the targets and the weights) may start on the SMs
+ * that the encoder's last round of tiles leaves idle, before the encoder has
+ * finished.  The targets must therefore be complete before the call's work
+ * starts on the stream, as for stca_encode's X.  Same Z as the two calls.
+ */
+int stca_encode_forward(stca_handle* handle, const void* X, const int64_t* offsets, int64_t R,
+                        int64_t N, const void* targets, const int64_t* target_offsets, int64_t T,
+                        float* Z, void* stream);
+
+/*
  * Prediction-head token of Eq. (9) ("Make It Long, Keep It Fast" digest,
  * §2.1, Eq. (9)) for T targets:
  *   zout[t] = SwiGLUFFN_z([Z[t, 0, :] || ... || Z[t, M-1, :] || x_t] W_Z)

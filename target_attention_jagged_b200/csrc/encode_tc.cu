@@ -169,6 +169,13 @@ encode_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   pdl_wait();                          // the predecessor's results are visible from here on
+  // Dependents may launch now: every CTA of this persistent grid is resident
+  // (a dependent launches only once all of them have passed this point), so a
+  // dependent CTA takes an SM only when an encoder CTA has left it.  Each
+  // dependent waits for this grid's completion before it reads what this grid
+  // writes, except the query init after stca_encode_forward, which reads none
+  // of it and uses the SMs of the CTAs that finish a round of tiles early.
+  pdl_trigger();
   const uint32_t sbase = smem_u32(sm);
 
   if (warp == 0) {
@@ -482,7 +489,6 @@ encode_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
   }
   tc_fence_before();
   __syncthreads();
-  pdl_trigger();
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);

@@ -511,8 +511,13 @@ static int encode_begin(stca_handle* H, const void* X, const int64_t* offsets, i
   H->encoded = false;
   H->R = R;
   H->N = N;
+  // the attention plan depends on the key layout: a batch with other offsets
+  // needs a new one, the same layout keeps the one on the device (no upload
+  // between the encoder and the forward's first launch)
+  if (H->offsets_h.size() != static_cast<size_t>(R + 1) ||
+      !std::equal(H->offsets_h.begin(), H->offsets_h.end(), offsets))
+    H->last_toff.clear();
   H->offsets_h.assign(offsets, offsets + R + 1);
-  H->last_toff.clear();          // plan must be rebuilt for the next forward
   H->launches = 0;
   if (H->dtype == STCA_BF16 && attn_tc_supported(H->d)) {
     for (int i = 0; i < H->M; ++i)
@@ -940,8 +945,11 @@ static bool naive_cheaper(const stca_handle* H, const int64_t* toff) {
 // The forward of stca_forward; with zout, also the prediction-head token of
 // Eq. (9), inside the last per-target step when that runs on the tensor cores,
 // else by the separate head kernel after it.
+// after_encode: the call directly follows this library's encoder launch on
+// the stream (stca_encode_forward, stca_run_host), so the two-half pipeline's
+// query init may overlap the encoder's last round of tiles.
 static int forward_impl(stca_handle* H, const void* targets, const int64_t* target_offsets,
-                        int64_t T, float* Z, float* zout, void* stream) {
+                        int64_t T, float* Z, float* zout, void* stream, bool after_encode = false) {
   if (!H) return set_error(STCA_EINVAL, "handle is NULL");
   if (!H->encoded) return set_error(STCA_ESTATE, "stca_forward before a successful stca_encode");
   if (T < 0) return set_error(STCA_EINVAL, "T must be >= 0");
@@ -1085,7 +1093,9 @@ static int forward_impl(stca_handle* H, const void* targets, const int64_t* targ
     PipeAttn aB{0, items_d, cta_d + H->pipe_gridA + 1, H->pipe_gridB, qs};
     {
       TimedLaunch tl(H, STCA_K_STEP, s);
-      if (int rc = launch_step_tc(H, -1, tg, TA, nullptr, &plan, H->part, H->last_G, Z, H->Ubf, s)) return rc;
+      if (int rc = launch_step_tc(H, -1, tg, TA, nullptr, &plan, H->part, H->last_G, Z, H->Ubf, s, nullptr,
+                                  nullptr, 0, nullptr, after_encode && !H->timing))
+        return rc;
     }
     if (int rc2 = check_launch("query init")) return rc2;
     for (int i = 0; i < M; ++i) {
@@ -1173,6 +1183,13 @@ static int forward_impl(stca_handle* H, const void* targets, const int64_t* targ
 extern "C" int stca_forward(stca_handle* H, const void* targets, const int64_t* target_offsets,
                             int64_t T, float* Z, void* stream) {
   return forward_impl(H, targets, target_offsets, T, Z, nullptr, stream);
+}
+
+extern "C" int stca_encode_forward(stca_handle* H, const void* X, const int64_t* offsets, int64_t R,
+                                   int64_t N, const void* targets, const int64_t* target_offsets,
+                                   int64_t T, float* Z, void* stream) {
+  if (int rc = stca_encode(H, X, offsets, R, N, stream)) return rc;
+  return forward_impl(H, targets, target_offsets, T, Z, nullptr, stream, true);
 }
 
 extern "C" int stca_forward_head(stca_handle* H, const void* targets, const int64_t* target_offsets,
@@ -1337,7 +1354,7 @@ extern "C" int stca_run_host(stca_handle* H, const void* X_host, const int64_t* 
     H->encoded = true;
   }
   if (T > 0) {
-    if (int rc = stca_forward(H, H->t_stage, target_offsets, T, H->z_stage, stream)) return rc;
+    if (int rc = forward_impl(H, H->t_stage, target_offsets, T, H->z_stage, nullptr, stream, true)) return rc;
     STCA_CUDA_TRY(cudaMemcpyAsync(Z_host, H->z_stage, zb, cudaMemcpyDeviceToHost, s));
   }
   STCA_CUDA_TRY(cudaStreamSynchronize(s));
@@ -1406,6 +1423,7 @@ extern "C" int stca_set_option(stca_handle* H, int option, int64_t value) {
     case STCA_OPT_SPLIT_KEYS:
       if (value < 0 || value % 128 || value > (int64_t(1) << 30))
         return set_error(STCA_EINVAL, "split must be 0 or a positive multiple of 128");
+      if (value != H->opt_split_keys) H->last_toff.clear();   // the plan cuts the keys by it
       H->opt_split_keys = value;
       return ok();
     default:

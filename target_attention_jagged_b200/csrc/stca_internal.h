@@ -265,11 +265,14 @@ struct NaiveStep {
 // proj: the attention already projected its rows by W_V (d_h-wide partials of
 // o_j): 1 cmerged holds the merged o_head (T x d); 2 cmerged is NULL and the
 // step merges the partials (part) itself, at most step_tc_max_items_proj()
-// items per query row.
+// items per query row.  defer_wait (query init only, layer < 0): the launch
+// directly follows this library's encoder launch on the stream, with nothing
+// in between, so the kernel waits for it at its end rather than its start.
 int launch_step_tc(const stca_handle* H, int layer, const void* targets, int64_t T,
                    const float* cmerged, const StepPlan* plan, const float* part, int64_t G,
                    float* Z, uint16_t* Ubf, cudaStream_t s, const NaiveStep* naive = nullptr,
-                   float* zout = nullptr, int proj = 0, const QslotBufs* qs = nullptr);
+                   float* zout = nullptr, int proj = 0, const QslotBufs* qs = nullptr,
+                   bool defer_wait = false);
 
 // One phase of the two-half pipeline (stca_forward at d = 128 with the
 // in-kernel projection): one launch runs the per-target step of one half of

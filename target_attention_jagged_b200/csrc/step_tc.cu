@@ -201,6 +201,8 @@ struct StepTcArgs {
   const int* qn;
   int wk_tc;                    // the W_K products run on the tensor cores (product kind kK)
   int qtot;                     // A tiles of this launch (kK's Pblk takes the next two ring slots)
+  int defer_wait;               // query init right after this library's encoder launch: wait for
+                                // the predecessor at the end, not the start (see launch_step_tc)
 };
 
 // Shared memory, in bytes (1024-aligned base): the A-tile ring, then the
@@ -320,7 +322,7 @@ __device__ __forceinline__ void step_tc_body(const StepTcArgs& a, uint8_t* smem_
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  pdl_wait();                          // the predecessor's results are visible from here on
+  if (!a.defer_wait) pdl_wait();       // the predecessor's results are visible from here on
 
   if (warp == 0) {
     // ------------------------------------------------------------ weight streamer
@@ -486,7 +488,7 @@ __device__ __forceinline__ void step_tc_body(const StepTcArgs& a, uint8_t* smem_
     if (L < 0) {
       for (int e = tid; e < kTgt * d; e += 32 * kWorkers) {
         const int t = e / d, k = e - t * d;
-        put_b1(bufs[kUG], t, k, t < nb ? bf2f(a.targets[(t0 + t) * d + k]) : 0.f);
+        put_b1(bufs[kUG], t, k, t < nb ? bf2f(__ldcg(a.targets + (t0 + t) * d + k)) : 0.f);
       }
     } else {
       if (concat && a.head_only) {
@@ -934,6 +936,9 @@ __device__ __forceinline__ void step_tc_body(const StepTcArgs& a, uint8_t* smem_
       }
     }
   }
+  // deferred: this grid completes only after its predecessor has, so the
+  // launches after it see the predecessor's results as well
+  if (a.defer_wait) pdl_wait();
   tc_fence_before();
   __syncthreads();
   pdl_trigger();
@@ -1126,7 +1131,7 @@ static_assert(kStepThreads <= kAttnThreads, "the pipeline kernel runs both bodie
 int launch_step_tc(const stca_handle* H, int layer, const void* targets, int64_t T,
                    const float* cmerged, const StepPlan* plan, const float* part, int64_t G,
                    float* Z, uint16_t* Ubf, cudaStream_t s, const NaiveStep* naive, float* zout,
-                   int proj, const QslotBufs* qs) {
+                   int proj, const QslotBufs* qs, bool defer_wait) {
   if (T <= 0) return STCA_OK;
   StepTcArgs a;
   size_t smem;
@@ -1134,6 +1139,12 @@ int launch_step_tc(const stca_handle* H, int layer, const void* targets, int64_t
   if (int rc = make_step_args(H, layer, targets, T, cmerged, plan, part, G, Z, Ubf, naive, zout, proj, qs, a,
                               smem, grid))
     return rc;
+  // The query init reads only the targets and the weights and writes only U
+  // rows, so right after this library's encoder launch (which triggers its
+  // dependents once its own wait is over) it may start on the SMs the
+  // encoder's last, shorter round of tiles leaves idle, and wait for the
+  // encoder at its end instead.
+  a.defer_wait = defer_wait && layer < 0 ? 1 : 0;
   cudaError_t e = cudaFuncSetAttribute(step_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return set_error(STCA_ECUDA, std::string("step_tc smem: ") + cudaGetErrorString(e));

@@ -36,7 +36,7 @@ STCA_K_ENCODE, STCA_K_ATTN, STCA_K_STEP, STCA_K_HEAD, STCA_K_PIPE, STCA_K_CLASSE
 _NAMES = {STCA_EINVAL: "EINVAL", STCA_ESTATE: "ESTATE", STCA_ENOMEM: "ENOMEM",
           STCA_ECUDA: "ECUDA", STCA_EDEVICE: "EDEVICE"}
 
-EXPORTS = ("stca_init", "stca_destroy", "stca_encode", "stca_forward", "stca_run_host",
+EXPORTS = ("stca_init", "stca_destroy", "stca_encode", "stca_forward", "stca_encode_forward", "stca_run_host",
            "stca_validate_offsets", "stca_device_status", "stca_set_option",
            "stca_get_option", "stca_kernel_times", "stca_get_encoded", "stca_plan_attention",
            "stca_forward_static", "stca_head", "stca_forward_head", "stca_sl_beta", "stca_sl_plan",
@@ -63,6 +63,7 @@ def _load():
     lib.stca_destroy.restype = None
     lib.stca_encode.argtypes = [P, P, PI64, I64, I64, P]
     lib.stca_forward.argtypes = [P, P, PI64, I64, P, P]
+    lib.stca_encode_forward.argtypes = [P, P, PI64, I64, I64, P, PI64, I64, P, P]
     lib.stca_forward_static.argtypes = [P, P, PI64, I64, P, P]
     lib.stca_head.argtypes = [P, P, I64, P, P, P]
     lib.stca_forward_head.argtypes = [P, P, PI64, I64, P, P, P]
@@ -223,6 +224,22 @@ def stca_forward(handle: int, targets, target_offsets, Z=None, stream=None):
     assert Z.dtype == torch.float32 and Z.is_cuda and Z.is_contiguous()
     _check(_lib.stca_forward(handle, targets.data_ptr() if T > 0 else None, _i64p(toff), T,
                              Z.data_ptr() if T > 0 else None, _stream_ptr(stream)))
+    return Z
+
+
+def stca_encode_forward(handle: int, X, offsets, targets, target_offsets, Z, stream=None):
+    """stca_encode then stca_forward in one call (see include/stca.h): X (N x d)
+    and targets (T x d) CUDA tensors in the handle's dtype, host int64 offsets;
+    fills and returns Z (T x M x d fp32 CUDA tensor)."""
+    import torch
+    off, toff = _offsets(offsets), _offsets(target_offsets)
+    R = off.shape[0] - 1
+    N = int(off[-1]) if R >= 0 else 0
+    T = int(toff[-1])
+    assert Z.dtype == torch.float32 and Z.is_cuda and Z.is_contiguous()
+    _check(_lib.stca_encode_forward(handle, X.data_ptr(), _i64p(off), R, N,
+                                    targets.data_ptr() if T > 0 else None, _i64p(toff), T,
+                                    Z.data_ptr() if T > 0 else None, _stream_ptr(stream)))
     return Z
 
 
@@ -525,6 +542,14 @@ class Stca:
         if Z is None:
             Z = torch.empty((T, self.M, self.d), dtype=torch.float32, device=targets.device)
         return stca_forward(self.handle, targets, target_offsets, Z, stream)
+
+    def encode_forward(self, X, offsets, targets, target_offsets, Z=None, stream=None):
+        """encode then forward in one call; returns Z."""
+        import torch
+        T = int(np.asarray(target_offsets)[-1])
+        if Z is None:
+            Z = torch.empty((T, self.M, self.d), dtype=torch.float32, device=targets.device)
+        return stca_encode_forward(self.handle, X, offsets, targets, target_offsets, Z, stream)
 
     def forward_head(self, targets, target_offsets, Z=None, zout=None, stream=None):
         """Z of the forward and z of Eq. (9) in one call."""

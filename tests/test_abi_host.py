@@ -101,6 +101,7 @@ def test_null_handle_calls_fail_cleanly():
     off = (ctypes.c_int64 * 2)(0, 4)
     assert lib.stca_encode(None, None, off, 1, 4, None) == B.STCA_EINVAL
     assert lib.stca_forward(None, None, off, 4, None, None) == B.STCA_EINVAL
+    assert lib.stca_encode_forward(None, None, off, 1, 4, None, off, 4, None, None) == B.STCA_EINVAL
     assert lib.stca_set_option(None, 1, 0) == B.STCA_EINVAL
     v = ctypes.c_int64()
     assert lib.stca_get_option(None, 1, ctypes.byref(v)) == B.STCA_EINVAL

@@ -338,6 +338,46 @@ def test_pipeline_matches_oracle(gpu, seed):
     assert normwise_err(a, b) <= 2e-2
 
 
+@pytest.mark.parametrize("big", [True, False])
+def test_encode_forward_matches_separate_calls(gpu, big):
+    """stca_encode_forward (one call: the first half's query init may overlap
+    the encoder's last tiles) gives the Z of stca_encode + stca_forward, bit
+    for bit, twice in a row; big: 80 requests of 4000..8000 keys (the two-half
+    pipeline engages), else a small ragged batch (one piece)."""
+    import torch
+    import target_attention_jagged_b200 as S
+    from tests.gpu_helpers import storage_weights, to_device
+    if big:
+        rng = np.random.default_rng(3)
+        wl = make_workload(lengths=rng.integers(4000, 8001, 80).tolist(), targets=[16] * 80, d=128, h=8,
+                           M=3, r=2, dtype="bf16", seed=450)
+    else:
+        wl = make_workload(lengths=EDGE_L, targets=EDGE_T, d=128, h=4, M=2, r=2, dtype="bf16", seed=451)
+    X, xt = to_device(wl, wl.X, gpu), to_device(wl, wl.targets, gpu)
+    with S.Stca(storage_weights(wl), wl.d, wl.h, wl.r, wl.M, wl.dtype) as st:
+        st.encode(X, wl.offsets)
+        want = torch.zeros((wl.T, wl.M, wl.d), dtype=torch.float32, device=gpu)
+        st.forward(xt, wl.target_offsets, want)
+        n0 = st.get_option(S.STCA_OPT_LAUNCHES)
+        for _ in range(2):
+            got = torch.full((wl.T, wl.M, wl.d), float("nan"), dtype=torch.float32, device=gpu)
+            st.encode_forward(X, wl.offsets, xt, wl.target_offsets, got)
+            torch.cuda.synchronize()
+            st.status()
+            assert torch.equal(got, want)
+        # the launches of one encode and one forward (the counter restarts at
+        # each encode): the encoder, then 2M + 2 launches with the pipeline,
+        # 2M + 1 without
+        assert st.get_option(S.STCA_OPT_LAUNCHES) == n0 == 1 + (2 * wl.M + 2 if big else 2 * wl.M + 1)
+        # T == 0: encodes only; a later forward reuses the encoding
+        S.stca_encode_forward(st.handle, X, wl.offsets, xt[:0], np.zeros(wl.R + 1, dtype=np.int64), want[:0])
+        again = torch.zeros_like(want)
+        st.forward(xt, wl.target_offsets, again)
+        torch.cuda.synchronize()
+        assert torch.equal(again, want)
+    check_sampled(wl, want.cpu().numpy(), 3, seed=6)
+
+
 def test_pipeline_skips_small_batches(gpu):
     """32 requests of 200..2000 keys, 8 targets each: too little attention
     work per SM for the pipeline to pay, so the forward runs in one piece (the
