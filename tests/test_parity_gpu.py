@@ -112,6 +112,34 @@ def test_split_sizes_agree(gpu, split, attn):
     check_full(wl, run_gpu(wl, gpu, split=split, attn_path=attn))
 
 
+def test_split_change_rebuilds_the_plan(gpu):
+    """The attention plan is kept on the device between forwards (and
+    encodes) of one layout; a new STCA_OPT_SPLIT_KEYS must replace it.  64
+    requests of 1280 keys (10 key tiles, one query tile): the default plan
+    cuts a pair into at most 2 items and the step merges the partials itself;
+    with 128-key items a pair has 10, more than the step merges, so each layer
+    adds a combine launch.  All match the oracle on sampled requests."""
+    import torch
+    import target_attention_jagged_b200 as S
+    from tests.gpu_helpers import storage_weights, to_device
+    wl = make_workload(lengths=[1280] * 64, targets=[3] * 64, d=128, h=4, M=2, r=2,
+                       dtype="bf16", seed=12)
+    X, xt = to_device(wl, wl.X, gpu), to_device(wl, wl.targets, gpu)
+    with S.Stca(storage_weights(wl), wl.d, wl.h, wl.r, wl.M, wl.dtype) as st:
+        st.encode(X, wl.offsets)
+        counts = []
+        for split in (0, 128, 0):
+            st.set_option(S.STCA_OPT_SPLIT_KEYS, split)
+            n0 = st.get_option(S.STCA_OPT_LAUNCHES)
+            Z = torch.zeros((wl.T, wl.M, wl.d), dtype=torch.float32, device=gpu)
+            st.forward(xt, wl.target_offsets, Z)
+            torch.cuda.synchronize()
+            st.status()
+            counts.append(st.get_option(S.STCA_OPT_LAUNCHES) - n0)
+            check_sampled(wl, Z.cpu().numpy(), 3, seed=len(counts))
+        assert counts[1] == counts[0] + wl.M and counts[2] == counts[0], counts
+
+
 def test_sharp_softmax_rescaling(gpu):
     # The first key tile of each request repeats one token, so its scores are
     # all equal and the running max jumps by far more than the lazy-rescale
