@@ -879,7 +879,8 @@ def main():
         run_reference(args, rank)
         return
     if args.attn_paths:
-        attn_paths_sweep()
+        if rank == 0:               # a one-GPU sweep: other ranks have nothing to do
+            attn_paths_sweep()
         return
     if world > 1:
         import torch
