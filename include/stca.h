@@ -152,6 +152,12 @@ int stca_encode(stca_handle* handle, const void* X, const int64_t* offsets,
  *   T               total targets (target_offsets[R]); T == 0 is a no-op
  *   Z               device pointer, caller-owned, T x M x d fp32; row t holds
  *                   [o(1); ...; o(M)] of target t (Eq. (8))
+ * The attention's work plan depends on the key layout (the offsets of the last
+ * encode), the target offsets and the options.  When one of them changed
+ * since the last forward, the call builds the plan on the host and uploads it
+ * on the stream (through a pinned buffer; the host first waits until the
+ * previous upload has left it); otherwise the plan already on the device
+ * serves, even across encodes of a batch with the same offsets.
  * Errors: STCA_ESTATE (no encode yet), STCA_EINVAL, STCA_ENOMEM, STCA_ECUDA.
  */
 int stca_forward(stca_handle* handle, const void* targets, const int64_t* target_offsets,
